@@ -1,0 +1,174 @@
+"""Plain float64 definition of Parallax attention (decode and causal prefill).
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).  Every function here is
+the explicit two-pass definition, written for a reader to check by eye against
+the method's statement; nothing is blocked, fused or reordered.
+
+The method ("Parallax: Breaking the Boundary Bias with Parameterized Local
+Linear Attention", section "The Core Insight: Covariance Correction"): the
+local linear estimate is softmax attention minus a KV-covariance term probed
+by a per-query vector rho.  Written out for one query q with key set {k_i},
+values {v_i}, softmax scale ``scale`` (the "bandwidth" of the newx.sg
+"Abstract") and probe rho:
+
+    w_i   = exp(s_i - max s) / sum_j exp(s_j - max s),   s_i = scale * q.k_i
+    vbar  = sum_i w_i v_i                 (softmax attention, the NW estimate)
+    kbar  = sum_i w_i k_i
+    S_KV  = sum_i w_i (k_i - kbar)(v_i - vbar)^T          (d_k x d_v)
+    out   = vbar - S_KV^T rho
+
+Readings taken where the pages are silent or garbled (each is listed in the
+design notes):
+  * rho lives in key space ("query-like projector", newx.sg "Abstract"), so it
+    contracts the key side of S_KV: out_j = vbar_j - sum_i w_i ((k_i-kbar).rho)
+    (v_ij - vbar_j).
+  * The covariance uses the same softmax weights as vbar.
+  * rho is used as given: ``scale`` multiplies q.k only.
+  * Causal prefill: key i is visible to query t iff i <= t.
+  * Grouped-query attention: query head h reads KV head h // (Hq / Hkv).
+  * An empty key set gives a zero output.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "softmax_weights",
+    "parallax_query",
+    "sigma_kv",
+    "decode",
+    "gather_paged_keys",
+    "prefill_rows",
+]
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+def softmax_weights(scores) -> np.ndarray:
+    """Softmax of a score vector, max-subtracted, in float64.
+
+    Softmax attention read as a Nadaraya-Watson (local constant) estimator:
+    wispaper blog, "Context: Why Softmax is Not Enough".
+    """
+    s = _f64(scores)
+    e = np.exp(s - s.max())
+    return e / e.sum()
+
+
+def sigma_kv(w, keys, values) -> np.ndarray:
+    """Softmax-weighted key/value cross-covariance, explicit d_k x d_v matrix.
+
+    "KV Covariance Estimation" (newx.sg, "Innovation"); the covariance that
+    the probe reads (wispaper blog, "The Core Insight").
+    """
+    w = _f64(w)
+    K = _f64(keys)
+    V = _f64(values)
+    kbar = w @ K
+    vbar = w @ V
+    Kc = K - kbar
+    Vc = V - vbar
+    return Kc.T @ (w[:, None] * Vc)
+
+
+def parallax_query(q, rho, keys, values, scale: float) -> np.ndarray:
+    """Parallax output for one query over the key set ``keys`` [n, d_k].
+
+    Two passes, as the definition reads: softmax weights first, then the
+    explicit covariance matrix, then its product with the probe.
+    (wispaper blog, "The Core Insight: Covariance Correction": output =
+    softmax attention - Sigma_KV rho.)
+    """
+    q = _f64(q)
+    rho = _f64(rho)
+    K = _f64(keys)
+    V = _f64(values)
+    if K.shape[0] == 0:
+        return np.zeros(V.shape[1], dtype=np.float64)
+    w = softmax_weights(scale * (K @ q))
+    vbar = w @ V
+    S = sigma_kv(w, K, V)
+    return vbar - S.T @ rho
+
+
+def gather_paged_keys(pool, page_table_row, length: int, kv_head: int) -> np.ndarray:
+    """Logical [length, d] rows of one sequence from a paged pool.
+
+    ``pool`` is [num_pages, Hkv, page_size, d]; ``page_table_row[j]`` is the
+    physical page that holds logical tokens j*page_size .. (j+1)*page_size-1.
+    The oracle's own addressing; it shares nothing with the CUDA path.
+    """
+    pool = np.asarray(pool)
+    page_size = pool.shape[2]
+    rows = []
+    n_pages = -(-length // page_size)
+    for j in range(n_pages):
+        page = int(page_table_row[j])
+        take = min(page_size, length - j * page_size)
+        rows.append(_f64(pool[page, kv_head, :take, :]))
+    if not rows:
+        return np.zeros((0, pool.shape[3]), dtype=np.float64)
+    return np.concatenate(rows, axis=0)
+
+
+def decode(q, rho, k_cache, v_cache, scale: float, seq_lens=None,
+           page_table=None, heads=None):
+    """Decode: one new query per (batch, query head) over its KV sequence.
+
+    q, rho: [B, Hq, d].  Contiguous cache: k_cache, v_cache [B, Hkv, L, d],
+    sequence b uses its first ``seq_lens[b]`` rows (all L when seq_lens is
+    None).  Paged cache (page_table given): pools [P, Hkv, page_size, d] and
+    page_table [B, max_pages].
+
+    ``heads``: optional iterable of (b, h) to evaluate; the others are NaN.
+    Returns float64 [B, Hq, d_v].
+    """
+    q = np.asarray(q)
+    rho = np.asarray(rho)
+    B, Hq, _ = q.shape
+    Hkv = k_cache.shape[1]
+    assert Hq % Hkv == 0
+    group = Hq // Hkv
+    dv = v_cache.shape[-1]
+    if page_table is None:
+        L = k_cache.shape[2]
+    if seq_lens is None:
+        assert page_table is None, "paged decode needs seq_lens"
+        seq_lens = [L] * B
+    out = np.full((B, Hq, dv), np.nan, dtype=np.float64)
+    todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    for b, h in todo:
+        kvh = h // group
+        n = int(seq_lens[b])
+        if page_table is None:
+            K = _f64(k_cache[b, kvh, :n, :])
+            V = _f64(v_cache[b, kvh, :n, :])
+        else:
+            K = gather_paged_keys(k_cache, page_table[b], n, kvh)
+            V = gather_paged_keys(v_cache, page_table[b], n, kvh)
+        out[b, h] = parallax_query(q[b, h], rho[b, h], K, V, scale)
+    return out
+
+
+def prefill_rows(q, rho, k, v, rows, scale: float, causal: bool = True):
+    """Prefill outputs for selected rows.
+
+    q, rho: [B, H, T, d]; k, v: [B, Hkv, T, d].  Row (b, h, t) attends to keys
+    0..t when ``causal`` (diagonal included), else to all T keys.
+    Returns float64 [len(rows), d_v] in the order of ``rows``.
+    """
+    q = np.asarray(q)
+    H = q.shape[1]
+    Hkv = k.shape[1]
+    group = H // Hkv
+    T = k.shape[2]
+    res = []
+    for b, h, t in rows:
+        kvh = h // group
+        n = t + 1 if causal else T
+        res.append(parallax_query(q[b, h, t], rho[b, h, t],
+                                  k[b, kvh, :n, :], v[b, kvh, :n, :], scale))
+    return np.stack(res) if res else np.zeros((0, v.shape[-1]))

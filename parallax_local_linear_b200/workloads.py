@@ -1,0 +1,273 @@
+"""Seeded synthetic inputs for Parallax decode and prefill.
+
+This module only draws and lays out inputs; it holds none of the method's
+arithmetic, and both the CUDA path and the float64 oracle consume what it
+returns.  Values are drawn as float32 with a torch generator seeded per
+workload (on the device that will hold them, so multi-GiB caches never cross
+PCIe), then rounded to bfloat16 with round-to-nearest-even.  The oracle reads
+back the very same rounded values.
+
+Named workloads (head_dim d, Hq query heads, Hkv KV heads):
+  decode_f32     B=1,   Hq=1,  Hkv=1, d=64,  L=256,   float32 throughout
+  decode_bf16    B=8,   Hq=16, Hkv=8, d=128, L=4096,  contiguous cache
+  decode_long    B=64,  Hq=32, Hkv=8, d=128, L=32768, keys offset per KV head
+  decode_paged   128 sequences, L ~ U{512..65536}, Hq=16, Hkv=4, d=128,
+                 64-token pages placed by a seeded permutation
+  prefill        B=4, H=16, T=8192, d=128, causal, rho scaled by 0.1
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import numpy as np
+import torch
+
+PAGE_SIZE = 64
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    batch: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    kv_len: int
+    dtype: str = "bf16"           # "bf16" or "f32"
+    key_offset_std: float = 0.0   # per-KV-head offset added to every key
+    paged: bool = False
+    min_len: int = 0              # paged: lengths uniform in [min_len, kv_len]
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+
+@dataclass(frozen=True)
+class PrefillWorkload:
+    name: str
+    batch: int
+    num_heads: int
+    seq_len: int
+    head_dim: int
+    num_kv_heads: int = 0
+    rho_scale: float = 0.1
+    causal: bool = True
+    seed: int = 0
+
+    @property
+    def kv_heads(self) -> int:
+        return self.num_kv_heads or self.num_heads
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+
+WORKLOADS = {
+    "decode_f32": DecodeWorkload("decode_f32", 1, 1, 1, 64, 256, dtype="f32", seed=1),
+    "decode_bf16": DecodeWorkload("decode_bf16", 8, 16, 8, 128, 4096, seed=2),
+    "decode_long": DecodeWorkload("decode_long", 64, 32, 8, 128, 32768, key_offset_std=0.5, seed=3),
+    "decode_paged": DecodeWorkload("decode_paged", 128, 16, 4, 128, 65536, paged=True,
+                                   min_len=512, seed=4),
+    "prefill": PrefillWorkload("prefill", 4, 16, 8192, 128, seed=5),
+}
+
+
+def _gen(device, seed):
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return g
+
+
+def _normal(shape, gen, device, out_dtype, chunk_dim0=True, add=None, mul=1.0):
+    """float32 N(0,1) draws, optionally scaled / offset, rounded to out_dtype.
+
+    Large tensors are drawn one leading-index slice at a time so the float32
+    staging copy stays small.
+    """
+    out = torch.empty(shape, dtype=out_dtype, device=device)
+    if chunk_dim0 and len(shape) > 1 and out.numel() > (1 << 26):
+        for i in range(shape[0]):
+            x = torch.randn(shape[1:], generator=gen, device=device, dtype=torch.float32)
+            if mul != 1.0:
+                x.mul_(mul)
+            if add is not None:
+                x.add_(add)
+            out[i].copy_(x)
+        return out
+    x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+    if mul != 1.0:
+        x.mul_(mul)
+    if add is not None:
+        x.add_(add)
+    out.copy_(x)
+    return out
+
+
+def paged_layout(batch, kv_len, min_len, seed, page_size=PAGE_SIZE):
+    """Sequence lengths, page count and page table of a ragged paged cache.
+
+    Lengths are integers uniform in [min_len, kv_len] (both ends included);
+    the pool has sum(ceil(L_b / page_size)) pages; a seeded permutation of the
+    pool gives each sequence its pages in order.  Unused table slots are -1.
+    """
+    rng = np.random.Generator(np.random.PCG64(seed))
+    lens = rng.integers(min_len, kv_len + 1, size=batch).astype(np.int32)
+    n_pages = -(-lens.astype(np.int64) // page_size)
+    total = int(n_pages.sum())
+    perm = rng.permutation(total).astype(np.int32)
+    max_pages = int(-(-kv_len // page_size))
+    table = np.full((batch, max_pages), -1, dtype=np.int32)
+    cur = 0
+    for b in range(batch):
+        table[b, : n_pages[b]] = perm[cur: cur + n_pages[b]]
+        cur += int(n_pages[b])
+    return lens, table, total
+
+
+def decode_inputs(w: DecodeWorkload, device="cpu", seed=None, nan_poison=True):
+    """Inputs of one decode call.
+
+    Returns a dict: q, rho [B, Hq, d]; k_cache, v_cache ([B, Hkv, L, d] or
+    the paged pool [P, Hkv, 64, d]); seq_lens (int32 [B] or None);
+    page_table (int32 [B, max_pages] or None); scale.  With ``nan_poison``
+    the unused tail of every last page is NaN, so any over-read shows.
+    """
+    seed = w.seed if seed is None else seed
+    dt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    gen = _gen(device, seed)
+    B, Hq, Hkv, d = w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim
+    q = _normal((B, Hq, d), gen, device, dt)
+    rho = _normal((B, Hq, d), gen, device, dt)
+    seq_lens = page_table = None
+    if w.paged:
+        lens, table, total = paged_layout(B, w.kv_len, w.min_len, seed)
+        shape = (total, Hkv, PAGE_SIZE, d)
+    else:
+        shape = (B, Hkv, w.kv_len, d)
+    offset = None
+    if w.key_offset_std:
+        # one d-vector per KV head, shared by every sequence and position
+        offset = (torch.randn((Hkv, d), generator=gen, device=device, dtype=torch.float32)
+                  * w.key_offset_std)
+    k = torch.empty(shape, dtype=dt, device=device)
+    v = torch.empty(shape, dtype=dt, device=device)
+    for i in range(shape[0]):
+        x = torch.randn(shape[1:], generator=gen, device=device, dtype=torch.float32)
+        if offset is not None:
+            x.add_(offset[:, None, :])
+        k[i].copy_(x)
+    for i in range(shape[0]):
+        v[i].copy_(torch.randn(shape[1:], generator=gen, device=device, dtype=torch.float32))
+    if w.paged:
+        seq_lens = torch.from_numpy(lens).to(device)
+        page_table = torch.from_numpy(table).to(device)
+        if nan_poison:
+            _poison_paged_tails(k, v, lens, table)
+    return dict(q=q, rho=rho, k_cache=k, v_cache=v, seq_lens=seq_lens,
+                page_table=page_table, scale=w.scale)
+
+
+def _poison_paged_tails(k, v, lens, table, page_size=PAGE_SIZE):
+    for b, n in enumerate(lens):
+        n = int(n)
+        if n % page_size:
+            last = int(table[b, (n - 1) // page_size])
+            k[last, :, n % page_size:, :] = float("nan")
+            v[last, :, n % page_size:, :] = float("nan")
+
+
+def small_decode_inputs(batch, num_q_heads, num_kv_heads, head_dim, kv_len, *, dtype="bf16",
+                        seq_lens=None, paged=False, page_size=PAGE_SIZE, key_offset_std=0.0,
+                        seed=0, device="cpu", nan_poison=True, value_offset=0.0):
+    """Decode inputs of arbitrary (small) shape for parity sweeps.
+
+    ``seq_lens``: optional list of lengths (each <= kv_len).  Contiguous
+    caches have their rows past each length set to NaN (with nan_poison).
+    ``paged``: the same logical cache, stored in pages placed by a seeded
+    permutation; returns the contiguous copy too (keys ``k_contig``,
+    ``v_contig``) so the two layouts can be compared.
+    """
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    gen = _gen("cpu", seed)
+    B, Hq, Hkv, d, L = batch, num_q_heads, num_kv_heads, head_dim, kv_len
+    q = torch.randn((B, Hq, d), generator=gen).to(dt)
+    rho = torch.randn((B, Hq, d), generator=gen).to(dt)
+    kx = torch.randn((B, Hkv, L, d), generator=gen)
+    if key_offset_std:
+        kx += torch.randn((Hkv, d), generator=gen)[None, :, None, :] * key_offset_std
+    vx = torch.randn((B, Hkv, L, d), generator=gen) + value_offset
+    k = kx.to(dt)
+    v = vx.to(dt)
+    lens = None if seq_lens is None else torch.tensor(seq_lens, dtype=torch.int32)
+    if lens is not None and nan_poison:
+        for b, n in enumerate(seq_lens):
+            k[b, :, n:] = float("nan")
+            v[b, :, n:] = float("nan")
+    res = dict(q=q, rho=rho, k_cache=k, v_cache=v, seq_lens=lens, page_table=None,
+               scale=1.0 / math.sqrt(d))
+    if paged:
+        lens_list = list(seq_lens) if seq_lens is not None else [L] * B
+        n_pages = [-(-n // page_size) for n in lens_list]
+        total = max(1, sum(n_pages))
+        rng = np.random.Generator(np.random.PCG64(seed + 7))
+        perm = rng.permutation(total)
+        max_pages = max(1, -(-L // page_size))
+        table = np.full((B, max_pages), -1, dtype=np.int32)
+        kp = torch.full((total, Hkv, page_size, d), float("nan"), dtype=dt)
+        vp = torch.full((total, Hkv, page_size, d), float("nan"), dtype=dt)
+        cur = 0
+        for b, n in enumerate(lens_list):
+            for j in range(n_pages[b]):
+                page = int(perm[cur])
+                cur += 1
+                table[b, j] = page
+                take = min(page_size, n - j * page_size)
+                kp[page, :, :take] = k[b, :, j * page_size: j * page_size + take]
+                vp[page, :, :take] = v[b, :, j * page_size: j * page_size + take]
+        res.update(k_contig=k, v_contig=v, k_cache=kp, v_cache=vp,
+                   page_table=torch.from_numpy(table),
+                   seq_lens=torch.tensor(lens_list, dtype=torch.int32))
+    return res
+
+
+def prefill_inputs(w: PrefillWorkload, device="cpu", seed=None):
+    """q, rho [B, H, T, d]; k, v [B, Hkv, T, d] (bfloat16); rho scaled by rho_scale."""
+    seed = w.seed if seed is None else seed
+    gen = _gen(device, seed)
+    B, H, T, d = w.batch, w.num_heads, w.seq_len, w.head_dim
+    q = _normal((B, H, T, d), gen, device, torch.bfloat16)
+    rho = _normal((B, H, T, d), gen, device, torch.bfloat16, mul=w.rho_scale)
+    k = _normal((B, w.kv_heads, T, d), gen, device, torch.bfloat16)
+    v = _normal((B, w.kv_heads, T, d), gen, device, torch.bfloat16)
+    return dict(q=q, rho=rho, k=k, v=v, scale=w.scale, causal=w.causal)
+
+
+def small_prefill_inputs(batch, num_heads, seq_len, head_dim, *, num_kv_heads=0, rho_scale=0.1,
+                         seed=0, device="cpu"):
+    w = PrefillWorkload("small", batch, num_heads, seq_len, head_dim,
+                        num_kv_heads=num_kv_heads, rho_scale=rho_scale, seed=seed)
+    return prefill_inputs(w, device=device)
+
+
+def kv_bytes(w: DecodeWorkload, seq_lens=None) -> int:
+    """Algorithmic K+V bytes one decode call reads: every row once."""
+    elt = 4 if w.dtype == "f32" else 2
+    if seq_lens is None:
+        tokens = w.batch * w.kv_len
+    else:
+        tokens = int(np.asarray(seq_lens, dtype=np.int64).sum())
+    return tokens * w.num_kv_heads * 2 * w.head_dim * elt
+
+
+def prefill_flops(w: PrefillWorkload) -> int:
+    """Algorithmic FLOP of one prefill call: 8*d per visible (query, key) pair
+    (q.k, rho.k, and the two weighted value products, 2*d each)."""
+    T = w.seq_len
+    pairs = T * (T + 1) // 2 if w.causal else T * T
+    return 8 * w.head_dim * pairs * w.batch * w.num_heads
+
