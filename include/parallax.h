@@ -1,0 +1,165 @@
+/*
+ * parallax.h -- C ABI of libparallax.so: Parallax attention forward on B200.
+ *
+ * Parallax is a parameterized Local Linear Attention.  For one query q with
+ * probe rho over keys k_i and values v_i (sources: the newx.sg page
+ * "Parallax: Parameterized Local Linear Attention for Language Modeling",
+ * section "Abstract"; the wispaper.ai blog "Parallax: Breaking the Boundary
+ * Bias with Parameterized Local Linear Attention", sections "The Core
+ * Insight: Covariance Correction" and "Hardware Efficiency"):
+ *
+ *     w_i  = softmax_i(scale * q.k_i)
+ *     vbar = sum_i w_i v_i,  kbar = sum_i w_i k_i
+ *     S_KV = sum_i w_i (k_i - kbar)(v_i - vbar)^T        (d x d)
+ *     out  = vbar - S_KV^T rho
+ *
+ * computed in one pass over the KV stream (the covariance matrix is never
+ * formed): with e_i = exp(scale q.k_i - m), a_i = rho.k_i,
+ *     out = (O1/l) (1 + c/l) - O2/l,
+ *     l = sum e_i, c = sum e_i a_i, O1 = sum e_i v_i, O2 = sum e_i a_i v_i.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named as device pointers are CUDA device memory of the
+ *     current device, owned by the caller, dense row-major with the last
+ *     dimension contiguous and 16-byte aligned.  The library keeps no
+ *     pointer after a call returns and allocates no device memory.
+ *   - Calls are asynchronous on `stream` (0 = legacy default stream).  They
+ *     validate on the host first and launch nothing when validation fails.
+ *   - Return values: plx_status.  Faults found by a kernel while it runs
+ *     (an out-of-range page id, a pipeline wait that ran out of time) set a
+ *     per-device error word read by parallax_last_device_error(); kernels
+ *     never trap.
+ *   - Not thread-safe across concurrent calls that share a workspace.
+ */
+#ifndef PARALLAX_H
+#define PARALLAX_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define PARALLAX_ABI_VERSION 1
+
+typedef enum plx_status {
+  PLX_OK = 0,
+  PLX_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer      */
+  PLX_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. head_dim 96)    */
+  PLX_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required      */
+  PLX_ERR_CUDA = 4,          /* a CUDA runtime / driver call or launch failed   */
+  PLX_ERR_DEVICE_FAULT = 5,  /* a kernel reported bad input (see error word)    */
+  PLX_ERR_TIMEOUT = 6        /* a kernel wait ran out of time (see error word)  */
+} plx_status;
+
+typedef enum plx_dtype { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
+
+/* Device error word codes (bit flags; several may be set). */
+#define PLX_DEVERR_BAD_PAGE   1   /* page_table entry outside [0, num_pages)     */
+#define PLX_DEVERR_TIMEOUT    2   /* an mbarrier / pipeline wait gave up         */
+#define PLX_DEVERR_BAD_LENGTH 4   /* seq_lens[b] < 0 or > kv_len                 */
+
+/* ------------------------------------------------------------------------
+ * Decode: one new query per (sequence, query head) over its KV cache.
+ * Defined by the single-pass decode of the "Hardware Efficiency" section of
+ * the wispaper.ai blog (softmax and covariance branches fused in one pass
+ * over the KV stream), on the definition above.
+ * ---------------------------------------------------------------------- */
+typedef struct plx_decode_params {
+  int32_t batch;              /* B >= 1                                        */
+  int32_t num_q_heads;        /* Hq, a multiple of num_kv_heads                */
+  int32_t num_kv_heads;       /* Hkv; query head h reads KV head h / (Hq/Hkv)  */
+  int32_t head_dim;           /* d: 64 or 128                                  */
+  int32_t kv_len;             /* contiguous: rows per sequence in the cache, L;
+                                 paged: upper bound of every seq_lens[b]       */
+  int32_t page_size;          /* 0: contiguous cache; 64: paged cache          */
+  int32_t num_pages;          /* paged: pages in the pool, P                   */
+  int32_t max_pages_per_seq;  /* paged: row stride of page_table (>= ceil(kv_len/64)) */
+  int32_t in_dtype;           /* plx_dtype of q, rho and the caches            */
+  int32_t out_dtype;          /* plx_dtype of out                              */
+  float scale;                /* softmax scale on q.k (e.g. 1/sqrt(d))         */
+  int32_t num_splits;         /* KV splits per sequence; 0 = choose            */
+} plx_decode_params;
+
+/* Number of KV splits a decode call with these parameters uses on a device
+ * with `num_sms` SMs (num_sms <= 0: the current device).  Host-only; makes
+ * no CUDA call when num_sms > 0.  Returns -1 for invalid parameters. */
+int32_t parallax_decode_num_splits(const plx_decode_params* p, int32_t num_sms);
+
+/* Workspace bytes parallax_decode needs (0 when it needs none), for
+ * `num_sms` as above.  Returns (size_t)-1 for invalid parameters.
+ * Layout: a counter region (one int32 per (sequence, KV head), padded to
+ * 256 B) followed by fp32 split partials.  The counter region must be zero
+ * before the workspace is first used (e.g. cudaMemsetAsync); every call
+ * that completes leaves it zero again, so one zeroing lasts for the
+ * workspace's lifetime. */
+size_t parallax_decode_workspace_size(const plx_decode_params* p, int32_t num_sms);
+
+/* Parallax decode.
+ *   q, rho      device, [B, Hq, d] of in_dtype: query and probe per head.
+ *   k_cache,    device, in_dtype.  Contiguous (page_size 0): [B, Hkv, L, d].
+ *   v_cache     Paged (page_size 64): pools [P, Hkv, 64, d]; logical token t
+ *               of sequence b is row t % 64 of page page_table[b][t / 64].
+ *   page_table  device int32 [B, max_pages_per_seq]; NULL when contiguous.
+ *               Entries past a sequence's last page are not read.
+ *   seq_lens    device int32 [B], 0 <= seq_lens[b] <= kv_len; NULL means
+ *               every sequence has kv_len tokens (required when paged).
+ *               A sequence of length 0 gets a zero output.
+ *   out         device, [B, Hq, d] of out_dtype (bf16 output is rounded to
+ *               nearest even from fp32).
+ *   workspace   device, >= parallax_decode_workspace_size() bytes, 256-byte
+ *               aligned; may be NULL when that size is 0.
+ * Rows of the cache past a sequence's length are never used in arithmetic
+ * (they may hold anything, NaN included). */
+plx_status parallax_decode(const void* q, const void* rho,
+                           const void* k_cache, const void* v_cache,
+                           const int32_t* page_table, const int32_t* seq_lens,
+                           void* out, void* workspace, size_t workspace_bytes,
+                           const plx_decode_params* p, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Prefill: every position of a sequence is a query; causal (key i visible
+ * to query t iff i <= t) or full.  The same definition per row; the dense
+ * contractions (q.K^T, rho.K^T, P.V, (P o A).V) run on tcgen05 tensor cores.
+ * ---------------------------------------------------------------------- */
+typedef struct plx_prefill_params {
+  int32_t batch;          /* B                                                */
+  int32_t num_heads;      /* H (query heads)                                  */
+  int32_t num_kv_heads;   /* Hkv, divides H; 0 means H                        */
+  int32_t seq_len;        /* T >= 1                                           */
+  int32_t head_dim;       /* d: 128                                           */
+  int32_t in_dtype;       /* PLX_BF16                                         */
+  int32_t out_dtype;      /* PLX_BF16 or PLX_F32                              */
+  float scale;            /* softmax scale on q.k                             */
+  int32_t causal;         /* 1: causal mask (diagonal included); 0: none      */
+} plx_prefill_params;
+
+/* Parallax prefill.
+ *   q, rho   device, [B, H, T, d] bf16.
+ *   k, v     device, [B, Hkv, T, d] bf16.
+ *   out      device, [B, H, T, d] of out_dtype. */
+plx_status parallax_prefill(const void* q, const void* rho, const void* k, const void* v,
+                            void* out, const plx_prefill_params* p, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Errors and introspection.
+ * ---------------------------------------------------------------------- */
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word into *code (0 = no fault, else PLX_DEVERR_* bits).  Returns PLX_OK,
+ * or PLX_ERR_CUDA if the synchronisation or the read failed. */
+plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code);
+
+/* Static string naming a status. */
+const char* parallax_status_string(plx_status s);
+
+/* PARALLAX_ABI_VERSION of the loaded library. */
+int32_t parallax_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PARALLAX_H */

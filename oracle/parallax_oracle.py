@@ -100,8 +100,9 @@ def gather_paged_keys(pool, page_table_row, length: int, kv_head: int) -> np.nda
     ``pool`` is [num_pages, Hkv, page_size, d]; ``page_table_row[j]`` is the
     physical page that holds logical tokens j*page_size .. (j+1)*page_size-1.
     The oracle's own addressing; it shares nothing with the CUDA path.
+    ``pool`` may be any object with ``.shape`` whose indexing returns arrays
+    (so a multi-GiB pool can be read one page at a time).
     """
-    pool = np.asarray(pool)
     page_size = pool.shape[2]
     rows = []
     n_pages = -(-length // page_size)
@@ -158,9 +159,9 @@ def prefill_rows(q, rho, k, v, rows, scale: float, causal: bool = True):
 
     q, rho: [B, H, T, d]; k, v: [B, Hkv, T, d].  Row (b, h, t) attends to keys
     0..t when ``causal`` (diagonal included), else to all T keys.
-    Returns float64 [len(rows), d_v] in the order of ``rows``.
+    Returns float64 [len(rows), d_v] in the order of ``rows``.  The inputs may
+    be arrays or any objects with ``.shape`` whose indexing returns arrays.
     """
-    q = np.asarray(q)
     H = q.shape[1]
     Hkv = k.shape[1]
     group = H // Hkv

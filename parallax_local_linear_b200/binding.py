@@ -1,0 +1,222 @@
+"""ctypes binding of libparallax.so (declared in include/parallax.h).
+
+Argument marshalling only: these functions read tensor pointers, shapes and
+the current torch stream, fill the C parameter structs and call the library.
+Every step of the computation runs in the library's CUDA kernels.  Importing
+this module loads the library and raises if it has not been built; there is
+no fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libparallax.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m parallax_local_linear_b200.build`")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+PLX_F32, PLX_BF16 = 0, 1
+STATUS = {0: "PLX_OK", 1: "PLX_ERR_INVALID_ARG", 2: "PLX_ERR_UNSUPPORTED", 3: "PLX_ERR_WORKSPACE",
+          4: "PLX_ERR_CUDA", 5: "PLX_ERR_DEVICE_FAULT", 6: "PLX_ERR_TIMEOUT"}
+DEVERR_BAD_PAGE, DEVERR_TIMEOUT, DEVERR_BAD_LENGTH = 1, 2, 4
+PAGE_SIZE = 64
+
+
+class DecodeParams(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("kv_len", ctypes.c_int32), ("page_size", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+                ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+                ("scale", ctypes.c_float), ("num_splits", ctypes.c_int32)]
+
+
+class PrefillParams(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("seq_len", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("in_dtype", ctypes.c_int32),
+                ("out_dtype", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("causal", ctypes.c_int32)]
+
+
+_vp, _i32p = ctypes.c_void_p, ctypes.c_void_p
+lib.parallax_abi_version.restype = ctypes.c_int32
+lib.parallax_status_string.restype = ctypes.c_char_p
+lib.parallax_status_string.argtypes = [ctypes.c_int]
+lib.parallax_decode_num_splits.restype = ctypes.c_int32
+lib.parallax_decode_num_splits.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_int32]
+lib.parallax_decode_workspace_size.restype = ctypes.c_size_t
+lib.parallax_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_int32]
+lib.parallax_decode.restype = ctypes.c_int
+lib.parallax_decode.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, _vp, ctypes.c_size_t,
+                                ctypes.POINTER(DecodeParams), _vp]
+lib.parallax_prefill.restype = ctypes.c_int
+lib.parallax_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(PrefillParams), _vp]
+lib.parallax_last_device_error.restype = ctypes.c_int
+lib.parallax_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
+
+SIZE_MAX = ctypes.c_size_t(-1).value
+
+
+class ParallaxError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)}")
+
+
+def _dtype_code(dt):
+    if dt == torch.bfloat16:
+        return PLX_BF16
+    if dt == torch.float32:
+        return PLX_F32
+    raise TypeError(f"unsupported dtype {dt}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _check_cuda(name, t, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+_ws_lock = threading.Lock()
+_workspaces = {}
+
+
+def _workspace(device, nbytes):
+    """A zero-initialised workspace per device, grown on demand.
+
+    The counter region must start at zero; the library leaves it zero after
+    every call, so the buffer is zeroed only when (re)allocated.
+    """
+    if nbytes == 0:
+        return None
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    with _ws_lock:
+        ws = _workspaces.get(idx)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+            _workspaces[idx] = ws
+        return ws
+
+
+def decode_params(q, k_cache, *, page_table=None, kv_len=None, scale=None, out_dtype=None,
+                  num_splits=0, num_pages=None):
+    B, Hq, d = q.shape
+    paged = page_table is not None
+    Hkv = k_cache.shape[1]
+    if paged:
+        if k_cache.shape[2] != PAGE_SIZE:
+            raise ValueError(f"paged caches hold {PAGE_SIZE}-token pages: got {tuple(k_cache.shape)}")
+        max_pages = page_table.shape[1]
+        L = kv_len if kv_len is not None else max_pages * PAGE_SIZE
+        n_pages = k_cache.shape[0] if num_pages is None else num_pages
+    else:
+        max_pages = 0
+        L = k_cache.shape[2] if kv_len is None else kv_len
+        n_pages = 0
+    scale = (1.0 / d ** 0.5) if scale is None else float(scale)
+    out_dtype = q.dtype if out_dtype is None else out_dtype
+    return DecodeParams(B, Hq, Hkv, d, L, PAGE_SIZE if paged else 0, n_pages, max_pages,
+                        _dtype_code(q.dtype), _dtype_code(out_dtype), scale, int(num_splits))
+
+
+def decode_workspace_size(params: DecodeParams, num_sms: int = 0) -> int:
+    n = lib.parallax_decode_workspace_size(ctypes.byref(params), int(num_sms))
+    if n == SIZE_MAX:
+        raise ParallaxError(1, "parallax_decode_workspace_size")
+    return n
+
+
+def decode_num_splits(params: DecodeParams, num_sms: int = 0) -> int:
+    return lib.parallax_decode_num_splits(ctypes.byref(params), int(num_sms))
+
+
+def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=None, out=None,
+           out_dtype=None, num_splits=0, kv_len=None):
+    """Parallax decode: out[b, h] = vbar - Sigma_KV^T rho[b, h] over sequence b.
+
+    q, rho: [B, Hq, d] (bfloat16 or float32, the cache's dtype).
+    Contiguous cache: k_cache, v_cache [B, Hkv, L, d]; ``seq_lens`` (int32
+    [B], optional) limits each sequence.  Paged cache: pools [P, Hkv, 64, d]
+    with ``page_table`` (int32 [B, max_pages]) and ``seq_lens`` (required).
+    Returns out [B, Hq, d] in ``out_dtype`` (default: the input dtype).
+    """
+    _check_cuda("q", q)
+    for name, t in (("rho", rho), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_cuda(name, t, q.dtype)
+    if rho.shape != q.shape or k_cache.shape != v_cache.shape:
+        raise ValueError("shape mismatch between q/rho or k_cache/v_cache")
+    if k_cache.dim() != 4 or k_cache.shape[-1] != q.shape[-1]:
+        raise ValueError("caches must be 4-D with the head_dim of q")
+    if page_table is not None:
+        _check_cuda("page_table", page_table, torch.int32)
+        if seq_lens is None:
+            raise ValueError("a paged cache needs seq_lens")
+    if seq_lens is not None:
+        _check_cuda("seq_lens", seq_lens, torch.int32)
+    p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale,
+                      out_dtype=out_dtype, num_splits=num_splits)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    else:
+        _check_cuda("out", out)
+    nbytes = decode_workspace_size(p)
+    ws = _workspace(q.device, nbytes)
+    st = lib.parallax_decode(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                             _ptr(seq_lens), _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                             ctypes.byref(p), _stream_ptr(q.device))
+    if st != 0:
+        raise ParallaxError(st, "parallax_decode")
+    return out
+
+
+def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):
+    """Parallax prefill.  q, rho: [B, H, T, d] bf16; k, v: [B, Hkv, T, d] bf16.
+    Row t attends to keys 0..t when causal, else to all T keys."""
+    for name, t in (("q", q), ("rho", rho), ("k", k), ("v", v)):
+        _check_cuda(name, t, torch.bfloat16)
+    B, H, T, d = q.shape
+    if rho.shape != q.shape or k.shape != v.shape or k.shape[0] != B or k.shape[2] != T or k.shape[3] != d:
+        raise ValueError("shape mismatch")
+    out_dtype = out_dtype or q.dtype
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    else:
+        _check_cuda("out", out, out_dtype)
+    scale = (1.0 / d ** 0.5) if scale is None else float(scale)
+    p = PrefillParams(B, H, k.shape[1], T, d, PLX_BF16, _dtype_code(out_dtype), scale, 1 if causal else 0)
+    st = lib.parallax_prefill(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(p),
+                              _stream_ptr(q.device))
+    if st != 0:
+        raise ParallaxError(st, "parallax_prefill")
+    return out
+
+
+def last_device_error(device=None) -> int:
+    """Synchronises the current stream and returns (and clears) the device error word."""
+    device = device or torch.device("cuda", torch.cuda.current_device())
+    code = ctypes.c_int32(0)
+    st = lib.parallax_last_device_error(_stream_ptr(device), ctypes.byref(code))
+    if st != 0:
+        raise ParallaxError(st, "parallax_last_device_error")
+    return code.value

@@ -1,0 +1,302 @@
+// libparallax.so: the C ABI declared in include/parallax.h.
+//
+// Host side of every entry point: argument validation, the split plan of a
+// decode call, TMA tensor maps, kernel launches.  All arithmetic of the path
+// runs in the kernels included below; nothing here touches tensor data.
+#include "parallax.h"
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include "ptx.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace {
+
+using namespace plx;
+
+constexpr int kMaxDevices = 64;
+
+// Decode kernel configuration (bf16 path): consumer warps and ring depth.
+constexpr int kDecodeNC = 4;
+constexpr int kDecodeStages128 = 4;
+constexpr int kDecodeStages64 = 6;
+constexpr int kDecodeF32Warps = 4;
+
+// Tiles per split: a split covers at least kMinTilesPerSplit and at most
+// kMaxTilesPerSplit 64-token tiles; within that range the split count aims at
+// kTargetCtasPerSm CTAs per SM over the device.
+constexpr int kMinTilesPerSplit = 2;
+constexpr int kMaxTilesPerSplit = 64;
+constexpr int kTargetCtasPerSm = 4;
+constexpr int kMaxSplits = 65535;   // gridDim.y limit
+
+std::mutex g_mu;
+int g_num_sms[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int current_device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_num_sms[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  return g_encode;
+}
+
+// Row-major [rows, cols] bf16 tensor, box [box_rows, box_cols], 128-byte swizzle.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                    uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ decode
+struct DecodePlan {
+  int splits, tiles_per_split;
+  size_t counter_bytes, partial_bytes;
+};
+
+plx_status validate_decode(const plx_decode_params* p) {
+  if (p == nullptr) return PLX_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->num_q_heads < 1 || p->num_kv_heads < 1) return PLX_ERR_INVALID_ARG;
+  if (p->num_q_heads % p->num_kv_heads != 0) return PLX_ERR_INVALID_ARG;
+  if (p->kv_len < 0 || p->num_splits < 0) return PLX_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return PLX_ERR_INVALID_ARG;
+  if (p->in_dtype != PLX_F32 && p->in_dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
+  if (p->out_dtype != PLX_F32 && p->out_dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
+  if (p->head_dim != 64 && p->head_dim != 128) return PLX_ERR_UNSUPPORTED;
+  if (p->page_size != 0 && p->page_size != kTile) return PLX_ERR_UNSUPPORTED;
+  if (p->in_dtype == PLX_BF16 && p->num_q_heads / p->num_kv_heads > kMaxGroup) return PLX_ERR_UNSUPPORTED;
+  if (p->page_size != 0) {
+    if (p->num_pages < 1) return PLX_ERR_INVALID_ARG;
+    if (p->max_pages_per_seq < (p->kv_len + kTile - 1) / kTile) return PLX_ERR_INVALID_ARG;
+    if ((int64_t)p->num_pages * p->num_kv_heads * kTile >= (int64_t)INT32_MAX) return PLX_ERR_UNSUPPORTED;
+  } else {
+    if ((int64_t)p->batch * p->num_kv_heads * ((int64_t)p->kv_len + kTile) >= (int64_t)INT32_MAX)
+      return PLX_ERR_UNSUPPORTED;
+  }
+  if ((int64_t)p->batch * p->num_q_heads >= (int64_t)INT32_MAX / 2) return PLX_ERR_UNSUPPORTED;
+  return PLX_OK;
+}
+
+DecodePlan plan_decode(const plx_decode_params* p, int num_sms) {
+  DecodePlan pl{};
+  const int tiles = (p->kv_len + kTile - 1) / kTile;
+  if (tiles == 0) {
+    pl.splits = 1;
+    pl.tiles_per_split = 1;
+    return pl;
+  }
+  int tps;
+  if (p->num_splits > 0) {
+    tps = (tiles + p->num_splits - 1) / p->num_splits;
+  } else {
+    const int64_t units = (int64_t)p->batch * (p->in_dtype == PLX_BF16 ? p->num_kv_heads : p->num_q_heads);
+    const int64_t target = (int64_t)kTargetCtasPerSm * (num_sms > 0 ? num_sms : 148);
+    const int64_t want_splits = (target + units - 1) / units;
+    tps = (int)((tiles + want_splits - 1) / want_splits);
+    tps = tps < kMinTilesPerSplit ? kMinTilesPerSplit : tps;
+    tps = tps > kMaxTilesPerSplit ? kMaxTilesPerSplit : tps;
+  }
+  if (tps > tiles) tps = tiles;
+  if (tps < 1) tps = 1;
+  if ((tiles + tps - 1) / tps > kMaxSplits) tps = (tiles + kMaxSplits - 1) / kMaxSplits;
+  pl.tiles_per_split = tps;
+  pl.splits = (tiles + tps - 1) / tps;
+  if (pl.splits > 1) {
+    pl.counter_bytes = (((size_t)p->batch * p->num_q_heads * 4) + 255) & ~size_t(255);
+    pl.partial_bytes = (size_t)pl.splits * p->batch * p->num_q_heads * (2 * p->head_dim + 4) * 4;
+  }
+  return pl;
+}
+
+template <int D, int STAGES, bool kLoInPad>
+plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
+                            cudaStream_t stream) {
+  constexpr int smem = tc_smem_bytes<D, STAGES, kDecodeNC>();
+  auto kern = decode_tc_kernel<D, STAGES, kDecodeNC, kLoInPad>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  kern<<<grid, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+template <int D>
+plx_status launch_decode_f32(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
+  decode_f32_kernel<D, kDecodeF32Warps><<<grid, kDecodeF32Warps * 32, 0, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+// ----------------------------------------------------------------- prefill
+plx_status validate_prefill(const plx_prefill_params* p) {
+  if (p == nullptr) return PLX_ERR_INVALID_ARG;
+  const int hkv = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
+  if (p->batch < 1 || p->num_heads < 1 || hkv < 1 || p->seq_len < 1) return PLX_ERR_INVALID_ARG;
+  if (p->num_heads % hkv != 0) return PLX_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale)) return PLX_ERR_INVALID_ARG;
+  if (p->in_dtype != PLX_BF16) return p->in_dtype == PLX_F32 ? PLX_ERR_UNSUPPORTED : PLX_ERR_INVALID_ARG;
+  if (p->out_dtype != PLX_F32 && p->out_dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
+  if (p->head_dim != 128) return PLX_ERR_UNSUPPORTED;
+  if (p->causal != 0 && p->causal != 1) return PLX_ERR_INVALID_ARG;
+  if ((int64_t)p->batch * p->num_heads * ((int64_t)p->seq_len + 128) >= (int64_t)INT32_MAX)
+    return PLX_ERR_UNSUPPORTED;
+  return PLX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t parallax_abi_version(void) { return PARALLAX_ABI_VERSION; }
+
+const char* parallax_status_string(plx_status s) {
+  switch (s) {
+    case PLX_OK: return "PLX_OK";
+    case PLX_ERR_INVALID_ARG: return "PLX_ERR_INVALID_ARG";
+    case PLX_ERR_UNSUPPORTED: return "PLX_ERR_UNSUPPORTED";
+    case PLX_ERR_WORKSPACE: return "PLX_ERR_WORKSPACE";
+    case PLX_ERR_CUDA: return "PLX_ERR_CUDA";
+    case PLX_ERR_DEVICE_FAULT: return "PLX_ERR_DEVICE_FAULT";
+    case PLX_ERR_TIMEOUT: return "PLX_ERR_TIMEOUT";
+  }
+  return "PLX_UNKNOWN_STATUS";
+}
+
+int32_t parallax_decode_num_splits(const plx_decode_params* p, int32_t num_sms) {
+  if (validate_decode(p) != PLX_OK) return -1;
+  if (num_sms <= 0) num_sms = current_device_sms();
+  if (num_sms <= 0) return -1;
+  return plan_decode(p, num_sms).splits;
+}
+
+size_t parallax_decode_workspace_size(const plx_decode_params* p, int32_t num_sms) {
+  if (validate_decode(p) != PLX_OK) return (size_t)-1;
+  if (num_sms <= 0) num_sms = current_device_sms();
+  if (num_sms <= 0) return (size_t)-1;
+  const DecodePlan pl = plan_decode(p, num_sms);
+  return pl.counter_bytes + pl.partial_bytes;
+}
+
+plx_status parallax_decode(const void* q, const void* rho, const void* k_cache, const void* v_cache,
+                           const int32_t* page_table, const int32_t* seq_lens, void* out, void* workspace,
+                           size_t workspace_bytes, const plx_decode_params* p, cudaStream_t stream) {
+  plx_status st = validate_decode(p);
+  if (st != PLX_OK) return st;
+  if (!q || !rho || !k_cache || !v_cache || !out) return PLX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
+    return PLX_ERR_INVALID_ARG;
+  const bool paged = p->page_size != 0;
+  if (paged && (page_table == nullptr || seq_lens == nullptr)) return PLX_ERR_INVALID_ARG;
+  if (!paged && page_table != nullptr) return PLX_ERR_INVALID_ARG;
+  if ((page_table && !aligned(page_table, 4)) || (seq_lens && !aligned(seq_lens, 4))) return PLX_ERR_INVALID_ARG;
+
+  const int num_sms = current_device_sms();
+  if (num_sms <= 0) return PLX_ERR_CUDA;
+  const DecodePlan pl = plan_decode(p, num_sms);
+  const size_t need = pl.counter_bytes + pl.partial_bytes;
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)))
+    return PLX_ERR_WORKSPACE;
+
+  const int D = p->head_dim;
+  if (p->kv_len == 0) {
+    // Every sequence is empty: the output is zero.
+    const size_t elt = p->out_dtype == PLX_BF16 ? 2 : 4;
+    return cudaMemsetAsync(out, 0, (size_t)p->batch * p->num_q_heads * D * elt, stream) == cudaSuccess
+               ? PLX_OK
+               : PLX_ERR_CUDA;
+  }
+
+  DecodeArgs a{};
+  a.q = q;
+  a.rho = rho;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.out = out;
+  a.counters = need ? reinterpret_cast<int32_t*>(workspace) : nullptr;
+  a.partials = need ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + pl.counter_bytes) : nullptr;
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.group = p->num_q_heads / p->num_kv_heads;
+  a.kv_len = p->kv_len;
+  a.paged = paged ? 1 : 0;
+  a.num_pages = paged ? p->num_pages : 0;
+  a.max_pages = paged ? p->max_pages_per_seq : 0;
+  a.splits = pl.splits;
+  a.tiles_per_split = pl.tiles_per_split;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
+
+  if (p->in_dtype == PLX_F32) {
+    const dim3 grid(p->batch * p->num_q_heads, pl.splits);
+    return D == 64 ? launch_decode_f32<64>(a, grid, stream) : launch_decode_f32<128>(a, grid, stream);
+  }
+  const uint64_t rows = paged ? (uint64_t)p->num_pages * p->num_kv_heads * kTile
+                              : (uint64_t)p->batch * p->num_kv_heads * p->kv_len;
+  CUtensorMap tk, tv;
+  if (!make_tmap_bf16(&tk, k_cache, D, rows, 64, kTile) || !make_tmap_bf16(&tv, v_cache, D, rows, 64, kTile))
+    return PLX_ERR_CUDA;
+  const dim3 grid(p->batch * p->num_kv_heads, pl.splits);
+  const bool pad = a.group <= kMaxGroup / 2;
+  if (D == 64)
+    return pad ? launch_decode_tc<64, kDecodeStages64, true>(a, tk, tv, grid, stream)
+               : launch_decode_tc<64, kDecodeStages64, false>(a, tk, tv, grid, stream);
+  return pad ? launch_decode_tc<128, kDecodeStages128, true>(a, tk, tv, grid, stream)
+             : launch_decode_tc<128, kDecodeStages128, false>(a, tk, tv, grid, stream);
+}
+
+plx_status parallax_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,
+                            const plx_prefill_params* p, cudaStream_t stream) {
+  plx_status st = validate_prefill(p);
+  if (st != PLX_OK) return st;
+  if (!q || !rho || !k || !v || !out) return PLX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
+    return PLX_ERR_INVALID_ARG;
+  return launch_prefill(q, rho, k, v, out, p, stream);
+}
+
+plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code) {
+  if (code == nullptr) return PLX_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return PLX_ERR_CUDA;
+  int32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, plx::g_device_error, sizeof(v)) != cudaSuccess) return PLX_ERR_CUDA;
+  if (cudaMemcpyToSymbol(plx::g_device_error, &zero, sizeof(zero)) != cudaSuccess) return PLX_ERR_CUDA;
+  *code = v;
+  return PLX_OK;
+}
+
+}  // extern "C"

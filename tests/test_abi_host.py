@@ -1,0 +1,139 @@
+"""Host-side checks of the C ABI that need no GPU.
+
+The library must load, export every function include/parallax.h declares, and
+reject bad arguments on the host before any CUDA call.  The split plan is
+pure host logic and is checked against its documented rule.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "parallax.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(parallax_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def binding():
+    from parallax_local_linear_b200 import binding as b
+    return b
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for must in ("parallax_decode", "parallax_prefill", "parallax_decode_workspace_size",
+                 "parallax_last_device_error", "parallax_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(binding):
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, f"not exported: {missing}"
+
+
+def test_abi_version_and_status_strings(binding):
+    assert binding.lib.parallax_abi_version() == 1
+    for code, name in binding.STATUS.items():
+        assert binding.lib.parallax_status_string(code).decode() == name
+
+
+def _params(binding, **kw):
+    base = dict(batch=8, num_q_heads=16, num_kv_heads=8, head_dim=128, kv_len=4096, page_size=0,
+                num_pages=0, max_pages_per_seq=0, in_dtype=1, out_dtype=1, scale=0.088, num_splits=0)
+    base.update(kw)
+    return binding.DecodeParams(**base)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(batch=0), dict(num_q_heads=12, num_kv_heads=8), dict(kv_len=-1), dict(in_dtype=7),
+    dict(out_dtype=9), dict(scale=float("inf")), dict(num_splits=-2),
+    dict(page_size=64, num_pages=0, max_pages_per_seq=64),
+    dict(page_size=64, num_pages=10, max_pages_per_seq=3),
+])
+def test_invalid_decode_params_are_rejected(binding, bad):
+    p = _params(binding, **bad)
+    assert binding.lib.parallax_decode_num_splits(ctypes.byref(p), 148) == -1
+    assert binding.lib.parallax_decode_workspace_size(ctypes.byref(p), 148) == binding.SIZE_MAX
+    st = binding.lib.parallax_decode(None, None, None, None, None, None, None, None, 0, ctypes.byref(p), None)
+    assert st == 1
+
+
+@pytest.mark.parametrize("unsup", [dict(head_dim=96), dict(page_size=32, num_pages=4, max_pages_per_seq=200),
+                                   dict(num_q_heads=32, num_kv_heads=2)])
+def test_unsupported_decode_params(binding, unsup):
+    p = _params(binding, **unsup)
+    st = binding.lib.parallax_decode(None, None, None, None, None, None, None, None, 0, ctypes.byref(p), None)
+    assert st == 2
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(binding):
+    p = _params(binding)
+    st = binding.lib.parallax_decode(None, None, None, None, None, None, None, None, 0, ctypes.byref(p), None)
+    assert st == 1
+    buf = ctypes.create_string_buffer(64)
+    addr = ctypes.addressof(buf)
+    odd = ctypes.c_void_p(addr + 2)
+    al = ctypes.c_void_p((addr + 15) & ~15)
+    st = binding.lib.parallax_decode(odd, al, al, al, None, None, al, None, 0, ctypes.byref(p), None)
+    assert st == 1
+    # contiguous cache given a page table
+    st = binding.lib.parallax_decode(al, al, al, al, al, None, al, None, 0, ctypes.byref(p), None)
+    assert st == 1
+    pp = _params(binding, page_size=64, num_pages=4, max_pages_per_seq=64)
+    st = binding.lib.parallax_decode(al, al, al, al, None, None, al, None, 0, ctypes.byref(pp), None)
+    assert st == 1   # paged without a page table / seq_lens
+
+
+@pytest.mark.parametrize("bad", [dict(seq_len=0), dict(head_dim=64), dict(in_dtype=0), dict(causal=2),
+                                 dict(num_heads=6, num_kv_heads=4)])
+def test_invalid_prefill_params_are_rejected(binding, bad):
+    base = dict(batch=1, num_heads=4, num_kv_heads=0, seq_len=16, head_dim=128, in_dtype=1, out_dtype=1,
+                scale=0.088, causal=1)
+    base.update(bad)
+    p = binding.PrefillParams(**base)
+    st = binding.lib.parallax_prefill(None, None, None, None, None, ctypes.byref(p), None)
+    assert st in (1, 2)
+
+
+def _expected_plan(B, units, L, num_sms=148, forced=0):
+    tiles = -(-L // 64)
+    if forced:
+        tps = -(-tiles // forced)
+    else:
+        want = -(-(4 * num_sms) // units)
+        tps = min(max(-(-tiles // want), 2), 64)
+    tps = max(1, min(tps, tiles))
+    return -(-tiles // tps)
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L,forced", [
+    (8, 16, 8, 4096, 0), (64, 32, 8, 32768, 0), (128, 16, 4, 65536, 0), (1, 1, 1, 256, 0),
+    (1, 4, 4, 65, 0), (8, 16, 8, 4096, 3), (2, 2, 1, 100, 16), (4, 8, 2, 1, 0),
+])
+def test_split_plan_and_workspace_size(binding, B, Hq, Hkv, L, forced):
+    p = _params(binding, batch=B, num_q_heads=Hq, num_kv_heads=Hkv, kv_len=L, num_splits=forced)
+    splits = binding.lib.parallax_decode_num_splits(ctypes.byref(p), 148)
+    assert splits == _expected_plan(B, B * Hkv, L, forced=forced)
+    ws = binding.lib.parallax_decode_workspace_size(ctypes.byref(p), 148)
+    if splits == 1:
+        assert ws == 0
+    else:
+        counters = -(-(B * Hq * 4) // 256) * 256
+        assert ws == counters + splits * B * Hq * (2 * 128 + 4) * 4
+
+
+def test_no_cpu_fallback(binding):
+    q = torch.zeros(1, 1, 64)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.decode(q, q, torch.zeros(1, 1, 4, 64), torch.zeros(1, 1, 4, 64))

@@ -1,0 +1,230 @@
+"""GPU parity of Parallax decode against the float64 oracle.
+
+Every case runs the CUDA path through the C ABI (the ctypes binding) and the
+oracle on the same seeded inputs, and checks
+    max |gpu - ref| <= tol * (1 + |ref|),  tol = 1e-5 (fp32), 2e-2 (bf16).
+Shapes span several 64-token tiles, ragged tails, GQA groups and split
+counts; the named workloads run at full size with sampled heads.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from parallax_local_linear_b200 import workloads as W
+from tests.helpers import TOL_BF16, TOL_F32, assert_parity, oracle_heads, parity_error
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def px():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from parallax_local_linear_b200 import binding
+    return binding
+
+
+def _to(inp, device=DEV):
+    return {k: (v.to(device) if torch.is_tensor(v) else v) for k, v in inp.items()}
+
+
+def _run(px, inp, **kw):
+    return px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"],
+                     seq_lens=inp.get("seq_lens"), page_table=inp.get("page_table"), **kw)
+
+
+def _all_heads(inp):
+    B, Hq, _ = inp["q"].shape
+    return [(b, h) for b in range(B) for h in range(Hq)]
+
+
+def _check_no_device_error(px):
+    assert px.last_device_error() == 0
+
+
+# ----------------------------------------------------------------- workloads
+
+def test_decode_f32_workload(px):
+    w = W.WORKLOADS["decode_f32"]
+    inp = W.decode_inputs(w, device=DEV)
+    out = _run(px, inp)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert out.dtype == torch.float32
+    assert_parity(out.cpu().numpy(), ref, TOL_F32, "decode_f32")
+    _check_no_device_error(px)
+
+
+def test_decode_bf16_workload(px):
+    w = W.WORKLOADS["decode_bf16"]
+    inp = W.decode_inputs(w, device=DEV)
+    out = _run(px, inp)
+    assert out.dtype == torch.bfloat16
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.float().cpu().numpy(), ref, TOL_BF16, "decode_bf16")
+    _check_no_device_error(px)
+
+
+def test_decode_long_workload_sampled(px):
+    w = W.WORKLOADS["decode_long"]
+    inp = W.decode_inputs(w, device=DEV)
+    out = _run(px, inp).float().cpu().numpy()
+    heads = [(0, 0), (0, 31), (17, 5), (40, 12), (63, 30), (63, 3)]
+    ref = oracle_heads(inp, heads)
+    for b, h in heads:
+        assert_parity(out[b, h], ref[b, h], TOL_BF16, f"decode_long ({b},{h})")
+    assert np.isfinite(out).all()
+    _check_no_device_error(px)
+    del inp
+    torch.cuda.empty_cache()
+
+
+def test_decode_paged_workload_sampled(px):
+    w = W.WORKLOADS["decode_paged"]
+    inp = W.decode_inputs(w, device=DEV)
+    out = _run(px, inp).float().cpu().numpy()
+    lens = inp["seq_lens"].cpu().numpy()
+    b_short, b_long = int(np.argmin(lens)), int(np.argmax(lens))
+    heads = [(b_short, 0), (b_short, 15), (b_long, 4), (b_long, 11), (7, 2), (100, 9)]
+    ref = oracle_heads(inp, heads)
+    for b, h in heads:
+        assert_parity(out[b, h], ref[b, h], TOL_BF16, f"decode_paged ({b},{h}) len={lens[b]}")
+    assert np.isfinite(out).all()
+    _check_no_device_error(px)
+    del inp
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------- sweeps
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("L", [1, 2, 63, 64, 65, 200, 1000, 4097])
+@pytest.mark.parametrize("group", [1, 2, 4, 8])
+def test_bf16_shapes(px, d, L, group):
+    inp = _to(W.small_decode_inputs(2, 2 * group, 2, d, L, seed=L * 10 + group))
+    out = _run(px, inp, out_dtype=torch.float32)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.cpu().numpy(), ref, TOL_BF16, f"d={d} L={L} g={group}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("L", [1, 31, 64, 65, 257, 1000])
+@pytest.mark.parametrize("group", [1, 3])
+def test_f32_shapes(px, d, L, group):
+    inp = _to(W.small_decode_inputs(2, 2 * group, 2, d, L, dtype="f32", seed=L + group))
+    out = _run(px, inp)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.cpu().numpy(), ref, TOL_F32, f"f32 d={d} L={L} g={group}")
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 16, 0])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_split_counts_agree(px, splits, dtype):
+    inp = _to(W.small_decode_inputs(3, 8, 2, 128, 1500, dtype=dtype, seq_lens=[1500, 700, 65], seed=5))
+    out = _run(px, inp, num_splits=splits, out_dtype=torch.float32)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.cpu().numpy(), ref, TOL_F32 if dtype == "f32" else TOL_BF16, f"splits={splits}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_ragged_lengths_with_nan_tails(px, dtype):
+    lens = [1, 63, 64, 65, 128, 129, 700, 0]
+    inp = _to(W.small_decode_inputs(8, 4, 2, 128, 768, dtype=dtype, seq_lens=lens, seed=11))
+    out = _run(px, inp, out_dtype=torch.float32).cpu().numpy()
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert np.isfinite(out).all(), "a NaN row past a sequence end leaked into the output"
+    assert_parity(out, ref, TOL_F32 if dtype == "f32" else TOL_BF16, "ragged")
+    np.testing.assert_array_equal(out[7], 0.0)   # empty sequence -> zero output
+
+
+@pytest.mark.parametrize("splits", [1, 4])
+def test_paged_is_bit_identical_to_contiguous(px, splits):
+    lens = [300, 64, 1, 129]
+    inp = _to(W.small_decode_inputs(4, 8, 2, 128, 320, seq_lens=lens, paged=True, seed=3))
+    paged = _run(px, inp, num_splits=splits, out_dtype=torch.float32)
+    contig = px.decode(inp["q"], inp["rho"], inp["k_contig"], inp["v_contig"], inp["scale"],
+                       seq_lens=inp["seq_lens"], num_splits=splits, out_dtype=torch.float32)
+    assert torch.equal(paged, contig)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(paged.cpu().numpy(), ref, TOL_BF16, "paged")
+
+
+def test_noncentred_keys_and_values(px):
+    # Keys share a large offset per KV head (the output is invariant to it)
+    # and values a common shift; the a_ref shift keeps the products small.
+    inp = _to(W.small_decode_inputs(2, 8, 2, 128, 2000, key_offset_std=4.0, value_offset=3.0, seed=9))
+    out = _run(px, inp, out_dtype=torch.float32)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.cpu().numpy(), ref, TOL_BF16, "non-centred")
+
+
+def test_rho_zero_matches_softmax_attention_reference(px):
+    inp = _to(W.small_decode_inputs(2, 4, 2, 128, 777, seed=21))
+    inp["rho"] = torch.zeros_like(inp["rho"])
+    out = _run(px, inp, out_dtype=torch.float32)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.cpu().numpy(), ref, TOL_BF16, "rho=0")
+
+
+def test_output_guard_bands_untouched(px):
+    inp = _to(W.small_decode_inputs(2, 4, 2, 128, 500, seed=4))
+    n = inp["q"].numel()
+    buf = torch.full((n + 2048,), 12345.0, dtype=torch.float32, device=DEV)
+    out = buf[1024:1024 + n].view(inp["q"].shape)
+    _run(px, inp, out=out, out_dtype=torch.float32, num_splits=3)
+    torch.cuda.synchronize()
+    assert (buf[:1024] == 12345.0).all() and (buf[1024 + n:] == 12345.0).all()
+
+
+def test_repeated_calls_are_deterministic(px):
+    inp = _to(W.small_decode_inputs(4, 8, 2, 128, 3000, seed=8))
+    a = _run(px, inp, num_splits=7)
+    b = _run(px, inp, num_splits=7)
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------ device errors
+
+def test_bad_page_id_sets_error_word(px):
+    inp = _to(W.small_decode_inputs(2, 4, 2, 128, 200, seq_lens=[200, 100], paged=True, seed=6))
+    assert px.last_device_error() == 0
+    table = inp["page_table"].clone()
+    table[1, 0] = 10 ** 6
+    px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"],
+              seq_lens=inp["seq_lens"], page_table=table)
+    assert px.last_device_error() & px.DEVERR_BAD_PAGE
+    assert px.last_device_error() == 0   # reading clears it
+
+
+def test_bad_length_sets_error_word(px):
+    inp = _to(W.small_decode_inputs(2, 4, 2, 128, 200, seed=6))
+    lens = torch.tensor([200, 500], dtype=torch.int32, device=DEV)
+    px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"], seq_lens=lens)
+    assert px.last_device_error() & px.DEVERR_BAD_LENGTH
+
+
+def test_workspace_too_small_is_rejected(px):
+    import ctypes
+    inp = _to(W.small_decode_inputs(2, 4, 2, 128, 2000, seed=1))
+    p = px.decode_params(inp["q"], inp["k_cache"], num_splits=4)
+    need = px.decode_workspace_size(p)
+    assert need > 0
+    ws = torch.zeros(need - 256, dtype=torch.uint8, device=DEV)
+    out = torch.empty_like(inp["q"])
+    st = px.lib.parallax_decode(px._ptr(inp["q"]), px._ptr(inp["rho"]), px._ptr(inp["k_cache"]),
+                                px._ptr(inp["v_cache"]), None, None, px._ptr(out), px._ptr(ws),
+                                ws.numel(), ctypes.byref(p), px._stream_ptr(inp["q"].device))
+    assert st == 3
+
+
+@pytest.mark.parametrize("L", [2, 3, 5, 9])
+@pytest.mark.parametrize("group", [2, 8])
+def test_short_sequences_keep_near_fp32_accuracy(px, L, group):
+    # With a handful of keys nothing averages out: the probe products e*a reach
+    # ~10 and must enter the value product without bf16 rounding.
+    inp = _to(W.small_decode_inputs(4, 2 * group, 2, 128, L, seed=100 + L))
+    out = _run(px, inp, out_dtype=torch.float32)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.cpu().numpy(), ref, 2e-3, f"short L={L} g={group}")
