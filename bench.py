@@ -1,0 +1,612 @@
+"""Benchmark of the Parallax attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the hot path over one batch: a decode call (single
+pass over the KV cache plus the split combine, one kernel launch) for the
+decode workloads, a causal prefill call for ``prefill``.  The default
+workload is decode_bf16: batch 8, 16 query / 8 KV heads, head_dim 128, KV
+length 4096, bf16 cache.
+
+Timing: W untimed warm-up steps, then exactly K steps between a barrier plus
+torch.cuda.synchronize() on both sides, timed with CUDA events on the stream
+the kernels run on; the max over ranks is reported.  Decode steps run as
+CUDA-graph replays (the library's kernels, captured once) so host launch cost
+does not hide the device time; every step reads a different copy of the KV
+cache, the copies totalling more than the 126 MB L2.  The ``e2e`` figure
+goes through the public Python API call by call, with the step's query and
+probe copied from pinned host memory and the output read back every step.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own copy of
+the workload (independent sequences, no collective on the data path), so
+scaling is weak and ``value`` is the total over ranks divided by the slowest
+rank's time.
+
+``--impl reference`` times the float64 CPU oracle on the host cores instead
+(rank 0 only), on a bounded sample of the same workload per step.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from parallax_local_linear_b200 import workloads as W  # noqa: E402
+
+METRIC = "decode KV GB/s & tokens/s (% of HBM peak); prefill TFLOP/s (% of bf16 peak)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {
+    "decode": ["parallax_local_linear_b200/csrc/decode.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "prefill": ["parallax_local_linear_b200/csrc/prefill.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
+}
+KV_COPIES = 4          # decode_bf16: 4 x 128 MiB of KV, more than L2
+GRAPH_STEPS = 64       # decode calls per captured graph
+
+
+# ---------------------------------------------------------------- helpers
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--workload", default="decode_bf16", choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args(argv)
+
+
+def default_steps(workload):
+    return {"decode_f32": 20000, "decode_bf16": 8192, "decode_long": 200, "decode_paged": 200,
+            "prefill": 20}[workload]
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_sha(kind):
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kind, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", f"{kind}-{workload}.md")
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and line.startswith("- "):
+                k, v = line[2:].split(":", 1)
+                fields[k.strip()] = v.strip().strip("`")
+    if fields.get("source_sha256") != source_sha(kind):
+        return None
+    try:
+        return float(fields["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index, period=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period
+        self._stop = threading.Event()
+        self._thr = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:   # NVML missing: report no clocks rather than guess
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for b, name in self.REASONS.items():
+                    if bits & b and b != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+class _F64View:
+    """float64 numpy slices of a (device) tensor, copied on indexing."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, idx):
+        return self.t[idx].double().cpu().numpy()
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i["num_threads"] for i in info if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ------------------------------------------------------------------ decode
+
+def decode_config(w, args, splits):
+    cfg = {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads,
+           "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "kv_len": w.kv_len,
+           "kv_dtype": w.dtype, "paged": w.paged, "num_splits": splits}
+    if w.paged:
+        cfg["seq_lens"] = f"uniform in [{w.min_len}, {w.kv_len}], 64-token pages, seeded permutation"
+    if w.key_offset_std:
+        cfg["key_offset_std"] = w.key_offset_std
+    return cfg
+
+
+def bench_decode(args, w, rank, world, dev, peaks, peaks_kind):
+    from parallax_local_linear_b200 import binding as px
+
+    copies = KV_COPIES if w.name in ("decode_bf16", "decode_f32") else 1
+    insts = [W.decode_inputs(w, device=dev, seed=w.seed + 1000 * rank + i) for i in range(copies)]
+    lens = [None if x["seq_lens"] is None else x["seq_lens"].cpu().numpy() for x in insts]
+    bytes_per_step = [W.kv_bytes(w, l) for l in lens]
+    outs = [torch.empty_like(x["q"]) for x in insts]
+    out_dtype = insts[0]["q"].dtype
+
+    def step(i):
+        x = insts[i % copies]
+        px.decode(x["q"], x["rho"], x["k_cache"], x["v_cache"], x["scale"], seq_lens=x["seq_lens"],
+                  page_table=x["page_table"], out=outs[i % copies], out_dtype=out_dtype,
+                  num_splits=args.num_splits)
+
+    p = px.decode_params(insts[0]["q"], insts[0]["k_cache"], page_table=insts[0]["page_table"],
+                         num_splits=args.num_splits)
+    splits = px.decode_num_splits(p)
+    stream = torch.cuda.current_stream()
+
+    # warm-up (also initialises the library and the workspace before capture)
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    assert px.last_device_error() == 0, "device error during warm-up"
+
+    K = args.steps
+    graphs = []
+    if w.name in ("decode_bf16", "decode_f32"):
+        g = torch.cuda.CUDAGraph()
+        n = min(GRAPH_STEPS, K)
+        with torch.cuda.graph(g):
+            for i in range(n):
+                step(i)
+        rem = K % n
+        gr = None
+        if rem:
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                for i in range(rem):
+                    step(i)
+        graphs = [(g, K // n), (gr, 1)] if gr is not None else [(g, K // n)]
+        for gg, _ in graphs:
+            gg.replay()
+        torch.cuda.synchronize()
+
+    def run_timed():
+        if graphs:
+            for gg, reps in graphs:
+                for _ in range(reps):
+                    gg.replay()
+        else:
+            for i in range(K):
+                step(i)
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record(stream)
+        run_timed()
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    assert px.last_device_error() == 0, "device error during the timed steps"
+    ms_max = ms
+    total_bytes = sum(bytes_per_step[i % copies] for i in range(K))
+    if world > 1:
+        t = torch.tensor([ms, float(total_bytes)], dtype=torch.float64, device=dev)
+        tm = t.clone()
+        torch.distributed.all_reduce(tm[:1], op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(t[1:], op=torch.distributed.ReduceOp.SUM)
+        ms_max, total_bytes = float(tm[0]), float(t[1])
+    gbs = total_bytes / (ms_max * 1e-3) / 1e9
+    tokens_per_s = w.batch * K * world / (ms_max * 1e-3)
+
+    # e2e: public API, q/rho from pinned host memory each step, output read back
+    e2e = e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world)
+
+    per_launch_bytes = sum(bytes_per_step) / copies
+    avg_launch_s = (ms * 1e-3) / K
+    achieved = per_launch_bytes / avg_launch_s / 1e9
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic("decode", w.name),
+                "peak_source": f"{peaks_kind} hbm_gbs", "kernel": "decode_tc_kernel" if w.dtype == "bf16"
+                else "decode_f32_kernel", "algorithmic_bytes_per_launch": int(per_launch_bytes)}
+    res = {
+        "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / K, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": dict(decode_config(w, args, splits),
+                       l2=("each step reads one of %d KV copies (%.0f MiB total > 126 MB L2)"
+                           % (copies, copies * per_launch_bytes / 2**20)) if copies > 1
+                       else "KV larger than L2", timing="CUDA-graph replay" if graphs else "stream"),
+        "tokens_per_s": round(tokens_per_s, 1),
+        "pct_of_hbm_peak": round(100 * gbs / world / peak, 2),
+        "roofline": roofline, "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
+    }
+    return res, insts
+
+
+def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
+    copies = len(insts)
+    host = []
+    for x in insts:
+        host.append({"q": x["q"].cpu().pin_memory(), "rho": x["rho"].cpu().pin_memory()})
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    K = min(args.steps, 2048)
+    dq = [torch.empty_like(x["q"]) for x in insts]
+    dr = [torch.empty_like(x["rho"]) for x in insts]
+
+    def one(i):
+        c = i % copies
+        x = insts[c]
+        dq[c].copy_(host[c]["q"], non_blocking=True)
+        dr[c].copy_(host[c]["rho"], non_blocking=True)
+        px.decode(dq[c], dr[c], x["k_cache"], x["v_cache"], x["scale"], seq_lens=x["seq_lens"],
+                  page_table=x["page_table"], out=outs[c], out_dtype=outs[c].dtype, num_splits=args.num_splits)
+        out_host[c].copy_(outs[c], non_blocking=True)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0 = time.perf_counter()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(K):
+        one(i)
+    end.record()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t[0])
+    total = sum(bytes_per_step[i % copies] for i in range(K)) * world
+    h2d = insts[0]["q"].numel() * insts[0]["q"].element_size() * 2
+    d2h = outs[0].numel() * outs[0].element_size()
+    return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "steps": K, "ms_per_step": round(ms / K, 6),
+            "host_wall_ms_per_step": round(1e3 * wall / K, 6),
+            "note": "query and probe copied from pinned host memory and output read back every step; "
+                    "the KV cache stays resident on the device"}
+
+
+# ----------------------------------------------------------------- prefill
+
+def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
+    from parallax_local_linear_b200 import binding as px
+
+    x = W.prefill_inputs(w, device=dev, seed=w.seed + 1000 * rank)
+    out = torch.empty_like(x["q"])
+
+    def step():
+        px.prefill(x["q"], x["rho"], x["k"], x["v"], causal=w.causal, scale=x["scale"], out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    assert px.last_device_error() == 0
+    K = args.steps
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record(stream)
+        for _ in range(K):
+            step()
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    ms_max = ms
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_max = float(t[0])
+    flops = W.prefill_flops(w)
+    tflops = flops * K * world / (ms_max * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved = flops / (ms * 1e-3 / K) / 1e12
+
+    # e2e through the public API: inputs copied from pinned host memory each step
+    hx = {k: x[k].cpu().pin_memory() for k in ("q", "rho", "k", "v")}
+    dx = {k: torch.empty_like(x[k]) for k in hx}
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    Ke = max(1, min(K, 10))
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(Ke):
+        for k in hx:
+            dx[k].copy_(hx[k], non_blocking=True)
+        px.prefill(dx["q"], dx["rho"], dx["k"], dx["v"], causal=w.causal, scale=x["scale"], out=out)
+        oh.copy_(out, non_blocking=True)
+    e2.record()
+    torch.cuda.synchronize()
+    ems = s2.elapsed_time(e2)
+    e2e = {"value": round(flops * Ke / (ems * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hx.values()),
+           "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": Ke}
+    res = {
+        "metric": METRIC, "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "num_heads": w.num_heads, "seq_len": w.seq_len,
+                   "head_dim": w.head_dim, "causal": w.causal, "rho_scale": w.rho_scale,
+                   "l2": "inputs 537 MB > 126 MB L2"},
+        "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic("prefill", w.name),
+                     "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_kernel",
+                     "algorithmic_flops_per_launch": flops},
+        "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
+    }
+    return res, x
+
+
+# ------------------------------------------------------------- CPU oracle
+
+def oracle_decode_sample(w, inp, budget_s, max_steps=None):
+    """Times the float64 oracle on whole KV-head units of the workload.
+
+    Returns (GB/s, seconds, units timed, description)."""
+    import oracle
+
+    B, Hq, Hkv = w.batch, w.num_q_heads, w.num_kv_heads
+    g = Hq // Hkv
+    units = [(b, kvh) for b in range(B) for kvh in range(Hkv)]
+    rng = np.random.default_rng(0)
+    rng.shuffle(units)
+    q = inp["q"].double().cpu().numpy()
+    rho = inp["rho"].double().cpu().numpy()
+    lens = None if inp["seq_lens"] is None else inp["seq_lens"].cpu().numpy()
+    table = None if inp["page_table"] is None else inp["page_table"].cpu().numpy()
+    done, secs, nbytes = 0, 0.0, 0
+    elt = 4 if w.dtype == "f32" else 2
+    for b, kvh in units:
+        n = w.kv_len if lens is None else int(lens[b])
+        if table is None:
+            K = inp["k_cache"][b, kvh, :n].double().cpu().numpy()
+            V = inp["v_cache"][b, kvh, :n].double().cpu().numpy()
+            kc = K[None, None]
+            vc = V[None, None]
+            heads = [(0, h) for h in range(g)]
+            qq, rr = q[b:b + 1, kvh * g:(kvh + 1) * g], rho[b:b + 1, kvh * g:(kvh + 1) * g]
+            t0 = time.perf_counter()
+            oracle.decode(qq, rr, kc, vc, w.scale, heads=heads)
+            secs += time.perf_counter() - t0
+        else:
+            kv = _F64View(inp["k_cache"])
+            vv = _F64View(inp["v_cache"])
+            t0 = time.perf_counter()
+            for h in range(kvh * g, (kvh + 1) * g):
+                oracle.decode(q, rho, kv, vv, w.scale, seq_lens=lens, page_table=table, heads=[(b, h)])
+            secs += time.perf_counter() - t0
+        nbytes += n * 2 * w.head_dim * elt
+        done += 1
+        if secs >= budget_s or (max_steps and done >= max_steps):
+            break
+    desc = (f"{done} of {len(units)} (sequence, KV head) units of {w.name}, all {g} query heads each "
+            f"({nbytes / 2**20:.1f} MiB of K+V), float64 numpy oracle")
+    return nbytes / secs / 1e9, secs, done, desc
+
+
+def cpu_baseline(w, inp, budget_s):
+    if w.name == "prefill":
+        return cpu_baseline_prefill(w, inp, budget_s)
+    gbs, secs, done, desc = oracle_decode_sample(w, inp, budget_s)
+    return {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": desc, "seconds": round(secs, 2)}
+
+
+def cpu_baseline_prefill(w, inp, budget_s):
+    import oracle
+    B, H, T = w.batch, w.num_heads, w.seq_len
+    rng = np.random.default_rng(1)
+    rows = [(int(rng.integers(B)), int(rng.integers(H)), int(t)) for t in rng.integers(0, T, size=4096)]
+    views = {k: _F64View(inp[k]) for k in ("q", "rho", "k", "v")}
+    secs, flops, n = 0.0, 0, 0
+    for r in rows:
+        t0 = time.perf_counter()
+        oracle.prefill_rows(views["q"], views["rho"], views["k"], views["v"], [r], w.scale, causal=True)
+        secs += time.perf_counter() - t0
+        flops += 8 * w.head_dim * (r[2] + 1)
+        n += 1
+        if secs >= budget_s:
+            break
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": f"{n} random rows of {w.name} (algorithmic FLOP of those rows)",
+            "seconds": round(secs, 2)}
+
+
+def reference_arm(args, w, rank, world):
+    """The float64 oracle on the host cores, on this workload's metric.
+
+    Each step times the oracle on a bounded sample of the workload (whole
+    (sequence, KV head) units for decode, random rows for prefill), sized so
+    that warm-up plus all steps take about two minutes."""
+    if rank != 0:
+        return None
+    budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
+    if w.name == "prefill":
+        sub = W.PrefillWorkload("prefill", 1, 1, w.seq_len, w.head_dim, rho_scale=w.rho_scale, seed=w.seed)
+        inp = W.prefill_inputs(sub, device="cpu")
+    elif w.batch * w.kv_len <= 2**20:
+        inp = W.decode_inputs(w, device="cpu")
+    else:
+        inp = _host_decode_sample(w)
+    vals, secs_all, desc = [], 0.0, ""
+    for i in range(args.warmup + args.steps):
+        if w.name == "prefill":
+            cb = cpu_baseline_prefill(w, inp, budget)
+            v, secs, desc = cb["value"], cb["seconds"], cb["sample"]
+        else:
+            sub_w = w if inp["q"].shape[0] == w.batch else W.DecodeWorkload(
+                w.name, inp["q"].shape[0], w.num_q_heads, w.num_kv_heads, w.head_dim, w.kv_len,
+                dtype=w.dtype, paged=w.paged, min_len=w.min_len)
+            v, secs, _, desc = oracle_decode_sample(sub_w, inp, budget)
+        if i >= args.warmup:
+            vals.append(v)
+            secs_all += secs
+    value = statistics.median(vals)
+    unit = "TFLOP/s" if w.name == "prefill" else "GB/s"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs_all / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name},
+            "cpu_baseline": {"value": round(value, 6), "unit": unit, "kind": "oracle", "cores": blas_threads(),
+                             "sample": "per step: " + desc},
+            "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def _host_decode_sample(w):
+    """Host-side inputs for a few sequences of a large decode workload (the
+    oracle's timing does not depend on which sequences are drawn)."""
+    n_seq = 2
+    sub = W.DecodeWorkload(w.name, n_seq, w.num_q_heads, w.num_kv_heads, w.head_dim, w.kv_len,
+                           dtype=w.dtype, key_offset_std=w.key_offset_std, paged=w.paged,
+                           min_len=w.min_len, seed=w.seed)
+    return W.decode_inputs(sub, device="cpu")
+
+
+# -------------------------------------------------------------------- main
+
+def main(argv=None):
+    args = parse_args(argv)
+    w = W.WORKLOADS[args.workload]
+    if args.steps is None:
+        args.steps = default_steps(args.workload) if args.impl == "ours" else 10
+    if args.warmup is None:
+        args.warmup = 20 if args.impl == "ours" else 2
+    rank, world, local = dist_env()
+
+    if args.impl == "reference":
+        res = reference_arm(args, w, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+
+    if not torch.cuda.is_available():
+        print(json.dumps({"error": "bench.py needs a CUDA device"}), flush=True)
+        return 1
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    peaks, kind = load_peaks()
+    try:
+        if w.name == "prefill":
+            res, inp = bench_prefill(args, w, rank, world, dev, peaks, kind)
+        else:
+            res, inp = bench_decode(args, w, rank, world, dev, peaks, kind)
+            inp = inp[0]
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
