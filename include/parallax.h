@@ -119,6 +119,34 @@ plx_status parallax_decode(const void* q, const void* rho,
                            void* out, void* workspace, size_t workspace_bytes,
                            const plx_decode_params* p, cudaStream_t stream);
 
+/* Decode that allocates nothing and takes no workspace.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory or own a workspace: a plugin running
+ * inside a host application that budgets all GPU memory itself, a binding
+ * from a language runtime that has no CUDA allocator of its own, or a
+ * latency-critical path that must not pay for cudaMalloc and the
+ * synchronisation it can imply.
+ *
+ * Same arguments and results as parallax_decode, minus the workspace.  The
+ * split partials live in a library-owned device array of
+ * PARALLAX_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library
+ * holds until the process exits.  The first call on a device looks up that
+ * array's device address (cudaGetSymbolAddress, with the device current);
+ * make that first call before any stream capture.  Each call clears the
+ * counter region of the array on `stream` before launching.  Calls share
+ * the one array: calls that overlap on the GPU (other streams, other host
+ * threads) race and give wrong results; serialise them.  Parameters whose
+ * parallax_decode_workspace_size() exceeds the array return
+ * PLX_ERR_WORKSPACE before any launch.  No cudaMalloc, cudaFree or
+ * allocating library routine is called. */
+#define PARALLAX_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+plx_status parallax_decode_noalloc(const void* q, const void* rho,
+                                   const void* k_cache, const void* v_cache,
+                                   const int32_t* page_table, const int32_t* seq_lens,
+                                   void* out, const plx_decode_params* p, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------
  * Prefill: every position of a sequence is a query; causal (key i visible
  * to query t iff i <= t) or full.  The same definition per row; the dense

@@ -61,6 +61,9 @@ lib.parallax_decode.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, _vp, ctyp
                                 ctypes.POINTER(DecodeParams), _vp]
 lib.parallax_prefill.restype = ctypes.c_int
 lib.parallax_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(PrefillParams), _vp]
+lib.parallax_decode_noalloc.restype = ctypes.c_int
+lib.parallax_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, ctypes.POINTER(DecodeParams), _vp]
+NOALLOC_SCRATCH_BYTES = 8 << 20
 lib.parallax_last_device_error.restype = ctypes.c_int
 lib.parallax_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
 
@@ -187,6 +190,25 @@ def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=No
                              ctypes.byref(p), _stream_ptr(q.device))
     if st != 0:
         raise ParallaxError(st, "parallax_decode")
+    return out
+
+
+def decode_noalloc(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=None, out, num_splits=0,
+                   kv_len=None):
+    """Decode through parallax_decode_noalloc: no workspace, no allocation.
+
+    For callers that cannot allocate device memory: ``out`` must be given,
+    and the library's fixed device scratch (NOALLOC_SCRATCH_BYTES per GPU)
+    holds the split partials.  Calls that overlap on the GPU race.
+    """
+    _check_cuda("q", q)
+    _check_cuda("out", out)
+    p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale, out_dtype=out.dtype,
+                      num_splits=num_splits)
+    st = lib.parallax_decode_noalloc(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                                     _ptr(seq_lens), _ptr(out), ctypes.byref(p), _stream_ptr(q.device))
+    if st != 0:
+        raise ParallaxError(st, "parallax_decode_noalloc")
     return out
 
 

@@ -175,6 +175,30 @@ plx_status validate_prefill(const plx_prefill_params* p) {
   return PLX_OK;
 }
 
+// ---------------------------------------------- decode without allocation
+// Scratch for parallax_decode_noalloc: split partials and their counters
+// live in this file-scope device array instead of a caller workspace.  Every
+// GPU that loads the library holds PARALLAX_NOALLOC_SCRATCH_BYTES of it
+// until the process exits.  In host code `g_noalloc_scratch` only names a
+// host-side stand-in for the symbol; its device address comes from
+// cudaGetSymbolAddress, looked up once per device with that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[PARALLAX_NOALLOC_SCRATCH_BYTES];
+
+void* g_noalloc_ptr[kMaxDevices];
+
+plx_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return PLX_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return PLX_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return PLX_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -287,6 +311,24 @@ plx_status parallax_prefill(const void* q, const void* rho, const void* k, const
   if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return PLX_ERR_INVALID_ARG;
   return launch_prefill(q, rho, k, v, out, p, stream);
+}
+
+plx_status parallax_decode_noalloc(const void* q, const void* rho, const void* k_cache, const void* v_cache,
+                                   const int32_t* page_table, const int32_t* seq_lens, void* out,
+                                   const plx_decode_params* p, cudaStream_t stream) {
+  plx_status st = validate_decode(p);
+  if (st != PLX_OK) return st;
+  const int num_sms = current_device_sms();
+  if (num_sms <= 0) return PLX_ERR_CUDA;
+  const DecodePlan pl = plan_decode(p, num_sms);
+  if (pl.counter_bytes + pl.partial_bytes > (size_t)PARALLAX_NOALLOC_SCRATCH_BYTES) return PLX_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != PLX_OK) return st;
+  // The counters must start at zero; the array keeps whatever the last call left.
+  if (pl.counter_bytes > 0 && cudaMemsetAsync(scratch, 0, pl.counter_bytes, stream) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  return parallax_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, scratch,
+                         (size_t)PARALLAX_NOALLOC_SCRATCH_BYTES, p, stream);
 }
 
 plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code) {
