@@ -67,7 +67,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=None)
     ap.add_argument("--workload", default="decode_bf16", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--num-ctas", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -202,10 +202,10 @@ def blas_threads():
 
 # ------------------------------------------------------------------ decode
 
-def decode_config(w, args, splits):
+def decode_config(w, args, ctas):
     cfg = {"workload": w.name, "batch": w.batch, "num_q_heads": w.num_q_heads,
            "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "kv_len": w.kv_len,
-           "kv_dtype": w.dtype, "paged": w.paged, "num_splits": splits}
+           "kv_dtype": w.dtype, "paged": w.paged, "num_ctas": ctas}
     if w.paged:
         cfg["seq_lens"] = f"uniform in [{w.min_len}, {w.kv_len}], 64-token pages, seeded permutation"
     if w.key_offset_std:
@@ -227,11 +227,11 @@ def bench_decode(args, w, rank, world, dev, peaks, peaks_kind):
         x = insts[i % copies]
         px.decode(x["q"], x["rho"], x["k_cache"], x["v_cache"], x["scale"], seq_lens=x["seq_lens"],
                   page_table=x["page_table"], out=outs[i % copies], out_dtype=out_dtype,
-                  num_splits=args.num_splits)
+                  num_ctas=args.num_ctas)
 
     p = px.decode_params(insts[0]["q"], insts[0]["k_cache"], page_table=insts[0]["page_table"],
-                         num_splits=args.num_splits)
-    splits = px.decode_num_splits(p)
+                         num_ctas=args.num_ctas)
+    ctas = px.decode_num_ctas(p)
     stream = torch.cuda.current_stream()
 
     # warm-up (also initialises the library and the workspace before capture)
@@ -308,7 +308,7 @@ def bench_decode(args, w, rank, world, dev, peaks, peaks_kind):
         "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms_max / K, 6), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": dict(decode_config(w, args, splits),
+        "config": dict(decode_config(w, args, ctas),
                        l2=("each step reads one of %d KV copies (%.0f MiB total > 126 MB L2)"
                            % (copies, copies * per_launch_bytes / 2**20)) if copies > 1
                        else "KV larger than L2", timing="CUDA-graph replay" if graphs else "stream"),
@@ -335,7 +335,7 @@ def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
         dq[c].copy_(host[c]["q"], non_blocking=True)
         dr[c].copy_(host[c]["rho"], non_blocking=True)
         px.decode(dq[c], dr[c], x["k_cache"], x["v_cache"], x["scale"], seq_lens=x["seq_lens"],
-                  page_table=x["page_table"], out=outs[c], out_dtype=outs[c].dtype, num_splits=args.num_splits)
+                  page_table=x["page_table"], out=outs[c], out_dtype=outs[c].dtype, num_ctas=args.num_ctas)
         out_host[c].copy_(outs[c], non_blocking=True)
 
     for i in range(3):

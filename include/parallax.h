@@ -68,7 +68,7 @@ typedef enum plx_dtype { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
  * over the KV stream), on the definition above.
  * ---------------------------------------------------------------------- */
 typedef struct plx_decode_params {
-  int32_t batch;              /* B >= 1                                        */
+  int32_t batch;              /* 1 <= B <= 8192                                */
   int32_t num_q_heads;        /* Hq, a multiple of num_kv_heads                */
   int32_t num_kv_heads;       /* Hkv; query head h reads KV head h / (Hq/Hkv)  */
   int32_t head_dim;           /* d: 64 or 128                                  */
@@ -80,21 +80,28 @@ typedef struct plx_decode_params {
   int32_t in_dtype;           /* plx_dtype of q, rho and the caches            */
   int32_t out_dtype;          /* plx_dtype of out                              */
   float scale;                /* softmax scale on q.k (e.g. 1/sqrt(d))         */
-  int32_t num_splits;         /* KV splits per sequence; 0 = choose            */
+  int32_t num_ctas;           /* persistent CTAs; 0 = one per SM (bf16) or
+                                 four per SM (fp32)                            */
 } plx_decode_params;
 
-/* Number of KV splits a decode call with these parameters uses on a device
- * with `num_sms` SMs (num_sms <= 0: the current device).  Host-only; makes
- * no CUDA call when num_sms > 0.  Returns -1 for invalid parameters. */
-int32_t parallax_decode_num_splits(const plx_decode_params* p, int32_t num_sms);
+/* Work decomposition.  The 64-token KV tiles of every (sequence, KV head)
+ * unit (bf16 caches; (sequence, query head) for fp32 caches) are laid end to
+ * end and cut into num_ctas equal contiguous chunks, one per persistent CTA
+ * (at most one CTA per tile).  A unit cut by chunk boundaries is finished by
+ * the last CTA to complete one of its pieces, in the same launch. */
 
-/* Workspace bytes parallax_decode needs (0 when it needs none), for
- * `num_sms` as above.  Returns (size_t)-1 for invalid parameters.
- * Layout: a counter region (one int32 per (sequence, KV head), padded to
- * 256 B) followed by fp32 split partials.  The counter region must be zero
- * before the workspace is first used (e.g. cudaMemsetAsync); every call
- * that completes leaves it zero again, so one zeroing lasts for the
- * workspace's lifetime. */
+/* CTAs a decode call with these parameters launches on a device with
+ * `num_sms` SMs (num_sms <= 0: the current device).  Host-only; makes no
+ * CUDA call when num_sms > 0.  Returns -1 for invalid parameters. */
+int32_t parallax_decode_num_ctas(const plx_decode_params* p, int32_t num_sms);
+
+/* Workspace bytes parallax_decode needs, for `num_sms` as above; it does not
+ * grow with the sequence lengths.  Returns (size_t)-1 for invalid
+ * parameters.  Layout: a counter region (one int32 per unit, padded to
+ * 256 B) followed by two fp32 partial slots per CTA.  The counter region
+ * must be zero before the workspace is first used (e.g. cudaMemsetAsync);
+ * every call that completes leaves it zero again, so one zeroing lasts for
+ * the workspace's lifetime. */
 size_t parallax_decode_workspace_size(const plx_decode_params* p, int32_t num_sms);
 
 /* Parallax decode.
@@ -110,7 +117,7 @@ size_t parallax_decode_workspace_size(const plx_decode_params* p, int32_t num_sm
  *   out         device, [B, Hq, d] of out_dtype (bf16 output is rounded to
  *               nearest even from fp32).
  *   workspace   device, >= parallax_decode_workspace_size() bytes, 256-byte
- *               aligned; may be NULL when that size is 0.
+ *               aligned.
  * Rows of the cache past a sequence's length are never used in arithmetic
  * (they may hold anything, NaN included). */
 plx_status parallax_decode(const void* q, const void* rho,

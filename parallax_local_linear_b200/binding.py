@@ -37,7 +37,7 @@ class DecodeParams(ctypes.Structure):
                 ("kv_len", ctypes.c_int32), ("page_size", ctypes.c_int32),
                 ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
                 ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
-                ("scale", ctypes.c_float), ("num_splits", ctypes.c_int32)]
+                ("scale", ctypes.c_float), ("num_ctas", ctypes.c_int32)]
 
 
 class PrefillParams(ctypes.Structure):
@@ -52,8 +52,8 @@ _vp, _i32p = ctypes.c_void_p, ctypes.c_void_p
 lib.parallax_abi_version.restype = ctypes.c_int32
 lib.parallax_status_string.restype = ctypes.c_char_p
 lib.parallax_status_string.argtypes = [ctypes.c_int]
-lib.parallax_decode_num_splits.restype = ctypes.c_int32
-lib.parallax_decode_num_splits.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_int32]
+lib.parallax_decode_num_ctas.restype = ctypes.c_int32
+lib.parallax_decode_num_ctas.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_int32]
 lib.parallax_decode_workspace_size.restype = ctypes.c_size_t
 lib.parallax_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_int32]
 lib.parallax_decode.restype = ctypes.c_int
@@ -123,7 +123,7 @@ def _workspace(device, nbytes):
 
 
 def decode_params(q, k_cache, *, page_table=None, kv_len=None, scale=None, out_dtype=None,
-                  num_splits=0, num_pages=None):
+                  num_ctas=0, num_pages=None):
     B, Hq, d = q.shape
     paged = page_table is not None
     Hkv = k_cache.shape[1]
@@ -140,7 +140,7 @@ def decode_params(q, k_cache, *, page_table=None, kv_len=None, scale=None, out_d
     scale = (1.0 / d ** 0.5) if scale is None else float(scale)
     out_dtype = q.dtype if out_dtype is None else out_dtype
     return DecodeParams(B, Hq, Hkv, d, L, PAGE_SIZE if paged else 0, n_pages, max_pages,
-                        _dtype_code(q.dtype), _dtype_code(out_dtype), scale, int(num_splits))
+                        _dtype_code(q.dtype), _dtype_code(out_dtype), scale, int(num_ctas))
 
 
 def decode_workspace_size(params: DecodeParams, num_sms: int = 0) -> int:
@@ -150,12 +150,12 @@ def decode_workspace_size(params: DecodeParams, num_sms: int = 0) -> int:
     return n
 
 
-def decode_num_splits(params: DecodeParams, num_sms: int = 0) -> int:
-    return lib.parallax_decode_num_splits(ctypes.byref(params), int(num_sms))
+def decode_num_ctas(params: DecodeParams, num_sms: int = 0) -> int:
+    return lib.parallax_decode_num_ctas(ctypes.byref(params), int(num_sms))
 
 
 def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=None, out=None,
-           out_dtype=None, num_splits=0, kv_len=None):
+           out_dtype=None, num_ctas=0, kv_len=None):
     """Parallax decode: out[b, h] = vbar - Sigma_KV^T rho[b, h] over sequence b.
 
     q, rho: [B, Hq, d] (bfloat16 or float32, the cache's dtype).
@@ -178,7 +178,7 @@ def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=No
     if seq_lens is not None:
         _check_cuda("seq_lens", seq_lens, torch.int32)
     p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale,
-                      out_dtype=out_dtype, num_splits=num_splits)
+                      out_dtype=out_dtype, num_ctas=num_ctas)
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     else:
@@ -193,7 +193,7 @@ def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=No
     return out
 
 
-def decode_noalloc(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=None, out, num_splits=0,
+def decode_noalloc(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=None, out, num_ctas=0,
                    kv_len=None):
     """Decode through parallax_decode_noalloc: no workspace, no allocation.
 
@@ -204,7 +204,7 @@ def decode_noalloc(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_
     _check_cuda("q", q)
     _check_cuda("out", out)
     p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale, out_dtype=out.dtype,
-                      num_splits=num_splits)
+                      num_ctas=num_ctas)
     st = lib.parallax_decode_noalloc(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
                                      _ptr(seq_lens), _ptr(out), ctypes.byref(p), _stream_ptr(q.device))
     if st != 0:

@@ -1,27 +1,31 @@
 // Parallax decode kernels for sm_100a.
 //
-// One CTA handles one split (a run of 64-token tiles) of one sequence for one
-// KV head (bf16 tensor-core path) or one query head (fp32 path).  It streams
-// every K and V row of its range exactly once and keeps, per query head, the
-// online-softmax running max m and the four sums of the single-pass form
-//     l = sum e_i,  c = sum e_i a_i,  O1 = sum e_i v_i,  O2 = sum e_i a_i v_i
-// with e_i = exp(scale q.k_i - m) and a_i = rho.k_i - a_ref.  The final
-// output is out = (O1/l)(1 + c/l) - O2/l, which equals vbar - S_KV^T rho
-// because the softmax weights sum to one (S_KV^T rho = O2/l - (c/l)(O1/l)).
-// This is the "single pass over the KV stream" that joins the softmax and
-// covariance branches (wispaper.ai blog "Parallax: Breaking the Boundary Bias
-// with Parameterized Local Linear Attention", section "Hardware Efficiency").
+// What one query computes.  For every KV token i, with e_i = exp(scale q.k_i - m)
+// and a_i = rho.k_i - a_ref, a CTA keeps the online-softmax running max m and
+// the four sums of the single-pass form
+//     l = sum e_i,  c = sum e_i a_i,  O1 = sum e_i v_i,  O2 = sum e_i a_i v_i,
+// and the output is out = (O1/l)(1 + c/l) - O2/l.  That equals vbar - S_KV^T rho
+// because the softmax weights sum to one (S_KV^T rho = O2/l - (c/l)(O1/l)), so
+// the covariance branch costs no byte beyond softmax attention's K and V: the
+// single pass over the KV stream that joins the softmax and covariance
+// branches (wispaper.ai blog "Parallax: Breaking the Boundary Bias with
+// Parameterized Local Linear Attention", section "Hardware Efficiency").
 //
-// a_ref = rho.k_0 (the first key of the sequence) is subtracted from every
-// a_i.  Any per-query constant leaves the output unchanged (O2 and c shift by
-// a_ref*O1 and a_ref*l, which cancel), and this one removes a common offset of
-// the keys from the products e*a before they are rounded and summed.
+// a_ref = rho.k_0 (first key of the sequence).  Any per-query constant leaves
+// the output unchanged (O2 and c shift by a_ref*O1 and a_ref*l, which cancel);
+// this one removes a common key offset from the products before they are
+// rounded and summed.
 //
-// Splits of one sequence combine like online softmax: with M = max_j m_j and
-// alpha_j = 2^(m_j - M), each of l, c, O1, O2 is the alpha-weighted sum.  The
-// last CTA of a sequence to finish (an atomic counter in the workspace, reset
-// by that CTA) combines the partials and writes the output, so one launch does
-// the whole decode.
+// Work decomposition (stream-K).  The 64-token tiles of all units (a unit is a
+// (sequence, KV head) on the bf16 path, a (sequence, query head) on the fp32
+// path) are laid end to end, unit after unit, and cut into gridDim.x equal
+// contiguous chunks, one per persistent CTA.  A CTA streams its chunk without
+// pause across unit boundaries.  A unit that lies inside one chunk is finished
+// by that CTA; a unit cut by chunk boundaries leaves one partial
+// (m, l, c, O1, O2) per piece, and the last CTA to finish a piece (an atomic
+// counter per unit, reset by that CTA) merges the pieces like online softmax:
+// with M = max_j m_j and alpha_j = 2^(m_j - M), each of l, c, O1, O2 is the
+// alpha-weighted sum.  One launch does the whole decode.
 #pragma once
 
 #include "ptx.cuh"
@@ -30,6 +34,7 @@ namespace plx {
 
 constexpr int kTile = 64;          // tokens per KV tile; equals the page size
 constexpr int kMaxGroup = 8;       // query heads per KV head on the bf16 path
+constexpr int kMaxBatch = 8192;    // sequences per call (prefix table in smem)
 
 struct DecodeArgs {
   const void* q;                   // [B, Hq, D]
@@ -39,25 +44,17 @@ struct DecodeArgs {
   const int32_t* page_table;       // [B, max_pages] or null
   const int32_t* seq_lens;         // [B] or null
   void* out;                       // [B, Hq, D]
-  float* partials;                 // [splits, B, Hq, 2D + 4]
-  int32_t* counters;               // [B * Hq]
+  float* slots;                    // [2 * gridDim.x][heads_per_unit][2D + 4]
+  int32_t* counters;               // [B * units_per_seq]
   int B, Hq, Hkv, group;
+  int units_per_seq;               // Hkv (bf16 path) or Hq (fp32 path)
+  int heads_per_unit;              // group (bf16 path) or 1 (fp32 path)
   int kv_len, paged, num_pages, max_pages;
-  int splits, tiles_per_split;
   float scale_log2;                // scale * log2(e)
   int out_bf16;
 };
 
-// Sequence length, clamped (and reported) when out of range.
-__device__ __forceinline__ int seq_len_of(const DecodeArgs& a, int b) {
-  if (a.seq_lens == nullptr) return a.kv_len;
-  int n = __ldg(a.seq_lens + b);
-  if (n < 0 || n > a.kv_len) {
-    report_error(4 /* PLX_DEVERR_BAD_LENGTH */);
-    n = n < 0 ? 0 : a.kv_len;
-  }
-  return n;
-}
+// ------------------------------------------------------------ addressing
 
 // Physical page of logical tile `tile` of sequence b (0 if out of range, reported).
 __device__ __forceinline__ int page_of(const DecodeArgs& a, int b, int tile) {
@@ -85,36 +82,132 @@ __device__ __forceinline__ void store_out(const DecodeArgs& a, size_t idx, float
     reinterpret_cast<float*>(a.out)[idx] = val;
 }
 
-// Merged state of one CTA: for each of its `nheads` heads, m, l, c and O1, O2.
+__device__ __forceinline__ float finalize(float o1, float o2, float l, float c) {
+  const float inv = 1.0f / l;
+  return o1 * inv * (1.0f + c * inv) - o2 * inv;
+}
+
+// ---------------------------------------------------------- the tile space
+//
+// pre[b] = number of tiles of all units of sequences before b; pre[B] = T.
+// lens[b] = length of sequence b (clamped to [0, kv_len], bad values reported).
+struct TileSpace {
+  const int* pre;
+  const int* lens;
+  int B, units;
+  long long T, G;
+
+  __device__ __forceinline__ int tiles_of(int b) const { return (pre[b + 1] - pre[b]) / units; }
+  __device__ __forceinline__ long long start(long long c) const { return c * T / G; }
+  // CTA whose chunk holds tile x.
+  __device__ __forceinline__ long long owner(long long x) const { return ((x + 1) * G + T - 1) / T - 1; }
+};
+
+// Fills pre[0..B] and lens[0..B) in shared memory; all threads of the CTA call it.
+__device__ void build_tile_space(const DecodeArgs& a, int* pre, int* lens, int* scratch) {
+  const int tid = threadIdx.x, nt = blockDim.x;
+  const int per = (a.B + nt - 1) / nt;
+  const int b0 = min(a.B, tid * per), b1 = min(a.B, b0 + per);
+  int sum = 0;
+  for (int b = b0; b < b1; ++b) {
+    int n = a.kv_len;
+    if (a.seq_lens != nullptr) {
+      n = __ldg(a.seq_lens + b);
+      if (n < 0 || n > a.kv_len) {
+        report_error(4 /* PLX_DEVERR_BAD_LENGTH */);
+        n = n < 0 ? 0 : a.kv_len;
+      }
+    }
+    lens[b] = n;
+    sum += ((n + kTile - 1) / kTile) * a.units_per_seq;
+  }
+  scratch[tid] = sum;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int i = 0; i < nt; ++i) {
+      const int v = scratch[i];
+      scratch[i] = run;
+      run += v;
+    }
+    pre[a.B] = run;
+  }
+  __syncthreads();
+  int run = scratch[tid];
+  for (int b = b0; b < b1; ++b) {
+    pre[b] = run;
+    run += ((lens[b] + kTile - 1) / kTile) * a.units_per_seq;
+  }
+  __syncthreads();
+}
+
+// Walks the units of a chunk in order.
+struct UnitCursor {
+  int b, hu, local, tiles;   // sequence, unit within it, tile within the unit, tiles per unit
+
+  __device__ __forceinline__ void seek(const TileSpace& ts, long long x) {
+    int lo = 0, hi = ts.B - 1;   // last b with pre[b] <= x
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (ts.pre[mid] <= x) lo = mid; else hi = mid - 1;
+    }
+    b = lo;
+    while (ts.pre[b + 1] <= x) ++b;   // skip empty sequences sharing the prefix
+    tiles = ts.tiles_of(b);
+    const int off = (int)(x - ts.pre[b]);
+    hu = off / tiles;
+    local = off % tiles;
+  }
+  __device__ __forceinline__ long long unit_begin(const TileSpace& ts) const {
+    return ts.pre[b] + (long long)hu * tiles;
+  }
+  __device__ __forceinline__ void next_tile(const TileSpace& ts) {
+    if (++local == tiles) next_unit(ts);
+  }
+  __device__ __forceinline__ void next_unit(const TileSpace& ts) {
+    local = 0;
+    if (++hu == ts.units) {
+      hu = 0;
+      do { ++b; } while (b < ts.B && ts.pre[b + 1] == ts.pre[b]);
+      if (b < ts.B) tiles = ts.tiles_of(b);
+    }
+  }
+};
+
+// Merged state of one unit: for each of its heads, m, l, c and O1, O2.
 template <int D>
 struct CtaState {
   float m[kMaxGroup], l[kMaxGroup], c[kMaxGroup];
   float o1[kMaxGroup][D], o2[kMaxGroup][D];
 };
 
-__device__ __forceinline__ float finalize(float o1, float o2, float l, float c) {
-  const float inv = 1.0f / l;
-  return o1 * inv * (1.0f + c * inv) - o2 * inv;
-}
-
-// Writes the CTA's result: the output directly when the sequence has one split,
-// otherwise a partial plus, in the last CTA to finish, the combine.  Called by
-// all `nthreads` threads of the CTA after `st` is complete and synchronised.
-template <int D>
-__device__ void finish_split(const DecodeArgs& a, const CtaState<D>& st, int nheads, int b, int hq0,
-                             int split, int nsplit, int counter_idx, int* s_flag) {
-  const int tid = threadIdx.x, nthreads = blockDim.x;
-  if (nsplit == 1) {
-    for (int i = tid; i < nheads * D; i += nthreads) {
+// Writes a unit's result: the output directly when this CTA holds the whole
+// unit, otherwise this piece's partial and, in the last CTA to finish a piece
+// of the unit, the merge of all pieces.  Called by the `nt` threads (ids
+// 0..nt-1) that synchronise through `bar`, after `st` is complete and
+// synchronised.
+template <int D, typename Bar>
+__device__ void finish_unit(const DecodeArgs& a, const TileSpace& ts, const CtaState<D>& st, int b, int hu,
+                            long long ua, long long ub, int tid, int nt, int* s_flag, Bar bar) {
+  const int nheads = a.heads_per_unit;
+  const int hq0 = hu * nheads;
+  const long long c = blockIdx.x;
+  const long long c0 = ts.owner(ua), c1 = ts.owner(ub - 1);
+  if (c0 == c1) {
+    for (int i = tid; i < nheads * D; i += nt) {
       const int h = i / D, d = i % D;
       store_out(a, ((size_t)b * a.Hq + hq0 + h) * D + d, finalize(st.o1[h][d], st.o2[h][d], st.l[h], st.c[h]));
     }
     return;
   }
   constexpr int P = 2 * D + 4;
-  for (int i = tid; i < nheads * (D + 1); i += nthreads) {
+  const size_t slot_stride = (size_t)nheads * P;
+  // Slot 2c holds a piece of CTA c's first unit, slot 2c + 1 of its last one.
+  auto slot_of = [&](long long cc) { return 2 * cc + (ts.start(cc) >= ua ? 0 : 1); };
+  float* mine = a.slots + slot_of(c) * slot_stride;
+  for (int i = tid; i < nheads * (D + 1); i += nt) {
     const int h = i / (D + 1), d = i % (D + 1);
-    float* part = a.partials + (((size_t)split * a.B + b) * a.Hq + hq0 + h) * P;
+    float* part = mine + h * P;
     if (d == D) {
       part[0] = st.m[h];
       part[1] = st.l[h];
@@ -125,25 +218,26 @@ __device__ void finish_split(const DecodeArgs& a, const CtaState<D>& st, int nhe
     }
   }
   __threadfence();
-  __syncthreads();
+  bar();
+  const int unit = b * a.units_per_seq + hu;
   if (tid == 0) {
-    const int prev = atomicAdd(a.counters + counter_idx, 1);
-    const int last = (prev == nsplit - 1);
-    if (last) atomicExch(a.counters + counter_idx, 0);
+    const int prev = atomicAdd(a.counters + unit, 1);
+    const int last = (prev == (int)(c1 - c0));
+    if (last) atomicExch(a.counters + unit, 0);
     *s_flag = last;
   }
-  __syncthreads();
-  if (!*s_flag) return;
+  bar();
+  const bool last = *s_flag != 0;
+  bar();   // everyone has read the flag before it can be reused
+  if (!last) return;
   __threadfence();
-  for (int i = tid; i < nheads * D; i += nthreads) {
+  for (int i = tid; i < nheads * D; i += nt) {
     const int h = i / D, d = i % D;
-    const float* base = a.partials + ((size_t)b * a.Hq + hq0 + h) * P;
-    const size_t sstride = (size_t)a.B * a.Hq * P;
     float M = -INFINITY;
-    for (int s = 0; s < nsplit; ++s) M = fmaxf(M, __ldcg(base + s * sstride));
+    for (long long cc = c0; cc <= c1; ++cc) M = fmaxf(M, __ldcg(a.slots + slot_of(cc) * slot_stride + h * P));
     float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
-    for (int s = 0; s < nsplit; ++s) {
-      const float* ps = base + s * sstride;
+    for (long long cc = c0; cc <= c1; ++cc) {
+      const float* ps = a.slots + slot_of(cc) * slot_stride + h * P;
       const float al = ex2(__ldcg(ps) - M);
       L += al * __ldcg(ps + 1);
       C += al * __ldcg(ps + 2);
@@ -154,44 +248,25 @@ __device__ void finish_split(const DecodeArgs& a, const CtaState<D>& st, int nhe
   }
 }
 
-// Split bookkeeping shared by both kernels.  Returns false when this CTA has no
-// work (after writing zeros for an empty sequence).
-struct SplitRange {
-  int len, nsplit, t_begin, t_end;  // tiles [t_begin, t_end) of the sequence
-};
-
-__device__ __forceinline__ bool split_range(const DecodeArgs& a, int b, int split, int hq0, int nheads,
-                                            int D, SplitRange& r) {
-  r.len = seq_len_of(a, b);
-  const int tiles = (r.len + kTile - 1) / kTile;
-  r.nsplit = (tiles + a.tiles_per_split - 1) / a.tiles_per_split;
-  if (r.len == 0) {
-    if (split == 0)
-      for (int i = threadIdx.x; i < nheads * D; i += blockDim.x)
-        store_out(a, ((size_t)b * a.Hq + hq0) * D + i, 0.f);
-    return false;
-  }
-  if (split >= r.nsplit) return false;
-  r.t_begin = split * a.tiles_per_split;
-  r.t_end = min(r.t_begin + a.tiles_per_split, tiles);
-  return true;
-}
-
 // =========================================================================
-// bf16 path: TMA ring + tensor cores (mma.sync m16n8k16, fp32 accumulate).
+// bf16 path: persistent CTAs, TMA ring, tensor cores (mma.sync m16n8k16,
+// bf16 inputs, fp32 accumulate).
 //
 // Warp roles: NC consumer warps and one producer warp.  The producer's lane 0
-// streams K and V tiles (64 tokens x D, bf16) into a STAGES-deep ring with
-// 2D TMA loads (128-byte swizzle, 64-column boxes).  Consumer warp w takes
-// tiles w, w + NC, ... of the split and keeps its own running state.
+// streams the chunk's K and V tiles (64 tokens x D, bf16) into a STAGES-deep
+// ring with 2D TMA loads (128-byte swizzle, 64-column boxes), straight across
+// unit boundaries.  Consumer warp w takes the chunk's tiles w, w + NC, ...;
+// each warp keeps its own running state per unit, and at the end of a unit
+// the consumer warps merge their states and finish the unit while the
+// producer keeps loading.
 //
 // Per tile a consumer computes, on tensor cores,
 //     [S; A] (16 x 64) = [Q; R] (16 x D) . K^T (D x 64)
 // where rows 0..g-1 of the 16-row operand are the group's queries and rows
 // 8..8+g-1 their probes (other rows zero).  The m16n8 accumulator layout then
 // gives each thread the score s and the probe value a of the same head (rows
-// h and h + 8) for the same two tokens.  It forms e and e*a in registers, packs
-// them as the A operand [P; P*A] of the second product
+// h and h + 8) for the same two tokens.  It forms e and e*a in registers and
+// packs them as the A operand [P; P*A] of the second product
 //     [O1; O2] (16 x D) += [P; P*A] (16 x 64) . V (64 x D)
 // so both accumulators come from one pass over each V tile.
 // =========================================================================
@@ -201,12 +276,15 @@ struct TcSmem {
   static constexpr int kBoxBytes = kTile * 128;              // 64 rows x 128 B
   static constexpr int kTileBytes = kBoxes * kBoxBytes;      // one K or V tile
   static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kWarpStateFloats = 16 * D + 24;       // m[8] l[8] c[8] O[16][D]
 };
 
 template <int D, int STAGES, int NC>
-constexpr int tc_smem_bytes() {
-  // ring + merged state + barriers + a_ref + flags + 1 KB alignment slack
-  return STAGES * TcSmem<D>::kStageBytes + (int)sizeof(CtaState<D>) + 2 * STAGES * 8 + 64 + 1024;
+constexpr int tc_smem_fixed_bytes() {
+  // ring + per-warp states + merged state + barriers + flags + scan scratch
+  // + 1 KB alignment slack (the prefix table, (2B + 1) ints, comes on top)
+  return STAGES * TcSmem<D>::kStageBytes + NC * TcSmem<D>::kWarpStateFloats * 4 + (int)sizeof(CtaState<D>) +
+         2 * STAGES * 8 + 16 + (NC + 1) * 32 * 4 + 1024;
 }
 
 template <int D, int STAGES, int NC, bool kLoInPad>
@@ -214,58 +292,44 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const DecodeArgs a) {
   using SM = TcSmem<D>;
-  static_assert(NC * (16 * D + 24) * 4 <= STAGES * SM::kStageBytes, "per-warp state must fit in the ring");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  CtaState<D>& st = *reinterpret_cast<CtaState<D>*>(ring + STAGES * SM::kStageBytes);
+  float* wstate = reinterpret_cast<float*>(ring + STAGES * SM::kStageBytes);
+  CtaState<D>& st = *reinterpret_cast<CtaState<D>*>(wstate + NC * SM::kWarpStateFloats);
   uint64_t* full = reinterpret_cast<uint64_t*>(&st + 1);
   uint64_t* empty = full + STAGES;
-  float* aref_s = reinterpret_cast<float*>(empty + STAGES);   // [8]
-  int* s_flag = reinterpret_cast<int*>(aref_s + 8);           // [0]: last-CTA flag, [1]: abort
+  int* s_flag = reinterpret_cast<int*>(empty + STAGES);    // [0]: last-piece flag, [1]: abort
+  int* scan = s_flag + 4;                                  // [(NC + 1) * 32]
+  int* pre = scan + (NC + 1) * 32;                          // [B + 1]
+  int* lens = pre + a.B + 1;                                // [B]
 
-  const int unit = blockIdx.x;
-  const int split = blockIdx.y;
-  const int b = unit / a.Hkv, kvh = unit % a.Hkv;
-  const int g = a.group;
-  const int hq0 = kvh * g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = a.group;
+  build_tile_space(a, pre, lens, scan);
 
-  SplitRange r;
-  if (!split_range(a, b, split, hq0, g, D, r)) return;
-  const int ntiles = r.t_end - r.t_begin;
+  // Sequences of length zero have no tiles: CTA b % gridDim.x writes their zeros.
+  for (int b = blockIdx.x; b < a.B; b += gridDim.x)
+    if (lens[b] == 0)
+      for (int i = threadIdx.x; i < a.Hq * D; i += blockDim.x) store_out(a, (size_t)b * a.Hq * D + i, 0.f);
+  // At most one CTA per tile, so that every chunk is non-empty.
+  const long long T = pre[a.B];
+  const long long G = T < (long long)gridDim.x ? T : (long long)gridDim.x;
+  if ((long long)blockIdx.x >= G) return;
+  TileSpace ts{pre, lens, a.B, a.units_per_seq, T, G};
+  const long long x0 = ts.start(blockIdx.x), x1 = ts.start(blockIdx.x + 1);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    s_flag[0] = 0;
     s_flag[1] = 0;
     fence_mbarrier_init();
   }
-  // a_ref[h] = rho_h . k_0, fp32, by warp 0.
-  if (warp == 0) {
-    const size_t row0 = cache_row(a, b, kvh, 0);
-    const __nv_bfloat16* k0 = reinterpret_cast<const __nv_bfloat16*>(a.k) + row0 * D;
-    for (int h = 0; h < kMaxGroup; ++h) {
-      float acc = 0.f;
-      if (h < g) {
-        const __nv_bfloat16* rh = reinterpret_cast<const __nv_bfloat16*>(a.rho) + ((size_t)b * a.Hq + hq0 + h) * D;
-        for (int d = lane; d < D; d += 32) acc += __bfloat162float(rh[d]) * __bfloat162float(k0[d]);
-        acc = warp_sum(acc);
-      }
-      if (lane == 0) aref_s[h] = acc;
-    }
-  }
   __syncthreads();
   volatile int* abort_flag = s_flag + 1;
-
-  // Consumer state (unused by the producer warp).
-  const int hr = lane >> 2;          // accumulator row (head) of this thread
-  const int qc = (lane & 3) * 2;     // column pair within an 8-wide chunk
-  float o[D / 8][4];
-#pragma unroll
-  for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_run = -INFINITY, l_part = 0.f, c_part = 0.f;
+  const int nchunk = (int)(x1 - x0);
 
   if (warp == NC) {
     // ------------------------------------------------------------ producer
@@ -273,17 +337,19 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
       prefetch_tmap(&tmap_k);
       prefetch_tmap(&tmap_v);
       const uint64_t pol = l2_policy_evict_first();
+      UnitCursor cur;
+      cur.seek(ts, x0);
       int issued = 0;
-      for (int t = 0; t < ntiles; ++t) {
+      for (int t = 0; t < nchunk; ++t) {
         const int s = t % STAGES;
         if (t >= STAGES && !mbar_wait_bounded(&empty[s], ((t / STAGES) - 1) & 1)) {
           *abort_flag = 1;
           break;
         }
         if (*abort_flag) break;
-        const int tile = r.t_begin + t;
-        const int row = a.paged ? (int)(((size_t)page_of(a, b, tile) * a.Hkv + kvh) * kTile)
-                                : (int)(((size_t)b * a.Hkv + kvh) * a.kv_len + (size_t)tile * kTile);
+        const int kvh = cur.hu;
+        const int row = a.paged ? (int)(((size_t)page_of(a, cur.b, cur.local) * a.Hkv + kvh) * kTile)
+                                : (int)(((size_t)cur.b * a.Hkv + kvh) * a.kv_len + (size_t)cur.local * kTile);
         uint8_t* kdst = ring + s * SM::kStageBytes;
         uint8_t* vdst = kdst + SM::kTileBytes;
         mbar_arrive_expect_tx(&full[s], SM::kStageBytes);
@@ -293,6 +359,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
           tma_load_2d(vdst + bx * SM::kBoxBytes, &tmap_v, bx * 64, row, &full[s], pol);
         }
         ++issued;
+        cur.next_tile(ts);
       }
       if (*abort_flag) {
         // Drain: wait (bounded) for the last load issued into each stage.
@@ -304,217 +371,256 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     }
   } else {
     // ------------------------------------------------------------ consumers
-    // [Q; R] A-operand fragments for every 16-wide k chunk.
-    uint32_t qa[D / 16][4];
-    {
-      const uint32_t* qrow = reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(a.q) +
-                                                               ((size_t)b * a.Hq + hq0 + hr) * D);
-      const uint32_t* rrow = reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(a.rho) +
-                                                               ((size_t)b * a.Hq + hq0 + hr) * D);
-      const bool live = hr < g;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const int c0 = (16 * kk + qc) / 2, c1 = (16 * kk + 8 + qc) / 2;
-        qa[kk][0] = live ? __ldg(qrow + c0) : 0u;
-        qa[kk][1] = live ? __ldg(rrow + c0) : 0u;
-        qa[kk][2] = live ? __ldg(qrow + c1) : 0u;
-        qa[kk][3] = live ? __ldg(rrow + c1) : 0u;
-      }
-    }
-    const float aref = aref_s[hr];
-
+    const int tid = threadIdx.x;
+    constexpr int NT = NC * 32;
+    auto bar = [] { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); };
+    const int hr = lane >> 2;          // accumulator row (head) of this thread
+    const int qc = (lane & 3) * 2;     // column pair within an 8-wide chunk
     const int rr = lane & 7, mi = lane >> 3;
-    for (int t = warp; t < ntiles; t += NC) {
-      const int s = t % STAGES;
-      if (*abort_flag) break;
-      if (!mbar_wait_bounded(&full[s], (t / STAGES) & 1)) {
-        *abort_flag = 1;
-        break;
-      }
-      uint8_t* kt = ring + s * SM::kStageBytes;
-      uint8_t* vt = kt + SM::kTileBytes;
-      const int tok0 = (r.t_begin + t) * kTile;
-      const int nvalid = min(kTile, r.len - tok0);
-      if (nvalid < kTile) {
-        // Zero V rows past the sequence end: their weight is 0, but 0 * NaN is not.
-        for (int i = lane; i < (kTile - nvalid) * SM::kBoxes * 8; i += 32) {
-          const int row = nvalid + i / (SM::kBoxes * 8);
-          const int rest = i % (SM::kBoxes * 8);
-          *reinterpret_cast<uint4*>(vt + (rest / 8) * SM::kBoxBytes + row * 128 + (rest % 8) * 16) =
-              make_uint4(0, 0, 0, 0);
+    float* ws = wstate + warp * SM::kWarpStateFloats;
+
+    UnitCursor cur;
+    cur.seek(ts, x0);
+    long long x = x0;
+    while (x < x1) {
+      const int b = cur.b, kvh = cur.hu, local0 = cur.local;
+      const long long ua = cur.unit_begin(ts), ub = ua + cur.tiles;
+      const long long seg_end = ub < x1 ? ub : x1;
+      const int len = lens[b];
+      const int hq0 = kvh * g;
+
+      // [Q; R] A-operand fragments of this unit, and a_ref = rho_h . k_0.
+      uint32_t qa[D / 16][4];
+      {
+        const bool live = hr < g;
+        const size_t qoff = ((size_t)b * a.Hq + hq0 + (live ? hr : 0)) * D;
+        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(a.q) + qoff);
+        const uint32_t* rrow =
+            reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(a.rho) + qoff);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int c0 = (16 * kk + qc) / 2, c1 = (16 * kk + 8 + qc) / 2;
+          qa[kk][0] = live ? __ldg(qrow + c0) : 0u;
+          qa[kk][1] = live ? __ldg(rrow + c0) : 0u;
+          qa[kk][2] = live ? __ldg(qrow + c1) : 0u;
+          qa[kk][3] = live ? __ldg(rrow + c1) : 0u;
         }
-        fence_proxy_async_smem();
-        __syncwarp();
       }
-      // ---- [S; A] = [Q; R] K^T
-      float sc[8][4];
+      float aref = 0.f;
+      {
+        const __nv_bfloat16* k0 = reinterpret_cast<const __nv_bfloat16*>(a.k) + cache_row(a, b, kvh, 0) * D;
+        float kv[D / 32];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
-      const uint32_t kb = smem_u32(kt);
+        for (int j = 0; j < D / 32; ++j) kv[j] = __bfloat162float(k0[lane + 32 * j]);
+        for (int h = 0; h < g; ++h) {
+          const __nv_bfloat16* rh = reinterpret_cast<const __nv_bfloat16*>(a.rho) + ((size_t)b * a.Hq + hq0 + h) * D;
+          float acc = 0.f;
 #pragma unroll
-      for (int k2 = 0; k2 < D / 32; ++k2) {
-        const uint32_t off = (k2 >> 1) * SM::kBoxBytes + rr * 128 + ((((k2 & 1) * 4 + mi) ^ rr) << 4);
+          for (int j = 0; j < D / 32; ++j) acc += __bfloat162float(rh[lane + 32 * j]) * kv[j];
+          acc = warp_sum(acc);
+          if (hr == h) aref = acc;
+        }
+      }
+
+      float o[D / 8][4];
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+      float m_run = -INFINITY, l_part = 0.f, c_part = 0.f;
+
+      const int i_begin = (int)(x - x0), i_end = (int)(seg_end - x0);
+      // first chunk-local tile index >= i_begin that this warp owns (t % NC == warp)
+      int t = i_begin + ((warp - i_begin % NC) + NC) % NC;
+      for (; t < i_end; t += NC) {
+        const int s = t % STAGES;
+        if (*abort_flag) break;
+        if (!mbar_wait_bounded(&full[s], (t / STAGES) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        uint8_t* kt = ring + s * SM::kStageBytes;
+        uint8_t* vt = kt + SM::kTileBytes;
+        const int tok0 = (local0 + (t - i_begin)) * kTile;
+        const int nvalid = min(kTile, len - tok0);
+        if (nvalid < kTile) {
+          // Zero V rows past the sequence end: their weight is 0, but 0 * NaN is not.
+          for (int i = lane; i < (kTile - nvalid) * SM::kBoxes * 8; i += 32) {
+            const int row = nvalid + i / (SM::kBoxes * 8);
+            const int rest = i % (SM::kBoxes * 8);
+            *reinterpret_cast<uint4*>(vt + (rest / 8) * SM::kBoxBytes + row * 128 + (rest % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        // ---- [S; A] = [Q; R] K^T
+        float sc[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+        const uint32_t kb = smem_u32(kt);
+#pragma unroll
+        for (int k2 = 0; k2 < D / 32; ++k2) {
+          const uint32_t off = (k2 >> 1) * SM::kBoxBytes + rr * 128 + ((((k2 & 1) * 4 + mi) ^ rr) << 4);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kb + off + j * 1024, b0, b1, b2, b3);
+            mma_bf16_16816(sc[j], qa[2 * k2], b0, b1);
+            mma_bf16_16816(sc[j], qa[2 * k2 + 1], b2, b3);
+          }
+        }
+        // ---- online softmax on this thread's row; mask tokens past the end
+        float mloc = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(kb + off + j * 1024, b0, b1, b2, b3);
-          mma_bf16_16816(sc[j], qa[2 * k2], b0, b1);
-          mma_bf16_16816(sc[j], qa[2 * k2 + 1], b2, b3);
-        }
-      }
-      // ---- online softmax on this thread's row; mask tokens past the end
-      float mloc = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const bool ok = 8 * j + qc + e < nvalid;
-          sc[j][e] = ok ? sc[j][e] * a.scale_log2 : -INFINITY;
-          sc[j][2 + e] = ok ? sc[j][2 + e] - aref : 0.f;
-          mloc = fmaxf(mloc, sc[j][e]);
-        }
-      }
-      mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
-      mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-      const float m_new = fmaxf(m_run, mloc);
-      const float alpha = ex2(m_run - m_new);
-      m_run = m_new;
-      l_part *= alpha;
-      c_part *= alpha;
-      // P and P*A enter the value product as bf16 hi + lo pairs (x = hi + lo
-      // with lo = x - bf16(x)), so the rounding of the weights stays near fp32
-      // level instead of 2^-9 relative: |a| is often ~10 for unit-scale
-      // probes, and a 2^-9 error on e*a would not average out for short
-      // sequences.  With g <= 4 the lo pairs ride in the zero-padding rows
-      // 4..7 / 12..15 (handed over from lane - 16), so they cost no extra
-      // MMA; otherwise a second MMA consumes them.
-      uint32_t pf[4][4], pl[4][4];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float p0 = ex2(sc[j][0] - m_new), p1 = ex2(sc[j][1] - m_new);
-        const float pa0 = p0 * sc[j][2], pa1 = p1 * sc[j][3];
-        l_part += p0 + p1;
-        c_part += pa0 + pa1;
-        const uint32_t hp = pack_bf16(p0, p1), ha = pack_bf16(pa0, pa1);
-        pf[j >> 1][(j & 1) * 2 + 0] = hp;
-        pf[j >> 1][(j & 1) * 2 + 1] = ha;
-        pl[j >> 1][(j & 1) * 2 + 0] = pack_bf16(p0 - bf16_lo_f(hp), p1 - bf16_hi_f(hp));
-        pl[j >> 1][(j & 1) * 2 + 1] = pack_bf16(pa0 - bf16_lo_f(ha), pa1 - bf16_hi_f(ha));
-      }
-      float alpha_o = alpha;
-      if (kLoInPad) {
-        const float a_from = __shfl_xor_sync(0xffffffffu, alpha, 16);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            const uint32_t from = __shfl_xor_sync(0xffffffffu, pl[jj][x], 16);
-            if (lane & 16) pf[jj][x] = from;
-          }
-        if (lane & 16) alpha_o = a_from;
-      }
-      if (alpha_o != 1.f) {
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-          o[i][0] *= alpha_o;
-          o[i][1] *= alpha_o;
-          o[i][2] *= alpha_o;
-          o[i][3] *= alpha_o;
-        }
-      }
-      // ---- [O1; O2] += [P; P*A] V
-      const uint32_t vb = smem_u32(vt);
-#pragma unroll
-      for (int n2 = 0; n2 < D / 16; ++n2) {
-        const int dcol = 16 * n2 + 8 * (mi >> 1);
-        const uint32_t off = (dcol >> 6) * SM::kBoxBytes + (rr + 8 * (mi & 1)) * 128 +
-                             ((((dcol & 63) >> 3) ^ rr) << 4);
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4_trans(vb + off + jj * 2048, b0, b1, b2, b3);
-          mma_bf16_16816(o[2 * n2], pf[jj], b0, b1);
-          mma_bf16_16816(o[2 * n2 + 1], pf[jj], b2, b3);
-          if (!kLoInPad) {
-            mma_bf16_16816(o[2 * n2], pl[jj], b0, b1);
-            mma_bf16_16816(o[2 * n2 + 1], pl[jj], b2, b3);
+          for (int e = 0; e < 2; ++e) {
+            const bool ok = 8 * j + qc + e < nvalid;
+            sc[j][e] = ok ? sc[j][e] * a.scale_log2 : -INFINITY;
+            sc[j][2 + e] = ok ? sc[j][2 + e] - aref : 0.f;
+            mloc = fmaxf(mloc, sc[j][e]);
           }
         }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-    }
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
-    l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
-    c_part += __shfl_xor_sync(0xffffffffu, c_part, 1);
-    c_part += __shfl_xor_sync(0xffffffffu, c_part, 2);
-  }
-  // The ring is idle from here on (every issued tile was consumed, or the
-  // producer drained what it issued): reuse it for the per-warp states.
-  __syncthreads();
-  if (warp < NC) {
-    float* ws = reinterpret_cast<float*>(ring) + warp * (16 * D + 3 * 8);
-    // layout per warp: m[8], l[8], c[8], O[16][D]
-    if ((lane & 3) == 0) {
-      ws[hr] = m_run;
-      ws[8 + hr] = l_part;
-      ws[16 + hr] = c_part;
-    }
-    float* wo = ws + 24;
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
+        mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
+        const float m_new = fmaxf(m_run, mloc);
+        const float alpha = ex2(m_run - m_new);
+        m_run = m_new;
+        l_part *= alpha;
+        c_part *= alpha;
+        // P and P*A enter the value product as bf16 hi + lo pairs (x = hi + lo
+        // with lo = x - bf16(x)), so the rounding of the weights stays near
+        // fp32 level instead of 2^-9 relative: |a| is often ~10 for unit-scale
+        // probes, and a 2^-9 error on e*a would not average out for short
+        // sequences.  With g <= 4 the lo pairs ride in the zero-padding rows
+        // 4..7 / 12..15 (handed over from lane - 16), so they cost no extra
+        // MMA; otherwise a second MMA consumes them.
+        uint32_t pf[4][4], pl[4][4];
 #pragma unroll
-    for (int i = 0; i < D / 8; ++i) {
-      wo[hr * D + 8 * i + qc] = o[i][0];
-      wo[hr * D + 8 * i + qc + 1] = o[i][1];
-      wo[(hr + 8) * D + 8 * i + qc] = o[i][2];
-      wo[(hr + 8) * D + 8 * i + qc + 1] = o[i][3];
-    }
-  }
-  __syncthreads();
-  // Merge the NC per-warp states into st (all threads).
-  {
-    const float* base = reinterpret_cast<const float*>(ring);
-    constexpr int W = 16 * D + 24;
-    for (int i = threadIdx.x; i < g * D; i += blockDim.x) {
-      const int h = i / D, d = i % D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < NC; ++w) M = fmaxf(M, base[w * W + h]);
-      float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
-#pragma unroll
-      for (int w = 0; w < NC; ++w) {
-        const float* ws = base + w * W;
-        const float al = ex2(ws[h] - M);   // a warp with no tiles has m = -inf -> 0
-        L += al * ws[8 + h];
-        C += al * ws[16 + h];
-        float o1 = ws[24 + h * D + d], o2 = ws[24 + (h + 8) * D + d];
-        if (kLoInPad) {   // rows h + 4 and h + 12 hold the lo-part products
-          o1 += ws[24 + (h + 4) * D + d];
-          o2 += ws[24 + (h + 12) * D + d];
+        for (int j = 0; j < 8; ++j) {
+          const float p0 = ex2(sc[j][0] - m_new), p1 = ex2(sc[j][1] - m_new);
+          const float pa0 = p0 * sc[j][2], pa1 = p1 * sc[j][3];
+          l_part += p0 + p1;
+          c_part += pa0 + pa1;
+          const uint32_t hp = pack_bf16(p0, p1), ha = pack_bf16(pa0, pa1);
+          pf[j >> 1][(j & 1) * 2 + 0] = hp;
+          pf[j >> 1][(j & 1) * 2 + 1] = ha;
+          pl[j >> 1][(j & 1) * 2 + 0] = pack_bf16(p0 - bf16_lo_f(hp), p1 - bf16_hi_f(hp));
+          pl[j >> 1][(j & 1) * 2 + 1] = pack_bf16(pa0 - bf16_lo_f(ha), pa1 - bf16_hi_f(ha));
         }
-        O1 += al * o1;
-        O2 += al * o2;
+        float alpha_o = alpha;
+        if (kLoInPad) {
+          const float a_from = __shfl_xor_sync(0xffffffffu, alpha, 16);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+            for (int xx = 0; xx < 4; ++xx) {
+              const uint32_t from = __shfl_xor_sync(0xffffffffu, pl[jj][xx], 16);
+              if (lane & 16) pf[jj][xx] = from;
+            }
+          if (lane & 16) alpha_o = a_from;
+        }
+        if (alpha_o != 1.f) {
+#pragma unroll
+          for (int i = 0; i < D / 8; ++i) {
+            o[i][0] *= alpha_o;
+            o[i][1] *= alpha_o;
+            o[i][2] *= alpha_o;
+            o[i][3] *= alpha_o;
+          }
+        }
+        // ---- [O1; O2] += [P; P*A] V
+        const uint32_t vb = smem_u32(vt);
+#pragma unroll
+        for (int n2 = 0; n2 < D / 16; ++n2) {
+          const int dcol = 16 * n2 + 8 * (mi >> 1);
+          const uint32_t off = (dcol >> 6) * SM::kBoxBytes + (rr + 8 * (mi & 1)) * 128 +
+                               ((((dcol & 63) >> 3) ^ rr) << 4);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_trans(vb + off + jj * 2048, b0, b1, b2, b3);
+            mma_bf16_16816(o[2 * n2], pf[jj], b0, b1);
+            mma_bf16_16816(o[2 * n2 + 1], pf[jj], b2, b3);
+            if (!kLoInPad) {
+              mma_bf16_16816(o[2 * n2], pl[jj], b0, b1);
+              mma_bf16_16816(o[2 * n2 + 1], pl[jj], b2, b3);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
       }
-      st.o1[h][d] = O1;
-      st.o2[h][d] = O2;
-      if (d == 0) {
-        st.m[h] = M;
-        st.l[h] = L;
-        st.c[h] = C;
+
+      // ---- end of this unit's segment: merge the warps, finish the unit
+      l_part += __shfl_xor_sync(0xffffffffu, l_part, 1);
+      l_part += __shfl_xor_sync(0xffffffffu, l_part, 2);
+      c_part += __shfl_xor_sync(0xffffffffu, c_part, 1);
+      c_part += __shfl_xor_sync(0xffffffffu, c_part, 2);
+      if ((lane & 3) == 0) {
+        ws[hr] = m_run;
+        ws[8 + hr] = l_part;
+        ws[16 + hr] = c_part;
       }
+      float* wo = ws + 24;
+#pragma unroll
+      for (int i = 0; i < D / 8; ++i) {
+        wo[hr * D + 8 * i + qc] = o[i][0];
+        wo[hr * D + 8 * i + qc + 1] = o[i][1];
+        wo[(hr + 8) * D + 8 * i + qc] = o[i][2];
+        wo[(hr + 8) * D + 8 * i + qc + 1] = o[i][3];
+      }
+      bar();
+      for (int i = tid; i < g * D; i += NT) {
+        const int h = i / D, d = i % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NC; ++w) M = fmaxf(M, wstate[w * SM::kWarpStateFloats + h]);
+        float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
+#pragma unroll
+        for (int w = 0; w < NC; ++w) {
+          const float* wsw = wstate + w * SM::kWarpStateFloats;
+          const float al = ex2(wsw[h] - M);   // a warp without tiles here has m = -inf -> 0
+          L += al * wsw[8 + h];
+          C += al * wsw[16 + h];
+          float o1 = wsw[24 + h * D + d], o2 = wsw[24 + (h + 8) * D + d];
+          if (kLoInPad) {   // rows h + 4 and h + 12 hold the lo-part products
+            o1 += wsw[24 + (h + 4) * D + d];
+            o2 += wsw[24 + (h + 12) * D + d];
+          }
+          O1 += al * o1;
+          O2 += al * o2;
+        }
+        st.o1[h][d] = O1;
+        st.o2[h][d] = O2;
+        if (d == 0) {
+          st.m[h] = M;
+          st.l[h] = L;
+          st.c[h] = C;
+        }
+      }
+      bar();
+      finish_unit<D>(a, ts, st, b, kvh, ua, ub, tid, NT, s_flag, bar);
+      bar();   // per-warp states and st are free again
+      x = seg_end;
+      cur.next_unit(ts);
     }
   }
   __syncthreads();
-  finish_split<D>(a, st, g, b, hq0, split, r.nsplit, b * a.Hq + hq0, s_flag);
 }
 
 // =========================================================================
-// fp32 path: CUDA-core FFMA, one CTA per (split, sequence, query head).
-//
-// Warp w takes 32-token chunks w, w + NW, ... of the split.  Lane j computes
-// the score and probe value of token j of the chunk (a full dot product over
-// D), the warp forms the chunk max and the weights, then every lane
-// accumulates O1 and O2 for its D/32 columns over the chunk's tokens.
+// fp32 path: CUDA-core FFMA, persistent CTAs over units (sequence, query
+// head).  Warp w takes the 32-token sub-chunks w, w + NW, ... of each unit
+// segment of the CTA's chunk.  Lane j computes the score and probe value of
+// token j of a sub-chunk (a full dot product over D); the warp forms the
+// sub-chunk max and the weights; then every lane accumulates O1 and O2 for
+// its D/32 columns over the sub-chunk's tokens.
 // =========================================================================
+template <int NW>
+constexpr int f32_smem_fixed_bytes() {
+  return (16 + NW * 32) * 4;   // flags + scan scratch (the prefix table, (2B + 1) ints, comes on top)
+}
+
 template <int D, int NW>
 __global__ void __launch_bounds__(NW * 32)
     decode_f32_kernel(const DecodeArgs a) {
@@ -522,114 +628,139 @@ __global__ void __launch_bounds__(NW * 32)
   __shared__ float s_qr[2][D];
   __shared__ float s_w[NW][3];
   __shared__ float s_o[NW][2][D];
-  __shared__ int s_flag[2];
+  extern __shared__ int smem_dyn[];
+  int* s_flag = smem_dyn;               // [0]: last-piece flag
+  int* scan = smem_dyn + 16;            // [NW * 32]
+  int* pre = scan + NW * 32;            // [B + 1]
+  int* lens = pre + a.B + 1;            // [B]
 
-  const int unit = blockIdx.x;    // b * Hq + hq
-  const int split = blockIdx.y;
-  const int b = unit / a.Hq, hq = unit % a.Hq;
-  const int kvh = hq / a.group;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+  constexpr int NT = NW * 32;
+  build_tile_space(a, pre, lens, scan);
+  for (int b = blockIdx.x; b < a.B; b += gridDim.x)
+    if (lens[b] == 0)
+      for (int i = tid; i < a.Hq * D; i += NT) store_out(a, (size_t)b * a.Hq * D + i, 0.f);
+  const long long T = pre[a.B];
+  const long long G = T < (long long)gridDim.x ? T : (long long)gridDim.x;
+  if ((long long)blockIdx.x >= G) return;
+  TileSpace ts{pre, lens, a.B, a.units_per_seq, T, G};
+  const long long x0 = ts.start(blockIdx.x), x1 = ts.start(blockIdx.x + 1);
+  auto bar = [] { __syncthreads(); };
 
-  SplitRange r;
-  if (!split_range(a, b, split, hq, 1, D, r)) return;
-
-  const float* qp = reinterpret_cast<const float*>(a.q) + ((size_t)b * a.Hq + hq) * D;
-  const float* rp = reinterpret_cast<const float*>(a.rho) + ((size_t)b * a.Hq + hq) * D;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    s_qr[0][d] = qp[d];
-    s_qr[1][d] = rp[d];
-  }
-  __syncthreads();
   const float* kc = reinterpret_cast<const float*>(a.k);
   const float* vc = reinterpret_cast<const float*>(a.v);
-  float aref;
-  {
-    const float* k0 = kc + cache_row(a, b, kvh, 0) * D;
-    float acc = 0.f;
-    for (int d = lane; d < D; d += 32) acc += s_qr[1][d] * k0[d];
-    aref = warp_sum(acc);
-  }
+  UnitCursor cur;
+  cur.seek(ts, x0);
+  long long x = x0;
+  while (x < x1) {
+    const int b = cur.b, hq = cur.hu, local0 = cur.local;
+    const int kvh = hq / a.group;
+    const long long ua = cur.unit_begin(ts), ub = ua + cur.tiles;
+    const long long seg_end = ub < x1 ? ub : x1;
+    const int len = lens[b];
 
-  float m_run = -INFINITY, l_lane = 0.f, c_lane = 0.f;
-  float o1[D / 32], o2[D / 32];
+    const float* qp = reinterpret_cast<const float*>(a.q) + ((size_t)b * a.Hq + hq) * D;
+    const float* rp = reinterpret_cast<const float*>(a.rho) + ((size_t)b * a.Hq + hq) * D;
+    for (int d = tid; d < D; d += NT) {
+      s_qr[0][d] = qp[d];
+      s_qr[1][d] = rp[d];
+    }
+    __syncthreads();
+    float aref;
+    {
+      const float* k0 = kc + cache_row(a, b, kvh, 0) * D;
+      float acc = 0.f;
+      for (int d = lane; d < D; d += 32) acc += s_qr[1][d] * k0[d];
+      aref = warp_sum(acc);
+    }
+
+    float m_run = -INFINITY, l_lane = 0.f, c_lane = 0.f;
+    float o1[D / 32], o2[D / 32];
 #pragma unroll
-  for (int i = 0; i < D / 32; ++i) o1[i] = o2[i] = 0.f;
+    for (int i = 0; i < D / 32; ++i) o1[i] = o2[i] = 0.f;
 
-  const int tok_begin = r.t_begin * kTile;
-  const int tok_end = min(r.t_end * kTile, r.len);
-  for (int c0 = tok_begin + warp * 32; c0 < tok_end; c0 += NW * 32) {
-    const int tok = c0 + lane;
-    const int nvalid = min(32, tok_end - c0);
-    float x = -INFINITY, av = 0.f;
-    if (lane < nvalid) {
-      const float4* kr = reinterpret_cast<const float4*>(kc + cache_row(a, b, kvh, tok) * D);
-      float s = 0.f, pr = 0.f;
+    const int tok_begin = local0 * kTile;
+    const int tok_end = min((local0 + (int)(seg_end - x)) * kTile, len);
+    for (int c0 = tok_begin + warp * 32; c0 < tok_end; c0 += NW * 32) {
+      const int tok = c0 + lane;
+      const int nvalid = min(32, tok_end - c0);
+      float xs = -INFINITY, av = 0.f;
+      if (lane < nvalid) {
+        const float4* kr = reinterpret_cast<const float4*>(kc + cache_row(a, b, kvh, tok) * D);
+        float s = 0.f, pr = 0.f;
 #pragma unroll 8
-      for (int d4 = 0; d4 < D / 4; ++d4) {
-        const float4 kv = kr[d4];
-        s += s_qr[0][4 * d4] * kv.x + s_qr[0][4 * d4 + 1] * kv.y + s_qr[0][4 * d4 + 2] * kv.z + s_qr[0][4 * d4 + 3] * kv.w;
-        pr += s_qr[1][4 * d4] * kv.x + s_qr[1][4 * d4 + 1] * kv.y + s_qr[1][4 * d4 + 2] * kv.z + s_qr[1][4 * d4 + 3] * kv.w;
+        for (int d4 = 0; d4 < D / 4; ++d4) {
+          const float4 kv = kr[d4];
+          s += s_qr[0][4 * d4] * kv.x + s_qr[0][4 * d4 + 1] * kv.y + s_qr[0][4 * d4 + 2] * kv.z +
+               s_qr[0][4 * d4 + 3] * kv.w;
+          pr += s_qr[1][4 * d4] * kv.x + s_qr[1][4 * d4 + 1] * kv.y + s_qr[1][4 * d4 + 2] * kv.z +
+                s_qr[1][4 * d4 + 3] * kv.w;
+        }
+        xs = s * a.scale_log2;
+        av = pr - aref;
       }
-      x = s * a.scale_log2;
-      av = pr - aref;
-    }
-    const float m_new = fmaxf(m_run, warp_max(x));
-    const float alpha = ex2(m_run - m_new);
-    m_run = m_new;
-    const float p = ex2(x - m_new);
-    const float pa = p * av;
-    l_lane = l_lane * alpha + p;
-    c_lane = c_lane * alpha + pa;
-#pragma unroll
-    for (int i = 0; i < D / 32; ++i) {
-      o1[i] *= alpha;
-      o2[i] *= alpha;
-    }
-    for (int j = 0; j < nvalid; ++j) {
-      const float pj = __shfl_sync(0xffffffffu, p, j);
-      const float paj = __shfl_sync(0xffffffffu, pa, j);
-      const float* vr = vc + cache_row(a, b, kvh, c0 + j) * D;
+      const float m_new = fmaxf(m_run, warp_max(xs));
+      const float alpha = ex2(m_run - m_new);
+      m_run = m_new;
+      const float p = ex2(xs - m_new);
+      const float pa = p * av;
+      l_lane = l_lane * alpha + p;
+      c_lane = c_lane * alpha + pa;
 #pragma unroll
       for (int i = 0; i < D / 32; ++i) {
-        const float vv = vr[lane + 32 * i];
-        o1[i] += pj * vv;
-        o2[i] += paj * vv;
+        o1[i] *= alpha;
+        o2[i] *= alpha;
+      }
+      for (int j = 0; j < nvalid; ++j) {
+        const float pj = __shfl_sync(0xffffffffu, p, j);
+        const float paj = __shfl_sync(0xffffffffu, pa, j);
+        const float* vr = vc + cache_row(a, b, kvh, c0 + j) * D;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) {
+          const float vv = vr[lane + 32 * i];
+          o1[i] += pj * vv;
+          o2[i] += paj * vv;
+        }
       }
     }
-  }
-  const float l_w = warp_sum(l_lane), c_w = warp_sum(c_lane);
-  if (lane == 0) {
-    s_w[warp][0] = m_run;
-    s_w[warp][1] = l_w;
-    s_w[warp][2] = c_w;
-  }
+    const float l_w = warp_sum(l_lane), c_w = warp_sum(c_lane);
+    if (lane == 0) {
+      s_w[warp][0] = m_run;
+      s_w[warp][1] = l_w;
+      s_w[warp][2] = c_w;
+    }
 #pragma unroll
-  for (int i = 0; i < D / 32; ++i) {
-    s_o[warp][0][lane + 32 * i] = o1[i];
-    s_o[warp][1][lane + 32 * i] = o2[i];
-  }
-  __syncthreads();
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float M = -INFINITY;
-    for (int w = 0; w < NW; ++w) M = fmaxf(M, s_w[w][0]);
-    float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
-    for (int w = 0; w < NW; ++w) {
-      const float al = ex2(s_w[w][0] - M);
-      L += al * s_w[w][1];
-      C += al * s_w[w][2];
-      O1 += al * s_o[w][0][d];
-      O2 += al * s_o[w][1][d];
+    for (int i = 0; i < D / 32; ++i) {
+      s_o[warp][0][lane + 32 * i] = o1[i];
+      s_o[warp][1][lane + 32 * i] = o2[i];
     }
-    st.o1[0][d] = O1;
-    st.o2[0][d] = O2;
-    if (d == 0) {
-      st.m[0] = M;
-      st.l[0] = L;
-      st.c[0] = C;
+    __syncthreads();
+    for (int d = tid; d < D; d += NT) {
+      float M = -INFINITY;
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, s_w[w][0]);
+      float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
+      for (int w = 0; w < NW; ++w) {
+        const float al = ex2(s_w[w][0] - M);
+        L += al * s_w[w][1];
+        C += al * s_w[w][2];
+        O1 += al * s_o[w][0][d];
+        O2 += al * s_o[w][1][d];
+      }
+      st.o1[0][d] = O1;
+      st.o2[0][d] = O2;
+      if (d == 0) {
+        st.m[0] = M;
+        st.l[0] = L;
+        st.c[0] = C;
+      }
     }
+    __syncthreads();
+    finish_unit<D>(a, ts, st, b, hq, ua, ub, tid, NT, s_flag, bar);
+    __syncthreads();
+    x = seg_end;
+    cur.next_unit(ts);
   }
-  __syncthreads();
-  finish_split<D>(a, st, 1, b, hq, split, r.nsplit, unit, s_flag);
 }
 
 }  // namespace plx

@@ -1,6 +1,6 @@
 // libparallax.so: the C ABI declared in include/parallax.h.
 //
-// Host side of every entry point: argument validation, the split plan of a
+// Host side of every entry point: argument validation, the work plan of a
 // decode call, TMA tensor maps, kernel launches.  All arithmetic of the path
 // runs in the kernels included below; nothing here touches tensor data.
 #include "parallax.h"
@@ -30,13 +30,8 @@ constexpr int kDecodeStages128 = 4;
 constexpr int kDecodeStages64 = 6;
 constexpr int kDecodeF32Warps = 4;
 
-// Tiles per split: a split covers at least kMinTilesPerSplit and at most
-// kMaxTilesPerSplit 64-token tiles; within that range the split count aims at
-// kTargetCtasPerSm CTAs per SM over the device.
-constexpr int kMinTilesPerSplit = 2;
-constexpr int kMaxTilesPerSplit = 64;
-constexpr int kTargetCtasPerSm = 4;
-constexpr int kMaxSplits = 65535;   // gridDim.y limit
+// Persistent grid of the fp32 path, in CTAs per SM (its CTAs are small).
+constexpr int kF32CtasPerSm = 4;
 
 std::mutex g_mu;
 int g_num_sms[kMaxDevices];
@@ -84,21 +79,23 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
 
 // ------------------------------------------------------------------ decode
 struct DecodePlan {
-  int splits, tiles_per_split;
-  size_t counter_bytes, partial_bytes;
+  int ctas;                  // persistent grid size
+  int units_per_seq, heads_per_unit;
+  size_t counter_bytes, slot_bytes;
 };
 
 plx_status validate_decode(const plx_decode_params* p) {
   if (p == nullptr) return PLX_ERR_INVALID_ARG;
   if (p->batch < 1 || p->num_q_heads < 1 || p->num_kv_heads < 1) return PLX_ERR_INVALID_ARG;
   if (p->num_q_heads % p->num_kv_heads != 0) return PLX_ERR_INVALID_ARG;
-  if (p->kv_len < 0 || p->num_splits < 0) return PLX_ERR_INVALID_ARG;
+  if (p->kv_len < 0 || p->num_ctas < 0) return PLX_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return PLX_ERR_INVALID_ARG;
   if (p->in_dtype != PLX_F32 && p->in_dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
   if (p->out_dtype != PLX_F32 && p->out_dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
   if (p->head_dim != 64 && p->head_dim != 128) return PLX_ERR_UNSUPPORTED;
   if (p->page_size != 0 && p->page_size != kTile) return PLX_ERR_UNSUPPORTED;
   if (p->in_dtype == PLX_BF16 && p->num_q_heads / p->num_kv_heads > kMaxGroup) return PLX_ERR_UNSUPPORTED;
+  if (p->batch > kMaxBatch) return PLX_ERR_UNSUPPORTED;
   if (p->page_size != 0) {
     if (p->num_pages < 1) return PLX_ERR_INVALID_ARG;
     if (p->max_pages_per_seq < (p->kv_len + kTile - 1) / kTile) return PLX_ERR_INVALID_ARG;
@@ -107,55 +104,52 @@ plx_status validate_decode(const plx_decode_params* p) {
     if ((int64_t)p->batch * p->num_kv_heads * ((int64_t)p->kv_len + kTile) >= (int64_t)INT32_MAX)
       return PLX_ERR_UNSUPPORTED;
   }
-  if ((int64_t)p->batch * p->num_q_heads >= (int64_t)INT32_MAX / 2) return PLX_ERR_UNSUPPORTED;
+  // total tiles of all units must fit an int
+  if ((int64_t)p->batch * p->num_q_heads * (((int64_t)p->kv_len + kTile - 1) / kTile) >= (int64_t)INT32_MAX / 2)
+    return PLX_ERR_UNSUPPORTED;
   return PLX_OK;
 }
 
 DecodePlan plan_decode(const plx_decode_params* p, int num_sms) {
   DecodePlan pl{};
-  const int tiles = (p->kv_len + kTile - 1) / kTile;
-  if (tiles == 0) {
-    pl.splits = 1;
-    pl.tiles_per_split = 1;
-    return pl;
-  }
-  int tps;
-  if (p->num_splits > 0) {
-    tps = (tiles + p->num_splits - 1) / p->num_splits;
-  } else {
-    const int64_t units = (int64_t)p->batch * (p->in_dtype == PLX_BF16 ? p->num_kv_heads : p->num_q_heads);
-    const int64_t target = (int64_t)kTargetCtasPerSm * (num_sms > 0 ? num_sms : 148);
-    const int64_t want_splits = (target + units - 1) / units;
-    tps = (int)((tiles + want_splits - 1) / want_splits);
-    tps = tps < kMinTilesPerSplit ? kMinTilesPerSplit : tps;
-    tps = tps > kMaxTilesPerSplit ? kMaxTilesPerSplit : tps;
-  }
-  if (tps > tiles) tps = tiles;
-  if (tps < 1) tps = 1;
-  if ((tiles + tps - 1) / tps > kMaxSplits) tps = (tiles + kMaxSplits - 1) / kMaxSplits;
-  pl.tiles_per_split = tps;
-  pl.splits = (tiles + tps - 1) / tps;
-  if (pl.splits > 1) {
-    pl.counter_bytes = (((size_t)p->batch * p->num_q_heads * 4) + 255) & ~size_t(255);
-    pl.partial_bytes = (size_t)pl.splits * p->batch * p->num_q_heads * (2 * p->head_dim + 4) * 4;
-  }
+  const bool bf16 = p->in_dtype == PLX_BF16;
+  pl.units_per_seq = bf16 ? p->num_kv_heads : p->num_q_heads;
+  pl.heads_per_unit = bf16 ? p->num_q_heads / p->num_kv_heads : 1;
+  const int64_t tiles = (int64_t)p->batch * pl.units_per_seq * ((p->kv_len + kTile - 1) / kTile);
+  int64_t ctas = p->num_ctas > 0 ? p->num_ctas : (int64_t)num_sms * (bf16 ? 1 : kF32CtasPerSm);
+  if (ctas > tiles) ctas = tiles;
+  if (ctas < 1) ctas = 1;
+  if (ctas > INT32_MAX / 4) ctas = INT32_MAX / 4;
+  pl.ctas = (int)ctas;
+  pl.counter_bytes = (((size_t)p->batch * pl.units_per_seq * 4) + 255) & ~size_t(255);
+  pl.slot_bytes = (size_t)2 * pl.ctas * pl.heads_per_unit * (2 * p->head_dim + 4) * 4;
   return pl;
 }
 
+size_t decode_smem_bytes(const plx_decode_params* p) {
+  const size_t table = (size_t)(2 * p->batch + 1) * 4;
+  if (p->in_dtype == PLX_F32) return f32_smem_fixed_bytes<kDecodeF32Warps>() + table;
+  return (p->head_dim == 64 ? tc_smem_fixed_bytes<64, kDecodeStages64, kDecodeNC>()
+                            : tc_smem_fixed_bytes<128, kDecodeStages128, kDecodeNC>()) +
+         table;
+}
+
 template <int D, int STAGES, bool kLoInPad>
-plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, dim3 grid,
-                            cudaStream_t stream) {
-  constexpr int smem = tc_smem_bytes<D, STAGES, kDecodeNC>();
+plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int ctas,
+                            size_t smem, cudaStream_t stream) {
   auto kern = decode_tc_kernel<D, STAGES, kDecodeNC, kLoInPad>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
-  kern<<<grid, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
+  kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
 template <int D>
-plx_status launch_decode_f32(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
-  decode_f32_kernel<D, kDecodeF32Warps><<<grid, kDecodeF32Warps * 32, 0, stream>>>(a);
+plx_status launch_decode_f32(const DecodeArgs& a, int ctas, size_t smem, cudaStream_t stream) {
+  auto kern = decode_f32_kernel<D, kDecodeF32Warps>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  kern<<<ctas, kDecodeF32Warps * 32, smem, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
@@ -218,11 +212,11 @@ const char* parallax_status_string(plx_status s) {
   return "PLX_UNKNOWN_STATUS";
 }
 
-int32_t parallax_decode_num_splits(const plx_decode_params* p, int32_t num_sms) {
+int32_t parallax_decode_num_ctas(const plx_decode_params* p, int32_t num_sms) {
   if (validate_decode(p) != PLX_OK) return -1;
   if (num_sms <= 0) num_sms = current_device_sms();
   if (num_sms <= 0) return -1;
-  return plan_decode(p, num_sms).splits;
+  return plan_decode(p, num_sms).ctas;
 }
 
 size_t parallax_decode_workspace_size(const plx_decode_params* p, int32_t num_sms) {
@@ -230,7 +224,7 @@ size_t parallax_decode_workspace_size(const plx_decode_params* p, int32_t num_sm
   if (num_sms <= 0) num_sms = current_device_sms();
   if (num_sms <= 0) return (size_t)-1;
   const DecodePlan pl = plan_decode(p, num_sms);
-  return pl.counter_bytes + pl.partial_bytes;
+  return pl.counter_bytes + pl.slot_bytes;
 }
 
 plx_status parallax_decode(const void* q, const void* rho, const void* k_cache, const void* v_cache,
@@ -249,9 +243,8 @@ plx_status parallax_decode(const void* q, const void* rho, const void* k_cache, 
   const int num_sms = current_device_sms();
   if (num_sms <= 0) return PLX_ERR_CUDA;
   const DecodePlan pl = plan_decode(p, num_sms);
-  const size_t need = pl.counter_bytes + pl.partial_bytes;
-  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)))
-    return PLX_ERR_WORKSPACE;
+  const size_t need = pl.counter_bytes + pl.slot_bytes;
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return PLX_ERR_WORKSPACE;
 
   const int D = p->head_dim;
   if (p->kv_len == 0) {
@@ -270,37 +263,36 @@ plx_status parallax_decode(const void* q, const void* rho, const void* k_cache, 
   a.page_table = page_table;
   a.seq_lens = seq_lens;
   a.out = out;
-  a.counters = need ? reinterpret_cast<int32_t*>(workspace) : nullptr;
-  a.partials = need ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + pl.counter_bytes) : nullptr;
+  a.counters = reinterpret_cast<int32_t*>(workspace);
+  a.slots = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + pl.counter_bytes);
   a.B = p->batch;
   a.Hq = p->num_q_heads;
   a.Hkv = p->num_kv_heads;
   a.group = p->num_q_heads / p->num_kv_heads;
+  a.units_per_seq = pl.units_per_seq;
+  a.heads_per_unit = pl.heads_per_unit;
   a.kv_len = p->kv_len;
   a.paged = paged ? 1 : 0;
   a.num_pages = paged ? p->num_pages : 0;
   a.max_pages = paged ? p->max_pages_per_seq : 0;
-  a.splits = pl.splits;
-  a.tiles_per_split = pl.tiles_per_split;
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
 
-  if (p->in_dtype == PLX_F32) {
-    const dim3 grid(p->batch * p->num_q_heads, pl.splits);
-    return D == 64 ? launch_decode_f32<64>(a, grid, stream) : launch_decode_f32<128>(a, grid, stream);
-  }
+  const size_t smem = decode_smem_bytes(p);
+  if (smem > 227 * 1024) return PLX_ERR_UNSUPPORTED;
+  if (p->in_dtype == PLX_F32)
+    return D == 64 ? launch_decode_f32<64>(a, pl.ctas, smem, stream) : launch_decode_f32<128>(a, pl.ctas, smem, stream);
   const uint64_t rows = paged ? (uint64_t)p->num_pages * p->num_kv_heads * kTile
                               : (uint64_t)p->batch * p->num_kv_heads * p->kv_len;
   CUtensorMap tk, tv;
   if (!make_tmap_bf16(&tk, k_cache, D, rows, 64, kTile) || !make_tmap_bf16(&tv, v_cache, D, rows, 64, kTile))
     return PLX_ERR_CUDA;
-  const dim3 grid(p->batch * p->num_kv_heads, pl.splits);
   const bool pad = a.group <= kMaxGroup / 2;
   if (D == 64)
-    return pad ? launch_decode_tc<64, kDecodeStages64, true>(a, tk, tv, grid, stream)
-               : launch_decode_tc<64, kDecodeStages64, false>(a, tk, tv, grid, stream);
-  return pad ? launch_decode_tc<128, kDecodeStages128, true>(a, tk, tv, grid, stream)
-             : launch_decode_tc<128, kDecodeStages128, false>(a, tk, tv, grid, stream);
+    return pad ? launch_decode_tc<64, kDecodeStages64, true>(a, tk, tv, pl.ctas, smem, stream)
+               : launch_decode_tc<64, kDecodeStages64, false>(a, tk, tv, pl.ctas, smem, stream);
+  return pad ? launch_decode_tc<128, kDecodeStages128, true>(a, tk, tv, pl.ctas, smem, stream)
+             : launch_decode_tc<128, kDecodeStages128, false>(a, tk, tv, pl.ctas, smem, stream);
 }
 
 plx_status parallax_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,
@@ -321,11 +313,11 @@ plx_status parallax_decode_noalloc(const void* q, const void* rho, const void* k
   const int num_sms = current_device_sms();
   if (num_sms <= 0) return PLX_ERR_CUDA;
   const DecodePlan pl = plan_decode(p, num_sms);
-  if (pl.counter_bytes + pl.partial_bytes > (size_t)PARALLAX_NOALLOC_SCRATCH_BYTES) return PLX_ERR_WORKSPACE;
+  if (pl.counter_bytes + pl.slot_bytes > (size_t)PARALLAX_NOALLOC_SCRATCH_BYTES) return PLX_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != PLX_OK) return st;
   // The counters must start at zero; the array keeps whatever the last call left.
-  if (pl.counter_bytes > 0 && cudaMemsetAsync(scratch, 0, pl.counter_bytes, stream) != cudaSuccess)
+  if (cudaMemsetAsync(scratch, 0, pl.counter_bytes, stream) != cudaSuccess)
     return PLX_ERR_CUDA;
   return parallax_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, scratch,
                          (size_t)PARALLAX_NOALLOC_SCRATCH_BYTES, p, stream);

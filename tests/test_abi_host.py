@@ -50,27 +50,27 @@ def test_abi_version_and_status_strings(binding):
 
 def _params(binding, **kw):
     base = dict(batch=8, num_q_heads=16, num_kv_heads=8, head_dim=128, kv_len=4096, page_size=0,
-                num_pages=0, max_pages_per_seq=0, in_dtype=1, out_dtype=1, scale=0.088, num_splits=0)
+                num_pages=0, max_pages_per_seq=0, in_dtype=1, out_dtype=1, scale=0.088, num_ctas=0)
     base.update(kw)
     return binding.DecodeParams(**base)
 
 
 @pytest.mark.parametrize("bad", [
     dict(batch=0), dict(num_q_heads=12, num_kv_heads=8), dict(kv_len=-1), dict(in_dtype=7),
-    dict(out_dtype=9), dict(scale=float("inf")), dict(num_splits=-2),
+    dict(out_dtype=9), dict(scale=float("inf")), dict(num_ctas=-2),
     dict(page_size=64, num_pages=0, max_pages_per_seq=64),
     dict(page_size=64, num_pages=10, max_pages_per_seq=3),
 ])
 def test_invalid_decode_params_are_rejected(binding, bad):
     p = _params(binding, **bad)
-    assert binding.lib.parallax_decode_num_splits(ctypes.byref(p), 148) == -1
+    assert binding.lib.parallax_decode_num_ctas(ctypes.byref(p), 148) == -1
     assert binding.lib.parallax_decode_workspace_size(ctypes.byref(p), 148) == binding.SIZE_MAX
     st = binding.lib.parallax_decode(None, None, None, None, None, None, None, None, 0, ctypes.byref(p), None)
     assert st == 1
 
 
 @pytest.mark.parametrize("unsup", [dict(head_dim=96), dict(page_size=32, num_pages=4, max_pages_per_seq=200),
-                                   dict(num_q_heads=32, num_kv_heads=2)])
+                                   dict(num_q_heads=32, num_kv_heads=2), dict(batch=9000)])
 def test_unsupported_decode_params(binding, unsup):
     p = _params(binding, **unsup)
     st = binding.lib.parallax_decode(None, None, None, None, None, None, None, None, 0, ctypes.byref(p), None)
@@ -106,31 +106,32 @@ def test_invalid_prefill_params_are_rejected(binding, bad):
     assert st in (1, 2)
 
 
-def _expected_plan(B, units, L, num_sms=148, forced=0):
-    tiles = -(-L // 64)
-    if forced:
-        tps = -(-tiles // forced)
-    else:
-        want = -(-(4 * num_sms) // units)
-        tps = min(max(-(-tiles // want), 2), 64)
-    tps = max(1, min(tps, tiles))
-    return -(-tiles // tps)
+def _expected_plan(B, units, heads_per_unit, L, d=128, num_sms=148, forced=0, per_sm=1):
+    tiles = B * units * (-(-L // 64))
+    ctas = forced if forced else num_sms * per_sm
+    ctas = max(1, min(ctas, tiles))
+    counters = -(-(B * units * 4) // 256) * 256
+    return ctas, counters + 2 * ctas * heads_per_unit * (2 * d + 4) * 4
 
 
-@pytest.mark.parametrize("B,Hq,Hkv,L,forced", [
-    (8, 16, 8, 4096, 0), (64, 32, 8, 32768, 0), (128, 16, 4, 65536, 0), (1, 1, 1, 256, 0),
-    (1, 4, 4, 65, 0), (8, 16, 8, 4096, 3), (2, 2, 1, 100, 16), (4, 8, 2, 1, 0),
+@pytest.mark.parametrize("B,Hq,Hkv,L,forced,dtype", [
+    (8, 16, 8, 4096, 0, 1), (64, 32, 8, 32768, 0, 1), (128, 16, 4, 65536, 0, 1), (1, 1, 1, 256, 0, 0),
+    (1, 4, 4, 65, 0, 1), (8, 16, 8, 4096, 3, 1), (2, 2, 1, 100, 16, 1), (4, 8, 2, 1, 0, 1), (2, 6, 2, 4096, 0, 0),
 ])
-def test_split_plan_and_workspace_size(binding, B, Hq, Hkv, L, forced):
-    p = _params(binding, batch=B, num_q_heads=Hq, num_kv_heads=Hkv, kv_len=L, num_splits=forced)
-    splits = binding.lib.parallax_decode_num_splits(ctypes.byref(p), 148)
-    assert splits == _expected_plan(B, B * Hkv, L, forced=forced)
-    ws = binding.lib.parallax_decode_workspace_size(ctypes.byref(p), 148)
-    if splits == 1:
-        assert ws == 0
-    else:
-        counters = -(-(B * Hq * 4) // 256) * 256
-        assert ws == counters + splits * B * Hq * (2 * 128 + 4) * 4
+def test_work_plan_and_workspace_size(binding, B, Hq, Hkv, L, forced, dtype):
+    p = _params(binding, batch=B, num_q_heads=Hq, num_kv_heads=Hkv, kv_len=L, num_ctas=forced, in_dtype=dtype,
+                out_dtype=dtype)
+    ctas = binding.lib.parallax_decode_num_ctas(ctypes.byref(p), 148)
+    units, hpu, per_sm = (Hkv, Hq // Hkv, 1) if dtype == 1 else (Hq, 1, 4)
+    exp_ctas, exp_ws = _expected_plan(B, units, hpu, L, forced=forced, per_sm=per_sm)
+    assert ctas == exp_ctas
+    assert binding.lib.parallax_decode_workspace_size(ctypes.byref(p), 148) == exp_ws
+
+
+def test_workspace_does_not_grow_with_length(binding):
+    sizes = [binding.lib.parallax_decode_workspace_size(ctypes.byref(_params(binding, kv_len=L)), 148)
+             for L in (4096, 65536, 1 << 20)]
+    assert sizes[0] == sizes[1] == sizes[2]
 
 
 def test_no_cpu_fallback(binding):

@@ -119,13 +119,14 @@ def test_f32_shapes(px, d, L, group):
     assert_parity(out.cpu().numpy(), ref, TOL_F32, f"f32 d={d} L={L} g={group}")
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 16, 0])
+@pytest.mark.parametrize("ctas", [1, 2, 3, 16, 0, 1000])
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_split_counts_agree(px, splits, dtype):
+def test_grid_sizes_agree(px, ctas, dtype):
+    # Different persistent grids cut the units into different pieces.
     inp = _to(W.small_decode_inputs(3, 8, 2, 128, 1500, dtype=dtype, seq_lens=[1500, 700, 65], seed=5))
-    out = _run(px, inp, num_splits=splits, out_dtype=torch.float32)
+    out = _run(px, inp, num_ctas=ctas, out_dtype=torch.float32)
     ref = oracle_heads(inp, _all_heads(inp))
-    assert_parity(out.cpu().numpy(), ref, TOL_F32 if dtype == "f32" else TOL_BF16, f"splits={splits}")
+    assert_parity(out.cpu().numpy(), ref, TOL_F32 if dtype == "f32" else TOL_BF16, f"ctas={ctas}")
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -139,13 +140,13 @@ def test_ragged_lengths_with_nan_tails(px, dtype):
     np.testing.assert_array_equal(out[7], 0.0)   # empty sequence -> zero output
 
 
-@pytest.mark.parametrize("splits", [1, 4])
-def test_paged_is_bit_identical_to_contiguous(px, splits):
+@pytest.mark.parametrize("ctas", [1, 4, 0])
+def test_paged_is_bit_identical_to_contiguous(px, ctas):
     lens = [300, 64, 1, 129]
     inp = _to(W.small_decode_inputs(4, 8, 2, 128, 320, seq_lens=lens, paged=True, seed=3))
-    paged = _run(px, inp, num_splits=splits, out_dtype=torch.float32)
+    paged = _run(px, inp, num_ctas=ctas, out_dtype=torch.float32)
     contig = px.decode(inp["q"], inp["rho"], inp["k_contig"], inp["v_contig"], inp["scale"],
-                       seq_lens=inp["seq_lens"], num_splits=splits, out_dtype=torch.float32)
+                       seq_lens=inp["seq_lens"], num_ctas=ctas, out_dtype=torch.float32)
     assert torch.equal(paged, contig)
     ref = oracle_heads(inp, _all_heads(inp))
     assert_parity(paged.cpu().numpy(), ref, TOL_BF16, "paged")
@@ -173,15 +174,15 @@ def test_output_guard_bands_untouched(px):
     n = inp["q"].numel()
     buf = torch.full((n + 2048,), 12345.0, dtype=torch.float32, device=DEV)
     out = buf[1024:1024 + n].view(inp["q"].shape)
-    _run(px, inp, out=out, out_dtype=torch.float32, num_splits=3)
+    _run(px, inp, out=out, out_dtype=torch.float32, num_ctas=3)
     torch.cuda.synchronize()
     assert (buf[:1024] == 12345.0).all() and (buf[1024 + n:] == 12345.0).all()
 
 
 def test_repeated_calls_are_deterministic(px):
     inp = _to(W.small_decode_inputs(4, 8, 2, 128, 3000, seed=8))
-    a = _run(px, inp, num_splits=7)
-    b = _run(px, inp, num_splits=7)
+    a = _run(px, inp, num_ctas=7)
+    b = _run(px, inp, num_ctas=7)
     assert torch.equal(a, b)
 
 
@@ -208,7 +209,7 @@ def test_bad_length_sets_error_word(px):
 def test_workspace_too_small_is_rejected(px):
     import ctypes
     inp = _to(W.small_decode_inputs(2, 4, 2, 128, 2000, seed=1))
-    p = px.decode_params(inp["q"], inp["k_cache"], num_splits=4)
+    p = px.decode_params(inp["q"], inp["k_cache"], num_ctas=4)
     need = px.decode_workspace_size(p)
     assert need > 0
     ws = torch.zeros(need - 256, dtype=torch.uint8, device=DEV)

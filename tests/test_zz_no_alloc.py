@@ -40,9 +40,9 @@ def _inputs(case):
     return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
 
 
-def _noalloc(px, inp, out, splits):
+def _noalloc(px, inp, out, ctas):
     p = px.decode_params(inp["q"], inp["k_cache"], page_table=inp.get("page_table"), scale=inp["scale"],
-                         out_dtype=out.dtype, num_splits=splits)
+                         out_dtype=out.dtype, num_ctas=ctas)
     return px.lib.parallax_decode_noalloc(
         px._ptr(inp["q"]), px._ptr(inp["rho"]), px._ptr(inp["k_cache"]), px._ptr(inp["v_cache"]),
         px._ptr(inp.get("page_table")), px._ptr(inp.get("seq_lens")), px._ptr(out), ctypes.byref(p),
@@ -52,14 +52,14 @@ def _noalloc(px, inp, out, splits):
 @pytest.mark.parametrize("case", ["contiguous_bf16", "paged_bf16", "f32"])
 def test_noalloc_matches_workspace_entry_point(px, case):
     inp = _inputs(case)
-    splits = 5   # several splits per sequence, so the scratch array is in use
+    ctas = 5   # several CTAs per sequence, so the scratch array is in use
     ref = px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"],
                     seq_lens=inp.get("seq_lens"), page_table=inp.get("page_table"),
-                    out_dtype=torch.float32, num_splits=splits)
+                    out_dtype=torch.float32, num_ctas=ctas)
     tol = TOL_F32 if case == "f32" else TOL_BF16
     for call in range(2):
         out = torch.full_like(ref, float("nan"))
-        assert _noalloc(px, inp, out, splits) == 0
+        assert _noalloc(px, inp, out, ctas) == 0
         torch.cuda.synchronize()
         assert_parity(out.cpu().numpy(), ref.cpu().numpy(), tol, f"{case} call {call}")
     assert px.last_device_error() == 0
@@ -70,7 +70,7 @@ def test_noalloc_back_to_back_different_shapes(px):
     for inp in (a, b, a):
         ref = px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"],
                         seq_lens=inp.get("seq_lens"), page_table=inp.get("page_table"),
-                        out_dtype=torch.float32, num_splits=7)
+                        out_dtype=torch.float32, num_ctas=7)
         out = torch.empty_like(ref)
         assert _noalloc(px, inp, out, 7) == 0
         assert_parity(out.cpu().numpy(), ref.cpu().numpy(), TOL_BF16, "back to back")
@@ -78,8 +78,8 @@ def test_noalloc_back_to_back_different_shapes(px):
 
 def test_noalloc_rejects_what_does_not_fit(px):
     inp = _inputs("contiguous_bf16")
-    p = px.decode_params(inp["q"], inp["k_cache"], num_splits=40)
-    big = px.DecodeParams(512, 64, 8, 128, 65536, 0, 0, 0, 1, 1, 0.088, 64)
+    p = px.decode_params(inp["q"], inp["k_cache"], num_ctas=40)
+    big = px.DecodeParams(512, 64, 8, 128, 65536, 0, 0, 0, 1, 1, 0.088, 100000)
     assert px.decode_workspace_size(big) > px.NOALLOC_SCRATCH_BYTES
     out = torch.empty(1, device="cuda")
     st = px.lib.parallax_decode_noalloc(px._ptr(out), px._ptr(out), px._ptr(out), px._ptr(out), None, None,
