@@ -68,6 +68,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="decode_bf16", choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--num-ctas", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -571,6 +573,9 @@ def _host_decode_sample(w):
 def main(argv=None):
     args = parse_args(argv)
     w = W.WORKLOADS[args.workload]
+    if args.batch > 0:
+        import dataclasses
+        w = dataclasses.replace(w, batch=args.batch)
     if args.steps is None:
         args.steps = default_steps(args.workload) if args.impl == "ours" else 10
     if args.warmup is None:

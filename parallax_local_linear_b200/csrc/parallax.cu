@@ -154,6 +154,34 @@ plx_status launch_decode_f32(const DecodeArgs& a, int ctas, size_t smem, cudaStr
 }
 
 // ----------------------------------------------------------------- prefill
+plx_status launch_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,
+                          const plx_prefill_params* p, cudaStream_t stream) {
+  const int hkv = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
+  const uint64_t rows_q = (uint64_t)p->batch * p->num_heads * p->seq_len;
+  const uint64_t rows_kv = (uint64_t)p->batch * hkv * p->seq_len;
+  CUtensorMap tq, tr, tk, tv;
+  if (!make_tmap_bf16(&tq, q, kPfD, rows_q, 64, kPfBM) || !make_tmap_bf16(&tr, rho, kPfD, rows_q, 64, kPfBM) ||
+      !make_tmap_bf16(&tk, k, kPfD, rows_kv, 64, kPfBN) || !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBN))
+    return PLX_ERR_CUDA;
+  PrefillArgs a{};
+  a.B = p->batch;
+  a.H = p->num_heads;
+  a.Hkv = hkv;
+  a.T = p->seq_len;
+  a.group = p->num_heads / hkv;
+  a.n_mblk = (p->seq_len + kPfBM - 1) / kPfBM;
+  a.causal = p->causal;
+  a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.out = out;
+  constexpr int smem = PfLayout::kBytes;
+  if (cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  const long long grid = (long long)a.n_mblk * a.B * a.H;
+  prefill_tc_kernel<<<(unsigned)grid, 192, smem, stream>>>(tq, tr, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
 plx_status validate_prefill(const plx_prefill_params* p) {
   if (p == nullptr) return PLX_ERR_INVALID_ARG;
   const int hkv = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
