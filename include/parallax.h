@@ -167,7 +167,7 @@ typedef struct plx_prefill_params {
   int32_t head_dim;       /* d: 128                                           */
   int32_t in_dtype;       /* PLX_BF16                                         */
   int32_t out_dtype;      /* PLX_BF16 or PLX_F32                              */
-  float scale;            /* softmax scale on q.k                             */
+  float scale;            /* softmax scale on q.k, > 0                        */
   int32_t causal;         /* 1: causal mask (diagonal included); 0: none      */
 } plx_prefill_params;
 

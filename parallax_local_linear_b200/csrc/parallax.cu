@@ -25,8 +25,11 @@ using namespace plx;
 constexpr int kMaxDevices = 64;
 
 // Decode kernel configuration (bf16 path): consumer warps and ring depth.
+#ifndef PLX_DECODE_STAGES
+#define PLX_DECODE_STAGES 4
+#endif
 constexpr int kDecodeNC = 4;
-constexpr int kDecodeStages128 = 4;
+constexpr int kDecodeStages128 = PLX_DECODE_STAGES;
 constexpr int kDecodeStages64 = 6;
 constexpr int kDecodeF32Warps = 4;
 
@@ -178,7 +181,7 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   if (cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return PLX_ERR_CUDA;
   const long long grid = (long long)a.n_mblk * a.B * a.H;
-  prefill_tc_kernel<<<(unsigned)grid, 192, smem, stream>>>(tq, tr, tk, tv, a);
+  prefill_tc_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
@@ -188,6 +191,7 @@ plx_status validate_prefill(const plx_prefill_params* p) {
   if (p->batch < 1 || p->num_heads < 1 || hkv < 1 || p->seq_len < 1) return PLX_ERR_INVALID_ARG;
   if (p->num_heads % hkv != 0) return PLX_ERR_INVALID_ARG;
   if (!std::isfinite(p->scale)) return PLX_ERR_INVALID_ARG;
+  if (!(p->scale > 0.f)) return PLX_ERR_INVALID_ARG;   // a softmax temperature is positive
   if (p->in_dtype != PLX_BF16) return p->in_dtype == PLX_F32 ? PLX_ERR_UNSUPPORTED : PLX_ERR_INVALID_ARG;
   if (p->out_dtype != PLX_F32 && p->out_dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
   if (p->head_dim != 128) return PLX_ERR_UNSUPPORTED;

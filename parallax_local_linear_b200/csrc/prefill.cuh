@@ -7,7 +7,7 @@
 // out = (O1/l)(1 + c/l) - O2/l, which equals vbar - S_KV^T rho (the
 // covariance correction of the wispaper.ai blog "Parallax: Breaking the
 // Boundary Bias with Parameterized Local Linear Attention", section "The Core
-// Insight: Covariance Correction"; computed "in a single pass" as in its
+// Insight: Covariance Correction"; computed in a single pass, as in its
 // "Hardware Efficiency" section).  a_ref = rho_t.k_0, read from the first key
 // tile (key 0 is visible to every row).
 //
@@ -17,14 +17,17 @@
 // with P = exp2(S * scale * log2(e) - m) and A' = A - a_ref.
 //
 // CTA = one 128-row query tile of one (sequence, head); key tiles of 64.
-// Warp roles (192 threads):
-//   warp 0       TMA producer: Q and R once, then a STAGES-deep K/V ring.
+// Warp roles (320 threads):
+//   warp 0       TMA producer: Q and R once, then separate K and V rings.
 //   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma.
-//   warps 2..5   softmax: thread = query row = TMEM lane.  Reads S and A
-//                from TMEM, forms P and P o A' in bf16, writes them back over
-//                the S and A columns (the A operand of the value products
-//                comes straight from TMEM), rescales O when the running max
-//                grows by more than 2^8, and finally writes the output.
+//   warps 2..9   softmax, two warpgroups.  Thread = query row = TMEM lane;
+//                warpgroup g takes key columns 32g..32g+31 of every tile.
+//                The two halves of a row exchange their max through shared
+//                memory once per tile, form P and P o A' in bf16 and write
+//                them back over the S and A columns (the A operand of the
+//                value products comes straight from TMEM).  When the running
+//                max grows by more than 2^8, warpgroup g rescales O1 (g = 0)
+//                or O2 (g = 1); at the end it writes output columns 64g..64g+63.
 //
 // TMEM columns (512 x 128 lanes x 32 bit): O1 [0,128), O2 [128,256), and two
 // buffers of S / A: S_b at 256 + 128 b, A_b at 320 + 128 b.  While the
@@ -39,20 +42,32 @@ namespace plx {
 constexpr int kPfBM = 128;        // query rows per CTA (= TMEM lanes)
 constexpr int kPfBN = 64;         // keys per tile
 constexpr int kPfD = 128;         // head dim
-constexpr int kPfStages = 3;      // K/V ring depth
+#ifndef PLX_PREFILL_STAGES
+#define PLX_PREFILL_STAGES 4
+#endif
+// Depth of each of the K and V rings.  A key tile must be in flight for the
+// L2 latency (~1.5 us) while the tensor cores work through the tiles ahead
+// of it, and K and V are released separately (K after the score products,
+// V after the value products), so each ring keeps several tiles in flight.
+constexpr int kPfStages = PLX_PREFILL_STAGES;
+constexpr int kPfThreads = 320;   // producer warp, MMA warp, two softmax warpgroups
+constexpr int kPfSoftmax = 256;   // softmax threads
 constexpr float kPfRescaleLog2 = 8.f;   // lazy rescale threshold (factor 256)
 // Key tiles whose P and P o A' also enter the value products as bf16 lo parts
-// (x = bf16(x) + lo).  A row with few keys has nothing to average the bf16
-// rounding of P o A' (|a| reaches ~10 for unit-scale probes) over; every
-// row's first 128 keys lie in tiles 0 and 1, so splitting those tiles keeps
-// short rows at fp32-level weights for ~1% more tensor work at T = 8192.
-constexpr int kPfSplitTiles = 2;
+// (x = bf16(x) + lo), in query tiles whose rows see fewer than 128 keys.  A
+// row with few keys has nothing to average the bf16 rounding of P o A' (|a|
+// reaches ~10 for unit-scale probes) over; such rows' keys all lie in tiles
+// 0 and 1.  Rows with 128 keys or more average it out.
+#ifndef PLX_PREFILL_SPLIT_TILES
+#define PLX_PREFILL_SPLIT_TILES 2
+#endif
+constexpr int kPfSplitTiles = PLX_PREFILL_SPLIT_TILES;
 
 struct PrefillArgs {
   int B, H, Hkv, T, group;
   int n_mblk;                     // ceil(T / 128)
   int causal, out_bf16;
-  float scale_log2;
+  float scale_log2;               // scale * log2(e), > 0
   void* out;                      // [B, H, T, D]
 };
 
@@ -64,17 +79,20 @@ struct PfLayout {
   static constexpr int kK = kR + kQBytes;
   static constexpr int kV = kK + kPfStages * kKVBytes;
   static constexpr int kBar = kV + kPfStages * kKVBytes;
-  // barriers: q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain
-  static constexpr int kNumBars = 1 + 3 * kPfStages + 2 + 2 + 1 + 1;
+  // barriers: q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2], o_done, drain
+  static constexpr int kNumBars = 1 + 4 * kPfStages + 2 + 2 + 1 + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;       // tmem base, abort flag
-  static constexpr int kBytes = kMisc + 16 + 1024;        // + alignment slack
+  static constexpr int kRedMax = kMisc + 16;              // float [2 tile parities][2 halves][128 rows]
+  static constexpr int kAref = kRedMax + 2 * 2 * 128 * 4; // float [128]
+  static constexpr int kLC = kAref + 128 * 4;             // float [2 halves][128 rows][2]
+  static constexpr int kBytes = kLC + 2 * 128 * 2 * 4 + 1024;   // + alignment slack
 };
 
 constexpr uint32_t kColO1 = 0, kColO2 = 128;
 __device__ __forceinline__ uint32_t col_s(int b) { return 256u + 128u * b; }
 __device__ __forceinline__ uint32_t col_a(int b) { return 320u + 128u * b; }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_r,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const PrefillArgs a) {
@@ -85,13 +103,17 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + kPfStages;
-  uint64_t* kv_empty = v_full + kPfStages;
-  uint64_t* s_full = kv_empty + kPfStages;
+  uint64_t* k_empty = v_full + kPfStages;
+  uint64_t* v_empty = k_empty + kPfStages;
+  uint64_t* s_full = v_empty + kPfStages;
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* drain = o_done + 1;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + L::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
+  float* red_max = reinterpret_cast<float*>(sm + L::kRedMax);
+  float* aref_s = reinterpret_cast<float*>(sm + L::kAref);
+  float* lc_s = reinterpret_cast<float*>(sm + L::kLC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Longest query tiles first: the last tile of every head, then the one before...
@@ -102,6 +124,10 @@ __global__ void __launch_bounds__(192, 1)
   const int m0 = mblk * kPfBM;
   const int kv_end = a.causal ? min(a.T, m0 + kPfBM) : a.T;
   const int n = (kv_end + kPfBN - 1) / kPfBN;
+  // Rows of this tile see at least min_keys keys; below 128 the bf16
+  // rounding of P o A' is not averaged away, so the first tiles are split.
+  const int min_keys = a.causal ? min(m0 + 1, a.T) : a.T;
+  const bool few_keys = min_keys < 2 * kPfBN;
   const int q_row = (b * a.H + h) * a.T + m0;
   const int kv_row = (b * a.Hkv + kvh) * a.T;
 
@@ -110,11 +136,12 @@ __global__ void __launch_bounds__(192, 1)
     for (int s = 0; s < kPfStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], kPfSoftmax);
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
@@ -144,169 +171,199 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_2d(sm + L::kQ + bx * (L::kQBytes / 2), &tm_q, bx * 64, q_row, q_full, once);
         tma_load_2d(sm + L::kR + bx * (L::kQBytes / 2), &tm_r, bx * 64, q_row, q_full, once);
       }
-      int issued = 0;
+      int issued = 0, issued_k = 0;   // V and K tiles issued
       for (int j = 0; j < n; ++j) {
         const int s = j % kPfStages;
-        if (j >= kPfStages && !mbar_wait_bounded(&kv_empty[s], ((j / kPfStages) - 1) & 1)) {
+        const uint32_t par = ((j / kPfStages) - 1) & 1;
+        const int row = kv_row + j * kPfBN;
+        if (j >= kPfStages && !mbar_wait_bounded(&k_empty[s], par)) {
           *abort_flag = 1;
           break;
         }
         if (*abort_flag) break;
-        const int row = kv_row + j * kPfBN;
         mbar_arrive_expect_tx(&k_full[s], L::kKVBytes);
-        mbar_arrive_expect_tx(&v_full[s], L::kKVBytes);
-        for (int bx = 0; bx < 2; ++bx) {
+        for (int bx = 0; bx < 2; ++bx)
           tma_load_2d(sm + L::kK + s * L::kKVBytes + bx * (L::kKVBytes / 2), &tm_k, bx * 64, row, &k_full[s], keep);
-          tma_load_2d(sm + L::kV + s * L::kKVBytes + bx * (L::kKVBytes / 2), &tm_v, bx * 64, row, &v_full[s], keep);
+        if (j >= kPfStages && !mbar_wait_bounded(&v_empty[s], par)) {
+          *abort_flag = 1;
+          ++issued_k;
+          break;
         }
+        mbar_arrive_expect_tx(&v_full[s], L::kKVBytes);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_2d(sm + L::kV + s * L::kKVBytes + bx * (L::kKVBytes / 2), &tm_v, bx * 64, row, &v_full[s], keep);
         ++issued;
+        ++issued_k;
       }
       // Every issued load must land before the CTA exits.
       mbar_wait_bounded(q_full, 0);
+      for (int s = 0; s < kPfStages && s < issued_k; ++s) {
+        const int last = s + ((issued_k - 1 - s) / kPfStages) * kPfStages;
+        mbar_wait_bounded(&k_full[s], (last / kPfStages) & 1);
+      }
       for (int s = 0; s < kPfStages && s < issued; ++s) {
         const int last = s + ((issued - 1 - s) / kPfStages) * kPfStages;
-        mbar_wait_bounded(&k_full[s], (last / kPfStages) & 1);
         mbar_wait_bounded(&v_full[s], (last / kPfStages) & 1);
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(kPfBM, kPfBN, false);   // 128 x 64, K-major B
-      constexpr uint32_t kIdPV = idesc_bf16(kPfBM, kPfD, true);    // 128 x 128, MN-major B (V)
-      const uint32_t q_base = smem_u32(sm + L::kQ), r_base = smem_u32(sm + L::kR);
-      const uint32_t k_base = smem_u32(sm + L::kK), v_base = smem_u32(sm + L::kV);
-      bool ok = mbar_wait_bounded(q_full, 0);
-      tc_fence_after();
-      for (int j = 0; ok && j <= n; ++j) {
-        if (*abort_flag) break;
-        if (j < n) {
-          const int s = j % kPfStages, b2 = j & 1;
-          if (!(ok = mbar_wait_bounded(&k_full[s], (j / kPfStages) & 1))) break;
-          tc_fence_after();
-          const uint32_t kb = k_base + s * L::kKVBytes;
+    // The whole warp runs this loop in lockstep (every branch is warp-uniform);
+    // one elected lane issues each tcgen05.mma / commit.
+    constexpr uint32_t kIdS = idesc_bf16(kPfBM, kPfBN, false);   // 128 x 64, K-major B
+    constexpr uint32_t kIdPV = idesc_bf16(kPfBM, kPfD, true);    // 128 x 128, MN-major B (V)
+    // Descriptors of every operand base; a k-step adds its byte offset / 16.
+    const uint64_t dq = smem_desc_sw128(smem_u32(sm + L::kQ), 16, 1024);
+    const uint64_t dr = smem_desc_sw128(smem_u32(sm + L::kR), 16, 1024);
+    const uint64_t dk = smem_desc_sw128(smem_u32(sm + L::kK), 16, 1024);
+    const uint64_t dv = smem_desc_sw128(smem_u32(sm + L::kV), L::kKVBytes / 2, 1024);
+    auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    };
+    bool ok = wait_warp(q_full, 0);
+    tc_fence_after();
+    for (int j = 0; ok && j <= n; ++j) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
+      if (j < n) {
+        const int s = j % kPfStages, b2 = j & 1;
+        if (!(ok = wait_warp(&k_full[s], (j / kPfStages) & 1))) break;
+        tc_fence_after();
+        const uint64_t dks = dk + (uint64_t)((s * L::kKVBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kPfD / 16; ++kk) {
-            // 16 columns of d per step: box kk / 4, 32 bytes into the 128-byte row per step
-            const uint32_t off_q = (kk >> 2) * (L::kQBytes / 2) + (kk & 3) * 32;
-            const uint32_t off_k = (kk >> 2) * (L::kKVBytes / 2) + (kk & 3) * 32;
-            tc_mma_ss(tmem + col_s(b2), smem_desc_sw128(q_base + off_q, 16, 1024),
-                      smem_desc_sw128(kb + off_k, 16, 1024), kIdS, kk > 0);
-          }
-#pragma unroll
-          for (int kk = 0; kk < kPfD / 16; ++kk) {
-            const uint32_t off_q = (kk >> 2) * (L::kQBytes / 2) + (kk & 3) * 32;
-            const uint32_t off_k = (kk >> 2) * (L::kKVBytes / 2) + (kk & 3) * 32;
-            tc_mma_ss(tmem + col_a(b2), smem_desc_sw128(r_base + off_q, 16, 1024),
-                      smem_desc_sw128(kb + off_k, 16, 1024), kIdS, kk > 0);
-          }
-          tc_commit(&s_full[b2]);
+        for (int kk = 0; kk < kPfD / 16; ++kk) {
+          // 16 columns of d per step: box kk / 4, 32 bytes into the 128-byte row per step
+          const uint64_t oq = (uint64_t)((kk >> 2) * (L::kQBytes / 2 / 16) + (kk & 3) * 2);
+          const uint64_t okk = (uint64_t)((kk >> 2) * (L::kKVBytes / 2 / 16) + (kk & 3) * 2);
+          tc_mma_ss(tmem + col_s(b2), dq + oq, dks + okk, kIdS, kk > 0);
+          tc_mma_ss(tmem + col_a(b2), dr + oq, dks + okk, kIdS, kk > 0);
         }
-        if (j >= 1) {
-          const int jp = j - 1, bp = jp & 1, sp = jp % kPfStages;
-          if (!(ok = mbar_wait_bounded(&p_full[bp], (jp >> 1) & 1))) break;
-          if (!(ok = mbar_wait_bounded(&v_full[sp], (jp / kPfStages) & 1))) break;
-          tc_fence_after();
-          const uint32_t vb = v_base + sp * L::kKVBytes;
+        tc_commit(&s_full[b2]);
+        tc_commit(&k_empty[s]);   // K(j) is free once the score products are done
+      }
+      if (j >= 1) {
+        const int jp = j - 1, bp = jp & 1, sp = jp % kPfStages;
+        if (!(ok = wait_warp(&p_full[bp], (jp >> 1) & 1))) break;
+        if (!(ok = wait_warp(&v_full[sp], (jp / kPfStages) & 1))) break;
+        tc_fence_after();
+        const uint64_t dvs = dv + (uint64_t)((sp * L::kKVBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kPfBN / 16; ++kk) {
+          // 16 keys per step: 8 TMEM columns of packed bf16 pairs, 16 rows of V
+          const uint64_t vd = dvs + (uint64_t)(kk * 16 * 128 / 16);
+          tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + kk * 8, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + kk * 8, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+        }
+        if (few_keys && jp < kPfSplitTiles) {   // lo parts sit in columns 32..63 of the S / A buffers
 #pragma unroll
           for (int kk = 0; kk < kPfBN / 16; ++kk) {
-            // 16 keys per step (8 TMEM columns of packed bf16 pairs; 16 rows of V)
-            const uint64_t vd = smem_desc_sw128(vb + kk * 16 * 128, L::kKVBytes / 2, 1024);
-            tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + kk * 8, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
-            tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + kk * 8, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t vd = dvs + (uint64_t)(kk * 16 * 128 / 16);
+            tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + 32 + kk * 8, vd, kIdPV, 1u);
+            tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + 32 + kk * 8, vd, kIdPV, 1u);
           }
-          if (jp < kPfSplitTiles) {   // lo parts sit in columns 32..63 of the S / A buffers
-#pragma unroll
-            for (int kk = 0; kk < kPfBN / 16; ++kk) {
-              const uint64_t vd = smem_desc_sw128(vb + kk * 16 * 128, L::kKVBytes / 2, 1024);
-              tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + 32 + kk * 8, vd, kIdPV, 1u);
-              tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + 32 + kk * 8, vd, kIdPV, 1u);
-            }
-          }
-          tc_commit(&kv_empty[sp]);
-          tc_commit(o_done);
         }
+        tc_commit(&v_empty[sp]);
+        tc_commit(o_done);
       }
-      if (!ok) *abort_flag = 1;
-      // Every issued MMA must complete before TMEM is released.
-      tc_commit(drain);
-      mbar_wait_bounded(drain, 0);
     }
+    if (!ok && lane == 0) *abort_flag = 1;
+    // Every issued MMA must complete before TMEM is released.
+    tc_commit(drain);
+    wait_warp(drain, 0);
   } else {
     // ------------------------------------------------------------ softmax
+    const int g = (warp - 2) >> 2;           // key-column half of every tile
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int r = wq * 32 + lane;            // query row within the tile
     const int t = m0 + r;                    // query position
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int key_lim = a.causal ? min(t + 1, a.T) : a.T;   // keys [0, key_lim) visible
-    float m_used = -INFINITY, l = 0.f, c = 0.f, aref = 0.f;
-    // tcgen05.ld / st are warp-collective: every wait outcome and abort
-    // decision is made uniform across the warp before acting on it.
-    auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
-      const bool w = !*abort_flag && mbar_wait_bounded(bar, parity);
-      return __all_sync(0xffffffffu, w);
-    };
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
+    const uint32_t cs = 32u * g;             // fp32 columns of this half in S / A
+    const int split_tiles = few_keys ? kPfSplitTiles : 0;
+    const uint32_t cp = 16u * g;             // packed bf16 columns of this half's P / P o A'
+    float m_used = -INFINITY, aref = 0.f;
+    float2 l2 = make_float2(0.f, 0.f), c2 = make_float2(0.f, 0.f);
+    // Each decision that gates a warp-collective tcgen05 op, or the shared
+    // barrier of the two warpgroups, is reduced over all 256 softmax threads
+    // (bar_and), so both halves always leave the loop together.
+    bool fine = true;
+    int j = 0;
+    for (; j < n; ++j) {
       const int b2 = j & 1;
-      if (!(ok = wait_warp(&s_full[b2], (j >> 1) & 1))) break;
+      const bool w = !*abort_flag && mbar_wait_bounded(&s_full[b2], (j >> 1) & 1);
       tc_fence_after();
-      uint32_t sr[64], ar[64];
-      tmem_ld32(tmem + lane_off + col_s(b2), *reinterpret_cast<uint32_t(*)[32]>(sr));
-      tmem_ld32(tmem + lane_off + col_s(b2) + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-      tmem_ld32(tmem + lane_off + col_a(b2), *reinterpret_cast<uint32_t(*)[32]>(ar));
-      tmem_ld32(tmem + lane_off + col_a(b2) + 32, *reinterpret_cast<uint32_t(*)[32]>(ar + 32));
+      uint32_t sr[32], ar[32];
+      tmem_ld32(tmem + lane_off + col_s(b2) + cs, sr);
+      tmem_ld32(tmem + lane_off + col_a(b2) + cs, ar);
       tmem_wait_ld();
-      const int key0 = j * kPfBN;
-      float mt = -INFINITY;
+      // Tiles that reach the diagonal or the sequence end need the mask.
+      const int key0 = j * kPfBN + (int)cs;
+      const bool masked = (a.causal && j * kPfBN + kPfBN - 1 > m0) || (j * kPfBN + kPfBN > a.T);
+      float mx = -INFINITY;
+      if (masked) {
 #pragma unroll
-      for (int cc = 0; cc < 64; ++cc) {
-        const float x = (key0 + cc < key_lim) ? __uint_as_float(sr[cc]) * a.scale_log2 : -INFINITY;
-        sr[cc] = __float_as_uint(x);
-        mt = fmaxf(mt, x);
+        for (int cc = 0; cc < 32; ++cc)
+          if (key0 + cc >= key_lim) sr[cc] = __float_as_uint(-INFINITY);
       }
-      if (j == 0) aref = __uint_as_float(ar[0]);
-      const float m_new = fmaxf(m_used, mt);
+#pragma unroll
+      for (int cc = 0; cc < 32; ++cc) mx = fmaxf(mx, __uint_as_float(sr[cc]));
+      red_max[((j & 1) * 2 + g) * 128 + r] = mx;
+      if (j == 0 && g == 0) aref_s[r] = __uint_as_float(ar[0]);
+      if (!bar_and(1, kPfSoftmax, w && fine)) {
+        fine = false;
+        break;
+      }
+      if (j == 0) aref = aref_s[r];
+      // scale > 0, so the max of the scaled scores is the scaled max
+      const float m_tile = fmaxf(mx, red_max[((j & 1) * 2 + (1 - g)) * 128 + r]) * a.scale_log2;
+      const float m_new = fmaxf(m_used, m_tile);
       const bool need = m_new > m_used + kPfRescaleLog2;
       float alpha = 1.f;
       if (need) {
         alpha = ex2(m_used - m_new);
         m_used = m_new;
       }
-      l *= alpha;
-      c *= alpha;
-      uint32_t pp[32], pa[32];
-      const bool split = j < kPfSplitTiles;
+      l2 = mul2(l2, make_float2(alpha, alpha));
+      c2 = mul2(c2, make_float2(alpha, alpha));
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
+      const float2 nm2 = make_float2(-m_used, -m_used);
+      const float2 na2 = make_float2(-aref, -aref);
+      const bool split = j < split_tiles;
+      uint32_t pp[16], pa[16];
 #pragma unroll
-      for (int cc = 0; cc < 32; ++cc) {
-        const float p0 = ex2(__uint_as_float(sr[2 * cc]) - m_used);
-        const float p1 = ex2(__uint_as_float(sr[2 * cc + 1]) - m_used);
-        const float q0 = p0 * (__uint_as_float(ar[2 * cc]) - aref);
-        const float q1 = p1 * (__uint_as_float(ar[2 * cc + 1]) - aref);
-        l += p0 + p1;
-        c += q0 + q1;
-        pp[cc] = pack_bf16(p0, p1);
-        pa[cc] = pack_bf16(q0, q1);
-        if (split) {   // the lo parts reuse sr / ar, already consumed
-          sr[cc] = pack_bf16(p0 - bf16_lo_f(pp[cc]), p1 - bf16_hi_f(pp[cc]));
-          ar[cc] = pack_bf16(q0 - bf16_lo_f(pa[cc]), q1 - bf16_hi_f(pa[cc]));
+      for (int i = 0; i < 16; ++i) {
+        const float2 x2 = fma2(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sc2, nm2);
+        const float2 p2 = make_float2(ex2(x2.x), ex2(x2.y));
+        l2 = add2(l2, p2);
+        const float2 q2 =
+            mul2(p2, add2(make_float2(__uint_as_float(ar[2 * i]), __uint_as_float(ar[2 * i + 1])), na2));
+        c2 = add2(c2, q2);
+        pp[i] = pack_bf16(p2.x, p2.y);
+        pa[i] = pack_bf16(q2.x, q2.y);
+        if (split) {   // lo parts reuse sr / ar entries already consumed
+          sr[i] = pack_bf16(p2.x - bf16_lo_f(pp[i]), p2.y - bf16_hi_f(pp[i]));
+          ar[i] = pack_bf16(q2.x - bf16_lo_f(pa[i]), q2.y - bf16_hi_f(pa[i]));
         }
       }
-      tmem_st32(tmem + lane_off + col_s(b2), pp);
-      tmem_st32(tmem + lane_off + col_a(b2), pa);
+      // Both halves have read S / A of this tile (the barrier above): overwrite.
+      tmem_st16(tmem + lane_off + col_s(b2) + cp, pp);
+      tmem_st16(tmem + lane_off + col_a(b2) + cp, pa);
       if (split) {
-        tmem_st32(tmem + lane_off + col_s(b2) + 32, *reinterpret_cast<uint32_t(*)[32]>(sr));
-        tmem_st32(tmem + lane_off + col_a(b2) + 32, *reinterpret_cast<uint32_t(*)[32]>(ar));
+        tmem_st16(tmem + lane_off + col_s(b2) + 32 + cp, sr);
+        tmem_st16(tmem + lane_off + col_a(b2) + 32 + cp, ar);
       }
       if (j >= 1) {
         // O may be touched only once the value products of tile j-1 are done.
-        if (!(ok = wait_warp(o_done, (j - 1) & 1))) break;
-        if (__any_sync(0xffffffffu, need)) {
+        const bool wo = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (j - 1) & 1));
+        fine = fine && wo;
+        if (wo && __any_sync(0xffffffffu, need)) {
           tc_fence_after();
 #pragma unroll 1
-          for (int part = 0; part < 8; ++part) {
+          for (int part = 0; part < 4; ++part) {
             uint32_t ov[32];
-            const uint32_t addr = tmem + lane_off + kColO1 + part * 32;   // O1 and O2 are contiguous
+            const uint32_t addr = tmem + lane_off + (g ? kColO2 : kColO1) + part * 32;
             tmem_ld32(addr, ov);
             tmem_wait_ld();
 #pragma unroll
@@ -319,18 +376,22 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_before();
       mbar_arrive(&p_full[b2]);
     }
-    if (!ok) *abort_flag = 1;
     // ---- epilogue: wait for the last value products, then write the rows
-    if (ok && wait_warp(o_done, (n - 1) & 1)) {
+    const bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(o_done, (n - 1) & 1);
+    lc_s[(g * 128 + r) * 2 + 0] = l2.x + l2.y;
+    lc_s[(g * 128 + r) * 2 + 1] = c2.x + c2.y;
+    if (bar_and(1, kPfSoftmax, wl)) {
       tc_fence_after();
-      const float inv = 1.f / l;
-      const float corr = 1.f + c * inv;
-      const size_t orow = ((size_t)(b * a.H + h) * a.T + t) * kPfD;
+      const float lt = lc_s[r * 2] + lc_s[(128 + r) * 2];
+      const float ct = lc_s[r * 2 + 1] + lc_s[(128 + r) * 2 + 1];
+      const float inv = 1.f / lt;
+      const float corr = 1.f + ct * inv;
+      const size_t orow = ((size_t)(b * a.H + h) * a.T + t) * kPfD + 64 * g;
 #pragma unroll 1
-      for (int part = 0; part < 4; ++part) {
+      for (int part = 0; part < 2; ++part) {
         uint32_t o1[32], o2[32];
-        tmem_ld32(tmem + lane_off + kColO1 + part * 32, o1);
-        tmem_ld32(tmem + lane_off + kColO2 + part * 32, o2);
+        tmem_ld32(tmem + lane_off + kColO1 + 64 * g + part * 32, o1);
+        tmem_ld32(tmem + lane_off + kColO2 + 64 * g + part * 32, o2);
         tmem_wait_ld();
         if (t < a.T) {
           float v[32];

@@ -96,7 +96,7 @@ def test_null_and_misaligned_pointers_rejected_before_launch(binding):
 
 
 @pytest.mark.parametrize("bad", [dict(seq_len=0), dict(head_dim=64), dict(in_dtype=0), dict(causal=2),
-                                 dict(num_heads=6, num_kv_heads=4)])
+                                 dict(num_heads=6, num_kv_heads=4), dict(scale=-0.1), dict(scale=0.0)])
 def test_invalid_prefill_params_are_rejected(binding, bad):
     base = dict(batch=1, num_heads=4, num_kv_heads=0, seq_len=16, head_dim=128, in_dtype=1, out_dtype=1,
                 scale=0.088, causal=1)
