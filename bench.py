@@ -190,6 +190,21 @@ class _F64View:
         return self.t[idx].double().cpu().numpy()
 
 
+def reduce_over_ranks(ms, total, device, world):
+    """Max of the per-rank times and sum of the per-rank work, over all ranks.
+
+    Every rank calls this with the same arguments shape (a collective);
+    world == 1 returns the inputs unchanged."""
+    if world == 1:
+        return float(ms), float(total)
+    t = torch.tensor([float(ms), float(total)], dtype=torch.float64, device=device)
+    tmax = t[:1].clone()
+    tsum = t[1:].clone()
+    torch.distributed.all_reduce(tmax, op=torch.distributed.ReduceOp.MAX)
+    torch.distributed.all_reduce(tsum, op=torch.distributed.ReduceOp.SUM)
+    return float(tmax[0]), float(tsum[0])
+
+
 def blas_threads():
     try:
         import threadpoolctl
@@ -284,14 +299,8 @@ def bench_decode(args, w, rank, world, dev, peaks, peaks_kind):
         torch.distributed.barrier()
     ms = start.elapsed_time(end)
     assert px.last_device_error() == 0, "device error during the timed steps"
-    ms_max = ms
     total_bytes = sum(bytes_per_step[i % copies] for i in range(K))
-    if world > 1:
-        t = torch.tensor([ms, float(total_bytes)], dtype=torch.float64, device=dev)
-        tm = t.clone()
-        torch.distributed.all_reduce(tm[:1], op=torch.distributed.ReduceOp.MAX)
-        torch.distributed.all_reduce(t[1:], op=torch.distributed.ReduceOp.SUM)
-        ms_max, total_bytes = float(tm[0]), float(t[1])
+    ms_max, total_bytes = reduce_over_ranks(ms, total_bytes, dev, world)
     gbs = total_bytes / (ms_max * 1e-3) / 1e9
     tokens_per_s = w.batch * K * world / (ms_max * 1e-3)
 
@@ -354,11 +363,7 @@ def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
     torch.cuda.synchronize()
     wall = time.perf_counter() - t0
     ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t[0])
-    total = sum(bytes_per_step[i % copies] for i in range(K)) * world
+    ms, total = reduce_over_ranks(ms, sum(bytes_per_step[i % copies] for i in range(K)), dev, world)
     h2d = insts[0]["q"].numel() * insts[0]["q"].element_size() * 2
     d2h = outs[0].numel() * outs[0].element_size()
     return {"value": round(total / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
@@ -398,13 +403,9 @@ def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
     if world > 1:
         torch.distributed.barrier()
     ms = start.elapsed_time(end)
-    ms_max = ms
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_max = float(t[0])
     flops = W.prefill_flops(w)
-    tflops = flops * K * world / (ms_max * 1e-3) / 1e12
+    ms_max, total_flops = reduce_over_ranks(ms, flops * K, dev, world)
+    tflops = total_flops / (ms_max * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     achieved = flops / (ms * 1e-3 / K) / 1e12
 

@@ -245,8 +245,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       if (j >= 1) {
         const int jp = j - 1, bp = jp & 1, sp = jp % kPfStages;
-        if (!(ok = wait_warp(&p_full[bp], (jp >> 1) & 1))) break;
+        // V(j-1) landed long ago; waiting on it first keeps it off the path
+        // from the softmax's arrival to the value products.
         if (!(ok = wait_warp(&v_full[sp], (jp / kPfStages) & 1))) break;
+        if (!(ok = wait_warp(&p_full[bp], (jp >> 1) & 1))) break;
         tc_fence_after();
         const uint64_t dvs = dv + (uint64_t)((sp * L::kKVBytes) >> 4);
 #pragma unroll
@@ -296,7 +298,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc_fence_after();
       uint32_t sr[32], ar[32];
       tmem_ld32(tmem + lane_off + col_s(b2) + cs, sr);
-      tmem_ld32(tmem + lane_off + col_a(b2) + cs, ar);
       tmem_wait_ld();
       // Tiles that reach the diagonal or the sequence end need the mask.
       const int key0 = j * kPfBN + (int)cs;
@@ -310,8 +311,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < 32; ++cc) mx = fmaxf(mx, __uint_as_float(sr[cc]));
       red_max[((j & 1) * 2 + g) * 128 + r] = mx;
-      if (j == 0 && g == 0) aref_s[r] = __uint_as_float(ar[0]);
-      if (!bar_and(1, kPfSoftmax, w && fine)) {
+      // The probe values are loaded while the two halves exchange their max.
+      tmem_ld32(tmem + lane_off + col_a(b2) + cs, ar);
+      if (j == 0 && g == 0) {
+        tmem_wait_ld();
+        aref_s[r] = __uint_as_float(ar[0]);
+      }
+      const bool go = bar_and(1, kPfSoftmax, w && fine);
+      tmem_wait_ld();
+      if (!go) {
         fine = false;
         break;
       }
@@ -354,8 +362,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_st16(tmem + lane_off + col_s(b2) + 32 + cp, sr);
         tmem_st16(tmem + lane_off + col_a(b2) + 32 + cp, ar);
       }
-      if (j >= 1) {
-        // O may be touched only once the value products of tile j-1 are done.
+      // O may be touched only once the value products of tile j-1 are done.
+      // Waiting on that one phase is exact without waiting on the earlier
+      // ones: s_full(j) was committed after the value products of tile j-2, so
+      // o_done has completed phase j-2, and tile j's value products cannot
+      // start before this warpgroup arrives on p_full(j); its phase is j-1 or
+      // j.  The wait is skipped unless O is rescaled, except at the last tile,
+      // which pins the phase for the epilogue's wait to n-1 or n.
+      if (j >= 1 && (j == n - 1 || __any_sync(0xffffffffu, need))) {
         const bool wo = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (j - 1) & 1));
         fine = fine && wo;
         if (wo && __any_sync(0xffffffffu, need)) {
