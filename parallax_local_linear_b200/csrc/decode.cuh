@@ -103,37 +103,53 @@ struct TileSpace {
   __device__ __forceinline__ long long owner(long long x) const { return ((x + 1) * G + T - 1) / T - 1; }
 };
 
-// Fills pre[0..B] and lens[0..B) in shared memory; all threads of the CTA call it.
+// Fills pre[0..B] and lens[0..B) in shared memory; all threads of the CTA
+// call it.  Without seq_lens the prefix is closed-form; otherwise it is a
+// block-wide scan (per-thread chunk sums, warp shuffles, warp totals).
 __device__ void build_tile_space(const DecodeArgs& a, int* pre, int* lens, int* scratch) {
   const int tid = threadIdx.x, nt = blockDim.x;
+  const int lane = tid & 31, wid = tid >> 5, nw = nt >> 5;
+  if (a.seq_lens == nullptr) {
+    const int per_seq = ((a.kv_len + kTile - 1) / kTile) * a.units_per_seq;
+    for (int b = tid; b <= a.B; b += nt) {
+      pre[b] = b * per_seq;
+      if (b < a.B) lens[b] = a.kv_len;
+    }
+    __syncthreads();
+    return;
+  }
   const int per = (a.B + nt - 1) / nt;
   const int b0 = min(a.B, tid * per), b1 = min(a.B, b0 + per);
   int sum = 0;
   for (int b = b0; b < b1; ++b) {
-    int n = a.kv_len;
-    if (a.seq_lens != nullptr) {
-      n = __ldg(a.seq_lens + b);
-      if (n < 0 || n > a.kv_len) {
-        report_error(4 /* PLX_DEVERR_BAD_LENGTH */);
-        n = n < 0 ? 0 : a.kv_len;
-      }
+    int n = __ldg(a.seq_lens + b);
+    if (n < 0 || n > a.kv_len) {
+      report_error(4 /* PLX_DEVERR_BAD_LENGTH */);
+      n = n < 0 ? 0 : a.kv_len;
     }
     lens[b] = n;
     sum += ((n + kTile - 1) / kTile) * a.units_per_seq;
   }
-  scratch[tid] = sum;
+  // inclusive scan of `sum` within the warp
+  int inc = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+  }
+  if (lane == 31) scratch[wid] = inc;
   __syncthreads();
   if (tid == 0) {
     int run = 0;
-    for (int i = 0; i < nt; ++i) {
-      const int v = scratch[i];
-      scratch[i] = run;
+    for (int w = 0; w < nw; ++w) {
+      const int v = scratch[w];
+      scratch[w] = run;
       run += v;
     }
     pre[a.B] = run;
   }
   __syncthreads();
-  int run = scratch[tid];
+  int run = scratch[wid] + inc - sum;   // exclusive prefix of this thread's chunk
   for (int b = b0; b < b1; ++b) {
     pre[b] = run;
     run += ((lens[b] + kTile - 1) / kTile) * a.units_per_seq;
@@ -185,10 +201,12 @@ struct CtaState {
 // unit, otherwise this piece's partial and, in the last CTA to finish a piece
 // of the unit, the merge of all pieces.  Called by the `nt` threads (ids
 // 0..nt-1) that synchronise through `bar`, after `st` is complete and
-// synchronised.
+// synchronised.  `scratch` is shared memory of `scratch_cap` floats that no
+// other code uses meanwhile.
 template <int D, typename Bar>
 __device__ void finish_unit(const DecodeArgs& a, const TileSpace& ts, const CtaState<D>& st, int b, int hu,
-                            long long ua, long long ub, int tid, int nt, int* s_flag, Bar bar) {
+                            long long ua, long long ub, int tid, int nt, int* s_flag, float* scratch,
+                            int scratch_cap, Bar bar) {
   const int nheads = a.heads_per_unit;
   const int hq0 = hu * nheads;
   const long long c = blockIdx.x;
@@ -231,14 +249,27 @@ __device__ void finish_unit(const DecodeArgs& a, const TileSpace& ts, const CtaS
   bar();   // everyone has read the flag before it can be reused
   if (!last) return;
   __threadfence();
+  // The pieces' maxima go to shared memory in one round of parallel loads;
+  // the sums are then read four pieces at a time, so the merge costs a few
+  // L2 round trips instead of one per piece.
+  const int np = (int)(c1 - c0 + 1);
+  const bool staged = np * nheads <= scratch_cap;
+  if (staged) {
+    for (int i = tid; i < np * nheads; i += nt)
+      scratch[i] = __ldcg(a.slots + slot_of(c0 + i / nheads) * slot_stride + (i % nheads) * P);
+    bar();
+  }
   for (int i = tid; i < nheads * D; i += nt) {
     const int h = i / D, d = i % D;
     float M = -INFINITY;
-    for (long long cc = c0; cc <= c1; ++cc) M = fmaxf(M, __ldcg(a.slots + slot_of(cc) * slot_stride + h * P));
+    for (int q = 0; q < np; ++q)
+      M = fmaxf(M, staged ? scratch[q * nheads + h] : __ldcg(a.slots + slot_of(c0 + q) * slot_stride + h * P));
     float L = 0.f, C = 0.f, O1 = 0.f, O2 = 0.f;
-    for (long long cc = c0; cc <= c1; ++cc) {
-      const float* ps = a.slots + slot_of(cc) * slot_stride + h * P;
-      const float al = ex2(__ldcg(ps) - M);
+#pragma unroll 4
+    for (int q = 0; q < np; ++q) {
+      const float* ps = a.slots + slot_of(c0 + q) * slot_stride + h * P;
+      const float mq = staged ? scratch[q * nheads + h] : __ldcg(ps);
+      const float al = ex2(mq - M);
       L += al * __ldcg(ps + 1);
       C += al * __ldcg(ps + 2);
       O1 += al * __ldcg(ps + 4 + d);
@@ -246,6 +277,7 @@ __device__ void finish_unit(const DecodeArgs& a, const TileSpace& ts, const CtaS
     }
     store_out(a, ((size_t)b * a.Hq + hq0 + h) * D + d, finalize(O1, O2, L, C));
   }
+  if (staged) bar();   // the scratch is free again
 }
 
 // =========================================================================
@@ -292,6 +324,12 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const DecodeArgs a) {
   using SM = TcSmem<D>;
+  // Consumer warp w takes tiles t = w (mod NC) and tile t sits in stage
+  // t % STAGES.  The parity wait on full[t % STAGES] is exact only if tile
+  // t - STAGES, the previous load into that stage, was consumed by the same
+  // warp, which holds exactly when NC divides STAGES: then each warp owns its
+  // stages and cannot run a whole ring ahead of a slower warp.
+  static_assert(STAGES % NC == 0, "each consumer warp must own whole stages");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* wstate = reinterpret_cast<float*>(ring + STAGES * SM::kStageBytes);
@@ -599,7 +637,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         }
       }
       bar();
-      finish_unit<D>(a, ts, st, b, kvh, ua, ub, tid, NT, s_flag, bar);
+      finish_unit<D>(a, ts, st, b, kvh, ua, ub, tid, NT, s_flag, wstate, NC * SM::kWarpStateFloats, bar);
       bar();   // per-warp states and st are free again
       x = seg_end;
       cur.next_unit(ts);
@@ -756,7 +794,7 @@ __global__ void __launch_bounds__(NW * 32)
       }
     }
     __syncthreads();
-    finish_unit<D>(a, ts, st, b, hq, ua, ub, tid, NT, s_flag, bar);
+    finish_unit<D>(a, ts, st, b, hq, ua, ub, tid, NT, s_flag, &s_o[0][0][0], NW * 2 * D, bar);
     __syncthreads();
     x = seg_end;
     cur.next_unit(ts);

@@ -29,8 +29,8 @@ constexpr int kMaxDevices = 64;
 #define PLX_DECODE_STAGES 4
 #endif
 constexpr int kDecodeNC = 4;
-constexpr int kDecodeStages128 = PLX_DECODE_STAGES;
-constexpr int kDecodeStages64 = 6;
+constexpr int kDecodeStages128 = PLX_DECODE_STAGES;   // a multiple of kDecodeNC
+constexpr int kDecodeStages64 = 8;
 constexpr int kDecodeF32Warps = 4;
 
 // Persistent grid of the fp32 path, in CTAs per SM (its CTAs are small).

@@ -229,3 +229,15 @@ def test_short_sequences_keep_near_fp32_accuracy(px, L, group):
     out = _run(px, inp, out_dtype=torch.float32)
     ref = oracle_heads(inp, _all_heads(inp))
     assert_parity(out.cpu().numpy(), ref, 2e-3, f"short L={L} g={group}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_long_chunks_let_warps_run_ahead(px, d):
+    # Few units and long sequences: every CTA streams tens of tiles, so its
+    # consumer warps can drift a full ring apart (the stage / warp ownership
+    # rule of the pipeline is what keeps their barrier waits exact).
+    inp = _to(W.small_decode_inputs(1, 4, 1, d, 60000, seed=77))
+    out = _run(px, inp, out_dtype=torch.float32, num_ctas=16)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.cpu().numpy(), ref, TOL_BF16, f"long chunks d={d}")
+    assert px.last_device_error() == 0
