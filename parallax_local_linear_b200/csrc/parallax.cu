@@ -118,8 +118,17 @@ DecodePlan plan_decode(const plx_decode_params* p, int num_sms) {
   const bool bf16 = p->in_dtype == PLX_BF16;
   pl.units_per_seq = bf16 ? p->num_kv_heads : p->num_q_heads;
   pl.heads_per_unit = bf16 ? p->num_q_heads / p->num_kv_heads : 1;
-  const int64_t tiles = (int64_t)p->batch * pl.units_per_seq * ((p->kv_len + kTile - 1) / kTile);
+  const int64_t units = (int64_t)p->batch * pl.units_per_seq;
+  const int64_t tiles = units * ((p->kv_len + kTile - 1) / kTile);
   int64_t ctas = p->num_ctas > 0 ? p->num_ctas : (int64_t)num_sms * (bf16 ? 1 : kF32CtasPerSm);
+  if (p->num_ctas == 0 && bf16 && p->page_size == 0 && units <= num_sms) {
+    // A contiguous cache usually holds equal-length sequences: cut each unit
+    // into k equal pieces, one per CTA, so that no CTA crosses a unit
+    // boundary, as long as that keeps most SMs busy.  Any grid is correct
+    // (stream-K handles ragged lengths); paged caches keep one CTA per SM.
+    const int64_t k = num_sms / units;
+    if (4 * units * k >= 3 * (int64_t)num_sms) ctas = units * k;
+  }
   if (ctas > tiles) ctas = tiles;
   if (ctas < 1) ctas = 1;
   if (ctas > INT32_MAX / 4) ctas = INT32_MAX / 4;

@@ -106,9 +106,14 @@ def test_invalid_prefill_params_are_rejected(binding, bad):
     assert st in (1, 2)
 
 
-def _expected_plan(B, units, heads_per_unit, L, d=128, num_sms=148, forced=0, per_sm=1):
+def _expected_plan(B, units, heads_per_unit, L, d=128, num_sms=148, forced=0, per_sm=1, paged=False):
     tiles = B * units * (-(-L // 64))
     ctas = forced if forced else num_sms * per_sm
+    n_units = B * units
+    if not forced and per_sm == 1 and not paged and n_units <= num_sms:
+        k = num_sms // n_units
+        if 4 * n_units * k >= 3 * num_sms:
+            ctas = n_units * k
     ctas = max(1, min(ctas, tiles))
     counters = -(-(B * units * 4) // 256) * 256
     return ctas, counters + 2 * ctas * heads_per_unit * (2 * d + 4) * 4
