@@ -52,6 +52,7 @@ struct DecodeArgs {
   int kv_len, paged, num_pages, max_pages;
   float scale_log2;                // scale * log2(e)
   int out_bf16;
+  int cluster;                     // > 1: each unit is one cluster of this many CTAs (bf16 path)
 };
 
 // ------------------------------------------------------------ addressing
@@ -311,12 +312,17 @@ struct TcSmem {
   static constexpr int kWarpStateFloats = 16 * D + 24;       // m[8] l[8] c[8] O[16][D]
 };
 
+// Cluster merge: the other CTAs of a unit's cluster deposit their state in
+// rank 0's receive area (at most kMaxClusterRecv states).
+constexpr int kMaxClusterRecv = 2;
+
 template <int D, int STAGES, int NC>
 constexpr int tc_smem_fixed_bytes() {
-  // ring + per-warp states + merged state + barriers + flags + scan scratch
-  // + 1 KB alignment slack (the prefix table, (2B + 1) ints, comes on top)
-  return STAGES * TcSmem<D>::kStageBytes + NC * TcSmem<D>::kWarpStateFloats * 4 + (int)sizeof(CtaState<D>) +
-         2 * STAGES * 8 + 16 + (NC + 1) * 32 * 4 + 1024;
+  // ring + per-warp states + merged state + cluster receive area + barriers +
+  // flags + scan scratch + 1 KB alignment slack (the prefix table, (2B + 1)
+  // ints, comes on top)
+  return STAGES * TcSmem<D>::kStageBytes + NC * TcSmem<D>::kWarpStateFloats * 4 +
+         (1 + kMaxClusterRecv) * (int)sizeof(CtaState<D>) + 2 * STAGES * 8 + 16 + (NC + 1) * 32 * 4 + 1024;
 }
 
 template <int D, int STAGES, int NC, bool kLoInPad>
@@ -334,7 +340,8 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* wstate = reinterpret_cast<float*>(ring + STAGES * SM::kStageBytes);
   CtaState<D>& st = *reinterpret_cast<CtaState<D>*>(wstate + NC * SM::kWarpStateFloats);
-  uint64_t* full = reinterpret_cast<uint64_t*>(&st + 1);
+  CtaState<D>* recv = &st + 1;                               // [kMaxClusterRecv]
+  uint64_t* full = reinterpret_cast<uint64_t*>(recv + kMaxClusterRecv);
   uint64_t* empty = full + STAGES;
   int* s_flag = reinterpret_cast<int*>(empty + STAGES);    // [0]: last-piece flag, [1]: abort
   int* scan = s_flag + 4;                                  // [(NC + 1) * 32]
@@ -366,6 +373,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     fence_mbarrier_init();
   }
   __syncthreads();
+  if (a.cluster > 1) cluster_arrive_relaxed();
   volatile int* abort_flag = s_flag + 1;
   const int nchunk = (int)(x1 - x0);
 
@@ -637,6 +645,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         }
       }
       bar();
+      if (a.cluster > 1) break;   // one unit per CTA; merged across the cluster below
       finish_unit<D>(a, ts, st, b, kvh, ua, ub, tid, NT, s_flag, wstate, NC * SM::kWarpStateFloats, bar);
       bar();   // per-warp states and st are free again
       x = seg_end;
@@ -644,6 +653,44 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     }
   }
   __syncthreads();
+  if (a.cluster > 1) {
+    // The cluster's CTAs hold one piece each of the same unit (the grid is
+    // unit-aligned).  Ranks >= 1 write their merged state into rank 0's
+    // receive area through distributed shared memory; after the cluster
+    // barrier (release / acquire) rank 0 merges and writes the output.
+    const int k = a.cluster;
+    const int rank = blockIdx.x % k;
+    const int unit = blockIdx.x / k;
+    const int b = unit / a.Hkv, kvh = unit % a.Hkv, hq0 = kvh * g;
+    cluster_wait();   // every CTA of the cluster has started
+    if (rank > 0) {
+      const uint32_t remote = dsmem_map(smem_u32(&recv[rank - 1]), 0);
+      const float* src = reinterpret_cast<const float*>(&st);
+      constexpr int kFloats = (int)(sizeof(CtaState<D>) / 4);
+      for (int i = threadIdx.x; i < kFloats; i += blockDim.x) {
+        // only the live heads' rows matter, but the state is small: copy it whole
+        dsmem_st_f32(remote + 4u * i, src[i]);
+      }
+    }
+    cluster_sync();
+    if (rank == 0) {
+      for (int i = threadIdx.x; i < g * D; i += blockDim.x) {
+        const int h = i / D, d = i % D;
+        float M = st.m[h];
+        for (int r = 0; r < k - 1; ++r) M = fmaxf(M, recv[r].m[h]);
+        const float a0 = ex2(st.m[h] - M);
+        float L = a0 * st.l[h], C = a0 * st.c[h], O1 = a0 * st.o1[h][d], O2 = a0 * st.o2[h][d];
+        for (int r = 0; r < k - 1; ++r) {
+          const float al = ex2(recv[r].m[h] - M);
+          L += al * recv[r].l[h];
+          C += al * recv[r].c[h];
+          O1 += al * recv[r].o1[h][d];
+          O2 += al * recv[r].o2[h][d];
+        }
+        store_out(a, ((size_t)b * a.Hq + hq0 + h) * D + d, finalize(O1, O2, L, C));
+      }
+    }
+  }
 }
 
 // =========================================================================

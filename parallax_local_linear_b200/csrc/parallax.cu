@@ -152,7 +152,29 @@ plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CU
   auto kern = decode_tc_kernel<D, STAGES, kDecodeNC, kLoInPad>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
-  kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
+  if (a.cluster <= 1) {
+    kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
+    return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas);
+  cfg.blockDim = dim3((kDecodeNC + 1) * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = a.cluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, tk, tv, a) == cudaSuccess) return PLX_OK;
+  // Clusters could not be scheduled (a launch-configuration error, which is
+  // not sticky): run the same grid with the global-memory merge instead.
+  (void)cudaGetLastError();
+  DecodeArgs b = a;
+  b.cluster = 1;
+  kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, b);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
@@ -319,6 +341,15 @@ plx_status parallax_decode(const void* q, const void* rho, const void* k_cache, 
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
 
+  // Units of equal length cut into k pieces each (the unit-aligned grid) are
+  // merged through distributed shared memory when each unit is one cluster.
+  a.cluster = 1;
+  if (p->in_dtype == PLX_BF16 && !paged && seq_lens == nullptr && p->num_ctas == 0) {
+    const int64_t units = (int64_t)p->batch * p->num_kv_heads;
+    const int64_t k = pl.ctas / units;
+    const int64_t tiles_per_unit = (p->kv_len + kTile - 1) / kTile;
+    if (k >= 2 && k <= 1 + kMaxClusterRecv && k * units == pl.ctas && tiles_per_unit >= k) a.cluster = (int)k;
+  }
   const size_t smem = decode_smem_bytes(p);
   if (smem > 227 * 1024) return PLX_ERR_UNSUPPORTED;
   if (p->in_dtype == PLX_F32)

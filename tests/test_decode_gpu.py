@@ -241,3 +241,22 @@ def test_long_chunks_let_warps_run_ahead(px, d):
     ref = oracle_heads(inp, _all_heads(inp))
     assert_parity(out.cpu().numpy(), ref, TOL_BF16, f"long chunks d={d}")
     assert px.last_device_error() == 0
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,L", [(8, 16, 8, 4096), (6, 32, 8, 1000), (4, 8, 2, 129), (16, 32, 8, 300)])
+def test_unit_aligned_grid_and_cluster_merge(px, B, Hq, Hkv, L):
+    # Equal-length contiguous caches run on a grid of k CTAs per (sequence,
+    # KV head); for k = 2 or 3 each unit is one thread-block cluster that
+    # merges its pieces through distributed shared memory.
+    import ctypes
+    inp = _to(W.small_decode_inputs(B, Hq, Hkv, 128, L, seed=B * 1000 + L))
+    p = px.decode_params(inp["q"], inp["k_cache"])
+    ctas = px.decode_num_ctas(p)
+    units = B * Hkv
+    assert ctas % units == 0 or ctas == min(148, units * (-(-L // 64)))
+    out = _run(px, inp, out_dtype=torch.float32)
+    ref = oracle_heads(inp, _all_heads(inp))
+    assert_parity(out.cpu().numpy(), ref, TOL_BF16, f"aligned B={B} Hkv={Hkv} L={L} ctas={ctas}")
+    again = _run(px, inp, out_dtype=torch.float32)
+    assert torch.equal(out, again)
+    assert px.last_device_error() == 0
