@@ -22,4 +22,5 @@ from .parallax_oracle import (  # noqa: F401
     decode,
     gather_paged_keys,
     prefill_rows,
+    prefill_paged_rows,
 )

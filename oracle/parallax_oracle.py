@@ -25,6 +25,9 @@ design notes):
   * The covariance uses the same softmax weights as vbar.
   * rho is used as given: ``scale`` multiplies q.k only.
   * Causal prefill: key i is visible to query t iff i <= t.
+  * Chunked prefill (a serving step the pages do not describe): the queries
+    of a chunk are the last positions of their sequence, and a query at
+    position t sees keys 0..t like any causal row.
   * Grouped-query attention: query head h reads KV head h // (Hq / Hkv).
   * An empty key set gives a zero output.
 """
@@ -40,6 +43,7 @@ __all__ = [
     "decode",
     "gather_paged_keys",
     "prefill_rows",
+    "prefill_paged_rows",
 ]
 
 
@@ -173,3 +177,36 @@ def prefill_rows(q, rho, k, v, rows, scale: float, causal: bool = True):
         res.append(parallax_query(q[b, h, t], rho[b, h, t],
                                   k[b, kvh, :n, :], v[b, kvh, :n, :], scale))
     return np.stack(res) if res else np.zeros((0, v.shape[-1]))
+
+
+def prefill_paged_rows(q, rho, k_pool, v_pool, page_table, cu_seqlens_q, seq_lens, rows,
+                       scale: float, causal: bool = True):
+    """Chunked (append) prefill over a paged cache, for selected rows.
+
+    Sequence b holds ``seq_lens[b]`` keys in the pools [P, Hkv, page_size, d]
+    through ``page_table[b]``.  Its q_len = cu_seqlens_q[b+1] - cu_seqlens_q[b]
+    queries are packed in q, rho [total_q, H, d] from row cu_seqlens_q[b] and
+    are the sequence's last positions: query i sits at position
+    t = seq_lens[b] - q_len + i and attends to keys 0..t when ``causal``,
+    else to all seq_lens[b] keys.  ``rows``: iterable of (b, i, h).
+    Returns float64 [len(rows), d_v] in the order of ``rows``.
+    """
+    H = q.shape[1]
+    Hkv = k_pool.shape[1]
+    group = H // Hkv
+    gathered = {}
+    res = []
+    for b, i, h in rows:
+        start = int(cu_seqlens_q[b])
+        q_len = int(cu_seqlens_q[b + 1]) - start
+        L = int(seq_lens[b])
+        assert 0 <= i < q_len <= L, (b, i, q_len, L)
+        t = L - q_len + i
+        n = t + 1 if causal else L
+        kvh = h // group
+        if (b, kvh) not in gathered:
+            gathered[(b, kvh)] = (gather_paged_keys(k_pool, page_table[b], L, kvh),
+                                  gather_paged_keys(v_pool, page_table[b], L, kvh))
+        K, V = gathered[(b, kvh)]
+        res.append(parallax_query(q[start + i, h], rho[start + i, h], K[:n], V[:n], scale))
+    return np.stack(res) if res else np.zeros((0, v_pool.shape[-1]))

@@ -276,6 +276,141 @@ def test_prefill_rows_equal_decode_over_prefix():
 
 
 # --------------------------------------------------------------------------
+# Chunked (append) prefill over a paged cache
+# --------------------------------------------------------------------------
+
+def _to_pages(seqs, ps, rng, fill=np.nan):
+    """Place per-sequence [Hkv, L_b, d] arrays into a permuted page pool."""
+    Hkv, d = seqs[0].shape[0], seqs[0].shape[2]
+    n_pages = [-(-s.shape[1] // ps) for s in seqs]
+    perm = rng.permutation(max(1, sum(n_pages)))
+    pool = np.full((max(1, sum(n_pages)), Hkv, ps, d), fill)
+    table = -np.ones((len(seqs), max(1, max(n_pages))), dtype=np.int64)
+    nxt = 0
+    for b, s in enumerate(seqs):
+        for j in range(n_pages[b]):
+            page = perm[nxt]
+            nxt += 1
+            table[b, j] = page
+            take = min(ps, s.shape[1] - j * ps)
+            pool[page, :, :take] = s[:, j * ps:j * ps + take]
+    return pool, table
+
+
+def _chunked_case(rng):
+    """Dense sequences plus a paged chunk holding each one's last q_len positions."""
+    H, Hkv, d, ps = 4, 2, 4, 8
+    lens, q_lens = [21, 8, 5, 17], [6, 8, 1, 17]
+    T = max(lens)
+    q = rng.standard_normal((len(lens), H, T, d))
+    rho = rng.standard_normal((len(lens), H, T, d))
+    k = rng.standard_normal((len(lens), Hkv, T, d))
+    v = rng.standard_normal((len(lens), Hkv, T, d))
+    kp, table = _to_pages([k[b, :, :n] for b, n in enumerate(lens)], ps, rng)
+    vp = np.full_like(kp, np.nan)   # V in the pages K's table names
+    for b, n in enumerate(lens):
+        for j in range(-(-n // ps)):
+            take = min(ps, n - j * ps)
+            vp[table[b, j], :, :take] = v[b, :, j * ps:j * ps + take]
+    cu = np.concatenate([[0], np.cumsum(q_lens)])
+    qp = np.concatenate([q[b, :, n - m:n].transpose(1, 0, 2) for b, (n, m) in enumerate(zip(lens, q_lens))])
+    rp = np.concatenate([rho[b, :, n - m:n].transpose(1, 0, 2) for b, (n, m) in enumerate(zip(lens, q_lens))])
+    return dict(q=q, rho=rho, k=k, v=v, qp=qp, rp=rp, kp=kp, vp=vp, table=table, cu=cu,
+                lens=lens, q_lens=q_lens, H=H)
+
+
+def _check_chunk_rows_equal_dense_rows(fn):
+    c = _chunked_case(np.random.default_rng(11))
+    rows = [(b, i, h) for b, m in enumerate(c["q_lens"]) for i in range(m) for h in range(c["H"])]
+    out = fn(c["qp"], c["rp"], c["kp"], c["vp"], c["table"], c["cu"], c["lens"], rows, 0.5, causal=True)
+    for (b, i, h), o in zip(rows, out):
+        t = c["lens"][b] - c["q_lens"][b] + i     # a chunk's queries are the sequence's last positions
+        ref = oracle.prefill_rows(c["q"][:, :, :c["lens"][b]], c["rho"][:, :, :c["lens"][b]],
+                                  c["k"][:, :, :c["lens"][b]], c["v"][:, :, :c["lens"][b]],
+                                  [(b, h, t)], 0.5, causal=True)[0]
+        np.testing.assert_array_equal(o, ref)
+    full = fn(c["qp"], c["rp"], c["kp"], c["vp"], c["table"], c["cu"], c["lens"], rows, 0.5, causal=False)
+    for (b, i, h), o in zip(rows, full):
+        t = c["lens"][b] - c["q_lens"][b] + i
+        n = c["lens"][b]
+        np.testing.assert_array_equal(
+            o, oracle.parallax_query(c["q"][b, h, t], c["rho"][b, h, t], c["k"][b, h // 2, :n],
+                                     c["v"][b, h // 2, :n], 0.5))
+
+
+def test_paged_chunk_rows_equal_dense_prefill_rows():
+    _check_chunk_rows_equal_dense_rows(oracle.prefill_paged_rows)
+
+
+def test_paged_chunk_of_one_token_is_paged_decode():
+    c = _chunked_case(np.random.default_rng(12))
+    q1 = np.stack([c["qp"][c["cu"][b + 1] - 1] for b in range(4)])
+    r1 = np.stack([c["rp"][c["cu"][b + 1] - 1] for b in range(4)])
+    dec = oracle.decode(q1, r1, c["kp"], c["vp"], 0.5, seq_lens=c["lens"], page_table=c["table"])
+    ones = np.arange(5)   # cu_seqlens_q of four one-token chunks
+    rows = [(b, 0, h) for b in range(4) for h in range(c["H"])]
+    out = oracle.prefill_paged_rows(q1.reshape(4, c["H"], -1), r1.reshape(4, c["H"], -1), c["kp"], c["vp"],
+                                    c["table"], ones, c["lens"], rows, 0.5, causal=True)
+    for (b, _, h), o in zip(rows, out):
+        np.testing.assert_array_equal(o, dec[b, h])
+
+
+def test_worked_example_as_paged_chunk():
+    # The three keys of [three_keys_unequal_weights] in two 2-token pages
+    # (physical order swapped); a chunk of two queries at positions 1 and 2:
+    # the last sees all three keys and must give the worked answer, the
+    # first sees keys 0 and 1 only.
+    c = load_worked_examples()["three_keys_unequal_weights"]
+    pool_k = np.full((2, 1, 2, 3), np.nan)
+    pool_v = np.full((2, 1, 2, 3), np.nan)
+    pool_k[1, 0, :2], pool_k[0, 0, :1] = c["k"][:2], c["k"][2:]
+    pool_v[1, 0, :2], pool_v[0, 0, :1] = c["v"][:2], c["v"][2:]
+    table = np.array([[1, 0]])
+    q = np.stack([np.array([0.0, 0.0, 0.0]), c["q"]])[:, None]
+    rho = np.stack([np.array([1.0, 0.0, 0.0]), c["rho"]])[:, None]
+    out = oracle.prefill_paged_rows(q, rho, pool_k, pool_v, table, [0, 2], [3], [(0, 0, 0), (0, 1, 0)],
+                                    c["scale"], causal=True)
+    np.testing.assert_allclose(out[1], c["out"], atol=1e-13)
+    # row 0: equal weights over keys 0, 1: vbar = (2, 4, 0), kbar = (1/2, 1/2, 0),
+    # (k - kbar).rho = +1/2, -1/2; Sigma^T rho = 1/2*(1/2)(2,-4,0) + 1/2*(-1/2)(-2,4,0) = (1, -2, 0)
+    np.testing.assert_allclose(out[0], [1.0, 6.0, 0.0], atol=1e-13)
+
+
+def _mutant_chunk_position(q, rho, k_pool, v_pool, page_table, cu, seq_lens, rows, scale, causal=True):
+    # places the chunk at the START of the sequence instead of its end
+    res = []
+    for b, i, h in rows:
+        start = int(cu[b])
+        kvh = h // (q.shape[1] // k_pool.shape[1])
+        n = i + 1 if causal else int(seq_lens[b])
+        K = po.gather_paged_keys(k_pool, page_table[b], n, kvh)
+        V = po.gather_paged_keys(v_pool, page_table[b], n, kvh)
+        res.append(po.parallax_query(q[start + i, h], rho[start + i, h], K, V, scale))
+    return np.stack(res)
+
+
+def _mutant_chunk_exclusive(q, rho, k_pool, v_pool, page_table, cu, seq_lens, rows, scale, causal=True):
+    # the diagonal left out: query at position t sees keys 0..t-1 (and key 0 at t = 0)
+    res = []
+    for b, i, h in rows:
+        start = int(cu[b])
+        L = int(seq_lens[b])
+        t = L - (int(cu[b + 1]) - start) + i
+        kvh = h // (q.shape[1] // k_pool.shape[1])
+        n = max(t, 1) if causal else L
+        K = po.gather_paged_keys(k_pool, page_table[b], n, kvh)
+        V = po.gather_paged_keys(v_pool, page_table[b], n, kvh)
+        res.append(po.parallax_query(q[start + i, h], rho[start + i, h], K, V, scale))
+    return np.stack(res)
+
+
+@pytest.mark.parametrize("mutant", [_mutant_chunk_position, _mutant_chunk_exclusive])
+def test_chunk_pin_catches_planted_mistakes(mutant):
+    with pytest.raises(AssertionError):
+        _check_chunk_rows_equal_dense_rows(mutant)
+
+
+# --------------------------------------------------------------------------
 # Mutation tests: plausible mistakes planted in the oracle must fail a pin
 # --------------------------------------------------------------------------
 
