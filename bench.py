@@ -78,7 +78,7 @@ def parse_args(argv=None):
 
 def default_steps(workload):
     return {"decode_f32": 20000, "decode_bf16": 8192, "decode_long": 200, "decode_paged": 200,
-            "prefill": 20}[workload]
+            "prefill": 20, "prefill_paged": 20}[workload]
 
 
 def dist_env():
@@ -444,6 +444,86 @@ def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
     return res, x
 
 
+def bench_prefill_paged(args, w, rank, world, dev, peaks, peaks_kind):
+    """Chunked prefill over the paged cache: one call per step."""
+    from parallax_local_linear_b200 import binding as px
+
+    x = W.chunked_prefill_inputs(w, device=dev, seed=w.seed + 1000 * rank)
+    out = torch.empty_like(x["q"])
+    meta = ("page_table", "cu_seqlens_q", "seq_lens")
+
+    def call(src):
+        px.prefill_paged(src["q"], src["rho"], x["k_cache"], x["v_cache"], src["page_table"],
+                         src["cu_seqlens_q"], src["seq_lens"], max_q_len=x["max_q_len"], scale=x["scale"],
+                         causal=w.causal, out=out)
+
+    for _ in range(max(args.warmup, 3)):
+        call(x)
+    torch.cuda.synchronize()
+    assert px.last_device_error() == 0
+    K = args.steps
+    stream = torch.cuda.current_stream()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record(stream)
+        for _ in range(K):
+            call(x)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    flops = W.chunked_prefill_flops(x["q_lens"], x["seq_lens_host"], w.num_heads, w.head_dim, w.causal)
+    ms_max, total_flops = reduce_over_ranks(ms, flops * K, dev, world)
+    tflops = total_flops / (ms_max * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved = flops / (ms * 1e-3 / K) / 1e12
+
+    # e2e through the public API: each step copies the chunk's queries, probes
+    # and the batch's page table / lengths from pinned host memory and reads
+    # the output back; the KV cache is resident device state.
+    hx = {k: x[k].cpu().pin_memory() for k in ("q", "rho") + meta}
+    dx = {k: torch.empty_like(x[k]) for k in hx}
+    oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    Ke = max(1, min(K, 10))
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(Ke):
+        for k in hx:
+            dx[k].copy_(hx[k], non_blocking=True)
+        call(dx)
+        oh.copy_(out, non_blocking=True)
+    e2.record()
+    torch.cuda.synchronize()
+    ems = s2.elapsed_time(e2)
+    e2e = {"value": round(flops * Ke / (ems * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hx.values()),
+           "d2h_bytes_per_step": out.numel() * out.element_size(), "steps": Ke,
+           "resident": "paged KV cache"}
+    kv_mb = 2 * x["k_cache"].numel() * 2 / 1e6
+    qr_mb = 2 * x["q"].numel() * 2 / 1e6
+    res = {
+        "metric": METRIC, "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "num_heads": w.num_heads,
+                   "num_kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "causal": w.causal,
+                   "q_lens": [int(v) for v in x["q_lens"]], "seq_lens": [int(v) for v in x["seq_lens_host"]],
+                   "page_size": W.PAGE_SIZE, "rho_scale": w.rho_scale,
+                   "l2": f"q+rho {qr_mb:.0f} MB + KV pages {kv_mb:.0f} MB > 126 MB L2"},
+        "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic("prefill", w.name),
+                     "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_kernel (paged)",
+                     "algorithmic_flops_per_launch": flops},
+        "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
+    }
+    return res, x
+
+
 # ------------------------------------------------------------- CPU oracle
 
 def oracle_decode_sample(w, inp, budget_s, max_steps=None):
@@ -494,6 +574,8 @@ def oracle_decode_sample(w, inp, budget_s, max_steps=None):
 def cpu_baseline(w, inp, budget_s):
     if w.name == "prefill":
         return cpu_baseline_prefill(w, inp, budget_s)
+    if w.name == "prefill_paged":
+        return cpu_baseline_prefill_paged(w, inp, budget_s)
     gbs, secs, done, desc = oracle_decode_sample(w, inp, budget_s)
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
             "sample": desc, "seconds": round(secs, 2)}
@@ -519,6 +601,36 @@ def cpu_baseline_prefill(w, inp, budget_s):
             "seconds": round(secs, 2)}
 
 
+def cpu_baseline_prefill_paged(w, inp, budget_s):
+    """The oracle on groups of 16 random rows of one (sequence, head); FLOP
+    counted for those rows.  Inputs are read from host copies."""
+    import oracle
+    host = {k: (inp[k].cpu() if inp[k].is_cuda else inp[k]) for k in ("q", "rho", "k_cache", "v_cache")}
+    views = {k: _F64View(v) for k, v in host.items()}
+    table = inp["page_table"].cpu().numpy()
+    cu = inp["cu_seqlens_q"].cpu().numpy()
+    lens, q_lens = inp["seq_lens_host"], inp["q_lens"]
+    rng = np.random.default_rng(1)
+    secs, flops, n = 0.0, 0, 0
+    while secs < budget_s:
+        b = int(rng.integers(w.batch))
+        if q_lens[b] == 0:
+            continue
+        h = int(rng.integers(w.num_heads))
+        rows = [(b, int(i), h) for i in rng.integers(0, q_lens[b], size=16)]
+        t0 = time.perf_counter()
+        oracle.prefill_paged_rows(views["q"], views["rho"], views["k_cache"], views["v_cache"], table, cu, lens,
+                                  rows, w.scale, causal=w.causal)
+        secs += time.perf_counter() - t0
+        flops += sum(8 * w.head_dim * (int(lens[b]) - int(q_lens[b]) + i + 1 if w.causal else int(lens[b]))
+                     for _, i, _ in rows)
+        n += len(rows)
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": f"{n} random rows of {w.name}, in groups of 16 per (sequence, head) "
+                                        "(algorithmic FLOP of those rows)",
+            "seconds": round(secs, 2)}
+
+
 def reference_arm(args, w, rank, world):
     """The float64 oracle on the host cores, on this workload's metric.
 
@@ -531,14 +643,16 @@ def reference_arm(args, w, rank, world):
     if w.name == "prefill":
         sub = W.PrefillWorkload("prefill", 1, 1, w.seq_len, w.head_dim, rho_scale=w.rho_scale, seed=w.seed)
         inp = W.prefill_inputs(sub, device="cpu")
+    elif w.name == "prefill_paged":
+        inp = W.chunked_prefill_inputs(w, device="cpu")
     elif w.batch * w.kv_len <= 2**20:
         inp = W.decode_inputs(w, device="cpu")
     else:
         inp = _host_decode_sample(w)
     vals, secs_all, desc = [], 0.0, ""
     for i in range(args.warmup + args.steps):
-        if w.name == "prefill":
-            cb = cpu_baseline_prefill(w, inp, budget)
+        if w.name in ("prefill", "prefill_paged"):
+            cb = cpu_baseline(w, inp, budget)
             v, secs, desc = cb["value"], cb["seconds"], cb["sample"]
         else:
             sub_w = w if inp["q"].shape[0] == w.batch else W.DecodeWorkload(
@@ -549,7 +663,7 @@ def reference_arm(args, w, rank, world):
             vals.append(v)
             secs_all += secs
     value = statistics.median(vals)
-    unit = "TFLOP/s" if w.name == "prefill" else "GB/s"
+    unit = "TFLOP/s" if w.name.startswith("prefill") else "GB/s"
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs_all / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -601,6 +715,8 @@ def main(argv=None):
     try:
         if w.name == "prefill":
             res, inp = bench_prefill(args, w, rank, world, dev, peaks, kind)
+        elif w.name == "prefill_paged":
+            res, inp = bench_prefill_paged(args, w, rank, world, dev, peaks, kind)
         else:
             res, inp = bench_decode(args, w, rank, world, dev, peaks, kind)
             inp = inp[0]

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define PARALLAX_ABI_VERSION 1
+#define PARALLAX_ABI_VERSION 2
 
 typedef enum plx_status {
   PLX_OK = 0,
@@ -59,7 +59,7 @@ typedef enum plx_dtype { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
 /* Device error word codes (bit flags; several may be set). */
 #define PLX_DEVERR_BAD_PAGE   1   /* page_table entry outside [0, num_pages)     */
 #define PLX_DEVERR_TIMEOUT    2   /* an mbarrier / pipeline wait gave up         */
-#define PLX_DEVERR_BAD_LENGTH 4   /* seq_lens[b] < 0 or > kv_len                 */
+#define PLX_DEVERR_BAD_LENGTH 4   /* a sequence length outside its allowed range */
 
 /* ------------------------------------------------------------------------
  * Decode: one new query per (sequence, query head) over its KV cache.
@@ -177,6 +177,60 @@ typedef struct plx_prefill_params {
  *   out      device, [B, H, T, d] of out_dtype. */
 plx_status parallax_prefill(const void* q, const void* rho, const void* k, const void* v,
                             void* out, const plx_prefill_params* p, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Chunked (append) prefill over the paged cache: the step between a prompt
+ * chunk and decode in a serving loop.  The same per-query definition as
+ * decode and prefill (out = vbar - S_KV^T rho over the query's visible keys;
+ * wispaper.ai blog "Parallax: Breaking the Boundary Bias with Parameterized
+ * Local Linear Attention", section "The Core Insight: Covariance Correction").
+ *
+ * Sequence b holds L_b = seq_lens[b] keys in 64-token pages, laid out as in
+ * paged decode.  Its q_len_b = cu_seqlens_q[b+1] - cu_seqlens_q[b] queries
+ * are the sequence's LAST q_len_b positions, L_b - q_len_b .. L_b - 1, so
+ * their own keys and values must already be in the cache.  Query i of
+ * sequence b sees keys 0 .. L_b - q_len_b + i (causal) or all L_b keys.
+ * A one-token chunk is a decode step; parallax_decode is the faster kernel
+ * for it.
+ * ---------------------------------------------------------------------- */
+typedef struct plx_prefill_paged_params {
+  int32_t batch;              /* B sequences                                  */
+  int32_t num_heads;          /* H query heads                                */
+  int32_t num_kv_heads;       /* Hkv, divides H                               */
+  int32_t head_dim;           /* d: 128                                       */
+  int32_t total_q;            /* rows of q, rho and out (= cu_seqlens_q[B])   */
+  int32_t max_q_len;          /* >= every q_len_b; sets the grid             */
+  int32_t page_size;          /* 64                                           */
+  int32_t num_pages;          /* P, pages in each pool                        */
+  int32_t max_pages_per_seq;  /* page_table row stride                        */
+  int32_t in_dtype;           /* PLX_BF16                                     */
+  int32_t out_dtype;          /* PLX_BF16 or PLX_F32                          */
+  float scale;                /* softmax scale on q.k, > 0                    */
+  int32_t causal;             /* 1: causal (diagonal included); 0: none       */
+} plx_prefill_paged_params;
+
+/* Paged chunked prefill.
+ *   q, rho        device, [total_q, H, d] bf16; sequence b's rows start at
+ *                 cu_seqlens_q[b].
+ *   k_cache,      device, pools [P, Hkv, 64, d] bf16.  Slots past L_b in a
+ *   v_cache       sequence's last page may hold anything, NaN included.
+ *   page_table    device int32 [B, max_pages_per_seq]; entries 0 ..
+ *                 ceil(L_b/64)-1 of row b are read.
+ *   cu_seqlens_q  device int32 [B + 1], non-decreasing, cu_seqlens_q[B] <= total_q.
+ *   seq_lens      device int32 [B], q_len_b <= L_b <= 64 * max_pages_per_seq.
+ *   out           device, [total_q, H, d] of out_dtype; rows that belong to
+ *                 no sequence are left untouched.
+ * All buffers are caller-owned; nothing is allocated.  Asynchronous on
+ * `stream`.  total_q == 0 or max_q_len == 0 returns PLX_OK without a launch.
+ * Errors: host checks give PLX_ERR_INVALID_ARG / PLX_ERR_UNSUPPORTED before
+ * any launch.  On the device, a sequence whose lengths break the rules
+ * above (or exceed max_q_len) sets PLX_DEVERR_BAD_LENGTH, one whose pages
+ * fall outside [0, P) sets PLX_DEVERR_BAD_PAGE; its rows are not written. */
+plx_status parallax_prefill_paged(const void* q, const void* rho,
+                                  const void* k_cache, const void* v_cache,
+                                  const int32_t* page_table, const int32_t* cu_seqlens_q,
+                                  const int32_t* seq_lens, void* out,
+                                  const plx_prefill_paged_params* p, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Errors and introspection.

@@ -48,6 +48,16 @@ class PrefillParams(ctypes.Structure):
                 ("causal", ctypes.c_int32)]
 
 
+class PrefillPagedParams(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("total_q", ctypes.c_int32), ("max_q_len", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
+                ("max_pages_per_seq", ctypes.c_int32), ("in_dtype", ctypes.c_int32),
+                ("out_dtype", ctypes.c_int32), ("scale", ctypes.c_float),
+                ("causal", ctypes.c_int32)]
+
+
 _vp, _i32p = ctypes.c_void_p, ctypes.c_void_p
 lib.parallax_abi_version.restype = ctypes.c_int32
 lib.parallax_status_string.restype = ctypes.c_char_p
@@ -61,6 +71,9 @@ lib.parallax_decode.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, _vp, ctyp
                                 ctypes.POINTER(DecodeParams), _vp]
 lib.parallax_prefill.restype = ctypes.c_int
 lib.parallax_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(PrefillParams), _vp]
+lib.parallax_prefill_paged.restype = ctypes.c_int
+lib.parallax_prefill_paged.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _i32p, _vp,
+                                       ctypes.POINTER(PrefillPagedParams), _vp]
 lib.parallax_decode_noalloc.restype = ctypes.c_int
 lib.parallax_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, ctypes.POINTER(DecodeParams), _vp]
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -220,7 +233,7 @@ def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):
     B, H, T, d = q.shape
     if rho.shape != q.shape or k.shape != v.shape or k.shape[0] != B or k.shape[2] != T or k.shape[3] != d:
         raise ValueError("shape mismatch")
-    out_dtype = out_dtype or q.dtype
+    out_dtype = out_dtype or (out.dtype if out is not None else q.dtype)
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
     else:
@@ -231,6 +244,46 @@ def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):
                               _stream_ptr(q.device))
     if st != 0:
         raise ParallaxError(st, "parallax_prefill")
+    return out
+
+
+def prefill_paged(q, rho, k_cache, v_cache, page_table, cu_seqlens_q, seq_lens, *, max_q_len, scale=None,
+                  causal=True, out=None, out_dtype=None):
+    """Chunked (append) prefill over the paged cache.
+
+    q, rho: [total_q, H, d] bf16, sequence b's queries at rows
+    cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1, which are the LAST positions of
+    its seq_lens[b] keys.  k_cache, v_cache: pools [P, Hkv, 64, d] bf16;
+    page_table: int32 [B, max_pages]; cu_seqlens_q: int32 [B+1]; seq_lens:
+    int32 [B] (all on the device).  ``max_q_len`` bounds every chunk length
+    (a host int, so the call needs no device read-back).  Returns out
+    [total_q, H, d]; rows outside every sequence are left as allocated.
+    """
+    for name, t in (("q", q), ("rho", rho), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_cuda(name, t, torch.bfloat16)
+    for name, t in (("page_table", page_table), ("cu_seqlens_q", cu_seqlens_q), ("seq_lens", seq_lens)):
+        _check_cuda(name, t, torch.int32)
+    total_q, H, d = q.shape
+    P, Hkv, ps, dk = k_cache.shape
+    B = seq_lens.shape[0]
+    if (rho.shape != q.shape or v_cache.shape != k_cache.shape or dk != d or page_table.dim() != 2
+            or page_table.shape[0] != B or cu_seqlens_q.shape != (B + 1,)):
+        raise ValueError("shape mismatch")
+    out_dtype = out_dtype or (out.dtype if out is not None else q.dtype)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    else:
+        _check_cuda("out", out, out_dtype)
+        if out.shape != q.shape:
+            raise ValueError("out shape mismatch")
+    scale = (1.0 / d ** 0.5) if scale is None else float(scale)
+    p = PrefillPagedParams(B, H, Hkv, d, total_q, int(max_q_len), ps, P, page_table.shape[1], PLX_BF16,
+                           _dtype_code(out_dtype), scale, 1 if causal else 0)
+    st = lib.parallax_prefill_paged(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                                    _ptr(cu_seqlens_q), _ptr(seq_lens), _ptr(out), ctypes.byref(p),
+                                    _stream_ptr(q.device))
+    if st != 0:
+        raise ParallaxError(st, "parallax_prefill_paged")
     return out
 
 

@@ -80,6 +80,21 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t ro
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, heads, cols] bf16 tensor (rows of `heads` head vectors), box
+// [box_rows, 1, box_cols]: box_rows rows of one head, 128-byte swizzle.
+bool make_tmap_bf16_heads(CUtensorMap* m, const void* base, uint64_t cols, uint64_t heads, uint64_t rows,
+                          uint32_t box_cols, uint32_t box_rows) {
+  auto enc = tensor_map_encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {cols, heads, rows};
+  cuuint64_t strides[2] = {cols * 2, heads * cols * 2};
+  cuuint32_t box[3] = {box_cols, 1, box_rows};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ------------------------------------------------------------------ decode
 struct DecodePlan {
   int ctas;                  // persistent grid size
@@ -188,6 +203,18 @@ plx_status launch_decode_f32(const DecodeArgs& a, int ctas, size_t smem, cudaStr
 }
 
 // ----------------------------------------------------------------- prefill
+template <bool kPaged>
+plx_status launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tr, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const PrefillArgs& a, cudaStream_t stream) {
+  constexpr int smem = PfLayout::kBytes;
+  if (cudaFuncSetAttribute(prefill_tc_kernel<kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess)
+    return PLX_ERR_CUDA;
+  const long long grid = (long long)a.n_mblk * a.B * a.H;
+  prefill_tc_kernel<kPaged><<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
 plx_status launch_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,
                           const plx_prefill_params* p, cudaStream_t stream) {
   const int hkv = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
@@ -208,12 +235,7 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.out = out;
-  constexpr int smem = PfLayout::kBytes;
-  if (cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return PLX_ERR_CUDA;
-  const long long grid = (long long)a.n_mblk * a.B * a.H;
-  prefill_tc_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return launch_prefill_kernel<false>(tq, tr, tk, tv, a, stream);
 }
 
 plx_status validate_prefill(const plx_prefill_params* p) {
@@ -228,6 +250,27 @@ plx_status validate_prefill(const plx_prefill_params* p) {
   if (p->head_dim != 128) return PLX_ERR_UNSUPPORTED;
   if (p->causal != 0 && p->causal != 1) return PLX_ERR_INVALID_ARG;
   if ((int64_t)p->batch * p->num_heads * ((int64_t)p->seq_len + 128) >= (int64_t)INT32_MAX)
+    return PLX_ERR_UNSUPPORTED;
+  return PLX_OK;
+}
+
+plx_status validate_prefill_paged(const plx_prefill_paged_params* p) {
+  if (p == nullptr) return PLX_ERR_INVALID_ARG;
+  if (p->batch < 1 || p->num_heads < 1 || p->num_kv_heads < 1) return PLX_ERR_INVALID_ARG;
+  if (p->num_heads % p->num_kv_heads != 0) return PLX_ERR_INVALID_ARG;
+  if (p->total_q < 0 || p->max_q_len < 0 || p->num_pages < 1 || p->max_pages_per_seq < 1)
+    return PLX_ERR_INVALID_ARG;
+  if (!std::isfinite(p->scale) || !(p->scale > 0.f)) return PLX_ERR_INVALID_ARG;
+  if (p->in_dtype != PLX_BF16) return p->in_dtype == PLX_F32 ? PLX_ERR_UNSUPPORTED : PLX_ERR_INVALID_ARG;
+  if (p->out_dtype != PLX_F32 && p->out_dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
+  if (p->head_dim != 128) return PLX_ERR_UNSUPPORTED;
+  if (p->page_size != kPfBN) return PLX_ERR_UNSUPPORTED;
+  if (p->causal != 0 && p->causal != 1) return PLX_ERR_INVALID_ARG;
+  // int32 TMA coordinates: pool rows and packed query rows; int32 key counts.
+  if ((int64_t)p->num_pages * p->num_kv_heads * kPfBN >= (int64_t)INT32_MAX) return PLX_ERR_UNSUPPORTED;
+  if ((int64_t)p->max_pages_per_seq * kPfBN >= (int64_t)INT32_MAX) return PLX_ERR_UNSUPPORTED;
+  if ((int64_t)p->total_q + kPfBM >= (int64_t)INT32_MAX) return PLX_ERR_UNSUPPORTED;
+  if (((int64_t)p->max_q_len + kPfBM - 1) / kPfBM * p->batch * p->num_heads >= (int64_t)INT32_MAX)
     return PLX_ERR_UNSUPPORTED;
   return PLX_OK;
 }
@@ -375,6 +418,45 @@ plx_status parallax_prefill(const void* q, const void* rho, const void* k, const
   if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return PLX_ERR_INVALID_ARG;
   return launch_prefill(q, rho, k, v, out, p, stream);
+}
+
+plx_status parallax_prefill_paged(const void* q, const void* rho, const void* k_cache, const void* v_cache,
+                                  const int32_t* page_table, const int32_t* cu_seqlens_q, const int32_t* seq_lens,
+                                  void* out, const plx_prefill_paged_params* p, cudaStream_t stream) {
+  plx_status st = validate_prefill_paged(p);
+  if (st != PLX_OK) return st;
+  if (p->total_q == 0 || p->max_q_len == 0) return PLX_OK;   // no query rows: nothing to do
+  if (!q || !rho || !k_cache || !v_cache || !page_table || !cu_seqlens_q || !seq_lens || !out)
+    return PLX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+      !aligned(out, 16) || !aligned(page_table, 4) || !aligned(cu_seqlens_q, 4) || !aligned(seq_lens, 4))
+    return PLX_ERR_INVALID_ARG;
+  const uint64_t pool_rows = (uint64_t)p->num_pages * p->num_kv_heads * kPfBN;
+  CUtensorMap tq, tr, tk, tv;
+  if (!make_tmap_bf16_heads(&tq, q, kPfD, p->num_heads, p->total_q, 64, kPfBM) ||
+      !make_tmap_bf16_heads(&tr, rho, kPfD, p->num_heads, p->total_q, 64, kPfBM) ||
+      !make_tmap_bf16(&tk, k_cache, kPfD, pool_rows, 64, kPfBN) ||
+      !make_tmap_bf16(&tv, v_cache, kPfD, pool_rows, 64, kPfBN))
+    return PLX_ERR_CUDA;
+  PrefillArgs a{};
+  a.B = p->batch;
+  a.H = p->num_heads;
+  a.Hkv = p->num_kv_heads;
+  a.T = 0;
+  a.group = p->num_heads / p->num_kv_heads;
+  a.n_mblk = (p->max_q_len + kPfBM - 1) / kPfBM;
+  a.causal = p->causal;
+  a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.out = out;
+  a.cu_q = cu_seqlens_q;
+  a.seq_lens = seq_lens;
+  a.page_table = page_table;
+  a.max_pages = p->max_pages_per_seq;
+  a.num_pages = p->num_pages;
+  a.total_q = p->total_q;
+  a.max_q = p->max_q_len;
+  return launch_prefill_kernel<true>(tq, tr, tk, tv, a, stream);
 }
 
 plx_status parallax_decode_noalloc(const void* q, const void* rho, const void* k_cache, const void* v_cache,

@@ -33,6 +33,18 @@
 // buffers of S / A: S_b at 256 + 128 b, A_b at 320 + 128 b.  While the
 // softmax warps work on tile j, the tensor cores run the value products of
 // tile j-1 and the score products of tile j+1.
+//
+// Two forms of the same kernel:
+//   dense   q, rho [B, H, T, d]; k, v [B, Hkv, T, d]; every position a query.
+//   paged   chunked (append) prefill: sequence b holds L_b = seq_lens[b] keys
+//           in 64-token pages of a pool [P, Hkv, 64, d]; its q_len_b queries
+//           are packed at rows cu_q[b] .. cu_q[b+1]-1 of q, rho, out
+//           [total_q, H, d] and sit at the LAST positions L_b - q_len_b ..
+//           L_b - 1 of the sequence (their keys are already in the cache).
+//           A key tile is one page.  The unused tail of a sequence's last
+//           page may hold anything, NaN included: masked columns get s = -inf
+//           and a = 0 (a select, since 0 * NaN is NaN), and the softmax warps
+//           zero those V rows in shared memory before the value products.
 #pragma once
 
 #include "ptx.cuh"
@@ -65,10 +77,15 @@ constexpr int kPfSplitTiles = PLX_PREFILL_SPLIT_TILES;
 
 struct PrefillArgs {
   int B, H, Hkv, T, group;
-  int n_mblk;                     // ceil(T / 128)
+  int n_mblk;                     // ceil(T / 128) (dense), ceil(max q_len / 128) (paged)
   int causal, out_bf16;
   float scale_log2;               // scale * log2(e), > 0
-  void* out;                      // [B, H, T, D]
+  void* out;                      // [B, H, T, D] (dense), [total_q, H, D] (paged)
+  // paged form only
+  const int32_t* cu_q;            // [B + 1] first packed query row of each sequence
+  const int32_t* seq_lens;        // [B] keys of each sequence, its queries included
+  const int32_t* page_table;      // [B, max_pages] physical page of each 64-key tile
+  int max_pages, num_pages, total_q, max_q;
 };
 
 struct PfLayout {
@@ -92,14 +109,15 @@ constexpr uint32_t kColO1 = 0, kColO2 = 128;
 __device__ __forceinline__ uint32_t col_s(int b) { return 256u + 128u * b; }
 __device__ __forceinline__ uint32_t col_a(int b) { return 320u + 128u * b; }
 
+template <bool kPaged>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_r,
                       const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                       const PrefillArgs a) {
-  using L = PfLayout;
+  using Ly = PfLayout;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::kBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + kPfStages;
@@ -109,11 +127,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* drain = o_done + 1;
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + L::kMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::kMisc + 4);
-  float* red_max = reinterpret_cast<float*>(sm + L::kRedMax);
-  float* aref_s = reinterpret_cast<float*>(sm + L::kAref);
-  float* lc_s = reinterpret_cast<float*>(sm + L::kLC);
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::kMisc + 4);
+  float* red_max = reinterpret_cast<float*>(sm + Ly::kRedMax);
+  float* aref_s = reinterpret_cast<float*>(sm + Ly::kAref);
+  float* lc_s = reinterpret_cast<float*>(sm + Ly::kLC);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Longest query tiles first: the last tile of every head, then the one before...
@@ -122,14 +140,45 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   const int bh = blockIdx.x % BH;
   const int b = bh / a.H, h = bh % a.H, kvh = h / a.group;
   const int m0 = mblk * kPfBM;
-  const int kv_end = a.causal ? min(a.T, m0 + kPfBM) : a.T;
+  // The sequence: q_len queries (first packed row q_first) at the last
+  // positions pos0 .. pos0 + q_len - 1 of its L keys.  Dense: q_len = L = T.
+  int q_len = a.T, L = a.T, q_first = 0;
+  const int32_t* pt = nullptr;
+  if constexpr (kPaged) {
+    q_first = a.cu_q[b];
+    q_len = a.cu_q[b + 1] - q_first;
+    L = a.seq_lens[b];
+    const bool bad = q_first < 0 || q_len < 0 || q_len > a.max_q ||
+                     (long long)q_first + q_len > (long long)a.total_q || L < q_len ||
+                     (long long)L > (long long)a.max_pages * kPfBN;
+    if (bad) {   // uniform over the CTA: nothing below has run yet
+      if (threadIdx.x == 0) report_error(4 /* PLX_DEVERR_BAD_LENGTH */);
+      return;
+    }
+    if (m0 >= q_len) return;
+    pt = a.page_table + (size_t)b * a.max_pages;
+  }
+  const int pos0 = L - q_len;
+  const int kv_end = a.causal ? min(L, pos0 + m0 + kPfBM) : L;
   const int n = (kv_end + kPfBN - 1) / kPfBN;
   // Rows of this tile see at least min_keys keys; below 128 the bf16
   // rounding of P o A' is not averaged away, so the first tiles are split.
-  const int min_keys = a.causal ? min(m0 + 1, a.T) : a.T;
+  const int min_keys = a.causal ? min(pos0 + m0 + 1, L) : L;
   const bool few_keys = min_keys < 2 * kPfBN;
-  const int q_row = (b * a.H + h) * a.T + m0;
-  const int kv_row = (b * a.Hkv + kvh) * a.T;
+  const int q_row = kPaged ? q_first + m0 : (b * a.H + h) * a.T + m0;
+  const int kv_row = (b * a.Hkv + kvh) * a.T;   // dense form only
+  if constexpr (kPaged) {
+    // Every page this tile reads must lie in the pool.
+    bool badp = false;
+    for (int i = threadIdx.x; i < n; i += kPfThreads) {
+      const int pg = pt[i];
+      badp |= pg < 0 || pg >= a.num_pages;
+    }
+    if (__syncthreads_or(badp)) {
+      if (threadIdx.x == 0) report_error(1 /* PLX_DEVERR_BAD_PAGE */);
+      return;
+    }
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -166,32 +215,38 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       prefetch_tmap(&tm_v);
       const uint64_t keep = l2_policy_evict_last();   // K/V tiles are re-read by other query tiles
       const uint64_t once = l2_policy_evict_first();
-      mbar_arrive_expect_tx(q_full, 2 * L::kQBytes);
+      mbar_arrive_expect_tx(q_full, 2 * Ly::kQBytes);
       for (int bx = 0; bx < 2; ++bx) {
-        tma_load_2d(sm + L::kQ + bx * (L::kQBytes / 2), &tm_q, bx * 64, q_row, q_full, once);
-        tma_load_2d(sm + L::kR + bx * (L::kQBytes / 2), &tm_r, bx * 64, q_row, q_full, once);
+        if constexpr (kPaged) {   // [total_q, H, D]: box of 128 rows of one head
+          tma_load_3d(sm + Ly::kQ + bx * (Ly::kQBytes / 2), &tm_q, bx * 64, h, q_row, q_full, once);
+          tma_load_3d(sm + Ly::kR + bx * (Ly::kQBytes / 2), &tm_r, bx * 64, h, q_row, q_full, once);
+        } else {
+          tma_load_2d(sm + Ly::kQ + bx * (Ly::kQBytes / 2), &tm_q, bx * 64, q_row, q_full, once);
+          tma_load_2d(sm + Ly::kR + bx * (Ly::kQBytes / 2), &tm_r, bx * 64, q_row, q_full, once);
+        }
       }
       int issued = 0, issued_k = 0;   // V and K tiles issued
       for (int j = 0; j < n; ++j) {
         const int s = j % kPfStages;
         const uint32_t par = ((j / kPfStages) - 1) & 1;
-        const int row = kv_row + j * kPfBN;
+        // pool rows [P * Hkv * 64] (paged; page ids checked above) or [B * Hkv * T]
+        const int row = kPaged ? (pt[j] * a.Hkv + kvh) * kPfBN : kv_row + j * kPfBN;
         if (j >= kPfStages && !mbar_wait_bounded(&k_empty[s], par)) {
           *abort_flag = 1;
           break;
         }
         if (*abort_flag) break;
-        mbar_arrive_expect_tx(&k_full[s], L::kKVBytes);
+        mbar_arrive_expect_tx(&k_full[s], Ly::kKVBytes);
         for (int bx = 0; bx < 2; ++bx)
-          tma_load_2d(sm + L::kK + s * L::kKVBytes + bx * (L::kKVBytes / 2), &tm_k, bx * 64, row, &k_full[s], keep);
+          tma_load_2d(sm + Ly::kK + s * Ly::kKVBytes + bx * (Ly::kKVBytes / 2), &tm_k, bx * 64, row, &k_full[s], keep);
         if (j >= kPfStages && !mbar_wait_bounded(&v_empty[s], par)) {
           *abort_flag = 1;
           ++issued_k;
           break;
         }
-        mbar_arrive_expect_tx(&v_full[s], L::kKVBytes);
+        mbar_arrive_expect_tx(&v_full[s], Ly::kKVBytes);
         for (int bx = 0; bx < 2; ++bx)
-          tma_load_2d(sm + L::kV + s * L::kKVBytes + bx * (L::kKVBytes / 2), &tm_v, bx * 64, row, &v_full[s], keep);
+          tma_load_2d(sm + Ly::kV + s * Ly::kKVBytes + bx * (Ly::kKVBytes / 2), &tm_v, bx * 64, row, &v_full[s], keep);
         ++issued;
         ++issued_k;
       }
@@ -213,10 +268,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     constexpr uint32_t kIdS = idesc_bf16(kPfBM, kPfBN, false);   // 128 x 64, K-major B
     constexpr uint32_t kIdPV = idesc_bf16(kPfBM, kPfD, true);    // 128 x 128, MN-major B (V)
     // Descriptors of every operand base; a k-step adds its byte offset / 16.
-    const uint64_t dq = smem_desc_sw128(smem_u32(sm + L::kQ), 16, 1024);
-    const uint64_t dr = smem_desc_sw128(smem_u32(sm + L::kR), 16, 1024);
-    const uint64_t dk = smem_desc_sw128(smem_u32(sm + L::kK), 16, 1024);
-    const uint64_t dv = smem_desc_sw128(smem_u32(sm + L::kV), L::kKVBytes / 2, 1024);
+    const uint64_t dq = smem_desc_sw128(smem_u32(sm + Ly::kQ), 16, 1024);
+    const uint64_t dr = smem_desc_sw128(smem_u32(sm + Ly::kR), 16, 1024);
+    const uint64_t dk = smem_desc_sw128(smem_u32(sm + Ly::kK), 16, 1024);
+    const uint64_t dv = smem_desc_sw128(smem_u32(sm + Ly::kV), Ly::kKVBytes / 2, 1024);
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
     };
@@ -231,12 +286,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int s = j % kPfStages, b2 = j & 1;
         if (!(ok = wait_warp(&k_full[s], (j / kPfStages) & 1))) break;
         tc_fence_after();
-        const uint64_t dks = dk + (uint64_t)((s * L::kKVBytes) >> 4);
+        const uint64_t dks = dk + (uint64_t)((s * Ly::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kPfD / 16; ++kk) {
           // 16 columns of d per step: box kk / 4, 32 bytes into the 128-byte row per step
-          const uint64_t oq = (uint64_t)((kk >> 2) * (L::kQBytes / 2 / 16) + (kk & 3) * 2);
-          const uint64_t okk = (uint64_t)((kk >> 2) * (L::kKVBytes / 2 / 16) + (kk & 3) * 2);
+          const uint64_t oq = (uint64_t)((kk >> 2) * (Ly::kQBytes / 2 / 16) + (kk & 3) * 2);
+          const uint64_t okk = (uint64_t)((kk >> 2) * (Ly::kKVBytes / 2 / 16) + (kk & 3) * 2);
           tc_mma_ss(tmem + col_s(b2), dq + oq, dks + okk, kIdS, kk > 0);
           tc_mma_ss(tmem + col_a(b2), dr + oq, dks + okk, kIdS, kk > 0);
         }
@@ -250,7 +305,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!(ok = wait_warp(&v_full[sp], (jp / kPfStages) & 1))) break;
         if (!(ok = wait_warp(&p_full[bp], (jp >> 1) & 1))) break;
         tc_fence_after();
-        const uint64_t dvs = dv + (uint64_t)((sp * L::kKVBytes) >> 4);
+        const uint64_t dvs = dv + (uint64_t)((sp * Ly::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kPfBN / 16; ++kk) {
           // 16 keys per step: 8 TMEM columns of packed bf16 pairs, 16 rows of V
@@ -279,9 +334,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int g = (warp - 2) >> 2;           // key-column half of every tile
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int r = wq * 32 + lane;            // query row within the tile
-    const int t = m0 + r;                    // query position
+    const int t = m0 + r;                    // query index within the sequence's queries
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const int key_lim = a.causal ? min(t + 1, a.T) : a.T;   // keys [0, key_lim) visible
+    const int key_lim = a.causal ? min(pos0 + t + 1, L) : L;   // keys [0, key_lim) visible
     const uint32_t cs = 32u * g;             // fp32 columns of this half in S / A
     const int split_tiles = few_keys ? kPfSplitTiles : 0;
     const uint32_t cp = 16u * g;             // packed bf16 columns of this half's P / P o A'
@@ -301,7 +356,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tmem_wait_ld();
       // Tiles that reach the diagonal or the sequence end need the mask.
       const int key0 = j * kPfBN + (int)cs;
-      const bool masked = (a.causal && j * kPfBN + kPfBN - 1 > m0) || (j * kPfBN + kPfBN > a.T);
+      const bool masked = (a.causal && j * kPfBN + kPfBN - 1 > pos0 + m0) || (j * kPfBN + kPfBN > L);
       float mx = -INFINITY;
       if (masked) {
 #pragma unroll
@@ -322,6 +377,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!go) {
         fine = false;
         break;
+      }
+      if constexpr (kPaged) {   // a page tail may hold NaN keys: select, do not multiply
+        if (masked) {
+#pragma unroll
+          for (int cc = 0; cc < 32; ++cc)
+            if (key0 + cc >= key_lim) ar[cc] = 0u;
+        }
       }
       if (j == 0) aref = aref_s[r];
       // scale > 0, so the max of the scaled scores is the scaled max
@@ -386,6 +448,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
+      if constexpr (kPaged) {
+        // The sequence ends inside this page: zero the V rows past its end
+        // (their weights are 0, but 0 * NaN is not) before the value
+        // products, which wait on this warpgroup's arrival below.
+        if (j * kPfBN + kPfBN > L) {
+          const int s = j % kPfStages, nv = L - j * kPfBN;
+          const bool wv = mbar_wait_bounded(&v_full[s], (j / kPfStages) & 1);
+          fine = fine && wv;
+          if (wv) {
+            uint8_t* vt = sm + Ly::kV + s * Ly::kKVBytes;
+            for (int i = (int)threadIdx.x - 64; i < (kPfBN - nv) * 16; i += kPfSoftmax) {
+              const int row = nv + (i >> 4), c = i & 15;   // c: box (c >> 3), 16-byte chunk (c & 7)
+              *reinterpret_cast<uint4*>(vt + (c >> 3) * (Ly::kKVBytes / 2) + row * 128 + (c & 7) * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+          }
+        }
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b2]);
@@ -400,14 +481,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const float ct = lc_s[r * 2 + 1] + lc_s[(128 + r) * 2 + 1];
       const float inv = 1.f / lt;
       const float corr = 1.f + ct * inv;
-      const size_t orow = ((size_t)(b * a.H + h) * a.T + t) * kPfD + 64 * g;
+      const size_t orow = (kPaged ? (size_t)(q_first + t) * a.H + h : (size_t)(b * a.H + h) * a.T + t) * kPfD + 64 * g;
 #pragma unroll 1
       for (int part = 0; part < 2; ++part) {
         uint32_t o1[32], o2[32];
         tmem_ld32(tmem + lane_off + kColO1 + 64 * g + part * 32, o1);
         tmem_ld32(tmem + lane_off + kColO2 + 64 * g + part * 32, o2);
         tmem_wait_ld();
-        if (t < a.T) {
+        if (t < q_len) {
           float v[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o1[i]) * inv * corr - __uint_as_float(o2[i]) * inv;

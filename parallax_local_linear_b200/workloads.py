@@ -14,6 +14,10 @@ Named workloads (head_dim d, Hq query heads, Hkv KV heads):
   decode_paged   128 sequences, L ~ U{512..65536}, Hq=16, Hkv=4, d=128,
                  64-token pages placed by a seeded permutation
   prefill        B=4, H=16, T=8192, d=128, causal, rho scaled by 0.1
+  prefill_paged  chunked (append) prefill over a paged cache: 8 sequences,
+                 H=16, Hkv=4, d=128; each appends a chunk of U{1024..4096}
+                 queries to a cached prefix of U{0..8192} tokens; 64-token
+                 pages placed by a seeded permutation; rho scaled by 0.1
 """
 
 from __future__ import annotations
@@ -67,6 +71,25 @@ class PrefillWorkload:
         return 1.0 / math.sqrt(self.head_dim)
 
 
+@dataclass(frozen=True)
+class ChunkedPrefillWorkload:
+    name: str
+    batch: int
+    num_heads: int
+    num_kv_heads: int
+    head_dim: int
+    q_min: int          # chunk lengths uniform in [q_min, q_max]
+    q_max: int
+    prefix_max: int     # cached prefix lengths uniform in [0, prefix_max]
+    rho_scale: float = 0.1
+    causal: bool = True
+    seed: int = 0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.head_dim)
+
+
 WORKLOADS = {
     "decode_f32": DecodeWorkload("decode_f32", 1, 1, 1, 64, 256, dtype="f32", seed=1),
     "decode_bf16": DecodeWorkload("decode_bf16", 8, 16, 8, 128, 4096, seed=2),
@@ -74,6 +97,7 @@ WORKLOADS = {
     "decode_paged": DecodeWorkload("decode_paged", 128, 16, 4, 128, 65536, paged=True,
                                    min_len=512, seed=4),
     "prefill": PrefillWorkload("prefill", 4, 16, 8192, 128, seed=5),
+    "prefill_paged": ChunkedPrefillWorkload("prefill_paged", 8, 16, 4, 128, 1024, 4096, 8192, seed=6),
 }
 
 
@@ -271,3 +295,92 @@ def prefill_flops(w: PrefillWorkload) -> int:
     pairs = T * (T + 1) // 2 if w.causal else T * T
     return 8 * w.head_dim * pairs * w.batch * w.num_heads
 
+
+
+def chunked_layout(q_lens, prefix_lens, seed, page_size=PAGE_SIZE):
+    """Offsets, lengths and page table of chunks appended to cached prefixes.
+
+    Sequence b holds prefix_lens[b] + q_lens[b] keys; its chunk is packed at
+    rows cu[b] .. cu[b+1]-1.  Pages come from a seeded permutation of a pool
+    of sum(ceil(L_b / page_size)) pages (at least one); unused slots are -1.
+    """
+    q_lens = np.asarray(q_lens, dtype=np.int64)
+    lens = q_lens + np.asarray(prefix_lens, dtype=np.int64)
+    cu = np.concatenate([[0], np.cumsum(q_lens)]).astype(np.int32)
+    n_pages = -(-lens // page_size)
+    total = max(1, int(n_pages.sum()))
+    perm = np.random.Generator(np.random.PCG64(seed)).permutation(total).astype(np.int32)
+    table = np.full((len(lens), max(1, int(n_pages.max(initial=0)))), -1, dtype=np.int32)
+    cur = 0
+    for b, n in enumerate(n_pages):
+        table[b, :n] = perm[cur: cur + n]
+        cur += int(n)
+    return cu, lens.astype(np.int32), table, total
+
+
+def chunked_prefill_inputs(w: ChunkedPrefillWorkload, device="cpu", seed=None, nan_poison=True):
+    """Inputs of one chunked prefill call.
+
+    Returns a dict: q, rho [total_q, H, d] bf16 (rho scaled by rho_scale);
+    pools k_cache, v_cache [P, Hkv, 64, d] bf16; page_table, cu_seqlens_q,
+    seq_lens (int32, on ``device``); their host copies q_lens, seq_lens_host;
+    max_q_len; scale; causal.  With ``nan_poison`` the unused tail of every
+    last page is NaN.
+    """
+    seed = w.seed if seed is None else seed
+    rng = np.random.Generator(np.random.PCG64(seed))
+    q_lens = rng.integers(w.q_min, w.q_max + 1, size=w.batch)
+    prefix = rng.integers(0, w.prefix_max + 1, size=w.batch)
+    cu, lens, table, total = chunked_layout(q_lens, prefix, seed + 1)
+    gen = _gen(device, seed)
+    H, Hkv, d = w.num_heads, w.num_kv_heads, w.head_dim
+    tq = int(cu[-1])
+    q = _normal((tq, H, d), gen, device, torch.bfloat16)
+    rho = _normal((tq, H, d), gen, device, torch.bfloat16, mul=w.rho_scale)
+    k = _normal((total, Hkv, PAGE_SIZE, d), gen, device, torch.bfloat16)
+    v = _normal((total, Hkv, PAGE_SIZE, d), gen, device, torch.bfloat16)
+    if nan_poison:
+        _poison_paged_tails(k, v, lens, table)
+    return dict(q=q, rho=rho, k_cache=k, v_cache=v,
+                page_table=torch.from_numpy(table).to(device),
+                cu_seqlens_q=torch.from_numpy(cu).to(device),
+                seq_lens=torch.from_numpy(lens).to(device),
+                q_lens=q_lens.astype(np.int64), seq_lens_host=lens.astype(np.int64),
+                max_q_len=int(q_lens.max(initial=0)), scale=w.scale, causal=w.causal)
+
+
+def small_chunked_prefill_inputs(q_lens, prefix_lens, num_heads, num_kv_heads, head_dim=128, *,
+                                 rho_scale=0.1, seed=0, device="cpu"):
+    """Chunked prefill inputs of arbitrary (small) shape; every pool slot
+    outside a sequence is NaN."""
+    cu, lens, table, total = chunked_layout(q_lens, prefix_lens, seed + 1)
+    gen = _gen("cpu", seed)
+    H, Hkv, d = num_heads, num_kv_heads, head_dim
+    tq = int(cu[-1])
+    q = torch.randn((tq, H, d), generator=gen).to(torch.bfloat16)
+    rho = (torch.randn((tq, H, d), generator=gen) * rho_scale).to(torch.bfloat16)
+    k = torch.full((total, Hkv, PAGE_SIZE, d), float("nan"), dtype=torch.bfloat16)
+    v = torch.full((total, Hkv, PAGE_SIZE, d), float("nan"), dtype=torch.bfloat16)
+    for b, n in enumerate(lens):
+        for j in range(-(-int(n) // PAGE_SIZE)):
+            take = min(PAGE_SIZE, int(n) - j * PAGE_SIZE)
+            k[table[b, j], :, :take] = torch.randn((Hkv, take, d), generator=gen).to(torch.bfloat16)
+            v[table[b, j], :, :take] = torch.randn((Hkv, take, d), generator=gen).to(torch.bfloat16)
+    res = dict(q=q, rho=rho, k_cache=k, v_cache=v, page_table=torch.from_numpy(table),
+               cu_seqlens_q=torch.from_numpy(cu), seq_lens=torch.from_numpy(lens),
+               q_lens=np.asarray(q_lens, dtype=np.int64), seq_lens_host=lens.astype(np.int64),
+               max_q_len=int(max(q_lens, default=0)), scale=1.0 / math.sqrt(d), causal=True)
+    if device != "cpu":
+        res = {kk: (vv.to(device) if torch.is_tensor(vv) else vv) for kk, vv in res.items()}
+    return res
+
+
+def chunked_prefill_flops(q_lens, seq_lens, num_heads, head_dim, causal=True) -> int:
+    """Algorithmic FLOP of one chunked prefill call: 8*d per visible
+    (query, key) pair.  Query i of a chunk of q rows over L keys sees
+    L - q + i + 1 keys (causal) or L."""
+    total = 0
+    for q, L in zip(q_lens, seq_lens):
+        q, L = int(q), int(L)
+        total += q * (L - q) + q * (q + 1) // 2 if causal else q * L
+    return 8 * head_dim * num_heads * total

@@ -31,7 +31,7 @@ def binding():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for must in ("parallax_decode", "parallax_prefill", "parallax_decode_workspace_size",
+    for must in ("parallax_decode", "parallax_prefill", "parallax_prefill_paged", "parallax_decode_workspace_size",
                  "parallax_last_device_error", "parallax_status_string"):
         assert must in names
 
@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(binding):
 
 
 def test_abi_version_and_status_strings(binding):
-    assert binding.lib.parallax_abi_version() == 1
+    assert binding.lib.parallax_abi_version() == 2
     for code, name in binding.STATUS.items():
         assert binding.lib.parallax_status_string(code).decode() == name
 
@@ -104,6 +104,42 @@ def test_invalid_prefill_params_are_rejected(binding, bad):
     p = binding.PrefillParams(**base)
     st = binding.lib.parallax_prefill(None, None, None, None, None, ctypes.byref(p), None)
     assert st in (1, 2)
+
+
+def _paged_prefill_params(binding, **kw):
+    base = dict(batch=2, num_heads=4, num_kv_heads=2, head_dim=128, total_q=300, max_q_len=200, page_size=64,
+                num_pages=20, max_pages_per_seq=10, in_dtype=1, out_dtype=0, scale=0.088, causal=1)
+    base.update(kw)
+    return binding.PrefillPagedParams(**base)
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(batch=0), 1), (dict(num_heads=6, num_kv_heads=4), 1), (dict(total_q=-1), 1),
+    (dict(max_q_len=-5), 1), (dict(num_pages=0), 1), (dict(max_pages_per_seq=0), 1),
+    (dict(scale=0.0), 1), (dict(scale=float("nan")), 1), (dict(in_dtype=3), 1), (dict(out_dtype=5), 1),
+    (dict(causal=-1), 1), (dict(head_dim=64), 2), (dict(page_size=16), 2), (dict(in_dtype=0), 2),
+    (dict(num_pages=1 << 24, num_kv_heads=4), 2), (dict(max_pages_per_seq=1 << 26), 2),
+])
+def test_invalid_paged_prefill_params_are_rejected(binding, bad, status):
+    p = _paged_prefill_params(binding, **bad)
+    st = binding.lib.parallax_prefill_paged(None, None, None, None, None, None, None, None, ctypes.byref(p), None)
+    assert st == status
+
+
+def test_paged_prefill_pointer_checks_and_empty_calls(binding):
+    p = _paged_prefill_params(binding)
+    nul = [None] * 8
+    assert binding.lib.parallax_prefill_paged(*nul, ctypes.byref(p), None) == 1
+    buf = ctypes.create_string_buffer(64)
+    addr = ctypes.addressof(buf)
+    al = ctypes.c_void_p((addr + 15) & ~15)
+    odd = ctypes.c_void_p(((addr + 15) & ~15) + 8)
+    args = [al, al, al, al, al, al, al, odd]          # out only 8-byte aligned
+    assert binding.lib.parallax_prefill_paged(*args, ctypes.byref(p), None) == 1
+    # no query rows: valid, and nothing is launched or dereferenced
+    for empty in (dict(total_q=0), dict(max_q_len=0)):
+        pe = _paged_prefill_params(binding, **empty)
+        assert binding.lib.parallax_prefill_paged(*nul, ctypes.byref(pe), None) == 0
 
 
 def _expected_plan(B, units, heads_per_unit, L, d=128, num_sms=148, forced=0, per_sm=1, paged=False):
