@@ -21,18 +21,22 @@
 //   warp 0       TMA producer: Q and R once, then separate K and V rings.
 //   warp 1       TMEM allocator; lane 0 issues every tcgen05.mma.
 //   warps 2..9   softmax, two warpgroups.  Thread = query row = TMEM lane;
-//                warpgroup g takes key columns 32g..32g+31 of every tile.
-//                The two halves of a row exchange their max through shared
-//                memory once per tile, form P and P o A' in bf16 and write
-//                them back over the S and A columns (the A operand of the
-//                value products comes straight from TMEM).  When the running
-//                max grows by more than 2^8, warpgroup g rescales O1 (g = 0)
-//                or O2 (g = 1); at the end it writes output columns 64g..64g+63.
+//                warpgroup g takes the key tiles j = g, g+2, ... (all 64
+//                columns), forms P and P o A' in bf16 and writes them back
+//                over its S and A buffer (the A operand of the value
+//                products comes straight from TMEM).  The two warpgroups
+//                work on consecutive tiles at once, so one's exponentials
+//                overlap the other's loads, reductions and waits.  The
+//                reference max of P passes from tile j-1's warpgroup to
+//                tile j's through shared memory and an mbarrier; when it
+//                grows by more than 2^8, that warpgroup rescales O1 and O2.
+//                At the end warpgroup g writes output columns 64g..64g+63.
 //
 // TMEM columns (512 x 128 lanes x 32 bit): O1 [0,128), O2 [128,256), and two
-// buffers of S / A: S_b at 256 + 128 b, A_b at 320 + 128 b.  While the
-// softmax warps work on tile j, the tensor cores run the value products of
-// tile j-1 and the score products of tile j+1.
+// buffers of S / A: S_b at 256 + 128 b, A_b at 320 + 128 b (buffer b holds
+// the tiles of warpgroup b).  While a warpgroup works on tile j, the tensor
+// cores run the value products of tile j-1 and the score products of tile
+// j+1, which the other warpgroup takes up as soon as they land.
 //
 // Two forms of the same kernel:
 //   dense   q, rho [B, H, T, d]; k, v [B, Hkv, T, d]; every position a query.
@@ -46,6 +50,8 @@
 //           and a = 0 (a select, since 0 * NaN is NaN), and the softmax warps
 //           zero those V rows in shared memory before the value products.
 #pragma once
+
+#include <type_traits>
 
 #include "ptx.cuh"
 
@@ -74,6 +80,12 @@ constexpr float kPfRescaleLog2 = 8.f;   // lazy rescale threshold (factor 256)
 #define PLX_PREFILL_SPLIT_TILES 2
 #endif
 constexpr int kPfSplitTiles = PLX_PREFILL_SPLIT_TILES;
+// Every kPfPolyEvery-th pair of exponentials is computed by ex2_poly2 on the
+// FMA pipe instead of the SFU (0: none), to balance the two pipes.
+#ifndef PLX_PREFILL_POLY_EVERY
+#define PLX_PREFILL_POLY_EVERY 0
+#endif
+constexpr int kPfPolyEvery = PLX_PREFILL_POLY_EVERY;
 
 struct PrefillArgs {
   int B, H, Hkv, T, group;
@@ -96,13 +108,14 @@ struct PfLayout {
   static constexpr int kK = kR + kQBytes;
   static constexpr int kV = kK + kPfStages * kKVBytes;
   static constexpr int kBar = kV + kPfStages * kKVBytes;
-  // barriers: q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2], o_done, drain
-  static constexpr int kNumBars = 1 + 4 * kPfStages + 2 + 2 + 1 + 1;
+  // barriers: q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_full[2], o_done,
+  // drain, hand[2] (hand[g]: the reference max for warpgroup g's next tile is in m_ref)
+  static constexpr int kNumBars = 1 + 4 * kPfStages + 2 + 2 + 1 + 1 + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;       // tmem base, abort flag
-  static constexpr int kRedMax = kMisc + 16;              // float [2 tile parities][2 halves][128 rows]
-  static constexpr int kAref = kRedMax + 2 * 2 * 128 * 4; // float [128]
-  static constexpr int kLC = kAref + 128 * 4;             // float [2 halves][128 rows][2]
-  static constexpr int kBytes = kLC + 2 * 128 * 2 * 4 + 1024;   // + alignment slack
+  static constexpr int kMref = kMisc + 16;                // float [128 rows]: reference max after the last tile
+  static constexpr int kAref = kMref + 128 * 4;           // float [128]
+  static constexpr int kLC = kAref + 128 * 4;             // float [2 warpgroups][128 rows][l, c, m]
+  static constexpr int kBytes = kLC + 2 * 128 * 3 * 4 + 1024;   // + alignment slack
 };
 
 constexpr uint32_t kColO1 = 0, kColO2 = 128;
@@ -127,9 +140,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;
   uint64_t* drain = o_done + 1;
+  uint64_t* hand = drain + 1;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::kMisc + 4);
-  float* red_max = reinterpret_cast<float*>(sm + Ly::kRedMax);
+  float* mref_s = reinterpret_cast<float*>(sm + Ly::kMref);
   float* aref_s = reinterpret_cast<float*>(sm + Ly::kAref);
   float* lc_s = reinterpret_cast<float*>(sm + Ly::kLC);
 
@@ -190,7 +204,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], kPfSoftmax);
+      mbar_init(&p_full[i], kPfSoftmax / 2);
+      mbar_init(&hand[i], kPfSoftmax / 2);
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
@@ -308,17 +323,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint64_t dvs = dv + (uint64_t)((sp * Ly::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kPfBN / 16; ++kk) {
-          // 16 keys per step: 8 TMEM columns of packed bf16 pairs, 16 rows of V
+          // 16 keys per step: 8 TMEM columns of packed bf16 pairs (keys 32q..32q+31
+          // sit in columns 32q..32q+15), 16 rows of V
           const uint64_t vd = dvs + (uint64_t)(kk * 16 * 128 / 16);
-          tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + kk * 8, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
-          tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + kk * 8, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t pc = 32u * (kk >> 1) + 8u * (kk & 1);
+          tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + pc, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + pc, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
         }
-        if (few_keys && jp < kPfSplitTiles) {   // lo parts sit in columns 32..63 of the S / A buffers
+        if (few_keys && jp < kPfSplitTiles) {   // lo parts: 16 columns after their hi parts
 #pragma unroll
           for (int kk = 0; kk < kPfBN / 16; ++kk) {
             const uint64_t vd = dvs + (uint64_t)(kk * 16 * 128 / 16);
-            tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + 32 + kk * 8, vd, kIdPV, 1u);
-            tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + 32 + kk * 8, vd, kIdPV, 1u);
+            const uint32_t pc = 32u * (kk >> 1) + 8u * (kk & 1) + 16u;
+            tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + pc, vd, kIdPV, 1u);
+            tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + pc, vd, kIdPV, 1u);
           }
         }
         tc_commit(&v_empty[sp]);
@@ -331,115 +349,148 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     wait_warp(drain, 0);
   } else {
     // ------------------------------------------------------------ softmax
-    const int g = (warp - 2) >> 2;           // key-column half of every tile
+    const int g = (warp - 2) >> 2;           // warpgroup: tiles j = g, g+2, ...; S / A buffer g
     const int wq = warp & 3;                 // TMEM lane quarter of this warp
     const int r = wq * 32 + lane;            // query row within the tile
     const int t = m0 + r;                    // query index within the sequence's queries
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int key_lim = a.causal ? min(pos0 + t + 1, L) : L;   // keys [0, key_lim) visible
-    const uint32_t cs = 32u * g;             // fp32 columns of this half in S / A
     const int split_tiles = few_keys ? kPfSplitTiles : 0;
-    const uint32_t cp = 16u * g;             // packed bf16 columns of this half's P / P o A'
-    float m_used = -INFINITY, aref = 0.f;
+    const uint32_t cS = tmem + lane_off + col_s(g), cA = tmem + lane_off + col_a(g);
+    // m_ref: reference max of P after the latest tile (both warpgroups' P
+    // enter the same O, so they share it).  m_mine: the reference this
+    // warpgroup's partial l and c are relative to.
+    float m_ref = -INFINITY, m_mine = -INFINITY, aref = 0.f;
     float2 l2 = make_float2(0.f, 0.f), c2 = make_float2(0.f, 0.f);
-    // Each decision that gates a warp-collective tcgen05 op, or the shared
-    // barrier of the two warpgroups, is reduced over all 256 softmax threads
-    // (bar_and), so both halves always leave the loop together.
+    // Each decision that gates a warp-collective tcgen05 op is reduced over
+    // the warpgroup (bar_and), so its four warps always run the same tiles.
     bool fine = true;
-    int j = 0;
-    for (; j < n; ++j) {
-      const int b2 = j & 1;
-      const bool w = !*abort_flag && mbar_wait_bounded(&s_full[b2], (j >> 1) & 1);
+    int j = g;
+    for (; j < n; j += 2) {
+      const bool w = !*abort_flag && mbar_wait_bounded(&s_full[g], (j >> 1) & 1);
       tc_fence_after();
-      uint32_t sr[32], ar[32];
-      tmem_ld32(tmem + lane_off + col_s(b2) + cs, sr);
+      uint32_t sr[64], ar[32];
+      tmem_ld32p(cS, sr);
+      tmem_ld32p(cS + 32, sr + 32);
       tmem_wait_ld();
       // Tiles that reach the diagonal or the sequence end need the mask.
-      const int key0 = j * kPfBN + (int)cs;
-      const bool masked = (a.causal && j * kPfBN + kPfBN - 1 > pos0 + m0) || (j * kPfBN + kPfBN > L);
-      float mx = -INFINITY;
+      const int key0 = j * kPfBN;
+      const bool masked = (a.causal && key0 + kPfBN - 1 > pos0 + m0) || (key0 + kPfBN > L);
       if (masked) {
 #pragma unroll
-        for (int cc = 0; cc < 32; ++cc)
+        for (int cc = 0; cc < 64; ++cc)
           if (key0 + cc >= key_lim) sr[cc] = __float_as_uint(-INFINITY);
       }
+      float mt[8];   // eight independent running maxima: a short dependency chain, few registers
 #pragma unroll
-      for (int cc = 0; cc < 32; ++cc) mx = fmaxf(mx, __uint_as_float(sr[cc]));
-      red_max[((j & 1) * 2 + g) * 128 + r] = mx;
-      // The probe values are loaded while the two halves exchange their max.
-      tmem_ld32(tmem + lane_off + col_a(b2) + cs, ar);
-      if (j == 0 && g == 0) {
-        tmem_wait_ld();
-        aref_s[r] = __uint_as_float(ar[0]);
-      }
-      const bool go = bar_and(1, kPfSoftmax, w && fine);
+      for (int i = 0; i < 8; ++i) mt[i] = fmaxf(__uint_as_float(sr[i]), __uint_as_float(sr[i + 8]));
+#pragma unroll
+      for (int i = 16; i < 64; ++i) mt[i & 7] = fmaxf(mt[i & 7], __uint_as_float(sr[i]));
+      mt[0] = fmaxf(fmaxf(fmaxf(mt[0], mt[4]), fmaxf(mt[1], mt[5])), fmaxf(fmaxf(mt[2], mt[6]), fmaxf(mt[3], mt[7])));
+      tmem_ld32(cA, ar);   // probe values of keys 0..31, loaded while the reference is handed over
+      // The reference after tile j-1 comes from the other warpgroup.
+      const bool wh = j == 0 || mbar_wait_bounded(&hand[g], ((j - 1) >> 1) & 1);
+      const bool go = bar_and(1 + g, kPfSoftmax / 2, w && wh && fine);
       tmem_wait_ld();
       if (!go) {
         fine = false;
         break;
       }
-      if constexpr (kPaged) {   // a page tail may hold NaN keys: select, do not multiply
-        if (masked) {
-#pragma unroll
-          for (int cc = 0; cc < 32; ++cc)
-            if (key0 + cc >= key_lim) ar[cc] = 0u;
-        }
+      if (j == 0) {
+        aref = __uint_as_float(ar[0]);   // a_ref = rho . k_0: key 0 is visible to every row
+      } else {
+        m_ref = mref_s[r];
+        if (j == 1) aref = aref_s[r];
       }
-      if (j == 0) aref = aref_s[r];
       // scale > 0, so the max of the scaled scores is the scaled max
-      const float m_tile = fmaxf(mx, red_max[((j & 1) * 2 + (1 - g)) * 128 + r]) * a.scale_log2;
-      const float m_new = fmaxf(m_used, m_tile);
-      const bool need = m_new > m_used + kPfRescaleLog2;
+      const float m_new = fmaxf(m_ref, mt[0] * a.scale_log2);
+      const bool need = m_new > m_ref + kPfRescaleLog2;
       float alpha = 1.f;
       if (need) {
-        alpha = ex2(m_used - m_new);
-        m_used = m_new;
+        alpha = ex2(m_ref - m_new);
+        m_ref = m_new;
       }
-      l2 = mul2(l2, make_float2(alpha, alpha));
-      c2 = mul2(c2, make_float2(alpha, alpha));
+      mref_s[r] = m_ref;
+      if (j == 0) aref_s[r] = aref;
+      mbar_arrive(&hand[1 - g]);
+      if (m_mine != m_ref) {   // bring this warpgroup's partial sums to the current reference
+        const float f = ex2(m_mine - m_ref);
+        l2 = mul2(l2, make_float2(f, f));
+        c2 = mul2(c2, make_float2(f, f));
+        m_mine = m_ref;
+      }
       const float2 sc2 = make_float2(a.scale_log2, a.scale_log2);
-      const float2 nm2 = make_float2(-m_used, -m_used);
+      const float2 nm2 = make_float2(-m_ref, -m_ref);
       const float2 na2 = make_float2(-aref, -aref);
-      const bool split = j < split_tiles;
-      uint32_t pp[16], pa[16];
+      // S of this tile is in registers and A is read half by half, so P and
+      // P o A' overwrite them in TMEM as they go: the bf16 pairs of keys
+      // 32q..32q+31 go to columns 32q..32q+15 of the S / A buffer, their lo
+      // parts (split tiles only) to 32q+16..32q+31 -- columns this half has
+      // already consumed.  The split is a separate instantiation so that
+      // ordinary tiles run a loop without it.
+      auto form_p = [&](auto split_tag) {
+        constexpr bool kSplit = decltype(split_tag)::value;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float2 x2 = fma2(make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])), sc2, nm2);
-        const float2 p2 = make_float2(ex2(x2.x), ex2(x2.y));
-        l2 = add2(l2, p2);
-        const float2 q2 =
-            mul2(p2, add2(make_float2(__uint_as_float(ar[2 * i]), __uint_as_float(ar[2 * i + 1])), na2));
-        c2 = add2(c2, q2);
-        pp[i] = pack_bf16(p2.x, p2.y);
-        pa[i] = pack_bf16(q2.x, q2.y);
-        if (split) {   // lo parts reuse sr / ar entries already consumed
-          sr[i] = pack_bf16(p2.x - bf16_lo_f(pp[i]), p2.y - bf16_hi_f(pp[i]));
-          ar[i] = pack_bf16(q2.x - bf16_lo_f(pa[i]), q2.y - bf16_hi_f(pa[i]));
+        for (int q = 0; q < 2; ++q) {
+          if (q == 1) {
+            tmem_ld32(cA + 32, ar);
+            tmem_wait_ld();
+          }
+          if constexpr (kPaged) {   // a page tail may hold NaN keys: select, not multiply
+            if (masked) {
+#pragma unroll
+              for (int cc = 0; cc < 32; ++cc)
+                if (key0 + 32 * q + cc >= key_lim) ar[cc] = 0u;
+            }
+          }
+          uint32_t pp[16], pa[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const int e = 32 * q + 2 * i;
+            const float2 x2 = fma2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sc2, nm2);
+            const float2 p2 = (kPfPolyEvery > 0 && i % (kPfPolyEvery > 0 ? kPfPolyEvery : 1) == kPfPolyEvery - 1)
+                                  ? ex2_poly2(x2)
+                                  : make_float2(ex2(x2.x), ex2(x2.y));
+            l2 = add2(l2, p2);
+            const float2 q2 =
+                mul2(p2, add2(make_float2(__uint_as_float(ar[2 * i]), __uint_as_float(ar[2 * i + 1])), na2));
+            c2 = add2(c2, q2);
+            pp[i] = pack_bf16(p2.x, p2.y);
+            pa[i] = pack_bf16(q2.x, q2.y);
+            if constexpr (kSplit) {   // lo parts reuse entries already consumed: sr[32q+i] (<= e), ar[i] (<= 2i)
+              sr[32 * q + i] = pack_bf16(p2.x - bf16_lo_f(pp[i]), p2.y - bf16_hi_f(pp[i]));
+              ar[i] = pack_bf16(q2.x - bf16_lo_f(pa[i]), q2.y - bf16_hi_f(pa[i]));
+            }
+          }
+          tmem_st16(cS + 32 * q, pp);
+          tmem_st16(cA + 32 * q, pa);
+          if constexpr (kSplit) {
+            tmem_st16(cS + 32 * q + 16, sr + 32 * q);
+            tmem_st16(cA + 32 * q + 16, ar);
+          }
         }
-      }
-      // Both halves have read S / A of this tile (the barrier above): overwrite.
-      tmem_st16(tmem + lane_off + col_s(b2) + cp, pp);
-      tmem_st16(tmem + lane_off + col_a(b2) + cp, pa);
-      if (split) {
-        tmem_st16(tmem + lane_off + col_s(b2) + 32 + cp, sr);
-        tmem_st16(tmem + lane_off + col_a(b2) + 32 + cp, ar);
-      }
+      };
+      if (j < split_tiles)
+        form_p(std::true_type{});
+      else
+        form_p(std::false_type{});
       // O may be touched only once the value products of tile j-1 are done.
       // Waiting on that one phase is exact without waiting on the earlier
-      // ones: s_full(j) was committed after the value products of tile j-2, so
-      // o_done has completed phase j-2, and tile j's value products cannot
-      // start before this warpgroup arrives on p_full(j); its phase is j-1 or
-      // j.  The wait is skipped unless O is rescaled, except at the last tile,
-      // which pins the phase for the epilogue's wait to n-1 or n.
-      if (j >= 1 && (j == n - 1 || __any_sync(0xffffffffu, need))) {
+      // ones: s_full(j) was committed after the value products of tile j-2,
+      // so o_done has completed phase j-2, and tile j's value products cannot
+      // start before this warpgroup arrives on p_full below; the phase is
+      // j-1 or j.  The wait is skipped unless O is rescaled, except at the
+      // last tile, which pins the phase for the epilogue's wait to n-1 or n.
+      const bool rescale = __any_sync(0xffffffffu, need) && j >= 1;
+      if (j >= 1 && (j == n - 1 || rescale)) {
         const bool wo = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (j - 1) & 1));
         fine = fine && wo;
-        if (wo && __any_sync(0xffffffffu, need)) {
+        if (wo && rescale) {
           tc_fence_after();
 #pragma unroll 1
-          for (int part = 0; part < 4; ++part) {
+          for (int part = 0; part < 8; ++part) {   // O1 then O2, 32 columns at a time
             uint32_t ov[32];
-            const uint32_t addr = tmem + lane_off + (g ? kColO2 : kColO1) + part * 32;
+            const uint32_t addr = tmem + lane_off + kColO1 + part * 32;
             tmem_ld32(addr, ov);
             tmem_wait_ld();
 #pragma unroll
@@ -452,13 +503,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // The sequence ends inside this page: zero the V rows past its end
         // (their weights are 0, but 0 * NaN is not) before the value
         // products, which wait on this warpgroup's arrival below.
-        if (j * kPfBN + kPfBN > L) {
-          const int s = j % kPfStages, nv = L - j * kPfBN;
+        if (key0 + kPfBN > L) {
+          const int s = j % kPfStages, nv = L - key0;
           const bool wv = mbar_wait_bounded(&v_full[s], (j / kPfStages) & 1);
           fine = fine && wv;
           if (wv) {
             uint8_t* vt = sm + Ly::kV + s * Ly::kKVBytes;
-            for (int i = (int)threadIdx.x - 64; i < (kPfBN - nv) * 16; i += kPfSoftmax) {
+            for (int i = (int)threadIdx.x - 64 - 128 * g; i < (kPfBN - nv) * 16; i += kPfSoftmax / 2) {
               const int row = nv + (i >> 4), c = i & 15;   // c: box (c >> 3), 16-byte chunk (c & 7)
               *reinterpret_cast<uint4*>(vt + (c >> 3) * (Ly::kKVBytes / 2) + row * 128 + (c & 7) * 16) =
                   make_uint4(0u, 0u, 0u, 0u);
@@ -469,16 +520,24 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full[b2]);
+      mbar_arrive(&p_full[g]);
     }
-    // ---- epilogue: wait for the last value products, then write the rows
-    const bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(o_done, (n - 1) & 1);
-    lc_s[(g * 128 + r) * 2 + 0] = l2.x + l2.y;
-    lc_s[(g * 128 + r) * 2 + 1] = c2.x + c2.y;
-    if (bar_and(1, kPfSoftmax, wl)) {
+    // ---- epilogue: the last tile's warpgroup waits for the last value
+    // products (its j == n-1 wait above made the phase exact), the barrier
+    // below releases the other; then the rows are written.
+    bool wl = fine && j >= n && !*abort_flag;
+    if (wl && ((n - 1) & 1) == g) wl = mbar_wait_bounded(o_done, (n - 1) & 1);
+    lc_s[(g * 128 + r) * 3 + 0] = l2.x + l2.y;
+    lc_s[(g * 128 + r) * 3 + 1] = c2.x + c2.y;
+    lc_s[(g * 128 + r) * 3 + 2] = m_mine;
+    if (bar_and(3, kPfSoftmax, wl)) {
       tc_fence_after();
-      const float lt = lc_s[r * 2] + lc_s[(128 + r) * 2];
-      const float ct = lc_s[r * 2 + 1] + lc_s[(128 + r) * 2 + 1];
+      // O is relative to the last reference, the larger of the two (references only grow).
+      const float ma = lc_s[r * 3 + 2], mb = lc_s[(128 + r) * 3 + 2];
+      const float mm = fmaxf(ma, mb);
+      const float fa = ex2(ma - mm), fb = ex2(mb - mm);   // a warpgroup with no tiles has l = c = 0
+      const float lt = lc_s[r * 3] * fa + lc_s[(128 + r) * 3] * fb;
+      const float ct = lc_s[r * 3 + 1] * fa + lc_s[(128 + r) * 3 + 1] * fb;
       const float inv = 1.f / lt;
       const float corr = 1.f + ct * inv;
       const size_t orow = (kPaged ? (size_t)(q_first + t) * a.H + h : (size_t)(b * a.H + h) * a.T + t) * kPfD + 64 * g;

@@ -263,6 +263,19 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
                : "memory");
 }
 
+// The same 32-column load / store on r[0..31] of a larger register array
+// (indices must be compile-time constants after unrolling).
+__device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32p(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
@@ -315,6 +328,32 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
       : "=f"(d.x), "=f"(d.y)
       : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
   return d;
+}
+
+// 2^x for a pair, on the FMA and integer pipes instead of the SFU, for
+// x <= 2^22 (-inf included).  Cody-Waite range reduction: x = n + f with
+// n = floor(x) (taken from the low mantissa bits of x + 1.5*2^23 rounded
+// toward -inf) and f in [0, 1); 2^f from a cubic fitted for least maximum
+// relative error on [0, 1] (Lawson's iteratively reweighted least squares;
+// error <= 7.5e-5); 2^n added into the exponent field.  x is clamped to
+// -125 first (so the exponent field stays >= 1), and very small results
+// come out as ~2^-125 rather than 0.
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.f;   // 1.5 * 2^23
+  x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
+  float2 y;
+  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rm.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(y.x), "=f"(y.y)
+      : "f"(x.x), "f"(x.y), "f"(kMagic), "f"(kMagic));
+  const float2 n = add2(y, make_float2(-kMagic, -kMagic));
+  const float2 f = add2(x, make_float2(-n.x, -n.y));
+  float2 p = fma2(make_float2(0.07802419364452362f, 0.07802419364452362f), f,
+                  make_float2(0.2260672152042389f, 0.2260672152042389f));
+  p = fma2(p, f, make_float2(0.6958337426185608f, 0.6958337426185608f));
+  p = fma2(p, f, make_float2(0.9999251961708069f, 0.9999251961708069f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23)));
 }
 
 // Named barrier over `nthreads` threads that also ANDs a predicate across them.
