@@ -80,12 +80,6 @@ constexpr float kPfRescaleLog2 = 8.f;   // lazy rescale threshold (factor 256)
 #define PLX_PREFILL_SPLIT_TILES 2
 #endif
 constexpr int kPfSplitTiles = PLX_PREFILL_SPLIT_TILES;
-// Every kPfPolyEvery-th pair of exponentials is computed by ex2_poly2 on the
-// FMA pipe instead of the SFU (0: none), to balance the two pipes.
-#ifndef PLX_PREFILL_POLY_EVERY
-#define PLX_PREFILL_POLY_EVERY 0
-#endif
-constexpr int kPfPolyEvery = PLX_PREFILL_POLY_EVERY;
 
 struct PrefillArgs {
   int B, H, Hkv, T, group;
@@ -448,9 +442,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           for (int i = 0; i < 16; ++i) {
             const int e = 32 * q + 2 * i;
             const float2 x2 = fma2(make_float2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1])), sc2, nm2);
-            const float2 p2 = (kPfPolyEvery > 0 && i % (kPfPolyEvery > 0 ? kPfPolyEvery : 1) == kPfPolyEvery - 1)
-                                  ? ex2_poly2(x2)
-                                  : make_float2(ex2(x2.x), ex2(x2.y));
+            const float2 p2 = make_float2(ex2(x2.x), ex2(x2.y));
             l2 = add2(l2, p2);
             const float2 q2 =
                 mul2(p2, add2(make_float2(__uint_as_float(ar[2 * i]), __uint_as_float(ar[2 * i + 1])), na2));

@@ -330,32 +330,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return d;
 }
 
-// 2^x for a pair, on the FMA and integer pipes instead of the SFU, for
-// x <= 2^22 (-inf included).  Cody-Waite range reduction: x = n + f with
-// n = floor(x) (taken from the low mantissa bits of x + 1.5*2^23 rounded
-// toward -inf) and f in [0, 1); 2^f from a cubic fitted for least maximum
-// relative error on [0, 1] (Lawson's iteratively reweighted least squares;
-// error <= 7.5e-5); 2^n added into the exponent field.  x is clamped to
-// -125 first (so the exponent field stays >= 1), and very small results
-// come out as ~2^-125 rather than 0.
-__device__ __forceinline__ float2 ex2_poly2(float2 x) {
-  constexpr float kMagic = 12582912.f;   // 1.5 * 2^23
-  x = make_float2(fmaxf(x.x, -125.f), fmaxf(x.y, -125.f));
-  float2 y;
-  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rm.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
-      : "=f"(y.x), "=f"(y.y)
-      : "f"(x.x), "f"(x.y), "f"(kMagic), "f"(kMagic));
-  const float2 n = add2(y, make_float2(-kMagic, -kMagic));
-  const float2 f = add2(x, make_float2(-n.x, -n.y));
-  float2 p = fma2(make_float2(0.07802419364452362f, 0.07802419364452362f), f,
-                  make_float2(0.2260672152042389f, 0.2260672152042389f));
-  p = fma2(p, f, make_float2(0.6958337426185608f, 0.6958337426185608f));
-  p = fma2(p, f, make_float2(0.9999251961708069f, 0.9999251961708069f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(y.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(y.y) << 23)));
-}
-
 // Named barrier over `nthreads` threads that also ANDs a predicate across them.
 __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t nthreads, bool v) {
   uint32_t r;
