@@ -23,4 +23,5 @@ from .parallax_oracle import (  # noqa: F401
     gather_paged_keys,
     prefill_rows,
     prefill_paged_rows,
+    prefill_grads,
 )

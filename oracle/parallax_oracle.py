@@ -44,6 +44,7 @@ __all__ = [
     "gather_paged_keys",
     "prefill_rows",
     "prefill_paged_rows",
+    "prefill_grads",
 ]
 
 
@@ -210,3 +211,47 @@ def prefill_paged_rows(q, rho, k_pool, v_pool, page_table, cu_seqlens_q, seq_len
         K, V = gathered[(b, kvh)]
         res.append(parallax_query(q[start + i, h], rho[start + i, h], K[:n], V[:n], scale))
     return np.stack(res) if res else np.zeros((0, v_pool.shape[-1]))
+
+
+def _prefill_out_torch(Q, R, K, V, scale: float, causal: bool):
+    """out of one (sequence, head) prefill from torch float64 tensors [T, d]:
+    softmax weights, the explicit d x d covariance of every row, its product
+    with the probe (the definition of ``parallax_query``, one row per t)."""
+    import torch
+    T = Q.shape[0]
+    s = scale * Q @ K.T
+    if causal:
+        s = s.masked_fill(torch.triu(torch.ones(T, T, dtype=torch.bool), diagonal=1), float("-inf"))
+    w = torch.softmax(s, dim=-1)                                   # [T, T]
+    vbar = w @ V
+    kbar = w @ K
+    kc = K[None, :, :] - kbar[:, None, :]                          # [T, T, d]
+    vc = V[None, :, :] - vbar[:, None, :]
+    sigma = torch.einsum("ti,tid,tie->tde", w, kc, vc)             # d_k x d_v per row
+    return vbar - torch.einsum("tde,td->te", sigma, R)
+
+
+def prefill_grads(q, rho, k, v, dout, scale: float, causal: bool = True):
+    """Gradients of sum(dout * out) for a prefill, in float64.
+
+    q, rho, dout: [B, H, T, d]; k, v: [B, Hkv, T, d].  ``out`` is built by
+    ``_prefill_out_torch`` from torch float64 tensors, and torch's
+    reverse-mode autograd (a library routine) differentiates it.  Returns
+    (dq, drho, dk, dv) as float64 numpy arrays shaped like the inputs.
+    """
+    import torch
+
+    def t(x):
+        return torch.tensor(np.asarray(x, dtype=np.float64), dtype=torch.float64, requires_grad=True)
+
+    Q, R, K, V = t(q), t(rho), t(k), t(v)
+    G = torch.tensor(np.asarray(dout, dtype=np.float64), dtype=torch.float64)
+    B, H = Q.shape[:2]
+    group = H // K.shape[1]
+    total = torch.zeros((), dtype=torch.float64)
+    for b in range(B):
+        for h in range(H):
+            out = _prefill_out_torch(Q[b, h], R[b, h], K[b, h // group], V[b, h // group], scale, causal)
+            total = total + (out * G[b, h]).sum()
+    total.backward()
+    return tuple(x.grad.numpy() for x in (Q, R, K, V))
