@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define PARALLAX_ABI_VERSION 2
+#define PARALLAX_ABI_VERSION 3
 
 typedef enum plx_status {
   PLX_OK = 0,
@@ -177,6 +177,50 @@ typedef struct plx_prefill_params {
  *   out      device, [B, H, T, d] of out_dtype. */
 plx_status parallax_prefill(const void* q, const void* rho, const void* k, const void* v,
                             void* out, const plx_prefill_params* p, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Training: the prefill forward with the per-row quantities its backward
+ * reads, and the backward.  For a row with weights w_i, probe values
+ * a_i = rho.k_i, abar = sum w_i a_i and vbar = sum w_i v_i the output is
+ * out = sum_i w_i (1 + abar - a_i) v_i (the covariance correction of the
+ * wispaper.ai blog "Parallax: Breaking the Boundary Bias with Parameterized
+ * Local Linear Attention", section "The Core Insight: Covariance Correction");
+ * the backward differentiates that expression (the pages print no
+ * gradient).
+ * ---------------------------------------------------------------------- */
+
+/* parallax_prefill, plus:
+ *   vbar    device float32 [B, H, T, d]: sum_i w_i v_i of every row.
+ *   stats   device float32 [B, H, T, 2]: (x, abar) per row, where
+ *           w_i = 2^(scale * log2(e) * q.k_i - x) (x = log2 of the softmax
+ *           normaliser of the scaled scores).
+ * out is written in out_dtype as by parallax_prefill.  Same errors. */
+plx_status parallax_prefill_train(const void* q, const void* rho, const void* k, const void* v,
+                                  void* out, float* vbar, float* stats,
+                                  const plx_prefill_params* p, cudaStream_t stream);
+
+/* Bytes of workspace parallax_prefill_backward needs (16 per row), or
+ * SIZE_MAX for invalid parameters. */
+size_t parallax_prefill_backward_workspace_size(const plx_prefill_params* p);
+
+/* Gradients of L through one prefill, given dout = dL/dout.
+ *   q, rho, k, v    the forward's inputs (bf16, layouts as parallax_prefill).
+ *   out, vbar, stats  the outputs of parallax_prefill_train for them (out
+ *                   in out_dtype).
+ *   dout            device bf16 [B, H, T, d].
+ *   dq, drho        device [B, H, T, d] of out_dtype.
+ *   dk, dv          device [B, Hkv, T, d] of out_dtype (summed over the
+ *                   query heads that share each KV head).
+ *   workspace       device, >= parallax_prefill_backward_workspace_size.
+ * Every output element is written exactly once (no atomics, deterministic).
+ * Three launches on `stream`.  Errors: PLX_ERR_INVALID_ARG (null or
+ * misaligned pointer, bad parameters), PLX_ERR_UNSUPPORTED (as
+ * parallax_prefill), PLX_ERR_WORKSPACE, PLX_ERR_CUDA. */
+plx_status parallax_prefill_backward(const void* q, const void* rho, const void* k, const void* v,
+                                     const void* out, const float* vbar, const float* stats,
+                                     const void* dout, void* dq, void* drho, void* dk, void* dv,
+                                     void* workspace, size_t workspace_bytes,
+                                     const plx_prefill_params* p, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Chunked (append) prefill over the paged cache: the step between a prompt

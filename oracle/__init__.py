@@ -24,4 +24,5 @@ from .parallax_oracle import (  # noqa: F401
     prefill_rows,
     prefill_paged_rows,
     prefill_grads,
+    query_grads,
 )

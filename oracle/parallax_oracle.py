@@ -45,6 +45,7 @@ __all__ = [
     "prefill_rows",
     "prefill_paged_rows",
     "prefill_grads",
+    "query_grads",
 ]
 
 
@@ -255,3 +256,25 @@ def prefill_grads(q, rho, k, v, dout, scale: float, causal: bool = True):
             total = total + (out * G[b, h]).sum()
     total.backward()
     return tuple(x.grad.numpy() for x in (Q, R, K, V))
+
+
+def query_grads(q, rho, keys, values, dout, scale: float):
+    """Gradients of dout . out for ONE query over the key set ``keys`` [n, d]
+    (the row of ``parallax_query``): returns (dq, drho, dkeys, dvalues) as
+    float64 numpy arrays.  Same construction as ``prefill_grads`` (torch
+    float64 autograd through the explicit covariance), for one row, so a
+    long prefill can be checked on sampled rows and keys."""
+    import torch
+
+    def t(x):
+        return torch.tensor(np.asarray(x, dtype=np.float64), dtype=torch.float64, requires_grad=True)
+
+    Q, R, K, V = t(np.asarray(q)[None]), t(np.asarray(rho)[None]), t(keys), t(values)
+    G = torch.tensor(np.asarray(dout, dtype=np.float64)[None], dtype=torch.float64)
+    w = torch.softmax(scale * Q @ K.T, dim=-1)                        # [1, n]
+    vbar = w @ V
+    kbar = w @ K
+    sigma = torch.einsum("ti,tid,tie->tde", w, K[None] - kbar[:, None], V[None] - vbar[:, None])
+    out = vbar - torch.einsum("tde,td->te", sigma, R)
+    (out * G).sum().backward()
+    return Q.grad.numpy()[0], R.grad.numpy()[0], K.grad.numpy(), V.grad.numpy()

@@ -74,6 +74,12 @@ lib.parallax_prefill.argtypes = [_vp, _vp, _vp, _vp, _vp, ctypes.POINTER(Prefill
 lib.parallax_prefill_paged.restype = ctypes.c_int
 lib.parallax_prefill_paged.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _i32p, _vp,
                                        ctypes.POINTER(PrefillPagedParams), _vp]
+lib.parallax_prefill_train.restype = ctypes.c_int
+lib.parallax_prefill_train.argtypes = [_vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.POINTER(PrefillParams), _vp]
+lib.parallax_prefill_backward_workspace_size.restype = ctypes.c_size_t
+lib.parallax_prefill_backward_workspace_size.argtypes = [ctypes.POINTER(PrefillParams)]
+lib.parallax_prefill_backward.restype = ctypes.c_int
+lib.parallax_prefill_backward.argtypes = [_vp] * 13 + [ctypes.c_size_t, ctypes.POINTER(PrefillParams), _vp]
 lib.parallax_decode_noalloc.restype = ctypes.c_int
 lib.parallax_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, ctypes.POINTER(DecodeParams), _vp]
 NOALLOC_SCRATCH_BYTES = 8 << 20
@@ -245,6 +251,87 @@ def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):
     if st != 0:
         raise ParallaxError(st, "parallax_prefill")
     return out
+
+
+def _prefill_params(q, k, causal, scale, out_dtype):
+    B, H, T, d = q.shape
+    scale = (1.0 / d ** 0.5) if scale is None else float(scale)
+    return PrefillParams(B, H, k.shape[1], T, d, PLX_BF16, _dtype_code(out_dtype), scale, 1 if causal else 0)
+
+
+def _check_prefill_inputs(q, rho, k, v):
+    for name, t in (("q", q), ("rho", rho), ("k", k), ("v", v)):
+        _check_cuda(name, t, torch.bfloat16)
+    B, H, T, d = q.shape
+    if rho.shape != q.shape or k.shape != v.shape or k.shape[0] != B or k.shape[2] != T or k.shape[3] != d:
+        raise ValueError("shape mismatch")
+
+
+def prefill_train(q, rho, k, v, causal=True, scale=None, *, out_dtype=None):
+    """Prefill forward for training: returns (out, vbar, stats).
+
+    vbar: float32 [B, H, T, d], the softmax average of the values of each
+    row; stats: float32 [B, H, T, 2], (x, abar) per row with weights
+    w_i = 2^(scale * log2(e) * q.k_i - x) and abar = sum_i w_i rho.k_i."""
+    _check_prefill_inputs(q, rho, k, v)
+    out_dtype = out_dtype or q.dtype
+    out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    vbar = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    stats = torch.empty(q.shape[:3] + (2,), dtype=torch.float32, device=q.device)
+    p = _prefill_params(q, k, causal, scale, out_dtype)
+    st = lib.parallax_prefill_train(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out), _ptr(vbar), _ptr(stats),
+                                    ctypes.byref(p), _stream_ptr(q.device))
+    if st != 0:
+        raise ParallaxError(st, "parallax_prefill_train")
+    return out, vbar, stats
+
+
+def prefill_backward(q, rho, k, v, out, vbar, stats, dout, causal=True, scale=None, *, grad_dtype=None):
+    """Gradients (dq, drho, dk, dv) of a prefill given dout = dL/dout.
+
+    ``out``, ``vbar``, ``stats`` come from prefill_train on the same inputs
+    (out in the dtype the loss saw).  Gradients are returned in
+    ``grad_dtype`` (default: out's dtype); dk, dv are summed over the query
+    heads that share a KV head."""
+    _check_prefill_inputs(q, rho, k, v)
+    _check_cuda("dout", dout, torch.bfloat16)
+    _check_cuda("out", out, out.dtype)
+    _check_cuda("vbar", vbar, torch.float32)
+    _check_cuda("stats", stats, torch.float32)
+    grad_dtype = grad_dtype or out.dtype
+    if grad_dtype != out.dtype:
+        raise ValueError("gradients are returned in out's dtype")
+    p = _prefill_params(q, k, causal, scale, out.dtype)
+    dq = torch.empty(q.shape, dtype=grad_dtype, device=q.device)
+    drho = torch.empty(q.shape, dtype=grad_dtype, device=q.device)
+    dk = torch.empty(k.shape, dtype=grad_dtype, device=q.device)
+    dv = torch.empty(v.shape, dtype=grad_dtype, device=q.device)
+    nbytes = lib.parallax_prefill_backward_workspace_size(ctypes.byref(p))
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    st = lib.parallax_prefill_backward(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out), _ptr(vbar), _ptr(stats),
+                                       _ptr(dout), _ptr(dq), _ptr(drho), _ptr(dk), _ptr(dv), _ptr(ws), nbytes,
+                                       ctypes.byref(p), _stream_ptr(q.device))
+    if st != 0:
+        raise ParallaxError(st, "parallax_prefill_backward")
+    return dq, drho, dk, dv
+
+
+class ParallaxPrefill(torch.autograd.Function):
+    """torch autograd node over prefill_train / prefill_backward (bf16 in and out)."""
+
+    @staticmethod
+    def forward(ctx, q, rho, k, v, causal=True, scale=None):
+        out, vbar, stats = prefill_train(q, rho, k, v, causal, scale)
+        ctx.save_for_backward(q, rho, k, v, out, vbar, stats)
+        ctx.causal, ctx.scale = causal, scale
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, rho, k, v, out, vbar, stats = ctx.saved_tensors
+        grads = prefill_backward(q, rho, k, v, out, vbar, stats, dout.to(torch.bfloat16).contiguous(),
+                                 ctx.causal, ctx.scale)
+        return grads + (None, None)
 
 
 def prefill_paged(q, rho, k_cache, v_cache, page_table, cu_seqlens_q, seq_lens, *, max_q_len, scale=None,

@@ -17,6 +17,7 @@
 #include "ptx.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill_bwd.cuh"
 
 namespace {
 
@@ -216,7 +217,8 @@ plx_status launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tr, c
 }
 
 plx_status launch_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,
-                          const plx_prefill_params* p, cudaStream_t stream) {
+                          const plx_prefill_params* p, cudaStream_t stream, float* vbar = nullptr,
+                          float2* stats = nullptr) {
   const int hkv = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
   const uint64_t rows_q = (uint64_t)p->batch * p->num_heads * p->seq_len;
   const uint64_t rows_kv = (uint64_t)p->batch * hkv * p->seq_len;
@@ -235,6 +237,8 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.out = out;
+  a.vbar = vbar;
+  a.stats = stats;
   return launch_prefill_kernel<false>(tq, tr, tk, tv, a, stream);
 }
 
@@ -272,6 +276,75 @@ plx_status validate_prefill_paged(const plx_prefill_paged_params* p) {
   if ((int64_t)p->total_q + kPfBM >= (int64_t)INT32_MAX) return PLX_ERR_UNSUPPORTED;
   if (((int64_t)p->max_q_len + kPfBM - 1) / kPfBM * p->batch * p->num_heads >= (int64_t)INT32_MAX)
     return PLX_ERR_UNSUPPORTED;
+  return PLX_OK;
+}
+
+// ----------------------------------------------------------- prefill backward
+size_t backward_rows_bytes(const plx_prefill_params* p) {
+  return ((size_t)p->batch * p->num_heads * p->seq_len * sizeof(float4) + 255) & ~size_t(255);
+}
+
+plx_status launch_prefill_backward(const void* q, const void* rho, const void* k, const void* v, const void* out,
+                                   const float* vbar, const float2* stats, const void* dout, void* dq, void* drho,
+                                   void* dk, void* dv, float4* rows, const plx_prefill_params* p,
+                                   cudaStream_t stream) {
+  const int hkv = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
+  const long long n_rows = (long long)p->batch * p->num_heads * p->seq_len;
+  const unsigned row_blocks = (unsigned)((n_rows + 7) / 8);
+  if (p->out_dtype == PLX_BF16)
+    prefill_bwd_rows_kernel<true><<<row_blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(dout), out, vbar, stats, rows, n_rows);
+  else
+    prefill_bwd_rows_kernel<false><<<row_blocks, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(dout), out, vbar, stats, rows, n_rows);
+  if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+
+  BwdArgs a{};
+  a.B = p->batch;
+  a.H = p->num_heads;
+  a.Hkv = hkv;
+  a.T = p->seq_len;
+  a.group = p->num_heads / hkv;
+  a.n_blk = (p->seq_len + kPfBM - 1) / kPfBM;
+  a.causal = p->causal;
+  a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
+  a.scale = p->scale;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.rows = rows;
+  a.dq = dq;
+  a.drho = drho;
+  a.dk = dk;
+  a.dv = dv;
+  const uint64_t rows_q = (uint64_t)n_rows;
+  const uint64_t rows_kv = (uint64_t)p->batch * hkv * p->seq_len;
+  {  // dq, drho: 128-row query tiles, 64-row key tiles
+    CUtensorMap tq, tr, tg, tk, tv;
+    if (!make_tmap_bf16(&tq, q, kPfD, rows_q, 64, kPfBM) || !make_tmap_bf16(&tr, rho, kPfD, rows_q, 64, kPfBM) ||
+        !make_tmap_bf16(&tg, dout, kPfD, rows_q, 64, kPfBM) || !make_tmap_bf16(&tk, k, kPfD, rows_kv, 64, kPfBN) ||
+        !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBN))
+      return PLX_ERR_CUDA;
+    constexpr int smem = BqLayout::kBytes;
+    if (cudaFuncSetAttribute(prefill_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return PLX_ERR_CUDA;
+    const long long grid = (long long)a.n_blk * a.B * a.H;
+    prefill_bwd_dq_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tg, tk, tv, a);
+    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+  }
+  {  // dk, dv: 128-row key tiles, 64-row query tiles
+    CUtensorMap tq, tr, tg, tk, tv;
+    if (!make_tmap_bf16(&tq, q, kPfD, rows_q, 64, kPfBN) || !make_tmap_bf16(&tr, rho, kPfD, rows_q, 64, kPfBN) ||
+        !make_tmap_bf16(&tg, dout, kPfD, rows_q, 64, kPfBN) || !make_tmap_bf16(&tk, k, kPfD, rows_kv, 64, kPfBM) ||
+        !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBM))
+      return PLX_ERR_CUDA;
+    constexpr int smem = BkLayout::kBytes;
+    if (cudaFuncSetAttribute(prefill_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+      return PLX_ERR_CUDA;
+    const long long grid = (long long)a.n_blk * a.B * hkv;
+    prefill_bwd_dkv_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tg, tk, tv, a);
+    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+  }
   return PLX_OK;
 }
 
@@ -418,6 +491,37 @@ plx_status parallax_prefill(const void* q, const void* rho, const void* k, const
   if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16))
     return PLX_ERR_INVALID_ARG;
   return launch_prefill(q, rho, k, v, out, p, stream);
+}
+
+plx_status parallax_prefill_train(const void* q, const void* rho, const void* k, const void* v, void* out,
+                                  float* vbar, float* stats, const plx_prefill_params* p, cudaStream_t stream) {
+  plx_status st = validate_prefill(p);
+  if (st != PLX_OK) return st;
+  if (!q || !rho || !k || !v || !out || !vbar || !stats) return PLX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      !aligned(vbar, 16) || !aligned(stats, 8))
+    return PLX_ERR_INVALID_ARG;
+  return launch_prefill(q, rho, k, v, out, p, stream, vbar, reinterpret_cast<float2*>(stats));
+}
+
+size_t parallax_prefill_backward_workspace_size(const plx_prefill_params* p) {
+  if (validate_prefill(p) != PLX_OK) return SIZE_MAX;
+  return backward_rows_bytes(p);
+}
+
+plx_status parallax_prefill_backward(const void* q, const void* rho, const void* k, const void* v,
+                                     const void* out, const float* vbar, const float* stats, const void* dout,
+                                     void* dq, void* drho, void* dk, void* dv, void* workspace,
+                                     size_t workspace_bytes, const plx_prefill_params* p, cudaStream_t stream) {
+  plx_status st = validate_prefill(p);
+  if (st != PLX_OK) return st;
+  const void* in[] = {q, rho, k, v, out, vbar, dout, dq, drho, dk, dv, workspace};
+  for (const void* x : in)
+    if (x == nullptr || !aligned(x, 16)) return PLX_ERR_INVALID_ARG;
+  if (stats == nullptr || !aligned(stats, 8)) return PLX_ERR_INVALID_ARG;
+  if (workspace_bytes < backward_rows_bytes(p)) return PLX_ERR_WORKSPACE;
+  return launch_prefill_backward(q, rho, k, v, out, vbar, reinterpret_cast<const float2*>(stats), dout, dq, drho,
+                                 dk, dv, static_cast<float4*>(workspace), p, stream);
 }
 
 plx_status parallax_prefill_paged(const void* q, const void* rho, const void* k_cache, const void* v_cache,

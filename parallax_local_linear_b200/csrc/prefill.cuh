@@ -92,6 +92,9 @@ struct PrefillArgs {
   const int32_t* seq_lens;        // [B] keys of each sequence, its queries included
   const int32_t* page_table;      // [B, max_pages] physical page of each 64-key tile
   int max_pages, num_pages, total_q, max_q;
+  // dense form, training: per-row quantities the backward pass reads (null: not written)
+  float* vbar;                    // [B, H, T, D]: vbar = O1 / l
+  float2* stats;                  // [B, H, T]: (m + log2 l, abar = c / l), weights w = 2^(s*scale*log2(e) - x)
 };
 
 struct PfLayout {
@@ -528,10 +531,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const float ma = lc_s[r * 3 + 2], mb = lc_s[(128 + r) * 3 + 2];
       const float mm = fmaxf(ma, mb);
       const float fa = ex2(ma - mm), fb = ex2(mb - mm);   // a warpgroup with no tiles has l = c = 0
-      const float lt = lc_s[r * 3] * fa + lc_s[(128 + r) * 3] * fb;
-      const float ct = lc_s[r * 3 + 1] * fa + lc_s[(128 + r) * 3 + 1] * fb;
+      // explicit fmaf throughout, so that both instantiations round alike
+      const float lt = fmaf(lc_s[r * 3], fa, lc_s[(128 + r) * 3] * fb);
+      const float ct = fmaf(lc_s[r * 3 + 1], fa, lc_s[(128 + r) * 3 + 1] * fb);
       const float inv = 1.f / lt;
-      const float corr = 1.f + ct * inv;
+      const float corr = fmaf(ct, inv, 1.f);
+      if constexpr (!kPaged) {
+        if (a.stats != nullptr && g == 0 && t < q_len)
+          // c accumulates e * (a - a_ref), so abar = c / l + a_ref
+          a.stats[(size_t)(b * a.H + h) * a.T + t] = make_float2(mm + __log2f(lt), ct * inv + aref);
+      }
       const size_t orow = (kPaged ? (size_t)(q_first + t) * a.H + h : (size_t)(b * a.H + h) * a.T + t) * kPfD + 64 * g;
 #pragma unroll 1
       for (int part = 0; part < 2; ++part) {
@@ -542,7 +551,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (t < q_len) {
           float v[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(o1[i]) * inv * corr - __uint_as_float(o2[i]) * inv;
+          for (int i = 0; i < 32; ++i) {
+            const float vb = __uint_as_float(o1[i]) * inv;   // vbar
+            v[i] = fmaf(vb, corr, -(__uint_as_float(o2[i]) * inv));
+            if constexpr (!kPaged) o1[i] = __float_as_uint(vb);
+          }
+          if constexpr (!kPaged) {
+            if (a.vbar != nullptr) {
+              float4* vbp = reinterpret_cast<float4*>(a.vbar + orow + part * 32);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                vbp[i] = make_float4(__uint_as_float(o1[4 * i]), __uint_as_float(o1[4 * i + 1]),
+                                     __uint_as_float(o1[4 * i + 2]), __uint_as_float(o1[4 * i + 3]));
+            }
+          }
           if (a.out_bf16) {
             uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + orow + part * 32);
 #pragma unroll

@@ -1,0 +1,691 @@
+// Parallax prefill backward on sm_100a: TMA, tcgen05.mma, tensor memory.
+//
+// For one query row t with visible keys i, softmax weights w_i, probe values
+// a_i = rho.k_i, abar = sum w_i a_i and vbar = sum w_i v_i, the forward output
+// (the covariance correction of the wispaper.ai blog "Parallax: Breaking the
+// Boundary Bias with Parameterized Local Linear Attention", section "The Core
+// Insight: Covariance Correction") can be written
+//     out = sum_i w_i (1 + abar - a_i) v_i.
+// With g = dL/dout, D_i = g.v_i, Gbar = g.vbar, Delta = g.out and
+// x_i = D_i - Gbar, differentiating gives (derived here, not printed on the
+// pages):
+//     dv_i   += w_i (1 + abar - a_i) g                     (u_i = w_i (1 + abar - a_i))
+//     dA_i    = -w_i x_i                                   (dL/da_i)
+//     dS_i    = w_i ((1 + abar - a_i) x_i + Gbar - Delta)  (dL/ds_i, s_i = scale q.k_i)
+//     dq      = scale sum_i dS_i k_i,      drho = sum_i dA_i k_i,
+//     dk_i   += scale dS_i q + dA_i rho.
+// w_i = 2^(s_i scale log2(e) - lse2) comes back from the forward's per-row
+// lse2 = m + log2(l); abar and vbar come from the forward too.
+//
+// Three launches:
+//   prefill_bwd_rows_kernel  per row: Gbar = g.vbar, Delta = g.out, packed
+//                            with (lse2, abar) into one float4.
+//   prefill_bwd_dq_kernel    query-stationary: one CTA per 128-row query tile
+//                            streams the key tiles it sees; S = QK^T,
+//                            A = RK^T, D = GV^T (tcgen05, fp32 in TMEM), the
+//                            elementwise warps form dS and dA in bf16, and
+//                            dQ += dS K, dR += dA K accumulate in TMEM.
+//   prefill_bwd_dkv_kernel   key-stationary: one CTA per 128-key tile of one
+//                            KV head streams the 64-row query tiles (of every
+//                            query head of its group) that see it;
+//                            S^T = KQ^T, A^T = KR^T, D^T = VG^T, and
+//                            dV += U^T G, dK += dS^T Q + dA^T R.
+// No atomics: every output element is written once, by one CTA.
+#pragma once
+
+#include "ptx.cuh"
+#include "prefill.cuh"
+
+namespace plx {
+
+struct BwdArgs {
+  int B, H, Hkv, T, group;
+  int n_blk;                      // dq: ceil(T / 128) query tiles; dkv: ceil(T / 128) key tiles
+  int causal, out_bf16;
+  float scale, scale_log2;
+  const float4* rows;             // [B, H, T]: (lse2, abar, Gbar, Delta)
+  void* dq;                       // [B, H, T, D]
+  void* drho;                     // [B, H, T, D]
+  void* dk;                       // [B, Hkv, T, D]
+  void* dv;                       // [B, Hkv, T, D]
+};
+
+// ---------------------------------------------------------------- per row
+// One warp per row: Gbar = g.vbar, Delta = g.out.  out is the forward output
+// in its own dtype (the loss saw those values).
+template <bool kOutBf16>
+__global__ void __launch_bounds__(256) prefill_bwd_rows_kernel(const __nv_bfloat16* __restrict__ dout,
+                                                               const void* __restrict__ out,
+                                                               const float* __restrict__ vbar,
+                                                               const float2* __restrict__ stats,
+                                                               float4* __restrict__ rows, long long n_rows) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const size_t base = (size_t)row * kPfD + lane * 4;
+  const uint2 gr = *reinterpret_cast<const uint2*>(dout + base);
+  const float g0 = bf16_lo_f(gr.x), g1 = bf16_hi_f(gr.x), g2 = bf16_lo_f(gr.y), g3 = bf16_hi_f(gr.y);
+  float o0, o1, o2, o3;
+  if constexpr (kOutBf16) {
+    const uint2 orw = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(out) + base);
+    o0 = bf16_lo_f(orw.x), o1 = bf16_hi_f(orw.x), o2 = bf16_lo_f(orw.y), o3 = bf16_hi_f(orw.y);
+  } else {
+    const float4 ov = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(out) + base);
+    o0 = ov.x, o1 = ov.y, o2 = ov.z, o3 = ov.w;
+  }
+  const float4 vb = *reinterpret_cast<const float4*>(vbar + base);
+  float delta = g0 * o0 + g1 * o1 + g2 * o2 + g3 * o3;
+  float gbar = g0 * vb.x + g1 * vb.y + g2 * vb.z + g3 * vb.w;
+  delta = warp_sum(delta);
+  gbar = warp_sum(gbar);
+  if (lane == 0) {
+    const float2 st = stats[row];
+    rows[row] = make_float4(st.x, st.y, gbar, delta);
+  }
+}
+
+// One element of the backward: u, scale * dS and dA of one (query, key)
+// pair.  A pair that is not visible gives zeros by selection: its inputs may
+// be anything (unloaded row records, keys past the end), NaN included.
+struct BwdElem {
+  float u, ds, da;
+};
+__device__ __forceinline__ BwdElem bwd_elem(float s, float a, float dv, float lse2, float abar, float gbar,
+                                            float gmd, float scale_log2, float scale, bool visible) {
+  const float w = ex2(s * scale_log2 - lse2);
+  const float e1 = 1.f + abar - a;
+  const float x = dv - gbar;
+  BwdElem r;
+  r.u = visible ? w * e1 : 0.f;
+  r.da = visible ? -w * x : 0.f;
+  r.ds = visible ? (w * scale) * fmaf(e1, x, gmd) : 0.f;   // gmd = Gbar - Delta
+  return r;
+}
+
+// TMEM columns shared by both kernels.
+constexpr uint32_t kBwAcc0 = 0, kBwAcc1 = 128;                 // dQ, dR  |  dK, dV
+constexpr uint32_t kBwS = 256, kBwA = 320, kBwD = 384;         // fp32 products of the current tile
+constexpr uint32_t kBwDS = 448, kBwDA = 480;                   // bf16 dS, dA of the current tile
+
+// ------------------------------------------------------------- dq kernel
+constexpr int kBqStages = 3;
+struct BqLayout {
+  static constexpr int kTile128 = 128 * kPfD * 2;   // 32 KB: two 64-column boxes of 128 rows
+  static constexpr int kTile64 = 64 * kPfD * 2;     // 16 KB: two 64-column boxes of 64 rows
+  static constexpr int kQ = 0, kR = kQ + kTile128, kG = kR + kTile128;
+  static constexpr int kK = kG + kTile128;
+  static constexpr int kV = kK + kBqStages * kTile64;
+  static constexpr int kBar = kV + kBqStages * kTile64;
+  // q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], sad_full, sad_free, dd_full, dd_free, drain
+  static constexpr int kNumBars = 1 + 4 * kBqStages + 5;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_r,
+                          const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
+  using Ly = BqLayout;
+  constexpr int S = kBqStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + S;
+  uint64_t* k_empty = v_full + S;
+  uint64_t* v_empty = k_empty + S;
+  uint64_t* sad_full = v_empty + S;   // S, A, D of the current tile are in TMEM
+  uint64_t* sad_free = sad_full + 1;  // the elementwise warps have read them
+  uint64_t* dd_full = sad_free + 1;   // dS, dA are in TMEM
+  uint64_t* dd_free = dd_full + 1;    // the products reading dS, dA are done
+  uint64_t* drain = dd_free + 1;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BH = a.B * a.H;
+  const int mblk = a.n_blk - 1 - (int)(blockIdx.x / BH);   // longest first
+  const int bh = blockIdx.x % BH;
+  const int b = bh / a.H, h = bh % a.H, kvh = h / a.group;
+  const int m0 = mblk * kPfBM;
+  const int kv_end = a.causal ? min(a.T, m0 + kPfBM) : a.T;
+  const int n = (kv_end + kPfBN - 1) / kPfBN;
+  const int q_row = (b * a.H + h) * a.T + m0;
+  const int kv_row = (b * a.Hkv + kvh) * a.T;
+  // Rows with fewer than 128 keys do not average out the bf16 rounding of
+  // dS and dA (dA is ~16/n per key and sums to zero): their key tiles (the
+  // first two) also enter the products as bf16 lo parts, kept in the D
+  // columns this half has already read.
+  const int split_tiles = (a.causal ? min(m0 + 1, a.T) : a.T) < 2 * kPfBN ? kPfSplitTiles : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    mbar_init(sad_full, 1);
+    mbar_init(sad_free, kPfSoftmax);
+    mbar_init(dd_full, kPfSoftmax);
+    mbar_init(dd_free, 1);
+    mbar_init(drain, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_s, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_r);
+      prefetch_tmap(&tm_g);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const uint64_t keep = l2_policy_evict_last();
+      const uint64_t once = l2_policy_evict_first();
+      mbar_arrive_expect_tx(q_full, 3 * Ly::kTile128);
+      for (int bx = 0; bx < 2; ++bx) {
+        tma_load_2d(sm + Ly::kQ + bx * (Ly::kTile128 / 2), &tm_q, bx * 64, q_row, q_full, once);
+        tma_load_2d(sm + Ly::kR + bx * (Ly::kTile128 / 2), &tm_r, bx * 64, q_row, q_full, once);
+        tma_load_2d(sm + Ly::kG + bx * (Ly::kTile128 / 2), &tm_g, bx * 64, q_row, q_full, once);
+      }
+      int issued_k = 0, issued_v = 0;
+      bool ok = true;
+      for (int j = 0; j < n && ok; ++j) {
+        const int s = j % S;
+        const uint32_t par = ((j / S) - 1) & 1;
+        const int row = kv_row + j * kPfBN;
+        if (j >= S && !(ok = mbar_wait_bounded(&k_empty[s], par))) break;
+        mbar_arrive_expect_tx(&k_full[s], Ly::kTile64);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_2d(sm + Ly::kK + s * Ly::kTile64 + bx * (Ly::kTile64 / 2), &tm_k, bx * 64, row, &k_full[s], keep);
+        ++issued_k;
+        if (j >= S && !(ok = mbar_wait_bounded(&v_empty[s], par))) break;
+        mbar_arrive_expect_tx(&v_full[s], Ly::kTile64);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_2d(sm + Ly::kV + s * Ly::kTile64 + bx * (Ly::kTile64 / 2), &tm_v, bx * 64, row, &v_full[s], keep);
+        ++issued_v;
+      }
+      // Every issued load must land before the CTA exits.
+      mbar_wait_bounded(q_full, 0);
+      for (int s = 0; s < S && s < issued_k; ++s)
+        mbar_wait_bounded(&k_full[s], ((s + ((issued_k - 1 - s) / S) * S) / S) & 1);
+      for (int s = 0; s < S && s < issued_v; ++s)
+        mbar_wait_bounded(&v_full[s], ((s + ((issued_v - 1 - s) / S) * S) / S) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdS = idesc_bf16(kPfBM, kPfBN, false);   // 128 x 64, K-major B
+    constexpr uint32_t kIdT = idesc_bf16(kPfBM, kPfD, true);     // 128 x 128, MN-major B
+    const uint64_t dq = smem_desc_sw128(smem_u32(sm + Ly::kQ), 16, 1024);
+    const uint64_t dr = smem_desc_sw128(smem_u32(sm + Ly::kR), 16, 1024);
+    const uint64_t dg = smem_desc_sw128(smem_u32(sm + Ly::kG), 16, 1024);
+    const uint64_t dk = smem_desc_sw128(smem_u32(sm + Ly::kK), 16, 1024);
+    const uint64_t dkt = smem_desc_sw128(smem_u32(sm + Ly::kK), Ly::kTile64 / 2, 1024);   // K as an MN-major B
+    const uint64_t dv = smem_desc_sw128(smem_u32(sm + Ly::kV), 16, 1024);
+    auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    };
+    bool ok = wait_warp(q_full, 0);
+    tc_fence_after();
+    // dQ += dS K, dR += dA K of tile jp (with the lo parts of a split tile)
+    auto value_products = [&](int jp) {
+      const int sp = jp % S;
+      const uint64_t kts = dkt + (uint64_t)((sp * Ly::kTile64) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < kPfBN / 16; ++kk) {
+        // 16 keys per step: 8 TMEM columns of packed bf16 pairs, 16 rows of K
+        const uint64_t kd = kts + (uint64_t)(kk * 16 * 128 / 16);
+        tc_mma_ts(tmem + kBwAcc0, tmem + kBwDS + kk * 8, kd, kIdT, (jp > 0 || kk > 0) ? 1u : 0u);
+        tc_mma_ts(tmem + kBwAcc1, tmem + kBwDA + kk * 8, kd, kIdT, (jp > 0 || kk > 0) ? 1u : 0u);
+      }
+      if (jp < split_tiles) {   // lo parts: keys 32h.. of dS at D + 32h, of dA at D + 32h + 16
+#pragma unroll
+        for (int kk = 0; kk < kPfBN / 16; ++kk) {
+          const uint64_t kd = kts + (uint64_t)(kk * 16 * 128 / 16);
+          const uint32_t pc = kBwD + 32u * (kk >> 1) + 8u * (kk & 1);
+          tc_mma_ts(tmem + kBwAcc0, tmem + pc, kd, kIdT, 1u);
+          tc_mma_ts(tmem + kBwAcc1, tmem + pc + 16, kd, kIdT, 1u);
+        }
+      }
+      tc_commit(dd_free);
+      tc_commit(&k_empty[sp]);   // K(jp) is done: scores and dQ, dR
+    };
+    for (int j = 0; ok && j <= n; ++j) {
+      // A split tile's lo parts sit in the D columns, so its value products
+      // go ahead of the next tile's score products (which rewrite D).
+      const bool early = j >= 1 && j - 1 < split_tiles;
+      if (early) {
+        if (!(ok = wait_warp(dd_full, (j - 1) & 1))) break;
+        tc_fence_after();
+        value_products(j - 1);
+      }
+      if (j < n) {
+        const int s = j % S;
+        if (!(ok = wait_warp(&k_full[s], (j / S) & 1))) break;
+        if (!(ok = wait_warp(&v_full[s], (j / S) & 1))) break;
+        if (j >= 1 && !(ok = wait_warp(sad_free, (j - 1) & 1))) break;
+        tc_fence_after();
+        const uint64_t dks = dk + (uint64_t)((s * Ly::kTile64) >> 4);
+        const uint64_t dvs = dv + (uint64_t)((s * Ly::kTile64) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < kPfD / 16; ++kk) {
+          const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTile128 / 2 / 16) + (kk & 3) * 2);
+          const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2);
+          tc_mma_ss(tmem + kBwS, dq + oa, dks + ob, kIdS, kk > 0);
+          tc_mma_ss(tmem + kBwA, dr + oa, dks + ob, kIdS, kk > 0);
+          tc_mma_ss(tmem + kBwD, dg + oa, dvs + ob, kIdS, kk > 0);
+        }
+        tc_commit(sad_full);
+        tc_commit(&v_empty[s]);   // V(j) only enters D
+      }
+      if (j >= 1 && !early) {
+        if (!(ok = wait_warp(dd_full, (j - 1) & 1))) break;
+        tc_fence_after();
+        value_products(j - 1);
+      }
+    }
+    if (!ok && lane == 0) report_error(2 /* PLX_DEVERR_TIMEOUT */);
+    tc_commit(drain);
+    wait_warp(drain, 0);
+  } else {
+    // ------------------------------------------------------------ elementwise
+    const int g = (warp - 2) >> 2;           // key-column half of every tile
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;            // query row within the tile
+    const int t = m0 + r;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const int key_lim = a.causal ? min(t + 1, a.T) : a.T;
+    const float4 rs = t < a.T ? a.rows[(size_t)(b * a.H + h) * a.T + t] : make_float4(0.f, 0.f, 0.f, 0.f);
+    const float lse2 = rs.x, abar = rs.y, gbar = rs.z, gmd = rs.z - rs.w;
+    bool fine = true;
+    int j = 0;
+    for (; j < n; ++j) {
+      fine = __all_sync(0xffffffffu, fine && mbar_wait_bounded(sad_full, j & 1));
+      if (!fine) break;
+      tc_fence_after();
+      uint32_t sr[32], ar[32], dr[32];
+      tmem_ld32(tmem + lane_off + kBwS + 32 * g, sr);
+      tmem_ld32(tmem + lane_off + kBwA + 32 * g, ar);
+      tmem_ld32(tmem + lane_off + kBwD + 32 * g, dr);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(sad_free);
+      const int key0 = j * kPfBN + 32 * g;
+      const bool split = j < split_tiles;
+      uint32_t pds[16], pda[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const BwdElem e0 = bwd_elem(__uint_as_float(sr[2 * i]), __uint_as_float(ar[2 * i]), __uint_as_float(dr[2 * i]),
+                                    lse2, abar, gbar, gmd, a.scale_log2, a.scale, key0 + 2 * i < key_lim);
+        const BwdElem e1 = bwd_elem(__uint_as_float(sr[2 * i + 1]), __uint_as_float(ar[2 * i + 1]),
+                                    __uint_as_float(dr[2 * i + 1]), lse2, abar, gbar, gmd, a.scale_log2, a.scale,
+                                    key0 + 2 * i + 1 < key_lim);
+        pds[i] = pack_bf16(e0.ds, e1.ds);
+        pda[i] = pack_bf16(e0.da, e1.da);
+        if (split) {   // lo parts reuse entries already consumed (sr[i], ar[i]: i <= 2i)
+          sr[i] = pack_bf16(e0.ds - bf16_lo_f(pds[i]), e1.ds - bf16_hi_f(pds[i]));
+          ar[i] = pack_bf16(e0.da - bf16_lo_f(pda[i]), e1.da - bf16_hi_f(pda[i]));
+        }
+      }
+      // The products of tile j-1 must be done with the dS / dA columns.
+      if (j >= 1) {
+        fine = __all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (j - 1) & 1));
+        if (!fine) break;
+        tc_fence_after();
+      }
+      tmem_st16(tmem + lane_off + kBwDS + 16 * g, pds);
+      tmem_st16(tmem + lane_off + kBwDA + 16 * g, pda);
+      if (split) {   // into this half's own D columns, already read
+        tmem_st16(tmem + lane_off + kBwD + 32 * g, sr);
+        tmem_st16(tmem + lane_off + kBwD + 32 * g + 16, ar);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(dd_full);
+    }
+    // ---- epilogue: the last dQ, dR products, then the rows
+    fine = __all_sync(0xffffffffu, fine && j == n && mbar_wait_bounded(dd_free, (n - 1) & 1));
+    if (fine) {
+      tc_fence_after();
+      const size_t orow = ((size_t)(b * a.H + h) * a.T + t) * kPfD + 64 * g;
+#pragma unroll 1
+      for (int part = 0; part < 4; ++part) {   // dQ cols 64g, 64g+32; dR cols 64g, 64g+32
+        uint32_t o[32];
+        const int acc = part >> 1, half = part & 1;
+        tmem_ld32(tmem + lane_off + (acc ? kBwAcc1 : kBwAcc0) + 64 * g + 32 * half, o);
+        tmem_wait_ld();
+        if (t < a.T) {
+          void* base = acc ? a.drho : a.dq;
+          if (a.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + orow + 32 * half);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16(__uint_as_float(o[8 * i]), __uint_as_float(o[8 * i + 1])),
+                                  pack_bf16(__uint_as_float(o[8 * i + 2]), __uint_as_float(o[8 * i + 3])),
+                                  pack_bf16(__uint_as_float(o[8 * i + 4]), __uint_as_float(o[8 * i + 5])),
+                                  pack_bf16(__uint_as_float(o[8 * i + 6]), __uint_as_float(o[8 * i + 7])));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + orow + 32 * half);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                   __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------ dkv kernel
+constexpr int kBkStages = 3;
+struct BkLayout {
+  static constexpr int kTile128 = 128 * kPfD * 2;   // 32 KB
+  static constexpr int kTile64 = 64 * kPfD * 2;     // 16 KB
+  static constexpr int kK = 0, kV = kK + kTile128;
+  // one stage: Q, R, G tiles of 64 query rows and their 64 row records
+  static constexpr int kStQ = 0, kStR = kTile64, kStG = 2 * kTile64, kStRows = 3 * kTile64;
+  static constexpr int kStage = 3 * kTile64 + 1024;   // 49 KB, a multiple of 1024
+  static constexpr int kRing = kV + kTile128;
+  static constexpr int kBar = kRing + kBkStages * kStage;
+  // kv_full, op_full[S], op_empty[S], sad_full, sad_free, dd_full, dd_free, drain
+  static constexpr int kNumBars = 1 + 2 * kBkStages + 5;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16 + 1024;
+};
+
+__global__ void __launch_bounds__(kPfThreads, 1)
+    prefill_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_r,
+                           const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_k,
+                           const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
+  using Ly = BkLayout;
+  constexpr int S = kBkStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
+  uint64_t* kv_full = bars;
+  uint64_t* op_full = bars + 1;
+  uint64_t* op_empty = op_full + S;
+  uint64_t* sad_full = op_empty + S;
+  uint64_t* sad_free = sad_full + 1;
+  uint64_t* dd_full = sad_free + 1;   // U, dS, dA are in TMEM
+  uint64_t* dd_free = dd_full + 1;    // the products reading them are done
+  uint64_t* drain = dd_free + 1;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int BHk = a.B * a.Hkv;
+  const int kb = (int)(blockIdx.x / BHk);   // causal: the first key tiles see the most queries
+  const int bk = blockIdx.x % BHk;
+  const int b = bk / a.Hkv, kvh = bk % a.Hkv;
+  const int k0 = kb * kPfBM;
+  const int nq_all = (a.T + kPfBN - 1) / kPfBN;
+  const int qb0 = a.causal ? k0 / kPfBN : 0;
+  const int nq = nq_all - qb0;                // query tiles per query head
+  const int N = a.group * nq;                  // iterations: (head of the group, query tile)
+  const int kv_row = (b * a.Hkv + kvh) * a.T + k0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&op_full[s], 1);
+      mbar_init(&op_empty[s], 1);
+    }
+    mbar_init(sad_full, 1);
+    mbar_init(sad_free, kPfSoftmax);
+    mbar_init(dd_full, kPfSoftmax);
+    mbar_init(dd_free, 1);
+    mbar_init(drain, 1);
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_s, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_s;
+
+  auto head_of = [&](int it) { return kvh * a.group + it / nq; };
+  auto tile_of = [&](int it) { return qb0 + it % nq; };
+  // Query tiles whose rows see fewer than 128 keys (the first two, causal)
+  // do not average out the bf16 rounding of U, dS and dA: they also enter
+  // the products as bf16 lo parts, kept in this half's A / D columns.
+  auto split_of = [&](int it) {
+    return a.causal ? tile_of(it) * kPfBN + 1 < 2 * kPfBN : a.T < 2 * kPfBN;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_q);
+      prefetch_tmap(&tm_r);
+      prefetch_tmap(&tm_g);
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const uint64_t keep = l2_policy_evict_last();
+      const uint64_t once = l2_policy_evict_first();
+      mbar_arrive_expect_tx(kv_full, 2 * Ly::kTile128);
+      for (int bx = 0; bx < 2; ++bx) {
+        tma_load_2d(sm + Ly::kK + bx * (Ly::kTile128 / 2), &tm_k, bx * 64, kv_row, kv_full, once);
+        tma_load_2d(sm + Ly::kV + bx * (Ly::kTile128 / 2), &tm_v, bx * 64, kv_row, kv_full, once);
+      }
+      int issued = 0;
+      for (int it = 0; it < N; ++it) {
+        const int s = it % S;
+        if (it >= S && !mbar_wait_bounded(&op_empty[s], ((it / S) - 1) & 1)) break;
+        const int hq = head_of(it), t0 = tile_of(it) * kPfBN;
+        const int row = (b * a.H + hq) * a.T + t0;
+        const int nrows = min(kPfBN, a.T - t0);   // row records past T are not read
+        uint8_t* st = sm + Ly::kRing + s * Ly::kStage;
+        mbar_arrive_expect_tx(&op_full[s], 3 * Ly::kTile64 + nrows * 16);
+        for (int bx = 0; bx < 2; ++bx) {
+          tma_load_2d(st + Ly::kStQ + bx * (Ly::kTile64 / 2), &tm_q, bx * 64, row, &op_full[s], keep);
+          tma_load_2d(st + Ly::kStR + bx * (Ly::kTile64 / 2), &tm_r, bx * 64, row, &op_full[s], keep);
+          tma_load_2d(st + Ly::kStG + bx * (Ly::kTile64 / 2), &tm_g, bx * 64, row, &op_full[s], keep);
+        }
+        bulk_load(st + Ly::kStRows, a.rows + (size_t)(b * a.H + hq) * a.T + t0, (uint32_t)nrows * 16, &op_full[s]);
+        ++issued;
+      }
+      mbar_wait_bounded(kv_full, 0);
+      for (int s = 0; s < S && s < issued; ++s)
+        mbar_wait_bounded(&op_full[s], ((s + ((issued - 1 - s) / S) * S) / S) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t kIdS = idesc_bf16(kPfBM, kPfBN, false);   // 128 keys x 64 queries, K-major B
+    constexpr uint32_t kIdT = idesc_bf16(kPfBM, kPfD, true);     // 128 keys x 128, MN-major B
+    const uint64_t dk = smem_desc_sw128(smem_u32(sm + Ly::kK), 16, 1024);
+    const uint64_t dvv = smem_desc_sw128(smem_u32(sm + Ly::kV), 16, 1024);
+    auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+    };
+    bool ok = wait_warp(kv_full, 0);
+    tc_fence_after();
+    // dV += U^T G, dK += dS^T Q + dA^T R of query tile ip (plus lo parts if split)
+    auto value_products = [&](int ip) {
+      const int sp = ip % S;
+      const uint32_t stp = smem_u32(sm + Ly::kRing + sp * Ly::kStage);
+      const uint64_t tq = smem_desc_sw128(stp + Ly::kStQ, Ly::kTile64 / 2, 1024);
+      const uint64_t tr = smem_desc_sw128(stp + Ly::kStR, Ly::kTile64 / 2, 1024);
+      const uint64_t tg = smem_desc_sw128(stp + Ly::kStG, Ly::kTile64 / 2, 1024);
+#pragma unroll
+      for (int kk = 0; kk < kPfBN / 16; ++kk) {
+        // 16 queries per step; U of queries 32h..32h+31 sits in columns 32h..32h+15
+        const uint64_t ko = (uint64_t)(kk * 16 * 128 / 16);
+        const uint32_t ph = 32u * (kk >> 1) + 8u * (kk & 1);
+        const uint32_t acc = (ip > 0 || kk > 0) ? 1u : 0u;
+        tc_mma_ts(tmem + kBwAcc1, tmem + kBwS + ph, tg + ko, kIdT, acc);
+        tc_mma_ts(tmem + kBwAcc0, tmem + kBwDS + kk * 8, tq + ko, kIdT, acc);
+        tc_mma_ts(tmem + kBwAcc0, tmem + kBwDA + kk * 8, tr + ko, kIdT, 1u);
+        if (split_of(ip)) {   // lo parts: U at A + 32h, dS at A + 32h + 16, dA at D + 32h
+          tc_mma_ts(tmem + kBwAcc1, tmem + kBwA + ph, tg + ko, kIdT, 1u);
+          tc_mma_ts(tmem + kBwAcc0, tmem + kBwA + 16 + ph, tq + ko, kIdT, 1u);
+          tc_mma_ts(tmem + kBwAcc0, tmem + kBwD + ph, tr + ko, kIdT, 1u);
+        }
+      }
+      tc_commit(dd_free);
+      tc_commit(&op_empty[sp]);
+    };
+    for (int it = 0; ok && it <= N; ++it) {
+      const int s = it % S;
+      const uint32_t st = smem_u32(sm + Ly::kRing + s * Ly::kStage);
+      // A split tile's lo parts sit in the A / D columns, so its products go
+      // ahead of this tile's A^T, D^T (which rewrite them).
+      const bool early = it >= 1 && split_of(it - 1);
+      if (early) {
+        if (!(ok = wait_warp(dd_full, (it - 1) & 1))) break;
+        tc_fence_after();
+        value_products(it - 1);
+      }
+      if (it < N) {
+        if (!(ok = wait_warp(&op_full[s], (it / S) & 1))) break;
+        if (it >= 1 && !(ok = wait_warp(sad_free, (it - 1) & 1))) break;
+        tc_fence_after();
+        const uint64_t br = smem_desc_sw128(st + Ly::kStR, 16, 1024);
+        const uint64_t bg = smem_desc_sw128(st + Ly::kStG, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kPfD / 16; ++kk) {
+          const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTile128 / 2 / 16) + (kk & 3) * 2);
+          const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2);
+          tc_mma_ss(tmem + kBwA, dk + oa, br + ob, kIdS, kk > 0);
+          tc_mma_ss(tmem + kBwD, dvv + oa, bg + ob, kIdS, kk > 0);
+        }
+      }
+      if (it >= 1 && !early) {
+        // U of the previous tile sits in the S^T columns, which S^T of this
+        // tile overwrites below.
+        if (!(ok = wait_warp(dd_full, (it - 1) & 1))) break;
+        tc_fence_after();
+        value_products(it - 1);
+      }
+      if (it < N) {
+        const uint64_t bq = smem_desc_sw128(st + Ly::kStQ, 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kPfD / 16; ++kk) {
+          const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTile128 / 2 / 16) + (kk & 3) * 2);
+          const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2);
+          tc_mma_ss(tmem + kBwS, dk + oa, bq + ob, kIdS, kk > 0);
+        }
+        tc_commit(sad_full);
+      }
+    }
+    if (!ok && lane == 0) report_error(2 /* PLX_DEVERR_TIMEOUT */);
+    tc_commit(drain);
+    wait_warp(drain, 0);
+  } else {
+    // ------------------------------------------------------------ elementwise
+    const int g = (warp - 2) >> 2;           // query-column half of every tile
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;            // key row within the tile
+    const int key = k0 + r;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    bool fine = true;
+    int it = 0;
+    for (; it < N; ++it) {
+      fine = __all_sync(0xffffffffu, fine && mbar_wait_bounded(sad_full, it & 1));
+      if (!fine) break;
+      tc_fence_after();
+      uint32_t sr[32], ar[32], dr[32];
+      tmem_ld32(tmem + lane_off + kBwS + 32 * g, sr);
+      tmem_ld32(tmem + lane_off + kBwA + 32 * g, ar);
+      tmem_ld32(tmem + lane_off + kBwD + 32 * g, dr);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(sad_free);
+      const int t0 = tile_of(it) * kPfBN + 32 * g;   // query of this thread's first column
+      const float4* rows = reinterpret_cast<const float4*>(sm + Ly::kRing + (it % S) * Ly::kStage + Ly::kStRows) + 32 * g;
+      const bool split = split_of(it);
+      uint32_t pu[16], pds[16], pda[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        BwdElem e[2];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int cc = 2 * i + c, tq = t0 + cc;
+          const bool vis = key < a.T && tq < a.T && (!a.causal || key <= tq);
+          const float4 rw = rows[cc];
+          e[c] = bwd_elem(__uint_as_float(sr[cc]), __uint_as_float(ar[cc]), __uint_as_float(dr[cc]), rw.x, rw.y,
+                          rw.z, rw.z - rw.w, a.scale_log2, a.scale, vis);
+        }
+        pu[i] = pack_bf16(e[0].u, e[1].u);
+        pds[i] = pack_bf16(e[0].ds, e[1].ds);
+        pda[i] = pack_bf16(e[0].da, e[1].da);
+        if (split) {   // lo parts reuse entries already consumed (sr[i], ar[i], dr[i]: i <= 2i)
+          sr[i] = pack_bf16(e[0].u - bf16_lo_f(pu[i]), e[1].u - bf16_hi_f(pu[i]));
+          ar[i] = pack_bf16(e[0].ds - bf16_lo_f(pds[i]), e[1].ds - bf16_hi_f(pds[i]));
+          dr[i] = pack_bf16(e[0].da - bf16_lo_f(pda[i]), e[1].da - bf16_hi_f(pda[i]));
+        }
+      }
+      if (it >= 1) {
+        fine = __all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (it - 1) & 1));
+        if (!fine) break;
+        tc_fence_after();
+      }
+      tmem_st16(tmem + lane_off + kBwS + 32 * g, pu);   // over this half's own S^T columns
+      tmem_st16(tmem + lane_off + kBwDS + 16 * g, pds);
+      tmem_st16(tmem + lane_off + kBwDA + 16 * g, pda);
+      if (split) {   // into this half's own A^T / D^T columns, already read
+        tmem_st16(tmem + lane_off + kBwA + 32 * g, sr);
+        tmem_st16(tmem + lane_off + kBwA + 32 * g + 16, ar);
+        tmem_st16(tmem + lane_off + kBwD + 32 * g, dr);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(dd_full);
+    }
+    // ---- epilogue: the last products, then the key rows
+    fine = __all_sync(0xffffffffu, fine && it == N && mbar_wait_bounded(dd_free, (N - 1) & 1));
+    if (fine) {
+      tc_fence_after();
+      const size_t orow = ((size_t)(b * a.Hkv + kvh) * a.T + key) * kPfD + 64 * g;
+#pragma unroll 1
+      for (int part = 0; part < 4; ++part) {   // dK cols 64g, 64g+32; dV cols 64g, 64g+32
+        uint32_t o[32];
+        const int acc = part >> 1, half = part & 1;
+        tmem_ld32(tmem + lane_off + (acc ? kBwAcc1 : kBwAcc0) + 64 * g + 32 * half, o);
+        tmem_wait_ld();
+        if (key < a.T) {
+          void* base = acc ? a.dv : a.dk;
+          if (a.out_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(base) + orow + 32 * half);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(pack_bf16(__uint_as_float(o[8 * i]), __uint_as_float(o[8 * i + 1])),
+                                  pack_bf16(__uint_as_float(o[8 * i + 2]), __uint_as_float(o[8 * i + 3])),
+                                  pack_bf16(__uint_as_float(o[8 * i + 4]), __uint_as_float(o[8 * i + 5])),
+                                  pack_bf16(__uint_as_float(o[8 * i + 6]), __uint_as_float(o[8 * i + 7])));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(base) + orow + 32 * half);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_float4(__uint_as_float(o[4 * i]), __uint_as_float(o[4 * i + 1]),
+                                   __uint_as_float(o[4 * i + 2]), __uint_as_float(o[4 * i + 3]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace plx

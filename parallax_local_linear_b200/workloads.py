@@ -384,3 +384,10 @@ def chunked_prefill_flops(q_lens, seq_lens, num_heads, head_dim, causal=True) ->
         q, L = int(q), int(L)
         total += q * (L - q) + q * (q + 1) // 2 if causal else q * L
     return 8 * head_dim * num_heads * total
+
+
+def dout_like(q, seed):
+    """dL/dout of a prefill: N(0, 1) draws rounded to bfloat16, shaped like q,
+    on q's device (a generator of its own, so q, rho, k, v are unchanged)."""
+    gen = _gen(q.device, seed)
+    return _normal(tuple(q.shape), gen, q.device, torch.bfloat16)

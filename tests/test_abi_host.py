@@ -43,7 +43,7 @@ def test_library_exports_every_declared_symbol(binding):
 
 
 def test_abi_version_and_status_strings(binding):
-    assert binding.lib.parallax_abi_version() == 2
+    assert binding.lib.parallax_abi_version() == 3
     for code, name in binding.STATUS.items():
         assert binding.lib.parallax_status_string(code).decode() == name
 
@@ -179,3 +179,25 @@ def test_no_cpu_fallback(binding):
     q = torch.zeros(1, 1, 64)
     with pytest.raises(ValueError, match="CUDA"):
         binding.decode(q, q, torch.zeros(1, 1, 4, 64), torch.zeros(1, 1, 4, 64))
+
+
+def _train_params(binding, **kw):
+    base = dict(batch=2, num_heads=4, num_kv_heads=2, seq_len=300, head_dim=128, in_dtype=1, out_dtype=0,
+                scale=0.088, causal=1)
+    base.update(kw)
+    return binding.PrefillParams(**base)
+
+
+def test_backward_workspace_size_and_validation(binding):
+    p = _train_params(binding)
+    assert binding.lib.parallax_prefill_backward_workspace_size(ctypes.byref(p)) == 2 * 4 * 300 * 16
+    bad = _train_params(binding, head_dim=64)
+    assert binding.lib.parallax_prefill_backward_workspace_size(ctypes.byref(bad)) == binding.SIZE_MAX
+    nul = [None] * 13
+    assert binding.lib.parallax_prefill_backward(*nul, 0, ctypes.byref(bad), None) == 2
+    assert binding.lib.parallax_prefill_backward(*nul, 0, ctypes.byref(p), None) == 1
+    assert binding.lib.parallax_prefill_train(*([None] * 7), ctypes.byref(p), None) == 1
+    buf = ctypes.create_string_buffer(64)
+    al = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
+    # every pointer present and aligned, workspace too small
+    assert binding.lib.parallax_prefill_backward(*([al] * 13), 16, ctypes.byref(p), None) == 3

@@ -97,6 +97,22 @@ def test_grouped_kv_heads_sum_their_queries_gradients():
         np.testing.assert_allclose(grads[i], rep[i].reshape(1, 2, 2, 6, 3).sum(2), rtol=1e-12)
 
 
+def test_row_gradients_sum_to_the_prefill_gradients():
+    q, rho, k, v, g = _case(H=2, Hkv=1, T=6, d=4)
+    dq, drho, dk, dv = oracle.prefill_grads(q, rho, k, v, g, 0.5, causal=True)
+    sk, sv = np.zeros_like(dk), np.zeros_like(dv)
+    for h in range(2):
+        for t in range(6):
+            rq, rr, rk, rv = oracle.query_grads(q[0, h, t], rho[0, h, t], k[0, 0, :t + 1], v[0, 0, :t + 1],
+                                                g[0, h, t], 0.5)
+            np.testing.assert_allclose(rq, dq[0, h, t], rtol=1e-12, atol=1e-14)
+            np.testing.assert_allclose(rr, drho[0, h, t], rtol=1e-12, atol=1e-14)
+            sk[0, 0, :t + 1] += rk
+            sv[0, 0, :t + 1] += rv
+    np.testing.assert_allclose(sk, dk, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(sv, dv, rtol=1e-12, atol=1e-14)
+
+
 def _mutant_transposed(Q, R, K, V, scale, causal):
     T = Q.shape[0]
     s = scale * Q @ K.T
