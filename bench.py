@@ -53,6 +53,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = {
     "decode": ["parallax_local_linear_b200/csrc/decode.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
     "prefill": ["parallax_local_linear_b200/csrc/prefill.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "prefill_bwd": ["parallax_local_linear_b200/csrc/prefill_bwd.cuh", "parallax_local_linear_b200/csrc/prefill.cuh",
+                    "parallax_local_linear_b200/csrc/ptx.cuh"],
 }
 KV_COPIES = 4          # decode_bf16: 4 x 128 MiB of KV, more than L2
 GRAPH_STEPS = 64       # decode calls per captured graph
@@ -78,7 +80,7 @@ def parse_args(argv=None):
 
 def default_steps(workload):
     return {"decode_f32": 20000, "decode_bf16": 8192, "decode_long": 200, "decode_paged": 200,
-            "prefill": 20, "prefill_paged": 20}[workload]
+            "prefill": 20, "prefill_paged": 20, "prefill_train": 10}[workload]
 
 
 def dist_env():
@@ -524,6 +526,89 @@ def bench_prefill_paged(args, w, rank, world, dev, peaks, peaks_kind):
     return res, x
 
 
+def bench_prefill_train(args, w, rank, world, dev, peaks, peaks_kind):
+    """Training step of the attention layer: forward with the backward's
+    row records, then the backward (4 launches per step)."""
+    from parallax_local_linear_b200 import binding as px
+
+    x = W.prefill_inputs(w, device=dev, seed=w.seed + 1000 * rank)
+    dout = W.dout_like(x["q"], w.seed + 2000 + rank)
+
+    def step(src, g):
+        out, vbar, stats = px.prefill_train(src["q"], src["rho"], src["k"], src["v"], w.causal, x["scale"])
+        return px.prefill_backward(src["q"], src["rho"], src["k"], src["v"], out, vbar, stats, g, w.causal,
+                                   x["scale"])
+
+    for _ in range(max(args.warmup, 3)):
+        step(x, dout)
+    torch.cuda.synchronize()
+    assert px.last_device_error() == 0
+    K = args.steps
+    stream = torch.cuda.current_stream()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        for i in range(K):
+            ev[i][0].record(stream)
+            out, vbar, stats = px.prefill_train(x["q"], x["rho"], x["k"], x["v"], w.causal, x["scale"])
+            ev[i][1].record(stream)
+            px.prefill_backward(x["q"], x["rho"], x["k"], x["v"], out, vbar, stats, dout, w.causal, x["scale"])
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = ev[0][0].elapsed_time(ev[-1][2])
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    f_fwd, f_bwd = W.prefill_flops(w), W.prefill_backward_flops(w)
+    flops = f_fwd + f_bwd
+    ms_max, total_flops = reduce_over_ranks(ms, flops * K, dev, world)
+    tflops = total_flops / (ms_max * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    achieved = f_bwd / (bwd_ms * 1e-3) / 1e12
+
+    # e2e through the public API: q, rho, k, v and dout copied in from pinned
+    # host memory each step, the four gradients read back.
+    hx = {k: x[k].cpu().pin_memory() for k in ("q", "rho", "k", "v")}
+    hx["dout"] = dout.cpu().pin_memory()
+    dx = {k: torch.empty_like(t, device=dev) for k, t in hx.items()}
+    oh = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (x["q"], x["rho"], x["k"], x["v"])]
+    Ke = max(1, min(K, 5))
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for _ in range(Ke):
+        for k in hx:
+            dx[k].copy_(hx[k], non_blocking=True)
+        grads = step(dx, dx["dout"])
+        for o, gg in zip(oh, grads):
+            o.copy_(gg, non_blocking=True)
+    e2.record()
+    torch.cuda.synchronize()
+    ems = s2.elapsed_time(e2)
+    e2e = {"value": round(flops * Ke / (ems * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in hx.values()),
+           "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in oh), "steps": Ke}
+    res = {
+        "metric": METRIC, "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "num_heads": w.num_heads, "seq_len": w.seq_len,
+                   "head_dim": w.head_dim, "causal": w.causal, "rho_scale": w.rho_scale,
+                   "flop_per_pair": "forward 8*d + backward 16*d", "fwd_ms": round(fwd_ms, 4),
+                   "bwd_ms": round(bwd_ms, 4), "l2": "inputs 671 MB > 126 MB L2"},
+        "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic("prefill_bwd", w.name),
+                     "peak_source": f"{peaks_kind} bf16_tflops_sustained",
+                     "kernel": "prefill backward: rows + dq + dkv kernels (one call)",
+                     "algorithmic_flops_per_launch": f_bwd},
+        "e2e": e2e, "gpu_launches": 4 * K, "clocks": clk.summary(),
+    }
+    return res, x
+
+
 # ------------------------------------------------------------- CPU oracle
 
 def oracle_decode_sample(w, inp, budget_s, max_steps=None):
@@ -576,6 +661,8 @@ def cpu_baseline(w, inp, budget_s):
         return cpu_baseline_prefill(w, inp, budget_s)
     if w.name == "prefill_paged":
         return cpu_baseline_prefill_paged(w, inp, budget_s)
+    if w.name == "prefill_train":
+        return cpu_baseline_prefill_train(w, inp, budget_s)
     gbs, secs, done, desc = oracle_decode_sample(w, inp, budget_s)
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
             "sample": desc, "seconds": round(secs, 2)}
@@ -631,6 +718,31 @@ def cpu_baseline_prefill_paged(w, inp, budget_s):
             "seconds": round(secs, 2)}
 
 
+def cpu_baseline_prefill_train(w, inp, budget_s):
+    """The oracle's forward rows plus its float64 autograd gradients on
+    (sequence, head) slices of the workload's first T' positions (T' = 256):
+    algorithmic FLOP 24*d per visible pair of those slices."""
+    import oracle
+    Tp = 256
+    rng = np.random.default_rng(2)
+    secs, flops, n = 0.0, 0, 0
+    while secs < budget_s:
+        b, h = int(rng.integers(w.batch)), int(rng.integers(w.num_heads))
+        sl = {k: inp[k][b:b + 1, h:h + 1, :Tp].double().cpu().numpy() for k in ("q", "rho", "k", "v")}
+        g = np.random.default_rng(n).standard_normal(sl["q"].shape)
+        t0 = time.perf_counter()
+        rows = [(0, 0, t) for t in range(Tp)]
+        oracle.prefill_rows(sl["q"], sl["rho"], sl["k"], sl["v"], rows, w.scale, causal=True)
+        oracle.prefill_grads(sl["q"], sl["rho"], sl["k"], sl["v"], g, w.scale, causal=True)
+        secs += time.perf_counter() - t0
+        flops += 24 * w.head_dim * Tp * (Tp + 1) // 2
+        n += 1
+    return {"value": round(flops / secs / 1e12, 6), "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{n} (sequence, head) slices of the first {Tp} positions: forward rows + float64 autograd "
+                      "gradients (algorithmic FLOP 24*d per visible pair)",
+            "seconds": round(secs, 2)}
+
+
 def reference_arm(args, w, rank, world):
     """The float64 oracle on the host cores, on this workload's metric.
 
@@ -640,8 +752,8 @@ def reference_arm(args, w, rank, world):
     if rank != 0:
         return None
     budget = max(0.05, 120.0 / max(1, args.steps + args.warmup))
-    if w.name == "prefill":
-        sub = W.PrefillWorkload("prefill", 1, 1, w.seq_len, w.head_dim, rho_scale=w.rho_scale, seed=w.seed)
+    if w.name in ("prefill", "prefill_train"):
+        sub = W.PrefillWorkload(w.name, 1, 1, w.seq_len, w.head_dim, rho_scale=w.rho_scale, seed=w.seed)
         inp = W.prefill_inputs(sub, device="cpu")
     elif w.name == "prefill_paged":
         inp = W.chunked_prefill_inputs(w, device="cpu")
@@ -651,8 +763,10 @@ def reference_arm(args, w, rank, world):
         inp = _host_decode_sample(w)
     vals, secs_all, desc = [], 0.0, ""
     for i in range(args.warmup + args.steps):
-        if w.name in ("prefill", "prefill_paged"):
-            cb = cpu_baseline(w, inp, budget)
+        if w.name in ("prefill", "prefill_paged", "prefill_train"):
+            sub_w = w if w.name != "prefill_train" else W.PrefillWorkload(w.name, 1, 1, w.seq_len, w.head_dim,
+                                                                          rho_scale=w.rho_scale, seed=w.seed)
+            cb = cpu_baseline(sub_w, inp, budget)
             v, secs, desc = cb["value"], cb["seconds"], cb["sample"]
         else:
             sub_w = w if inp["q"].shape[0] == w.batch else W.DecodeWorkload(
@@ -717,6 +831,8 @@ def main(argv=None):
             res, inp = bench_prefill(args, w, rank, world, dev, peaks, kind)
         elif w.name == "prefill_paged":
             res, inp = bench_prefill_paged(args, w, rank, world, dev, peaks, kind)
+        elif w.name == "prefill_train":
+            res, inp = bench_prefill_train(args, w, rank, world, dev, peaks, kind)
         else:
             res, inp = bench_decode(args, w, rank, world, dev, peaks, kind)
             inp = inp[0]

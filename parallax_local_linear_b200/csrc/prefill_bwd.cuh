@@ -322,34 +322,41 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc_fence_before();
       mbar_arrive(sad_free);
       const int key0 = j * kPfBN + 32 * g;
-      const bool split = j < split_tiles;
-      uint32_t pds[16], pda[16];
+      // The split is a separate instantiation so that ordinary tiles run a
+      // loop without it.
+      auto form = [&](auto split_tag) -> bool {
+        constexpr bool kSplit = decltype(split_tag)::value;
+        uint32_t pds[16], pda[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const BwdElem e0 = bwd_elem(__uint_as_float(sr[2 * i]), __uint_as_float(ar[2 * i]), __uint_as_float(dr[2 * i]),
-                                    lse2, abar, gbar, gmd, a.scale_log2, a.scale, key0 + 2 * i < key_lim);
-        const BwdElem e1 = bwd_elem(__uint_as_float(sr[2 * i + 1]), __uint_as_float(ar[2 * i + 1]),
-                                    __uint_as_float(dr[2 * i + 1]), lse2, abar, gbar, gmd, a.scale_log2, a.scale,
-                                    key0 + 2 * i + 1 < key_lim);
-        pds[i] = pack_bf16(e0.ds, e1.ds);
-        pda[i] = pack_bf16(e0.da, e1.da);
-        if (split) {   // lo parts reuse entries already consumed (sr[i], ar[i]: i <= 2i)
-          sr[i] = pack_bf16(e0.ds - bf16_lo_f(pds[i]), e1.ds - bf16_hi_f(pds[i]));
-          ar[i] = pack_bf16(e0.da - bf16_lo_f(pda[i]), e1.da - bf16_hi_f(pda[i]));
+        for (int i = 0; i < 16; ++i) {
+          const BwdElem e0 = bwd_elem(__uint_as_float(sr[2 * i]), __uint_as_float(ar[2 * i]),
+                                      __uint_as_float(dr[2 * i]), lse2, abar, gbar, gmd, a.scale_log2, a.scale,
+                                      key0 + 2 * i < key_lim);
+          const BwdElem e1 = bwd_elem(__uint_as_float(sr[2 * i + 1]), __uint_as_float(ar[2 * i + 1]),
+                                      __uint_as_float(dr[2 * i + 1]), lse2, abar, gbar, gmd, a.scale_log2, a.scale,
+                                      key0 + 2 * i + 1 < key_lim);
+          pds[i] = pack_bf16(e0.ds, e1.ds);
+          pda[i] = pack_bf16(e0.da, e1.da);
+          if constexpr (kSplit) {   // lo parts reuse entries already consumed (sr[i], ar[i]: i <= 2i)
+            sr[i] = pack_bf16(e0.ds - bf16_lo_f(pds[i]), e1.ds - bf16_hi_f(pds[i]));
+            ar[i] = pack_bf16(e0.da - bf16_lo_f(pda[i]), e1.da - bf16_hi_f(pda[i]));
+          }
         }
-      }
-      // The products of tile j-1 must be done with the dS / dA columns.
-      if (j >= 1) {
-        fine = __all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (j - 1) & 1));
-        if (!fine) break;
-        tc_fence_after();
-      }
-      tmem_st16(tmem + lane_off + kBwDS + 16 * g, pds);
-      tmem_st16(tmem + lane_off + kBwDA + 16 * g, pda);
-      if (split) {   // into this half's own D columns, already read
-        tmem_st16(tmem + lane_off + kBwD + 32 * g, sr);
-        tmem_st16(tmem + lane_off + kBwD + 32 * g + 16, ar);
-      }
+        // The products of tile j-1 must be done with the dS / dA columns.
+        if (j >= 1) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (j - 1) & 1))) return false;
+          tc_fence_after();
+        }
+        tmem_st16(tmem + lane_off + kBwDS + 16 * g, pds);
+        tmem_st16(tmem + lane_off + kBwDA + 16 * g, pda);
+        if constexpr (kSplit) {   // into this half's own D columns, already read
+          tmem_st16(tmem + lane_off + kBwD + 32 * g, sr);
+          tmem_st16(tmem + lane_off + kBwD + 32 * g + 16, ar);
+        }
+        return true;
+      };
+      fine = j < split_tiles ? form(std::true_type{}) : form(std::false_type{});
+      if (!fine) break;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(dd_full);
@@ -611,41 +618,47 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_arrive(sad_free);
       const int t0 = tile_of(it) * kPfBN + 32 * g;   // query of this thread's first column
       const float4* rows = reinterpret_cast<const float4*>(sm + Ly::kRing + (it % S) * Ly::kStage + Ly::kStRows) + 32 * g;
-      const bool split = split_of(it);
-      uint32_t pu[16], pds[16], pda[16];
+      // The split is a separate instantiation so that ordinary tiles run a
+      // loop without it.
+      auto form = [&](auto split_tag) -> bool {
+        constexpr bool kSplit = decltype(split_tag)::value;
+        uint32_t pu[16], pds[16], pda[16];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        BwdElem e[2];
+        for (int i = 0; i < 16; ++i) {
+          BwdElem e[2];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          const int cc = 2 * i + c, tq = t0 + cc;
-          const bool vis = key < a.T && tq < a.T && (!a.causal || key <= tq);
-          const float4 rw = rows[cc];
-          e[c] = bwd_elem(__uint_as_float(sr[cc]), __uint_as_float(ar[cc]), __uint_as_float(dr[cc]), rw.x, rw.y,
-                          rw.z, rw.z - rw.w, a.scale_log2, a.scale, vis);
+          for (int c = 0; c < 2; ++c) {
+            const int cc = 2 * i + c, tq = t0 + cc;
+            const bool vis = key < a.T && tq < a.T && (!a.causal || key <= tq);
+            const float4 rw = rows[cc];
+            e[c] = bwd_elem(__uint_as_float(sr[cc]), __uint_as_float(ar[cc]), __uint_as_float(dr[cc]), rw.x, rw.y,
+                            rw.z, rw.z - rw.w, a.scale_log2, a.scale, vis);
+          }
+          pu[i] = pack_bf16(e[0].u, e[1].u);
+          pds[i] = pack_bf16(e[0].ds, e[1].ds);
+          pda[i] = pack_bf16(e[0].da, e[1].da);
+          if constexpr (kSplit) {   // lo parts reuse entries already consumed (sr[i], ar[i], dr[i]: i <= 2i)
+            sr[i] = pack_bf16(e[0].u - bf16_lo_f(pu[i]), e[1].u - bf16_hi_f(pu[i]));
+            ar[i] = pack_bf16(e[0].ds - bf16_lo_f(pds[i]), e[1].ds - bf16_hi_f(pds[i]));
+            dr[i] = pack_bf16(e[0].da - bf16_lo_f(pda[i]), e[1].da - bf16_hi_f(pda[i]));
+          }
         }
-        pu[i] = pack_bf16(e[0].u, e[1].u);
-        pds[i] = pack_bf16(e[0].ds, e[1].ds);
-        pda[i] = pack_bf16(e[0].da, e[1].da);
-        if (split) {   // lo parts reuse entries already consumed (sr[i], ar[i], dr[i]: i <= 2i)
-          sr[i] = pack_bf16(e[0].u - bf16_lo_f(pu[i]), e[1].u - bf16_hi_f(pu[i]));
-          ar[i] = pack_bf16(e[0].ds - bf16_lo_f(pds[i]), e[1].ds - bf16_hi_f(pds[i]));
-          dr[i] = pack_bf16(e[0].da - bf16_lo_f(pda[i]), e[1].da - bf16_hi_f(pda[i]));
+        if (it >= 1) {
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (it - 1) & 1))) return false;
+          tc_fence_after();
         }
-      }
-      if (it >= 1) {
-        fine = __all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (it - 1) & 1));
-        if (!fine) break;
-        tc_fence_after();
-      }
-      tmem_st16(tmem + lane_off + kBwS + 32 * g, pu);   // over this half's own S^T columns
-      tmem_st16(tmem + lane_off + kBwDS + 16 * g, pds);
-      tmem_st16(tmem + lane_off + kBwDA + 16 * g, pda);
-      if (split) {   // into this half's own A^T / D^T columns, already read
-        tmem_st16(tmem + lane_off + kBwA + 32 * g, sr);
-        tmem_st16(tmem + lane_off + kBwA + 32 * g + 16, ar);
-        tmem_st16(tmem + lane_off + kBwD + 32 * g, dr);
-      }
+        tmem_st16(tmem + lane_off + kBwS + 32 * g, pu);   // over this half's own S^T columns
+        tmem_st16(tmem + lane_off + kBwDS + 16 * g, pds);
+        tmem_st16(tmem + lane_off + kBwDA + 16 * g, pda);
+        if constexpr (kSplit) {   // into this half's own A^T / D^T columns, already read
+          tmem_st16(tmem + lane_off + kBwA + 32 * g, sr);
+          tmem_st16(tmem + lane_off + kBwA + 32 * g + 16, ar);
+          tmem_st16(tmem + lane_off + kBwD + 32 * g, dr);
+        }
+        return true;
+      };
+      fine = split_of(it) ? form(std::true_type{}) : form(std::false_type{});
+      if (!fine) break;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(dd_full);

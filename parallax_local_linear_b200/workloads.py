@@ -14,6 +14,8 @@ Named workloads (head_dim d, Hq query heads, Hkv KV heads):
   decode_paged   128 sequences, L ~ U{512..65536}, Hq=16, Hkv=4, d=128,
                  64-token pages placed by a seeded permutation
   prefill        B=4, H=16, T=8192, d=128, causal, rho scaled by 0.1
+  prefill_train  the same shapes, forward for training plus backward, with
+                 dL/dout ~ N(0, 1)
   prefill_paged  chunked (append) prefill over a paged cache: 8 sequences,
                  H=16, Hkv=4, d=128; each appends a chunk of U{1024..4096}
                  queries to a cached prefix of U{0..8192} tokens; 64-token
@@ -97,6 +99,7 @@ WORKLOADS = {
     "decode_paged": DecodeWorkload("decode_paged", 128, 16, 4, 128, 65536, paged=True,
                                    min_len=512, seed=4),
     "prefill": PrefillWorkload("prefill", 4, 16, 8192, 128, seed=5),
+    "prefill_train": PrefillWorkload("prefill_train", 4, 16, 8192, 128, seed=5),
     "prefill_paged": ChunkedPrefillWorkload("prefill_paged", 8, 16, 4, 128, 1024, 4096, 8192, seed=6),
 }
 
@@ -391,3 +394,10 @@ def dout_like(q, seed):
     on q's device (a generator of its own, so q, rho, k, v are unchanged)."""
     gen = _gen(q.device, seed)
     return _normal(tuple(q.shape), gen, q.device, torch.bfloat16)
+
+
+def prefill_backward_flops(w: PrefillWorkload) -> int:
+    """Algorithmic FLOP of one prefill backward: 16*d per visible pair, one
+    pass over each product the gradients need (S, A, D = g.v, dQ, dR, dV and
+    the two dK products, 2*d each)."""
+    return 2 * prefill_flops(w)
