@@ -29,7 +29,10 @@
 //                            KV head streams the 64-row query tiles (of every
 //                            query head of its group) that see it;
 //                            S^T = KQ^T, A^T = KR^T, D^T = VG^T, and
-//                            dV += U^T G, dK += dS^T Q + dA^T R.
+//                            dV += U^T G, dK += dS^T Q + dA^T R.  Its
+//                            elementwise warps take 16 query columns at a
+//                            time; the queries' row records come with their
+//                            Q, R, G tiles.
 // No atomics: every output element is written once, by one CTA.
 #pragma once
 
@@ -43,7 +46,7 @@ struct BwdArgs {
   int n_blk;                      // dq: ceil(T / 128) query tiles; dkv: ceil(T / 128) key tiles
   int causal, out_bf16;
   float scale, scale_log2;
-  const float4* rows;             // [B, H, T]: (lse2, abar, Gbar, Delta)
+  const float4* rows;             // [B, H, T]: (lse2, 1 + abar, Gbar, Gbar - Delta)
   void* dq;                       // [B, H, T, D]
   void* drho;                     // [B, H, T, D]
   void* dk;                       // [B, Hkv, T, D]
@@ -52,7 +55,9 @@ struct BwdArgs {
 
 // ---------------------------------------------------------------- per row
 // One warp per row: Gbar = g.vbar, Delta = g.out.  out is the forward output
-// in its own dtype (the loss saw those values).
+// in its own dtype (the loss saw those values).  The record holds the
+// row's constants in the form the elementwise warps use:
+// (lse2, 1 + abar, Gbar, Gbar - Delta).
 template <bool kOutBf16>
 __global__ void __launch_bounds__(256) prefill_bwd_rows_kernel(const __nv_bfloat16* __restrict__ dout,
                                                                const void* __restrict__ out,
@@ -80,7 +85,7 @@ __global__ void __launch_bounds__(256) prefill_bwd_rows_kernel(const __nv_bfloat
   gbar = warp_sum(gbar);
   if (lane == 0) {
     const float2 st = stats[row];
-    rows[row] = make_float4(st.x, st.y, gbar, delta);
+    rows[row] = make_float4(st.x, 1.f + st.y, gbar, gbar - delta);
   }
 }
 
@@ -90,16 +95,32 @@ __global__ void __launch_bounds__(256) prefill_bwd_rows_kernel(const __nv_bfloat
 struct BwdElem {
   float u, ds, da;
 };
-__device__ __forceinline__ BwdElem bwd_elem(float s, float a, float dv, float lse2, float abar, float gbar,
+__device__ __forceinline__ BwdElem bwd_elem(float s, float a, float dv, float lse2, float c1a, float gbar,
                                             float gmd, float scale_log2, float scale, bool visible) {
   const float w = ex2(s * scale_log2 - lse2);
-  const float e1 = 1.f + abar - a;
+  const float e1 = c1a - a;   // c1a = 1 + abar
   const float x = dv - gbar;
   BwdElem r;
   r.u = visible ? w * e1 : 0.f;
   r.da = visible ? -w * x : 0.f;
   r.ds = visible ? (w * scale) * fmaf(e1, x, gmd) : 0.f;   // gmd = Gbar - Delta
   return r;
+}
+
+// The same for two pairs at once, on packed f32x2 arithmetic, every pair
+// visible.  s2, a2, d2: the two columns' S, A, D; r0, r1: the two queries'
+// records.  Returns packed bf16 (u, scale*dS, dA) pairs.
+__device__ __forceinline__ uint3 bwd_pair_visible(float2 s2, float2 a2, float2 d2, float4 r0, float4 r1,
+                                                  float scale_log2, float scale) {
+  const float2 x2 = fma2(s2, make_float2(scale_log2, scale_log2), make_float2(-r0.x, -r1.x));
+  const float2 w2 = make_float2(ex2(x2.x), ex2(x2.y));
+  const float2 e1 = add2(make_float2(r0.y, r1.y), make_float2(-a2.x, -a2.y));      // 1 + abar - a
+  const float2 nx = add2(make_float2(r0.z, r1.z), make_float2(-d2.x, -d2.y));      // Gbar - D = -x
+  const float2 u = mul2(w2, e1);
+  const float2 da = mul2(w2, nx);
+  const float2 t = fma2(e1, make_float2(-nx.x, -nx.y), make_float2(r0.w, r1.w));   // e1 x + Gbar - Delta
+  const float2 ds = mul2(mul2(w2, make_float2(scale, scale)), t);
+  return make_uint3(pack_bf16(u.x, u.y), pack_bf16(ds.x, ds.y), pack_bf16(da.x, da.y));
 }
 
 // TMEM columns shared by both kernels.
@@ -307,7 +328,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int key_lim = a.causal ? min(t + 1, a.T) : a.T;
     const float4 rs = t < a.T ? a.rows[(size_t)(b * a.H + h) * a.T + t] : make_float4(0.f, 0.f, 0.f, 0.f);
-    const float lse2 = rs.x, abar = rs.y, gbar = rs.z, gmd = rs.z - rs.w;
+    const float lse2 = rs.x, abar = rs.y, gbar = rs.z, gmd = rs.w;   // abar holds 1 + abar
     bool fine = true;
     int j = 0;
     for (; j < n; ++j) {
@@ -406,6 +427,7 @@ struct BkLayout {
   static constexpr int kTile64 = 64 * kPfD * 2;     // 16 KB
   static constexpr int kK = 0, kV = kK + kTile128;
   // one stage: Q, R, G tiles of 64 query rows and their 64 row records
+  // (they arrive with the tiles, long before the elementwise warps read them)
   static constexpr int kStQ = 0, kStR = kTile64, kStG = 2 * kTile64, kStRows = 3 * kTile64;
   static constexpr int kStage = 3 * kTile64 + 1024;   // 49 KB, a multiple of 1024
   static constexpr int kRing = kV + kTile128;
@@ -534,17 +556,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t tg = smem_desc_sw128(stp + Ly::kStG, Ly::kTile64 / 2, 1024);
 #pragma unroll
       for (int kk = 0; kk < kPfBN / 16; ++kk) {
-        // 16 queries per step; U of queries 32h..32h+31 sits in columns 32h..32h+15
+        // 16 queries per step.  U of queries 16kk.. sits in columns 16kk..16kk+7
+        // of the S^T block (its lo parts in 16kk+8..), dS / dA in 8kk..8kk+7 of
+        // their own blocks (lo parts: 16kk.. and 16kk+8.. of the A^T block).
         const uint64_t ko = (uint64_t)(kk * 16 * 128 / 16);
-        const uint32_t ph = 32u * (kk >> 1) + 8u * (kk & 1);
         const uint32_t acc = (ip > 0 || kk > 0) ? 1u : 0u;
-        tc_mma_ts(tmem + kBwAcc1, tmem + kBwS + ph, tg + ko, kIdT, acc);
+        tc_mma_ts(tmem + kBwAcc1, tmem + kBwS + 16 * kk, tg + ko, kIdT, acc);
         tc_mma_ts(tmem + kBwAcc0, tmem + kBwDS + kk * 8, tq + ko, kIdT, acc);
         tc_mma_ts(tmem + kBwAcc0, tmem + kBwDA + kk * 8, tr + ko, kIdT, 1u);
-        if (split_of(ip)) {   // lo parts: U at A + 32h, dS at A + 32h + 16, dA at D + 32h
-          tc_mma_ts(tmem + kBwAcc1, tmem + kBwA + ph, tg + ko, kIdT, 1u);
-          tc_mma_ts(tmem + kBwAcc0, tmem + kBwA + 16 + ph, tq + ko, kIdT, 1u);
-          tc_mma_ts(tmem + kBwAcc0, tmem + kBwD + ph, tr + ko, kIdT, 1u);
+        if (split_of(ip)) {
+          tc_mma_ts(tmem + kBwAcc1, tmem + kBwS + 16 * kk + 8, tg + ko, kIdT, 1u);
+          tc_mma_ts(tmem + kBwAcc0, tmem + kBwA + 16 * kk, tq + ko, kIdT, 1u);
+          tc_mma_ts(tmem + kBwAcc0, tmem + kBwA + 16 * kk + 8, tr + ko, kIdT, 1u);
         }
       }
       tc_commit(dd_free);
@@ -609,55 +632,94 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       fine = __all_sync(0xffffffffu, fine && mbar_wait_bounded(sad_full, it & 1));
       if (!fine) break;
       tc_fence_after();
-      uint32_t sr[32], ar[32], dr[32];
-      tmem_ld32(tmem + lane_off + kBwS + 32 * g, sr);
-      tmem_ld32(tmem + lane_off + kBwA + 32 * g, ar);
-      tmem_ld32(tmem + lane_off + kBwD + 32 * g, dr);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(sad_free);
       const int t0 = tile_of(it) * kPfBN + 32 * g;   // query of this thread's first column
-      const float4* rows = reinterpret_cast<const float4*>(sm + Ly::kRing + (it % S) * Ly::kStage + Ly::kStRows) + 32 * g;
-      // The split is a separate instantiation so that ordinary tiles run a
-      // loop without it.
-      auto form = [&](auto split_tag) -> bool {
+      // this half's 32 queries' row records, in the stage (entries past T are stale and masked)
+      const float4* rows_s =
+          reinterpret_cast<const float4*>(sm + Ly::kRing + (it % S) * Ly::kStage + Ly::kStRows) + 32 * g;
+      // every pair of this warp's 32 keys and this half's 32 queries visible?
+      const int kw0 = k0 + wq * 32;
+      const bool all_vis = kw0 + 31 < a.T && t0 + 31 < a.T && (!a.causal || t0 >= kw0 + 31);
+      const bool split = split_of(it);   // rare: the first two query tiles of the first key tile
+      // Two passes of 16 query columns, so that their S, A, D (48 registers)
+      // and their 16 row records (64) are all in flight at once.  Every
+      // output lands in columns this pass has already read: U of queries
+      // 16kk.. (kk = 2g + q) in S^T columns 16kk..16kk+7 (lo parts 16kk+8..),
+      // dS / dA in their own blocks, the lo parts of dS / dA in A^T columns
+      // 16kk.. and 16kk+8..
+      auto pass = [&](int q, auto split_tag, auto mask_tag) -> bool {
         constexpr bool kSplit = decltype(split_tag)::value;
-        uint32_t pu[16], pds[16], pda[16];
+        constexpr bool kMask = decltype(mask_tag)::value;
+        const uint32_t col = 32u * g + 16u * q;
+        uint32_t sr[16], ar[16], dr[16];
+        tmem_ld16(tmem + lane_off + kBwS + col, sr);
+        tmem_ld16(tmem + lane_off + kBwA + col, ar);
+        tmem_ld16(tmem + lane_off + kBwD + col, dr);
+        float4 rw[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          BwdElem e[2];
+        for (int c = 0; c < 16; ++c) rw[c] = rows_s[16 * q + c];
+        tmem_wait_ld();
+        if (q == 1) {   // S^T, A^T, D^T of this tile are all read
+          tc_fence_before();
+          mbar_arrive(sad_free);
+        }
+        uint32_t pu[8], pds[8], pda[8];
 #pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int cc = 2 * i + c, tq = t0 + cc;
-            const bool vis = key < a.T && tq < a.T && (!a.causal || key <= tq);
-            const float4 rw = rows[cc];
-            e[c] = bwd_elem(__uint_as_float(sr[cc]), __uint_as_float(ar[cc]), __uint_as_float(dr[cc]), rw.x, rw.y,
-                            rw.z, rw.z - rw.w, a.scale_log2, a.scale, vis);
+        for (int i = 0; i < 8; ++i) {
+          const int cc = 2 * i;
+          [[maybe_unused]] float2 uf, dsf, daf;
+          if constexpr (!kMask) {
+            const uint3 pk = bwd_pair_visible(make_float2(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])),
+                                              make_float2(__uint_as_float(ar[cc]), __uint_as_float(ar[cc + 1])),
+                                              make_float2(__uint_as_float(dr[cc]), __uint_as_float(dr[cc + 1])),
+                                              rw[cc], rw[cc + 1], a.scale_log2, a.scale);
+            pu[i] = pk.x;
+            pds[i] = pk.y;
+            pda[i] = pk.z;
+            static_assert(!kSplit || kMask, "split tiles take the masked path, which keeps fp32 values");
+          } else {
+            BwdElem e[2];
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int tq = t0 + 16 * q + cc + c;
+              const bool vis = key < a.T && tq < a.T && (!a.causal || key <= tq);
+              e[c] = bwd_elem(__uint_as_float(sr[cc + c]), __uint_as_float(ar[cc + c]), __uint_as_float(dr[cc + c]),
+                              rw[cc + c].x, rw[cc + c].y, rw[cc + c].z, rw[cc + c].w, a.scale_log2, a.scale, vis);
+            }
+            uf = make_float2(e[0].u, e[1].u);
+            dsf = make_float2(e[0].ds, e[1].ds);
+            daf = make_float2(e[0].da, e[1].da);
+            pu[i] = pack_bf16(uf.x, uf.y);
+            pds[i] = pack_bf16(dsf.x, dsf.y);
+            pda[i] = pack_bf16(daf.x, daf.y);
           }
-          pu[i] = pack_bf16(e[0].u, e[1].u);
-          pds[i] = pack_bf16(e[0].ds, e[1].ds);
-          pda[i] = pack_bf16(e[0].da, e[1].da);
-          if constexpr (kSplit) {   // lo parts reuse entries already consumed (sr[i], ar[i], dr[i]: i <= 2i)
-            sr[i] = pack_bf16(e[0].u - bf16_lo_f(pu[i]), e[1].u - bf16_hi_f(pu[i]));
-            ar[i] = pack_bf16(e[0].ds - bf16_lo_f(pds[i]), e[1].ds - bf16_hi_f(pds[i]));
-            dr[i] = pack_bf16(e[0].da - bf16_lo_f(pda[i]), e[1].da - bf16_hi_f(pda[i]));
+          if constexpr (kSplit && kMask) {   // lo parts reuse entries already consumed (i <= 2i)
+            sr[i] = pack_bf16(uf.x - bf16_lo_f(pu[i]), uf.y - bf16_hi_f(pu[i]));
+            ar[i] = pack_bf16(dsf.x - bf16_lo_f(pds[i]), dsf.y - bf16_hi_f(pds[i]));
+            dr[i] = pack_bf16(daf.x - bf16_lo_f(pda[i]), daf.y - bf16_hi_f(pda[i]));
           }
         }
-        if (it >= 1) {
+        // The products of the previous tile must be done with the dS / dA columns.
+        if (q == 0 && it >= 1) {
           if (!__all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (it - 1) & 1))) return false;
           tc_fence_after();
         }
-        tmem_st16(tmem + lane_off + kBwS + 32 * g, pu);   // over this half's own S^T columns
-        tmem_st16(tmem + lane_off + kBwDS + 16 * g, pds);
-        tmem_st16(tmem + lane_off + kBwDA + 16 * g, pda);
-        if constexpr (kSplit) {   // into this half's own A^T / D^T columns, already read
-          tmem_st16(tmem + lane_off + kBwA + 32 * g, sr);
-          tmem_st16(tmem + lane_off + kBwA + 32 * g + 16, ar);
-          tmem_st16(tmem + lane_off + kBwD + 32 * g, dr);
+        tmem_st8(tmem + lane_off + kBwS + col, pu);
+        tmem_st8(tmem + lane_off + kBwDS + 16 * g + 8 * q, pds);
+        tmem_st8(tmem + lane_off + kBwDA + 16 * g + 8 * q, pda);
+        if constexpr (kSplit) {
+          tmem_st8(tmem + lane_off + kBwS + col + 8, sr);
+          tmem_st8(tmem + lane_off + kBwA + col, ar);
+          tmem_st8(tmem + lane_off + kBwA + col + 8, dr);
         }
         return true;
       };
-      fine = split_of(it) ? form(std::true_type{}) : form(std::false_type{});
+#pragma unroll 1
+      for (int q = 0; q < 2 && fine; ++q) {
+        if (split)
+          fine = pass(q, std::true_type{}, std::true_type{});
+        else
+          fine = all_vis ? pass(q, std::false_type{}, std::false_type{}) : pass(q, std::false_type{}, std::true_type{});
+      }
       if (!fine) break;
       tmem_wait_st();
       tc_fence_before();
