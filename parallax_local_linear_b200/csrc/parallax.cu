@@ -280,8 +280,12 @@ plx_status validate_prefill_paged(const plx_prefill_paged_params* p) {
 }
 
 // ----------------------------------------------------------- prefill backward
-size_t backward_rows_bytes(const plx_prefill_params* p) {
+// Workspace of the backward: per row a float4 record and a 128-byte slab row.
+size_t backward_records_bytes(const plx_prefill_params* p) {
   return ((size_t)p->batch * p->num_heads * p->seq_len * sizeof(float4) + 255) & ~size_t(255);
+}
+size_t backward_rows_bytes(const plx_prefill_params* p) {
+  return backward_records_bytes(p) + (size_t)p->batch * p->num_heads * p->seq_len * 128;
 }
 
 plx_status launch_prefill_backward(const void* q, const void* rho, const void* k, const void* v, const void* out,
@@ -291,12 +295,14 @@ plx_status launch_prefill_backward(const void* q, const void* rho, const void* k
   const int hkv = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
   const long long n_rows = (long long)p->batch * p->num_heads * p->seq_len;
   const unsigned row_blocks = (unsigned)((n_rows + 7) / 8);
+  uint32_t* slab = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(rows) + backward_records_bytes(p));
+  const float scale_log2 = p->scale * 1.4426950408889634f;
   if (p->out_dtype == PLX_BF16)
     prefill_bwd_rows_kernel<true><<<row_blocks, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(dout), out, vbar, stats, rows, n_rows);
+        static_cast<const __nv_bfloat16*>(dout), out, vbar, stats, rows, slab, scale_log2, n_rows);
   else
     prefill_bwd_rows_kernel<false><<<row_blocks, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(dout), out, vbar, stats, rows, n_rows);
+        static_cast<const __nv_bfloat16*>(dout), out, vbar, stats, rows, slab, scale_log2, n_rows);
   if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
 
   BwdArgs a{};
@@ -331,18 +337,18 @@ plx_status launch_prefill_backward(const void* q, const void* rho, const void* k
     prefill_bwd_dq_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tg, tk, tv, a);
     if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
   }
-  {  // dk, dv: 128-row key tiles, 64-row query tiles
-    CUtensorMap tq, tr, tg, tk, tv;
+  {  // dk, dv: 128-row key tiles, 64-row query tiles (and their 64-column offset slab rows)
+    CUtensorMap tq, tr, tg, tk, tv, ts;
     if (!make_tmap_bf16(&tq, q, kPfD, rows_q, 64, kPfBN) || !make_tmap_bf16(&tr, rho, kPfD, rows_q, 64, kPfBN) ||
         !make_tmap_bf16(&tg, dout, kPfD, rows_q, 64, kPfBN) || !make_tmap_bf16(&tk, k, kPfD, rows_kv, 64, kPfBM) ||
-        !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBM))
+        !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBM) || !make_tmap_bf16(&ts, slab, 64, rows_q, 64, kPfBN))
       return PLX_ERR_CUDA;
     constexpr int smem = BkLayout::kBytes;
     if (cudaFuncSetAttribute(prefill_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
       return PLX_ERR_CUDA;
     const long long grid = (long long)a.n_blk * a.B * hkv;
-    prefill_bwd_dkv_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tg, tk, tv, a);
+    prefill_bwd_dkv_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tg, tk, tv, ts, a);
     if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
   }
   return PLX_OK;

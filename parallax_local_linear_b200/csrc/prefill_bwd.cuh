@@ -58,12 +58,20 @@ struct BwdArgs {
 // in its own dtype (the loss saw those values).  The record holds the
 // row's constants in the form the elementwise warps use:
 // (lse2, 1 + abar, Gbar, Gbar - Delta).
+//
+// It also writes the row's offsets for the key-stationary kernel's products,
+// as bf16 hi / lo pairs in a 64-column row: columns 0, 1 hold -lse2 / c
+// (c = scale * log2(e)), 16, 17 hold -(1 + abar), 32, 33 hold -Gbar, the rest
+// 0.  A product's extra k-step against a block of ones adds them, so that
+// kernel reads S - lse2 / c, A - (1 + abar) and D - Gbar straight from TMEM.
 template <bool kOutBf16>
 __global__ void __launch_bounds__(256) prefill_bwd_rows_kernel(const __nv_bfloat16* __restrict__ dout,
                                                                const void* __restrict__ out,
                                                                const float* __restrict__ vbar,
                                                                const float2* __restrict__ stats,
-                                                               float4* __restrict__ rows, long long n_rows) {
+                                                               float4* __restrict__ rows,
+                                                               uint32_t* __restrict__ slab, float scale_log2,
+                                                               long long n_rows) {
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= n_rows) return;
@@ -83,10 +91,16 @@ __global__ void __launch_bounds__(256) prefill_bwd_rows_kernel(const __nv_bfloat
   float gbar = g0 * vb.x + g1 * vb.y + g2 * vb.z + g3 * vb.w;
   delta = warp_sum(delta);
   gbar = warp_sum(gbar);
-  if (lane == 0) {
-    const float2 st = stats[row];
-    rows[row] = make_float4(st.x, 1.f + st.y, gbar, gbar - delta);
-  }
+  const float2 st = stats[row];
+  if (lane == 0) rows[row] = make_float4(st.x, 1.f + st.y, gbar, gbar - delta);
+  // lane j writes bf16 columns 2j, 2j+1 of the slab row
+  float off = 0.f;
+  if (lane == 0) off = -st.x / scale_log2;
+  if (lane == 8) off = -(1.f + st.y);
+  if (lane == 16) off = -gbar;
+  const uint32_t hi = pack_bf16(off, 0.f) & 0xffffu;
+  const float lo = off - bf16_lo_f(hi);
+  slab[(size_t)row * 32 + lane] = (lane == 0 || lane == 8 || lane == 16) ? (hi | (pack_bf16(lo, 0.f) << 16)) : 0u;
 }
 
 // One element of the backward: u, scale * dS and dA of one (query, key)
@@ -121,6 +135,30 @@ __device__ __forceinline__ uint3 bwd_pair_visible(float2 s2, float2 a2, float2 d
   const float2 t = fma2(e1, make_float2(-nx.x, -nx.y), make_float2(r0.w, r1.w));   // e1 x + Gbar - Delta
   const float2 ds = mul2(mul2(w2, make_float2(scale, scale)), t);
   return make_uint3(pack_bf16(u.x, u.y), pack_bf16(ds.x, ds.y), pack_bf16(da.x, da.y));
+}
+
+// The key-stationary kernel's version, on products whose offsets are folded
+// in: sp = S - lse2 / c, ap = A - (1 + abar) = -(1 + abar - a),
+// dp = D - Gbar = x; gmd = Gbar - Delta.  Then u = -w ap, dA = -w dp and
+// scale * dS = -w scale (ap dp - gmd).
+__device__ __forceinline__ uint3 bwd_pair_folded(float2 sp, float2 ap, float2 dp, float2 gmd, float scale_log2,
+                                                 float scale) {
+  const float2 x2 = mul2(sp, make_float2(scale_log2, scale_log2));
+  const float2 nw = make_float2(-ex2(x2.x), -ex2(x2.y));
+  const float2 u = mul2(nw, ap);
+  const float2 da = mul2(nw, dp);
+  const float2 t = fma2(ap, dp, make_float2(-gmd.x, -gmd.y));
+  const float2 ds = mul2(mul2(nw, make_float2(scale, scale)), t);
+  return make_uint3(pack_bf16(u.x, u.y), pack_bf16(ds.x, ds.y), pack_bf16(da.x, da.y));
+}
+__device__ __forceinline__ BwdElem bwd_elem_folded(float sp, float ap, float dp, float gmd, float scale_log2,
+                                                   float scale, bool visible) {
+  const float nw = -ex2(sp * scale_log2);
+  BwdElem r;
+  r.u = visible ? nw * ap : 0.f;
+  r.da = visible ? nw * dp : 0.f;
+  r.ds = visible ? (nw * scale) * fmaf(ap, dp, -gmd) : 0.f;
+  return r;
 }
 
 // TMEM columns shared by both kernels.
@@ -421,19 +459,22 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 }
 
 // ------------------------------------------------------------ dkv kernel
-constexpr int kBkStages = 3;
+constexpr int kBkStages = 2;
 struct BkLayout {
   static constexpr int kTile128 = 128 * kPfD * 2;   // 32 KB
   static constexpr int kTile64 = 64 * kPfD * 2;     // 16 KB
+  static constexpr int kSlab64 = 64 * 64 * 2;       // 8 KB: 64 rows of 64 bf16 columns
   static constexpr int kK = 0, kV = kK + kTile128;
-  // one stage: Q, R, G tiles of 64 query rows and their 64 row records
-  // (they arrive with the tiles, long before the elementwise warps read them)
-  static constexpr int kStQ = 0, kStR = kTile64, kStG = 2 * kTile64, kStRows = 3 * kTile64;
-  static constexpr int kStage = 3 * kTile64 + 1024;   // 49 KB, a multiple of 1024
-  static constexpr int kRing = kV + kTile128;
+  static constexpr int kOnes = kV + kTile128;       // 128 rows of 64 bf16 ones (the A side of the offset k-step)
+  // one stage: Q, R, G tiles of 64 query rows, their offset slab and their
+  // 64 row records (they arrive with the tiles, long before they are read)
+  static constexpr int kStQ = 0, kStR = kTile64, kStG = 2 * kTile64, kStSlab = 3 * kTile64;
+  static constexpr int kStRows = kStSlab + kSlab64;
+  static constexpr int kStage = kStRows + 1024;       // 57 KB, a multiple of 1024
+  static constexpr int kRing = kOnes + 2 * kSlab64;
   static constexpr int kBar = kRing + kBkStages * kStage;
-  // kv_full, op_full[S], op_empty[S], sad_full, sad_free, dd_full, dd_free, drain
-  static constexpr int kNumBars = 1 + 2 * kBkStages + 5;
+  // kv_full, op_full[S], op_empty[S], sad_full, sad_free, dd_full[2], dd_free, drain
+  static constexpr int kNumBars = 1 + 2 * kBkStages + 6;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16 + 1024;
 };
@@ -441,7 +482,8 @@ struct BkLayout {
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_r,
                            const __grid_constant__ CUtensorMap tm_g, const __grid_constant__ CUtensorMap tm_k,
-                           const __grid_constant__ CUtensorMap tm_v, const BwdArgs a) {
+                           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_slab,
+                           const BwdArgs a) {
   using Ly = BkLayout;
   constexpr int S = kBkStages;
   extern __shared__ uint8_t smem_raw[];
@@ -452,8 +494,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* op_empty = op_full + S;
   uint64_t* sad_full = op_empty + S;
   uint64_t* sad_free = sad_full + 1;
-  uint64_t* dd_full = sad_free + 1;   // U, dS, dA are in TMEM
-  uint64_t* dd_free = dd_full + 1;    // the products reading them are done
+  uint64_t* dd_full = sad_free + 1;   // [2]: U, dS, dA of pass 0 / 1 are in TMEM
+  uint64_t* dd_free = dd_full + 2;    // the products reading them are done
   uint64_t* drain = dd_free + 1;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
 
@@ -477,7 +519,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     mbar_init(sad_full, 1);
     mbar_init(sad_free, kPfSoftmax);
-    mbar_init(dd_full, kPfSoftmax);
+    mbar_init(&dd_full[0], kPfSoftmax);
+    mbar_init(&dd_full[1], kPfSoftmax);
     mbar_init(dd_free, 1);
     mbar_init(drain, 1);
     fence_mbarrier_init();
@@ -486,6 +529,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     tmem_alloc(tmem_base_s, 512);
     tmem_relinquish();
   }
+  // The A side of the offset k-step: bf16 ones (every column, so the swizzle
+  // does not matter).
+  for (int i = threadIdx.x; i < 2 * Ly::kSlab64 / 16; i += kPfThreads)
+    reinterpret_cast<uint4*>(sm + Ly::kOnes)[i] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -508,6 +556,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       prefetch_tmap(&tm_g);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
+      prefetch_tmap(&tm_slab);
       const uint64_t keep = l2_policy_evict_last();
       const uint64_t once = l2_policy_evict_first();
       mbar_arrive_expect_tx(kv_full, 2 * Ly::kTile128);
@@ -523,12 +572,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int row = (b * a.H + hq) * a.T + t0;
         const int nrows = min(kPfBN, a.T - t0);   // row records past T are not read
         uint8_t* st = sm + Ly::kRing + s * Ly::kStage;
-        mbar_arrive_expect_tx(&op_full[s], 3 * Ly::kTile64 + nrows * 16);
+        mbar_arrive_expect_tx(&op_full[s], 3 * Ly::kTile64 + Ly::kSlab64 + nrows * 16);
         for (int bx = 0; bx < 2; ++bx) {
           tma_load_2d(st + Ly::kStQ + bx * (Ly::kTile64 / 2), &tm_q, bx * 64, row, &op_full[s], keep);
           tma_load_2d(st + Ly::kStR + bx * (Ly::kTile64 / 2), &tm_r, bx * 64, row, &op_full[s], keep);
           tma_load_2d(st + Ly::kStG + bx * (Ly::kTile64 / 2), &tm_g, bx * 64, row, &op_full[s], keep);
         }
+        tma_load_2d(st + Ly::kStSlab, &tm_slab, 0, row, &op_full[s], keep);
         bulk_load(st + Ly::kStRows, a.rows + (size_t)(b * a.H + hq) * a.T + t0, (uint32_t)nrows * 16, &op_full[s]);
         ++issued;
       }
@@ -542,23 +592,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     constexpr uint32_t kIdT = idesc_bf16(kPfBM, kPfD, true);     // 128 keys x 128, MN-major B
     const uint64_t dk = smem_desc_sw128(smem_u32(sm + Ly::kK), 16, 1024);
     const uint64_t dvv = smem_desc_sw128(smem_u32(sm + Ly::kV), 16, 1024);
+    const uint64_t dones = smem_desc_sw128(smem_u32(sm + Ly::kOnes), 16, 1024);
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
     };
     bool ok = wait_warp(kv_full, 0);
     tc_fence_after();
-    // dV += U^T G, dK += dS^T Q + dA^T R of query tile ip (plus lo parts if split)
-    auto value_products = [&](int ip) {
+    // dV += U^T G, dK += dS^T Q + dA^T R of query tile ip, for the queries of
+    // elementwise pass q: 16q.. (first warpgroup) and 32 + 16q.. (second),
+    // i.e. k-steps kk = q and q + 2 (plus lo parts if split).
+    auto value_products = [&](int ip, int q) {
       const int sp = ip % S;
       const uint32_t stp = smem_u32(sm + Ly::kRing + sp * Ly::kStage);
       const uint64_t tq = smem_desc_sw128(stp + Ly::kStQ, Ly::kTile64 / 2, 1024);
       const uint64_t tr = smem_desc_sw128(stp + Ly::kStR, Ly::kTile64 / 2, 1024);
       const uint64_t tg = smem_desc_sw128(stp + Ly::kStG, Ly::kTile64 / 2, 1024);
 #pragma unroll
-      for (int kk = 0; kk < kPfBN / 16; ++kk) {
+      for (int h = 0; h < 2; ++h) {
         // 16 queries per step.  U of queries 16kk.. sits in columns 16kk..16kk+7
         // of the S^T block (its lo parts in 16kk+8..), dS / dA in 8kk..8kk+7 of
         // their own blocks (lo parts: 16kk.. and 16kk+8.. of the A^T block).
+        const int kk = q + 2 * h;
         const uint64_t ko = (uint64_t)(kk * 16 * 128 / 16);
         const uint32_t acc = (ip > 0 || kk > 0) ? 1u : 0u;
         tc_mma_ts(tmem + kBwAcc1, tmem + kBwS + 16 * kk, tg + ko, kIdT, acc);
@@ -570,20 +624,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc_mma_ts(tmem + kBwAcc0, tmem + kBwA + 16 * kk + 8, tr + ko, kIdT, 1u);
         }
       }
-      tc_commit(dd_free);
-      tc_commit(&op_empty[sp]);
+      if (q == 1) {
+        tc_commit(dd_free);
+        tc_commit(&op_empty[sp]);
+      }
+    };
+    auto both_passes = [&](int ip) -> bool {
+      for (int q = 0; q < 2; ++q) {
+        if (!wait_warp(&dd_full[q], ip & 1)) return false;
+        tc_fence_after();
+        value_products(ip, q);
+      }
+      return true;
     };
     for (int it = 0; ok && it <= N; ++it) {
       const int s = it % S;
       const uint32_t st = smem_u32(sm + Ly::kRing + s * Ly::kStage);
-      // A split tile's lo parts sit in the A / D columns, so its products go
+      // A split tile's lo parts sit in the A columns, so its products go
       // ahead of this tile's A^T, D^T (which rewrite them).
       const bool early = it >= 1 && split_of(it - 1);
-      if (early) {
-        if (!(ok = wait_warp(dd_full, (it - 1) & 1))) break;
-        tc_fence_after();
-        value_products(it - 1);
-      }
+      if (early && !(ok = both_passes(it - 1))) break;
       if (it < N) {
         if (!(ok = wait_warp(&op_full[s], (it / S) & 1))) break;
         if (it >= 1 && !(ok = wait_warp(sad_free, (it - 1) & 1))) break;
@@ -597,14 +657,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tc_mma_ss(tmem + kBwA, dk + oa, br + ob, kIdS, kk > 0);
           tc_mma_ss(tmem + kBwD, dvv + oa, bg + ob, kIdS, kk > 0);
         }
+        // offsets: A^T -= 1 + abar (slab columns 16..31), D^T -= Gbar (32..47)
+        const uint64_t bsl = smem_desc_sw128(st + Ly::kStSlab, 16, 1024);
+        tc_mma_ss(tmem + kBwA, dones, bsl + 2, kIdS, 1u);
+        tc_mma_ss(tmem + kBwD, dones, bsl + 4, kIdS, 1u);
       }
-      if (it >= 1 && !early) {
-        // U of the previous tile sits in the S^T columns, which S^T of this
-        // tile overwrites below.
-        if (!(ok = wait_warp(dd_full, (it - 1) & 1))) break;
-        tc_fence_after();
-        value_products(it - 1);
-      }
+      // U of the previous tile sits in the S^T columns, which S^T of this
+      // tile overwrites below.
+      if (it >= 1 && !early && !(ok = both_passes(it - 1))) break;
       if (it < N) {
         const uint64_t bq = smem_desc_sw128(st + Ly::kStQ, 16, 1024);
 #pragma unroll
@@ -613,6 +673,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2);
           tc_mma_ss(tmem + kBwS, dk + oa, bq + ob, kIdS, kk > 0);
         }
+        tc_mma_ss(tmem + kBwS, dones, smem_desc_sw128(st + Ly::kStSlab, 16, 1024), kIdS, 1u);   // S^T -= lse2 / c
         tc_commit(sad_full);
       }
     }
@@ -640,38 +701,37 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const int kw0 = k0 + wq * 32;
       const bool all_vis = kw0 + 31 < a.T && t0 + 31 < a.T && (!a.causal || t0 >= kw0 + 31);
       const bool split = split_of(it);   // rare: the first two query tiles of the first key tile
-      // Two passes of 16 query columns, so that their S, A, D (48 registers)
-      // and their 16 row records (64) are all in flight at once.  Every
-      // output lands in columns this pass has already read: U of queries
-      // 16kk.. (kk = 2g + q) in S^T columns 16kk..16kk+7 (lo parts 16kk+8..),
-      // dS / dA in their own blocks, the lo parts of dS / dA in A^T columns
-      // 16kk.. and 16kk+8..
-      auto pass = [&](int q, auto split_tag, auto mask_tag) -> bool {
+      // S^T, A^T, D^T of this half's 32 queries, all read at once so that the
+      // next tile's A^T, D^T products can start while this tile is worked on.
+      uint32_t sr[32], ar[32], dr[32];
+      tmem_ld32(tmem + lane_off + kBwS + 32 * g, sr);
+      tmem_ld32(tmem + lane_off + kBwA + 32 * g, ar);
+      tmem_ld32(tmem + lane_off + kBwD + 32 * g, dr);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(sad_free);
+      // Two passes of 16 queries; after each, the value products of its
+      // queries may start (dd_full[q]).  Every output lands in columns
+      // already read: U of queries 16kk.. (kk = 2g + q) in S^T columns
+      // 16kk..16kk+7 (lo parts 16kk+8..), dS / dA in their own blocks, the lo
+      // parts of dS / dA in A^T columns 16kk.. and 16kk+8..
+      auto pass = [&](auto q_tag, auto split_tag, auto mask_tag) -> bool {
+        constexpr int q = decltype(q_tag)::value;
         constexpr bool kSplit = decltype(split_tag)::value;
         constexpr bool kMask = decltype(mask_tag)::value;
         const uint32_t col = 32u * g + 16u * q;
-        uint32_t sr[16], ar[16], dr[16];
-        tmem_ld16(tmem + lane_off + kBwS + col, sr);
-        tmem_ld16(tmem + lane_off + kBwA + col, ar);
-        tmem_ld16(tmem + lane_off + kBwD + col, dr);
-        float4 rw[16];
+        float gw[16];   // Gbar - Delta of the pass's 16 queries (the rest is folded into S, A, D)
 #pragma unroll
-        for (int c = 0; c < 16; ++c) rw[c] = rows_s[16 * q + c];
-        tmem_wait_ld();
-        if (q == 1) {   // S^T, A^T, D^T of this tile are all read
-          tc_fence_before();
-          mbar_arrive(sad_free);
-        }
-        uint32_t pu[8], pds[8], pda[8];
+        for (int c = 0; c < 16; ++c) gw[c] = rows_s[16 * q + c].w;
+        uint32_t pu[8], pds[8], pda[8], lu[8], lds[8], lda[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          const int cc = 2 * i;
-          [[maybe_unused]] float2 uf, dsf, daf;
+          const int cc = 16 * q + 2 * i;
           if constexpr (!kMask) {
-            const uint3 pk = bwd_pair_visible(make_float2(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])),
-                                              make_float2(__uint_as_float(ar[cc]), __uint_as_float(ar[cc + 1])),
-                                              make_float2(__uint_as_float(dr[cc]), __uint_as_float(dr[cc + 1])),
-                                              rw[cc], rw[cc + 1], a.scale_log2, a.scale);
+            const uint3 pk = bwd_pair_folded(make_float2(__uint_as_float(sr[cc]), __uint_as_float(sr[cc + 1])),
+                                             make_float2(__uint_as_float(ar[cc]), __uint_as_float(ar[cc + 1])),
+                                             make_float2(__uint_as_float(dr[cc]), __uint_as_float(dr[cc + 1])),
+                                             make_float2(gw[2 * i], gw[2 * i + 1]), a.scale_log2, a.scale);
             pu[i] = pk.x;
             pds[i] = pk.y;
             pda[i] = pk.z;
@@ -680,22 +740,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             BwdElem e[2];
 #pragma unroll
             for (int c = 0; c < 2; ++c) {
-              const int tq = t0 + 16 * q + cc + c;
+              const int tq = t0 + cc + c;
               const bool vis = key < a.T && tq < a.T && (!a.causal || key <= tq);
-              e[c] = bwd_elem(__uint_as_float(sr[cc + c]), __uint_as_float(ar[cc + c]), __uint_as_float(dr[cc + c]),
-                              rw[cc + c].x, rw[cc + c].y, rw[cc + c].z, rw[cc + c].w, a.scale_log2, a.scale, vis);
+              e[c] = bwd_elem_folded(__uint_as_float(sr[cc + c]), __uint_as_float(ar[cc + c]),
+                                     __uint_as_float(dr[cc + c]), gw[2 * i + c], a.scale_log2, a.scale, vis);
             }
-            uf = make_float2(e[0].u, e[1].u);
-            dsf = make_float2(e[0].ds, e[1].ds);
-            daf = make_float2(e[0].da, e[1].da);
-            pu[i] = pack_bf16(uf.x, uf.y);
-            pds[i] = pack_bf16(dsf.x, dsf.y);
-            pda[i] = pack_bf16(daf.x, daf.y);
-          }
-          if constexpr (kSplit && kMask) {   // lo parts reuse entries already consumed (i <= 2i)
-            sr[i] = pack_bf16(uf.x - bf16_lo_f(pu[i]), uf.y - bf16_hi_f(pu[i]));
-            ar[i] = pack_bf16(dsf.x - bf16_lo_f(pds[i]), dsf.y - bf16_hi_f(pds[i]));
-            dr[i] = pack_bf16(daf.x - bf16_lo_f(pda[i]), daf.y - bf16_hi_f(pda[i]));
+            pu[i] = pack_bf16(e[0].u, e[1].u);
+            pds[i] = pack_bf16(e[0].ds, e[1].ds);
+            pda[i] = pack_bf16(e[0].da, e[1].da);
+            if constexpr (kSplit) {
+              lu[i] = pack_bf16(e[0].u - bf16_lo_f(pu[i]), e[1].u - bf16_hi_f(pu[i]));
+              lds[i] = pack_bf16(e[0].ds - bf16_lo_f(pds[i]), e[1].ds - bf16_hi_f(pds[i]));
+              lda[i] = pack_bf16(e[0].da - bf16_lo_f(pda[i]), e[1].da - bf16_hi_f(pda[i]));
+            }
           }
         }
         // The products of the previous tile must be done with the dS / dA columns.
@@ -707,23 +764,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tmem_st8(tmem + lane_off + kBwDS + 16 * g + 8 * q, pds);
         tmem_st8(tmem + lane_off + kBwDA + 16 * g + 8 * q, pda);
         if constexpr (kSplit) {
-          tmem_st8(tmem + lane_off + kBwS + col + 8, sr);
-          tmem_st8(tmem + lane_off + kBwA + col, ar);
-          tmem_st8(tmem + lane_off + kBwA + col + 8, dr);
+          tmem_st8(tmem + lane_off + kBwS + col + 8, lu);
+          tmem_st8(tmem + lane_off + kBwA + col, lds);
+          tmem_st8(tmem + lane_off + kBwA + col + 8, lda);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&dd_full[q]);
         return true;
       };
-#pragma unroll 1
-      for (int q = 0; q < 2 && fine; ++q) {
+      auto run_pass = [&](auto q_tag) {
         if (split)
-          fine = pass(q, std::true_type{}, std::true_type{});
-        else
-          fine = all_vis ? pass(q, std::false_type{}, std::false_type{}) : pass(q, std::false_type{}, std::true_type{});
-      }
+          return pass(q_tag, std::true_type{}, std::true_type{});
+        return all_vis ? pass(q_tag, std::false_type{}, std::false_type{})
+                       : pass(q_tag, std::false_type{}, std::true_type{});
+      };
+      fine = run_pass(std::integral_constant<int, 0>{}) && run_pass(std::integral_constant<int, 1>{});
       if (!fine) break;
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(dd_full);
     }
     // ---- epilogue: the last products, then the key rows
     fine = __all_sync(0xffffffffu, fine && it == N && mbar_wait_bounded(dd_free, (N - 1) & 1));
