@@ -381,24 +381,38 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tc_fence_before();
       mbar_arrive(sad_free);
       const int key0 = j * kPfBN + 32 * g;
-      // The split is a separate instantiation so that ordinary tiles run a
-      // loop without it.
-      auto form = [&](auto split_tag) -> bool {
+      // The split and the mask are separate instantiations so that ordinary
+      // tiles (every key of this half visible to every row of this warp) run
+      // a loop without either, on f32x2 pair arithmetic.
+      auto form = [&](auto split_tag, auto mask_tag) -> bool {
         constexpr bool kSplit = decltype(split_tag)::value;
+        constexpr bool kMask = decltype(mask_tag)::value;
         uint32_t pds[16], pda[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const BwdElem e0 = bwd_elem(__uint_as_float(sr[2 * i]), __uint_as_float(ar[2 * i]),
-                                      __uint_as_float(dr[2 * i]), lse2, abar, gbar, gmd, a.scale_log2, a.scale,
-                                      key0 + 2 * i < key_lim);
-          const BwdElem e1 = bwd_elem(__uint_as_float(sr[2 * i + 1]), __uint_as_float(ar[2 * i + 1]),
-                                      __uint_as_float(dr[2 * i + 1]), lse2, abar, gbar, gmd, a.scale_log2, a.scale,
-                                      key0 + 2 * i + 1 < key_lim);
-          pds[i] = pack_bf16(e0.ds, e1.ds);
-          pda[i] = pack_bf16(e0.da, e1.da);
-          if constexpr (kSplit) {   // lo parts reuse entries already consumed (sr[i], ar[i]: i <= 2i)
-            sr[i] = pack_bf16(e0.ds - bf16_lo_f(pds[i]), e1.ds - bf16_hi_f(pds[i]));
-            ar[i] = pack_bf16(e0.da - bf16_lo_f(pda[i]), e1.da - bf16_hi_f(pda[i]));
+          if constexpr (!kMask) {
+            const float4 r4 = make_float4(lse2, abar, gbar, gmd);
+            const uint3 pk = bwd_pair_visible(
+                make_float2(__uint_as_float(sr[2 * i]), __uint_as_float(sr[2 * i + 1])),
+                make_float2(__uint_as_float(ar[2 * i]), __uint_as_float(ar[2 * i + 1])),
+                make_float2(__uint_as_float(dr[2 * i]), __uint_as_float(dr[2 * i + 1])), r4, r4, a.scale_log2,
+                a.scale);
+            pds[i] = pk.y;
+            pda[i] = pk.z;
+            static_assert(!kSplit || kMask, "split tiles take the masked path, which keeps fp32 values");
+          } else {
+            const BwdElem e0 = bwd_elem(__uint_as_float(sr[2 * i]), __uint_as_float(ar[2 * i]),
+                                        __uint_as_float(dr[2 * i]), lse2, abar, gbar, gmd, a.scale_log2, a.scale,
+                                        key0 + 2 * i < key_lim);
+            const BwdElem e1 = bwd_elem(__uint_as_float(sr[2 * i + 1]), __uint_as_float(ar[2 * i + 1]),
+                                        __uint_as_float(dr[2 * i + 1]), lse2, abar, gbar, gmd, a.scale_log2,
+                                        a.scale, key0 + 2 * i + 1 < key_lim);
+            pds[i] = pack_bf16(e0.ds, e1.ds);
+            pda[i] = pack_bf16(e0.da, e1.da);
+            if constexpr (kSplit) {   // lo parts reuse entries already consumed (sr[i], ar[i]: i <= 2i)
+              sr[i] = pack_bf16(e0.ds - bf16_lo_f(pds[i]), e1.ds - bf16_hi_f(pds[i]));
+              ar[i] = pack_bf16(e0.da - bf16_lo_f(pda[i]), e1.da - bf16_hi_f(pda[i]));
+            }
           }
         }
         // The products of tile j-1 must be done with the dS / dA columns.
@@ -414,7 +428,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         return true;
       };
-      fine = j < split_tiles ? form(std::true_type{}) : form(std::false_type{});
+      // rows t0w..t0w+31 of this warp against keys key0..key0+31 of this half
+      const int t0w = m0 + wq * 32;
+      const bool all_vis = key0 + 31 < a.T && (a.causal ? key0 + 31 <= t0w : true);
+      if (j < split_tiles)
+        fine = form(std::true_type{}, std::true_type{});
+      else
+        fine = all_vis ? form(std::false_type{}, std::false_type{}) : form(std::false_type{}, std::true_type{});
       if (!fine) break;
       tmem_wait_st();
       tc_fence_before();
