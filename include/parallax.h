@@ -199,8 +199,9 @@ plx_status parallax_prefill_train(const void* q, const void* rho, const void* k,
                                   void* out, float* vbar, float* stats,
                                   const plx_prefill_params* p, cudaStream_t stream);
 
-/* Bytes of workspace parallax_prefill_backward needs (16 per row), or
- * SIZE_MAX for invalid parameters. */
+/* Bytes of workspace parallax_prefill_backward needs, or SIZE_MAX for
+ * invalid parameters: per row (B * H * T rows) a 16-byte record (rounded up
+ * to 256 bytes in total) and a 128-byte row of bf16 offsets. */
 size_t parallax_prefill_backward_workspace_size(const plx_prefill_params* p);
 
 /* Gradients of L through one prefill, given dout = dL/dout.
