@@ -97,6 +97,42 @@ struct PrefillArgs {
   float2* stats;                  // [B, H, T]: (m + log2 l, abar = c / l), weights w = 2^(s*scale*log2(e) - x)
 };
 
+// Four MMAs under one elect.sync: the issuing warp spends fewer instructions
+// per MMA, which matters when it shares its sub-partition with busy warps
+// (the tensor pipe's queue is short, so a late issue leaves it idle).
+// MMAs 0 and 1 take accumulate flag acc01, MMAs 2 and 3 acc23.
+__device__ __forceinline__ void tc_mma_ss4(uint32_t d0, uint64_t a0, uint64_t b0, uint32_t d1, uint64_t a1,
+                                           uint64_t b1, uint32_t d2, uint64_t a2, uint64_t b2, uint32_t d3,
+                                           uint64_t a3, uint64_t b3, uint32_t idesc, uint32_t acc01,
+                                           uint32_t acc23) {
+  asm volatile(
+      "{\n\t.reg .pred p01, p23, e;\n\tsetp.ne.b32 p01, %13, 0;\n\tsetp.ne.b32 p23, %14, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %12, p01;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], %4, %5, %12, p01;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%6], %7, %8, %12, p23;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%9], %10, %11, %12, p23;\n\t}" ::"r"(d0),
+      "l"(a0), "l"(b0), "r"(d1), "l"(a1), "l"(b1), "r"(d2), "l"(a2), "l"(b2), "r"(d3), "l"(a3), "l"(b3),
+      "r"(idesc), "r"(acc01), "r"(acc23)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_mma_ts4(uint32_t d0, uint32_t a0, uint64_t b0, uint32_t d1, uint32_t a1,
+                                           uint64_t b1, uint32_t d2, uint32_t a2, uint64_t b2, uint32_t d3,
+                                           uint32_t a3, uint64_t b3, uint32_t idesc, uint32_t acc01,
+                                           uint32_t acc23) {
+  asm volatile(
+      "{\n\t.reg .pred p01, p23, e;\n\tsetp.ne.b32 p01, %13, 0;\n\tsetp.ne.b32 p23, %14, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %12, p01;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], [%4], %5, %12, p01;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%6], [%7], %8, %12, p23;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%9], [%10], %11, %12, p23;\n\t}" ::"r"(d0),
+      "r"(a0), "l"(b0), "r"(d1), "r"(a1), "l"(b1), "r"(d2), "r"(a2), "l"(b2), "r"(d3), "r"(a3), "l"(b3),
+      "r"(idesc), "r"(acc01), "r"(acc23)
+      : "memory");
+}
+
 struct PfLayout {
   static constexpr int kQBytes = kPfBM * kPfD * 2;       // 32 KB: two 64-column boxes of 128 rows
   static constexpr int kKVBytes = kPfBN * kPfD * 2;      // 16 KB: two 64-column boxes of 64 rows
@@ -300,12 +336,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
         const uint64_t dks = dk + (uint64_t)((s * Ly::kKVBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kPfD / 16; ++kk) {
-          // 16 columns of d per step: box kk / 4, 32 bytes into the 128-byte row per step
-          const uint64_t oq = (uint64_t)((kk >> 2) * (Ly::kQBytes / 2 / 16) + (kk & 3) * 2);
-          const uint64_t okk = (uint64_t)((kk >> 2) * (Ly::kKVBytes / 2 / 16) + (kk & 3) * 2);
-          tc_mma_ss(tmem + col_s(b2), dq + oq, dks + okk, kIdS, kk > 0);
-          tc_mma_ss(tmem + col_a(b2), dr + oq, dks + okk, kIdS, kk > 0);
+        for (int kk = 0; kk < kPfD / 16; kk += 2) {
+          // 16 columns of d per step: box kk / 4, 32 bytes into the 128-byte row per
+          // step; S and A of two steps per issue
+          const uint64_t oq0 = (uint64_t)((kk >> 2) * (Ly::kQBytes / 2 / 16) + (kk & 3) * 2);
+          const uint64_t ok0 = (uint64_t)((kk >> 2) * (Ly::kKVBytes / 2 / 16) + (kk & 3) * 2);
+          const uint64_t oq1 = oq0 + 2, ok1 = ok0 + 2;   // kk + 1 stays in the same box
+          tc_mma_ss4(tmem + col_s(b2), dq + oq0, dks + ok0, tmem + col_a(b2), dr + oq0, dks + ok0,
+                     tmem + col_s(b2), dq + oq1, dks + ok1, tmem + col_a(b2), dr + oq1, dks + ok1, kIdS,
+                     kk > 0 ? 1u : 0u, 1u);
         }
         tc_commit(&s_full[b2]);
         tc_commit(&k_empty[s]);   // K(j) is free once the score products are done
@@ -319,21 +358,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
         const uint64_t dvs = dv + (uint64_t)((sp * Ly::kKVBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < kPfBN / 16; ++kk) {
+        for (int kk = 0; kk < kPfBN / 16; kk += 2) {
           // 16 keys per step: 8 TMEM columns of packed bf16 pairs (keys 32q..32q+31
-          // sit in columns 32q..32q+15), 16 rows of V
-          const uint64_t vd = dvs + (uint64_t)(kk * 16 * 128 / 16);
-          const uint32_t pc = 32u * (kk >> 1) + 8u * (kk & 1);
-          tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + pc, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
-          tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + pc, vd, kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+          // sit in columns 32q..32q+15), 16 rows of V; O1 and O2 of two steps per issue
+          const uint64_t vd0 = dvs + (uint64_t)(kk * 16 * 128 / 16), vd1 = vd0 + 16 * 128 / 16;
+          const uint32_t pc0 = 32u * (kk >> 1), pc1 = pc0 + 8u;   // kk even: (kk & 1) = 0, kk + 1 odd
+          tc_mma_ts4(tmem + kColO1, tmem + col_s(bp) + pc0, vd0, tmem + kColO2, tmem + col_a(bp) + pc0, vd0,
+                     tmem + kColO1, tmem + col_s(bp) + pc1, vd1, tmem + kColO2, tmem + col_a(bp) + pc1, vd1, kIdPV,
+                     (jp > 0 || kk > 0) ? 1u : 0u, 1u);
         }
         if (few_keys && jp < kPfSplitTiles) {   // lo parts: 16 columns after their hi parts
 #pragma unroll
-          for (int kk = 0; kk < kPfBN / 16; ++kk) {
-            const uint64_t vd = dvs + (uint64_t)(kk * 16 * 128 / 16);
-            const uint32_t pc = 32u * (kk >> 1) + 8u * (kk & 1) + 16u;
-            tc_mma_ts(tmem + kColO1, tmem + col_s(bp) + pc, vd, kIdPV, 1u);
-            tc_mma_ts(tmem + kColO2, tmem + col_a(bp) + pc, vd, kIdPV, 1u);
+          for (int kk = 0; kk < kPfBN / 16; kk += 2) {
+            const uint64_t vd0 = dvs + (uint64_t)(kk * 16 * 128 / 16), vd1 = vd0 + 16 * 128 / 16;
+            const uint32_t pc0 = 32u * (kk >> 1) + 16u, pc1 = pc0 + 8u;
+            tc_mma_ts4(tmem + kColO1, tmem + col_s(bp) + pc0, vd0, tmem + kColO2, tmem + col_a(bp) + pc0, vd0,
+                       tmem + kColO1, tmem + col_s(bp) + pc1, vd1, tmem + kColO2, tmem + col_a(bp) + pc1, vd1,
+                       kIdPV, 1u, 1u);
           }
         }
         tc_commit(&v_empty[sp]);
