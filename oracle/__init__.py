@@ -25,4 +25,7 @@ from .parallax_oracle import (  # noqa: F401
     prefill_paged_rows,
     prefill_grads,
     query_grads,
+    round_bf16,
+    project_heads,
+    decode_projected,
 )

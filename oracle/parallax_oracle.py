@@ -30,6 +30,13 @@ design notes):
     position t sees keys 0..t like any causal row.
   * Grouped-query attention: query head h reads KV head h // (Hq / Hkv).
   * An empty key set gives a zero output.
+  * The probe is a learned linear map of the layer input ("Parallax learns it
+    via a projection of the input", wispaper blog, "The Core Insight:
+    Covariance Correction"): rho_h = W_R^(h) x, and likewise q_h = W_Q^(h) x,
+    with no bias and no positional rotation (the pages name neither); row
+    n of a weight matrix is head n // d, component n % d.  Like every
+    activation of the bf16 path, q and rho are stored in bfloat16 (rounded to
+    nearest, ties to even) before attention reads them.
 """
 
 from __future__ import annotations
@@ -46,6 +53,9 @@ __all__ = [
     "prefill_paged_rows",
     "prefill_grads",
     "query_grads",
+    "round_bf16",
+    "project_heads",
+    "decode_projected",
 ]
 
 
@@ -278,3 +288,60 @@ def query_grads(q, rho, keys, values, dout, scale: float):
     out = vbar - torch.einsum("tde,td->te", sigma, R)
     (out * G).sum().backward()
     return Q.grad.numpy()[0], R.grad.numpy()[0], K.grad.numpy(), V.grad.numpy()
+
+
+# --------------------------------------------------------------- projection
+
+_BF16_MIN_ULP = 2.0 ** -133          # spacing of the subnormal bfloat16 values
+_BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
+
+
+def round_bf16(x) -> np.ndarray:
+    """float64 values rounded to the nearest bfloat16, ties to even, returned
+    as float64.
+
+    bfloat16 is float32 with 8 significant bits: a value with leading bit
+    2^(e-1) (``numpy.frexp`` gives x = m 2^e, 1/2 <= |m| < 1) has spacing
+    2^(e-8), never below the subnormal spacing 2^-133.  x / spacing is exact
+    in float64; ``numpy.round`` takes it to the nearest integer with ties to
+    even; magnitudes past the largest finite bfloat16 become infinite.
+    NaN stays NaN.
+    """
+    x = _f64(x)
+    _, e = np.frexp(x)
+    ulp = np.maximum(np.ldexp(1.0, e - 8), _BF16_MIN_ULP)
+    with np.errstate(invalid="ignore"):
+        y = np.round(x / ulp) * ulp
+        y = np.where(np.abs(y) > _BF16_MAX, np.copysign(np.inf, x), y)
+    return np.where(np.isfinite(x), y, x)
+
+
+def project_heads(x, weight, num_heads: int, head_dim: int) -> np.ndarray:
+    """Per-head linear projection of the layer input, in float64:
+    y[b, h, j] = sum_c weight[h * head_dim + j, c] * x[b, c].
+
+    x: [B, hidden]; weight: [num_heads * head_dim, hidden] (output feature
+    by input feature).  Returns float64 [B, num_heads, head_dim], unrounded.
+    """
+    x = _f64(x)
+    weight = _f64(weight)
+    assert weight.shape == (num_heads * head_dim, x.shape[1])
+    return (x @ weight.T).reshape(x.shape[0], num_heads, head_dim)
+
+
+def decode_projected(x, w_q, w_rho, k_cache, v_cache, scale: float, seq_lens=None,
+                     page_table=None, heads=None):
+    """Decode whose query and probe come from the new token's layer input:
+    q = bf16(W_Q x), rho = bf16(W_R x) per head (``project_heads`` then
+    ``round_bf16``), then ``decode``.
+
+    x: [B, hidden]; w_q, w_rho: [Hq * d, hidden]; caches as in ``decode``.
+    Returns (q, rho, out): the rounded projections [B, Hq, d] and the float64
+    output [B, Hq, d_v].
+    """
+    d = k_cache.shape[-1]
+    Hq = np.asarray(w_q).shape[0] // d
+    q = round_bf16(project_heads(x, w_q, Hq, d))
+    rho = round_bf16(project_heads(x, w_rho, Hq, d))
+    return q, rho, decode(q, rho, k_cache, v_cache, scale, seq_lens=seq_lens,
+                          page_table=page_table, heads=heads)

@@ -46,6 +46,7 @@ class DecodeWorkload:
     paged: bool = False
     min_len: int = 0              # paged: lengths uniform in [min_len, kv_len]
     seed: int = 0
+    hidden: int = 0               # > 0: q and rho are projected from a [B, hidden] input
 
     @property
     def scale(self) -> float:
@@ -95,6 +96,8 @@ class ChunkedPrefillWorkload:
 WORKLOADS = {
     "decode_f32": DecodeWorkload("decode_f32", 1, 1, 1, 64, 256, dtype="f32", seed=1),
     "decode_bf16": DecodeWorkload("decode_bf16", 8, 16, 8, 128, 4096, seed=2),
+    # decode_bf16's cache with q and rho projected from a model width of Hq * d
+    "decode_projected": DecodeWorkload("decode_projected", 8, 16, 8, 128, 4096, seed=2, hidden=2048),
     "decode_long": DecodeWorkload("decode_long", 64, 32, 8, 128, 32768, key_offset_std=0.5, seed=3),
     "decode_paged": DecodeWorkload("decode_paged", 128, 16, 4, 128, 65536, paged=True,
                                    min_len=512, seed=4),
@@ -197,6 +200,39 @@ def decode_inputs(w: DecodeWorkload, device="cpu", seed=None, nan_poison=True):
             _poison_paged_tails(k, v, lens, table)
     return dict(q=q, rho=rho, k_cache=k, v_cache=v, seq_lens=seq_lens,
                 page_table=page_table, scale=w.scale)
+
+
+def projection_inputs(batch, num_q_heads, head_dim, hidden, device="cpu", seed=0):
+    """Layer input and projection weights of a projected decode.
+
+    x [B, hidden] ~ N(0, 1); w_q, w_rho [Hq * d, hidden] ~ N(0, 1 / hidden)
+    (so every projected component has unit variance, like the q and rho
+    draws of the plain decode inputs); all rounded to bfloat16.  Drawn from
+    their own generator, seeded ``seed``, in the order x, w_q, w_rho.
+    """
+    gen = _gen(device, seed)
+    n = num_q_heads * head_dim
+    x = _normal((batch, hidden), gen, device, torch.bfloat16)
+    w_q = _normal((n, hidden), gen, device, torch.bfloat16, mul=hidden ** -0.5)
+    w_rho = _normal((n, hidden), gen, device, torch.bfloat16, mul=hidden ** -0.5)
+    return dict(x=x, w_q=w_q, w_rho=w_rho)
+
+
+def projected_decode_inputs(w: DecodeWorkload, device="cpu", seed=None):
+    """Inputs of one projected decode call: ``decode_inputs`` (its q and rho
+    unused) plus ``projection_inputs`` drawn with seed + 104729."""
+    seed = w.seed if seed is None else seed
+    inp = decode_inputs(w, device=device, seed=seed)
+    inp.update(projection_inputs(w.batch, w.num_q_heads, w.head_dim, w.hidden, device=device,
+                                 seed=seed + 104729))
+    return inp
+
+
+def projection_bytes(batch, num_q_heads, head_dim, hidden) -> int:
+    """Bytes a projected decode moves beyond the KV cache: both weight
+    matrices and x read once, q and rho written once (bf16)."""
+    n = num_q_heads * head_dim
+    return 2 * (2 * n * hidden + batch * hidden + 2 * batch * n)
 
 
 def _poison_paged_tails(k, v, lens, table, page_size=PAGE_SIZE):
