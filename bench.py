@@ -55,6 +55,8 @@ KERNEL_SOURCES = {
     "prefill": ["parallax_local_linear_b200/csrc/prefill.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
     "prefill_bwd": ["parallax_local_linear_b200/csrc/prefill_bwd.cuh", "parallax_local_linear_b200/csrc/prefill.cuh",
                     "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "decode_projected": ["parallax_local_linear_b200/csrc/project.cuh", "parallax_local_linear_b200/csrc/decode.cuh",
+                         "parallax_local_linear_b200/csrc/ptx.cuh"],
 }
 KV_COPIES = 4          # decode_bf16: 4 x 128 MiB of KV, more than L2
 GRAPH_STEPS = 64       # decode calls per captured graph
@@ -79,8 +81,8 @@ def parse_args(argv=None):
 
 
 def default_steps(workload):
-    return {"decode_f32": 20000, "decode_bf16": 8192, "decode_long": 200, "decode_paged": 200,
-            "prefill": 20, "prefill_paged": 20, "prefill_train": 10}[workload]
+    return {"decode_f32": 20000, "decode_bf16": 8192, "decode_projected": 8192, "decode_long": 200,
+            "decode_paged": 200, "prefill": 20, "prefill_paged": 20, "prefill_train": 10}[workload]
 
 
 def dist_env():
@@ -375,6 +377,138 @@ def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
                     "the KV cache stays resident on the device"}
 
 
+def bench_decode_projected(args, w, rank, world, dev, peaks, peaks_kind):
+    """Decode with q and rho projected from the layer input in the same call
+    (projection kernel, then the decode kernel with a programmatic dependency
+    on it).  The plain decode of the same projections is timed beside it."""
+    from parallax_local_linear_b200 import binding as px
+
+    copies = KV_COPIES
+    insts = [W.projected_decode_inputs(w, device=dev, seed=w.seed + 1000 * rank + i) for i in range(copies)]
+    B, Hq, d = w.batch, w.num_q_heads, w.head_dim
+    kv = W.kv_bytes(w)
+    proj = W.projection_bytes(B, Hq, d, w.hidden)
+    step_bytes = kv + proj
+    qo = [torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+    ro = [torch.empty_like(t) for t in qo]
+    outs = [torch.empty_like(t) for t in qo]
+
+    def step(i):
+        c = i % copies
+        x = insts[c]
+        px.decode_projected(x["x"], x["w_q"], x["w_rho"], x["k_cache"], x["v_cache"], x["scale"],
+                            q_out=qo[c], rho_out=ro[c], out=outs[c], num_ctas=args.num_ctas)
+
+    def plain(i):
+        c = i % copies
+        x = insts[c]
+        px.decode(qo[c], ro[c], x["k_cache"], x["v_cache"], x["scale"], out=outs[c], num_ctas=args.num_ctas)
+
+    ctas = px.decode_num_ctas(px.decode_params(qo[0], insts[0]["k_cache"], num_ctas=args.num_ctas))
+    stream = torch.cuda.current_stream()
+    for i in range(max(args.warmup, 3)):
+        step(i)
+        plain(i)
+    torch.cuda.synchronize()
+    assert px.last_device_error() == 0, "device error during warm-up"
+
+    K = args.steps
+    n = min(GRAPH_STEPS, K)
+
+    def capture(fn, count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(count):
+                fn(i)
+        return g
+
+    def timed(fn):
+        graphs = [(capture(fn, n), K // n)]
+        if K % n:
+            graphs.append((capture(fn, K % n), 1))
+        for gg, _ in graphs:
+            gg.replay()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        with ClockSampler(dev.index) as clk:
+            start.record(stream)
+            for gg, reps in graphs:
+                for _ in range(reps):
+                    gg.replay()
+            end.record(stream)
+            torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        return start.elapsed_time(end), clk
+
+    ms, clk = timed(step)
+    ms_plain, _ = timed(plain)
+    assert px.last_device_error() == 0, "device error during the timed steps"
+    ms_max, total_bytes = reduce_over_ranks(ms, step_bytes * K, dev, world)
+    gbs = total_bytes / (ms_max * 1e-3) / 1e9
+    achieved = step_bytes / (ms * 1e-3 / K) / 1e9
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+
+    # e2e: x from pinned host memory each step, output read back; cache and weights resident
+    x_host = [x["x"].cpu().pin_memory() for x in insts]
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    x_dev = [torch.empty_like(x["x"]) for x in insts]
+    Ke = min(K, 2048)
+
+    def one(i):
+        c = i % copies
+        x = insts[c]
+        x_dev[c].copy_(x_host[c], non_blocking=True)
+        px.decode_projected(x_dev[c], x["w_q"], x["w_rho"], x["k_cache"], x["v_cache"], x["scale"],
+                            q_out=qo[c], rho_out=ro[c], out=outs[c], num_ctas=args.num_ctas)
+        out_host[c].copy_(outs[c], non_blocking=True)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    t0 = time.perf_counter()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(Ke):
+        one(i)
+    end.record()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - t0
+    ms_e, tot_e = reduce_over_ranks(start.elapsed_time(end), step_bytes * Ke, dev, world)
+    e2e = {"value": round(tot_e / (ms_e * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": insts[0]["x"].numel() * 2, "d2h_bytes_per_step": outs[0].numel() * 2,
+           "steps": Ke, "ms_per_step": round(ms_e / Ke, 6), "host_wall_ms_per_step": round(1e3 * wall / Ke, 6),
+           "note": "the layer input copied from pinned host memory and the output read back every step; "
+                   "cache and weights stay resident on the device"}
+
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": profiled_traffic("decode_projected", w.name),
+                "peak_source": f"{peaks_kind} hbm_gbs",
+                "kernel": "project_qr_kernel + decode_tc_kernel (one call)",
+                "algorithmic_bytes_per_launch": int(step_bytes)}
+    cfg = dict(decode_config(w, args, ctas), hidden=w.hidden,
+               l2="each step reads one of %d copies of cache and weights (%.0f MiB total > 126 MB L2)"
+                  % (copies, copies * step_bytes / 2**20),
+               timing="CUDA-graph replay", bytes="K + V + W_Q + W_R + x read, q and rho written",
+               kv_bytes_per_step=int(kv), projection_bytes_per_step=int(proj),
+               plain_decode_ms_per_step=round(ms_plain / K, 6),
+               added_ms_per_step=round((ms - ms_plain) / K, 6))
+    res = {
+        "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / K, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "tokens_per_s": round(B * K * world / (ms_max * 1e-3), 1),
+        "pct_of_hbm_peak": round(100 * gbs / world / peak, 2),
+        "roofline": roofline, "e2e": e2e, "gpu_launches": 2 * K, "clocks": clk.summary(),
+    }
+    return res, insts
+
+
 # ----------------------------------------------------------------- prefill
 
 def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
@@ -624,6 +758,11 @@ def oracle_decode_sample(w, inp, budget_s, max_steps=None):
     rng.shuffle(units)
     q = inp["q"].double().cpu().numpy()
     rho = inp["rho"].double().cpu().numpy()
+    projected = w.hidden > 0
+    if projected:
+        x = inp["x"].double().cpu().numpy()
+        wq = _F64View(inp["w_q"])
+        wr = _F64View(inp["w_rho"])
     lens = None if inp["seq_lens"] is None else inp["seq_lens"].cpu().numpy()
     table = None if inp["page_table"] is None else inp["page_table"].cpu().numpy()
     done, secs, nbytes = 0, 0.0, 0
@@ -637,9 +776,16 @@ def oracle_decode_sample(w, inp, budget_s, max_steps=None):
             vc = V[None, None]
             heads = [(0, h) for h in range(g)]
             qq, rr = q[b:b + 1, kvh * g:(kvh + 1) * g], rho[b:b + 1, kvh * g:(kvh + 1) * g]
-            t0 = time.perf_counter()
-            oracle.decode(qq, rr, kc, vc, w.scale, heads=heads)
-            secs += time.perf_counter() - t0
+            if projected:
+                rows = slice(kvh * g * w.head_dim, (kvh + 1) * g * w.head_dim)
+                wqu, wru = wq[rows], wr[rows]
+                t0 = time.perf_counter()
+                oracle.decode_projected(x[b:b + 1], wqu, wru, kc, vc, w.scale, heads=heads)
+                secs += time.perf_counter() - t0
+            else:
+                t0 = time.perf_counter()
+                oracle.decode(qq, rr, kc, vc, w.scale, heads=heads)
+                secs += time.perf_counter() - t0
         else:
             kv = _F64View(inp["k_cache"])
             vv = _F64View(inp["v_cache"])
@@ -651,8 +797,13 @@ def oracle_decode_sample(w, inp, budget_s, max_steps=None):
         done += 1
         if secs >= budget_s or (max_steps and done >= max_steps):
             break
+    if projected:
+        # the workload's metric counts the weights once per step: credit the
+        # sample with the fraction of the step's projection bytes it covers
+        nbytes += W.projection_bytes(B, Hq, w.head_dim, w.hidden) * done // len(units)
+    what = "K+V, plus its share of the projection bytes" if projected else "K+V"
     desc = (f"{done} of {len(units)} (sequence, KV head) units of {w.name}, all {g} query heads each "
-            f"({nbytes / 2**20:.1f} MiB of K+V), float64 numpy oracle")
+            f"({nbytes / 2**20:.1f} MiB of {what}), float64 numpy oracle")
     return nbytes / secs / 1e9, secs, done, desc
 
 
@@ -757,6 +908,8 @@ def reference_arm(args, w, rank, world):
         inp = W.prefill_inputs(sub, device="cpu")
     elif w.name == "prefill_paged":
         inp = W.chunked_prefill_inputs(w, device="cpu")
+    elif w.hidden:
+        inp = W.projected_decode_inputs(w, device="cpu")
     elif w.batch * w.kv_len <= 2**20:
         inp = W.decode_inputs(w, device="cpu")
     else:
@@ -771,7 +924,7 @@ def reference_arm(args, w, rank, world):
         else:
             sub_w = w if inp["q"].shape[0] == w.batch else W.DecodeWorkload(
                 w.name, inp["q"].shape[0], w.num_q_heads, w.num_kv_heads, w.head_dim, w.kv_len,
-                dtype=w.dtype, paged=w.paged, min_len=w.min_len)
+                dtype=w.dtype, paged=w.paged, min_len=w.min_len, hidden=w.hidden)
             v, secs, _, desc = oracle_decode_sample(sub_w, inp, budget)
         if i >= args.warmup:
             vals.append(v)
@@ -833,6 +986,9 @@ def main(argv=None):
             res, inp = bench_prefill_paged(args, w, rank, world, dev, peaks, kind)
         elif w.name == "prefill_train":
             res, inp = bench_prefill_train(args, w, rank, world, dev, peaks, kind)
+        elif w.hidden:
+            res, inp = bench_decode_projected(args, w, rank, world, dev, peaks, kind)
+            inp = inp[0]
         else:
             res, inp = bench_decode(args, w, rank, world, dev, peaks, kind)
             inp = inp[0]

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define PARALLAX_ABI_VERSION 3
+#define PARALLAX_ABI_VERSION 4
 
 typedef enum plx_status {
   PLX_OK = 0,
@@ -125,6 +125,40 @@ plx_status parallax_decode(const void* q, const void* rho,
                            const int32_t* page_table, const int32_t* seq_lens,
                            void* out, void* workspace, size_t workspace_bytes,
                            const plx_decode_params* p, cudaStream_t stream);
+
+/* Decode whose query and probe are projected from the new token's layer
+ * input in the same call.
+ *
+ * Parallax learns the probe as a linear projection of the input (wispaper
+ * blog, "The Core Insight: Covariance Correction"; the newx.sg "Abstract"
+ * calls it an extra query-like projector).  For every sequence b and query
+ * head h, with d = head_dim and n = h*d + j:
+ *     q[b, h, j]   = bf16( sum_c w_q[n, c]   x[b, c] )
+ *     rho[b, h, j] = bf16( sum_c w_rho[n, c] x[b, c] )
+ * (fp32 sums, rounded to nearest even), then parallax_decode(q, rho, ...).
+ *
+ *   x            device bf16 [B, hidden]: the new token's layer input.
+ *   w_q, w_rho   device bf16 [Hq * d, hidden]: output feature by input
+ *                feature (row n belongs to head n / d, component n % d).
+ *   hidden       > 0 and a multiple of 32 (else PLX_ERR_UNSUPPORTED).
+ *   q, rho       device bf16 [B, Hq, d]: written with the projections, then
+ *                read by the decode.  They must not overlap x or the weights.
+ *   the rest     as parallax_decode; in_dtype must be PLX_BF16 (the cache
+ *                is bf16), else PLX_ERR_UNSUPPORTED.  Workspace size: as
+ *                parallax_decode_workspace_size().
+ *
+ * Two launches on `stream`: the projection kernel, then the decode kernel
+ * with a programmatic dependency on it, so that the decode's set-up and its
+ * first K/V loads overlap the projection; the decode reads q and rho only
+ * after the projection grid has completed.  Every check of parallax_decode
+ * runs before the first launch; if the second launch fails, q and rho are
+ * written and out is not (PLX_ERR_CUDA). */
+plx_status parallax_decode_projected(const void* x, const void* w_q, const void* w_rho, int32_t hidden,
+                                     const void* k_cache, const void* v_cache,
+                                     const int32_t* page_table, const int32_t* seq_lens,
+                                     void* q, void* rho, void* out,
+                                     void* workspace, size_t workspace_bytes,
+                                     const plx_decode_params* p, cudaStream_t stream);
 
 /* Decode that allocates nothing and takes no workspace.
  *

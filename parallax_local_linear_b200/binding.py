@@ -81,6 +81,9 @@ lib.parallax_prefill_backward_workspace_size.argtypes = [ctypes.POINTER(PrefillP
 lib.parallax_prefill_backward.restype = ctypes.c_int
 lib.parallax_prefill_backward.argtypes = [_vp] * 13 + [ctypes.c_size_t, ctypes.POINTER(PrefillParams), _vp]
 lib.parallax_decode_noalloc.restype = ctypes.c_int
+lib.parallax_decode_projected.argtypes = [_vp, _vp, _vp, ctypes.c_int32, _vp, _vp, _i32p, _i32p, _vp, _vp, _vp,
+                                          _vp, ctypes.c_size_t, ctypes.POINTER(DecodeParams), _vp]
+lib.parallax_decode_projected.restype = ctypes.c_int
 lib.parallax_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, ctypes.POINTER(DecodeParams), _vp]
 NOALLOC_SCRATCH_BYTES = 8 << 20
 lib.parallax_last_device_error.restype = ctypes.c_int
@@ -210,6 +213,59 @@ def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=No
     if st != 0:
         raise ParallaxError(st, "parallax_decode")
     return out
+
+
+def decode_projected(x, w_q, w_rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=None,
+                     q_out=None, rho_out=None, out=None, out_dtype=None, num_ctas=0, kv_len=None):
+    """Decode with q and rho projected from the new token's layer input in the
+    same call: q[b, h] = bf16(W_Q[h] x[b]), rho[b, h] = bf16(W_R[h] x[b]),
+    then ``decode``.
+
+    x: [B, hidden] bf16; w_q, w_rho: [Hq * d, hidden] bf16 (d = the cache's
+    head_dim); caches and options as in ``decode``.  Returns (out, q, rho):
+    out [B, Hq, d] in ``out_dtype`` (default bf16) and the projections
+    [B, Hq, d] bf16 (written into ``q_out`` / ``rho_out`` when given).
+    """
+    _check_cuda("x", x, torch.bfloat16)
+    for name, t in (("w_q", w_q), ("w_rho", w_rho), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_cuda(name, t, torch.bfloat16)
+    if x.dim() != 2 or w_q.dim() != 2 or w_q.shape != w_rho.shape or w_q.shape[1] != x.shape[1]:
+        raise ValueError("x must be [B, hidden] and w_q, w_rho [Hq * d, hidden]")
+    if k_cache.dim() != 4 or k_cache.shape != v_cache.shape:
+        raise ValueError("caches must be 4-D and alike")
+    d = k_cache.shape[-1]
+    if w_q.shape[0] % d:
+        raise ValueError("w_q rows must be a multiple of head_dim")
+    B, Hq = x.shape[0], w_q.shape[0] // d
+    if q_out is None:
+        q_out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=x.device)
+    if rho_out is None:
+        rho_out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=x.device)
+    for name, t in (("q_out", q_out), ("rho_out", rho_out)):
+        _check_cuda(name, t, torch.bfloat16)
+        if t.shape != (B, Hq, d):
+            raise ValueError(f"{name} must be [B, Hq, d] = {(B, Hq, d)}")
+    if page_table is not None:
+        _check_cuda("page_table", page_table, torch.int32)
+        if seq_lens is None:
+            raise ValueError("a paged cache needs seq_lens")
+    if seq_lens is not None:
+        _check_cuda("seq_lens", seq_lens, torch.int32)
+    p = decode_params(q_out, k_cache, page_table=page_table, kv_len=kv_len, scale=scale,
+                      out_dtype=out_dtype, num_ctas=num_ctas)
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=out_dtype or torch.bfloat16, device=x.device)
+    else:
+        _check_cuda("out", out)
+    nbytes = decode_workspace_size(p)
+    ws = _workspace(x.device, nbytes)
+    st = lib.parallax_decode_projected(_ptr(x), _ptr(w_q), _ptr(w_rho), int(x.shape[1]), _ptr(k_cache),
+                                       _ptr(v_cache), _ptr(page_table), _ptr(seq_lens), _ptr(q_out),
+                                       _ptr(rho_out), _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                                       ctypes.byref(p), _stream_ptr(x.device))
+    if st != 0:
+        raise ParallaxError(st, "parallax_decode_projected")
+    return out, q_out, rho_out
 
 
 def decode_noalloc(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=None, out, num_ctas=0,

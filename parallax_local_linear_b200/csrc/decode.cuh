@@ -417,6 +417,11 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     }
   } else {
     // ------------------------------------------------------------ consumers
+    // q and rho may come from the grid launched just before this one (the
+    // projection of a projected decode, with a programmatic dependency): wait
+    // for it to complete before reading them.  Without such a dependency the
+    // wait returns at once.  The producer warp streams K and V meanwhile.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int tid = threadIdx.x;
     constexpr int NT = NC * 32;
     auto bar = [] { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); };

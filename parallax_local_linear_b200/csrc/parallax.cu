@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "prefill_bwd.cuh"
+#include "project.cuh"
 
 namespace {
 
@@ -162,13 +163,16 @@ size_t decode_smem_bytes(const plx_decode_params* p) {
          table;
 }
 
+// `pdl`: launch with a programmatic dependency on the previous kernel in the
+// stream, which may then still be running when this grid starts (the
+// consumers wait for it before reading q and rho).
 template <int D, int STAGES, bool kLoInPad>
 plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int ctas,
-                            size_t smem, cudaStream_t stream) {
+                            size_t smem, cudaStream_t stream, bool pdl) {
   auto kern = decode_tc_kernel<D, STAGES, kDecodeNC, kLoInPad>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
-  if (a.cluster <= 1) {
+  if (a.cluster <= 1 && !pdl) {
     kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
     return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
   }
@@ -177,21 +181,34 @@ plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CU
   cfg.blockDim = dim3((kDecodeNC + 1) * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = a.cluster;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  const int cluster_attr = n;
+  if (a.cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = a.cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = n;
   if (cudaLaunchKernelEx(&cfg, kern, tk, tv, a) == cudaSuccess) return PLX_OK;
+  (void)cudaGetLastError();
+  if (a.cluster <= 1) return PLX_ERR_CUDA;
   // Clusters could not be scheduled (a launch-configuration error, which is
   // not sticky): run the same grid with the global-memory merge instead.
-  (void)cudaGetLastError();
   DecodeArgs b = a;
   b.cluster = 1;
-  kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, b);
-  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  cfg.numAttrs = cluster_attr;
+  if (cudaLaunchKernelEx(&cfg, kern, tk, tv, b) == cudaSuccess) return PLX_OK;
+  (void)cudaGetLastError();
+  return PLX_ERR_CUDA;
 }
 
 template <int D>
@@ -202,6 +219,119 @@ plx_status launch_decode_f32(const DecodeArgs& a, int ctas, size_t smem, cudaStr
   kern<<<ctas, kDecodeF32Warps * 32, smem, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
+
+// A validated decode call: kernel arguments, plan and tensor maps.
+struct DecodeLaunch {
+  DecodeArgs a;
+  DecodePlan pl;
+  size_t smem;
+  CUtensorMap tk, tv;   // bf16 path only
+  bool empty;           // every sequence is empty: the output is zero
+};
+
+// Validates a decode call and builds its kernel arguments and tensor maps;
+// launches nothing.
+plx_status prepare_decode(const void* q, const void* rho, const void* k_cache, const void* v_cache,
+                          const int32_t* page_table, const int32_t* seq_lens, void* out, void* workspace,
+                          size_t workspace_bytes, const plx_decode_params* p, DecodeLaunch* L) {
+  plx_status st = validate_decode(p);
+  if (st != PLX_OK) return st;
+  if (!q || !rho || !k_cache || !v_cache || !out) return PLX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
+    return PLX_ERR_INVALID_ARG;
+  const bool paged = p->page_size != 0;
+  if (paged && (page_table == nullptr || seq_lens == nullptr)) return PLX_ERR_INVALID_ARG;
+  if (!paged && page_table != nullptr) return PLX_ERR_INVALID_ARG;
+  if ((page_table && !aligned(page_table, 4)) || (seq_lens && !aligned(seq_lens, 4))) return PLX_ERR_INVALID_ARG;
+
+  const int num_sms = current_device_sms();
+  if (num_sms <= 0) return PLX_ERR_CUDA;
+  const DecodePlan pl = plan_decode(p, num_sms);
+  const size_t need = pl.counter_bytes + pl.slot_bytes;
+  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return PLX_ERR_WORKSPACE;
+
+  const int D = p->head_dim;
+  L->pl = pl;
+  L->empty = p->kv_len == 0;   // every sequence is empty: the output is zero
+  DecodeArgs& a = L->a;
+  a = DecodeArgs{};
+  a.q = q;
+  a.rho = rho;
+  a.k = k_cache;
+  a.v = v_cache;
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.out = out;
+  a.counters = reinterpret_cast<int32_t*>(workspace);
+  a.slots = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + pl.counter_bytes);
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.group = p->num_q_heads / p->num_kv_heads;
+  a.units_per_seq = pl.units_per_seq;
+  a.heads_per_unit = pl.heads_per_unit;
+  a.kv_len = p->kv_len;
+  a.paged = paged ? 1 : 0;
+  a.num_pages = paged ? p->num_pages : 0;
+  a.max_pages = paged ? p->max_pages_per_seq : 0;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
+
+  // Units of equal length cut into k pieces each (the unit-aligned grid) are
+  // merged through distributed shared memory when each unit is one cluster.
+  a.cluster = 1;
+  if (p->in_dtype == PLX_BF16 && !paged && seq_lens == nullptr && p->num_ctas == 0) {
+    const int64_t units = (int64_t)p->batch * p->num_kv_heads;
+    const int64_t k = pl.ctas / units;
+    const int64_t tiles_per_unit = (p->kv_len + kTile - 1) / kTile;
+    if (k >= 2 && k <= 1 + kMaxClusterRecv && k * units == pl.ctas && tiles_per_unit >= k) a.cluster = (int)k;
+  }
+  L->smem = decode_smem_bytes(p);
+  if (L->smem > 227 * 1024) return PLX_ERR_UNSUPPORTED;
+  if (L->empty || p->in_dtype == PLX_F32) return PLX_OK;
+  const uint64_t rows = paged ? (uint64_t)p->num_pages * p->num_kv_heads * kTile
+                              : (uint64_t)p->batch * p->num_kv_heads * p->kv_len;
+  if (!make_tmap_bf16(&L->tk, k_cache, D, rows, 64, kTile) || !make_tmap_bf16(&L->tv, v_cache, D, rows, 64, kTile))
+    return PLX_ERR_CUDA;
+  return PLX_OK;
+}
+
+plx_status launch_decode(const DecodeLaunch& L, const plx_decode_params* p, cudaStream_t stream, bool pdl) {
+  const DecodeArgs& a = L.a;
+  const int D = p->head_dim;
+  if (L.empty) {
+    const size_t elt = p->out_dtype == PLX_BF16 ? 2 : 4;
+    return cudaMemsetAsync(a.out, 0, (size_t)p->batch * p->num_q_heads * D * elt, stream) == cudaSuccess
+               ? PLX_OK
+               : PLX_ERR_CUDA;
+  }
+  if (p->in_dtype == PLX_F32)
+    return D == 64 ? launch_decode_f32<64>(a, L.pl.ctas, L.smem, stream)
+                   : launch_decode_f32<128>(a, L.pl.ctas, L.smem, stream);
+  const bool pad = a.group <= kMaxGroup / 2;
+  if (D == 64)
+    return pad ? launch_decode_tc<64, kDecodeStages64, true>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl)
+               : launch_decode_tc<64, kDecodeStages64, false>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl);
+  return pad ? launch_decode_tc<128, kDecodeStages128, true>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl)
+             : launch_decode_tc<128, kDecodeStages128, false>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl);
+}
+
+// q and rho projections of a projected decode (project.cuh).
+plx_status launch_project(const ProjArgs& pa, cudaStream_t stream) {
+  const int tiles = (pa.B + 7) / 8;
+  const int bt = tiles <= 1 ? 1 : tiles <= 2 ? 2 : tiles <= 4 ? 4 : kPjMaxTiles;
+  const dim3 grid(2 * pa.n1 / kPjRows, (pa.B + 8 * bt - 1) / (8 * bt));
+  const dim3 block(kPjWarps * 32);
+  switch (bt) {
+    case 1: project_qr_kernel<1, 8><<<grid, block, 0, stream>>>(pa); break;
+    case 2: project_qr_kernel<2, 4><<<grid, block, 0, stream>>>(pa); break;
+    case 4: project_qr_kernel<4, 4><<<grid, block, 0, stream>>>(pa); break;
+    default: project_qr_kernel<kPjMaxTiles, 2><<<grid, block, 0, stream>>>(pa); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+}
+
+
 
 // ----------------------------------------------------------------- prefill
 template <bool kPaged>
@@ -415,78 +545,39 @@ size_t parallax_decode_workspace_size(const plx_decode_params* p, int32_t num_sm
 plx_status parallax_decode(const void* q, const void* rho, const void* k_cache, const void* v_cache,
                            const int32_t* page_table, const int32_t* seq_lens, void* out, void* workspace,
                            size_t workspace_bytes, const plx_decode_params* p, cudaStream_t stream) {
+  DecodeLaunch L;
+  const plx_status st =
+      prepare_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, workspace, workspace_bytes, p, &L);
+  if (st != PLX_OK) return st;
+  return launch_decode(L, p, stream, false);
+}
+
+plx_status parallax_decode_projected(const void* x, const void* w_q, const void* w_rho, int32_t hidden,
+                                     const void* k_cache, const void* v_cache, const int32_t* page_table,
+                                     const int32_t* seq_lens, void* q, void* rho, void* out, void* workspace,
+                                     size_t workspace_bytes, const plx_decode_params* p, cudaStream_t stream) {
   plx_status st = validate_decode(p);
   if (st != PLX_OK) return st;
-  if (!q || !rho || !k_cache || !v_cache || !out) return PLX_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(rho, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16))
-    return PLX_ERR_INVALID_ARG;
-  const bool paged = p->page_size != 0;
-  if (paged && (page_table == nullptr || seq_lens == nullptr)) return PLX_ERR_INVALID_ARG;
-  if (!paged && page_table != nullptr) return PLX_ERR_INVALID_ARG;
-  if ((page_table && !aligned(page_table, 4)) || (seq_lens && !aligned(seq_lens, 4))) return PLX_ERR_INVALID_ARG;
-
-  const int num_sms = current_device_sms();
-  if (num_sms <= 0) return PLX_ERR_CUDA;
-  const DecodePlan pl = plan_decode(p, num_sms);
-  const size_t need = pl.counter_bytes + pl.slot_bytes;
-  if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256)) return PLX_ERR_WORKSPACE;
-
-  const int D = p->head_dim;
-  if (p->kv_len == 0) {
-    // Every sequence is empty: the output is zero.
-    const size_t elt = p->out_dtype == PLX_BF16 ? 2 : 4;
-    return cudaMemsetAsync(out, 0, (size_t)p->batch * p->num_q_heads * D * elt, stream) == cudaSuccess
-               ? PLX_OK
-               : PLX_ERR_CUDA;
-  }
-
-  DecodeArgs a{};
-  a.q = q;
-  a.rho = rho;
-  a.k = k_cache;
-  a.v = v_cache;
-  a.page_table = page_table;
-  a.seq_lens = seq_lens;
-  a.out = out;
-  a.counters = reinterpret_cast<int32_t*>(workspace);
-  a.slots = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + pl.counter_bytes);
-  a.B = p->batch;
-  a.Hq = p->num_q_heads;
-  a.Hkv = p->num_kv_heads;
-  a.group = p->num_q_heads / p->num_kv_heads;
-  a.units_per_seq = pl.units_per_seq;
-  a.heads_per_unit = pl.heads_per_unit;
-  a.kv_len = p->kv_len;
-  a.paged = paged ? 1 : 0;
-  a.num_pages = paged ? p->num_pages : 0;
-  a.max_pages = paged ? p->max_pages_per_seq : 0;
-  a.scale_log2 = p->scale * 1.4426950408889634f;
-  a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
-
-  // Units of equal length cut into k pieces each (the unit-aligned grid) are
-  // merged through distributed shared memory when each unit is one cluster.
-  a.cluster = 1;
-  if (p->in_dtype == PLX_BF16 && !paged && seq_lens == nullptr && p->num_ctas == 0) {
-    const int64_t units = (int64_t)p->batch * p->num_kv_heads;
-    const int64_t k = pl.ctas / units;
-    const int64_t tiles_per_unit = (p->kv_len + kTile - 1) / kTile;
-    if (k >= 2 && k <= 1 + kMaxClusterRecv && k * units == pl.ctas && tiles_per_unit >= k) a.cluster = (int)k;
-  }
-  const size_t smem = decode_smem_bytes(p);
-  if (smem > 227 * 1024) return PLX_ERR_UNSUPPORTED;
-  if (p->in_dtype == PLX_F32)
-    return D == 64 ? launch_decode_f32<64>(a, pl.ctas, smem, stream) : launch_decode_f32<128>(a, pl.ctas, smem, stream);
-  const uint64_t rows = paged ? (uint64_t)p->num_pages * p->num_kv_heads * kTile
-                              : (uint64_t)p->batch * p->num_kv_heads * p->kv_len;
-  CUtensorMap tk, tv;
-  if (!make_tmap_bf16(&tk, k_cache, D, rows, 64, kTile) || !make_tmap_bf16(&tv, v_cache, D, rows, 64, kTile))
-    return PLX_ERR_CUDA;
-  const bool pad = a.group <= kMaxGroup / 2;
-  if (D == 64)
-    return pad ? launch_decode_tc<64, kDecodeStages64, true>(a, tk, tv, pl.ctas, smem, stream)
-               : launch_decode_tc<64, kDecodeStages64, false>(a, tk, tv, pl.ctas, smem, stream);
-  return pad ? launch_decode_tc<128, kDecodeStages128, true>(a, tk, tv, pl.ctas, smem, stream)
-             : launch_decode_tc<128, kDecodeStages128, false>(a, tk, tv, pl.ctas, smem, stream);
+  if (!x || !w_q || !w_rho || hidden <= 0) return PLX_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_q, 16) || !aligned(w_rho, 16)) return PLX_ERR_INVALID_ARG;
+  if (p->in_dtype != PLX_BF16 || hidden % 32 != 0) return PLX_ERR_UNSUPPORTED;
+  const int64_t n1 = (int64_t)p->num_q_heads * p->head_dim;
+  if (2 * n1 > (int64_t)INT32_MAX) return PLX_ERR_UNSUPPORTED;
+  DecodeLaunch L;
+  if ((st = prepare_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, workspace, workspace_bytes, p,
+                           &L)) != PLX_OK)
+    return st;
+  ProjArgs pa{};
+  pa.x = static_cast<const __nv_bfloat16*>(x);
+  pa.wq = static_cast<const __nv_bfloat16*>(w_q);
+  pa.wr = static_cast<const __nv_bfloat16*>(w_rho);
+  pa.q = static_cast<__nv_bfloat16*>(q);
+  pa.rho = static_cast<__nv_bfloat16*>(rho);
+  pa.B = p->batch;
+  pa.n1 = (int)n1;
+  pa.hidden = hidden;
+  if ((st = launch_project(pa, stream)) != PLX_OK) return st;
+  return launch_decode(L, p, stream, true);
 }
 
 plx_status parallax_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,

@@ -31,7 +31,8 @@ def binding():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for must in ("parallax_decode", "parallax_prefill", "parallax_prefill_paged", "parallax_decode_workspace_size",
+    for must in ("parallax_decode", "parallax_decode_projected", "parallax_prefill", "parallax_prefill_paged",
+                 "parallax_decode_workspace_size",
                  "parallax_last_device_error", "parallax_status_string"):
         assert must in names
 
@@ -43,7 +44,7 @@ def test_library_exports_every_declared_symbol(binding):
 
 
 def test_abi_version_and_status_strings(binding):
-    assert binding.lib.parallax_abi_version() == 3
+    assert binding.lib.parallax_abi_version() == 4
     for code, name in binding.STATUS.items():
         assert binding.lib.parallax_status_string(code).decode() == name
 
@@ -93,6 +94,27 @@ def test_null_and_misaligned_pointers_rejected_before_launch(binding):
     pp = _params(binding, page_size=64, num_pages=4, max_pages_per_seq=64)
     st = binding.lib.parallax_decode(al, al, al, al, None, None, al, None, 0, ctypes.byref(pp), None)
     assert st == 1   # paged without a page table / seq_lens
+
+
+def test_projected_decode_rejects_bad_arguments_before_launch(binding):
+    buf = ctypes.create_string_buffer(256)
+    addr = ctypes.addressof(buf)
+    al = ctypes.c_void_p((addr + 15) & ~15)
+    odd = ctypes.c_void_p(((addr + 15) & ~15) + 2)
+    p = _params(binding)
+
+    def call(x=al, wq=al, wr=al, hidden=2048, params=p):
+        return binding.lib.parallax_decode_projected(x, wq, wr, hidden, al, al, None, None, al, al, al, None, 0,
+                                                     ctypes.byref(params), None)
+
+    assert call(params=_params(binding, batch=0)) == 1          # decode parameters checked first
+    assert call(x=None) == 1
+    assert call(wr=None) == 1
+    assert call(wq=odd) == 1
+    assert call(hidden=0) == 1
+    assert call(hidden=-32) == 1
+    assert call(hidden=48) == 2                                 # not a multiple of 32
+    assert call(params=_params(binding, in_dtype=0, out_dtype=0)) == 2   # fp32 cache
 
 
 @pytest.mark.parametrize("bad", [dict(seq_len=0), dict(head_dim=64), dict(in_dtype=0), dict(causal=2),
