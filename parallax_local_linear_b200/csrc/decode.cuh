@@ -325,6 +325,13 @@ constexpr int tc_smem_fixed_bytes() {
          (1 + kMaxClusterRecv) * (int)sizeof(CtaState<D>) + 2 * STAGES * 8 + 16 + (NC + 1) * 32 * 4 + 1024;
 }
 
+// 16-byte store to distributed shared memory (a shared::cluster address).
+__device__ __forceinline__ void dsmem_st_v4(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
+}
+
 template <int D, int STAGES, int NC, bool kLoInPad>
 __global__ void __launch_bounds__((NC + 1) * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
@@ -669,12 +676,17 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     const int b = unit / a.Hkv, kvh = unit % a.Hkv, hq0 = kvh * g;
     cluster_wait();   // every CTA of the cluster has started
     if (rank > 0) {
+      // m, l, c of every head slot, then the O1 and O2 rows of the g live
+      // heads, in 16-byte stores (the states are 16-byte aligned: the ring
+      // is, and every block before them is a multiple of 16 bytes)
       const uint32_t remote = dsmem_map(smem_u32(&recv[rank - 1]), 0);
-      const float* src = reinterpret_cast<const float*>(&st);
-      constexpr int kFloats = (int)(sizeof(CtaState<D>) / 4);
-      for (int i = threadIdx.x; i < kFloats; i += blockDim.x) {
-        // only the live heads' rows matter, but the state is small: copy it whole
-        dsmem_st_f32(remote + 4u * i, src[i]);
+      const float4* src = reinterpret_cast<const float4*>(&st);
+      constexpr int kHead = 3 * kMaxGroup / 4;             // m, l, c
+      constexpr int kO2 = (3 * kMaxGroup + kMaxGroup * D) / 4;
+      const int live = g * D / 4;
+      for (int i = threadIdx.x; i < kHead + 2 * live; i += blockDim.x) {
+        const int v = i < kHead + live ? i : kO2 + (i - kHead - live);
+        dsmem_st_v4(remote + 16u * v, src[v]);
       }
     }
     cluster_sync();
