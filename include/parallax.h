@@ -142,7 +142,8 @@ plx_status parallax_decode(const void* q, const void* rho,
  *                feature (row n belongs to head n / d, component n % d).
  *   hidden       > 0 and a multiple of 32 (else PLX_ERR_UNSUPPORTED).
  *   q, rho       device bf16 [B, Hq, d]: written with the projections, then
- *                read by the decode.  They must not overlap x or the weights.
+ *                read by the decode.  Neither may overlap x, the weights or
+ *                the other (PLX_ERR_INVALID_ARG); out may be q itself.
  *   the rest     as parallax_decode; in_dtype must be PLX_BF16 (the cache
  *                is bf16), else PLX_ERR_UNSUPPORTED.  Workspace size: as
  *                parallax_decode_workspace_size().

@@ -44,6 +44,12 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Do the byte ranges [a, a + na) and [b, b + nb) share a byte?
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
 int current_device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return -1;
@@ -563,6 +569,17 @@ plx_status parallax_decode_projected(const void* x, const void* w_q, const void*
   if (p->in_dtype != PLX_BF16 || hidden % 32 != 0) return PLX_ERR_UNSUPPORTED;
   const int64_t n1 = (int64_t)p->num_q_heads * p->head_dim;
   if (2 * n1 > (int64_t)INT32_MAX) return PLX_ERR_UNSUPPORTED;
+  // The projection writes q and rho while other CTAs still read x and the
+  // weights: the outputs must not overlap the inputs or each other.
+  const size_t qr_bytes = (size_t)p->batch * n1 * 2, x_bytes = (size_t)p->batch * hidden * 2,
+               w_bytes = (size_t)n1 * hidden * 2;
+  for (const void* o : {q, rho}) {
+    if (o == nullptr) return PLX_ERR_INVALID_ARG;
+    if (overlaps(o, qr_bytes, x, x_bytes) || overlaps(o, qr_bytes, w_q, w_bytes) ||
+        overlaps(o, qr_bytes, w_rho, w_bytes))
+      return PLX_ERR_INVALID_ARG;
+  }
+  if (overlaps(q, qr_bytes, rho, qr_bytes)) return PLX_ERR_INVALID_ARG;
   DecodeLaunch L;
   if ((st = prepare_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, workspace, workspace_bytes, p,
                            &L)) != PLX_OK)

@@ -117,6 +117,28 @@ def test_projected_decode_rejects_bad_arguments_before_launch(binding):
     assert call(params=_params(binding, in_dtype=0, out_dtype=0)) == 2   # fp32 cache
 
 
+def test_projected_decode_rejects_overlapping_outputs_before_launch(binding):
+    # Fake, 16-byte aligned device addresses: the overlap checks run on the
+    # host before any CUDA call.  B=8, Hq*d=2048, hidden=2048: q and rho are
+    # 32 KiB each, x 32 KiB, each weight 8 MiB.
+    p = _params(binding)
+    X, WQ, WR = 1 << 32, 2 << 32, 3 << 32
+    Q, R, OUT = 4 << 32, 5 << 32, 6 << 32
+    V = ctypes.c_void_p
+
+    def call(q=Q, r=R, x=X, wq=WQ, wr=WR):
+        return binding.lib.parallax_decode_projected(V(x), V(wq), V(wr), 2048, V(7 << 32), V(8 << 32), None, None,
+                                                     V(q), V(r), V(OUT), None, 0, ctypes.byref(p), None)
+
+    # disjoint buffers pass these checks and fail later: no device (CPU) or no workspace (GPU)
+    assert call() in (3, 4)
+    assert call(q=X + 16) == 1                 # q inside x
+    assert call(r=WQ + (8 << 20) - 16) == 1    # rho straddles the end of w_q
+    assert call(q=WR) == 1                     # q on w_rho
+    assert call(r=Q + 32768 - 16) == 1         # rho overlaps q
+    assert call(q=None) == 1
+
+
 @pytest.mark.parametrize("bad", [dict(seq_len=0), dict(head_dim=64), dict(in_dtype=0), dict(causal=2),
                                  dict(num_heads=6, num_kv_heads=4), dict(scale=-0.1), dict(scale=0.0)])
 def test_invalid_prefill_params_are_rejected(binding, bad):
