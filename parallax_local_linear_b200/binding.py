@@ -123,6 +123,37 @@ def _check_cuda(name, t, dtype=None):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def _check_sequences(batch, seq_lens, page_table):
+    """seq_lens [B] int32 and page_table [B, max_pages] int32 on the device
+    (either may be None): the kernels read one entry / row per sequence."""
+    if seq_lens is not None and tuple(seq_lens.shape) != (batch,):
+        raise ValueError(f"seq_lens must have shape ({batch},), got {tuple(seq_lens.shape)}")
+    if page_table is not None:
+        if page_table.dim() != 2 or page_table.shape[0] != batch:
+            raise ValueError(f"page_table must be [{batch}, max_pages], got {tuple(page_table.shape)}")
+        if seq_lens is None:
+            raise ValueError("a paged cache needs seq_lens")
+        _check_cuda("page_table", page_table, torch.int32)
+    if seq_lens is not None:
+        _check_cuda("seq_lens", seq_lens, torch.int32)
+
+
+def _output(out, out_dtype, shape, default_dtype, device):
+    """The call's output tensor and dtype.  A caller's ``out`` must have
+    ``shape`` (the kernels write every element of it) and, when
+    ``out_dtype`` is given, that dtype; otherwise its own dtype is the
+    output dtype.  Without ``out`` a new tensor is allocated."""
+    if out is None:
+        dt = out_dtype or default_dtype
+        return torch.empty(tuple(shape), dtype=dt, device=device), dt
+    if tuple(out.shape) != tuple(shape):
+        raise ValueError(f"out must have shape {tuple(shape)}, got {tuple(out.shape)}")
+    if out_dtype is not None and out.dtype != out_dtype:
+        raise TypeError(f"out is {out.dtype} but out_dtype is {out_dtype}")
+    _check_cuda("out", out)
+    return out, out.dtype
+
+
 _ws_lock = threading.Lock()
 _workspaces = {}
 
@@ -193,18 +224,10 @@ def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=No
         raise ValueError("shape mismatch between q/rho or k_cache/v_cache")
     if k_cache.dim() != 4 or k_cache.shape[-1] != q.shape[-1]:
         raise ValueError("caches must be 4-D with the head_dim of q")
-    if page_table is not None:
-        _check_cuda("page_table", page_table, torch.int32)
-        if seq_lens is None:
-            raise ValueError("a paged cache needs seq_lens")
-    if seq_lens is not None:
-        _check_cuda("seq_lens", seq_lens, torch.int32)
+    _check_sequences(q.shape[0], seq_lens, page_table)
+    out, out_dtype = _output(out, out_dtype, q.shape, q.dtype, q.device)
     p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale,
                       out_dtype=out_dtype, num_ctas=num_ctas)
-    if out is None:
-        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
-    else:
-        _check_cuda("out", out)
     nbytes = decode_workspace_size(p)
     ws = _workspace(q.device, nbytes)
     st = lib.parallax_decode(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
@@ -245,18 +268,10 @@ def decode_projected(x, w_q, w_rho, k_cache, v_cache, scale=None, *, seq_lens=No
         _check_cuda(name, t, torch.bfloat16)
         if t.shape != (B, Hq, d):
             raise ValueError(f"{name} must be [B, Hq, d] = {(B, Hq, d)}")
-    if page_table is not None:
-        _check_cuda("page_table", page_table, torch.int32)
-        if seq_lens is None:
-            raise ValueError("a paged cache needs seq_lens")
-    if seq_lens is not None:
-        _check_cuda("seq_lens", seq_lens, torch.int32)
+    _check_sequences(B, seq_lens, page_table)
+    out, out_dtype = _output(out, out_dtype, (B, Hq, d), torch.bfloat16, x.device)
     p = decode_params(q_out, k_cache, page_table=page_table, kv_len=kv_len, scale=scale,
                       out_dtype=out_dtype, num_ctas=num_ctas)
-    if out is None:
-        out = torch.empty((B, Hq, d), dtype=out_dtype or torch.bfloat16, device=x.device)
-    else:
-        _check_cuda("out", out)
     nbytes = decode_workspace_size(p)
     ws = _workspace(x.device, nbytes)
     st = lib.parallax_decode_projected(_ptr(x), _ptr(w_q), _ptr(w_rho), int(x.shape[1]), _ptr(k_cache),
@@ -277,8 +292,15 @@ def decode_noalloc(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_
     holds the split partials.  Calls that overlap on the GPU race.
     """
     _check_cuda("q", q)
-    _check_cuda("out", out)
-    p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale, out_dtype=out.dtype,
+    for name, t in (("rho", rho), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_cuda(name, t, q.dtype)
+    if rho.shape != q.shape or k_cache.shape != v_cache.shape:
+        raise ValueError("shape mismatch between q/rho or k_cache/v_cache")
+    _check_sequences(q.shape[0], seq_lens, page_table)
+    if out is None:
+        raise ValueError("decode_noalloc needs out")
+    out, out_dtype = _output(out, None, q.shape, q.dtype, q.device)
+    p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale, out_dtype=out_dtype,
                       num_ctas=num_ctas)
     st = lib.parallax_decode_noalloc(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
                                      _ptr(seq_lens), _ptr(out), ctypes.byref(p), _stream_ptr(q.device))
@@ -295,11 +317,7 @@ def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):
     B, H, T, d = q.shape
     if rho.shape != q.shape or k.shape != v.shape or k.shape[0] != B or k.shape[2] != T or k.shape[3] != d:
         raise ValueError("shape mismatch")
-    out_dtype = out_dtype or (out.dtype if out is not None else q.dtype)
-    if out is None:
-        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
-    else:
-        _check_cuda("out", out, out_dtype)
+    out, out_dtype = _output(out, out_dtype, q.shape, q.dtype, q.device)
     scale = (1.0 / d ** 0.5) if scale is None else float(scale)
     p = PrefillParams(B, H, k.shape[1], T, d, PLX_BF16, _dtype_code(out_dtype), scale, 1 if causal else 0)
     st = lib.parallax_prefill(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(p),
@@ -354,6 +372,11 @@ def prefill_backward(q, rho, k, v, out, vbar, stats, dout, causal=True, scale=No
     _check_cuda("out", out, out.dtype)
     _check_cuda("vbar", vbar, torch.float32)
     _check_cuda("stats", stats, torch.float32)
+    rows = tuple(q.shape[:3])
+    for name, t, shape in (("dout", dout, q.shape), ("out", out, q.shape), ("vbar", vbar, q.shape),
+                           ("stats", stats, rows + (2,))):
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
     grad_dtype = grad_dtype or out.dtype
     if grad_dtype != out.dtype:
         raise ValueError("gradients are returned in out's dtype")
@@ -412,13 +435,7 @@ def prefill_paged(q, rho, k_cache, v_cache, page_table, cu_seqlens_q, seq_lens, 
     if (rho.shape != q.shape or v_cache.shape != k_cache.shape or dk != d or page_table.dim() != 2
             or page_table.shape[0] != B or cu_seqlens_q.shape != (B + 1,)):
         raise ValueError("shape mismatch")
-    out_dtype = out_dtype or (out.dtype if out is not None else q.dtype)
-    if out is None:
-        out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
-    else:
-        _check_cuda("out", out, out_dtype)
-        if out.shape != q.shape:
-            raise ValueError("out shape mismatch")
+    out, out_dtype = _output(out, out_dtype, q.shape, q.dtype, q.device)
     scale = (1.0 / d ** 0.5) if scale is None else float(scale)
     p = PrefillPagedParams(B, H, Hkv, d, total_q, int(max_q_len), ps, P, page_table.shape[1], PLX_BF16,
                            _dtype_code(out_dtype), scale, 1 if causal else 0)

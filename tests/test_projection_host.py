@@ -61,3 +61,33 @@ def test_oracle_leg_counts_the_projection_once_per_step():
     want = (W.kv_bytes(w) + W.projection_bytes(w.batch, w.num_q_heads, w.head_dim, w.hidden)) / secs / 1e9
     assert np.isclose(gbs, want, rtol=1e-9)
     assert "projection" in desc
+
+
+# --------------------------------------------------------------------------
+# Binding checks of caller buffers (host logic; the CUDA check comes last)
+# --------------------------------------------------------------------------
+
+def test_output_buffer_shape_and_dtype_are_checked_before_any_launch():
+    from parallax_local_linear_b200 import binding as px
+    with pytest.raises(ValueError, match="shape"):
+        px._output(torch.empty(2, 3, 4), None, (2, 3, 5), torch.bfloat16, "cpu")
+    with pytest.raises(TypeError, match="out_dtype"):
+        px._output(torch.empty(2, 3, 4), torch.bfloat16, (2, 3, 4), torch.bfloat16, "cpu")
+    with pytest.raises(ValueError, match="CUDA"):   # right shape and dtype: only the device is wrong
+        px._output(torch.empty(2, 3, 4), None, (2, 3, 4), torch.bfloat16, "cpu")
+    out, dt = px._output(None, None, (2, 3), torch.float32, "cpu")
+    assert out.shape == (2, 3) and dt == torch.float32
+
+
+def test_sequence_tables_are_checked_against_the_batch():
+    from parallax_local_linear_b200 import binding as px
+    lens = torch.zeros(3, dtype=torch.int32)
+    table = torch.zeros(3, 5, dtype=torch.int32)
+    with pytest.raises(ValueError, match="seq_lens must have shape"):
+        px._check_sequences(4, lens, None)
+    with pytest.raises(ValueError, match="page_table must be"):
+        px._check_sequences(4, torch.zeros(4, dtype=torch.int32), table)
+    with pytest.raises(ValueError, match="needs seq_lens"):
+        px._check_sequences(3, None, table)
+    with pytest.raises(ValueError, match="CUDA"):
+        px._check_sequences(3, lens, table)
