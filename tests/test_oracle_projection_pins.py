@@ -199,3 +199,18 @@ def test_projection_pins_catch_planted_mistakes(name, mutant, monkeypatch):
                 assert oracle.round_bf16(np.array([x]))[0] == want
     else:
         assert caught > 0
+
+
+def test_decode_projected_paged_equals_contiguous():
+    # the same logical cache stored in pages placed by a permutation
+    from parallax_local_linear_b200 import workloads as W
+    inp = W.small_decode_inputs(3, 4, 2, 64, 150, seq_lens=[150, 1, 77], paged=True, seed=12,
+                                nan_poison=True)
+    pj = W.projection_inputs(3, 4, 64, 96, seed=13)
+    args = [pj[k].double().numpy() for k in ("x", "w_q", "w_rho")]
+    lens = inp["seq_lens"].numpy()
+    _, _, paged = oracle.decode_projected(*args, inp["k_cache"].double().numpy(), inp["v_cache"].double().numpy(),
+                                          inp["scale"], seq_lens=lens, page_table=inp["page_table"].numpy())
+    _, _, contig = oracle.decode_projected(*args, inp["k_contig"].double().numpy(),
+                                           inp["v_contig"].double().numpy(), inp["scale"], seq_lens=lens)
+    np.testing.assert_array_equal(paged, contig)
