@@ -138,6 +138,51 @@ def _check_sequences(batch, seq_lens, page_table):
         _check_cuda("seq_lens", seq_lens, torch.int32)
 
 
+def _check_cache_layout(batch, num_q_heads, head_dim, k_cache, v_cache, seq_lens, page_table, kv_len):
+    """Shape checks of a decode's cache and sequence tables (host-only, so
+    they run before any device check): the library reads the caches through
+    these shapes, so a mismatch would read outside them."""
+    if k_cache.dim() != 4 or tuple(k_cache.shape) != tuple(v_cache.shape):
+        raise ValueError(f"k_cache and v_cache must be 4-D and alike, got {tuple(k_cache.shape)} "
+                         f"and {tuple(v_cache.shape)}")
+    if k_cache.shape[-1] != head_dim:
+        raise ValueError(f"the caches' head_dim {k_cache.shape[-1]} differs from the queries' {head_dim}")
+    if k_cache.shape[1] < 1 or num_q_heads % k_cache.shape[1]:
+        raise ValueError(f"{num_q_heads} query heads do not split into {k_cache.shape[1]} KV heads")
+    if page_table is None:
+        if k_cache.shape[0] != batch:
+            raise ValueError(f"a contiguous cache holds one sequence per row: {k_cache.shape[0]} != {batch}")
+        # The library addresses token t of (b, kv head) as row (b * Hkv + kvh) * kv_len + t,
+        # so kv_len must be the cache's own row count; seq_lens limits each sequence.
+        if kv_len is not None and int(kv_len) != k_cache.shape[2]:
+            raise ValueError(f"kv_len {kv_len} must equal the contiguous cache's length {k_cache.shape[2]} "
+                             "(use seq_lens for shorter sequences)")
+    else:
+        if k_cache.shape[2] != PAGE_SIZE:
+            raise ValueError(f"paged caches hold {PAGE_SIZE}-token pages: got {tuple(k_cache.shape)}")
+        if page_table.dim() == 2 and kv_len is not None and int(kv_len) > page_table.shape[1] * PAGE_SIZE:
+            raise ValueError(f"kv_len {kv_len} exceeds the page table's {page_table.shape[1]} pages")
+    if seq_lens is not None and tuple(seq_lens.shape) != (batch,):
+        raise ValueError(f"seq_lens must have shape ({batch},), got {tuple(seq_lens.shape)}")
+    if page_table is not None:
+        if page_table.dim() != 2 or page_table.shape[0] != batch:
+            raise ValueError(f"page_table must be [{batch}, max_pages], got {tuple(page_table.shape)}")
+        if seq_lens is None:
+            raise ValueError("a paged cache needs seq_lens")
+
+
+def _check_decode_inputs(q, rho, k_cache, v_cache, seq_lens, page_table, kv_len):
+    """Every check of a decode call's inputs: shapes first, then devices and dtypes."""
+    if q.dim() != 3 or tuple(rho.shape) != tuple(q.shape):
+        raise ValueError(f"q and rho must be [B, Hq, d] and alike, got {tuple(q.shape)} and {tuple(rho.shape)}")
+    B, Hq, d = q.shape
+    _check_cache_layout(B, Hq, d, k_cache, v_cache, seq_lens, page_table, kv_len)
+    _check_cuda("q", q)
+    for name, t in (("rho", rho), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_cuda(name, t, q.dtype)
+    _check_sequences(B, seq_lens, page_table)
+
+
 def _output(out, out_dtype, shape, default_dtype, device):
     """The call's output tensor and dtype.  A caller's ``out`` must have
     ``shape`` (the kernels write every element of it) and, when
@@ -217,14 +262,7 @@ def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=No
     with ``page_table`` (int32 [B, max_pages]) and ``seq_lens`` (required).
     Returns out [B, Hq, d] in ``out_dtype`` (default: the input dtype).
     """
-    _check_cuda("q", q)
-    for name, t in (("rho", rho), ("k_cache", k_cache), ("v_cache", v_cache)):
-        _check_cuda(name, t, q.dtype)
-    if rho.shape != q.shape or k_cache.shape != v_cache.shape:
-        raise ValueError("shape mismatch between q/rho or k_cache/v_cache")
-    if k_cache.dim() != 4 or k_cache.shape[-1] != q.shape[-1]:
-        raise ValueError("caches must be 4-D with the head_dim of q")
-    _check_sequences(q.shape[0], seq_lens, page_table)
+    _check_decode_inputs(q, rho, k_cache, v_cache, seq_lens, page_table, kv_len)
     out, out_dtype = _output(out, out_dtype, q.shape, q.dtype, q.device)
     p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale,
                       out_dtype=out_dtype, num_ctas=num_ctas)
@@ -249,9 +287,6 @@ def decode_projected(x, w_q, w_rho, k_cache, v_cache, scale=None, *, seq_lens=No
     out [B, Hq, d] in ``out_dtype`` (default bf16) and the projections
     [B, Hq, d] bf16 (written into ``q_out`` / ``rho_out`` when given).
     """
-    _check_cuda("x", x, torch.bfloat16)
-    for name, t in (("w_q", w_q), ("w_rho", w_rho), ("k_cache", k_cache), ("v_cache", v_cache)):
-        _check_cuda(name, t, torch.bfloat16)
     if x.dim() != 2 or w_q.dim() != 2 or w_q.shape != w_rho.shape or w_q.shape[1] != x.shape[1]:
         raise ValueError("x must be [B, hidden] and w_q, w_rho [Hq * d, hidden]")
     if k_cache.dim() != 4 or k_cache.shape != v_cache.shape:
@@ -260,6 +295,10 @@ def decode_projected(x, w_q, w_rho, k_cache, v_cache, scale=None, *, seq_lens=No
     if w_q.shape[0] % d:
         raise ValueError("w_q rows must be a multiple of head_dim")
     B, Hq = x.shape[0], w_q.shape[0] // d
+    _check_cache_layout(B, Hq, d, k_cache, v_cache, seq_lens, page_table, kv_len)
+    _check_cuda("x", x, torch.bfloat16)
+    for name, t in (("w_q", w_q), ("w_rho", w_rho), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _check_cuda(name, t, torch.bfloat16)
     if q_out is None:
         q_out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=x.device)
     if rho_out is None:
@@ -291,12 +330,7 @@ def decode_noalloc(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_
     and the library's fixed device scratch (NOALLOC_SCRATCH_BYTES per GPU)
     holds the split partials.  Calls that overlap on the GPU race.
     """
-    _check_cuda("q", q)
-    for name, t in (("rho", rho), ("k_cache", k_cache), ("v_cache", v_cache)):
-        _check_cuda(name, t, q.dtype)
-    if rho.shape != q.shape or k_cache.shape != v_cache.shape:
-        raise ValueError("shape mismatch between q/rho or k_cache/v_cache")
-    _check_sequences(q.shape[0], seq_lens, page_table)
+    _check_decode_inputs(q, rho, k_cache, v_cache, seq_lens, page_table, kv_len)
     if out is None:
         raise ValueError("decode_noalloc needs out")
     out, out_dtype = _output(out, None, q.shape, q.dtype, q.device)

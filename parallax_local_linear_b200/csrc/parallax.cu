@@ -688,11 +688,14 @@ plx_status parallax_decode_noalloc(const void* q, const void* rho, const void* k
   if (pl.counter_bytes + pl.slot_bytes > (size_t)PARALLAX_NOALLOC_SCRATCH_BYTES) return PLX_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch)) != PLX_OK) return st;
+  // Every check runs before anything is queued on the stream.
+  DecodeLaunch L;
+  if ((st = prepare_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, scratch,
+                           (size_t)PARALLAX_NOALLOC_SCRATCH_BYTES, p, &L)) != PLX_OK)
+    return st;
   // The counters must start at zero; the array keeps whatever the last call left.
-  if (cudaMemsetAsync(scratch, 0, pl.counter_bytes, stream) != cudaSuccess)
-    return PLX_ERR_CUDA;
-  return parallax_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, scratch,
-                         (size_t)PARALLAX_NOALLOC_SCRATCH_BYTES, p, stream);
+  if (cudaMemsetAsync(scratch, 0, L.pl.counter_bytes, stream) != cudaSuccess) return PLX_ERR_CUDA;
+  return launch_decode(L, p, stream, false);
 }
 
 plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code) {

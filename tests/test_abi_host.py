@@ -245,3 +245,37 @@ def test_backward_workspace_size_and_validation(binding):
     al = ctypes.c_void_p((ctypes.addressof(buf) + 15) & ~15)
     # every pointer present and aligned, workspace too small
     assert binding.lib.parallax_prefill_backward(*([al] * 13), 16, ctypes.byref(p), None) == 3
+
+
+def test_decode_binding_checks_cache_shapes_before_any_launch(binding):
+    # Host tensors: each call must fail on the shape check, which runs before
+    # the device checks, so no launch is ever reached.
+    q = torch.zeros((2, 4, 128), dtype=torch.bfloat16)
+    k = torch.zeros((2, 2, 256, 64), dtype=torch.bfloat16)        # head_dim 64 against q's 128
+    out = torch.zeros_like(q)
+    for fn in (lambda: binding.decode(q, q, k, k),
+               lambda: binding.decode_noalloc(q, q, k, k, out=out)):
+        with pytest.raises(ValueError, match="head_dim"):
+            fn()
+    k = torch.zeros((2, 2, 256, 128), dtype=torch.bfloat16)
+    for kv_len in (100, 300):   # a contiguous cache is addressed with its own length
+        for fn in (lambda: binding.decode(q, q, k, k, kv_len=kv_len),
+                   lambda: binding.decode_noalloc(q, q, k, k, out=out, kv_len=kv_len)):
+            with pytest.raises(ValueError, match="kv_len"):
+                fn()
+    with pytest.raises(ValueError, match="one sequence per row"):
+        binding.decode(q, q, torch.zeros((3, 2, 256, 128), dtype=torch.bfloat16),
+                       torch.zeros((3, 2, 256, 128), dtype=torch.bfloat16))
+    with pytest.raises(ValueError, match="KV heads"):
+        binding.decode(q, q, torch.zeros((2, 3, 256, 128), dtype=torch.bfloat16),
+                       torch.zeros((2, 3, 256, 128), dtype=torch.bfloat16))
+    x = torch.zeros((2, 256), dtype=torch.bfloat16)
+    w = torch.zeros((4 * 128, 256), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="kv_len"):
+        binding.decode_projected(x, w, w, k, k, kv_len=100)
+    # a paged pool must hold 64-token pages, and kv_len fits the page table
+    pool = torch.zeros((8, 2, 64, 128), dtype=torch.bfloat16)
+    table = torch.zeros((2, 4), dtype=torch.int32)
+    lens = torch.zeros((2,), dtype=torch.int32)
+    with pytest.raises(ValueError, match="kv_len"):
+        binding.decode(q, q, pool, pool, seq_lens=lens, page_table=table, kv_len=4 * 64 + 1)

@@ -65,6 +65,28 @@ def test_noalloc_matches_workspace_entry_point(px, case):
     assert px.last_device_error() == 0
 
 
+@pytest.mark.parametrize("case", ["default_grid", "empty_sequence"])
+def test_noalloc_default_grid_and_empty_sequences(px, case):
+    # The default grid (num_ctas 0) of an equal-length contiguous cache is
+    # unit-aligned and may merge a unit's pieces inside a thread-block
+    # cluster; a zero-length sequence gets a zero output without any tile.
+    if case == "default_grid":
+        inp = W.small_decode_inputs(8, 16, 8, 128, 4096, seed=34)
+    else:
+        inp = W.small_decode_inputs(4, 8, 2, 128, 1500, seq_lens=[1500, 0, 700, 0], seed=35)
+    inp = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+    ref = px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"],
+                    seq_lens=inp.get("seq_lens"), out_dtype=torch.float32, num_ctas=0)
+    for call in range(2):
+        out = torch.full_like(ref, float("nan"))
+        assert _noalloc(px, inp, out, 0) == 0
+        torch.cuda.synchronize()
+        assert_parity(out.cpu().numpy(), ref.cpu().numpy(), TOL_BF16, f"{case} call {call}")
+    if case == "empty_sequence":
+        assert torch.equal(out[1], torch.zeros_like(out[1])) and torch.equal(out[3], torch.zeros_like(out[3]))
+    assert px.last_device_error() == 0
+
+
 def test_noalloc_back_to_back_different_shapes(px):
     a, b = _inputs("contiguous_bf16"), _inputs("paged_bf16")
     for inp in (a, b, a):
