@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define PARALLAX_ABI_VERSION 4
+#define PARALLAX_ABI_VERSION 5
 
 typedef enum plx_status {
   PLX_OK = 0,
@@ -320,6 +320,20 @@ plx_status parallax_prefill_paged(const void* q, const void* rho,
  * word into *code (0 = no fault, else PLX_DEVERR_* bits).  Returns PLX_OK,
  * or PLX_ERR_CUDA if the synchronisation or the read failed. */
 plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code);
+
+/* Sets the limit of one pipeline wait in the kernels launched afterwards on
+ * the current device, in nanoseconds, and returns the previous limit in
+ * *previous (if not NULL).  A pipeline wait is one role of a CTA waiting for
+ * another's data or buffer (a TMA load to land, tensor-core results, a freed
+ * stage); the default limit is 2 s, far above any healthy wait.  When a wait
+ * runs out, the kernel sets PLX_DEVERR_TIMEOUT in the error word, abandons
+ * its work, waits for its own copies and tensor-core operations still in
+ * flight (those waits keep a fixed 2 s limit) and exits; its outputs are
+ * then undefined.  0 makes every wait give up unless its phase is already
+ * complete, which exercises that path deliberately.  A serving loop may set
+ * a shorter limit to learn sooner that a kernel is stuck.  Host-only; takes
+ * effect at the next launch.  Errors: PLX_ERR_CUDA (no current device). */
+plx_status parallax_set_wait_limit_ns(uint64_t limit_ns, uint64_t* previous);
 
 /* Static string naming a status. */
 const char* parallax_status_string(plx_status s);

@@ -86,6 +86,8 @@ lib.parallax_decode_projected.argtypes = [_vp, _vp, _vp, ctypes.c_int32, _vp, _v
 lib.parallax_decode_projected.restype = ctypes.c_int
 lib.parallax_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, ctypes.POINTER(DecodeParams), _vp]
 NOALLOC_SCRATCH_BYTES = 8 << 20
+lib.parallax_set_wait_limit_ns.restype = ctypes.c_int
+lib.parallax_set_wait_limit_ns.argtypes = [ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64)]
 lib.parallax_last_device_error.restype = ctypes.c_int
 lib.parallax_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
 
@@ -489,3 +491,13 @@ def last_device_error(device=None) -> int:
     if st != 0:
         raise ParallaxError(st, "parallax_last_device_error")
     return code.value
+
+
+def set_wait_limit_ns(limit_ns: int) -> int:
+    """Sets the pipeline wait limit of the current device's kernels (ns) and
+    returns the previous one (see parallax_set_wait_limit_ns)."""
+    prev = ctypes.c_uint64(0)
+    st = lib.parallax_set_wait_limit_ns(int(limit_ns), ctypes.byref(prev))
+    if st != 0:
+        raise ParallaxError(st, "parallax_set_wait_limit_ns")
+    return prev.value

@@ -53,6 +53,7 @@ struct DecodeArgs {
   float scale_log2;                // scale * log2(e)
   int out_bf16;
   int cluster;                     // > 1: each unit is one cluster of this many CTAs (bf16 path)
+  unsigned long long wait_ns;      // limit of one pipeline wait (0: give up unless complete)
 };
 
 // ------------------------------------------------------------ addressing
@@ -395,7 +396,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
       int issued = 0;
       for (int t = 0; t < nchunk; ++t) {
         const int s = t % STAGES;
-        if (t >= STAGES && !mbar_wait_bounded(&empty[s], ((t / STAGES) - 1) & 1)) {
+        if (t >= STAGES && !mbar_wait_bounded(a.wait_ns, &empty[s], ((t / STAGES) - 1) & 1)) {
           *abort_flag = 1;
           break;
         }
@@ -418,7 +419,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         // Drain: wait (bounded) for the last load issued into each stage.
         for (int s = 0; s < STAGES && s < issued; ++s) {
           const int last_t = s + ((issued - 1 - s) / STAGES) * STAGES;
-          mbar_wait_bounded(&full[s], (last_t / STAGES) & 1);
+          mbar_wait_drain(&full[s], (last_t / STAGES) & 1);
         }
       }
     }
@@ -491,7 +492,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
       for (; t < i_end; t += NC) {
         const int s = t % STAGES;
         if (*abort_flag) break;
-        if (!mbar_wait_bounded(&full[s], (t / STAGES) & 1)) {
+        if (!mbar_wait_bounded(a.wait_ns, &full[s], (t / STAGES) & 1)) {
           *abort_flag = 1;
           break;
         }

@@ -40,6 +40,17 @@ constexpr int kF32CtasPerSm = 4;
 
 std::mutex g_mu;
 int g_num_sms[kMaxDevices];
+// Pipeline wait limit of each device's kernels (parallax_set_wait_limit_ns).
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+unsigned long long g_wait_ns[kMaxDevices];
+bool g_wait_set[kMaxDevices];
+
+unsigned long long current_wait_ns() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return kDefaultWaitNs;
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_wait_set[dev] ? g_wait_ns[dev] : kDefaultWaitNs;
+}
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
@@ -282,6 +293,7 @@ plx_status prepare_decode(const void* q, const void* rho, const void* k_cache, c
   a.max_pages = paged ? p->max_pages_per_seq : 0;
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
+  a.wait_ns = current_wait_ns();
 
   // Units of equal length cut into k pieces each (the unit-aligned grid) are
   // merged through distributed shared memory when each unit is one cluster.
@@ -373,6 +385,7 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.out = out;
+  a.wait_ns = current_wait_ns();
   a.vbar = vbar;
   a.stats = stats;
   return launch_prefill_kernel<false>(tq, tr, tk, tv, a, stream);
@@ -457,6 +470,7 @@ plx_status launch_prefill_backward(const void* q, const void* rho, const void* k
   a.drho = drho;
   a.dk = dk;
   a.dv = dv;
+  a.wait_ns = current_wait_ns();
   const uint64_t rows_q = (uint64_t)n_rows;
   const uint64_t rows_kv = (uint64_t)p->batch * hkv * p->seq_len;
   {  // dq, drho: 128-row query tiles, 64-row key tiles
@@ -667,6 +681,7 @@ plx_status parallax_prefill_paged(const void* q, const void* rho, const void* k_
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
   a.scale_log2 = p->scale * 1.4426950408889634f;
   a.out = out;
+  a.wait_ns = current_wait_ns();
   a.cu_q = cu_seqlens_q;
   a.seq_lens = seq_lens;
   a.page_table = page_table;
@@ -696,6 +711,17 @@ plx_status parallax_decode_noalloc(const void* q, const void* rho, const void* k
   // The counters must start at zero; the array keeps whatever the last call left.
   if (cudaMemsetAsync(scratch, 0, L.pl.counter_bytes, stream) != cudaSuccess) return PLX_ERR_CUDA;
   return launch_decode(L, p, stream, false);
+}
+
+plx_status parallax_set_wait_limit_ns(uint64_t limit_ns, uint64_t* previous) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PLX_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PLX_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (previous != nullptr) *previous = g_wait_set[dev] ? g_wait_ns[dev] : kDefaultWaitNs;
+  g_wait_ns[dev] = limit_ns;
+  g_wait_set[dev] = true;
+  return PLX_OK;
 }
 
 plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code) {

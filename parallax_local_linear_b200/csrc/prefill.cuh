@@ -95,6 +95,7 @@ struct PrefillArgs {
   // dense form, training: per-row quantities the backward pass reads (null: not written)
   float* vbar;                    // [B, H, T, D]: vbar = O1 / l
   float2* stats;                  // [B, H, T]: (m + log2 l, abar = c / l), weights w = 2^(s*scale*log2(e) - x)
+  unsigned long long wait_ns;     // limit of one pipeline wait (0: give up unless complete)
 };
 
 // Four MMAs under one elect.sync: the issuing warp spends fewer instructions
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t par = ((j / kPfStages) - 1) & 1;
         // pool rows [P * Hkv * 64] (paged; page ids checked above) or [B * Hkv * T]
         const int row = kPaged ? (pt[j] * a.Hkv + kvh) * kPfBN : kv_row + j * kPfBN;
-        if (j >= kPfStages && !mbar_wait_bounded(&k_empty[s], par)) {
+        if (j >= kPfStages && !mbar_wait_bounded(a.wait_ns, &k_empty[s], par)) {
           *abort_flag = 1;
           break;
         }
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         mbar_arrive_expect_tx(&k_full[s], Ly::kKVBytes);
         for (int bx = 0; bx < 2; ++bx)
           tma_load_2d(sm + Ly::kK + s * Ly::kKVBytes + bx * (Ly::kKVBytes / 2), &tm_k, bx * 64, row, &k_full[s], keep);
-        if (j >= kPfStages && !mbar_wait_bounded(&v_empty[s], par)) {
+        if (j >= kPfStages && !mbar_wait_bounded(a.wait_ns, &v_empty[s], par)) {
           *abort_flag = 1;
           ++issued_k;
           break;
@@ -299,14 +300,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ++issued_k;
       }
       // Every issued load must land before the CTA exits.
-      mbar_wait_bounded(q_full, 0);
+      mbar_wait_drain(q_full, 0);
       for (int s = 0; s < kPfStages && s < issued_k; ++s) {
         const int last = s + ((issued_k - 1 - s) / kPfStages) * kPfStages;
-        mbar_wait_bounded(&k_full[s], (last / kPfStages) & 1);
+        mbar_wait_drain(&k_full[s], (last / kPfStages) & 1);
       }
       for (int s = 0; s < kPfStages && s < issued; ++s) {
         const int last = s + ((issued - 1 - s) / kPfStages) * kPfStages;
-        mbar_wait_bounded(&v_full[s], (last / kPfStages) & 1);
+        mbar_wait_drain(&v_full[s], (last / kPfStages) & 1);
       }
     }
   } else if (warp == 1) {
@@ -321,7 +322,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint64_t dk = smem_desc_sw128(smem_u32(sm + Ly::kK), 16, 1024);
     const uint64_t dv = smem_desc_sw128(smem_u32(sm + Ly::kV), Ly::kKVBytes / 2, 1024);
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+      return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
     bool ok = wait_warp(q_full, 0);
     tc_fence_after();
@@ -384,7 +385,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     if (!ok && lane == 0) *abort_flag = 1;
     // Every issued MMA must complete before TMEM is released.
     tc_commit(drain);
-    wait_warp(drain, 0);
+    __syncwarp();
+    mbar_wait_drain(drain, 0);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
     const int g = (warp - 2) >> 2;           // warpgroup: tiles j = g, g+2, ...; S / A buffer g
@@ -405,7 +408,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     bool fine = true;
     int j = g;
     for (; j < n; j += 2) {
-      const bool w = !*abort_flag && mbar_wait_bounded(&s_full[g], (j >> 1) & 1);
+      const bool w = !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[g], (j >> 1) & 1);
       tc_fence_after();
       uint32_t sr[64], ar[32];
       tmem_ld32p(cS, sr);
@@ -427,7 +430,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mt[0] = fmaxf(fmaxf(fmaxf(mt[0], mt[4]), fmaxf(mt[1], mt[5])), fmaxf(fmaxf(mt[2], mt[6]), fmaxf(mt[3], mt[7])));
       tmem_ld32(cA, ar);   // probe values of keys 0..31, loaded while the reference is handed over
       // The reference after tile j-1 comes from the other warpgroup.
-      const bool wh = j == 0 || mbar_wait_bounded(&hand[g], ((j - 1) >> 1) & 1);
+      const bool wh = j == 0 || mbar_wait_bounded(a.wait_ns, &hand[g], ((j - 1) >> 1) & 1);
       const bool go = bar_and(1 + g, kPfSoftmax / 2, w && wh && fine);
       tmem_wait_ld();
       if (!go) {
@@ -519,7 +522,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // last tile, which pins the phase for the epilogue's wait to n-1 or n.
       const bool rescale = __any_sync(0xffffffffu, need) && j >= 1;
       if (j >= 1 && (j == n - 1 || rescale)) {
-        const bool wo = __all_sync(0xffffffffu, mbar_wait_bounded(o_done, (j - 1) & 1));
+        const bool wo = __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, o_done, (j - 1) & 1));
         fine = fine && wo;
         if (wo && rescale) {
           tc_fence_after();
@@ -541,7 +544,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // products, which wait on this warpgroup's arrival below.
         if (key0 + kPfBN > L) {
           const int s = j % kPfStages, nv = L - key0;
-          const bool wv = mbar_wait_bounded(&v_full[s], (j / kPfStages) & 1);
+          const bool wv = mbar_wait_bounded(a.wait_ns, &v_full[s], (j / kPfStages) & 1);
           fine = fine && wv;
           if (wv) {
             uint8_t* vt = sm + Ly::kV + s * Ly::kKVBytes;
@@ -562,7 +565,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // products (its j == n-1 wait above made the phase exact), the barrier
     // below releases the other; then the rows are written.
     bool wl = fine && j >= n && !*abort_flag;
-    if (wl && ((n - 1) & 1) == g) wl = mbar_wait_bounded(o_done, (n - 1) & 1);
+    if (wl && ((n - 1) & 1) == g) wl = mbar_wait_bounded(a.wait_ns, o_done, (n - 1) & 1);
     lc_s[(g * 128 + r) * 3 + 0] = l2.x + l2.y;
     lc_s[(g * 128 + r) * 3 + 1] = c2.x + c2.y;
     lc_s[(g * 128 + r) * 3 + 2] = m_mine;

@@ -51,6 +51,7 @@ struct BwdArgs {
   void* drho;                     // [B, H, T, D]
   void* dk;                       // [B, Hkv, T, D]
   void* dv;                       // [B, Hkv, T, D]
+  unsigned long long wait_ns;     // limit of one pipeline wait (0: give up unless complete)
 };
 
 // ---------------------------------------------------------------- per row
@@ -264,23 +265,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int s = j % S;
         const uint32_t par = ((j / S) - 1) & 1;
         const int row = kv_row + j * kPfBN;
-        if (j >= S && !(ok = mbar_wait_bounded(&k_empty[s], par))) break;
+        if (j >= S && !(ok = mbar_wait_bounded(a.wait_ns, &k_empty[s], par))) break;
         mbar_arrive_expect_tx(&k_full[s], Ly::kTile64);
         for (int bx = 0; bx < 2; ++bx)
           tma_load_2d(sm + Ly::kK + s * Ly::kTile64 + bx * (Ly::kTile64 / 2), &tm_k, bx * 64, row, &k_full[s], keep);
         ++issued_k;
-        if (j >= S && !(ok = mbar_wait_bounded(&v_empty[s], par))) break;
+        if (j >= S && !(ok = mbar_wait_bounded(a.wait_ns, &v_empty[s], par))) break;
         mbar_arrive_expect_tx(&v_full[s], Ly::kTile64);
         for (int bx = 0; bx < 2; ++bx)
           tma_load_2d(sm + Ly::kV + s * Ly::kTile64 + bx * (Ly::kTile64 / 2), &tm_v, bx * 64, row, &v_full[s], keep);
         ++issued_v;
       }
       // Every issued load must land before the CTA exits.
-      mbar_wait_bounded(q_full, 0);
+      mbar_wait_drain(q_full, 0);
       for (int s = 0; s < S && s < issued_k; ++s)
-        mbar_wait_bounded(&k_full[s], ((s + ((issued_k - 1 - s) / S) * S) / S) & 1);
+        mbar_wait_drain(&k_full[s], ((s + ((issued_k - 1 - s) / S) * S) / S) & 1);
       for (int s = 0; s < S && s < issued_v; ++s)
-        mbar_wait_bounded(&v_full[s], ((s + ((issued_v - 1 - s) / S) * S) / S) & 1);
+        mbar_wait_drain(&v_full[s], ((s + ((issued_v - 1 - s) / S) * S) / S) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -293,7 +294,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint64_t dkt = smem_desc_sw128(smem_u32(sm + Ly::kK), Ly::kTile64 / 2, 1024);   // K as an MN-major B
     const uint64_t dv = smem_desc_sw128(smem_u32(sm + Ly::kV), 16, 1024);
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+      return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
     bool ok = wait_warp(q_full, 0);
     tc_fence_after();
@@ -356,7 +357,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     if (!ok && lane == 0) report_error(2 /* PLX_DEVERR_TIMEOUT */);
     tc_commit(drain);
-    wait_warp(drain, 0);
+    __syncwarp();
+    mbar_wait_drain(drain, 0);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise
     const int g = (warp - 2) >> 2;           // key-column half of every tile
@@ -370,7 +373,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     bool fine = true;
     int j = 0;
     for (; j < n; ++j) {
-      fine = __all_sync(0xffffffffu, fine && mbar_wait_bounded(sad_full, j & 1));
+      fine = __all_sync(0xffffffffu, fine && mbar_wait_bounded(a.wait_ns, sad_full, j & 1));
       if (!fine) break;
       tc_fence_after();
       uint32_t sr[32], ar[32], dr[32];
@@ -417,7 +420,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         // The products of tile j-1 must be done with the dS / dA columns.
         if (j >= 1) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (j - 1) & 1))) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, dd_free, (j - 1) & 1))) return false;
           tc_fence_after();
         }
         tmem_st16(tmem + lane_off + kBwDS + 16 * g, pds);
@@ -441,7 +444,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_arrive(dd_full);
     }
     // ---- epilogue: the last dQ, dR products, then the rows
-    fine = __all_sync(0xffffffffu, fine && j == n && mbar_wait_bounded(dd_free, (n - 1) & 1));
+    fine = __all_sync(0xffffffffu, fine && j == n && mbar_wait_bounded(a.wait_ns, dd_free, (n - 1) & 1));
     if (fine) {
       tc_fence_after();
       const size_t orow = ((size_t)(b * a.H + h) * a.T + t) * kPfD + 64 * g;
@@ -587,7 +590,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int issued = 0;
       for (int it = 0; it < N; ++it) {
         const int s = it % S;
-        if (it >= S && !mbar_wait_bounded(&op_empty[s], ((it / S) - 1) & 1)) break;
+        if (it >= S && !mbar_wait_bounded(a.wait_ns, &op_empty[s], ((it / S) - 1) & 1)) break;
         const int hq = head_of(it), t0 = tile_of(it) * kPfBN;
         const int row = (b * a.H + hq) * a.T + t0;
         const int nrows = min(kPfBN, a.T - t0);   // row records past T are not read
@@ -602,9 +605,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         bulk_load(st + Ly::kStRows, a.rows + (size_t)(b * a.H + hq) * a.T + t0, (uint32_t)nrows * 16, &op_full[s]);
         ++issued;
       }
-      mbar_wait_bounded(kv_full, 0);
+      mbar_wait_drain(kv_full, 0);
       for (int s = 0; s < S && s < issued; ++s)
-        mbar_wait_bounded(&op_full[s], ((s + ((issued - 1 - s) / S) * S) / S) & 1);
+        mbar_wait_drain(&op_full[s], ((s + ((issued - 1 - s) / S) * S) / S) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -614,7 +617,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const uint64_t dvv = smem_desc_sw128(smem_u32(sm + Ly::kV), 16, 1024);
     const uint64_t dones = smem_desc_sw128(smem_u32(sm + Ly::kOnes), 16, 1024);
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
-      return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity));
+      return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
     bool ok = wait_warp(kv_full, 0);
     tc_fence_after();
@@ -699,7 +702,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     if (!ok && lane == 0) report_error(2 /* PLX_DEVERR_TIMEOUT */);
     tc_commit(drain);
-    wait_warp(drain, 0);
+    __syncwarp();
+    mbar_wait_drain(drain, 0);
+    __syncwarp();
   } else {
     // ------------------------------------------------------------ elementwise
     const int g = (warp - 2) >> 2;           // query-column half of every tile
@@ -710,7 +715,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     bool fine = true;
     int it = 0;
     for (; it < N; ++it) {
-      fine = __all_sync(0xffffffffu, fine && mbar_wait_bounded(sad_full, it & 1));
+      fine = __all_sync(0xffffffffu, fine && mbar_wait_bounded(a.wait_ns, sad_full, it & 1));
       if (!fine) break;
       tc_fence_after();
       const int t0 = tile_of(it) * kPfBN + 32 * g;   // query of this thread's first column
@@ -777,7 +782,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         // The products of the previous tile must be done with the dS / dA columns.
         if (q == 0 && it >= 1) {
-          if (!__all_sync(0xffffffffu, mbar_wait_bounded(dd_free, (it - 1) & 1))) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, dd_free, (it - 1) & 1))) return false;
           tc_fence_after();
         }
         tmem_st8(tmem + lane_off + kBwS + col, pu);
@@ -803,7 +808,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!fine) break;
     }
     // ---- epilogue: the last products, then the key rows
-    fine = __all_sync(0xffffffffu, fine && it == N && mbar_wait_bounded(dd_free, (N - 1) & 1));
+    fine = __all_sync(0xffffffffu, fine && it == N && mbar_wait_bounded(a.wait_ns, dd_free, (N - 1) & 1));
     if (fine) {
       tc_fence_after();
       const size_t orow = ((size_t)(b * a.Hkv + kvh) * a.T + key) * kPfD + 64 * g;

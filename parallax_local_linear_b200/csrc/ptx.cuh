@@ -25,9 +25,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Upper bound of any single pipeline wait.  A healthy wait lasts micro- to
-// milliseconds; past this the kernel records PLX_DEVERR_TIMEOUT and unwinds.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Upper bound of a drain wait: a CTA that unwinds waits for its own copies
+// and tensor-core operations still in flight before it exits or frees tensor
+// memory.  Those complete on their own, so this limit is fixed and long.
+// Pipeline waits (a role waiting for another role's data or buffer) take
+// their limit from the kernel's arguments instead (parallax_set_wait_limit_ns).
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -59,19 +62,43 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete.  Returns false (and
-// records PLX_DEVERR_TIMEOUT) if it has not after kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete, for at most
+// `limit_ns` nanoseconds (0: only if it is complete already).  Returns false,
+// and records PLX_DEVERR_TIMEOUT, if it has not.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t limit_ns, uint64_t* bar, uint32_t parity) {
+  if (limit_ns == 0) {
+    if (mbar_test_wait(bar, parity)) return true;
+    report_error(2 /* PLX_DEVERR_TIMEOUT */);
+    return false;
+  }
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t it = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if ((++it & 255u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((++it & 255u) == 0 && globaltimer_ns() - t0 > limit_ns) {
       report_error(2 /* PLX_DEVERR_TIMEOUT */);
       return false;
     }
   }
   return true;
+}
+
+// A drain wait (see kDrainLimitNs).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  return mbar_wait_bounded(kDrainLimitNs, bar, parity);
 }
 
 // ------------------------------------------------------------------- TMA

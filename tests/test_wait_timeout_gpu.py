@@ -1,0 +1,107 @@
+"""A kernel wait that runs out of time is reported and leaves the device usable.
+
+Every wait of one CTA role on another (a TMA load landing, tensor-core
+results, a freed ring stage) is bounded by the device's pipeline wait limit.
+These tests set that limit to 0, so the first wait that does not find its
+phase complete gives up: the kernel must set PLX_DEVERR_TIMEOUT, wait for its
+own copies and tensor-core operations in flight (those waits keep their own
+long limit), free its tensor memory and return.  The next call with the
+default limit, on the same stream and workspace, must then match the float64
+oracle.  No GPU fault is involved: the failure is an ordinary bounded wait
+that returns false.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parallax_local_linear_b200 import workloads as W
+from tests.helpers import TOL_BF16, F64View, assert_parity, oracle_heads, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def px():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from parallax_local_linear_b200 import binding
+    return binding
+
+
+def _timed_out(px, call):
+    """Runs `call` with a zero wait limit; returns the error word it left."""
+    assert px.last_device_error() == 0
+    prev = px.set_wait_limit_ns(0)
+    try:
+        call()
+        code = px.last_device_error()   # synchronises: the call has returned on the device
+    finally:
+        px.set_wait_limit_ns(prev)
+    assert prev == 2_000_000_000
+    return code
+
+
+@pytest.mark.parametrize("ctas", [3, 0])
+def test_decode_wait_timeout_then_recovery(px, ctas):
+    # ctas 3: pieces merged through the workspace; 0: the unit-aligned grid,
+    # whose clusters merge through distributed shared memory.
+    inp = W.small_decode_inputs(2, 4, 2, 128, 8192, seed=51)
+    inp = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+
+    def run():
+        return px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"],
+                         out_dtype=torch.float32, num_ctas=ctas)
+
+    code = _timed_out(px, run)
+    assert code & px.DEVERR_TIMEOUT, f"error word {code}"
+    out = run()
+    assert px.last_device_error() == 0
+    ref = oracle_heads(inp, [(b, h) for b in range(2) for h in range(4)])
+    assert_parity(out.cpu().numpy(), ref, TOL_BF16, f"decode after a timeout, ctas={ctas}")
+
+
+def test_prefill_wait_timeout_then_recovery(px):
+    inp = W.small_prefill_inputs(1, 2, 1000, 128, seed=52)
+    inp = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+
+    def run():
+        return px.prefill(inp["q"], inp["rho"], inp["k"], inp["v"], causal=True, scale=inp["scale"],
+                          out_dtype=torch.float32)
+
+    code = _timed_out(px, run)
+    assert code & px.DEVERR_TIMEOUT, f"error word {code}"
+    out = run().cpu().numpy()
+    assert px.last_device_error() == 0
+    rows = [(0, h, t) for h in range(2) for t in (0, 1, 127, 128, 500, 999)]
+    views = {k: F64View(inp[k]) for k in ("q", "rho", "k", "v")}
+    ref = oracle.prefill_rows(views["q"], views["rho"], views["k"], views["v"], rows, inp["scale"])
+    assert_parity(np.stack([out[b, h, t] for b, h, t in rows]), ref, TOL_BF16, "prefill after a timeout")
+
+
+def test_backward_wait_timeout_then_recovery(px):
+    x = W.small_prefill_inputs(1, 2, 300, 128, seed=53)
+    x = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in x.items()}
+    dout = W.dout_like(x["q"], 54)
+    out, vbar, stats = px.prefill_train(x["q"], x["rho"], x["k"], x["v"], True, x["scale"], out_dtype=torch.float32)
+
+    def run():
+        return px.prefill_backward(x["q"], x["rho"], x["k"], x["v"], out, vbar, stats, dout, True, x["scale"])
+
+    code = _timed_out(px, run)
+    assert code & px.DEVERR_TIMEOUT, f"error word {code}"
+    grads = run()
+    assert px.last_device_error() == 0
+    ref = oracle.prefill_grads(*(to_f64(t) for t in (x["q"], x["rho"], x["k"], x["v"], dout)), x["scale"],
+                               causal=True)
+    for name, g, r in zip(("dq", "drho", "dk", "dv"), grads, ref):
+        assert_parity(g.cpu().numpy(), r, TOL_BF16, f"{name} after a timeout")
+
+
+def test_wait_limit_setter_round_trips(px):
+    prev = px.set_wait_limit_ns(123456)
+    try:
+        assert px.set_wait_limit_ns(prev) == 123456
+    finally:
+        px.set_wait_limit_ns(prev)
