@@ -22,6 +22,12 @@ the workload (independent sequences, no collective on the data path), so
 scaling is weak and ``value`` is the total over ranks divided by the slowest
 rank's time.
 
+The default run (decode_bf16) then times every other workload the same way
+(``per_config`` in the JSON line: decode_f32, decode_long, decode_paged,
+prefill, prefill_paged, prefill_train, decode_projected), each with its
+roofline against the measured and the nominal peak, its clocks and its
+oracle baseline; ``--no-per-config`` skips them.
+
 ``--impl reference`` times the float64 CPU oracle on the host cores instead
 (rank 0 only), on a bounded sample of the same workload per step.
 """
@@ -77,6 +83,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--cpu-seconds-per-config", type=float, default=4.0,
+                    help="target CPU time of each other workload's oracle baseline sample")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="time only --workload (by default the decode_bf16 run also times every other workload)")
     return ap.parse_args(argv)
 
 
@@ -112,22 +122,32 @@ def source_sha(kind):
 
 def profiled_traffic(kind, workload):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
-    path = os.path.join(ROOT, "profiles", f"{kind}-{workload}.md")
+    on the current kernel source.  Returns (bytes or None, provenance)."""
+    rel = os.path.join("profiles", f"{kind}-{workload}.md")
+    path = os.path.join(ROOT, rel)
     if not os.path.exists(path):
-        return None
+        return None, f"no ncu summary at {rel}"
     fields = {}
     with open(path) as f:
         for line in f:
             if ":" in line and line.startswith("- "):
                 k, v = line[2:].split(":", 1)
                 fields[k.strip()] = v.strip().strip("`")
-    if fields.get("source_sha256") != source_sha(kind):
-        return None
+    sha = source_sha(kind)
+    if fields.get("source_sha256") != sha:
+        return None, (f"{rel} was captured on kernel source {fields.get('source_sha256')}, "
+                      f"not the current {sha}: no counters for this source")
     try:
-        return float(fields["dram_bytes_per_launch"])
+        return float(fields["dram_bytes_per_launch"]), (
+            f"read from {rel} (ncu dram__bytes_read.sum + dram__bytes_write.sum, kernel source {sha}); "
+            "not measured in this run")
     except (KeyError, ValueError):
-        return None
+        return None, f"{rel} holds no dram_bytes_per_launch"
+
+
+def traffic_fields(kind, workload):
+    t, src = profiled_traffic(kind, workload)
+    return {"traffic": t, "traffic_source": src}
 
 
 class ClockSampler:
@@ -316,7 +336,7 @@ def bench_decode(args, w, rank, world, dev, peaks, peaks_kind):
     achieved = per_launch_bytes / avg_launch_s / 1e9
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": profiled_traffic("decode", w.name),
+                "frac": round(achieved / peak, 4), **traffic_fields("decode", w.name),
                 "peak_source": f"{peaks_kind} hbm_gbs", "kernel": "decode_tc_kernel" if w.dtype == "bf16"
                 else "decode_f32_kernel", "algorithmic_bytes_per_launch": int(per_launch_bytes)}
     res = {
@@ -487,7 +507,7 @@ def bench_decode_projected(args, w, rank, world, dev, peaks, peaks_kind):
                    "cache and weights stay resident on the device"}
 
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": profiled_traffic("decode_projected", w.name),
+                "frac": round(achieved / peak, 4), **traffic_fields("decode_projected", w.name),
                 "peak_source": f"{peaks_kind} hbm_gbs",
                 "kernel": "project_qr_kernel + decode_tc_kernel (one call)",
                 "algorithmic_bytes_per_launch": int(step_bytes)}
@@ -572,7 +592,7 @@ def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
                    "l2": "inputs 537 MB > 126 MB L2"},
         "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic("prefill", w.name),
+                     "frac": round(achieved / peak, 4), **traffic_fields("prefill", w.name),
                      "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_kernel",
                      "algorithmic_flops_per_launch": flops},
         "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
@@ -652,7 +672,7 @@ def bench_prefill_paged(args, w, rank, world, dev, peaks, peaks_kind):
                    "l2": f"q+rho {qr_mb:.0f} MB + KV pages {kv_mb:.0f} MB > 126 MB L2"},
         "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic("prefill", w.name),
+                     "frac": round(achieved / peak, 4), **traffic_fields("prefill", w.name),
                      "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_kernel (paged)",
                      "algorithmic_flops_per_launch": flops},
         "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
@@ -734,7 +754,7 @@ def bench_prefill_train(args, w, rank, world, dev, peaks, peaks_kind):
                    "bwd_ms": round(bwd_ms, 4), "l2": "inputs 671 MB > 126 MB L2"},
         "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": profiled_traffic("prefill_bwd", w.name),
+                     "frac": round(achieved / peak, 4), **traffic_fields("prefill_bwd", w.name),
                      "peak_source": f"{peaks_kind} bf16_tflops_sustained",
                      "kernel": "prefill backward: rows + dq + dkv kernels (one call)",
                      "algorithmic_flops_per_launch": f_bwd},
@@ -952,12 +972,54 @@ def _host_decode_sample(w):
 
 # -------------------------------------------------------------------- main
 
+# Workloads timed after the headline one in the default run, each with its
+# own roofline, clocks and oracle baseline (the four other configurations of
+# the method's targets first, then the serving and training steps beyond them).
+PER_CONFIG = ("decode_f32", "decode_long", "decode_paged", "prefill", "prefill_paged", "prefill_train",
+              "decode_projected")
+NOMINAL_PEAKS = {"GB/s": 8000.0, "TFLOP/s": 2250.0}   # B200 HBM3e and dense bf16, NVIDIA's figures
+
+
+def run_workload(args, w, rank, world, dev, peaks, kind):
+    if w.name == "prefill":
+        return bench_prefill(args, w, rank, world, dev, peaks, kind)
+    if w.name == "prefill_paged":
+        return bench_prefill_paged(args, w, rank, world, dev, peaks, kind)
+    if w.name == "prefill_train":
+        return bench_prefill_train(args, w, rank, world, dev, peaks, kind)
+    if w.hidden:
+        res, inp = bench_decode_projected(args, w, rank, world, dev, peaks, kind)
+        return res, inp[0]
+    res, inp = bench_decode(args, w, rank, world, dev, peaks, kind)
+    return res, inp[0]
+
+
+def config_summary(res):
+    """The per-workload record of the default run: throughput, its roofline
+    against the measured and the nominal peak, clocks, e2e and the oracle."""
+    rf = dict(res["roofline"])
+    nominal = NOMINAL_PEAKS[rf["unit"]]
+    rf["nominal_peak"] = nominal
+    rf["frac_of_nominal"] = round(rf["achieved"] / nominal, 4)
+    out = {k: res[k] for k in ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config", "clocks",
+                               "gpu_launches") if k in res}
+    out["roofline"] = rf
+    if "tokens_per_s" in res:
+        out["tokens_per_s"] = res["tokens_per_s"]
+    if "e2e" in res:
+        out["e2e"] = {k: res["e2e"][k] for k in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step")}
+    if "cpu_baseline" in res:
+        out["cpu_baseline"] = res["cpu_baseline"]
+    return out
+
+
 def main(argv=None):
     args = parse_args(argv)
     w = W.WORKLOADS[args.workload]
     if args.batch > 0:
         import dataclasses
         w = dataclasses.replace(w, batch=args.batch)
+    steps_given, warmup_given = args.steps, args.warmup
     if args.steps is None:
         args.steps = default_steps(args.workload) if args.impl == "ours" else 10
     if args.warmup is None:
@@ -980,21 +1042,33 @@ def main(argv=None):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     peaks, kind = load_peaks()
     try:
-        if w.name == "prefill":
-            res, inp = bench_prefill(args, w, rank, world, dev, peaks, kind)
-        elif w.name == "prefill_paged":
-            res, inp = bench_prefill_paged(args, w, rank, world, dev, peaks, kind)
-        elif w.name == "prefill_train":
-            res, inp = bench_prefill_train(args, w, rank, world, dev, peaks, kind)
-        elif w.hidden:
-            res, inp = bench_decode_projected(args, w, rank, world, dev, peaks, kind)
-            inp = inp[0]
-        else:
-            res, inp = bench_decode(args, w, rank, world, dev, peaks, kind)
-            inp = inp[0]
+        res, inp = run_workload(args, w, rank, world, dev, peaks, kind)
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_seconds)
+        del inp
+        per_config = {}
+        if args.per_config and args.workload == "decode_bf16" and args.batch == 0:
+            import copy
+            for name in PER_CONFIG:
+                torch.cuda.empty_cache()
+                wc = W.WORKLOADS[name]
+                ac = copy.copy(args)
+                ac.steps = steps_given if steps_given is not None else default_steps(name)
+                ac.warmup = warmup_given if warmup_given is not None else 5
+                rc, ic = run_workload(ac, wc, rank, world, dev, peaks, kind)
+                if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                    rc["cpu_baseline"] = cpu_baseline(wc, ic, args.cpu_seconds_per_config)
+                del ic
+                per_config[name] = config_summary(rc)
         if rank == 0:
+            res["roofline"]["nominal_peak"] = NOMINAL_PEAKS[res["roofline"]["unit"]]
+            res["roofline"]["frac_of_nominal"] = round(res["roofline"]["achieved"] /
+                                                       res["roofline"]["nominal_peak"], 4)
+            if per_config:
+                res["per_config"] = per_config
+                res["per_config_note"] = ("each workload timed in this same run on the same GPU after the "
+                                          "headline, with its own timed region, launches, clocks and oracle "
+                                          "sample; the top-level keys describe the headline alone")
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

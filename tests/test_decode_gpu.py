@@ -68,10 +68,17 @@ def test_decode_bf16_workload(px):
 
 
 def test_decode_long_workload_sampled(px):
+    # 64 (sequence, query head) pairs: every sequence's first and last
+    # sequences, all four query heads of some KV heads, the rest seeded.
     w = W.WORKLOADS["decode_long"]
     inp = W.decode_inputs(w, device=DEV)
     out = _run(px, inp).float().cpu().numpy()
-    heads = [(0, 0), (0, 31), (17, 5), (40, 12), (63, 30), (63, 3)]
+    rng = np.random.default_rng(3)
+    heads = {(0, 0), (0, 31), (63, 0), (63, 31), (17, 4), (17, 5), (17, 6), (17, 7), (40, 28), (40, 29),
+             (40, 30), (40, 31)}
+    while len(heads) < 64:
+        heads.add((int(rng.integers(w.batch)), int(rng.integers(w.num_q_heads))))
+    heads = sorted(heads)
     ref = oracle_heads(inp, heads)
     for b, h in heads:
         assert_parity(out[b, h], ref[b, h], TOL_BF16, f"decode_long ({b},{h})")
@@ -82,12 +89,18 @@ def test_decode_long_workload_sampled(px):
 
 
 def test_decode_paged_workload_sampled(px):
+    # Every one of the 128 sequences at one query head (so the shortest, the
+    # longest and every length residue mod the 64-token page that the seed
+    # draws are covered), plus all 16 heads of the shortest and the longest.
     w = W.WORKLOADS["decode_paged"]
     inp = W.decode_inputs(w, device=DEV)
     out = _run(px, inp).float().cpu().numpy()
     lens = inp["seq_lens"].cpu().numpy()
     b_short, b_long = int(np.argmin(lens)), int(np.argmax(lens))
-    heads = [(b_short, 0), (b_short, 15), (b_long, 4), (b_long, 11), (7, 2), (100, 9)]
+    heads = {(b, b % w.num_q_heads) for b in range(w.batch)}
+    heads |= {(b, h) for b in (b_short, b_long) for h in range(w.num_q_heads)}
+    heads = sorted(heads)
+    assert len({int(n) % 64 for n in lens}) > 32   # many page-boundary residues
     ref = oracle_heads(inp, heads)
     for b, h in heads:
         assert_parity(out[b, h], ref[b, h], TOL_BF16, f"decode_paged ({b},{h}) len={lens[b]}")

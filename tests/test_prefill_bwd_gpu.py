@@ -108,6 +108,7 @@ def test_deterministic(px):
 
 
 def test_full_prefill_workload_sampled(px):
+    from tests.test_prefill_gpu import full_workload_rows
     w = W.WORKLOADS["prefill"]
     x = W.prefill_inputs(w, device="cuda")
     dout = W.dout_like(x["q"], w.seed + 1000)
@@ -116,24 +117,33 @@ def test_full_prefill_workload_sampled(px):
                                            x["scale"])
     for gg in (dq, drho, dk, dv):
         assert torch.isfinite(gg.float()).all()
-    T = w.seq_len
-    views = {n: F64View(x[n]) for n in ("q", "rho", "k", "v")}
-    gv = F64View(dout)
-    # dq, drho of sampled rows: each depends on its own row only
-    for b, h, t in [(0, 0, 0), (1, 3, 127), (2, 9, 128), (3, 15, T - 1), (0, 7, 4000)]:
-        rq, rr, _, _ = oracle.query_grads(views["q"][b, h, t], views["rho"][b, h, t], views["k"][b, h, :t + 1],
-                                          views["v"][b, h, :t + 1], gv[b, h, t], x["scale"])
-        assert_parity(dq[b, h, t].float().cpu().numpy(), rq, TOL_BF16, f"dq {(b, h, t)}")
-        assert_parity(drho[b, h, t].float().cpu().numpy(), rr, TOL_BF16, f"drho {(b, h, t)}")
-    # dk, dv of keys near the end: the sum over the rows that see them
-    for b, h, i in [(1, 5, T - 1), (3, 2, T - 3)]:
-        sk = np.zeros(128)
-        sv = np.zeros(128)
-        for t in range(i, T):
-            _, _, rk, rv = oracle.query_grads(views["q"][b, h, t], views["rho"][b, h, t], views["k"][b, h, :t + 1],
-                                              views["v"][b, h, :t + 1], gv[b, h, t], x["scale"])
-            sk += rk[i]
-            sv += rv[i]
-        assert_parity(dk[b, h, i].float().cpu().numpy(), sk, TOL_BF16, f"dk {(b, h, i)}")
-        assert_parity(dv[b, h, i].float().cpu().numpy(), sv, TOL_BF16, f"dv {(b, h, i)}")
+    T, tail = w.seq_len, 65
+    rows = full_workload_rows(w.batch, w.num_heads, T)
+    pairs = sorted({(b, h) for b, h, _ in rows})
+    for n_pair, (b, h) in enumerate(pairs):
+        sl = {k: x[k][b, h].double().cpu().numpy() for k in ("q", "rho", "k", "v")}
+        g = dout[b, h].double().cpu().numpy()
+        ts = sorted({t for bb, hh, t in rows if (bb, hh) == (b, h)})
+        # in half of the pairs the last `tail` rows are all computed: they give
+        # dk, dv of the last `tail` keys exactly (no earlier row sees them)
+        full_tail = n_pair % 2 == 0
+        if full_tail:
+            ts = sorted(set(ts) | set(range(T - tail, T)))
+        sk = np.zeros((tail, 128))
+        sv = np.zeros((tail, 128))
+        rq_all, rr_all = {}, {}
+        for t in ts:
+            rq, rr, rk, rv = oracle.query_grads(sl["q"][t], sl["rho"][t], sl["k"][:t + 1], sl["v"][:t + 1], g[t],
+                                                x["scale"])
+            rq_all[t], rr_all[t] = rq, rr
+            if full_tail and t >= T - tail:
+                sk[: t + 1 - (T - tail)] += rk[T - tail:]
+                sv[: t + 1 - (T - tail)] += rv[T - tail:]
+        got_q = dq[b, h, ts].float().cpu().numpy()
+        got_r = drho[b, h, ts].float().cpu().numpy()
+        assert_parity(got_q, np.stack([rq_all[t] for t in ts]), TOL_BF16, f"dq (b={b}, h={h})")
+        assert_parity(got_r, np.stack([rr_all[t] for t in ts]), TOL_BF16, f"drho (b={b}, h={h})")
+        if full_tail:
+            assert_parity(dk[b, h, T - tail:].float().cpu().numpy(), sk, TOL_BF16, f"dk (b={b}, h={h})")
+            assert_parity(dv[b, h, T - tail:].float().cpu().numpy(), sv, TOL_BF16, f"dv (b={b}, h={h})")
     assert px.last_device_error() == 0
