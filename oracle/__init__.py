@@ -13,6 +13,8 @@ Sources (web pages on the method):
     Attention" (wispaper.ai blog), sections "Context: Why Softmax is Not
     Enough", "The Core Insight: Covariance Correction" and "Hardware
     Efficiency".
+  * Local Linear Attention with the solved probe (``lla_*``): the newx.sg
+    "Abstract" and the blog's "Context" section.
 """
 
 from .parallax_oracle import (  # noqa: F401
@@ -28,4 +30,8 @@ from .parallax_oracle import (  # noqa: F401
     round_bf16,
     project_heads,
     decode_projected,
+    sigma_kk,
+    lla_probe,
+    lla_query,
+    lla_decode,
 )

@@ -56,6 +56,10 @@ __all__ = [
     "round_bf16",
     "project_heads",
     "decode_projected",
+    "sigma_kk",
+    "lla_probe",
+    "lla_query",
+    "lla_decode",
 ]
 
 
@@ -345,3 +349,77 @@ def decode_projected(x, w_q, w_rho, k_cache, v_cache, scale: float, seq_lens=Non
     rho = round_bf16(project_heads(x, w_rho, Hq, d))
     return q, rho, decode(q, rho, k_cache, v_cache, scale, seq_lens=seq_lens,
                           page_table=page_table, heads=heads)
+
+
+# ------------------------------------------------- LLA with the solved probe
+
+def sigma_kk(w, keys) -> np.ndarray:
+    """Softmax-weighted key covariance, explicit d_k x d_k matrix:
+    sum_i w_i (k_i - kbar)(k_i - kbar)^T with kbar = sum_i w_i k_i."""
+    w = _f64(w)
+    K = _f64(keys)
+    Kc = K - w @ K
+    return Kc.T @ (w[:, None] * Kc)
+
+
+def lla_probe(q, keys, scale: float, ridge: float) -> np.ndarray:
+    """The probe Local Linear Attention solves for, per query.
+
+    LLA is the local linear estimate: the intercept of the softmax-weighted
+    least-squares fit v ~ a + M^T (k - q) (newx.sg "Abstract": it upgrades
+    the local constant estimate of softmax attention to a local linear one;
+    wispaper blog, "Context: Why Softmax is Not Enough": it solves a linear
+    system for every token).  Its intercept is vbar - S_KV^T rho* with
+        (S_KK + ridge I) rho* = kbar - q,
+    where ``ridge`` >= 0 penalises the slope M (ridge * ||M||^2; the pages
+    name no regularisation, so it is a parameter and 0 is plain LLA).  The
+    system is solved exactly (numpy.linalg.solve); the pages' solver is
+    conjugate gradients, whose converged answer is the same.  An empty key
+    set gives rho* = 0.
+    """
+    q = _f64(q)
+    K = _f64(keys)
+    if K.shape[0] == 0:
+        return np.zeros(K.shape[1], dtype=np.float64)
+    w = softmax_weights(scale * (K @ q))
+    kbar = w @ K
+    A = sigma_kk(w, K) + ridge * np.eye(K.shape[1])
+    return np.linalg.solve(A, kbar - q)
+
+
+def lla_query(q, keys, values, scale: float, ridge: float):
+    """LLA output for one query: (rho*, vbar - S_KV^T rho*), the Parallax
+    output of ``parallax_query`` with the solved probe in place of a learned
+    one."""
+    rho = lla_probe(q, keys, scale, ridge)
+    return rho, parallax_query(q, rho, keys, values, scale)
+
+
+def lla_decode(q, k_cache, v_cache, scale: float, ridge: float, seq_lens=None, page_table=None, heads=None):
+    """Decode with LLA's solved probe: for every (sequence, query head),
+    ``lla_query`` over the sequence's keys (contiguous or paged caches, GQA
+    and ``heads`` as in ``decode``).  Returns (rho*, out), float64
+    [B, Hq, d_k] and [B, Hq, d_v]; heads not evaluated are NaN."""
+    q = np.asarray(q)
+    B, Hq, dk = q.shape
+    Hkv = k_cache.shape[1]
+    group = Hq // Hkv
+    dv = v_cache.shape[-1]
+    if seq_lens is None:
+        assert page_table is None, "paged decode needs seq_lens"
+        seq_lens = [k_cache.shape[2]] * B
+    rho = np.full((B, Hq, dk), np.nan, dtype=np.float64)
+    out = np.full((B, Hq, dv), np.nan, dtype=np.float64)
+    todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hq)]
+    for b, h in todo:
+        kvh = h // group
+        n = int(seq_lens[b])
+        if page_table is None:
+            K = _f64(k_cache[b, kvh, :n, :])
+            V = _f64(v_cache[b, kvh, :n, :])
+        else:
+            K = gather_paged_keys(k_cache, page_table[b], n, kvh)
+            V = gather_paged_keys(v_cache, page_table[b], n, kvh)
+        rho[b, h], out[b, h] = lla_query(q[b, h], K, V, scale, ridge)
+    return rho, out
+
