@@ -63,6 +63,7 @@ KERNEL_SOURCES = {
                     "parallax_local_linear_b200/csrc/ptx.cuh"],
     "decode_projected": ["parallax_local_linear_b200/csrc/project.cuh", "parallax_local_linear_b200/csrc/decode.cuh",
                          "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "lla": ["parallax_local_linear_b200/csrc/lla.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
 }
 KV_COPIES = 4          # decode_bf16: 4 x 128 MiB of KV, more than L2
 GRAPH_STEPS = 64       # decode calls per captured graph
@@ -91,7 +92,7 @@ def parse_args(argv=None):
 
 
 def default_steps(workload):
-    return {"decode_f32": 20000, "decode_bf16": 8192, "decode_projected": 8192, "decode_long": 200,
+    return {"decode_f32": 20000, "decode_bf16": 8192, "decode_projected": 8192, "lla_decode": 2048, "decode_long": 200,
             "decode_paged": 200, "prefill": 20, "prefill_paged": 20, "prefill_train": 10}[workload]
 
 
@@ -529,6 +530,148 @@ def bench_decode_projected(args, w, rank, world, dev, peaks, peaks_kind):
     return res, insts
 
 
+def bench_lla(args, w, rank, world, dev, peaks, peaks_kind):
+    """Local Linear Attention with the solved probe over decode_bf16's inputs:
+    the moments pass over K and V, then the per-head solve (two launches)."""
+    from parallax_local_linear_b200 import binding as px
+
+    ridge = 0.0
+    copies = KV_COPIES
+    insts = [W.decode_inputs(w, device=dev, seed=w.seed + 1000 * rank + i) for i in range(copies)]
+    outs = [torch.empty_like(x["q"]) for x in insts]
+    rhos = [torch.empty(x["q"].shape, dtype=torch.float32, device=dev) for x in insts]
+    kv = W.kv_bytes(w)
+    flops = W.lla_decode_flops(w)
+
+    def step(i):
+        c = i % copies
+        x = insts[c]
+        px.lla_decode(x["q"], x["k_cache"], x["v_cache"], x["scale"], ridge, out=outs[c], rho_out=rhos[c],
+                      num_ctas=args.num_ctas)
+
+    stream = torch.cuda.current_stream()
+    for i in range(max(args.warmup, 3)):
+        step(i)
+    torch.cuda.synchronize()
+    assert px.last_device_error() == 0, "device error during warm-up"
+    K = args.steps
+    n = min(GRAPH_STEPS, K)
+
+    def capture(count):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(count):
+                step(i)
+        return g
+
+    graphs = [(capture(n), K // n)]
+    if K % n:
+        graphs.append((capture(K % n), 1))
+    for gg, _ in graphs:
+        gg.replay()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record(stream)
+        for gg, reps in graphs:
+            for _ in range(reps):
+                gg.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    ms = start.elapsed_time(end)
+    assert px.last_device_error() == 0, "device error during the timed steps"
+    ms_max, total_bytes = reduce_over_ranks(ms, kv * K, dev, world)
+    gbs = total_bytes / (ms_max * 1e-3) / 1e9
+    step_s = ms * 1e-3 / K
+    tflops = flops / step_s / 1e12
+    hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    tc_peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    hbm_frac, tc_frac = kv / step_s / 1e9 / hbm_peak, tflops / tc_peak
+    if tc_frac >= hbm_frac:
+        roofline = {"bound": "tensor", "achieved": round(tflops, 1), "peak": tc_peak, "unit": "TFLOP/s",
+                    "frac": round(tc_frac, 4), "peak_source": f"{peaks_kind} bf16_tflops",
+                    "algorithmic_flops_per_launch": flops}
+    else:
+        roofline = {"bound": "hbm", "achieved": round(kv / step_s / 1e9, 1), "peak": hbm_peak, "unit": "GB/s",
+                    "frac": round(hbm_frac, 4), "peak_source": f"{peaks_kind} hbm_gbs",
+                    "algorithmic_bytes_per_launch": kv}
+    roofline.update(traffic_fields("lla", w.name))
+    roofline["kernel"] = "lla_moments_kernel + lla_solve_kernel (one call)"
+    roofline["other_bound"] = ({"unit": "GB/s", "achieved": round(kv / step_s / 1e9, 1), "frac": round(hbm_frac, 4)}
+                               if roofline["bound"] == "tensor" else
+                               {"unit": "TFLOP/s", "achieved": round(tflops, 1), "frac": round(tc_frac, 4)})
+
+    # e2e: q from pinned host memory each step, output read back; cache resident
+    host_q = [x["q"].cpu().pin_memory() for x in insts]
+    out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+    dq = [torch.empty_like(x["q"]) for x in insts]
+    Ke = min(K, 2048)
+
+    def one(i):
+        c = i % copies
+        x = insts[c]
+        dq[c].copy_(host_q[c], non_blocking=True)
+        px.lla_decode(dq[c], x["k_cache"], x["v_cache"], x["scale"], ridge, out=outs[c], rho_out=rhos[c],
+                      num_ctas=args.num_ctas)
+        out_host[c].copy_(outs[c], non_blocking=True)
+
+    for i in range(3):
+        one(i)
+    torch.cuda.synchronize()
+    s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s2.record()
+    for i in range(Ke):
+        one(i)
+    e2.record()
+    torch.cuda.synchronize()
+    ms_e, tot_e = reduce_over_ranks(s2.elapsed_time(e2), kv * Ke, dev, world)
+    e2e = {"value": round(tot_e / (ms_e * 1e-3) / 1e9, 2), "unit": "GB/s",
+           "h2d_bytes_per_step": insts[0]["q"].numel() * 2, "d2h_bytes_per_step": outs[0].numel() * 2,
+           "steps": Ke, "ms_per_step": round(ms_e / Ke, 6)}
+    cfg = dict(decode_config(w, args, None), ridge=ridge,
+        l2="each step reads one of %d KV copies (%.0f MiB total > 126 MB L2)" % (copies, copies * kv / 2**20),
+        timing="CUDA-graph replay", tflops=round(tflops, 1), algorithmic_flops_per_step=flops)
+    cfg.pop("num_ctas", None)
+    res = {
+        "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": round(ms_max / K, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+        "tokens_per_s": round(w.batch * K * world / (ms_max * 1e-3), 1),
+        "roofline": roofline, "e2e": e2e, "gpu_launches": 2 * K, "clocks": clk.summary(),
+    }
+    return res, insts
+
+
+def oracle_lla_sample(w, inp, budget_s):
+    """Times the float64 LLA oracle on whole (sequence, query head) pairs;
+    returns (GB/s of their K+V, seconds, pairs, description)."""
+    import oracle
+    B, Hq, Hkv = w.batch, w.num_q_heads, w.num_kv_heads
+    g = Hq // Hkv
+    pairs = [(b, h) for b in range(B) for h in range(Hq)]
+    np.random.default_rng(0).shuffle(pairs)
+    q = inp["q"].double().cpu().numpy()
+    secs, nbytes, done = 0.0, 0, 0
+    for b, h in pairs:
+        K = inp["k_cache"][b, h // g].double().cpu().numpy()
+        V = inp["v_cache"][b, h // g].double().cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.lla_query(q[b, h], K, V, w.scale, 0.0)
+        secs += time.perf_counter() - t0
+        nbytes += K.shape[0] * 2 * w.head_dim * 2
+        done += 1
+        if secs >= budget_s:
+            break
+    desc = (f"{done} of {len(pairs)} (sequence, query head) pairs of {w.name} ({nbytes / 2**20:.1f} MiB of K+V), "
+            "float64 numpy LLA oracle (explicit S_KK, S_KV, numpy.linalg.solve)")
+    return nbytes / secs / 1e9, secs, done, desc
+
+
 # ----------------------------------------------------------------- prefill
 
 def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
@@ -834,6 +977,10 @@ def cpu_baseline(w, inp, budget_s):
         return cpu_baseline_prefill_paged(w, inp, budget_s)
     if w.name == "prefill_train":
         return cpu_baseline_prefill_train(w, inp, budget_s)
+    if w.name == "lla_decode":
+        gbs, secs, done, desc = oracle_lla_sample(w, inp, budget_s)
+        return {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                "sample": desc, "seconds": round(secs, 2)}
     gbs, secs, done, desc = oracle_decode_sample(w, inp, budget_s)
     return {"value": round(gbs, 4), "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
             "sample": desc, "seconds": round(secs, 2)}
@@ -945,7 +1092,8 @@ def reference_arm(args, w, rank, world):
             sub_w = w if inp["q"].shape[0] == w.batch else W.DecodeWorkload(
                 w.name, inp["q"].shape[0], w.num_q_heads, w.num_kv_heads, w.head_dim, w.kv_len,
                 dtype=w.dtype, paged=w.paged, min_len=w.min_len, hidden=w.hidden)
-            v, secs, _, desc = oracle_decode_sample(sub_w, inp, budget)
+            sample = oracle_lla_sample if w.name == "lla_decode" else oracle_decode_sample
+            v, secs, _, desc = sample(sub_w, inp, budget)
         if i >= args.warmup:
             vals.append(v)
             secs_all += secs
@@ -976,7 +1124,7 @@ def _host_decode_sample(w):
 # own roofline, clocks and oracle baseline (the four other configurations of
 # the method's targets first, then the serving and training steps beyond them).
 PER_CONFIG = ("decode_f32", "decode_long", "decode_paged", "prefill", "prefill_paged", "prefill_train",
-              "decode_projected")
+              "decode_projected", "lla_decode")
 NOMINAL_PEAKS = {"GB/s": 8000.0, "TFLOP/s": 2250.0}   # B200 HBM3e and dense bf16, NVIDIA's figures
 
 
@@ -989,6 +1137,9 @@ def run_workload(args, w, rank, world, dev, peaks, kind):
         return bench_prefill_train(args, w, rank, world, dev, peaks, kind)
     if w.hidden:
         res, inp = bench_decode_projected(args, w, rank, world, dev, peaks, kind)
+        return res, inp[0]
+    if w.name == "lla_decode":
+        res, inp = bench_lla(args, w, rank, world, dev, peaks, kind)
         return res, inp[0]
     res, inp = bench_decode(args, w, rank, world, dev, peaks, kind)
     return res, inp[0]

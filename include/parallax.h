@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define PARALLAX_ABI_VERSION 5
+#define PARALLAX_ABI_VERSION 6
 
 typedef enum plx_status {
   PLX_OK = 0,
@@ -60,6 +60,7 @@ typedef enum plx_dtype { PLX_F32 = 0, PLX_BF16 = 1 } plx_dtype;
 #define PLX_DEVERR_BAD_PAGE   1   /* page_table entry outside [0, num_pages)     */
 #define PLX_DEVERR_TIMEOUT    2   /* an mbarrier / pipeline wait gave up         */
 #define PLX_DEVERR_BAD_LENGTH 4   /* a sequence length outside its allowed range */
+#define PLX_DEVERR_SINGULAR   8   /* LLA: S_KK + ridge I not positive definite     */
 
 /* ------------------------------------------------------------------------
  * Decode: one new query per (sequence, query head) over its KV cache.
@@ -188,6 +189,59 @@ plx_status parallax_decode_noalloc(const void* q, const void* rho,
                                    const void* k_cache, const void* v_cache,
                                    const int32_t* page_table, const int32_t* seq_lens,
                                    void* out, const plx_decode_params* p, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Local Linear Attention (LLA) with the solved probe, decode form.
+ *
+ * LLA is the local linear estimate at the query: the intercept of the
+ * softmax-weighted least-squares fit v ~ a + M^T (k - q) (newx.sg page,
+ * section "Abstract": softmax attention's local constant estimate upgraded
+ * to a local linear one; wispaper.ai blog, section "Context: Why Softmax is
+ * Not Enough": LLA solves a linear system for every token).  It is Parallax
+ * with the probe solved instead of learned:
+ *     (S_KK + ridge I) rho* = kbar - q,     out = vbar - S_KV^T rho*,
+ *     S_KK = sum_i w_i (k_i - kbar)(k_i - kbar)^T,
+ * with w, kbar, vbar and S_KV as in the definition at the top.  `ridge`
+ * (>= 0, finite) penalises the slope M; the pages name no regularisation,
+ * and 0 is plain LLA, which needs more effectively weighted keys than d.
+ * The pages solve by conjugate gradients; here each query head's system is
+ * formed in fp32 and solved exactly by a Cholesky factorisation.
+ *
+ * Two launches on `stream`: a single pass over each query head's K and V
+ * that accumulates sum w k k^T and sum w k v^T on the tensor cores (with
+ * the first moments), then one solve per query head that also writes out.
+ *
+ *   q            device bf16 [B, Hq, 128].
+ *   k_cache,     device bf16, contiguous [B, Hkv, L, 128] or paged pools
+ *   v_cache      [P, Hkv, 64, 128], with page_table / seq_lens exactly as
+ *                for parallax_decode (a sequence of length 0 gets out = 0
+ *                and rho* = 0).
+ *   rho          device float32 [B, Hq, 128]: the solved probe, or NULL.
+ *   out          device [B, Hq, 128] of out_dtype.  Neither out nor rho may
+ *                overlap q or each other (PLX_ERR_INVALID_ARG).
+ *   workspace    device, >= parallax_lla_decode_workspace_size() bytes,
+ *                256-byte aligned; no initialisation needed.
+ *   p            as parallax_decode; in_dtype PLX_BF16 and head_dim 128
+ *                (else PLX_ERR_UNSUPPORTED).  num_ctas 0 picks how many
+ *                pieces each query head's keys are cut into (one CTA each);
+ *                num_ctas > 0 asks for about that many CTAs in total.
+ * A query head whose factorisation meets a pivot that is not positive
+ * (S_KK + ridge I not numerically positive definite, e.g. ridge 0 and one
+ * key) sets PLX_DEVERR_SINGULAR and gets rho* = 0, out = vbar.  With ridge 0
+ * and fewer effectively weighted keys than d the system is ill-posed even
+ * when every pivot is positive: pass ridge > 0 for short sequences.  Other
+ * errors as parallax_decode. */
+
+/* Workspace bytes of parallax_lla_decode for these parameters on a device
+ * with `num_sms` SMs (<= 0: the current device), or (size_t)-1 for invalid
+ * ones: 132 KB per (query head, piece) -- the two d x d sums, the first
+ * moments, the running max and the normaliser. */
+size_t parallax_lla_decode_workspace_size(const plx_decode_params* p, float ridge, int32_t num_sms);
+
+plx_status parallax_lla_decode(const void* q, const void* k_cache, const void* v_cache,
+                               const int32_t* page_table, const int32_t* seq_lens, float ridge,
+                               float* rho, void* out, void* workspace, size_t workspace_bytes,
+                               const plx_decode_params* p, cudaStream_t stream);
 
 /* ------------------------------------------------------------------------
  * Prefill: every position of a sequence is a query; causal (key i visible

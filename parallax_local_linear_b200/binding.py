@@ -27,7 +27,7 @@ lib = ctypes.CDLL(LIB_PATH)
 PLX_F32, PLX_BF16 = 0, 1
 STATUS = {0: "PLX_OK", 1: "PLX_ERR_INVALID_ARG", 2: "PLX_ERR_UNSUPPORTED", 3: "PLX_ERR_WORKSPACE",
           4: "PLX_ERR_CUDA", 5: "PLX_ERR_DEVICE_FAULT", 6: "PLX_ERR_TIMEOUT"}
-DEVERR_BAD_PAGE, DEVERR_TIMEOUT, DEVERR_BAD_LENGTH = 1, 2, 4
+DEVERR_BAD_PAGE, DEVERR_TIMEOUT, DEVERR_BAD_LENGTH, DEVERR_SINGULAR = 1, 2, 4, 8
 PAGE_SIZE = 64
 
 
@@ -86,6 +86,11 @@ lib.parallax_decode_projected.argtypes = [_vp, _vp, _vp, ctypes.c_int32, _vp, _v
 lib.parallax_decode_projected.restype = ctypes.c_int
 lib.parallax_decode_noalloc.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, ctypes.POINTER(DecodeParams), _vp]
 NOALLOC_SCRATCH_BYTES = 8 << 20
+lib.parallax_lla_decode_workspace_size.restype = ctypes.c_size_t
+lib.parallax_lla_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams), ctypes.c_float, ctypes.c_int32]
+lib.parallax_lla_decode.restype = ctypes.c_int
+lib.parallax_lla_decode.argtypes = [_vp, _vp, _vp, _i32p, _i32p, ctypes.c_float, _vp, _vp, _vp, ctypes.c_size_t,
+                                    ctypes.POINTER(DecodeParams), _vp]
 lib.parallax_set_wait_limit_ns.restype = ctypes.c_int
 lib.parallax_set_wait_limit_ns.argtypes = [ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64)]
 lib.parallax_last_device_error.restype = ctypes.c_int
@@ -343,6 +348,38 @@ def decode_noalloc(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_
     if st != 0:
         raise ParallaxError(st, "parallax_decode_noalloc")
     return out
+
+
+def lla_decode(q, k_cache, v_cache, scale=None, ridge=0.0, *, seq_lens=None, page_table=None, out=None,
+               out_dtype=None, rho_out=None, num_ctas=0, kv_len=None):
+    """Local Linear Attention with the solved probe (decode).
+
+    Per (sequence, query head): rho* solves (S_KK + ridge I) rho* = kbar - q
+    and out = vbar - S_KV^T rho*.  q: [B, Hq, 128] bf16; caches as in
+    ``decode`` (bf16).  Returns (out [B, Hq, 128] in ``out_dtype``, default
+    bf16; rho* [B, Hq, 128] float32, written into ``rho_out`` when given).
+    """
+    _check_decode_inputs(q, q, k_cache, v_cache, seq_lens, page_table, kv_len)
+    if q.dtype != torch.bfloat16:
+        raise TypeError("lla_decode takes bfloat16 queries and caches")
+    out, out_dtype = _output(out, out_dtype, q.shape, torch.bfloat16, q.device)
+    if rho_out is None:
+        rho_out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    _check_cuda("rho_out", rho_out, torch.float32)
+    if tuple(rho_out.shape) != tuple(q.shape):
+        raise ValueError(f"rho_out must have shape {tuple(q.shape)}")
+    p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale, out_dtype=out_dtype,
+                      num_ctas=num_ctas)
+    nbytes = lib.parallax_lla_decode_workspace_size(ctypes.byref(p), float(ridge), 0)
+    if nbytes == SIZE_MAX:
+        raise ParallaxError(1, "parallax_lla_decode_workspace_size")
+    ws = _workspace(q.device, nbytes)
+    st = lib.parallax_lla_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table), _ptr(seq_lens),
+                                 float(ridge), _ptr(rho_out), _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                                 ctypes.byref(p), _stream_ptr(q.device))
+    if st != 0:
+        raise ParallaxError(st, "parallax_lla_decode")
+    return out, rho_out
 
 
 def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):

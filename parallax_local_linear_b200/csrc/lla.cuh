@@ -1,0 +1,576 @@
+// Local Linear Attention (LLA) with the solved probe, decode form, sm_100a.
+//
+// LLA is the local linear estimate at the query: the intercept of the
+// softmax-weighted least-squares fit v ~ a + M^T (k - q) (newx.sg page
+// "Parallax: Parameterized Local Linear Attention for Language Modeling",
+// section "Abstract"; the wispaper.ai blog "Parallax: Breaking the Boundary
+// Bias with Parameterized Local Linear Attention", section "Context: Why
+// Softmax is Not Enough", where LLA solves a linear system for every token).
+// With weights w_i = softmax(scale q.k_i), kbar = sum w k, vbar = sum w v,
+//     S_KK = sum w (k - kbar)(k - kbar)^T,  S_KV = sum w (k - kbar)(v - vbar)^T,
+//     (S_KK + ridge I) rho* = kbar - q,       out = vbar - S_KV^T rho*,
+// the same output as Parallax with the probe solved instead of learned.
+// `ridge` penalises the slope (the pages name no regularisation; 0 is plain
+// LLA).
+//
+// Two kernels per call:
+//
+//   lla_moments_kernel  one CTA per (sequence, query head, piece of its keys):
+//     a single pass over the piece's K and V tiles accumulates, relative to
+//     a running max m (2^(s - m) weights, rescaled lazily as in the prefill),
+//         l = sum e,  ks = sum e k,  vs = sum e v,
+//         D_KK = sum e k k^T,  D_KV = sum e k v^T          (128 x 128 each)
+//     The two d x d sums are dense contractions over the keys and run on the
+//     tensor cores: D += A . B with A = (e o K)^T, 128 x 16 keys per step,
+//     written by the compute warps into tensor memory (thread a holds
+//     column a of the tile: e_i k_ia for its 64 keys, packed bf16 pairs),
+//     and B = the K or V tile in shared memory (keys x 128, MN-major).  For
+//     sequences shorter than kLlaSplitLen the bf16 rounding of e o K is not
+//     averaged away (the solve amplifies it along directions the few keys do
+//     not span), so a second product adds its lo part (x = hi + lo).
+//     The piece's record goes to the workspace.
+//
+//   lla_solve_kernel  one CTA per (sequence, query head): merges the pieces
+//     like online softmax (weights 2^(m_j - M)), forms S_KK + ridge I and
+//     kbar - q in fp32, solves by Cholesky, and writes rho* and
+//         out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a,
+//     which is vbar - S_KV^T rho* (S_KV = D_KV / l - kbar vbar^T).
+#pragma once
+
+#include "ptx.cuh"
+#include "decode.cuh"    // kTile (64-token tiles and pages)
+#include "prefill.cuh"   // tc_mma_ts4
+
+namespace plx {
+
+constexpr int kLlaD = 128;
+constexpr int kLlaStages = 4;            // K and V ring depth (tiles)
+constexpr int kLlaThreads = 192;         // TMA producer warp, MMA warp, four compute warps
+constexpr int kLlaCompute = 128;
+constexpr int kLlaSplitLen = 1024;       // shorter sequences add the lo part of e o K
+constexpr float kLlaRescaleLog2 = 8.f;   // lazy rescale threshold (factor 256)
+constexpr int kLlaMaxPieces = 16;
+// Record of one piece: D_KK, D_KV (row-major [a][b]), ks, vs, then m, l.
+constexpr int kLlaRecKK = 0;
+constexpr int kLlaRecKV = kLlaD * kLlaD;
+constexpr int kLlaRecKs = 2 * kLlaD * kLlaD;
+constexpr int kLlaRecVs = kLlaRecKs + kLlaD;
+constexpr int kLlaRecM = kLlaRecVs + kLlaD;
+constexpr int kLlaRecFloats = kLlaRecM + 16;
+
+#define PLX_DEVERR_SINGULAR_BIT 8   // PLX_DEVERR_SINGULAR in parallax.h
+
+struct LlaArgs {
+  const __nv_bfloat16* q;          // [B, Hq, D]
+  const int32_t* page_table;       // [B, max_pages] or null (contiguous)
+  const int32_t* seq_lens;         // [B] or null (every sequence kv_len)
+  float* rec;                      // [B * Hq * pieces][kLlaRecFloats]
+  void* out;                       // [B, Hq, D] of out dtype
+  float* rho;                      // [B, Hq, D] or null
+  int B, Hq, Hkv, group, kv_len, paged, num_pages, max_pages, pieces;
+  float scale_log2, ridge;
+  int out_bf16;
+  unsigned long long wait_ns;      // limit of one pipeline wait
+};
+
+struct LlaLayout {
+  static constexpr int kTileBytes = kTile * kLlaD * 2;   // 16 KB: two 64-column boxes of 64 rows
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kLlaStages * kTileBytes;
+  static constexpr int kQ = kV + kLlaStages * kTileBytes;   // float [128]: q * scale * log2(e)
+  static constexpr int kE = kQ + kLlaD * 4;                 // float [64]: weights of the tile
+  static constexpr int kRed = kE + kTile * 4;               // float [4 warps][2]
+  static constexpr int kBar = kRed + 64;
+  // full[S], empty[S], a_full[2], a_free[2], acc_done, drain
+  static constexpr int kNumBars = 2 * kLlaStages + 6;
+  static constexpr int kMisc = kBar + kNumBars * 8;         // tmem base, abort flag
+  static constexpr int kBytes = kMisc + 16 + 1024;          // + alignment slack
+};
+
+// TMEM columns: D_KK [0, 128), D_KV [128, 256); A buffer b: hi words at
+// 256 + 64 b, lo words at 288 + 64 b (keys 2c, 2c+1 in word c).
+constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128;
+__device__ __forceinline__ uint32_t lla_col_a(int buf) { return 256u + 64u * buf; }
+
+__device__ __forceinline__ int lla_seq_len(const LlaArgs& a, int b) {
+  if (a.seq_lens == nullptr) return a.kv_len;
+  int n = __ldg(a.seq_lens + b);
+  if (n < 0 || n > a.kv_len) {
+    report_error(4 /* PLX_DEVERR_BAD_LENGTH */);
+    n = n < 0 ? 0 : a.kv_len;
+  }
+  return n;
+}
+
+__global__ void __launch_bounds__(kLlaThreads, 1)
+    lla_moments_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                       const LlaArgs a) {
+  using Ly = LlaLayout;
+  constexpr int S = kLlaStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
+  uint64_t* empty = full + S;
+  uint64_t* a_full = empty + S;
+  uint64_t* a_free = a_full + 2;
+  uint64_t* acc_done = a_free + 2;
+  uint64_t* drain = acc_done + 1;
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::kMisc + 4);
+  float* q_s = reinterpret_cast<float*>(sm + Ly::kQ);
+  float* e_s = reinterpret_cast<float*>(sm + Ly::kE);
+  float* red_s = reinterpret_cast<float*>(sm + Ly::kRed);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int piece = blockIdx.x % a.pieces;
+  const int bh = blockIdx.x / a.pieces;
+  const int b = bh / a.Hq, h = bh % a.Hq, kvh = h / a.group;
+  float* rec = a.rec + (size_t)blockIdx.x * kLlaRecFloats;
+  const int len = lla_seq_len(a, b);
+  const int tiles = (len + kTile - 1) / kTile;
+  const int t0 = (int)((long long)piece * tiles / a.pieces);
+  const int n = (int)((long long)(piece + 1) * tiles / a.pieces) - t0;
+  if (n == 0) {   // no keys in this piece: an empty record
+    if (threadIdx.x == 0) {
+      rec[kLlaRecM] = -INFINITY;
+      rec[kLlaRecM + 1] = 0.f;
+    }
+    return;
+  }
+  const int32_t* pt = a.paged ? a.page_table + (size_t)b * a.max_pages : nullptr;
+  if (a.paged) {   // every page this piece reads must lie in the pool
+    bool bad = false;
+    for (int i = threadIdx.x; i < n; i += kLlaThreads) {
+      const int pg = __ldg(pt + t0 + i);
+      bad |= pg < 0 || pg >= a.num_pages;
+    }
+    if (__syncthreads_or(bad)) {
+      if (threadIdx.x == 0) {
+        report_error(1 /* PLX_DEVERR_BAD_PAGE */);
+        rec[kLlaRecM] = -INFINITY;
+        rec[kLlaRecM + 1] = 0.f;
+      }
+      return;
+    }
+  }
+  const bool split_lo = len < kLlaSplitLen;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], kLlaCompute);
+      mbar_init(&a_free[i], 1);
+    }
+    mbar_init(acc_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (threadIdx.x < kLlaD)
+    q_s[threadIdx.x] = __bfloat162float(a.q[(size_t)bh * kLlaD + threadIdx.x]) * a.scale_log2;
+  if (warp == 1) {
+    tmem_alloc(tmem_base_s, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_s;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_k);
+      prefetch_tmap(&tm_v);
+      const uint64_t pol = l2_policy_evict_first();
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int s = j % S;
+        if (j >= S && !mbar_wait_bounded(a.wait_ns, &empty[s], ((j / S) - 1) & 1)) {
+          *abort_flag = 1;
+          break;
+        }
+        if (*abort_flag) break;
+        const int tile = t0 + j;
+        const int row = a.paged ? (__ldg(pt + tile) * a.Hkv + kvh) * kTile   // page ids checked above
+                                : (b * a.Hkv + kvh) * a.kv_len + tile * kTile;
+        mbar_arrive_expect_tx(&full[s], 2 * Ly::kTileBytes);
+        for (int bx = 0; bx < 2; ++bx) {
+          tma_load_2d(sm + Ly::kK + s * Ly::kTileBytes + bx * (Ly::kTileBytes / 2), &tm_k, bx * 64, row,
+                      &full[s], pol);
+          tma_load_2d(sm + Ly::kV + s * Ly::kTileBytes + bx * (Ly::kTileBytes / 2), &tm_v, bx * 64, row,
+                      &full[s], pol);
+        }
+        ++issued;
+      }
+      // Every issued load must land before the CTA exits.
+      for (int s = 0; s < S && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / S) * S;
+        mbar_wait_drain(&full[s], (last / S) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    // D_KK += A . K and D_KV += A . V, A = (e o K)^T from tensor memory
+    // (128 x 16 keys per step), K and V MN-major from shared memory.
+    constexpr uint32_t kId = idesc_bf16(128, kLlaD, true);
+    const uint64_t dk = smem_desc_sw128(smem_u32(sm + Ly::kK), Ly::kTileBytes / 2, 1024);
+    const uint64_t dv = smem_desc_sw128(smem_u32(sm + Ly::kV), Ly::kTileBytes / 2, 1024);
+    auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
+    };
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
+      const int s = j % S, buf = j & 1;
+      if (!(ok = wait_warp(&full[s], (j / S) & 1))) break;
+      if (!(ok = wait_warp(&a_full[buf], (j >> 1) & 1))) break;
+      tc_fence_after();
+      const uint64_t ks = dk + (uint64_t)((s * Ly::kTileBytes) >> 4);
+      const uint64_t vs = dv + (uint64_t)((s * Ly::kTileBytes) >> 4);
+      const uint32_t ahi = tmem + lla_col_a(buf);
+#pragma unroll
+      for (int kk = 0; kk < 4; kk += 2) {   // 16 keys per step: 8 A words, 16 B rows (2048 bytes)
+        const uint64_t o0 = (uint64_t)(kk * 128), o1 = o0 + 128;
+        tc_mma_ts4(tmem + kLlaColKK, ahi + 8u * kk, ks + o0, tmem + kLlaColKV, ahi + 8u * kk, vs + o0,
+                   tmem + kLlaColKK, ahi + 8u * (kk + 1), ks + o1, tmem + kLlaColKV, ahi + 8u * (kk + 1), vs + o1,
+                   kId, (j > 0 || kk > 0) ? 1u : 0u, 1u);
+      }
+      if (split_lo) {
+#pragma unroll
+        for (int kk = 0; kk < 4; kk += 2) {
+          const uint64_t o0 = (uint64_t)(kk * 128), o1 = o0 + 128;
+          const uint32_t alo = ahi + 32u;
+          tc_mma_ts4(tmem + kLlaColKK, alo + 8u * kk, ks + o0, tmem + kLlaColKV, alo + 8u * kk, vs + o0,
+                     tmem + kLlaColKK, alo + 8u * (kk + 1), ks + o1, tmem + kLlaColKV, alo + 8u * (kk + 1),
+                     vs + o1, kId, 1u, 1u);
+        }
+      }
+      tc_commit(&a_free[buf]);
+      tc_commit(&empty[s]);
+      tc_commit(acc_done);
+    }
+    if (!ok && lane == 0) *abort_flag = 1;
+    // Every issued MMA must complete before tensor memory is released.
+    tc_commit(drain);
+    __syncwarp();
+    mbar_wait_drain(drain, 0);
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ compute
+    const int c = threadIdx.x - 64;            // 0..127
+    const int cw = warp - 2;                   // compute warp 0..3
+    const int wq = warp & 3;                   // TMEM lane quarter of this warp
+    const int row = wq * 32 + lane;            // this thread's column of K / V = TMEM lane of D
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const int ki = c >> 1, hf = c & 1;         // score phase: key, half of the head dim
+    // this thread's column in a swizzled tile: box, 16-byte chunk, element
+    const int cbox = row >> 6, cch = (row & 63) >> 3, cel = row & 7;
+    float m_ref = -INFINITY, l_acc = 0.f, ksum = 0.f, vsum = 0.f;
+    bool fine = true;
+    int j = 0;
+    for (; j < n; ++j) {
+      const int s = j % S, buf = j & 1;
+      const bool w = !*abort_flag && mbar_wait_bounded(a.wait_ns, &full[s], (j / S) & 1);
+      if (!bar_and(1, kLlaCompute, w && fine)) {
+        fine = false;
+        break;
+      }
+      uint8_t* kt = sm + Ly::kK + s * Ly::kTileBytes;
+      uint8_t* vt = sm + Ly::kV + s * Ly::kTileBytes;
+      const int nvalid = min(kTile, len - (t0 + j) * kTile);
+      // ---- scaled score of key ki: half hf of q . k
+      float dot = 0.f;
+      {
+        const uint8_t* krow = kt + hf * (Ly::kTileBytes / 2) + ki * 128;
+        const float* qh = q_s + 64 * hf;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 v4 = *reinterpret_cast<const uint4*>(krow + ((ch ^ (ki & 7)) << 4));
+          const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            dot = fmaf(qh[8 * ch + 2 * e], bf16_lo_f(w4[e]), dot);
+            dot = fmaf(qh[8 * ch + 2 * e + 1], bf16_hi_f(w4[e]), dot);
+          }
+        }
+      }
+      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      const float sc = ki < nvalid ? dot : -INFINITY;
+      const float wmax = warp_max(sc);
+      if (lane == 0) red_s[cw] = wmax;
+      bar_and(2, kLlaCompute, true);
+      const float tmax = fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3]));
+      // ---- running max; rescale D, ks, vs, l when it grows past the threshold
+      bool rescale = false;
+      float alpha = 1.f;
+      if (j == 0) {
+        m_ref = tmax;   // the piece's first tile holds a key: tmax is finite
+      } else if (tmax > m_ref + kLlaRescaleLog2) {
+        alpha = ex2(m_ref - tmax);
+        m_ref = tmax;
+        rescale = true;
+      }
+      if (rescale) {   // uniform: every compute thread saw the same maxima
+        const bool wd = mbar_wait_bounded(a.wait_ns, acc_done, (j - 1) & 1);   // D holds tiles < j
+        if (!bar_and(3, kLlaCompute, wd)) {
+          fine = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll 1
+        for (int part = 0; part < 8; ++part) {   // D_KK then D_KV, 32 columns at a time
+          uint32_t r[32];
+          const uint32_t addr = tmem + lane_off + (uint32_t)(part * 32);
+          tmem_ld32(addr, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(addr, r);
+        }
+        tmem_wait_st();
+        l_acc *= alpha;
+        ksum *= alpha;
+        vsum *= alpha;
+      }
+      const float e = ki < nvalid ? ex2(sc - m_ref) : 0.f;
+      if (hf == 0) {
+        e_s[ki] = e;
+        l_acc += e;
+      }
+      // The A buffer is free once the products of tile j - 2 are done.
+      const bool wa = j < 2 || mbar_wait_bounded(a.wait_ns, &a_free[buf], ((j >> 1) - 1) & 1);
+      if (!bar_and(2, kLlaCompute, wa)) {   // also publishes e_s
+        fine = false;
+        break;
+      }
+      // ---- A = (e o K)^T: this thread's column, 64 keys as 32 bf16 pairs (hi, lo)
+      uint32_t hi[32], lo[32];
+      {
+        const uint8_t* kc = kt + cbox * (Ly::kTileBytes / 2) + cel * 2;
+        const uint8_t* vc = vt + cbox * (Ly::kTileBytes / 2) + cel * 2;
+#pragma unroll
+        for (int p = 0; p < 32; ++p) {
+          const int i0 = 2 * p, i1 = 2 * p + 1;
+          const bool v0 = i0 < nvalid, v1 = i1 < nvalid;   // rows past the end may hold NaN: select
+          const int o0 = i0 * 128 + ((cch ^ (i0 & 7)) << 4), o1 = i1 * 128 + ((cch ^ (i1 & 7)) << 4);
+          const float k0 = v0 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kc + o0)) : 0.f;
+          const float k1 = v1 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kc + o1)) : 0.f;
+          const float x0 = v0 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vc + o0)) : 0.f;
+          const float x1 = v1 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vc + o1)) : 0.f;
+          const float e0 = e_s[i0], e1 = e_s[i1];
+          const float p0 = e0 * k0, p1 = e1 * k1;
+          ksum += p0 + p1;
+          vsum = fmaf(e0, x0, fmaf(e1, x1, vsum));
+          hi[p] = pack_bf16(p0, p1);
+          lo[p] = pack_bf16(p0 - bf16_lo_f(hi[p]), p1 - bf16_hi_f(hi[p]));
+        }
+      }
+      tmem_st32(tmem + lane_off + lla_col_a(buf), hi);
+      if (split_lo) tmem_st32(tmem + lane_off + lla_col_a(buf) + 32u, lo);
+      if (nvalid < kTile) {
+        // Rows past the end are B operands of the products (their A entries are
+        // 0, but 0 * NaN is not): zero them in K and V.  No thread reads them
+        // after the scores above.
+        for (int i = c; i < (kTile - nvalid) * 16; i += kLlaCompute) {
+          const int r = nvalid + (i >> 4), cc = i & 15;   // cc: box (cc >> 3), chunk (cc & 7)
+          const int off = (cc >> 3) * (Ly::kTileBytes / 2) + r * 128 + (cc & 7) * 16;
+          *reinterpret_cast<uint4*>(kt + off) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(vt + off) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&a_full[buf]);
+    }
+    // ---- the piece's record: wait for the last products, then write
+    bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, acc_done, (n - 1) & 1);
+    wl = bar_and(3, kLlaCompute, wl);
+    const float lw = warp_sum(l_acc);
+    if (lane == 0) red_s[4 + cw] = lw;
+    bar_and(2, kLlaCompute, true);
+    if (wl) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int part = 0; part < 8; ++part) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + (uint32_t)(part * 32), r);
+        tmem_wait_ld();
+        float* dst = rec + (part < 4 ? kLlaRecKK : kLlaRecKV) + row * kLlaD + (part & 3) * 32;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                                          __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+      }
+      rec[kLlaRecKs + row] = ksum;
+      rec[kLlaRecVs + row] = vsum;
+      if (c == 0) {
+        rec[kLlaRecM] = m_ref;
+        rec[kLlaRecM + 1] = red_s[4] + red_s[5] + red_s[6] + red_s[7];
+      }
+    } else if (c == 0) {   // abandoned after a wait ran out (already reported): an empty record
+      rec[kLlaRecM] = -INFINITY;
+      rec[kLlaRecM + 1] = 0.f;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- solve
+// One CTA (256 threads) per (sequence, query head).
+constexpr int kLlaSolveThreads = 256;
+constexpr int kLlaLd = kLlaD + 1;   // padded row stride of the matrix in shared memory
+
+__global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaArgs a) {
+  extern __shared__ float smf[];
+  float* A = smf;                          // [128][129]: S_KK + ridge I, then its Cholesky factor
+  float* kb = A + kLlaD * kLlaLd;          // kbar
+  float* vb = kb + kLlaD;                  // vbar
+  float* y = vb + kLlaD;                   // right-hand side, then rho*
+  float* piv = y + kLlaD;                  // diagonal of the factor
+  float* part = piv + kLlaD;               // [2][128] partial matrix-vector products
+  float* wts = part + 2 * kLlaD;           // [kLlaMaxPieces] piece weights 2^(m_j - M)
+  float* misc = wts + kLlaMaxPieces;       // [0] l, [1] kbar . rho*, [2] singular flag
+
+  const int tid = threadIdx.x;
+  const int bh = blockIdx.x, b = bh / a.Hq;
+  const size_t orow = (size_t)bh * kLlaD;
+  const int len = lla_seq_len(a, b);
+  auto store_out = [&](int i, float v) {
+    if (a.out_bf16)
+      reinterpret_cast<__nv_bfloat16*>(a.out)[orow + i] = __float2bfloat16_rn(v);
+    else
+      reinterpret_cast<float*>(a.out)[orow + i] = v;
+  };
+  if (len == 0) {   // no keys: out = 0, rho* = 0
+    if (tid < kLlaD) {
+      store_out(tid, 0.f);
+      if (a.rho) a.rho[orow + tid] = 0.f;
+    }
+    return;
+  }
+  const float* rec0 = a.rec + (size_t)bh * a.pieces * kLlaRecFloats;
+  if (tid == 0) {
+    float M = -INFINITY;
+    for (int p = 0; p < a.pieces; ++p) {
+      const float* r = rec0 + (size_t)p * kLlaRecFloats;
+      if (r[kLlaRecM + 1] > 0.f) M = fmaxf(M, r[kLlaRecM]);
+    }
+    float L = 0.f;
+    for (int p = 0; p < a.pieces; ++p) {
+      const float* r = rec0 + (size_t)p * kLlaRecFloats;
+      const float w = r[kLlaRecM + 1] > 0.f ? ex2(r[kLlaRecM] - M) : 0.f;
+      wts[p] = w;
+      L += w * r[kLlaRecM + 1];
+    }
+    misc[0] = L;
+    misc[2] = 0.f;
+  }
+  __syncthreads();
+  const float L = misc[0];
+  const float invL = 1.f / L;
+  if (tid < kLlaD) {
+    float ks = 0.f, vs = 0.f;
+    for (int p = 0; p < a.pieces; ++p) {
+      if (wts[p] == 0.f) continue;
+      const float* r = rec0 + (size_t)p * kLlaRecFloats;
+      ks = fmaf(wts[p], r[kLlaRecKs + tid], ks);
+      vs = fmaf(wts[p], r[kLlaRecVs + tid], vs);
+    }
+    kb[tid] = ks * invL;
+    vb[tid] = vs * invL;
+  }
+  __syncthreads();
+  for (int idx = tid; idx < kLlaD * kLlaD; idx += kLlaSolveThreads) {
+    const int i = idx >> 7, jj = idx & (kLlaD - 1);
+    float d = 0.f;
+    for (int p = 0; p < a.pieces; ++p)
+      if (wts[p] != 0.f) d = fmaf(wts[p], rec0[(size_t)p * kLlaRecFloats + kLlaRecKK + idx], d);
+    A[i * kLlaLd + jj] = fmaf(d, invL, -kb[i] * kb[jj]) + (i == jj ? a.ridge : 0.f);
+  }
+  if (tid < kLlaD) y[tid] = kb[tid] - __bfloat162float(a.q[orow + tid]);
+
+  // ---- Cholesky, lower: column k of the factor is A[i][k] / piv[k] (i >= k)
+  const int ti = tid >> 4, tj = tid & 15;
+  bool bad = false;
+  for (int k = 0; k < kLlaD; ++k) {
+    __syncthreads();
+    const float akk = A[k * kLlaLd + k];
+    if (!(akk > 0.f) || !isfinite(akk)) {   // not numerically positive definite (uniform)
+      bad = true;
+      break;
+    }
+    const float dk = sqrtf(akk), inv = 1.f / dk;
+    if (tid == 0) piv[k] = dk;
+    for (int i = k + 1 + ti; i < kLlaD; i += 16) {
+      const float lik = A[i * kLlaLd + k] * inv;
+      for (int jj = k + 1 + tj; jj <= i; jj += 16) A[i * kLlaLd + jj] -= lik * (A[jj * kLlaLd + k] * inv);
+    }
+  }
+  __syncthreads();
+  if (bad) {
+    if (tid == 0) report_error(PLX_DEVERR_SINGULAR_BIT);
+    if (tid < kLlaD) {   // rho* = 0: the output falls back to vbar
+      store_out(tid, vb[tid]);
+      if (a.rho) a.rho[orow + tid] = 0.f;
+    }
+    return;
+  }
+  // ---- forward (L z = y) and back (L^T rho = z) substitution, one warp
+  if (tid < 32) {
+    for (int k = 0; k < kLlaD; ++k) {
+      const float zk = y[k] / piv[k];
+      __syncwarp();
+      if (tid == 0) y[k] = zk;
+      for (int i = k + 1 + tid; i < kLlaD; i += 32) y[i] -= (A[i * kLlaLd + k] / piv[k]) * zk;
+      __syncwarp();
+    }
+    for (int k = kLlaD - 1; k >= 0; --k) {
+      const float xk = y[k] / piv[k];
+      __syncwarp();
+      if (tid == 0) y[k] = xk;
+      for (int jj = tid; jj < k; jj += 32) y[jj] -= (A[k * kLlaLd + jj] / piv[jj]) * xk;
+      __syncwarp();
+    }
+    float kr = 0.f;
+    for (int i = tid; i < kLlaD; i += 32) kr = fmaf(kb[i], y[i], kr);
+    kr = warp_sum(kr);
+    if (tid == 0) misc[1] = kr;
+  }
+  __syncthreads();
+  // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a
+  {
+    const int col = tid & (kLlaD - 1), half = tid >> 7;
+    float acc = 0.f;
+    for (int p = 0; p < a.pieces; ++p) {
+      if (wts[p] == 0.f) continue;
+      const float* dkv = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV;
+      float sp = 0.f;
+      for (int r = half * 64; r < half * 64 + 64; ++r) sp = fmaf(dkv[r * kLlaD + col], y[r], sp);
+      acc = fmaf(wts[p], sp, acc);
+    }
+    part[half * kLlaD + col] = acc;
+  }
+  __syncthreads();
+  if (tid < kLlaD) {
+    const float corr = (part[tid] + part[kLlaD + tid]) * invL;
+    store_out(tid, fmaf(vb[tid], 1.f + misc[1], -corr));
+    if (a.rho) a.rho[orow + tid] = y[tid];
+  }
+}
+
+constexpr int lla_solve_smem_bytes() {
+  return (kLlaD * kLlaLd + 4 * kLlaD + 2 * kLlaD + kLlaMaxPieces + 4) * 4;
+}
+
+}  // namespace plx

@@ -19,6 +19,7 @@
 #include "prefill.cuh"
 #include "prefill_bwd.cuh"
 #include "project.cuh"
+#include "lla.cuh"
 
 namespace {
 
@@ -528,6 +529,33 @@ plx_status noalloc_scratch(void** out) {
   return PLX_OK;
 }
 
+// ------------------------------------------------ LLA with the solved probe
+plx_status validate_lla(const plx_decode_params* p, float ridge) {
+  plx_status st = validate_decode(p);
+  if (st != PLX_OK) return st;
+  if (!std::isfinite(ridge) || ridge < 0.f) return PLX_ERR_INVALID_ARG;
+  if (p->in_dtype != PLX_BF16 || p->head_dim != kLlaD) return PLX_ERR_UNSUPPORTED;
+  if ((int64_t)p->batch * p->num_q_heads * kLlaMaxPieces >= (int64_t)INT32_MAX) return PLX_ERR_UNSUPPORTED;
+  return PLX_OK;
+}
+
+// Pieces each query head's keys are cut into: enough CTAs to fill the SMs
+// (or num_ctas of them), at least four tiles per piece.
+int lla_pieces(const plx_decode_params* p, int num_sms) {
+  const int64_t heads = (int64_t)p->batch * p->num_q_heads;
+  const int64_t want = p->num_ctas > 0 ? p->num_ctas : num_sms;
+  int64_t k = want / heads;
+  const int64_t tiles = ((int64_t)p->kv_len + kTile - 1) / kTile;
+  if (k > tiles / 4) k = tiles / 4;
+  if (k > kLlaMaxPieces) k = kLlaMaxPieces;
+  if (k < 1) k = 1;
+  return (int)k;
+}
+
+size_t lla_workspace_bytes(const plx_decode_params* p, int pieces) {
+  return (size_t)p->batch * p->num_q_heads * pieces * kLlaRecFloats * sizeof(float);
+}
+
 }  // namespace
 
 extern "C" {
@@ -722,6 +750,78 @@ plx_status parallax_set_wait_limit_ns(uint64_t limit_ns, uint64_t* previous) {
   g_wait_ns[dev] = limit_ns;
   g_wait_set[dev] = true;
   return PLX_OK;
+}
+
+size_t parallax_lla_decode_workspace_size(const plx_decode_params* p, float ridge, int32_t num_sms) {
+  if (validate_lla(p, ridge) != PLX_OK) return (size_t)-1;
+  if (num_sms <= 0) num_sms = current_device_sms();
+  if (num_sms <= 0) return (size_t)-1;
+  return lla_workspace_bytes(p, lla_pieces(p, num_sms));
+}
+
+plx_status parallax_lla_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* page_table,
+                               const int32_t* seq_lens, float ridge, float* rho, void* out, void* workspace,
+                               size_t workspace_bytes, const plx_decode_params* p, cudaStream_t stream) {
+  plx_status st = validate_lla(p, ridge);
+  if (st != PLX_OK) return st;
+  if (!q || !k_cache || !v_cache || !out) return PLX_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      (rho && !aligned(rho, 16)))
+    return PLX_ERR_INVALID_ARG;
+  const bool paged = p->page_size != 0;
+  if (paged && (page_table == nullptr || seq_lens == nullptr)) return PLX_ERR_INVALID_ARG;
+  if (!paged && page_table != nullptr) return PLX_ERR_INVALID_ARG;
+  if ((page_table && !aligned(page_table, 4)) || (seq_lens && !aligned(seq_lens, 4))) return PLX_ERR_INVALID_ARG;
+  // The solve writes out and rho while other CTAs still read q.
+  const size_t heads = (size_t)p->batch * p->num_q_heads;
+  const size_t q_bytes = heads * kLlaD * 2, out_bytes = heads * kLlaD * (p->out_dtype == PLX_BF16 ? 2 : 4),
+               rho_bytes = heads * kLlaD * 4;
+  if (overlaps(out, out_bytes, q, q_bytes)) return PLX_ERR_INVALID_ARG;
+  if (rho && (overlaps(rho, rho_bytes, q, q_bytes) || overlaps(rho, rho_bytes, out, out_bytes)))
+    return PLX_ERR_INVALID_ARG;
+  const int num_sms = current_device_sms();
+  if (num_sms <= 0) return PLX_ERR_CUDA;
+  const int pieces = lla_pieces(p, num_sms);
+  if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < lla_workspace_bytes(p, pieces))
+    return PLX_ERR_WORKSPACE;
+
+  LlaArgs a{};
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.rec = static_cast<float*>(workspace);
+  a.out = out;
+  a.rho = rho;
+  a.B = p->batch;
+  a.Hq = p->num_q_heads;
+  a.Hkv = p->num_kv_heads;
+  a.group = p->num_q_heads / p->num_kv_heads;
+  a.kv_len = p->kv_len;
+  a.paged = paged ? 1 : 0;
+  a.num_pages = paged ? p->num_pages : 0;
+  a.max_pages = paged ? p->max_pages_per_seq : 0;
+  a.pieces = pieces;
+  a.scale_log2 = p->scale * 1.4426950408889634f;
+  a.ridge = ridge;
+  a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
+  a.wait_ns = current_wait_ns();
+  if (p->kv_len > 0) {   // kv_len 0: every sequence is empty and the solve writes zeros
+    const uint64_t rows = paged ? (uint64_t)p->num_pages * p->num_kv_heads * kTile
+                                : (uint64_t)p->batch * p->num_kv_heads * p->kv_len;
+    CUtensorMap tk, tv;
+    if (!make_tmap_bf16(&tk, k_cache, kLlaD, rows, 64, kTile) || !make_tmap_bf16(&tv, v_cache, kLlaD, rows, 64, kTile))
+      return PLX_ERR_CUDA;
+    constexpr int smem = LlaLayout::kBytes;
+    if (cudaFuncSetAttribute(lla_moments_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      return PLX_ERR_CUDA;
+    lla_moments_kernel<<<(unsigned)(heads * pieces), kLlaThreads, smem, stream>>>(tk, tv, a);
+    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+  }
+  constexpr int ssmem = lla_solve_smem_bytes();
+  if (cudaFuncSetAttribute(lla_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ssmem) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  lla_solve_kernel<<<(unsigned)heads, kLlaSolveThreads, ssmem, stream>>>(a);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
 plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code) {

@@ -13,6 +13,8 @@ Named workloads (head_dim d, Hq query heads, Hkv KV heads):
   decode_long    B=64,  Hq=32, Hkv=8, d=128, L=32768, keys offset per KV head
   decode_paged   128 sequences, L ~ U{512..65536}, Hq=16, Hkv=4, d=128,
                  64-token pages placed by a seeded permutation
+  lla_decode     decode_bf16's inputs through Local Linear Attention with the
+                 solved probe (ridge 0)
   prefill        B=4, H=16, T=8192, d=128, causal, rho scaled by 0.1
   prefill_train  the same shapes, forward for training plus backward, with
                  dL/dout ~ N(0, 1)
@@ -101,6 +103,8 @@ WORKLOADS = {
     "decode_long": DecodeWorkload("decode_long", 64, 32, 8, 128, 32768, key_offset_std=0.5, seed=3),
     "decode_paged": DecodeWorkload("decode_paged", 128, 16, 4, 128, 65536, paged=True,
                                    min_len=512, seed=4),
+    # decode_bf16's cache and queries through Local Linear Attention with the solved probe
+    "lla_decode": DecodeWorkload("lla_decode", 8, 16, 8, 128, 4096, seed=2),
     "prefill": PrefillWorkload("prefill", 4, 16, 8192, 128, seed=5),
     "prefill_train": PrefillWorkload("prefill_train", 4, 16, 8192, 128, seed=5),
     "prefill_paged": ChunkedPrefillWorkload("prefill_paged", 8, 16, 4, 128, 1024, 4096, 8192, seed=6),
@@ -437,3 +441,17 @@ def prefill_backward_flops(w: PrefillWorkload) -> int:
     pass over each product the gradients need (S, A, D = g.v, dQ, dR, dV and
     the two dK products, 2*d each)."""
     return 2 * prefill_flops(w)
+
+
+def lla_decode_flops(w: DecodeWorkload, seq_lens=None) -> int:
+    """Algorithmic FLOP of one LLA decode call: per (sequence, query head)
+    with n keys, the scores (2*d*n), the two d x d weighted sums
+    sum e k k^T and sum e k v^T (2 * 2*d*d*n), the first moments (2 * 2*d*n),
+    the Cholesky factorisation and two triangular solves (d^3/3 + 2*d^2)
+    and the output's matrix-vector product (2*d*d)."""
+    d = w.head_dim
+    lens = [w.kv_len] * w.batch if seq_lens is None else [int(x) for x in seq_lens]
+    per_key = 2 * d + 4 * d * d + 4 * d
+    per_head = d ** 3 // 3 + 4 * d * d
+    return sum(w.num_q_heads * (n * per_key + (per_head if n else 0)) for n in lens)
+
