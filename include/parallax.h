@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define PARALLAX_ABI_VERSION 6
+#define PARALLAX_ABI_VERSION 7
 
 typedef enum plx_status {
   PLX_OK = 0,
@@ -126,6 +126,36 @@ plx_status parallax_decode(const void* q, const void* rho,
                            const int32_t* page_table, const int32_t* seq_lens,
                            void* out, void* workspace, size_t workspace_bytes,
                            const plx_decode_params* p, cudaStream_t stream);
+
+/* Prepared decode: the validation, work plan, kernel arguments and TMA
+ * descriptors of one parallax_decode call, kept for repeated launches on
+ * the same buffers (a serving loop that decodes into fixed q / rho / out
+ * buffers over a resident cache pays the host-side preparation once).
+ *
+ * parallax_decode_plan_create takes exactly the arguments of
+ * parallax_decode, minus the stream, checks them as parallax_decode does
+ * and returns a host-allocated plan in *plan (NULL on error).  The plan
+ * keeps the pointers, not the data: every buffer must stay allocated, at the
+ * same address, for the plan's lifetime, and the contents (q, rho, the
+ * cache, page_table, seq_lens) are read at each run.  The workspace follows
+ * parallax_decode's rule (counter region zero before the first run; every
+ * completed run leaves it zero); runs that share a workspace must not
+ * overlap on the GPU.  The plan is bound to the device current at creation
+ * (PLX_ERR_INVALID_ARG if another device is current at a run) and to the
+ * pipeline wait limit in force then.
+ *
+ * parallax_decode_plan_run launches the decode on `stream` (one launch,
+ * asynchronous); parallax_decode_plan_destroy frees the plan (NULL is a
+ * no-op).  Host-only otherwise: no CUDA allocation. */
+typedef struct plx_decode_plan plx_decode_plan;
+
+plx_status parallax_decode_plan_create(const void* q, const void* rho,
+                                      const void* k_cache, const void* v_cache,
+                                      const int32_t* page_table, const int32_t* seq_lens,
+                                      void* out, void* workspace, size_t workspace_bytes,
+                                      const plx_decode_params* p, plx_decode_plan** plan);
+plx_status parallax_decode_plan_run(const plx_decode_plan* plan, cudaStream_t stream);
+void parallax_decode_plan_destroy(plx_decode_plan* plan);
 
 /* Decode whose query and probe are projected from the new token's layer
  * input in the same call.

@@ -91,6 +91,13 @@ lib.parallax_lla_decode_workspace_size.argtypes = [ctypes.POINTER(DecodeParams),
 lib.parallax_lla_decode.restype = ctypes.c_int
 lib.parallax_lla_decode.argtypes = [_vp, _vp, _vp, _i32p, _i32p, ctypes.c_float, _vp, _vp, _vp, ctypes.c_size_t,
                                     ctypes.POINTER(DecodeParams), _vp]
+lib.parallax_decode_plan_create.restype = ctypes.c_int
+lib.parallax_decode_plan_create.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _vp, _vp, ctypes.c_size_t,
+                                            ctypes.POINTER(DecodeParams), ctypes.POINTER(ctypes.c_void_p)]
+lib.parallax_decode_plan_run.restype = ctypes.c_int
+lib.parallax_decode_plan_run.argtypes = [_vp, _vp]
+lib.parallax_decode_plan_destroy.restype = None
+lib.parallax_decode_plan_destroy.argtypes = [_vp]
 lib.parallax_set_wait_limit_ns.restype = ctypes.c_int
 lib.parallax_set_wait_limit_ns.argtypes = [ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64)]
 lib.parallax_last_device_error.restype = ctypes.c_int
@@ -281,6 +288,50 @@ def decode(q, rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=No
     if st != 0:
         raise ParallaxError(st, "parallax_decode")
     return out
+
+
+class DecodePlan:
+    """A prepared decode over fixed buffers (parallax_decode_plan_*).
+
+    Checks and prepares ``decode(q, rho, k_cache, v_cache, ..., out=out)``
+    once; each ``run()`` is one kernel launch on the current stream that
+    reads the buffers' current contents.  The plan keeps references to every
+    tensor it was made from (so they stay allocated at the same address) and
+    owns a zeroed workspace of its own.  Runs of one plan must not overlap on
+    the GPU (they share that workspace).
+    """
+
+    def __init__(self, q, rho, k_cache, v_cache, scale=None, *, out, seq_lens=None, page_table=None, num_ctas=0,
+                 kv_len=None):
+        _check_decode_inputs(q, rho, k_cache, v_cache, seq_lens, page_table, kv_len)
+        out, out_dtype = _output(out, None, q.shape, q.dtype, q.device)
+        p = decode_params(q, k_cache, page_table=page_table, kv_len=kv_len, scale=scale, out_dtype=out_dtype,
+                          num_ctas=num_ctas)
+        nbytes = decode_workspace_size(p)
+        ws = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+        handle = ctypes.c_void_p()
+        st = lib.parallax_decode_plan_create(_ptr(q), _ptr(rho), _ptr(k_cache), _ptr(v_cache), _ptr(page_table),
+                                             _ptr(seq_lens), _ptr(out), _ptr(ws), ws.numel(), ctypes.byref(p),
+                                             ctypes.byref(handle))
+        if st != 0:
+            raise ParallaxError(st, "parallax_decode_plan_create")
+        self._handle = handle
+        self._keep = (q, rho, k_cache, v_cache, seq_lens, page_table, ws)
+        self.out = out
+        self._device = q.device
+        self._run = lib.parallax_decode_plan_run
+
+    def run(self):
+        st = self._run(self._handle, ctypes.c_void_p(torch.cuda.current_stream(self._device).cuda_stream))
+        if st != 0:
+            raise ParallaxError(st, "parallax_decode_plan_run")
+        return self.out
+
+    def __del__(self):
+        h = getattr(self, "_handle", None)
+        if h is not None and h.value:
+            lib.parallax_decode_plan_destroy(h)
+            self._handle = None
 
 
 def decode_projected(x, w_q, w_rho, k_cache, v_cache, scale=None, *, seq_lens=None, page_table=None,

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -17,6 +18,7 @@
 #include "ptx.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill2.cuh"
 #include "prefill_bwd.cuh"
 #include "project.cuh"
 #include "lla.cuh"
@@ -186,9 +188,10 @@ size_t decode_smem_bytes(const plx_decode_params* p) {
 // consumers wait for it before reading q and rho).
 template <int D, int STAGES, bool kLoInPad>
 plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int ctas,
-                            size_t smem, cudaStream_t stream, bool pdl) {
+                            size_t smem, cudaStream_t stream, bool pdl, bool set_attr) {
   auto kern = decode_tc_kernel<D, STAGES, kDecodeNC, kLoInPad>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  if (set_attr &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
   if (a.cluster <= 1 && !pdl) {
     kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
@@ -230,9 +233,10 @@ plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CU
 }
 
 template <int D>
-plx_status launch_decode_f32(const DecodeArgs& a, int ctas, size_t smem, cudaStream_t stream) {
+plx_status launch_decode_f32(const DecodeArgs& a, int ctas, size_t smem, cudaStream_t stream, bool set_attr) {
   auto kern = decode_f32_kernel<D, kDecodeF32Warps>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+  if (set_attr &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
   kern<<<ctas, kDecodeF32Warps * 32, smem, stream>>>(a);
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
@@ -315,7 +319,10 @@ plx_status prepare_decode(const void* q, const void* rho, const void* k_cache, c
   return PLX_OK;
 }
 
-plx_status launch_decode(const DecodeLaunch& L, const plx_decode_params* p, cudaStream_t stream, bool pdl) {
+// `set_attr`: set the kernel's dynamic shared-memory limit first (a prepared
+// plan did that once when it was made).
+plx_status launch_decode(const DecodeLaunch& L, const plx_decode_params* p, cudaStream_t stream, bool pdl,
+                         bool set_attr = true) {
   const DecodeArgs& a = L.a;
   const int D = p->head_dim;
   if (L.empty) {
@@ -325,14 +332,40 @@ plx_status launch_decode(const DecodeLaunch& L, const plx_decode_params* p, cuda
                : PLX_ERR_CUDA;
   }
   if (p->in_dtype == PLX_F32)
-    return D == 64 ? launch_decode_f32<64>(a, L.pl.ctas, L.smem, stream)
-                   : launch_decode_f32<128>(a, L.pl.ctas, L.smem, stream);
+    return D == 64 ? launch_decode_f32<64>(a, L.pl.ctas, L.smem, stream, set_attr)
+                   : launch_decode_f32<128>(a, L.pl.ctas, L.smem, stream, set_attr);
   const bool pad = a.group <= kMaxGroup / 2;
   if (D == 64)
-    return pad ? launch_decode_tc<64, kDecodeStages64, true>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl)
-               : launch_decode_tc<64, kDecodeStages64, false>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl);
-  return pad ? launch_decode_tc<128, kDecodeStages128, true>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl)
-             : launch_decode_tc<128, kDecodeStages128, false>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl);
+    return pad ? launch_decode_tc<64, kDecodeStages64, true>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl, set_attr)
+               : launch_decode_tc<64, kDecodeStages64, false>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl,
+                                                               set_attr);
+  return pad ? launch_decode_tc<128, kDecodeStages128, true>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl, set_attr)
+             : launch_decode_tc<128, kDecodeStages128, false>(a, L.tk, L.tv, L.pl.ctas, L.smem, stream, pdl,
+                                                              set_attr);
+}
+
+// Sets the dynamic shared-memory limit of the kernel a launch will use.
+plx_status set_decode_attr(const DecodeLaunch& L, const plx_decode_params* p) {
+  if (L.empty) return PLX_OK;
+  const int smem = (int)L.smem;
+  cudaError_t e;
+  const bool pad = L.a.group <= kMaxGroup / 2;
+  if (p->in_dtype == PLX_F32)
+    e = p->head_dim == 64 ? cudaFuncSetAttribute(decode_f32_kernel<64, kDecodeF32Warps>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+                          : cudaFuncSetAttribute(decode_f32_kernel<128, kDecodeF32Warps>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  else if (p->head_dim == 64)
+    e = pad ? cudaFuncSetAttribute(decode_tc_kernel<64, kDecodeStages64, kDecodeNC, true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+            : cudaFuncSetAttribute(decode_tc_kernel<64, kDecodeStages64, kDecodeNC, false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  else
+    e = pad ? cudaFuncSetAttribute(decode_tc_kernel<128, kDecodeStages128, kDecodeNC, true>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
+            : cudaFuncSetAttribute(decode_tc_kernel<128, kDecodeStages128, kDecodeNC, false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
 // q and rho projections of a projected decode (project.cuh).
@@ -365,6 +398,8 @@ plx_status launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tr, c
   return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
+// Dense prefill: the two-CTA kernel (prefill2.cuh), 256 query rows per
+// cluster of two SMs.
 plx_status launch_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,
                           const plx_prefill_params* p, cudaStream_t stream, float* vbar = nullptr,
                           float2* stats = nullptr) {
@@ -373,7 +408,7 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   const uint64_t rows_kv = (uint64_t)p->batch * hkv * p->seq_len;
   CUtensorMap tq, tr, tk, tv;
   if (!make_tmap_bf16(&tq, q, kPfD, rows_q, 64, kPfBM) || !make_tmap_bf16(&tr, rho, kPfD, rows_q, 64, kPfBM) ||
-      !make_tmap_bf16(&tk, k, kPfD, rows_kv, 64, kPfBN) || !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBN))
+      !make_tmap_bf16(&tk, k, kPfD, rows_kv, 64, kPfBN / 2) || !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBN))
     return PLX_ERR_CUDA;
   PrefillArgs a{};
   a.B = p->batch;
@@ -381,7 +416,7 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   a.Hkv = hkv;
   a.T = p->seq_len;
   a.group = p->num_heads / hkv;
-  a.n_mblk = (p->seq_len + kPfBM - 1) / kPfBM;
+  a.n_mblk = (p->seq_len + 2 * kPfBM - 1) / (2 * kPfBM);   // pairs of 128-row tiles
   a.causal = p->causal;
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
   a.scale_log2 = p->scale * 1.4426950408889634f;
@@ -389,7 +424,12 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   a.wait_ns = current_wait_ns();
   a.vbar = vbar;
   a.stats = stats;
-  return launch_prefill_kernel<false>(tq, tr, tk, tv, a, stream);
+  constexpr int smem = P2Layout::kBytes;
+  if (cudaFuncSetAttribute(prefill_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return PLX_ERR_CUDA;
+  const long long grid = 2LL * a.n_mblk * a.B * a.H;
+  prefill_tc2_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
 plx_status validate_prefill(const plx_prefill_params* p) {
@@ -558,6 +598,14 @@ size_t lla_workspace_bytes(const plx_decode_params* p, int pieces) {
 
 }  // namespace
 
+// A validated decode call whose kernel arguments and tensor maps are kept
+// for repeated launches (parallax_decode_plan_*).
+struct plx_decode_plan {
+  DecodeLaunch L;
+  plx_decode_params p;
+  int device;
+};
+
 extern "C" {
 
 int32_t parallax_abi_version(void) { return PARALLAX_ABI_VERSION; }
@@ -599,6 +647,37 @@ plx_status parallax_decode(const void* q, const void* rho, const void* k_cache, 
   if (st != PLX_OK) return st;
   return launch_decode(L, p, stream, false);
 }
+
+plx_status parallax_decode_plan_create(const void* q, const void* rho, const void* k_cache, const void* v_cache,
+                                      const int32_t* page_table, const int32_t* seq_lens, void* out,
+                                      void* workspace, size_t workspace_bytes, const plx_decode_params* p,
+                                      plx_decode_plan** plan) {
+  if (plan == nullptr) return PLX_ERR_INVALID_ARG;
+  *plan = nullptr;
+  plx_decode_plan* P = new (std::nothrow) plx_decode_plan;
+  if (P == nullptr) return PLX_ERR_CUDA;
+  plx_status st =
+      prepare_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, workspace, workspace_bytes, p, &P->L);
+  if (st == PLX_OK && cudaGetDevice(&P->device) != cudaSuccess) st = PLX_ERR_CUDA;
+  if (st == PLX_OK) st = set_decode_attr(P->L, p);
+  if (st != PLX_OK) {
+    delete P;
+    return st;
+  }
+  P->p = *p;
+  *plan = P;
+  return PLX_OK;
+}
+
+plx_status parallax_decode_plan_run(const plx_decode_plan* plan, cudaStream_t stream) {
+  if (plan == nullptr) return PLX_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PLX_ERR_CUDA;
+  if (dev != plan->device) return PLX_ERR_INVALID_ARG;
+  return launch_decode(plan->L, &plan->p, stream, false, false);
+}
+
+void parallax_decode_plan_destroy(plx_decode_plan* plan) { delete plan; }
 
 plx_status parallax_decode_projected(const void* x, const void* w_q, const void* w_rho, int32_t hidden,
                                      const void* k_cache, const void* v_cache, const int32_t* page_table,

@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(binding):
 
 
 def test_abi_version_and_status_strings(binding):
-    assert binding.lib.parallax_abi_version() == 6
+    assert binding.lib.parallax_abi_version() == 7
     for code, name in binding.STATUS.items():
         assert binding.lib.parallax_status_string(code).decode() == name
 
@@ -279,3 +279,16 @@ def test_decode_binding_checks_cache_shapes_before_any_launch(binding):
     lens = torch.zeros((2,), dtype=torch.int32)
     with pytest.raises(ValueError, match="kv_len"):
         binding.decode(q, q, pool, pool, seq_lens=lens, page_table=table, kv_len=4 * 64 + 1)
+
+
+def test_decode_plan_rejects_bad_arguments_before_any_launch(binding):
+    p = _params(binding)
+    handle = ctypes.c_void_p(1234)
+    st = binding.lib.parallax_decode_plan_create(None, None, None, None, None, None, None, None, 0,
+                                                 ctypes.byref(p), ctypes.byref(handle))
+    assert st == 1 and not handle.value   # the plan pointer is cleared on error
+    bad = _params(binding, batch=0)
+    assert binding.lib.parallax_decode_plan_create(None, None, None, None, None, None, None, None, 0,
+                                                   ctypes.byref(bad), ctypes.byref(handle)) == 1
+    assert binding.lib.parallax_decode_plan_run(None, None) == 1
+    binding.lib.parallax_decode_plan_destroy(None)   # a no-op

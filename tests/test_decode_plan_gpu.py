@@ -1,0 +1,77 @@
+"""The prepared decode (parallax_decode_plan_*) against the one-shot call.
+
+A plan made from fixed buffers must give, at every run, bit for bit what
+parallax_decode gives on the buffers' current contents: it reuses the
+validated arguments and tensor maps, not any data.  parallax_decode itself is
+checked against the float64 oracle in test_decode_gpu.py; one case here is
+checked against the oracle directly as well.
+"""
+
+import pytest
+import torch
+
+from parallax_local_linear_b200 import workloads as W
+from tests.helpers import TOL_BF16, assert_parity, oracle_heads
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def px():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from parallax_local_linear_b200 import binding
+    return binding
+
+
+def _cuda(inp):
+    return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+
+
+CASES = {
+    "cluster_grid": dict(args=(8, 16, 8, 128, 4096), kw={}, ctas=0),
+    "workspace_merge": dict(args=(4, 8, 2, 128, 3000), kw=dict(seq_lens=[3000, 1200, 65, 0]), ctas=5),
+    "paged": dict(args=(3, 16, 4, 128, 2500), kw=dict(seq_lens=[2500, 700, 64], paged=True), ctas=7),
+    "f32": dict(args=(2, 4, 2, 64, 1000), kw=dict(dtype="f32"), ctas=3),
+}
+
+
+@pytest.mark.parametrize("case", sorted(CASES))
+def test_plan_runs_match_the_one_shot_call(px, case):
+    c = CASES[case]
+    inp = _cuda(W.small_decode_inputs(*c["args"], seed=61, **c["kw"]))
+    out = torch.empty_like(inp["q"])
+    plan = px.DecodePlan(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"], out=out,
+                         seq_lens=inp.get("seq_lens"), page_table=inp.get("page_table"), num_ctas=c["ctas"])
+    for step in range(3):
+        if step == 2:   # new contents in the same buffers: the plan reads them at the run
+            inp["q"].copy_(torch.randn_like(inp["q"].float()).to(inp["q"].dtype))
+        plan.run()
+        ref = px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"],
+                        seq_lens=inp.get("seq_lens"), page_table=inp.get("page_table"), num_ctas=c["ctas"])
+        assert torch.equal(out, ref), f"{case} step {step}"
+    assert px.last_device_error() == 0
+
+
+def test_plan_against_the_oracle(px):
+    inp = _cuda(W.small_decode_inputs(2, 8, 2, 128, 777, seed=62))
+    out = torch.empty(inp["q"].shape, dtype=torch.bfloat16, device="cuda")
+    plan = px.DecodePlan(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"], out=out)
+    plan.run()
+    ref = oracle_heads(inp, [(b, h) for b in range(2) for h in range(8)])
+    assert_parity(out.float().cpu().numpy(), ref, TOL_BF16, "plan")
+
+
+def test_plan_in_a_cuda_graph(px):
+    inp = _cuda(W.small_decode_inputs(4, 8, 4, 128, 2048, seed=63))
+    out = torch.empty_like(inp["q"])
+    plan = px.DecodePlan(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"], out=out)
+    plan.run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        plan.run()
+    out.zero_()
+    g.replay()
+    ref = px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"])
+    assert torch.equal(out, ref)

@@ -3,8 +3,9 @@
 Rows of the CUDA output are compared with the oracle's explicit two-pass
 definition over keys 0..t (causal) or all keys, on the same seeded inputs:
     max |gpu - ref| <= 2e-2 * (1 + |ref|)   (bf16 inputs, fp32 accumulation).
-Lengths cover one row, partial and full 64-key and 128-row tiles and ragged
-tails; the full B=4, H=16, T=8192 workload is checked on sampled rows.
+Lengths cover one row, partial and full 64-key tiles, the 128-row tile of
+each CTA and the 256 rows of each two-CTA cluster, and ragged tails; the full
+B=4, H=16, T=8192 workload is checked on 512 sampled rows.
 """
 
 import numpy as np
@@ -51,7 +52,7 @@ def _rows(B, H, T, limit=None, seed=0):
     return rows
 
 
-@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 128, 129, 200, 1000])
+@pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 128, 129, 200, 255, 256, 257, 383, 1000])
 def test_causal_lengths(px, T):
     inp = _cuda(W.small_prefill_inputs(1, 2, T, 128, seed=T))
     out = _run(px, inp).cpu().numpy()
@@ -61,7 +62,7 @@ def test_causal_lengths(px, T):
     assert_parity(got, ref, TOL_BF16, f"T={T}")
 
 
-@pytest.mark.parametrize("T", [1, 100, 300])
+@pytest.mark.parametrize("T", [1, 100, 300, 513])
 def test_non_causal(px, T):
     inp = _cuda(W.small_prefill_inputs(2, 2, T, 128, seed=7 + T))
     out = _run(px, inp, causal=False).cpu().numpy()
