@@ -58,12 +58,15 @@ METRIC = "decode KV GB/s & tokens/s (% of HBM peak); prefill TFLOP/s (% of bf16 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
     "decode": ["parallax_local_linear_b200/csrc/decode.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
-    "prefill": ["parallax_local_linear_b200/csrc/prefill.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "prefill": ["parallax_local_linear_b200/csrc/prefill2.cuh", "parallax_local_linear_b200/csrc/prefill.cuh",
+                "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "prefill_paged": ["parallax_local_linear_b200/csrc/prefill.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
     "prefill_bwd": ["parallax_local_linear_b200/csrc/prefill_bwd.cuh", "parallax_local_linear_b200/csrc/prefill.cuh",
                     "parallax_local_linear_b200/csrc/ptx.cuh"],
     "decode_projected": ["parallax_local_linear_b200/csrc/project.cuh", "parallax_local_linear_b200/csrc/decode.cuh",
                          "parallax_local_linear_b200/csrc/ptx.cuh"],
-    "lla": ["parallax_local_linear_b200/csrc/lla.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "lla": ["parallax_local_linear_b200/csrc/lla.cuh", "parallax_local_linear_b200/csrc/prefill.cuh",
+            "parallax_local_linear_b200/csrc/ptx.cuh"],
 }
 KV_COPIES = 4          # decode_bf16: 4 x 128 MiB of KV, more than L2
 GRAPH_STEPS = 64       # decode calls per captured graph
@@ -758,7 +761,7 @@ def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
         "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
                      "frac": round(achieved / peak, 4), **traffic_fields("prefill", w.name),
-                     "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_kernel",
+                     "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_tc2_kernel",
                      "algorithmic_flops_per_launch": flops},
         "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
     }
@@ -837,8 +840,8 @@ def bench_prefill_paged(args, w, rank, world, dev, peaks, peaks_kind):
                    "l2": f"q+rho {qr_mb:.0f} MB + KV pages {kv_mb:.0f} MB > 126 MB L2"},
         "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), **traffic_fields("prefill", w.name),
-                     "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_kernel (paged)",
+                     "frac": round(achieved / peak, 4), **traffic_fields("prefill_paged", w.name),
+                     "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_tc_kernel (paged)",
                      "algorithmic_flops_per_launch": flops},
         "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
     }

@@ -41,6 +41,8 @@
 #include "decode.cuh"    // kTile (64-token tiles and pages)
 #include "prefill.cuh"   // tc_mma_ts4
 
+#include <type_traits>
+
 namespace plx {
 
 constexpr int kLlaD = 128;
@@ -350,13 +352,20 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         fine = false;
         break;
       }
-      // ---- A = (e o K)^T: this thread's column, 64 keys as 32 bf16 pairs (hi, lo)
-      uint32_t hi[32], lo[32];
-      {
+      // ---- A = (e o K)^T: this thread's column, 64 keys as 32 bf16 pairs (hi,
+      // and lo for short sequences -- a separate instantiation, so that the
+      // long-sequence loop does not compute it)
+      auto form_a = [&](auto split_tag) {
+        constexpr bool kSplit = decltype(split_tag)::value;
         const uint8_t* kc = kt + cbox * (Ly::kTileBytes / 2) + cel * 2;
         const uint8_t* vc = vt + cbox * (Ly::kTileBytes / 2) + cel * 2;
+        const float2* e2s = reinterpret_cast<const float2*>(e_s);
 #pragma unroll
-        for (int p = 0; p < 32; ++p) {
+        for (int half = 0; half < 2; ++half) {   // keys 32 half .. 32 half + 31: words 16 half ..
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int pp = 0; pp < 16; ++pp) {
+          const int p = 16 * half + pp;
           const int i0 = 2 * p, i1 = 2 * p + 1;
           const bool v0 = i0 < nvalid, v1 = i1 < nvalid;   // rows past the end may hold NaN: select
           const int o0 = i0 * 128 + ((cch ^ (i0 & 7)) << 4), o1 = i1 * 128 + ((cch ^ (i1 & 7)) << 4);
@@ -364,16 +373,21 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
           const float k1 = v1 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kc + o1)) : 0.f;
           const float x0 = v0 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vc + o0)) : 0.f;
           const float x1 = v1 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vc + o1)) : 0.f;
-          const float e0 = e_s[i0], e1 = e_s[i1];
-          const float p0 = e0 * k0, p1 = e1 * k1;
+          const float2 e01 = e2s[p];
+          const float p0 = e01.x * k0, p1 = e01.y * k1;
           ksum += p0 + p1;
-          vsum = fmaf(e0, x0, fmaf(e1, x1, vsum));
-          hi[p] = pack_bf16(p0, p1);
-          lo[p] = pack_bf16(p0 - bf16_lo_f(hi[p]), p1 - bf16_hi_f(hi[p]));
+          vsum = fmaf(e01.x, x0, fmaf(e01.y, x1, vsum));
+          hi[pp] = pack_bf16(p0, p1);
+          if constexpr (kSplit) lo[pp] = pack_bf16(p0 - bf16_lo_f(hi[pp]), p1 - bf16_hi_f(hi[pp]));
         }
-      }
-      tmem_st32(tmem + lane_off + lla_col_a(buf), hi);
-      if (split_lo) tmem_st32(tmem + lane_off + lla_col_a(buf) + 32u, lo);
+        tmem_st16(tmem + lane_off + lla_col_a(buf) + 16u * half, hi);
+        if constexpr (kSplit) tmem_st16(tmem + lane_off + lla_col_a(buf) + 32u + 16u * half, lo);
+        }
+      };
+      if (split_lo)
+        form_a(std::true_type{});
+      else
+        form_a(std::false_type{});
       if (nvalid < kTile) {
         // Rows past the end are B operands of the products (their A entries are
         // 0, but 0 * NaN is not): zero them in K and V.  No thread reads them
@@ -427,20 +441,27 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
 }
 
 // ---------------------------------------------------------------- solve
-// One CTA (256 threads) per (sequence, query head).
+// One CTA (256 threads) per (sequence, query head).  Thread (bi, bj) of a
+// 16 x 16 grid holds the 8 x 8 block of S_KK + ridge I at rows 8 bi.., columns
+// 8 bj.. in registers (blocks on or below the diagonal; the others idle in
+// the factorisation).  Right-looking Cholesky, one column per step: the
+// column's owners publish it in shared memory, every thread updates its
+// block with the column's outer product.  The factor's columns are kept in
+// shared memory for the two triangular solves, which one warp runs with the
+// right-hand side in registers.
 constexpr int kLlaSolveThreads = 256;
-constexpr int kLlaLd = kLlaD + 1;   // padded row stride of the matrix in shared memory
+constexpr int kLlaLd = kLlaD + 1;   // padded row stride of the factor in shared memory
 
 __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaArgs a) {
   extern __shared__ float smf[];
-  float* A = smf;                          // [128][129]: S_KK + ridge I, then its Cholesky factor
-  float* kb = A + kLlaD * kLlaLd;          // kbar
+  float* Lm = smf;                         // [128][129]: column k of the factor, rows >= k
+  float* colb = Lm + kLlaD * kLlaLd;       // [2][128]: the current column, double-buffered
+  float* kb = colb + 2 * kLlaD;            // kbar
   float* vb = kb + kLlaD;                  // vbar
-  float* y = vb + kLlaD;                   // right-hand side, then rho*
-  float* piv = y + kLlaD;                  // diagonal of the factor
-  float* part = piv + kLlaD;               // [2][128] partial matrix-vector products
-  float* wts = part + 2 * kLlaD;           // [kLlaMaxPieces] piece weights 2^(m_j - M)
-  float* misc = wts + kLlaMaxPieces;       // [0] l, [1] kbar . rho*, [2] singular flag
+  float* rho_s = vb + kLlaD;               // rho*
+  float* part = rho_s + kLlaD;             // [8][128] partial matrix-vector products
+  float* wts = part + 8 * kLlaD;           // [kLlaMaxPieces] piece weights 2^(m_j - M)
+  float* misc = wts + kLlaMaxPieces;       // [0] l, [1] kbar . rho*
 
   const int tid = threadIdx.x;
   const int bh = blockIdx.x, b = bh / a.Hq;
@@ -474,11 +495,9 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
       L += w * r[kLlaRecM + 1];
     }
     misc[0] = L;
-    misc[2] = 0.f;
   }
   __syncthreads();
-  const float L = misc[0];
-  const float invL = 1.f / L;
+  const float invL = 1.f / misc[0];
   if (tid < kLlaD) {
     float ks = 0.f, vs = 0.f;
     for (int p = 0; p < a.pieces; ++p) {
@@ -491,30 +510,80 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     vb[tid] = vs * invL;
   }
   __syncthreads();
-  for (int idx = tid; idx < kLlaD * kLlaD; idx += kLlaSolveThreads) {
-    const int i = idx >> 7, jj = idx & (kLlaD - 1);
-    float d = 0.f;
-    for (int p = 0; p < a.pieces; ++p)
-      if (wts[p] != 0.f) d = fmaf(wts[p], rec0[(size_t)p * kLlaRecFloats + kLlaRecKK + idx], d);
-    A[i * kLlaLd + jj] = fmaf(d, invL, -kb[i] * kb[jj]) + (i == jj ? a.ridge : 0.f);
-  }
-  if (tid < kLlaD) y[tid] = kb[tid] - __bfloat162float(a.q[orow + tid]);
 
-  // ---- Cholesky, lower: column k of the factor is A[i][k] / piv[k] (i >= k)
-  const int ti = tid >> 4, tj = tid & 15;
+  // ---- this thread's block of S_KK + ridge I = D_KK / l - kbar kbar^T + ridge I
+  const int bi = tid >> 4, bj = tid & 15, r0 = 8 * bi, c0 = 8 * bj;
+  const bool active = bi >= bj;
+  float blk[8][8];
+#pragma unroll
+  for (int r = 0; r < 8; ++r)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) blk[r][c] = 0.f;
+  if (active) {
+    for (int p = 0; p < a.pieces; ++p) {
+      if (wts[p] == 0.f) continue;
+      const float* d = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKK + r0 * kLlaD + c0;
+      float4 v[8][2];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {   // all 16 loads in flight before any use
+        v[r][0] = *reinterpret_cast<const float4*>(d + r * kLlaD);
+        v[r][1] = *reinterpret_cast<const float4*>(d + r * kLlaD + 4);
+      }
+      const float w = wts[p];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        blk[r][0] = fmaf(w, v[r][0].x, blk[r][0]);
+        blk[r][1] = fmaf(w, v[r][0].y, blk[r][1]);
+        blk[r][2] = fmaf(w, v[r][0].z, blk[r][2]);
+        blk[r][3] = fmaf(w, v[r][0].w, blk[r][3]);
+        blk[r][4] = fmaf(w, v[r][1].x, blk[r][4]);
+        blk[r][5] = fmaf(w, v[r][1].y, blk[r][5]);
+        blk[r][6] = fmaf(w, v[r][1].z, blk[r][6]);
+        blk[r][7] = fmaf(w, v[r][1].w, blk[r][7]);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        blk[r][c] = fmaf(blk[r][c], invL, -kb[r0 + r] * kb[c0 + c]) + (r0 + r == c0 + c ? a.ridge : 0.f);
+  }
+
+  // ---- Cholesky: after step k, Lm[i][k] = L[i][k] for i >= k
   bool bad = false;
+#pragma unroll 1
   for (int k = 0; k < kLlaD; ++k) {
+    const int bc = k >> 3, cc = k & 7;
+    float* col = colb + (k & 1) * kLlaD;
+    if (active && bj == bc) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          if (c == cc) col[r0 + r] = blk[r][c];
+    }
     __syncthreads();
-    const float akk = A[k * kLlaLd + k];
+    const float akk = col[k];
     if (!(akk > 0.f) || !isfinite(akk)) {   // not numerically positive definite (uniform)
       bad = true;
       break;
     }
-    const float dk = sqrtf(akk), inv = 1.f / dk;
-    if (tid == 0) piv[k] = dk;
-    for (int i = k + 1 + ti; i < kLlaD; i += 16) {
-      const float lik = A[i * kLlaLd + k] * inv;
-      for (int jj = k + 1 + tj; jj <= i; jj += 16) A[i * kLlaLd + jj] -= lik * (A[jj * kLlaLd + k] * inv);
+    const float invd = 1.f / sqrtf(akk);
+    if (active && bj == bc) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+        if (r0 + r >= k) Lm[(r0 + r) * kLlaLd + k] = col[r0 + r] * invd;
+    }
+    if (active && bi >= bc && bj >= bc) {   // blocks that hold rows and columns past k
+      float li[8], lj[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) li[r] = r0 + r > k ? col[r0 + r] * invd : 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) lj[c] = c0 + c > k ? col[c0 + c] * invd : 0.f;
+#pragma unroll
+      for (int r = 0; r < 8; ++r)
+#pragma unroll
+        for (int c = 0; c < 8; ++c) blk[r][c] = fmaf(-li[r], lj[c], blk[r][c]);
     }
   }
   __syncthreads();
@@ -526,51 +595,86 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     }
     return;
   }
-  // ---- forward (L z = y) and back (L^T rho = z) substitution, one warp
+  // ---- L z = kbar - q, then L^T rho = z: one warp, rows lane + 32u in registers
   if (tid < 32) {
-    for (int k = 0; k < kLlaD; ++k) {
-      const float zk = y[k] / piv[k];
-      __syncwarp();
-      if (tid == 0) y[k] = zk;
-      for (int i = k + 1 + tid; i < kLlaD; i += 32) y[i] -= (A[i * kLlaLd + k] / piv[k]) * zk;
-      __syncwarp();
+    const int lane = tid;
+    float yv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) yv[u] = kb[lane + 32 * u] - __bfloat162float(a.q[orow + lane + 32 * u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll 1
+      for (int kk = 0; kk < 32; ++kk) {
+        const int k = 32 * u + kk;
+        const float zk = __shfl_sync(0xffffffffu, yv[u], kk) / Lm[k * kLlaLd + k];
+        if (lane == kk) yv[u] = zk;
+#pragma unroll
+        for (int v = u; v < 4; ++v) {
+          const int i = lane + 32 * v;
+          if (i > k) yv[v] = fmaf(-Lm[i * kLlaLd + k], zk, yv[v]);
+        }
+      }
     }
-    for (int k = kLlaD - 1; k >= 0; --k) {
-      const float xk = y[k] / piv[k];
-      __syncwarp();
-      if (tid == 0) y[k] = xk;
-      for (int jj = tid; jj < k; jj += 32) y[jj] -= (A[k * kLlaLd + jj] / piv[jj]) * xk;
-      __syncwarp();
+#pragma unroll
+    for (int u = 3; u >= 0; --u) {
+#pragma unroll 1
+      for (int kk = 31; kk >= 0; --kk) {
+        const int k = 32 * u + kk;
+        const float xk = __shfl_sync(0xffffffffu, yv[u], kk) / Lm[k * kLlaLd + k];
+        if (lane == kk) yv[u] = xk;
+#pragma unroll
+        for (int v = 0; v <= u; ++v) {
+          const int jj = lane + 32 * v;
+          if (jj < k) yv[v] = fmaf(-Lm[k * kLlaLd + jj], xk, yv[v]);
+        }
+      }
     }
     float kr = 0.f;
-    for (int i = tid; i < kLlaD; i += 32) kr = fmaf(kb[i], y[i], kr);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      rho_s[lane + 32 * u] = yv[u];
+      kr = fmaf(kb[lane + 32 * u], yv[u], kr);
+    }
     kr = warp_sum(kr);
-    if (tid == 0) misc[1] = kr;
+    if (lane == 0) misc[1] = kr;
   }
   __syncthreads();
   // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a
   {
-    const int col = tid & (kLlaD - 1), half = tid >> 7;
-    float acc = 0.f;
+    const int cq = tid & 31, rg = tid >> 5;   // columns 4 cq .. 4 cq + 3, rows rg + 8 u
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int p = 0; p < a.pieces; ++p) {
       if (wts[p] == 0.f) continue;
-      const float* dkv = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV;
-      float sp = 0.f;
-      for (int r = half * 64; r < half * 64 + 64; ++r) sp = fmaf(dkv[r * kLlaD + col], y[r], sp);
-      acc = fmaf(wts[p], sp, acc);
+      const float* dkv = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + 4 * cq;
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = *reinterpret_cast<const float4*>(dkv + (rg + 8 * u) * kLlaD);
+      float4 sp = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float r = rho_s[rg + 8 * u];
+        sp.x = fmaf(v[u].x, r, sp.x);
+        sp.y = fmaf(v[u].y, r, sp.y);
+        sp.z = fmaf(v[u].z, r, sp.z);
+        sp.w = fmaf(v[u].w, r, sp.w);
+      }
+      const float w = wts[p];
+      acc = make_float4(fmaf(w, sp.x, acc.x), fmaf(w, sp.y, acc.y), fmaf(w, sp.z, acc.z), fmaf(w, sp.w, acc.w));
     }
-    part[half * kLlaD + col] = acc;
+    *reinterpret_cast<float4*>(part + rg * kLlaD + 4 * cq) = acc;
   }
   __syncthreads();
   if (tid < kLlaD) {
-    const float corr = (part[tid] + part[kLlaD + tid]) * invL;
-    store_out(tid, fmaf(vb[tid], 1.f + misc[1], -corr));
-    if (a.rho) a.rho[orow + tid] = y[tid];
+    float corr = 0.f;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) corr += part[g * kLlaD + tid];
+    store_out(tid, fmaf(vb[tid], 1.f + misc[1], -corr * invL));
+    if (a.rho) a.rho[orow + tid] = rho_s[tid];
   }
 }
 
 constexpr int lla_solve_smem_bytes() {
-  return (kLlaD * kLlaLd + 4 * kLlaD + 2 * kLlaD + kLlaMaxPieces + 4) * 4;
+  return (kLlaD * kLlaLd + 2 * kLlaD + 3 * kLlaD + 8 * kLlaD + kLlaMaxPieces + 4) * 4;
 }
 
 }  // namespace plx
