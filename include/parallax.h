@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define PARALLAX_ABI_VERSION 7
+#define PARALLAX_ABI_VERSION 8
 
 typedef enum plx_status {
   PLX_OK = 0,
@@ -418,6 +418,13 @@ plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code);
  * a shorter limit to learn sooner that a kernel is stuck.  Host-only; takes
  * effect at the next launch.  Errors: PLX_ERR_CUDA (no current device). */
 plx_status parallax_set_wait_limit_ns(uint64_t limit_ns, uint64_t* previous);
+
+/* The CUDA error (a cudaError_t value) behind the last PLX_ERR_CUDA that a
+ * call on this host thread returned, or 0; reading it clears it. */
+int32_t parallax_last_cuda_error(void);
+
+/* CUDA's description of a cudaError_t value. */
+const char* parallax_cuda_error_string(int32_t code);
 
 /* Static string naming a status. */
 const char* parallax_status_string(plx_status s);

@@ -100,6 +100,10 @@ lib.parallax_decode_plan_destroy.restype = None
 lib.parallax_decode_plan_destroy.argtypes = [_vp]
 lib.parallax_set_wait_limit_ns.restype = ctypes.c_int
 lib.parallax_set_wait_limit_ns.argtypes = [ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint64)]
+lib.parallax_last_cuda_error.restype = ctypes.c_int32
+lib.parallax_last_cuda_error.argtypes = []
+lib.parallax_cuda_error_string.restype = ctypes.c_char_p
+lib.parallax_cuda_error_string.argtypes = [ctypes.c_int32]
 lib.parallax_last_device_error.restype = ctypes.c_int
 lib.parallax_last_device_error.argtypes = [_vp, ctypes.POINTER(ctypes.c_int32)]
 
@@ -109,7 +113,12 @@ SIZE_MAX = ctypes.c_size_t(-1).value
 class ParallaxError(RuntimeError):
     def __init__(self, status, what):
         self.status = status
-        super().__init__(f"{what}: {STATUS.get(status, status)}")
+        msg = f"{what}: {STATUS.get(status, status)}"
+        if status == 4:   # PLX_ERR_CUDA: name the CUDA error behind it
+            code = lib.parallax_last_cuda_error()
+            if code:
+                msg += f" ({lib.parallax_cuda_error_string(code).decode()}, cudaError {code})"
+        super().__init__(msg)
 
 
 def _dtype_code(dt):

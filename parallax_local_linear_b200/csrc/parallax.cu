@@ -56,6 +56,19 @@ unsigned long long current_wait_ns() {
 }
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+// The last CUDA error a call of this thread met (parallax_last_cuda_error).
+thread_local int g_last_cuda_error = 0;
+
+cudaError_t note(cudaError_t e) {
+  if (e != cudaSuccess) g_last_cuda_error = (int)e;
+  return e;
+}
+
+template <typename Kernel>
+cudaError_t set_smem(Kernel kern, int bytes) {
+  return note(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 // Do the byte ranges [a, a + na) and [b, b + nb) share a byte?
@@ -191,11 +204,11 @@ plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CU
                             size_t smem, cudaStream_t stream, bool pdl, bool set_attr) {
   auto kern = decode_tc_kernel<D, STAGES, kDecodeNC, kLoInPad>;
   if (set_attr &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      set_smem(kern, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
   if (a.cluster <= 1 && !pdl) {
     kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
-    return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+    return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas);
@@ -219,7 +232,7 @@ plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CU
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  if (cudaLaunchKernelEx(&cfg, kern, tk, tv, a) == cudaSuccess) return PLX_OK;
+  if (note(cudaLaunchKernelEx(&cfg, kern, tk, tv, a)) == cudaSuccess) return PLX_OK;
   (void)cudaGetLastError();
   if (a.cluster <= 1) return PLX_ERR_CUDA;
   // Clusters could not be scheduled (a launch-configuration error, which is
@@ -227,7 +240,7 @@ plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CU
   DecodeArgs b = a;
   b.cluster = 1;
   cfg.numAttrs = cluster_attr;
-  if (cudaLaunchKernelEx(&cfg, kern, tk, tv, b) == cudaSuccess) return PLX_OK;
+  if (note(cudaLaunchKernelEx(&cfg, kern, tk, tv, b)) == cudaSuccess) return PLX_OK;
   (void)cudaGetLastError();
   return PLX_ERR_CUDA;
 }
@@ -236,10 +249,10 @@ template <int D>
 plx_status launch_decode_f32(const DecodeArgs& a, int ctas, size_t smem, cudaStream_t stream, bool set_attr) {
   auto kern = decode_f32_kernel<D, kDecodeF32Warps>;
   if (set_attr &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      set_smem(kern, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
   kern<<<ctas, kDecodeF32Warps * 32, smem, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
 // A validated decode call: kernel arguments, plan and tensor maps.
@@ -351,20 +364,14 @@ plx_status set_decode_attr(const DecodeLaunch& L, const plx_decode_params* p) {
   cudaError_t e;
   const bool pad = L.a.group <= kMaxGroup / 2;
   if (p->in_dtype == PLX_F32)
-    e = p->head_dim == 64 ? cudaFuncSetAttribute(decode_f32_kernel<64, kDecodeF32Warps>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-                          : cudaFuncSetAttribute(decode_f32_kernel<128, kDecodeF32Warps>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = p->head_dim == 64 ? set_smem(decode_f32_kernel<64, kDecodeF32Warps>, smem)
+                          : set_smem(decode_f32_kernel<128, kDecodeF32Warps>, smem);
   else if (p->head_dim == 64)
-    e = pad ? cudaFuncSetAttribute(decode_tc_kernel<64, kDecodeStages64, kDecodeNC, true>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-            : cudaFuncSetAttribute(decode_tc_kernel<64, kDecodeStages64, kDecodeNC, false>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = pad ? set_smem(decode_tc_kernel<64, kDecodeStages64, kDecodeNC, true>, smem)
+            : set_smem(decode_tc_kernel<64, kDecodeStages64, kDecodeNC, false>, smem);
   else
-    e = pad ? cudaFuncSetAttribute(decode_tc_kernel<128, kDecodeStages128, kDecodeNC, true>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem)
-            : cudaFuncSetAttribute(decode_tc_kernel<128, kDecodeStages128, kDecodeNC, false>,
-                                   cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = pad ? set_smem(decode_tc_kernel<128, kDecodeStages128, kDecodeNC, true>, smem)
+            : set_smem(decode_tc_kernel<128, kDecodeStages128, kDecodeNC, false>, smem);
   return e == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
@@ -380,7 +387,7 @@ plx_status launch_project(const ProjArgs& pa, cudaStream_t stream) {
     case 4: project_qr_kernel<4, 4><<<grid, block, 0, stream>>>(pa); break;
     default: project_qr_kernel<kPjMaxTiles, 2><<<grid, block, 0, stream>>>(pa); break;
   }
-  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
 
@@ -390,12 +397,12 @@ template <bool kPaged>
 plx_status launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tr, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const PrefillArgs& a, cudaStream_t stream) {
   constexpr int smem = PfLayout::kBytes;
-  if (cudaFuncSetAttribute(prefill_tc_kernel<kPaged>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+  if (set_smem(prefill_tc_kernel<kPaged>, smem) !=
       cudaSuccess)
     return PLX_ERR_CUDA;
   const long long grid = (long long)a.n_mblk * a.B * a.H;
   prefill_tc_kernel<kPaged><<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
 // Dense prefill: the two-CTA kernel (prefill2.cuh), 256 query rows per
@@ -425,11 +432,23 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   a.vbar = vbar;
   a.stats = stats;
   constexpr int smem = P2Layout::kBytes;
-  if (cudaFuncSetAttribute(prefill_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+  if (set_smem(prefill_tc2_kernel, smem) != cudaSuccess)
     return PLX_ERR_CUDA;
   const long long grid = 2LL * a.n_mblk * a.B * a.H;
-  prefill_tc2_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kPfThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return note(cudaLaunchKernelEx(&cfg, prefill_tc2_kernel, tq, tr, tk, tv, a)) == cudaSuccess ? PLX_OK
+                                                                                         : PLX_ERR_CUDA;
 }
 
 plx_status validate_prefill(const plx_prefill_params* p) {
@@ -493,7 +512,7 @@ plx_status launch_prefill_backward(const void* q, const void* rho, const void* k
   else
     prefill_bwd_rows_kernel<false><<<row_blocks, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(dout), out, vbar, stats, rows, slab, scale_log2, n_rows);
-  if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+  if (note(cudaGetLastError()) != cudaSuccess) return PLX_ERR_CUDA;
 
   BwdArgs a{};
   a.B = p->batch;
@@ -521,12 +540,12 @@ plx_status launch_prefill_backward(const void* q, const void* rho, const void* k
         !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBN))
       return PLX_ERR_CUDA;
     constexpr int smem = BqLayout::kBytes;
-    if (cudaFuncSetAttribute(prefill_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+    if (set_smem(prefill_bwd_dq_kernel, smem) !=
         cudaSuccess)
       return PLX_ERR_CUDA;
     const long long grid = (long long)a.n_blk * a.B * a.H;
     prefill_bwd_dq_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tg, tk, tv, a);
-    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+    if (note(cudaGetLastError()) != cudaSuccess) return PLX_ERR_CUDA;
   }
   {  // dk, dv: 128-row key tiles, 64-row query tiles (and their 64-column offset slab rows)
     CUtensorMap tq, tr, tg, tk, tv, ts;
@@ -535,12 +554,12 @@ plx_status launch_prefill_backward(const void* q, const void* rho, const void* k
         !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBM) || !make_tmap_bf16(&ts, slab, 64, rows_q, 64, kPfBN))
       return PLX_ERR_CUDA;
     constexpr int smem = BkLayout::kBytes;
-    if (cudaFuncSetAttribute(prefill_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+    if (set_smem(prefill_bwd_dkv_kernel, smem) !=
         cudaSuccess)
       return PLX_ERR_CUDA;
     const long long grid = (long long)a.n_blk * a.B * hkv;
     prefill_bwd_dkv_kernel<<<(unsigned)grid, kPfThreads, smem, stream>>>(tq, tr, tg, tk, tv, ts, a);
-    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+    if (note(cudaGetLastError()) != cudaSuccess) return PLX_ERR_CUDA;
   }
   return PLX_OK;
 }
@@ -891,17 +910,25 @@ plx_status parallax_lla_decode(const void* q, const void* k_cache, const void* v
     if (!make_tmap_bf16(&tk, k_cache, kLlaD, rows, 64, kTile) || !make_tmap_bf16(&tv, v_cache, kLlaD, rows, 64, kTile))
       return PLX_ERR_CUDA;
     constexpr int smem = LlaLayout::kBytes;
-    if (cudaFuncSetAttribute(lla_moments_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    if (set_smem(lla_moments_kernel, smem) != cudaSuccess)
       return PLX_ERR_CUDA;
     lla_moments_kernel<<<(unsigned)(heads * pieces), kLlaThreads, smem, stream>>>(tk, tv, a);
-    if (cudaGetLastError() != cudaSuccess) return PLX_ERR_CUDA;
+    if (note(cudaGetLastError()) != cudaSuccess) return PLX_ERR_CUDA;
   }
   constexpr int ssmem = lla_solve_smem_bytes();
-  if (cudaFuncSetAttribute(lla_solve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, ssmem) != cudaSuccess)
+  if (set_smem(lla_solve_kernel, ssmem) != cudaSuccess)
     return PLX_ERR_CUDA;
   lla_solve_kernel<<<(unsigned)heads, kLlaSolveThreads, ssmem, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
+
+int32_t parallax_last_cuda_error(void) {
+  const int e = g_last_cuda_error;
+  g_last_cuda_error = 0;
+  return e;
+}
+
+const char* parallax_cuda_error_string(int32_t code) { return cudaGetErrorString((cudaError_t)code); }
 
 plx_status parallax_last_device_error(cudaStream_t stream, int32_t* code) {
   if (code == nullptr) return PLX_ERR_INVALID_ARG;

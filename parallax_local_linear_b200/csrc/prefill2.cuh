@@ -173,7 +173,10 @@ struct P2Layout {
 
 // Grid: 2 CTAs per 256 query rows of a (sequence, head), clusters of 2,
 // longest pairs first.  a.n_mblk = ceil(T / 256).
-__global__ void __cluster_dims__(2, 1, 1) __maxnreg__(200)
+// Launched with a cluster dimension of 2 (cudaLaunchKernelEx).  320 threads
+// are 10 warps, so three share an SM sub-partition's 16K registers: at most
+// 168 registers a thread.
+__global__ void __launch_bounds__(kPfThreads, 1)
     prefill_tc2_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_r,
                        const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const PrefillArgs a) {

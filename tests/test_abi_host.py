@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(binding):
 
 
 def test_abi_version_and_status_strings(binding):
-    assert binding.lib.parallax_abi_version() == 7
+    assert binding.lib.parallax_abi_version() == 8
     for code, name in binding.STATUS.items():
         assert binding.lib.parallax_status_string(code).decode() == name
 
