@@ -102,7 +102,9 @@ int32_t parallax_decode_num_ctas(const plx_decode_params* p, int32_t num_sms);
  * 256 B) followed by two fp32 partial slots per CTA.  The counter region
  * must be zero before the workspace is first used (e.g. cudaMemsetAsync);
  * every call that completes leaves it zero again, so one zeroing lasts for
- * the workspace's lifetime. */
+ * the workspace's lifetime -- as long as nothing else writes it: memory
+ * lent to another call in between (parallax_lla_decode's workspace, say)
+ * must be zeroed again. */
 size_t parallax_decode_workspace_size(const plx_decode_params* p, int32_t num_sms);
 
 /* Parallax decode.

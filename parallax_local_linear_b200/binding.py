@@ -243,6 +243,22 @@ def _workspace(device, nbytes):
         return ws
 
 
+_lla_workspaces = {}
+
+
+def _lla_workspace(device, nbytes):
+    """The LLA pass's scratch per device, grown on demand.  It is kept apart
+    from the decode workspace: LLA writes its records over the whole buffer,
+    while a decode workspace's counter region must stay zero between calls."""
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    with _ws_lock:
+        ws = _lla_workspaces.get(idx)
+        if ws is None or ws.numel() < nbytes:
+            ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+            _lla_workspaces[idx] = ws
+        return ws
+
+
 def decode_params(q, k_cache, *, page_table=None, kv_len=None, scale=None, out_dtype=None,
                   num_ctas=0, num_pages=None):
     B, Hq, d = q.shape
@@ -433,7 +449,7 @@ def lla_decode(q, k_cache, v_cache, scale=None, ridge=0.0, *, seq_lens=None, pag
     nbytes = lib.parallax_lla_decode_workspace_size(ctypes.byref(p), float(ridge), 0)
     if nbytes == SIZE_MAX:
         raise ParallaxError(1, "parallax_lla_decode_workspace_size")
-    ws = _workspace(q.device, nbytes)
+    ws = _lla_workspace(q.device, nbytes)
     st = lib.parallax_lla_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(page_table), _ptr(seq_lens),
                                  float(ridge), _ptr(rho_out), _ptr(out), _ptr(ws), 0 if ws is None else ws.numel(),
                                  ctypes.byref(p), _stream_ptr(q.device))

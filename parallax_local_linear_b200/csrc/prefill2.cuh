@@ -28,8 +28,10 @@
 //     (acquire.cluster), issues the MMAs, and commits their completion to the
 //     barriers of both CTAs at once (tcgen05.commit multicast): s_full (S/A
 //     ready), k_empty / v_empty (the stage may be refilled), o_done, drain;
-//   * each CTA's softmax warps arrive on the first CTA's p_full when their P
-//     is in their TMEM (remote arrive from the second CTA).
+//   * each softmax warp of either CTA arrives once on the first CTA's p_full
+//     when its lanes' P is in their TMEM (a remote arrive from the second).
+// Barriers that only tcgen05.commit arrives on are waited with CTA scope;
+// those that threads of the other CTA arrive on, with cluster scope.
 // Tensor memory is allocated and freed for the pair (cta_group::2); a
 // cluster barrier precedes the release.
 #pragma once
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], kPfSoftmax);   // both CTAs' warpgroup of this buffer (first CTA's barrier)
+      mbar_init(&p_full[i], 8);   // the 4 warps of this buffer's warpgroup in each CTA (first CTA's barrier)
       mbar_init(&hand[i], kPfSoftmax / 2);
     }
     mbar_init(o_done, 1);
@@ -273,7 +275,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int s = j % S;
         const uint32_t par = ((j / S) - 1) & 1;
         const int row = kv_row + j * kPfBN;
-        if (j >= S && !mbar_wait_cl(a.wait_ns, &k_empty[s], par)) {
+        if (j >= S && !mbar_wait_bounded(a.wait_ns, &k_empty[s], par)) {
           *abort_flag = 1;
           break;
         }
@@ -283,7 +285,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           tma_load_2d(sm + Ly::kK + s * Ly::kKBytes + bx * (Ly::kKBytes / 2), &tm_k, bx * 64,
                       row + (kPfBN / 2) * (int)rank, &k_full[s], keep);
         ++issued_k;
-        if (j >= S && !mbar_wait_cl(a.wait_ns, &v_empty[s], par)) {
+        if (j >= S && !mbar_wait_bounded(a.wait_ns, &v_empty[s], par)) {
           *abort_flag = 1;
           break;
         }
@@ -323,7 +325,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     __syncwarp();
     // The first CTA's MMAs write this CTA's TMEM: wait for all of them.
-    mbar_wait_cl(kDrainLimitNs, drain, 0);
+    mbar_wait_drain(drain, 0);
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer (first CTA)
@@ -396,7 +398,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // Every issued MMA must complete before either CTA releases tensor memory.
     tc2_commit_mc(drain, kBoth);
     __syncwarp();
-    mbar_wait_cl(kDrainLimitNs, drain, 0);
+    mbar_wait_drain(drain, 0);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax (both CTAs)
@@ -410,13 +412,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     const int key_lim = a.causal ? min(t + 1, T) : T;
     const int split_tiles = few_keys ? kPfSplitTiles : 0;
     const uint32_t cS = tmem + lane_off + col_s(g), cA = tmem + lane_off + col_a(g);
-    const uint32_t p_full_first = dsmem_map(smem_u32(&p_full[g]), 0);
     float m_ref = -INFINITY, m_mine = -INFINITY, aref = 0.f;
     float2 l2 = make_float2(0.f, 0.f), c2 = make_float2(0.f, 0.f);
     bool fine = true;
     int j = g;
     for (; j < n; j += 2) {
-      const bool w = !*abort_flag && mbar_wait_cl(a.wait_ns, &s_full[g], (j >> 1) & 1);
+      const bool w = !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[g], (j >> 1) & 1);
       tc_fence_after();
       uint32_t sr[64], ar[32];
       tmem_ld32p(cS, sr);
@@ -509,7 +510,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         form_p(std::false_type{});
       const bool rescale = __any_sync(0xffffffffu, need) && j >= 1;
       if (j >= 1 && (j == n - 1 || rescale)) {
-        const bool wo = __all_sync(0xffffffffu, mbar_wait_cl(a.wait_ns, o_done, (j - 1) & 1));
+        const bool wo = __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, o_done, (j - 1) & 1));
         fine = fine && wo;
         if (wo && rescale) {
           tc_fence_after();
@@ -525,15 +526,19 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
+      // One arrive per warp, after every lane's TMEM stores have completed.
       tmem_wait_st();
       tc_fence_before();
-      if (rank == 0)
-        mbar_arrive(&p_full[g]);
-      else
-        mbar_arrive_remote(p_full_first);
+      __syncwarp();
+      if (lane == 0) {
+        if (cluster_ctarank() == 0)
+          mbar_arrive(&p_full[g]);
+        else
+          mbar_arrive_remote(dsmem_map(smem_u32(&p_full[g]), 0));
+      }
     }
     bool wl = fine && j >= n && !*abort_flag;
-    if (wl && ((n - 1) & 1) == g) wl = mbar_wait_cl(a.wait_ns, o_done, (n - 1) & 1);
+    if (wl && ((n - 1) & 1) == g) wl = mbar_wait_bounded(a.wait_ns, o_done, (n - 1) & 1);
     lc_s[(g * 128 + r) * 3 + 0] = l2.x + l2.y;
     lc_s[(g * 128 + r) * 3 + 1] = c2.x + c2.y;
     lc_s[(g * 128 + r) * 3 + 2] = m_mine;

@@ -15,7 +15,7 @@ import torch
 
 import oracle
 from parallax_local_linear_b200 import workloads as W
-from tests.helpers import TOL_BF16, F64View, assert_parity, to_f64
+from tests.helpers import TOL_BF16, F64View, assert_parity, oracle_heads, to_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -134,3 +134,14 @@ def test_decode_long_workload_sampled(px):
     _check(px, inp, 0.0, "decode_long workload", heads=heads)
     del inp
     torch.cuda.empty_cache()
+
+
+def test_decode_after_lla_is_unaffected(px):
+    # LLA's scratch is not the decode's workspace: a decode whose units are
+    # split over CTAs (merged through the workspace counters) right after an
+    # LLA call must still match the oracle.
+    inp = _cuda(W.small_decode_inputs(1, 2, 2, 128, 500, seed=48))
+    _run(px, inp, 0.1)
+    out = px.decode(inp["q"], inp["q"], inp["k_cache"], inp["v_cache"], inp["scale"], out_dtype=torch.float32)
+    ref = oracle_heads(dict(inp, rho=inp["q"]), [(0, 0), (0, 1)])
+    assert_parity(out.cpu().numpy(), ref, TOL_BF16, "decode after LLA")
