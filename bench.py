@@ -58,8 +58,9 @@ METRIC = "decode KV GB/s & tokens/s (% of HBM peak); prefill TFLOP/s (% of bf16 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = {
     "decode": ["parallax_local_linear_b200/csrc/decode.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
-    "prefill": ["parallax_local_linear_b200/csrc/prefill2.cuh", "parallax_local_linear_b200/csrc/prefill.cuh",
-                "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "prefill": ["parallax_local_linear_b200/csrc/prefill.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
+    "prefill_pair": ["parallax_local_linear_b200/csrc/prefill2.cuh", "parallax_local_linear_b200/csrc/prefill.cuh",
+                     "parallax_local_linear_b200/csrc/ptx.cuh"],
     "prefill_paged": ["parallax_local_linear_b200/csrc/prefill.cuh", "parallax_local_linear_b200/csrc/ptx.cuh"],
     "prefill_bwd": ["parallax_local_linear_b200/csrc/prefill_bwd.cuh", "parallax_local_linear_b200/csrc/prefill.cuh",
                     "parallax_local_linear_b200/csrc/ptx.cuh"],
@@ -84,6 +85,8 @@ def parse_args(argv=None):
     ap.add_argument("--num-ctas", type=int, default=0)
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--cta-pair", action="store_true",
+                    help="prefill workloads: run the two-SM (cta_group::2) dense prefill kernel")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
@@ -706,7 +709,8 @@ def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
     out = torch.empty_like(x["q"])
 
     def step():
-        px.prefill(x["q"], x["rho"], x["k"], x["v"], causal=w.causal, scale=x["scale"], out=out)
+        px.prefill(x["q"], x["rho"], x["k"], x["v"], causal=w.causal, scale=x["scale"], out=out,
+                   cta_pair=args.cta_pair)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -743,7 +747,8 @@ def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
     for _ in range(Ke):
         for k in hx:
             dx[k].copy_(hx[k], non_blocking=True)
-        px.prefill(dx["q"], dx["rho"], dx["k"], dx["v"], causal=w.causal, scale=x["scale"], out=out)
+        px.prefill(dx["q"], dx["rho"], dx["k"], dx["v"], causal=w.causal, scale=x["scale"], out=out,
+                   cta_pair=args.cta_pair)
         oh.copy_(out, non_blocking=True)
     e2.record()
     torch.cuda.synchronize()
@@ -757,11 +762,13 @@ def bench_prefill(args, w, rank, world, dev, peaks, peaks_kind):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "batch": w.batch, "num_heads": w.num_heads, "seq_len": w.seq_len,
                    "head_dim": w.head_dim, "causal": w.causal, "rho_scale": w.rho_scale,
-                   "l2": "inputs 537 MB > 126 MB L2"},
+                   "cta_pair": bool(args.cta_pair), "l2": "inputs 537 MB > 126 MB L2"},
         "pct_of_bf16_peak": round(100 * tflops / world / peak, 2),
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), **traffic_fields("prefill", w.name),
-                     "peak_source": f"{peaks_kind} bf16_tflops_sustained", "kernel": "prefill_tc2_kernel",
+                     "frac": round(achieved / peak, 4),
+                     **traffic_fields("prefill_pair" if args.cta_pair else "prefill", w.name),
+                     "peak_source": f"{peaks_kind} bf16_tflops_sustained",
+                     "kernel": "prefill_tc2_kernel (cta_pair)" if args.cta_pair else "prefill_tc_kernel",
                      "algorithmic_flops_per_launch": flops},
         "e2e": e2e, "gpu_launches": K, "clocks": clk.summary(),
     }
@@ -1148,8 +1155,8 @@ def _host_decode_sample(w):
 # Workloads timed after the headline one in the default run, each with its
 # own roofline, clocks and oracle baseline (the four other configurations of
 # the method's targets first, then the serving and training steps beyond them).
-PER_CONFIG = ("decode_f32", "decode_long", "decode_paged", "prefill", "prefill_paged", "prefill_train",
-              "decode_projected", "lla_decode")
+PER_CONFIG = ("decode_f32", "decode_long", "decode_paged", "prefill", "prefill_cta_pair", "prefill_paged",
+              "prefill_train", "decode_projected", "lla_decode")
 NOMINAL_PEAKS = {"GB/s": 8000.0, "TFLOP/s": 2250.0}   # B200 HBM3e and dense bf16, NVIDIA's figures
 
 
@@ -1225,17 +1232,19 @@ def main(argv=None):
         per_config = {}
         if args.per_config and args.workload == "decode_bf16" and args.batch == 0:
             import copy
-            for name in PER_CONFIG:
+            for key in PER_CONFIG:
                 torch.cuda.empty_cache()
+                name = "prefill" if key == "prefill_cta_pair" else key
                 wc = W.WORKLOADS[name]
                 ac = copy.copy(args)
+                ac.cta_pair = key == "prefill_cta_pair"
                 ac.steps = steps_given if steps_given is not None else default_steps(name)
                 ac.warmup = warmup_given if warmup_given is not None else 5
                 rc, ic = run_workload(ac, wc, rank, world, dev, peaks, kind)
-                if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                if rank == 0 and world == 1 and not args.no_cpu_baseline and not ac.cta_pair:
                     rc["cpu_baseline"] = cpu_baseline(wc, ic, args.cpu_seconds_per_config)
                 del ic
-                per_config[name] = config_summary(rc)
+                per_config[key] = config_summary(rc)
         if rank == 0:
             res["roofline"]["nominal_peak"] = NOMINAL_PEAKS[res["roofline"]["unit"]]
             res["roofline"]["frac_of_nominal"] = round(res["roofline"]["achieved"] /

@@ -42,7 +42,7 @@
 extern "C" {
 #endif
 
-#define PARALLAX_ABI_VERSION 8
+#define PARALLAX_ABI_VERSION 10
 
 typedef enum plx_status {
   PLX_OK = 0,
@@ -157,6 +157,16 @@ plx_status parallax_decode_plan_create(const void* q, const void* rho,
                                       void* out, void* workspace, size_t workspace_bytes,
                                       const plx_decode_params* p, plx_decode_plan** plan);
 plx_status parallax_decode_plan_run(const plx_decode_plan* plan, cudaStream_t stream);
+
+/* One serving step from host memory: on `stream`, copies host_q and
+ * host_rho ([B, Hq, d] of in_dtype) into the plan's q and rho buffers, runs
+ * the decode, and copies the plan's out buffer into host_out ([B, Hq, d] of
+ * out_dtype); three copies and one launch, all asynchronous (the host
+ * buffers must be page-locked for the copies to overlap other work, and
+ * must stay valid until the stream reaches them).  Errors as
+ * parallax_decode_plan_run; PLX_ERR_INVALID_ARG for a null host pointer. */
+plx_status parallax_decode_plan_run_io(const plx_decode_plan* plan, const void* host_q, const void* host_rho,
+                                      void* host_out, cudaStream_t stream);
 void parallax_decode_plan_destroy(plx_decode_plan* plan);
 
 /* Decode whose query and probe are projected from the new token's layer
@@ -290,6 +300,11 @@ typedef struct plx_prefill_params {
   int32_t out_dtype;      /* PLX_BF16 or PLX_F32                              */
   float scale;            /* softmax scale on q.k, > 0                        */
   int32_t causal;         /* 1: causal mask (diagonal included); 0: none      */
+  int32_t cta_pair;       /* 0: one CTA (one SM) per 128 query rows; 1: a
+                             cluster of two CTAs per 256 rows, one tcgen05
+                             instruction (cta_group::2) for both, each SM
+                             loading half of every K and V tile.  Same
+                             results; 0 is the faster one as measured.      */
 } plx_prefill_params;
 
 /* Parallax prefill.

@@ -45,7 +45,7 @@ class PrefillParams(ctypes.Structure):
                 ("num_kv_heads", ctypes.c_int32), ("seq_len", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("in_dtype", ctypes.c_int32),
                 ("out_dtype", ctypes.c_int32), ("scale", ctypes.c_float),
-                ("causal", ctypes.c_int32)]
+                ("causal", ctypes.c_int32), ("cta_pair", ctypes.c_int32)]
 
 
 class PrefillPagedParams(ctypes.Structure):
@@ -96,6 +96,8 @@ lib.parallax_decode_plan_create.argtypes = [_vp, _vp, _vp, _vp, _i32p, _i32p, _v
                                             ctypes.POINTER(DecodeParams), ctypes.POINTER(ctypes.c_void_p)]
 lib.parallax_decode_plan_run.restype = ctypes.c_int
 lib.parallax_decode_plan_run.argtypes = [_vp, _vp]
+lib.parallax_decode_plan_run_io.restype = ctypes.c_int
+lib.parallax_decode_plan_run_io.argtypes = [_vp, _vp, _vp, _vp, _vp]
 lib.parallax_decode_plan_destroy.restype = None
 lib.parallax_decode_plan_destroy.argtypes = [_vp]
 lib.parallax_set_wait_limit_ns.restype = ctypes.c_int
@@ -352,6 +354,21 @@ class DecodePlan:
             raise ParallaxError(st, "parallax_decode_plan_run")
         return self.out
 
+    def run_io(self, host_q, host_rho, host_out):
+        """One step from host memory: copies ``host_q`` and ``host_rho`` in,
+        runs the decode and copies the output into ``host_out``, all queued
+        on the current stream (host tensors: contiguous, pinned, shaped and
+        typed like q / out)."""
+        q, rho = self._keep[0], self._keep[1]
+        for name, t, like in (("host_q", host_q, q), ("host_rho", host_rho, rho), ("host_out", host_out, self.out)):
+            if t.is_cuda or not t.is_contiguous() or t.dtype != like.dtype or tuple(t.shape) != tuple(like.shape):
+                raise ValueError(f"{name} must be a contiguous host tensor like {tuple(like.shape)} {like.dtype}")
+        st = lib.parallax_decode_plan_run_io(self._handle, _ptr(host_q), _ptr(host_rho), _ptr(host_out),
+                                             ctypes.c_void_p(torch.cuda.current_stream(self._device).cuda_stream))
+        if st != 0:
+            raise ParallaxError(st, "parallax_decode_plan_run_io")
+        return host_out
+
     def __del__(self):
         h = getattr(self, "_handle", None)
         if h is not None and h.value:
@@ -458,9 +475,11 @@ def lla_decode(q, k_cache, v_cache, scale=None, ridge=0.0, *, seq_lens=None, pag
     return out, rho_out
 
 
-def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):
+def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None, cta_pair=False):
     """Parallax prefill.  q, rho: [B, H, T, d] bf16; k, v: [B, Hkv, T, d] bf16.
-    Row t attends to keys 0..t when causal, else to all T keys."""
+    Row t attends to keys 0..t when causal, else to all T keys.  ``cta_pair``
+    runs the two-SM kernel (tcgen05 cta_group::2) instead of one CTA per 128
+    rows; the results are the same."""
     for name, t in (("q", q), ("rho", rho), ("k", k), ("v", v)):
         _check_cuda(name, t, torch.bfloat16)
     B, H, T, d = q.shape
@@ -468,7 +487,8 @@ def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):
         raise ValueError("shape mismatch")
     out, out_dtype = _output(out, out_dtype, q.shape, q.dtype, q.device)
     scale = (1.0 / d ** 0.5) if scale is None else float(scale)
-    p = PrefillParams(B, H, k.shape[1], T, d, PLX_BF16, _dtype_code(out_dtype), scale, 1 if causal else 0)
+    p = PrefillParams(B, H, k.shape[1], T, d, PLX_BF16, _dtype_code(out_dtype), scale, 1 if causal else 0,
+                      1 if cta_pair else 0)
     st = lib.parallax_prefill(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out), ctypes.byref(p),
                               _stream_ptr(q.device))
     if st != 0:
@@ -476,10 +496,11 @@ def prefill(q, rho, k, v, causal=True, scale=None, *, out=None, out_dtype=None):
     return out
 
 
-def _prefill_params(q, k, causal, scale, out_dtype):
+def _prefill_params(q, k, causal, scale, out_dtype, cta_pair=False):
     B, H, T, d = q.shape
     scale = (1.0 / d ** 0.5) if scale is None else float(scale)
-    return PrefillParams(B, H, k.shape[1], T, d, PLX_BF16, _dtype_code(out_dtype), scale, 1 if causal else 0)
+    return PrefillParams(B, H, k.shape[1], T, d, PLX_BF16, _dtype_code(out_dtype), scale, 1 if causal else 0,
+                         1 if cta_pair else 0)
 
 
 def _check_prefill_inputs(q, rho, k, v):
@@ -490,7 +511,7 @@ def _check_prefill_inputs(q, rho, k, v):
         raise ValueError("shape mismatch")
 
 
-def prefill_train(q, rho, k, v, causal=True, scale=None, *, out_dtype=None):
+def prefill_train(q, rho, k, v, causal=True, scale=None, *, out_dtype=None, cta_pair=False):
     """Prefill forward for training: returns (out, vbar, stats).
 
     vbar: float32 [B, H, T, d], the softmax average of the values of each
@@ -501,7 +522,7 @@ def prefill_train(q, rho, k, v, causal=True, scale=None, *, out_dtype=None):
     out = torch.empty(q.shape, dtype=out_dtype, device=q.device)
     vbar = torch.empty(q.shape, dtype=torch.float32, device=q.device)
     stats = torch.empty(q.shape[:3] + (2,), dtype=torch.float32, device=q.device)
-    p = _prefill_params(q, k, causal, scale, out_dtype)
+    p = _prefill_params(q, k, causal, scale, out_dtype, cta_pair)
     st = lib.parallax_prefill_train(_ptr(q), _ptr(rho), _ptr(k), _ptr(v), _ptr(out), _ptr(vbar), _ptr(stats),
                                     ctypes.byref(p), _stream_ptr(q.device))
     if st != 0:

@@ -405,17 +405,19 @@ plx_status launch_prefill_kernel(const CUtensorMap& tq, const CUtensorMap& tr, c
   return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
 }
 
-// Dense prefill: the two-CTA kernel (prefill2.cuh), 256 query rows per
-// cluster of two SMs.
+// Dense prefill: one CTA per 128 query rows (prefill_tc_kernel), or with
+// p->cta_pair a cluster of two CTAs per 256 rows (prefill_tc2_kernel).
 plx_status launch_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,
                           const plx_prefill_params* p, cudaStream_t stream, float* vbar = nullptr,
                           float2* stats = nullptr) {
   const int hkv = p->num_kv_heads == 0 ? p->num_heads : p->num_kv_heads;
   const uint64_t rows_q = (uint64_t)p->batch * p->num_heads * p->seq_len;
   const uint64_t rows_kv = (uint64_t)p->batch * hkv * p->seq_len;
+  const bool pair = p->cta_pair != 0;
   CUtensorMap tq, tr, tk, tv;
   if (!make_tmap_bf16(&tq, q, kPfD, rows_q, 64, kPfBM) || !make_tmap_bf16(&tr, rho, kPfD, rows_q, 64, kPfBM) ||
-      !make_tmap_bf16(&tk, k, kPfD, rows_kv, 64, kPfBN / 2) || !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBN))
+      !make_tmap_bf16(&tk, k, kPfD, rows_kv, 64, pair ? kPfBN / 2 : kPfBN) ||
+      !make_tmap_bf16(&tv, v, kPfD, rows_kv, 64, kPfBN))
     return PLX_ERR_CUDA;
   PrefillArgs a{};
   a.B = p->batch;
@@ -423,7 +425,8 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   a.Hkv = hkv;
   a.T = p->seq_len;
   a.group = p->num_heads / hkv;
-  a.n_mblk = (p->seq_len + 2 * kPfBM - 1) / (2 * kPfBM);   // pairs of 128-row tiles
+  a.n_mblk = pair ? (p->seq_len + 2 * kPfBM - 1) / (2 * kPfBM)   // pairs of 128-row tiles
+                  : (p->seq_len + kPfBM - 1) / kPfBM;
   a.causal = p->causal;
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
   a.scale_log2 = p->scale * 1.4426950408889634f;
@@ -431,6 +434,7 @@ plx_status launch_prefill(const void* q, const void* rho, const void* k, const v
   a.wait_ns = current_wait_ns();
   a.vbar = vbar;
   a.stats = stats;
+  if (!pair) return launch_prefill_kernel<false>(tq, tr, tk, tv, a, stream);
   constexpr int smem = P2Layout::kBytes;
   if (set_smem(prefill_tc2_kernel, smem) != cudaSuccess)
     return PLX_ERR_CUDA;
@@ -462,7 +466,8 @@ plx_status validate_prefill(const plx_prefill_params* p) {
   if (p->out_dtype != PLX_F32 && p->out_dtype != PLX_BF16) return PLX_ERR_INVALID_ARG;
   if (p->head_dim != 128) return PLX_ERR_UNSUPPORTED;
   if (p->causal != 0 && p->causal != 1) return PLX_ERR_INVALID_ARG;
-  if ((int64_t)p->batch * p->num_heads * ((int64_t)p->seq_len + 128) >= (int64_t)INT32_MAX)
+  if (p->cta_pair != 0 && p->cta_pair != 1) return PLX_ERR_INVALID_ARG;
+  if ((int64_t)p->batch * p->num_heads * ((int64_t)p->seq_len + 256) >= (int64_t)INT32_MAX)
     return PLX_ERR_UNSUPPORTED;
   return PLX_OK;
 }
@@ -694,6 +699,28 @@ plx_status parallax_decode_plan_run(const plx_decode_plan* plan, cudaStream_t st
   if (cudaGetDevice(&dev) != cudaSuccess) return PLX_ERR_CUDA;
   if (dev != plan->device) return PLX_ERR_INVALID_ARG;
   return launch_decode(plan->L, &plan->p, stream, false, false);
+}
+
+plx_status parallax_decode_plan_run_io(const plx_decode_plan* plan, const void* host_q, const void* host_rho,
+                                      void* host_out, cudaStream_t stream) {
+  if (plan == nullptr || host_q == nullptr || host_rho == nullptr || host_out == nullptr) return PLX_ERR_INVALID_ARG;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PLX_ERR_CUDA;
+  if (dev != plan->device) return PLX_ERR_INVALID_ARG;
+  const plx_decode_params& p = plan->p;
+  const size_t heads = (size_t)p.batch * p.num_q_heads * p.head_dim;
+  const size_t in_bytes = heads * (p.in_dtype == PLX_BF16 ? 2 : 4);
+  const size_t out_bytes = heads * (p.out_dtype == PLX_BF16 ? 2 : 4);
+  const DecodeArgs& a = plan->L.a;
+  if (note(cudaMemcpyAsync(const_cast<void*>(a.q), host_q, in_bytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
+      note(cudaMemcpyAsync(const_cast<void*>(a.rho), host_rho, in_bytes, cudaMemcpyHostToDevice, stream)) !=
+          cudaSuccess)
+    return PLX_ERR_CUDA;
+  const plx_status st = launch_decode(plan->L, &plan->p, stream, false, false);
+  if (st != PLX_OK) return st;
+  return note(cudaMemcpyAsync(host_out, a.out, out_bytes, cudaMemcpyDeviceToHost, stream)) == cudaSuccess
+             ? PLX_OK
+             : PLX_ERR_CUDA;
 }
 
 void parallax_decode_plan_destroy(plx_decode_plan* plan) { delete plan; }

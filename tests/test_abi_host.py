@@ -44,7 +44,7 @@ def test_library_exports_every_declared_symbol(binding):
 
 
 def test_abi_version_and_status_strings(binding):
-    assert binding.lib.parallax_abi_version() == 8
+    assert binding.lib.parallax_abi_version() == 10
     for code, name in binding.STATUS.items():
         assert binding.lib.parallax_status_string(code).decode() == name
 
@@ -139,7 +139,7 @@ def test_projected_decode_rejects_overlapping_outputs_before_launch(binding):
     assert call(q=None) == 1
 
 
-@pytest.mark.parametrize("bad", [dict(seq_len=0), dict(head_dim=64), dict(in_dtype=0), dict(causal=2),
+@pytest.mark.parametrize("bad", [dict(seq_len=0), dict(head_dim=64), dict(in_dtype=0), dict(causal=2), dict(cta_pair=2),
                                  dict(num_heads=6, num_kv_heads=4), dict(scale=-0.1), dict(scale=0.0)])
 def test_invalid_prefill_params_are_rejected(binding, bad):
     base = dict(batch=1, num_heads=4, num_kv_heads=0, seq_len=16, head_dim=128, in_dtype=1, out_dtype=1,

@@ -75,3 +75,20 @@ def test_plan_in_a_cuda_graph(px):
     g.replay()
     ref = px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"])
     assert torch.equal(out, ref)
+
+
+def test_plan_step_from_host_memory(px):
+    # run_io: q and rho copied in from pinned host memory, the decode, the
+    # output copied back, on one stream: the result equals the device-side run.
+    inp = _cuda(W.small_decode_inputs(8, 16, 8, 128, 1024, seed=64))
+    dq, dr = torch.empty_like(inp["q"]), torch.empty_like(inp["rho"])
+    out = torch.empty_like(inp["q"])
+    plan = px.DecodePlan(dq, dr, inp["k_cache"], inp["v_cache"], inp["scale"], out=out)
+    hq, hr = inp["q"].cpu().pin_memory(), inp["rho"].cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    plan.run_io(hq, hr, hout)
+    torch.cuda.synchronize()
+    ref = px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"])
+    assert torch.equal(hout, ref.cpu())
+    with pytest.raises(ValueError):
+        plan.run_io(inp["q"], hr, hout)   # a device tensor where a host one belongs

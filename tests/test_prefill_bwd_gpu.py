@@ -68,10 +68,13 @@ def test_unit_scale_probe(px):
     _check(px, _inputs(1, 2, 150, seed=6, rho_scale=1.0), what="unit rho")
 
 
-def test_training_forward_outputs(px):
+@pytest.mark.parametrize("pair", [False, True])
+def test_training_forward_outputs(px, pair):
     x = _inputs(1, 2, 300, seed=7)
-    out, vbar, stats = px.prefill_train(x["q"], x["rho"], x["k"], x["v"], True, x["scale"], out_dtype=torch.float32)
-    plain = px.prefill(x["q"], x["rho"], x["k"], x["v"], causal=True, scale=x["scale"], out_dtype=torch.float32)
+    out, vbar, stats = px.prefill_train(x["q"], x["rho"], x["k"], x["v"], True, x["scale"], out_dtype=torch.float32,
+                                        cta_pair=pair)
+    plain = px.prefill(x["q"], x["rho"], x["k"], x["v"], causal=True, scale=x["scale"], out_dtype=torch.float32,
+                       cta_pair=pair)
     assert torch.equal(out, plain)
     q, rho, k, v = (to_f64(x[n]) for n in ("q", "rho", "k", "v"))
     st = stats.cpu().numpy().astype(np.float64)

@@ -31,9 +31,9 @@ def _cuda(inp):
     return {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
 
 
-def _run(px, inp, causal=True, out_dtype=torch.float32):
+def _run(px, inp, causal=True, out_dtype=torch.float32, pair=False):
     return px.prefill(inp["q"], inp["rho"], inp["k"], inp["v"], causal=causal, scale=inp["scale"],
-                      out_dtype=out_dtype)
+                      out_dtype=out_dtype, cta_pair=pair)
 
 
 def _ref_rows(inp, rows, causal=True):
@@ -52,29 +52,32 @@ def _rows(B, H, T, limit=None, seed=0):
     return rows
 
 
+@pytest.mark.parametrize("pair", [False, True])
 @pytest.mark.parametrize("T", [1, 2, 63, 64, 65, 127, 128, 129, 200, 255, 256, 257, 383, 1000])
-def test_causal_lengths(px, T):
+def test_causal_lengths(px, T, pair):
     inp = _cuda(W.small_prefill_inputs(1, 2, T, 128, seed=T))
-    out = _run(px, inp).cpu().numpy()
+    out = _run(px, inp, pair=pair).cpu().numpy()
     rows = _rows(1, 2, T, limit=160, seed=T)
     ref = _ref_rows(inp, rows)
     got = np.stack([out[b, h, t] for b, h, t in rows])
     assert_parity(got, ref, TOL_BF16, f"T={T}")
 
 
+@pytest.mark.parametrize("pair", [False, True])
 @pytest.mark.parametrize("T", [1, 100, 300, 513])
-def test_non_causal(px, T):
+def test_non_causal(px, T, pair):
     inp = _cuda(W.small_prefill_inputs(2, 2, T, 128, seed=7 + T))
-    out = _run(px, inp, causal=False).cpu().numpy()
+    out = _run(px, inp, causal=False, pair=pair).cpu().numpy()
     rows = _rows(2, 2, T, limit=120)
     ref = _ref_rows(inp, rows, causal=False)
     got = np.stack([out[b, h, t] for b, h, t in rows])
     assert_parity(got, ref, TOL_BF16, f"non-causal T={T}")
 
 
-def test_gqa_heads(px):
+@pytest.mark.parametrize("pair", [False, True])
+def test_gqa_heads(px, pair):
     inp = _cuda(W.small_prefill_inputs(2, 4, 300, 128, num_kv_heads=2, seed=11))
-    out = _run(px, inp).cpu().numpy()
+    out = _run(px, inp, pair=pair).cpu().numpy()
     rows = _rows(2, 4, 300, limit=200)
     ref = _ref_rows(inp, rows)
     got = np.stack([out[b, h, t] for b, h, t in rows])
@@ -119,10 +122,11 @@ def full_workload_rows(B, H, T, pairs=8, per_pair=64, seed=5):
     return rows
 
 
-def test_full_prefill_workload_sampled(px):
+@pytest.mark.parametrize("pair", [False, True])
+def test_full_prefill_workload_sampled(px, pair):
     w = W.WORKLOADS["prefill"]
     inp = W.prefill_inputs(w, device="cuda")
-    out = px.prefill(inp["q"], inp["rho"], inp["k"], inp["v"], causal=True, scale=inp["scale"])
+    out = px.prefill(inp["q"], inp["rho"], inp["k"], inp["v"], causal=True, scale=inp["scale"], cta_pair=pair)
     assert out.dtype == torch.bfloat16
     rows = full_workload_rows(w.batch, w.num_heads, w.seq_len)
     assert len(rows) == 512
@@ -133,6 +137,6 @@ def test_full_prefill_workload_sampled(px):
         ts = [t for bb, hh, t in rows if (bb, hh) == (b, h)]
         ref = oracle.prefill_rows(sl["q"], sl["rho"], sl["k"], sl["v"], [(0, 0, t) for t in ts], inp["scale"])
         got = o[b, h, ts].cpu().numpy()
-        assert_parity(got, ref, TOL_BF16, f"prefill workload (b={b}, h={h})")
+        assert_parity(got, ref, TOL_BF16, f"prefill workload (b={b}, h={h}, pair={pair})")
     assert torch.isfinite(o).all()
     assert px.last_device_error() == 0
