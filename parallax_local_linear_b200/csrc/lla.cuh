@@ -20,15 +20,17 @@
 //     a running max m (2^(s - m) weights, rescaled lazily as in the prefill),
 //         l = sum e,  ks = sum e k,  vs = sum e v,
 //         D_KK = sum e k k^T,  D_KV = sum e k v^T          (128 x 128 each)
-//     The two d x d sums are dense contractions over the keys and run on the
-//     tensor cores: D += A . B with A = (e o K)^T, 128 x 16 keys per step,
-//     written by the compute warps into tensor memory (thread a holds
-//     column a of the tile: e_i k_ia for its 64 keys, packed bf16 pairs),
-//     and B = the K or V tile in shared memory (keys x 128, MN-major).  For
-//     sequences shorter than kLlaSplitLen the bf16 rounding of e o K is not
-//     averaged away (the solve amplifies it along directions the few keys do
-//     not span), so a second product adds its lo part (x = hi + lo).
-//     The piece's record goes to the workspace.
+//     All of it runs on the tensor cores except the scores: per 64-key tile
+//     the weights e (rounded to bf16 once, so that every sum uses the same
+//     values) go into diag(e) and the column [e 0 ..] in shared memory; the
+//     MMAs G = K^T diag(e) (so row a of G holds e_i k_ia, exact in fp32),
+//     ks += K^T [e 0 ..] and vs += V^T [e 0 ..] read the K and V tiles as
+//     MN-major A operands; the compute warps pack G into A = (e o K)^T in
+//     tensor memory (bf16 pairs); then D_KK += A . K and D_KV += A . V (K, V
+//     as MN-major B operands).  For sequences shorter than kLlaSplitLen the
+//     bf16 rounding of e o K is not averaged away (the solve amplifies it
+//     along directions the few keys do not span), so a second product adds
+//     its lo part (x = hi + lo).  The piece's record goes to the workspace.
 //
 //   lla_solve_kernel  one CTA per (sequence, query head): merges the pieces
 //     like online softmax (weights 2^(m_j - M)), forms S_KK + ridge I and
@@ -47,12 +49,13 @@ namespace plx {
 
 constexpr int kLlaD = 128;
 constexpr int kLlaStages = 4;            // K and V ring depth (tiles)
-constexpr int kLlaThreads = 192;         // TMA producer warp, MMA warp, four compute warps
-constexpr int kLlaCompute = 128;
+constexpr int kLlaThreads = 320;         // TMA producer warp, MMA warp, eight compute warps
+constexpr int kLlaCompute = 256;
 constexpr int kLlaSplitLen = 1024;       // shorter sequences add the lo part of e o K
 constexpr float kLlaRescaleLog2 = 8.f;   // lazy rescale threshold (factor 256)
 constexpr int kLlaMaxPieces = 16;
-// Record of one piece: D_KK, D_KV (row-major [a][b]), ks, vs, then m, l.
+// Record of one piece: D_KK, D_KV (column-major: [a][b] at b * 128 + a), ks,
+// vs, then m, l.
 constexpr int kLlaRecKK = 0;
 constexpr int kLlaRecKV = kLlaD * kLlaD;
 constexpr int kLlaRecKs = 2 * kLlaD * kLlaD;
@@ -79,20 +82,29 @@ struct LlaLayout {
   static constexpr int kTileBytes = kTile * kLlaD * 2;   // 16 KB: two 64-column boxes of 64 rows
   static constexpr int kK = 0;
   static constexpr int kV = kK + kLlaStages * kTileBytes;
-  static constexpr int kQ = kV + kLlaStages * kTileBytes;   // float [128]: q * scale * log2(e)
-  static constexpr int kE = kQ + kLlaD * 4;                 // float [64]: weights of the tile
-  static constexpr int kRed = kE + kTile * 4;               // float [4 warps][2]
+  static constexpr int kDiag = kV + kLlaStages * kTileBytes;   // bf16 [64][64]: diag(e), 128-byte swizzle
+  static constexpr int kEcol = kDiag + kTile * kTile * 2;      // bf16 [16][64]: row 0 = e, rows 1.. zero
+  static constexpr int kQ = kEcol + 16 * kTile * 2;           // float [128]: q * scale * log2(e)
+  static constexpr int kRed = kQ + kLlaD * 4;                 // float [8 warps][2]
   static constexpr int kBar = kRed + 64;
-  // full[S], empty[S], a_full[2], a_free[2], acc_done, drain
-  static constexpr int kNumBars = 2 * kLlaStages + 6;
-  static constexpr int kMisc = kBar + kNumBars * 8;         // tmem base, abort flag
-  static constexpr int kBytes = kMisc + 16 + 1024;          // + alignment slack
+  // full[S], empty[S], e_ready, da_full, da_free, a_full[2], a_free[2], acc_done, drain
+  static constexpr int kNumBars = 2 * kLlaStages + 9;
+  static constexpr int kMisc = kBar + kNumBars * 8;           // tmem base, abort flag
+  static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
 
 // TMEM columns: D_KK [0, 128), D_KV [128, 256); A buffer b: hi words at
-// 256 + 64 b, lo words at 288 + 64 b (keys 2c, 2c+1 in word c).
-constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128;
+// 256 + 64 b, lo words at 288 + 64 b (keys 2c, 2c+1 in word c); the gather
+// G = K^T diag(e) at [384, 448); sum e k at column 448, sum e v at 464 (the
+// first of 16 columns each).
+constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128, kLlaColG = 384, kLlaColKs = 448, kLlaColVs = 464;
 __device__ __forceinline__ uint32_t lla_col_a(int buf) { return 256u + 64u * buf; }
+
+__device__ __forceinline__ float4 lds_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
 
 __device__ __forceinline__ int lla_seq_len(const LlaArgs& a, int b) {
   if (a.seq_lens == nullptr) return a.kv_len;
@@ -104,6 +116,19 @@ __device__ __forceinline__ int lla_seq_len(const LlaArgs& a, int b) {
   return n;
 }
 
+// Byte offset of element (row, col) of a [rows][64] bf16 tile with the
+// 128-byte swizzle (16-byte chunks XORed with the row within each 8 rows).
+__device__ __forceinline__ int sw128_off(int row, int col) {
+  return row * 128 + ((((col >> 3) ^ (row & 7)) << 4)) + (col & 7) * 2;
+}
+
+// Instruction descriptor of kind::f16 with both operands' majorness given
+// (bf16 A and B, fp32 accumulator, shape M x N).
+__host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
 __global__ void __launch_bounds__(kLlaThreads, 1)
     lla_moments_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const LlaArgs a) {
@@ -113,15 +138,19 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
   uint64_t* empty = full + S;
-  uint64_t* a_full = empty + S;
+  uint64_t* e_ready = empty + S;
+  uint64_t* da_full = e_ready + 1;
+  uint64_t* da_free = da_full + 1;
+  uint64_t* a_full = da_free + 1;
   uint64_t* a_free = a_full + 2;
   uint64_t* acc_done = a_free + 2;
   uint64_t* drain = acc_done + 1;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::kMisc + 4);
   float* q_s = reinterpret_cast<float*>(sm + Ly::kQ);
-  float* e_s = reinterpret_cast<float*>(sm + Ly::kE);
   float* red_s = reinterpret_cast<float*>(sm + Ly::kRed);
+  __nv_bfloat16* diag_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kDiag);
+  __nv_bfloat16* ecol_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kEcol);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int piece = blockIdx.x % a.pieces;
@@ -162,6 +191,9 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
+    mbar_init(e_ready, kLlaCompute);
+    mbar_init(da_full, 1);
+    mbar_init(da_free, kLlaCompute);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&a_full[i], kLlaCompute);
       mbar_init(&a_free[i], 1);
@@ -173,6 +205,10 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   }
   if (threadIdx.x < kLlaD)
     q_s[threadIdx.x] = __bfloat162float(a.q[(size_t)bh * kLlaD + threadIdx.x]) * a.scale_log2;
+  // diag(e) and [e; 0] start as zeros; only their e entries change per tile
+  for (int i = threadIdx.x; i < (kTile * kTile + 16 * kTile) / 8; i += kLlaThreads)
+    reinterpret_cast<uint4*>(sm + Ly::kDiag)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_base_s, 512);
     tmem_relinquish();
@@ -216,11 +252,18 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // D_KK += A . K and D_KV += A . V, A = (e o K)^T from tensor memory
-    // (128 x 16 keys per step), K and V MN-major from shared memory.
+    // Per tile: the gather G = K^T diag(e) (128 x 64, A = the K tile read as
+    // MN-major, B = diag(e)), the first moments sum e k += K^T [e 0..] and
+    // sum e v += V^T [e 0..] (128 x 16); once the compute warps have packed
+    // G into A = (e o K)^T: D_KK += A . K and D_KV += A . V (TS, K and V as
+    // MN-major B operands).
+    constexpr uint32_t kIdG = idesc_bf16_ab(128, kTile, true, false);
+    constexpr uint32_t kIdM = idesc_bf16_ab(128, 16, true, false);
     constexpr uint32_t kId = idesc_bf16(128, kLlaD, true);
-    const uint64_t dk = smem_desc_sw128(smem_u32(sm + Ly::kK), Ly::kTileBytes / 2, 1024);
-    const uint64_t dv = smem_desc_sw128(smem_u32(sm + Ly::kV), Ly::kTileBytes / 2, 1024);
+    const uint64_t dkA = smem_desc_sw128(smem_u32(sm + Ly::kK), Ly::kTileBytes / 2, 1024);   // K^T, MN-major A
+    const uint64_t dvA = smem_desc_sw128(smem_u32(sm + Ly::kV), Ly::kTileBytes / 2, 1024);   // V^T, MN-major A
+    const uint64_t dd = smem_desc_sw128(smem_u32(sm + Ly::kDiag), 16, 1024);                // diag(e), K-major B
+    const uint64_t de = smem_desc_sw128(smem_u32(sm + Ly::kEcol), 16, 1024);                // [e 0..], K-major B
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
@@ -232,16 +275,30 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       }
       const int s = j % S, buf = j & 1;
       if (!(ok = wait_warp(&full[s], (j / S) & 1))) break;
+      if (!(ok = wait_warp(e_ready, j & 1))) break;
+      if (j > 0 && !(ok = wait_warp(da_free, (j - 1) & 1))) break;
+      tc_fence_after();
+      const uint64_t ks = dkA + (uint64_t)((s * Ly::kTileBytes) >> 4);
+      const uint64_t vs = dvA + (uint64_t)((s * Ly::kTileBytes) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {   // 16 keys per step: 16 rows (2048 bytes) of K, V; 32 bytes of diag, e
+        const uint64_t o0 = (uint64_t)(kk * 128), b0 = (uint64_t)(kk * 2);
+        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;   // the first moments accumulate over tiles
+        tc_mma_ss(tmem + kLlaColG, ks + o0, dd + b0, kIdG, kk > 0 ? 1u : 0u);
+        tc_mma_ss(tmem + kLlaColKs, ks + o0, de + b0, kIdM, acc);
+        tc_mma_ss(tmem + kLlaColVs, vs + o0, de + b0, kIdM, acc);
+      }
+      tc_commit(da_full);
       if (!(ok = wait_warp(&a_full[buf], (j >> 1) & 1))) break;
       tc_fence_after();
-      const uint64_t ks = dk + (uint64_t)((s * Ly::kTileBytes) >> 4);
-      const uint64_t vs = dv + (uint64_t)((s * Ly::kTileBytes) >> 4);
+      const uint64_t kb = dkA + (uint64_t)((s * Ly::kTileBytes) >> 4);   // the same tiles as MN-major B
+      const uint64_t vb = dvA + (uint64_t)((s * Ly::kTileBytes) >> 4);
       const uint32_t ahi = tmem + lla_col_a(buf);
 #pragma unroll
       for (int kk = 0; kk < 4; kk += 2) {   // 16 keys per step: 8 A words, 16 B rows (2048 bytes)
         const uint64_t o0 = (uint64_t)(kk * 128), o1 = o0 + 128;
-        tc_mma_ts4(tmem + kLlaColKK, ahi + 8u * kk, ks + o0, tmem + kLlaColKV, ahi + 8u * kk, vs + o0,
-                   tmem + kLlaColKK, ahi + 8u * (kk + 1), ks + o1, tmem + kLlaColKV, ahi + 8u * (kk + 1), vs + o1,
+        tc_mma_ts4(tmem + kLlaColKK, ahi + 8u * kk, kb + o0, tmem + kLlaColKV, ahi + 8u * kk, vb + o0,
+                   tmem + kLlaColKK, ahi + 8u * (kk + 1), kb + o1, tmem + kLlaColKV, ahi + 8u * (kk + 1), vb + o1,
                    kId, (j > 0 || kk > 0) ? 1u : 0u, 1u);
       }
       if (split_lo) {
@@ -249,9 +306,9 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         for (int kk = 0; kk < 4; kk += 2) {
           const uint64_t o0 = (uint64_t)(kk * 128), o1 = o0 + 128;
           const uint32_t alo = ahi + 32u;
-          tc_mma_ts4(tmem + kLlaColKK, alo + 8u * kk, ks + o0, tmem + kLlaColKV, alo + 8u * kk, vs + o0,
-                     tmem + kLlaColKK, alo + 8u * (kk + 1), ks + o1, tmem + kLlaColKV, alo + 8u * (kk + 1),
-                     vs + o1, kId, 1u, 1u);
+          tc_mma_ts4(tmem + kLlaColKK, alo + 8u * kk, kb + o0, tmem + kLlaColKV, alo + 8u * kk, vb + o0,
+                     tmem + kLlaColKK, alo + 8u * (kk + 1), kb + o1, tmem + kLlaColKV, alo + 8u * (kk + 1),
+                     vb + o1, kId, 1u, 1u);
         }
       }
       tc_commit(&a_free[buf]);
@@ -266,15 +323,17 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ compute
-    const int c = threadIdx.x - 64;            // 0..127
-    const int cw = warp - 2;                   // compute warp 0..3
+    // Two warps per TMEM lane quarter: warp cw (0..7) takes rows 32 (warp % 4)
+    // .. of the accumulators and the keys 32 kh .. 32 kh + 31 of each tile's
+    // gather (kh = cw / 4).
+    const int c = threadIdx.x - 64;            // 0..255
+    const int cw = warp - 2;                   // compute warp 0..7
+    const int kh = cw >> 2;                    // key half of the gather this thread packs
     const int wq = warp & 3;                   // TMEM lane quarter of this warp
-    const int row = wq * 32 + lane;            // this thread's column of K / V = TMEM lane of D
+    const int row = wq * 32 + lane;            // TMEM lane = component a of k
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const int ki = c >> 1, hf = c & 1;         // score phase: key, half of the head dim
-    // this thread's column in a swizzled tile: box, 16-byte chunk, element
-    const int cbox = row >> 6, cch = (row & 63) >> 3, cel = row & 7;
-    float m_ref = -INFINITY, l_acc = 0.f, ksum = 0.f, vsum = 0.f;
+    const int ki = c >> 2, hf = c & 3;         // score phase: key, quarter of the head dim
+    float m_ref = -INFINITY, l_acc = 0.f;
     bool fine = true;
     int j = 0;
     for (; j < n; ++j) {
@@ -287,29 +346,36 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       uint8_t* kt = sm + Ly::kK + s * Ly::kTileBytes;
       uint8_t* vt = sm + Ly::kV + s * Ly::kTileBytes;
       const int nvalid = min(kTile, len - (t0 + j) * kTile);
-      // ---- scaled score of key ki: half hf of q . k
-      float dot = 0.f;
+      // ---- scaled score of key ki: quarter hf of q . k (four partial sums)
+      float dot;
       {
-        const uint8_t* krow = kt + hf * (Ly::kTileBytes / 2) + ki * 128;
-        const float* qh = q_s + 64 * hf;
+        float d4[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint8_t* krow = kt + (hf >> 1) * (Ly::kTileBytes / 2) + ki * 128;
+        const uint32_t qh = smem_u32(q_s + 32 * hf);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
+        for (int cq = 0; cq < 4; ++cq) {
+          const int ch = 4 * (hf & 1) + cq;
           const uint4 v4 = *reinterpret_cast<const uint4*>(krow + ((ch ^ (ki & 7)) << 4));
           const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
+          const float4 qa = lds_f4(qh + 32 * cq), qb = lds_f4(qh + 32 * cq + 16);
+          const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            dot = fmaf(qh[8 * ch + 2 * e], bf16_lo_f(w4[e]), dot);
-            dot = fmaf(qh[8 * ch + 2 * e + 1], bf16_hi_f(w4[e]), dot);
+            d4[e] = fmaf(qv[2 * e], bf16_lo_f(w4[e]), d4[e]);
+            d4[e] = fmaf(qv[2 * e + 1], bf16_hi_f(w4[e]), d4[e]);
           }
         }
+        dot = (d4[0] + d4[1]) + (d4[2] + d4[3]);
       }
       dot += __shfl_xor_sync(0xffffffffu, dot, 1);
+      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
       const float sc = ki < nvalid ? dot : -INFINITY;
       const float wmax = warp_max(sc);
       if (lane == 0) red_s[cw] = wmax;
       bar_and(2, kLlaCompute, true);
-      const float tmax = fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3]));
-      // ---- running max; rescale D, ks, vs, l when it grows past the threshold
+      const float tmax = fmaxf(fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3])),
+                               fmaxf(fmaxf(red_s[4], red_s[5]), fmaxf(red_s[6], red_s[7])));
+      // ---- running max; rescale the accumulators and l when it grows past the threshold
       bool rescale = false;
       float alpha = 1.f;
       if (j == 0) {
@@ -320,14 +386,14 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         rescale = true;
       }
       if (rescale) {   // uniform: every compute thread saw the same maxima
-        const bool wd = mbar_wait_bounded(a.wait_ns, acc_done, (j - 1) & 1);   // D holds tiles < j
+        const bool wd = mbar_wait_bounded(a.wait_ns, acc_done, (j - 1) & 1);   // products of tiles < j are in
         if (!bar_and(3, kLlaCompute, wd)) {
           fine = false;
           break;
         }
         tc_fence_after();
 #pragma unroll 1
-        for (int part = 0; part < 8; ++part) {   // D_KK then D_KV, 32 columns at a time
+        for (int part = 4 * kh; part < 4 * kh + 4; ++part) {   // D_KK (kh 0) or D_KV (kh 1), 32 columns at a time
           uint32_t r[32];
           const uint32_t addr = tmem + lane_off + (uint32_t)(part * 32);
           tmem_ld32(addr, r);
@@ -336,70 +402,66 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
           tmem_st32(addr, r);
         }
+        {   // the first moments: column 0 of sum e k (kh 0) or sum e v (kh 1); the other 15 are zero
+          uint32_t r[16];
+          const uint32_t addr = tmem + lane_off + (kh ? kLlaColVs : kLlaColKs);
+          tmem_ld16(addr, r);
+          tmem_wait_ld();
+          r[0] = __float_as_uint(__uint_as_float(r[0]) * alpha);
+          tmem_st16(addr, r);
+        }
         tmem_wait_st();
         l_acc *= alpha;
-        ksum *= alpha;
-        vsum *= alpha;
       }
-      const float e = ki < nvalid ? ex2(sc - m_ref) : 0.f;
+      // ---- the weights, rounded to bf16: every product below uses these values
+      const float e = ki < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f;
       if (hf == 0) {
-        e_s[ki] = e;
         l_acc += e;
+        diag_s[sw128_off(ki, ki) >> 1] = __float2bfloat16_rn(e);
+        ecol_s[ki] = __float2bfloat16_rn(e);   // row 0 of [e 0..]: unswizzled
       }
-      // The A buffer is free once the products of tile j - 2 are done.
-      const bool wa = j < 2 || mbar_wait_bounded(a.wait_ns, &a_free[buf], ((j >> 1) - 1) & 1);
-      if (!bar_and(2, kLlaCompute, wa)) {   // also publishes e_s
-        fine = false;
-        break;
-      }
-      // ---- A = (e o K)^T: this thread's column, 64 keys as 32 bf16 pairs (hi,
-      // and lo for short sequences -- a separate instantiation, so that the
-      // long-sequence loop does not compute it)
-      auto form_a = [&](auto split_tag) {
-        constexpr bool kSplit = decltype(split_tag)::value;
-        const uint8_t* kc = kt + cbox * (Ly::kTileBytes / 2) + cel * 2;
-        const uint8_t* vc = vt + cbox * (Ly::kTileBytes / 2) + cel * 2;
-        const float2* e2s = reinterpret_cast<const float2*>(e_s);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {   // keys 32 half .. 32 half + 31: words 16 half ..
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int pp = 0; pp < 16; ++pp) {
-          const int p = 16 * half + pp;
-          const int i0 = 2 * p, i1 = 2 * p + 1;
-          const bool v0 = i0 < nvalid, v1 = i1 < nvalid;   // rows past the end may hold NaN: select
-          const int o0 = i0 * 128 + ((cch ^ (i0 & 7)) << 4), o1 = i1 * 128 + ((cch ^ (i1 & 7)) << 4);
-          const float k0 = v0 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kc + o0)) : 0.f;
-          const float k1 = v1 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(kc + o1)) : 0.f;
-          const float x0 = v0 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vc + o0)) : 0.f;
-          const float x1 = v1 ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(vc + o1)) : 0.f;
-          const float2 e01 = e2s[p];
-          const float p0 = e01.x * k0, p1 = e01.y * k1;
-          ksum += p0 + p1;
-          vsum = fmaf(e01.x, x0, fmaf(e01.y, x1, vsum));
-          hi[pp] = pack_bf16(p0, p1);
-          if constexpr (kSplit) lo[pp] = pack_bf16(p0 - bf16_lo_f(hi[pp]), p1 - bf16_hi_f(hi[pp]));
-        }
-        tmem_st16(tmem + lane_off + lla_col_a(buf) + 16u * half, hi);
-        if constexpr (kSplit) tmem_st16(tmem + lane_off + lla_col_a(buf) + 32u + 16u * half, lo);
-        }
-      };
-      if (split_lo)
-        form_a(std::true_type{});
-      else
-        form_a(std::false_type{});
       if (nvalid < kTile) {
-        // Rows past the end are B operands of the products (their A entries are
-        // 0, but 0 * NaN is not): zero them in K and V.  No thread reads them
-        // after the scores above.
+        // Rows past the end are operands of the gather and the products
+        // (their weights are 0, but 0 * NaN is not): zero them in K and V.
+        // Every score read of this tile has happened (the barrier above).
         for (int i = c; i < (kTile - nvalid) * 16; i += kLlaCompute) {
           const int r = nvalid + (i >> 4), cc = i & 15;   // cc: box (cc >> 3), chunk (cc & 7)
           const int off = (cc >> 3) * (Ly::kTileBytes / 2) + r * 128 + (cc & 7) * 16;
           *reinterpret_cast<uint4*>(kt + off) = make_uint4(0u, 0u, 0u, 0u);
           *reinterpret_cast<uint4*>(vt + off) = make_uint4(0u, 0u, 0u, 0u);
         }
-        fence_proxy_async_smem();
       }
+      fence_proxy_async_smem();
+      mbar_arrive(e_ready);
+      // ---- pack this thread's 32 keys of the gather into A = (e o K)^T
+      const bool wg = mbar_wait_bounded(a.wait_ns, da_full, j & 1);
+      const bool wa = j < 2 || mbar_wait_bounded(a.wait_ns, &a_free[buf], ((j >> 1) - 1) & 1);
+      if (!bar_and(2, kLlaCompute, wg && wa)) {
+        fine = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t g[32];
+      tmem_ld32(tmem + lane_off + kLlaColG + 32u * kh, g);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(da_free);
+      auto pack = [&](auto split_tag) {
+        constexpr bool kSplit = decltype(split_tag)::value;
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int p = 0; p < 16; ++p) {
+          const float p0 = __uint_as_float(g[2 * p]), p1 = __uint_as_float(g[2 * p + 1]);
+          hi[p] = pack_bf16(p0, p1);
+          if constexpr (kSplit) lo[p] = pack_bf16(p0 - bf16_lo_f(hi[p]), p1 - bf16_hi_f(hi[p]));
+        }
+        tmem_st16(tmem + lane_off + lla_col_a(buf) + 16u * kh, hi);
+        if constexpr (kSplit) tmem_st16(tmem + lane_off + lla_col_a(buf) + 32u + 16u * kh, lo);
+      };
+      if (split_lo)
+        pack(std::true_type{});
+      else
+        pack(std::false_type{});
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&a_full[buf]);
@@ -408,26 +470,32 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, acc_done, (n - 1) & 1);
     wl = bar_and(3, kLlaCompute, wl);
     const float lw = warp_sum(l_acc);
-    if (lane == 0) red_s[4 + cw] = lw;
+    if (lane == 0) red_s[8 + cw] = lw;
     bar_and(2, kLlaCompute, true);
     if (wl) {
       tc_fence_after();
 #pragma unroll 1
-      for (int part = 0; part < 8; ++part) {
+      for (int part = 4 * kh; part < 4 * kh + 4; ++part) {
         uint32_t r[32];
         tmem_ld32(tmem + lane_off + (uint32_t)(part * 32), r);
         tmem_wait_ld();
-        float* dst = rec + (part < 4 ? kLlaRecKK : kLlaRecKV) + row * kLlaD + (part & 3) * 32;
+        // column-major: element [a][b] at b * 128 + a, so that the warp's 32
+        // lanes (consecutive a) write 128 contiguous bytes per column
+        float* dst = rec + (part < 4 ? kLlaRecKK : kLlaRecKV) + (part & 3) * 32 * kLlaD + row;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          reinterpret_cast<float4*>(dst)[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
-                                                          __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+        for (int i = 0; i < 32; ++i) dst[i * kLlaD] = __uint_as_float(r[i]);
       }
-      rec[kLlaRecKs + row] = ksum;
-      rec[kLlaRecVs + row] = vsum;
+      {
+        uint32_t r[16];
+        tmem_ld16(tmem + lane_off + (kh ? kLlaColVs : kLlaColKs), r);
+        tmem_wait_ld();
+        rec[(kh ? kLlaRecVs : kLlaRecKs) + row] = __uint_as_float(r[0]);
+      }
       if (c == 0) {
+        float lt = 0.f;
+        for (int w = 0; w < 8; ++w) lt += red_s[8 + w];
         rec[kLlaRecM] = m_ref;
-        rec[kLlaRecM + 1] = red_s[4] + red_s[5] + red_s[6] + red_s[7];
+        rec[kLlaRecM + 1] = lt;
       }
     } else if (c == 0) {   // abandoned after a wait ran out (already reported): an empty record
       rec[kLlaRecM] = -INFINITY;
@@ -446,9 +514,10 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
 // 8 bj.. in registers (blocks on or below the diagonal; the others idle in
 // the factorisation).  Right-looking Cholesky, one column per step: the
 // column's owners publish it in shared memory, every thread updates its
-// block with the column's outer product.  The factor's columns are kept in
-// shared memory for the two triangular solves, which one warp runs with the
-// right-hand side in registers.
+// block with the column's outer product, and the owners also apply the
+// column to the right-hand side (the forward solve L z = kbar - q, one step
+// behind).  The factor's columns stay in shared memory for the back
+// substitution, which one warp runs with the vector in registers.
 constexpr int kLlaSolveThreads = 256;
 constexpr int kLlaLd = kLlaD + 1;   // padded row stride of the factor in shared memory
 
@@ -458,8 +527,10 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
   float* colb = Lm + kLlaD * kLlaLd;       // [2][128]: the current column, double-buffered
   float* kb = colb + 2 * kLlaD;            // kbar
   float* vb = kb + kLlaD;                  // vbar
-  float* rho_s = vb + kLlaD;               // rho*
-  float* part = rho_s + kLlaD;             // [8][128] partial matrix-vector products
+  float* rho_s = vb + kLlaD;               // kbar - q, reduced in place to L^-1 (kbar - q), then rho*
+  float* zs = rho_s + kLlaD;               // z = L^-1 (kbar - q)
+  float* invp = zs + kLlaD;                // 1 / L[k][k]
+  float* part = invp + kLlaD;              // [8][128] partial matrix-vector products
   float* wts = part + 8 * kLlaD;           // [kLlaMaxPieces] piece weights 2^(m_j - M)
   float* misc = wts + kLlaMaxPieces;       // [0] l, [1] kbar . rho*
 
@@ -522,24 +593,25 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
   if (active) {
     for (int p = 0; p < a.pieces; ++p) {
       if (wts[p] == 0.f) continue;
-      const float* d = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKK + r0 * kLlaD + c0;
+      // column c0 + c of the block: rows r0 .. r0 + 7 are contiguous
+      const float* d = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKK + c0 * kLlaD + r0;
       float4 v[8][2];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {   // all 16 loads in flight before any use
-        v[r][0] = *reinterpret_cast<const float4*>(d + r * kLlaD);
-        v[r][1] = *reinterpret_cast<const float4*>(d + r * kLlaD + 4);
+      for (int c = 0; c < 8; ++c) {   // all 16 loads in flight before any use
+        v[c][0] = *reinterpret_cast<const float4*>(d + c * kLlaD);
+        v[c][1] = *reinterpret_cast<const float4*>(d + c * kLlaD + 4);
       }
       const float w = wts[p];
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        blk[r][0] = fmaf(w, v[r][0].x, blk[r][0]);
-        blk[r][1] = fmaf(w, v[r][0].y, blk[r][1]);
-        blk[r][2] = fmaf(w, v[r][0].z, blk[r][2]);
-        blk[r][3] = fmaf(w, v[r][0].w, blk[r][3]);
-        blk[r][4] = fmaf(w, v[r][1].x, blk[r][4]);
-        blk[r][5] = fmaf(w, v[r][1].y, blk[r][5]);
-        blk[r][6] = fmaf(w, v[r][1].z, blk[r][6]);
-        blk[r][7] = fmaf(w, v[r][1].w, blk[r][7]);
+      for (int c = 0; c < 8; ++c) {
+        blk[0][c] = fmaf(w, v[c][0].x, blk[0][c]);
+        blk[1][c] = fmaf(w, v[c][0].y, blk[1][c]);
+        blk[2][c] = fmaf(w, v[c][0].z, blk[2][c]);
+        blk[3][c] = fmaf(w, v[c][0].w, blk[3][c]);
+        blk[4][c] = fmaf(w, v[c][1].x, blk[4][c]);
+        blk[5][c] = fmaf(w, v[c][1].y, blk[5][c]);
+        blk[6][c] = fmaf(w, v[c][1].z, blk[6][c]);
+        blk[7][c] = fmaf(w, v[c][1].w, blk[7][c]);
       }
     }
 #pragma unroll
@@ -549,7 +621,10 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
         blk[r][c] = fmaf(blk[r][c], invL, -kb[r0 + r] * kb[c0 + c]) + (r0 + r == c0 + c ? a.ridge : 0.f);
   }
 
-  // ---- Cholesky: after step k, Lm[i][k] = L[i][k] for i >= k
+  if (tid < kLlaD) rho_s[tid] = kb[tid] - __bfloat162float(a.q[orow + tid]);
+  // ---- Cholesky with the forward solve L z = kbar - q folded in: after step
+  // k, Lm[i][k] = L[i][k] for i >= k, z_k is final, and rho_s[i] (i > k)
+  // holds kbar_i - q_i - sum_{j <= k} L[i][j] z_j.
   bool bad = false;
 #pragma unroll 1
   for (int k = 0; k < kLlaD; ++k) {
@@ -568,11 +643,22 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
       bad = true;
       break;
     }
-    const float invd = 1.f / sqrtf(akk);
-    if (active && bj == bc) {
+    const float invd = rsqrtf(akk);
+    const float zk = rho_s[k] * invd;   // z_k: its updates from columns < k are in
+    if (tid == 0) {
+      zs[k] = zk;
+      invp[k] = invd;
+    }
+    if (active && bj == bc) {   // this column's rows: the factor, and their right-hand sides
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-        if (r0 + r >= k) Lm[(r0 + r) * kLlaLd + k] = col[r0 + r] * invd;
+      for (int r = 0; r < 8; ++r) {
+        const int i = r0 + r;
+        if (i >= k) {
+          const float lik = col[i] * invd;
+          Lm[i * kLlaLd + k] = lik;
+          if (i > k) rho_s[i] = fmaf(-lik, zk, rho_s[i]);
+        }
+      }
     }
     if (active && bi >= bc && bj >= bc) {   // blocks that hold rows and columns past k
       float li[8], lj[8];
@@ -595,32 +681,18 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     }
     return;
   }
-  // ---- L z = kbar - q, then L^T rho = z: one warp, rows lane + 32u in registers
+  // ---- L^T rho = z: one warp, rows lane + 32u in registers
   if (tid < 32) {
     const int lane = tid;
     float yv[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) yv[u] = kb[lane + 32 * u] - __bfloat162float(a.q[orow + lane + 32 * u]);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-#pragma unroll 1
-      for (int kk = 0; kk < 32; ++kk) {
-        const int k = 32 * u + kk;
-        const float zk = __shfl_sync(0xffffffffu, yv[u], kk) / Lm[k * kLlaLd + k];
-        if (lane == kk) yv[u] = zk;
-#pragma unroll
-        for (int v = u; v < 4; ++v) {
-          const int i = lane + 32 * v;
-          if (i > k) yv[v] = fmaf(-Lm[i * kLlaLd + k], zk, yv[v]);
-        }
-      }
-    }
+    for (int u = 0; u < 4; ++u) yv[u] = zs[lane + 32 * u];
 #pragma unroll
     for (int u = 3; u >= 0; --u) {
 #pragma unroll 1
       for (int kk = 31; kk >= 0; --kk) {
         const int k = 32 * u + kk;
-        const float xk = __shfl_sync(0xffffffffu, yv[u], kk) / Lm[k * kLlaLd + k];
+        const float xk = __shfl_sync(0xffffffffu, yv[u], kk) * invp[k];
         if (lane == kk) yv[u] = xk;
 #pragma unroll
         for (int v = 0; v <= u; ++v) {
@@ -641,40 +713,35 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
   __syncthreads();
   // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a
   {
-    const int cq = tid & 31, rg = tid >> 5;   // columns 4 cq .. 4 cq + 3, rows rg + 8 u
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int col = tid >> 1, half = tid & 1;   // rows a = 64 half .. 64 half + 63 of column col
+    float acc = 0.f;
     for (int p = 0; p < a.pieces; ++p) {
       if (wts[p] == 0.f) continue;
-      const float* dkv = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + 4 * cq;
+      const float* dkv = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + col * kLlaD + 64 * half;
       float4 v[16];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = *reinterpret_cast<const float4*>(dkv + (rg + 8 * u) * kLlaD);
-      float4 sp = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int u = 0; u < 16; ++u) v[u] = *reinterpret_cast<const float4*>(dkv + 4 * u);
+      float sp = 0.f;
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        const float r = rho_s[rg + 8 * u];
-        sp.x = fmaf(v[u].x, r, sp.x);
-        sp.y = fmaf(v[u].y, r, sp.y);
-        sp.z = fmaf(v[u].z, r, sp.z);
-        sp.w = fmaf(v[u].w, r, sp.w);
+        const float* rr = rho_s + 64 * half + 4 * u;
+        sp = fmaf(v[u].x, rr[0], fmaf(v[u].y, rr[1], fmaf(v[u].z, rr[2], fmaf(v[u].w, rr[3], sp))));
       }
-      const float w = wts[p];
-      acc = make_float4(fmaf(w, sp.x, acc.x), fmaf(w, sp.y, acc.y), fmaf(w, sp.z, acc.z), fmaf(w, sp.w, acc.w));
+      acc = fmaf(wts[p], sp, acc);
     }
-    *reinterpret_cast<float4*>(part + rg * kLlaD + 4 * cq) = acc;
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    if (half == 0) part[col] = acc;
   }
   __syncthreads();
   if (tid < kLlaD) {
-    float corr = 0.f;
-#pragma unroll
-    for (int g = 0; g < 8; ++g) corr += part[g * kLlaD + tid];
+    const float corr = part[tid];
     store_out(tid, fmaf(vb[tid], 1.f + misc[1], -corr * invL));
     if (a.rho) a.rho[orow + tid] = rho_s[tid];
   }
 }
 
 constexpr int lla_solve_smem_bytes() {
-  return (kLlaD * kLlaLd + 2 * kLlaD + 3 * kLlaD + 8 * kLlaD + kLlaMaxPieces + 4) * 4;
+  return (kLlaD * kLlaLd + 2 * kLlaD + 5 * kLlaD + 8 * kLlaD + kLlaMaxPieces + 4) * 4;
 }
 
 }  // namespace plx
