@@ -364,9 +364,11 @@ def bench_decode(args, w, rank, world, dev, peaks, peaks_kind):
 def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
     """End to end through the public API: each step copies the step's q and
     rho from pinned host memory, runs the decode and reads the output back.
-    The headline figure runs a prepared decode (DecodePlan, made once per
-    buffer set, as a serving loop with fixed buffers would); the one-shot
-    decode() call is timed the same way beside it."""
+    The headline figure is one call per step of a prepared decode
+    (DecodePlan.run_io: both copies in, the launch and the copy out, queued
+    by the library; the plan is made once per buffer set, as a serving loop
+    with fixed buffers would); the one-shot decode() call with torch copies
+    around it is timed the same way beside it."""
     copies = len(insts)
     host = []
     for x in insts:
@@ -381,10 +383,7 @@ def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
 
     def one_plan(i):
         c = i % copies
-        dq[c].copy_(host[c]["q"], non_blocking=True)
-        dr[c].copy_(host[c]["rho"], non_blocking=True)
-        plans[c].run()
-        out_host[c].copy_(outs[c], non_blocking=True)
+        plans[c].run_io(host[c]["q"], host[c]["rho"], out_host[c])
 
     def one_call(i):
         c = i % copies
@@ -419,7 +418,7 @@ def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
     d2h = outs[0].numel() * outs[0].element_size()
     return {"value": round(gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "steps": K, "ms_per_step": round(ms, 6),
-            "host_wall_ms_per_step": round(wall, 6), "api": "DecodePlan.run (parallax_decode_plan_run)",
+            "host_wall_ms_per_step": round(wall, 6), "api": "DecodePlan.run_io (parallax_decode_plan_run_io)",
             "one_shot_call": {"value": round(gbs_call, 2), "ms_per_step": round(ms_call, 6),
                               "host_wall_ms_per_step": round(wall_call, 6), "api": "decode (parallax_decode)"},
             "note": "query and probe copied from pinned host memory and output read back every step; "

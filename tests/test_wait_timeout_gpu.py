@@ -105,3 +105,19 @@ def test_wait_limit_setter_round_trips(px):
         assert px.set_wait_limit_ns(prev) == 123456
     finally:
         px.set_wait_limit_ns(prev)
+
+
+def test_lla_wait_timeout_then_recovery(px):
+    inp = W.small_decode_inputs(2, 4, 2, 128, 4096, seed=55)
+    inp = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
+
+    def run():
+        return px.lla_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["scale"], 0.01, out_dtype=torch.float32)
+
+    code = _timed_out(px, run)
+    assert code & px.DEVERR_TIMEOUT, f"error word {code}"
+    out, rho = run()
+    assert px.last_device_error() == 0
+    rho_ref, ref = oracle.lla_decode(to_f64(inp["q"]), F64View(inp["k_cache"]), F64View(inp["v_cache"]),
+                                     inp["scale"], 0.01)
+    assert_parity(out.cpu().numpy(), ref, TOL_BF16, "LLA after a timeout")
