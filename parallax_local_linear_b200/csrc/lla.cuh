@@ -510,26 +510,22 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
 
 // ---------------------------------------------------------------- solve
 // One CTA (256 threads) per (sequence, query head).  Thread (bi, bj) of a
-// 16 x 16 grid holds the 8 x 8 block of S_KK + ridge I at rows 8 bi.., columns
-// 8 bj.. in registers (blocks on or below the diagonal; the others idle in
-// the factorisation).  Right-looking Cholesky, one column per step: the
-// column's owners publish it in shared memory, every thread updates its
-// block with the column's outer product, and the owners also apply the
-// column to the right-hand side (the forward solve L z = kbar - q, one step
-// behind).  The factor's columns stay in shared memory for the back
-// substitution, which one warp runs with the vector in registers.
+// 16 x 16 grid holds the 8 x 8 block of S_KK + ridge I at rows 8 bi..,
+// columns 8 bj.. in registers (blocks on or below the diagonal; the others
+// idle in the factorisation).  Blocked right-looking Cholesky, 8 columns per
+// step: 16 steps of two barriers each.  The factor goes to shared memory for
+// the two triangular solves, which one warp runs with the vector in
+// registers.
 constexpr int kLlaSolveThreads = 256;
 constexpr int kLlaLd = kLlaD + 1;   // padded row stride of the factor in shared memory
 
 __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaArgs a) {
   extern __shared__ float smf[];
   float* Lm = smf;                         // [128][129]: column k of the factor, rows >= k
-  float* colb = Lm + kLlaD * kLlaLd;       // [2][128]: the current column, double-buffered
-  float* kb = colb + 2 * kLlaD;            // kbar
+  float* kb = Lm + kLlaD * kLlaLd;         // kbar
   float* vb = kb + kLlaD;                  // vbar
-  float* rho_s = vb + kLlaD;               // kbar - q, reduced in place to L^-1 (kbar - q), then rho*
-  float* zs = rho_s + kLlaD;               // z = L^-1 (kbar - q)
-  float* invp = zs + kLlaD;                // 1 / L[k][k]
+  float* rho_s = vb + kLlaD;               // rho*
+  float* invp = rho_s + kLlaD;             // 1 / L[k][k]
   float* part = invp + kLlaD;              // [8][128] partial matrix-vector products
   float* wts = part + 8 * kLlaD;           // [kLlaMaxPieces] piece weights 2^(m_j - M)
   float* misc = wts + kLlaMaxPieces;       // [0] l, [1] kbar . rho*
@@ -621,55 +617,74 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
         blk[r][c] = fmaf(blk[r][c], invL, -kb[r0 + r] * kb[c0 + c]) + (r0 + r == c0 + c ? a.ridge : 0.f);
   }
 
-  if (tid < kLlaD) rho_s[tid] = kb[tid] - __bfloat162float(a.q[orow + tid]);
-  // ---- Cholesky with the forward solve L z = kbar - q folded in: after step
-  // k, Lm[i][k] = L[i][k] for i >= k, z_k is final, and rho_s[i] (i > k)
-  // holds kbar_i - q_i - sum_{j <= k} L[i][j] z_j.
+  // ---- blocked Cholesky, one panel of 8 columns per step P: the diagonal
+  // block's owner factors it in registers; the blocks below it solve
+  // against that factor (X L_PP^T = A); the blocks right of the panel and
+  // on or below the diagonal take the rank-8 update.  Lm ends up holding L.
+  int* flag_s = reinterpret_cast<int*>(misc + 2);
+  if (tid == 0) *flag_s = 0;
   bool bad = false;
 #pragma unroll 1
-  for (int k = 0; k < kLlaD; ++k) {
-    const int bc = k >> 3, cc = k & 7;
-    float* col = colb + (k & 1) * kLlaD;
-    if (active && bj == bc) {
+  for (int P = 0; P < 16; ++P) {
+    if (bi == P && bj == P) {   // the diagonal block: L_PP L_PP^T = A_PP
+      bool ok = true;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float akk = blk[k][k];
+        ok = ok && akk > 0.f && isfinite(akk);
+        const float invd = rsqrtf(akk);
+        blk[k][k] = akk * invd;
+        invp[8 * P + k] = invd;
+#pragma unroll
+        for (int i = k + 1; i < 8; ++i) blk[i][k] *= invd;
+#pragma unroll
+        for (int i = k + 1; i < 8; ++i)
+#pragma unroll
+          for (int jj = k + 1; jj <= i; ++jj) blk[i][jj] = fmaf(-blk[i][k], blk[jj][k], blk[i][jj]);
+      }
+      if (!ok) *flag_s = 1;
 #pragma unroll
       for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          if (c == cc) col[r0 + r] = blk[r][c];
+        for (int c = 0; c <= r; ++c) Lm[(r0 + r) * kLlaLd + c0 + c] = blk[r][c];
     }
     __syncthreads();
-    const float akk = col[k];
-    if (!(akk > 0.f) || !isfinite(akk)) {   // not numerically positive definite (uniform)
+    if (*flag_s != 0) {   // not numerically positive definite (uniform)
       bad = true;
       break;
     }
-    const float invd = rsqrtf(akk);
-    const float zk = rho_s[k] * invd;   // z_k: its updates from columns < k are in
-    if (tid == 0) {
-      zs[k] = zk;
-      invp[k] = invd;
-    }
-    if (active && bj == bc) {   // this column's rows: the factor, and their right-hand sides
+    if (bj == P && bi > P) {   // the panel: X L_PP^T = A, column by column
+      const float* lpp = Lm + (8 * P) * kLlaLd + 8 * P;
 #pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int i = r0 + r;
-        if (i >= k) {
-          const float lik = col[i] * invd;
-          Lm[i * kLlaLd + k] = lik;
-          if (i > k) rho_s[i] = fmaf(-lik, zk, rho_s[i]);
+      for (int c = 0; c < 8; ++c) {
+        const float invd = invp[8 * P + c];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+          float x = blk[r][c];
+#pragma unroll
+          for (int m = 0; m < c; ++m) x = fmaf(-blk[r][m], lpp[c * kLlaLd + m], x);
+          blk[r][c] = x * invd;
         }
       }
-    }
-    if (active && bi >= bc && bj >= bc) {   // blocks that hold rows and columns past k
-      float li[8], lj[8];
-#pragma unroll
-      for (int r = 0; r < 8; ++r) li[r] = r0 + r > k ? col[r0 + r] * invd : 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) lj[c] = c0 + c > k ? col[c0 + c] * invd : 0.f;
 #pragma unroll
       for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int c = 0; c < 8; ++c) blk[r][c] = fmaf(-li[r], lj[c], blk[r][c]);
+        for (int c = 0; c < 8; ++c) Lm[(r0 + r) * kLlaLd + c0 + c] = blk[r][c];
+    }
+    __syncthreads();
+    if (active && bj > P) {   // rank-8 update of the trailing blocks
+#pragma unroll
+      for (int m = 0; m < 8; ++m) {
+        float li[8], lj[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) li[r] = Lm[(r0 + r) * kLlaLd + 8 * P + m];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) lj[c] = Lm[(c0 + c) * kLlaLd + 8 * P + m];
+#pragma unroll
+        for (int r = 0; r < 8; ++r)
+#pragma unroll
+          for (int c = 0; c < 8; ++c) blk[r][c] = fmaf(-li[r], lj[c], blk[r][c]);
+      }
     }
   }
   __syncthreads();
@@ -681,12 +696,26 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     }
     return;
   }
-  // ---- L^T rho = z: one warp, rows lane + 32u in registers
+  // ---- L z = kbar - q, then L^T rho = z: one warp, rows lane + 32u in registers
   if (tid < 32) {
     const int lane = tid;
     float yv[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) yv[u] = zs[lane + 32 * u];
+    for (int u = 0; u < 4; ++u) yv[u] = kb[lane + 32 * u] - __bfloat162float(a.q[orow + lane + 32 * u]);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+#pragma unroll 1
+      for (int kk = 0; kk < 32; ++kk) {
+        const int k = 32 * u + kk;
+        const float zk = __shfl_sync(0xffffffffu, yv[u], kk) * invp[k];
+        if (lane == kk) yv[u] = zk;
+#pragma unroll
+        for (int v = u; v < 4; ++v) {
+          const int i = lane + 32 * v;
+          if (i > k) yv[v] = fmaf(-Lm[i * kLlaLd + k], zk, yv[v]);
+        }
+      }
+    }
 #pragma unroll
     for (int u = 3; u >= 0; --u) {
 #pragma unroll 1
@@ -741,7 +770,7 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
 }
 
 constexpr int lla_solve_smem_bytes() {
-  return (kLlaD * kLlaLd + 2 * kLlaD + 5 * kLlaD + 8 * kLlaD + kLlaMaxPieces + 4) * 4;
+  return (kLlaD * kLlaLd + 4 * kLlaD + 8 * kLlaD + kLlaMaxPieces + 4) * 4;
 }
 
 }  // namespace plx
