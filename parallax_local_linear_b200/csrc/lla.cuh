@@ -82,23 +82,27 @@ struct LlaLayout {
   static constexpr int kTileBytes = kTile * kLlaD * 2;   // 16 KB: two 64-column boxes of 64 rows
   static constexpr int kK = 0;
   static constexpr int kV = kK + kLlaStages * kTileBytes;
-  static constexpr int kDiag = kV + kLlaStages * kTileBytes;   // bf16 [64][64]: diag(e), 128-byte swizzle
-  static constexpr int kEcol = kDiag + kTile * kTile * 2;      // bf16 [16][64]: row 0 = e, rows 1.. zero
-  static constexpr int kQ = kEcol + 16 * kTile * 2;           // float [128]: q * scale * log2(e)
+  static constexpr int kDiagBytes = kTile * kTile * 2;        // bf16 [64][64]: diag(e), 128-byte swizzle
+  static constexpr int kEcolBytes = 16 * kTile * 2;           // bf16 [16][64]: row 0 = e, rows 1.. zero
+  static constexpr int kDiag = kV + kLlaStages * kTileBytes;  // two buffers (tile parity)
+  static constexpr int kEcol = kDiag + 2 * kDiagBytes;        // two buffers
+  static constexpr int kQ = kEcol + 2 * kEcolBytes;           // float [128]: q * scale * log2(e)
   static constexpr int kRed = kQ + kLlaD * 4;                 // float [8 warps][2]
   static constexpr int kBar = kRed + 64;
-  // full[S], empty[S], e_ready, da_full, da_free, a_full[2], a_free[2], acc_done, drain
+  // full[S], empty[S], e_ready[2], da_full[2], da_free[2], a_full, a_free, drain
+  // (the three per-tile hand-offs that run a tile ahead alternate between
+  // two barriers by tile parity, so neither side can be two phases ahead)
   static constexpr int kNumBars = 2 * kLlaStages + 9;
   static constexpr int kMisc = kBar + kNumBars * 8;           // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
 
-// TMEM columns: D_KK [0, 128), D_KV [128, 256); A buffer b: hi words at
-// 256 + 64 b, lo words at 288 + 64 b (keys 2c, 2c+1 in word c); the gather
-// G = K^T diag(e) at [384, 448); sum e k at column 448, sum e v at 464 (the
+// TMEM columns: D_KK [0, 128), D_KV [128, 256); A: hi words at 256, lo
+// words at 288 (keys 2c, 2c+1 in word c); the gather G = K^T diag(e) of
+// tile j at 320 + 64 (j % 2); sum e k at column 448, sum e v at 464 (the
 // first of 16 columns each).
-constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128, kLlaColG = 384, kLlaColKs = 448, kLlaColVs = 464;
-__device__ __forceinline__ uint32_t lla_col_a(int buf) { return 256u + 64u * buf; }
+constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128, kLlaColA = 256, kLlaColKs = 448, kLlaColVs = 464;
+__device__ __forceinline__ uint32_t lla_col_g(int buf) { return 320u + 64u * buf; }
 
 __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   float4 v;
@@ -139,18 +143,15 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
   uint64_t* empty = full + S;
   uint64_t* e_ready = empty + S;
-  uint64_t* da_full = e_ready + 1;
-  uint64_t* da_free = da_full + 1;
-  uint64_t* a_full = da_free + 1;
-  uint64_t* a_free = a_full + 2;
-  uint64_t* acc_done = a_free + 2;
-  uint64_t* drain = acc_done + 1;
+  uint64_t* da_full = e_ready + 2;
+  uint64_t* da_free = da_full + 2;
+  uint64_t* a_full = da_free + 2;
+  uint64_t* a_free = a_full + 1;
+  uint64_t* drain = a_free + 1;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::kMisc + 4);
   float* q_s = reinterpret_cast<float*>(sm + Ly::kQ);
   float* red_s = reinterpret_cast<float*>(sm + Ly::kRed);
-  __nv_bfloat16* diag_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kDiag);
-  __nv_bfloat16* ecol_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kEcol);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int piece = blockIdx.x % a.pieces;
@@ -191,14 +192,13 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(e_ready, kLlaCompute);
-    mbar_init(da_full, 1);
-    mbar_init(da_free, kLlaCompute);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&a_full[i], kLlaCompute);
-      mbar_init(&a_free[i], 1);
+      mbar_init(&e_ready[i], kLlaCompute);
+      mbar_init(&da_full[i], 1);
+      mbar_init(&da_free[i], kLlaCompute);
     }
-    mbar_init(acc_done, 1);
+    mbar_init(a_full, kLlaCompute);
+    mbar_init(a_free, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -206,7 +206,7 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   if (threadIdx.x < kLlaD)
     q_s[threadIdx.x] = __bfloat162float(a.q[(size_t)bh * kLlaD + threadIdx.x]) * a.scale_log2;
   // diag(e) and [e; 0] start as zeros; only their e entries change per tile
-  for (int i = threadIdx.x; i < (kTile * kTile + 16 * kTile) / 8; i += kLlaThreads)
+  for (int i = threadIdx.x; i < 2 * (Ly::kDiagBytes + Ly::kEcolBytes) / 16; i += kLlaThreads)
     reinterpret_cast<uint4*>(sm + Ly::kDiag)[i] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
   if (warp == 1) {
@@ -267,39 +267,20 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-        ok = false;
-        break;
-      }
-      const int s = j % S, buf = j & 1;
-      if (!(ok = wait_warp(&full[s], (j / S) & 1))) break;
-      if (!(ok = wait_warp(e_ready, j & 1))) break;
-      if (j > 0 && !(ok = wait_warp(da_free, (j - 1) & 1))) break;
-      tc_fence_after();
-      const uint64_t ks = dkA + (uint64_t)((s * Ly::kTileBytes) >> 4);
-      const uint64_t vs = dvA + (uint64_t)((s * Ly::kTileBytes) >> 4);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {   // 16 keys per step: 16 rows (2048 bytes) of K, V; 32 bytes of diag, e
-        const uint64_t o0 = (uint64_t)(kk * 128), b0 = (uint64_t)(kk * 2);
-        const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;   // the first moments accumulate over tiles
-        tc_mma_ss(tmem + kLlaColG, ks + o0, dd + b0, kIdG, kk > 0 ? 1u : 0u);
-        tc_mma_ss(tmem + kLlaColKs, ks + o0, de + b0, kIdM, acc);
-        tc_mma_ss(tmem + kLlaColVs, vs + o0, de + b0, kIdM, acc);
-      }
-      tc_commit(da_full);
-      if (!(ok = wait_warp(&a_full[buf], (j >> 1) & 1))) break;
-      tc_fence_after();
-      const uint64_t kb = dkA + (uint64_t)((s * Ly::kTileBytes) >> 4);   // the same tiles as MN-major B
-      const uint64_t vb = dvA + (uint64_t)((s * Ly::kTileBytes) >> 4);
-      const uint32_t ahi = tmem + lla_col_a(buf);
+    // main(j) = D_KK += A . K(j), D_KV += A . V(j); A holds tile j's packed
+    // gather.  Issue order G(0), G(1), main(0), G(2), main(1), ...: the
+    // gather of the next tile runs while the compute warps pack this one.
+    auto issue_main = [&](int jm) {
+      const int sm_ = jm % S;
+      const uint64_t kb = dkA + (uint64_t)((sm_ * Ly::kTileBytes) >> 4);   // the tiles as MN-major B
+      const uint64_t vb = dvA + (uint64_t)((sm_ * Ly::kTileBytes) >> 4);
+      const uint32_t ahi = tmem + kLlaColA;
 #pragma unroll
       for (int kk = 0; kk < 4; kk += 2) {   // 16 keys per step: 8 A words, 16 B rows (2048 bytes)
         const uint64_t o0 = (uint64_t)(kk * 128), o1 = o0 + 128;
         tc_mma_ts4(tmem + kLlaColKK, ahi + 8u * kk, kb + o0, tmem + kLlaColKV, ahi + 8u * kk, vb + o0,
                    tmem + kLlaColKK, ahi + 8u * (kk + 1), kb + o1, tmem + kLlaColKV, ahi + 8u * (kk + 1), vb + o1,
-                   kId, (j > 0 || kk > 0) ? 1u : 0u, 1u);
+                   kId, (jm > 0 || kk > 0) ? 1u : 0u, 1u);
       }
       if (split_lo) {
 #pragma unroll
@@ -311,9 +292,40 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
                      vb + o1, kId, 1u, 1u);
         }
       }
-      tc_commit(&a_free[buf]);
-      tc_commit(&empty[s]);
-      tc_commit(acc_done);
+      tc_commit(a_free);
+      tc_commit(&empty[sm_]);
+    };
+    bool ok = true;
+    for (int j = 0; j <= n; ++j) {
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
+      if (j < n) {   // G(j) and the first moments of tile j
+        const int s = j % S, gb = j & 1;
+        if (!(ok = wait_warp(&full[s], (j / S) & 1))) break;
+        if (!(ok = wait_warp(&e_ready[gb], (j >> 1) & 1))) break;
+        if (j >= 2 && !(ok = wait_warp(&da_free[gb], ((j >> 1) - 1) & 1))) break;   // G buffer gb was read
+        tc_fence_after();
+        const uint64_t ks = dkA + (uint64_t)((s * Ly::kTileBytes) >> 4);
+        const uint64_t vs = dvA + (uint64_t)((s * Ly::kTileBytes) >> 4);
+        const uint64_t ddb = dd + (uint64_t)((gb * Ly::kDiagBytes) >> 4);
+        const uint64_t deb = de + (uint64_t)((gb * Ly::kEcolBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {   // 16 keys per step: 16 rows (2048 bytes) of K, V; 32 bytes of diag, e
+          const uint64_t o0 = (uint64_t)(kk * 128), b0 = (uint64_t)(kk * 2);
+          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;   // the first moments accumulate over tiles
+          tc_mma_ss(tmem + lla_col_g(gb), ks + o0, ddb + b0, kIdG, kk > 0 ? 1u : 0u);
+          tc_mma_ss(tmem + kLlaColKs, ks + o0, deb + b0, kIdM, acc);
+          tc_mma_ss(tmem + kLlaColVs, vs + o0, deb + b0, kIdM, acc);
+        }
+        tc_commit(&da_full[gb]);
+      }
+      if (j >= 1) {   // main(j - 1), once the compute warps have packed tile j - 1
+        if (!(ok = wait_warp(a_full, (j - 1) & 1))) break;
+        tc_fence_after();
+        issue_main(j - 1);
+      }
     }
     if (!ok && lane == 0) *abort_flag = 1;
     // Every issued MMA must complete before tensor memory is released.
@@ -334,18 +346,17 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const int ki = c >> 2, hf = c & 3;         // score phase: key, quarter of the head dim
     float m_ref = -INFINITY, l_acc = 0.f;
-    bool fine = true;
-    int j = 0;
-    for (; j < n; ++j) {
-      const int s = j % S, buf = j & 1;
-      const bool w = !*abort_flag && mbar_wait_bounded(a.wait_ns, &full[s], (j / S) & 1);
-      if (!bar_and(1, kLlaCompute, w && fine)) {
-        fine = false;
-        break;
-      }
+    // Tile t's scores, weights, diag(e) and [e 0 ..] (buffers t % 2), then
+    // e_ready.  A new running max rescales sum e k, sum e v (after G(t - 1),
+    // before G(t)) at once, and returns the factor that D_KK, D_KV take
+    // after main(t - 1) and before main(t).
+    auto scores_phase = [&](int t, float& alpha_d) -> bool {
+      const int s = t % S, gb = t & 1;
+      const bool w = !*abort_flag && mbar_wait_bounded(a.wait_ns, &full[s], (t / S) & 1);
+      if (!bar_and(1, kLlaCompute, w)) return false;
       uint8_t* kt = sm + Ly::kK + s * Ly::kTileBytes;
       uint8_t* vt = sm + Ly::kV + s * Ly::kTileBytes;
-      const int nvalid = min(kTile, len - (t0 + j) * kTile);
+      const int nvalid = min(kTile, len - (t0 + t) * kTile);
       // ---- scaled score of key ki: quarter hf of q . k (four partial sums)
       float dot;
       {
@@ -375,48 +386,33 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       bar_and(2, kLlaCompute, true);
       const float tmax = fmaxf(fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3])),
                                fmaxf(fmaxf(red_s[4], red_s[5]), fmaxf(red_s[6], red_s[7])));
-      // ---- running max; rescale the accumulators and l when it grows past the threshold
-      bool rescale = false;
-      float alpha = 1.f;
-      if (j == 0) {
+      alpha_d = 1.f;
+      if (t == 0) {
         m_ref = tmax;   // the piece's first tile holds a key: tmax is finite
-      } else if (tmax > m_ref + kLlaRescaleLog2) {
-        alpha = ex2(m_ref - tmax);
+      } else if (tmax > m_ref + kLlaRescaleLog2) {   // uniform: every compute thread saw the same maxima
+        const float alpha = ex2(m_ref - tmax);
         m_ref = tmax;
-        rescale = true;
-      }
-      if (rescale) {   // uniform: every compute thread saw the same maxima
-        const bool wd = mbar_wait_bounded(a.wait_ns, acc_done, (j - 1) & 1);   // products of tiles < j are in
-        if (!bar_and(3, kLlaCompute, wd)) {
-          fine = false;
-          break;
-        }
+        alpha_d = alpha;
+        // sum e k, sum e v hold tiles < t once G(t - 1) is done
+        const bool wd = mbar_wait_bounded(a.wait_ns, &da_full[(t - 1) & 1], ((t - 1) >> 1) & 1);
+        if (!bar_and(3, kLlaCompute, wd)) return false;
         tc_fence_after();
-#pragma unroll 1
-        for (int part = 4 * kh; part < 4 * kh + 4; ++part) {   // D_KK (kh 0) or D_KV (kh 1), 32 columns at a time
-          uint32_t r[32];
-          const uint32_t addr = tmem + lane_off + (uint32_t)(part * 32);
-          tmem_ld32(addr, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(addr, r);
-        }
-        {   // the first moments: column 0 of sum e k (kh 0) or sum e v (kh 1); the other 15 are zero
-          uint32_t r[16];
-          const uint32_t addr = tmem + lane_off + (kh ? kLlaColVs : kLlaColKs);
-          tmem_ld16(addr, r);
-          tmem_wait_ld();
-          r[0] = __float_as_uint(__uint_as_float(r[0]) * alpha);
-          tmem_st16(addr, r);
-        }
+        uint32_t r[16];   // column 0 of sum e k (kh 0) or sum e v (kh 1); the other 15 are zero
+        const uint32_t addr = tmem + lane_off + (kh ? kLlaColVs : kLlaColKs);
+        tmem_ld16(addr, r);
+        tmem_wait_ld();
+        r[0] = __float_as_uint(__uint_as_float(r[0]) * alpha);
+        tmem_st16(addr, r);
         tmem_wait_st();
+        tc_fence_before();
         l_acc *= alpha;
       }
       // ---- the weights, rounded to bf16: every product below uses these values
       const float e = ki < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f;
       if (hf == 0) {
         l_acc += e;
+        __nv_bfloat16* diag_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kDiag + gb * Ly::kDiagBytes);
+        __nv_bfloat16* ecol_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kEcol + gb * Ly::kEcolBytes);
         diag_s[sw128_off(ki, ki) >> 1] = __float2bfloat16_rn(e);
         ecol_s[ki] = __float2bfloat16_rn(e);   // row 0 of [e 0..]: unswizzled
       }
@@ -432,20 +428,33 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      mbar_arrive(e_ready);
-      // ---- pack this thread's 32 keys of the gather into A = (e o K)^T
-      const bool wg = mbar_wait_bounded(a.wait_ns, da_full, j & 1);
-      const bool wa = j < 2 || mbar_wait_bounded(a.wait_ns, &a_free[buf], ((j >> 1) - 1) & 1);
-      if (!bar_and(2, kLlaCompute, wg && wa)) {
-        fine = false;
-        break;
-      }
+      mbar_arrive(&e_ready[gb]);
+      return true;
+    };
+    // Tile t's gather into A = (e o K)^T (after main(t - 1) has read A), and
+    // the deferred rescale of D_KK, D_KV.
+    auto pack_phase = [&](int t, float alpha_d) -> bool {
+      const bool wg = mbar_wait_bounded(a.wait_ns, &da_full[t & 1], (t >> 1) & 1);
+      const bool wa = t == 0 || mbar_wait_bounded(a.wait_ns, a_free, (t - 1) & 1);
+      if (!bar_and(2, kLlaCompute, wg && wa)) return false;
       tc_fence_after();
+      if (alpha_d != 1.f) {   // uniform; main(t - 1) is done
+#pragma unroll 1
+        for (int part = 4 * kh; part < 4 * kh + 4; ++part) {   // D_KK (kh 0) or D_KV (kh 1), 32 columns at a time
+          uint32_t r[32];
+          const uint32_t addr = tmem + lane_off + (uint32_t)(part * 32);
+          tmem_ld32(addr, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha_d);
+          tmem_st32(addr, r);
+        }
+      }
       uint32_t g[32];
-      tmem_ld32(tmem + lane_off + kLlaColG + 32u * kh, g);
+      tmem_ld32(tmem + lane_off + lla_col_g(t & 1) + 32u * kh, g);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(da_free);
+      mbar_arrive(&da_free[t & 1]);
       auto pack = [&](auto split_tag) {
         constexpr bool kSplit = decltype(split_tag)::value;
         uint32_t hi[16], lo[16];
@@ -455,8 +464,8 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
           hi[p] = pack_bf16(p0, p1);
           if constexpr (kSplit) lo[p] = pack_bf16(p0 - bf16_lo_f(hi[p]), p1 - bf16_hi_f(hi[p]));
         }
-        tmem_st16(tmem + lane_off + lla_col_a(buf) + 16u * kh, hi);
-        if constexpr (kSplit) tmem_st16(tmem + lane_off + lla_col_a(buf) + 32u + 16u * kh, lo);
+        tmem_st16(tmem + lane_off + kLlaColA + 16u * kh, hi);
+        if constexpr (kSplit) tmem_st16(tmem + lane_off + kLlaColA + 32u + 16u * kh, lo);
       };
       if (split_lo)
         pack(std::true_type{});
@@ -464,10 +473,22 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         pack(std::false_type{});
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&a_full[buf]);
+      mbar_arrive(a_full);
+      return true;
+    };
+    // scores(t + 1) runs before pack(t), so the gather of tile t + 1 overlaps
+    // the packing of tile t and main(t).
+    float alpha_pack = 1.f;   // D's rescale before main(t), decided by scores(t)
+    bool fine = scores_phase(0, alpha_pack);
+    int j = 0;
+    for (; fine && j < n; ++j) {
+      float alpha_next = 1.f;
+      if (j + 1 < n && !(fine = scores_phase(j + 1, alpha_next))) break;
+      if (!(fine = pack_phase(j, alpha_pack))) break;
+      alpha_pack = alpha_next;
     }
     // ---- the piece's record: wait for the last products, then write
-    bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, acc_done, (n - 1) & 1);
+    bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, a_free, (n - 1) & 1);
     wl = bar_and(3, kLlaCompute, wl);
     const float lw = warp_sum(l_acc);
     if (lane == 0) red_s[8 + cw] = lw;
