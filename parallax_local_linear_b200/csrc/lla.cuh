@@ -20,10 +20,12 @@
 //     a running max m (2^(s - m) weights, rescaled lazily as in the prefill),
 //         l = sum e,  ks = sum e k,  vs = sum e v,
 //         D_KK = sum e k k^T,  D_KV = sum e k v^T          (128 x 128 each)
-//     All of it runs on the tensor cores except the scores: per 64-key tile
-//     the weights e (rounded to bf16 once, so that every sum uses the same
-//     values) go into diag(e) and the column [e 0 ..] in shared memory; the
-//     MMAs G = K^T diag(e) (so row a of G holds e_i k_ia, exact in fp32),
+//     All of the arithmetic over keys runs on the tensor cores: per 64-key
+//     tile the scores S = K q (M = 64 keys, N = 8: q is row 0 of an 8-row
+//     operand), read back by four warps, 16 keys each; the weights e
+//     (rounded to bf16 once, so that every sum uses the same values) go into
+//     diag(e) and the column [e 0 ..] in shared memory; the MMAs
+//     G = K^T diag(e) (so row a of G holds e_i k_ia, exact in fp32),
 //     ks += K^T [e 0 ..] and vs += V^T [e 0 ..] read the K and V tiles as
 //     MN-major A operands; the compute warps pack G into A = (e o K)^T in
 //     tensor memory (bf16 pairs); then D_KK += A . K and D_KV += A . V (K, V
@@ -86,13 +88,15 @@ struct LlaLayout {
   static constexpr int kEcolBytes = 16 * kTile * 2;           // bf16 [16][64]: row 0 = e, rows 1.. zero
   static constexpr int kDiag = kV + kLlaStages * kTileBytes;  // two buffers (tile parity)
   static constexpr int kEcol = kDiag + 2 * kDiagBytes;        // two buffers
-  static constexpr int kQ = kEcol + 2 * kEcolBytes;           // float [128]: q * scale * log2(e)
-  static constexpr int kRed = kQ + kLlaD * 4;                 // float [8 warps][2]
+  static constexpr int kQBytes = 8 * kLlaD * 2;               // bf16 [8][128]: row 0 = q, rows 1.. zero
+  static constexpr int kQ = kEcol + 2 * kEcolBytes;           // K-major B operand, two 64-column atoms
+  static constexpr int kRed = kQ + kQBytes;                   // float [8 warps][2]
   static constexpr int kBar = kRed + 64;
-  // full[S], empty[S], e_ready[2], da_full[2], da_free[2], a_full, a_free, drain
-  // (the three per-tile hand-offs that run a tile ahead alternate between
-  // two barriers by tile parity, so neither side can be two phases ahead)
-  static constexpr int kNumBars = 2 * kLlaStages + 9;
+  // full[S], empty[S], e_ready[2], da_full[2], da_free[2], a_full, a_free,
+  // drain, s_full[2] (the per-tile hand-offs that run a tile ahead alternate
+  // between two barriers by tile parity, so neither side can be two phases
+  // ahead)
+  static constexpr int kNumBars = 2 * kLlaStages + 11;
   static constexpr int kMisc = kBar + kNumBars * 8;           // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
@@ -100,9 +104,30 @@ struct LlaLayout {
 // TMEM columns: D_KK [0, 128), D_KV [128, 256); A: hi words at 256, lo
 // words at 288 (keys 2c, 2c+1 in word c); the gather G = K^T diag(e) of
 // tile j at 320 + 64 (j % 2); sum e k at column 448, sum e v at 464 (the
-// first of 16 columns each).
+// first of 16 columns each); the scores of tile j at 480 + 8 (j % 2) (M = 64:
+// key r in lane (r % 16) + 32 (r / 16), column 0).
 constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128, kLlaColA = 256, kLlaColKs = 448, kLlaColVs = 464;
 __device__ __forceinline__ uint32_t lla_col_g(int buf) { return 320u + 64u * buf; }
+__device__ __forceinline__ uint32_t lla_col_s(int buf) { return 480u + 8u * buf; }
+
+// One 32-bit column of this thread's TMEM lane.
+__device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return r;
+}
+
+// Named barrier over nthreads threads; true in all of them if v is true in any.
+__device__ __forceinline__ bool bar_or(uint32_t id, uint32_t nthreads, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\tsetp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.or.pred po, %2, %3, pi;\n\tselp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
 
 __device__ __forceinline__ float4 lds_f4(uint32_t addr) {
   float4 v;
@@ -148,9 +173,9 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   uint64_t* a_full = da_free + 2;
   uint64_t* a_free = a_full + 1;
   uint64_t* drain = a_free + 1;
+  uint64_t* s_full = drain + 1;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::kMisc + 4);
-  float* q_s = reinterpret_cast<float*>(sm + Ly::kQ);
   float* red_s = reinterpret_cast<float*>(sm + Ly::kRed);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -200,11 +225,21 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     mbar_init(a_full, kLlaCompute);
     mbar_init(a_free, 1);
     mbar_init(drain, 1);
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (threadIdx.x < kLlaD)
-    q_s[threadIdx.x] = __bfloat162float(a.q[(size_t)bh * kLlaD + threadIdx.x]) * a.scale_log2;
+  if (threadIdx.x < Ly::kQBytes / 16) {
+    // 16-byte chunk i of the q operand: atom i / 64 (components 64 (i / 64) ..),
+    // row (i / 8) % 8, chunk i % 8; row 0 is not swizzled and holds q
+    const int i = threadIdx.x;
+    alignas(16) __nv_bfloat16 v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      v[e] = ((i >> 3) & 7) == 0 ? a.q[(size_t)bh * kLlaD + (i >> 6) * 64 + (i & 7) * 8 + e] : __float2bfloat16_rn(0.f);
+    *reinterpret_cast<uint4*>(sm + Ly::kQ + i * 16) = *reinterpret_cast<const uint4*>(v);
+  }
   // diag(e) and [e; 0] start as zeros; only their e entries change per tile
   for (int i = threadIdx.x; i < 2 * (Ly::kDiagBytes + Ly::kEcolBytes) / 16; i += kLlaThreads)
     reinterpret_cast<uint4*>(sm + Ly::kDiag)[i] = make_uint4(0u, 0u, 0u, 0u);
@@ -252,14 +287,18 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per tile: the gather G = K^T diag(e) (128 x 64, A = the K tile read as
+    // Per tile: the scores S = K q (M = 64 keys, N = 8, K-major A and B), the
+    // gather G = K^T diag(e) (128 x 64, A = the K tile read as
     // MN-major, B = diag(e)), the first moments sum e k += K^T [e 0..] and
     // sum e v += V^T [e 0..] (128 x 16); once the compute warps have packed
     // G into A = (e o K)^T: D_KK += A . K and D_KV += A . V (TS, K and V as
     // MN-major B operands).
+    constexpr uint32_t kIdS = idesc_bf16_ab(kTile, 8, false, false);
     constexpr uint32_t kIdG = idesc_bf16_ab(128, kTile, true, false);
     constexpr uint32_t kIdM = idesc_bf16_ab(128, 16, true, false);
     constexpr uint32_t kId = idesc_bf16(128, kLlaD, true);
+    const uint64_t dkS = smem_desc_sw128(smem_u32(sm + Ly::kK), 16, 1024);                  // K, K-major A
+    const uint64_t dqS = smem_desc_sw128(smem_u32(sm + Ly::kQ), 16, 1024);                  // q, K-major B
     const uint64_t dkA = smem_desc_sw128(smem_u32(sm + Ly::kK), Ly::kTileBytes / 2, 1024);   // K^T, MN-major A
     const uint64_t dvA = smem_desc_sw128(smem_u32(sm + Ly::kV), Ly::kTileBytes / 2, 1024);   // V^T, MN-major A
     const uint64_t dd = smem_desc_sw128(smem_u32(sm + Ly::kDiag), 16, 1024);                // diag(e), K-major B
@@ -268,8 +307,9 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
     // main(j) = D_KK += A . K(j), D_KV += A . V(j); A holds tile j's packed
-    // gather.  Issue order G(0), G(1), main(0), G(2), main(1), ...: the
-    // gather of the next tile runs while the compute warps pack this one.
+    // gather.  Issue order S(0), S(1), then per tile j: G(j), main(j - 1),
+    // S(j + 2): the gather of the next tile runs while the compute warps
+    // pack this one, and the scores are two tiles ahead.
     auto issue_main = [&](int jm) {
       const int sm_ = jm % S;
       const uint64_t kb = dkA + (uint64_t)((sm_ * Ly::kTileBytes) >> 4);   // the tiles as MN-major B
@@ -295,15 +335,30 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       tc_commit(a_free);
       tc_commit(&empty[sm_]);
     };
-    bool ok = true;
-    for (int j = 0; j <= n; ++j) {
+    // S(js) once tile js has landed (buffer js % 2: the scores of tile js - 2
+    // have been read, which e_ready(js - 2) reported before G(js - 2)).
+    auto issue_s = [&](int js) -> bool {
+      const int s = js % S;
+      if (!wait_warp(&full[s], (js / S) & 1)) return false;
+      tc_fence_after();
+      const uint64_t ka = dkS + (uint64_t)((s * Ly::kTileBytes) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < kLlaD / 16; ++kk) {   // 16 components per step: box kk / 4, 32 bytes into the row
+        const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTileBytes / 2 / 16) + (kk & 3) * 2);
+        const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kQBytes / 2 / 16) + (kk & 3) * 2);
+        tc_mma_ss(tmem + lla_col_s(js & 1), ka + oa, dqS + ob, kIdS, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(&s_full[js & 1]);
+      return true;
+    };
+    bool ok = issue_s(0) && (n < 2 || issue_s(1));
+    for (int j = 0; ok && j <= n; ++j) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) {
         ok = false;
         break;
       }
-      if (j < n) {   // G(j) and the first moments of tile j
+      if (j < n) {   // G(j) and the first moments of tile j (tile j has landed: S(j) waited for it)
         const int s = j % S, gb = j & 1;
-        if (!(ok = wait_warp(&full[s], (j / S) & 1))) break;
         if (!(ok = wait_warp(&e_ready[gb], (j >> 1) & 1))) break;
         if (j >= 2 && !(ok = wait_warp(&da_free[gb], ((j >> 1) - 1) & 1))) break;   // G buffer gb was read
         tc_fence_after();
@@ -326,6 +381,7 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         tc_fence_after();
         issue_main(j - 1);
       }
+      if (j + 2 < n && !(ok = issue_s(j + 2))) break;
     }
     if (!ok && lane == 0) *abort_flag = 1;
     // Every issued MMA must complete before tensor memory is released.
@@ -344,82 +400,72 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     const int wq = warp & 3;                   // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;            // TMEM lane = component a of k
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    const int ki = c >> 2, hf = c & 3;         // score phase: key, quarter of the head dim
+    // Score phase: warps with cw < 4 read the scores of keys 16 wq .. 16 wq + 15
+    // (TMEM lanes 32 wq .. 32 wq + 15 of the M = 64 product), one per lane.
+    const bool skey = cw < 4 && lane < 16;
+    const int key = 16 * wq + lane;
     float m_ref = -INFINITY, l_acc = 0.f;
     // Tile t's scores, weights, diag(e) and [e 0 ..] (buffers t % 2), then
-    // e_ready.  A new running max rescales sum e k, sum e v (after G(t - 1),
-    // before G(t)) at once, and returns the factor that D_KK, D_KV take
-    // after main(t - 1) and before main(t).
+    // e_ready.  The running max moves only when a score passes it by
+    // kLlaRescaleLog2 (one barrier reduction per tile decides; the first
+    // tile always takes its max).  A new running max rescales sum e k,
+    // sum e v (after G(t - 1), before G(t)) at once, and returns the factor
+    // that D_KK, D_KV take after main(t - 1) and before main(t).
     auto scores_phase = [&](int t, float& alpha_d) -> bool {
       const int s = t % S, gb = t & 1;
-      const bool w = !*abort_flag && mbar_wait_bounded(a.wait_ns, &full[s], (t / S) & 1);
-      if (!bar_and(1, kLlaCompute, w)) return false;
+      const bool w = __all_sync(0xffffffffu, !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[gb], (t >> 1) & 1));
       uint8_t* kt = sm + Ly::kK + s * Ly::kTileBytes;
       uint8_t* vt = sm + Ly::kV + s * Ly::kTileBytes;
       const int nvalid = min(kTile, len - (t0 + t) * kTile);
-      // ---- scaled score of key ki: quarter hf of q . k (four partial sums)
-      float dot;
-      {
-        float d4[4] = {0.f, 0.f, 0.f, 0.f};
-        const uint8_t* krow = kt + (hf >> 1) * (Ly::kTileBytes / 2) + ki * 128;
-        const uint32_t qh = smem_u32(q_s + 32 * hf);
-#pragma unroll
-        for (int cq = 0; cq < 4; ++cq) {
-          const int ch = 4 * (hf & 1) + cq;
-          const uint4 v4 = *reinterpret_cast<const uint4*>(krow + ((ch ^ (ki & 7)) << 4));
-          const uint32_t w4[4] = {v4.x, v4.y, v4.z, v4.w};
-          const float4 qa = lds_f4(qh + 32 * cq), qb = lds_f4(qh + 32 * cq + 16);
-          const float qv[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            d4[e] = fmaf(qv[2 * e], bf16_lo_f(w4[e]), d4[e]);
-            d4[e] = fmaf(qv[2 * e + 1], bf16_hi_f(w4[e]), d4[e]);
-          }
-        }
-        dot = (d4[0] + d4[1]) + (d4[2] + d4[3]);
-      }
-      dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-      dot += __shfl_xor_sync(0xffffffffu, dot, 2);
-      const float sc = ki < nvalid ? dot : -INFINITY;
-      const float wmax = warp_max(sc);
-      if (lane == 0) red_s[cw] = wmax;
-      bar_and(2, kLlaCompute, true);
-      const float tmax = fmaxf(fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3])),
-                               fmaxf(fmaxf(red_s[4], red_s[5]), fmaxf(red_s[6], red_s[7])));
-      alpha_d = 1.f;
-      if (t == 0) {
-        m_ref = tmax;   // the piece's first tile holds a key: tmax is finite
-      } else if (tmax > m_ref + kLlaRescaleLog2) {   // uniform: every compute thread saw the same maxima
-        const float alpha = ex2(m_ref - tmax);
-        m_ref = tmax;
-        alpha_d = alpha;
-        // sum e k, sum e v hold tiles < t once G(t - 1) is done
-        const bool wd = mbar_wait_bounded(a.wait_ns, &da_full[(t - 1) & 1], ((t - 1) >> 1) & 1);
-        if (!bar_and(3, kLlaCompute, wd)) return false;
+      float sc = -INFINITY;
+      if (w && cw < 4) {   // warp-uniform
         tc_fence_after();
-        uint32_t r[16];   // column 0 of sum e k (kh 0) or sum e v (kh 1); the other 15 are zero
-        const uint32_t addr = tmem + lane_off + (kh ? kLlaColVs : kLlaColKs);
-        tmem_ld16(addr, r);
+        const uint32_t r = tmem_ld1(tmem + lane_off + lla_col_s(gb));
         tmem_wait_ld();
-        r[0] = __float_as_uint(__uint_as_float(r[0]) * alpha);
-        tmem_st16(addr, r);
-        tmem_wait_st();
-        tc_fence_before();
-        l_acc *= alpha;
+        if (skey && key < nvalid) sc = __uint_as_float(r) * a.scale_log2;
+      }
+      alpha_d = 1.f;
+      if (bar_or(1, kLlaCompute, t == 0 || !w || sc > m_ref + kLlaRescaleLog2)) {   // uniform
+        if (!bar_and(2, kLlaCompute, w)) return false;
+        const float wmax = warp_max(sc);
+        if (lane == 0) red_s[cw] = wmax;
+        bar_and(3, kLlaCompute, true);
+        const float tmax = fmaxf(fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3])),
+                                 fmaxf(fmaxf(red_s[4], red_s[5]), fmaxf(red_s[6], red_s[7])));
+        if (t == 0) {
+          m_ref = tmax;   // the piece's first tile holds a key: tmax is finite
+        } else if (tmax > m_ref + kLlaRescaleLog2) {   // uniform: every compute thread saw the same maxima
+          const float alpha = ex2(m_ref - tmax);
+          m_ref = tmax;
+          alpha_d = alpha;
+          // sum e k, sum e v hold tiles < t once G(t - 1) is done
+          const bool wd = mbar_wait_bounded(a.wait_ns, &da_full[(t - 1) & 1], ((t - 1) >> 1) & 1);
+          if (!bar_and(2, kLlaCompute, wd)) return false;
+          tc_fence_after();
+          uint32_t r[16];   // column 0 of sum e k (kh 0) or sum e v (kh 1); the other 15 are zero
+          const uint32_t addr = tmem + lane_off + (kh ? kLlaColVs : kLlaColKs);
+          tmem_ld16(addr, r);
+          tmem_wait_ld();
+          r[0] = __float_as_uint(__uint_as_float(r[0]) * alpha);
+          tmem_st16(addr, r);
+          tmem_wait_st();
+          tc_fence_before();
+          l_acc *= alpha;
+        }
       }
       // ---- the weights, rounded to bf16: every product below uses these values
-      const float e = ki < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f;
-      if (hf == 0) {
+      if (skey) {   // every key of the tile, its weight 0 past the end
+        const float e = key < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f;
         l_acc += e;
         __nv_bfloat16* diag_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kDiag + gb * Ly::kDiagBytes);
         __nv_bfloat16* ecol_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kEcol + gb * Ly::kEcolBytes);
-        diag_s[sw128_off(ki, ki) >> 1] = __float2bfloat16_rn(e);
-        ecol_s[ki] = __float2bfloat16_rn(e);   // row 0 of [e 0..]: unswizzled
+        diag_s[sw128_off(key, key) >> 1] = __float2bfloat16_rn(e);
+        ecol_s[key] = __float2bfloat16_rn(e);   // row 0 of [e 0..]: unswizzled
       }
       if (nvalid < kTile) {
         // Rows past the end are operands of the gather and the products
         // (their weights are 0, but 0 * NaN is not): zero them in K and V.
-        // Every score read of this tile has happened (the barrier above).
+        // S(t), the only earlier reader of the tile, is done (s_full).
         for (int i = c; i < (kTile - nvalid) * 16; i += kLlaCompute) {
           const int r = nvalid + (i >> 4), cc = i & 15;   // cc: box (cc >> 3), chunk (cc & 7)
           const int off = (cc >> 3) * (Ly::kTileBytes / 2) + r * 128 + (cc & 7) * 16;
