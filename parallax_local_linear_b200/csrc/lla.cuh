@@ -20,19 +20,22 @@
 //     a running max m (2^(s - m) weights, rescaled lazily as in the prefill),
 //         l = sum e,  ks = sum e k,  vs = sum e v,
 //         D_KK = sum e k k^T,  D_KV = sum e k v^T          (128 x 128 each)
-//     All of the arithmetic over keys runs on the tensor cores: per 64-key
-//     tile the scores S = K q (M = 64 keys, N = 8: q is row 0 of an 8-row
-//     operand), read back by four warps, 16 keys each; the weights e
-//     (rounded to bf16 once, so that every sum uses the same values) go into
-//     diag(e) and the column [e 0 ..] in shared memory; the MMAs
-//     G = K^T diag(e) (so row a of G holds e_i k_ia, exact in fp32),
-//     ks += K^T [e 0 ..] and vs += V^T [e 0 ..] read the K and V tiles as
-//     MN-major A operands; the compute warps pack G into A = (e o K)^T in
-//     tensor memory (bf16 pairs); then D_KK += A . K and D_KV += A . V (K, V
-//     as MN-major B operands).  For sequences shorter than kLlaSplitLen the
-//     bf16 rounding of e o K is not averaged away (the solve amplifies it
-//     along directions the few keys do not span), so a second product adds
-//     its lo part (x = hi + lo).  The piece's record goes to the workspace.
+//     The products over keys run on the tensor cores: per 64-key tile the
+//     scores S = K q (M = 64 keys, N = 8: q is row 0 of an 8-row operand),
+//     read back by four warps, 16 keys each; the weights e (rounded to bf16
+//     once, so that every sum uses the same values) go into diag(e) in
+//     shared memory; the MMA G = K^T diag(e) (the K tile read as an MN-major
+//     A operand) puts e_i k_ia, exact in fp32, in row a of G; the compute
+//     warps pack G into A = (e o K)^T in tensor memory (bf16 pairs) and sum
+//     its rows into ks; then [D_KK | D_KV] += A . [K | V] (N = 256: a
+//     stage's K and V tiles are one MN-major B operand).  The issuing warp
+//     spends ~40 cycles per MMA, so the count matters more than the size:
+//     sixteen per tile.  vs is summed on the CUDA cores from the V tile
+//     while the compute warps wait for the gather.  For sequences shorter
+//     than kLlaSplitLen the bf16 rounding of e o K is not averaged away (the
+//     solve amplifies it along directions the few keys do not span), so a
+//     second product adds its lo part (x = hi + lo).  The piece's record
+//     goes to the workspace.
 //
 //   lla_solve_kernel  one CTA per (sequence, query head): merges the pieces
 //     like online softmax (weights 2^(m_j - M)), forms S_KK + ridge I and
@@ -82,15 +85,16 @@ struct LlaArgs {
 
 struct LlaLayout {
   static constexpr int kTileBytes = kTile * kLlaD * 2;   // 16 KB: two 64-column boxes of 64 rows
-  static constexpr int kK = 0;
-  static constexpr int kV = kK + kLlaStages * kTileBytes;
+  // Stage s: the K tile, then the V tile, so that the four 64-column boxes
+  // [K lo | K hi | V lo | V hi] are one MN-major operand of 256 columns.
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kKV = 0;
   static constexpr int kDiagBytes = kTile * kTile * 2;        // bf16 [64][64]: diag(e), 128-byte swizzle
-  static constexpr int kEcolBytes = 16 * kTile * 2;           // bf16 [16][64]: row 0 = e, rows 1.. zero
-  static constexpr int kDiag = kV + kLlaStages * kTileBytes;  // two buffers (tile parity)
-  static constexpr int kEcol = kDiag + 2 * kDiagBytes;        // two buffers
+  static constexpr int kDiag = kKV + kLlaStages * kStageBytes;   // two buffers (tile parity)
   static constexpr int kQBytes = 8 * kLlaD * 2;               // bf16 [8][128]: row 0 = q, rows 1.. zero
-  static constexpr int kQ = kEcol + 2 * kEcolBytes;           // K-major B operand, two 64-column atoms
-  static constexpr int kRed = kQ + kQBytes;                   // float [8 warps][2]
+  static constexpr int kQ = kDiag + 2 * kDiagBytes;           // K-major B operand, two 64-column atoms
+  static constexpr int kE = kQ + kQBytes;                     // float [2][64]: the tile's weights e
+  static constexpr int kRed = kE + 2 * kTile * 4;             // float [8 warps][2]
   static constexpr int kBar = kRed + 64;
   // full[S], empty[S], e_ready[2], da_full[2], da_free[2], a_full, a_free,
   // drain, s_full[2] (the per-tile hand-offs that run a tile ahead alternate
@@ -101,14 +105,43 @@ struct LlaLayout {
   static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
 
-// TMEM columns: D_KK [0, 128), D_KV [128, 256); A: hi words at 256, lo
-// words at 288 (keys 2c, 2c+1 in word c); the gather G = K^T diag(e) of
-// tile j at 320 + 64 (j % 2); sum e k at column 448, sum e v at 464 (the
-// first of 16 columns each); the scores of tile j at 480 + 8 (j % 2) (M = 64:
-// key r in lane (r % 16) + 32 (r / 16), column 0).
-constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128, kLlaColA = 256, kLlaColKs = 448, kLlaColVs = 464;
+// TMEM columns: D = [D_KK | D_KV] in [0, 256); A: hi words at 256, lo words
+// at 288 (keys 2c, 2c+1 in word c); the gather G = K^T diag(e) of tile j at
+// 320 + 64 (j % 2); the scores of tile j at 480 + 8 (j % 2) (M = 64: key r
+// in lane (r % 16) + 32 (r / 16), column 0).
+constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128, kLlaColA = 256;
 __device__ __forceinline__ uint32_t lla_col_g(int buf) { return 320u + 64u * buf; }
 __device__ __forceinline__ uint32_t lla_col_s(int buf) { return 480u + 8u * buf; }
+
+// Four MMAs into one accumulator under one elect.sync (four k-steps): the
+// first takes the accumulate flag acc0, the others accumulate.
+__device__ __forceinline__ void lla_mma4_ss(uint32_t d, uint64_t a0, uint64_t b0, uint64_t a1, uint64_t b1,
+                                            uint64_t a2, uint64_t b2, uint64_t a3, uint64_t b3, uint32_t idesc,
+                                            uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1, e;\n\tsetp.ne.b32 p0, %10, 0;\n\tsetp.eq.b32 p1, %10, %10;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %9, p0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %9, p1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %9, p1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %9, p1;\n\t}" ::"r"(d),
+      "l"(a0), "l"(b0), "l"(a1), "l"(b1), "l"(a2), "l"(b2), "l"(a3), "l"(b3), "r"(idesc), "r"(acc0)
+      : "memory");
+}
+
+__device__ __forceinline__ void lla_mma4_ts(uint32_t d, uint32_t a0, uint64_t b0, uint32_t a1, uint64_t b1,
+                                            uint32_t a2, uint64_t b2, uint32_t a3, uint64_t b3, uint32_t idesc,
+                                            uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1, e;\n\tsetp.ne.b32 p0, %10, 0;\n\tsetp.eq.b32 p1, %10, %10;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %9, p0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %4, %9, p1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %9, p1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %9, p1;\n\t}" ::"r"(d),
+      "r"(a0), "l"(b0), "r"(a1), "l"(b1), "r"(a2), "l"(b2), "r"(a3), "l"(b3), "r"(idesc), "r"(acc0)
+      : "memory");
+}
 
 // One 32-bit column of this thread's TMEM lane.
 __device__ __forceinline__ uint32_t tmem_ld1(uint32_t taddr) {
@@ -221,12 +254,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       mbar_init(&e_ready[i], kLlaCompute);
       mbar_init(&da_full[i], 1);
       mbar_init(&da_free[i], kLlaCompute);
+      mbar_init(&s_full[i], 1);
     }
     mbar_init(a_full, kLlaCompute);
     mbar_init(a_free, 1);
     mbar_init(drain, 1);
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -240,8 +272,8 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       v[e] = ((i >> 3) & 7) == 0 ? a.q[(size_t)bh * kLlaD + (i >> 6) * 64 + (i & 7) * 8 + e] : __float2bfloat16_rn(0.f);
     *reinterpret_cast<uint4*>(sm + Ly::kQ + i * 16) = *reinterpret_cast<const uint4*>(v);
   }
-  // diag(e) and [e; 0] start as zeros; only their e entries change per tile
-  for (int i = threadIdx.x; i < 2 * (Ly::kDiagBytes + Ly::kEcolBytes) / 16; i += kLlaThreads)
+  // diag(e) starts as zeros; only its diagonal changes per tile
+  for (int i = threadIdx.x; i < 2 * Ly::kDiagBytes / 16; i += kLlaThreads)
     reinterpret_cast<uint4*>(sm + Ly::kDiag)[i] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
   if (warp == 1) {
@@ -270,12 +302,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         const int tile = t0 + j;
         const int row = a.paged ? (__ldg(pt + tile) * a.Hkv + kvh) * kTile   // page ids checked above
                                 : (b * a.Hkv + kvh) * a.kv_len + tile * kTile;
-        mbar_arrive_expect_tx(&full[s], 2 * Ly::kTileBytes);
+        uint8_t* st = sm + Ly::kKV + s * Ly::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], Ly::kStageBytes);
         for (int bx = 0; bx < 2; ++bx) {
-          tma_load_2d(sm + Ly::kK + s * Ly::kTileBytes + bx * (Ly::kTileBytes / 2), &tm_k, bx * 64, row,
-                      &full[s], pol);
-          tma_load_2d(sm + Ly::kV + s * Ly::kTileBytes + bx * (Ly::kTileBytes / 2), &tm_v, bx * 64, row,
-                      &full[s], pol);
+          tma_load_2d(st + bx * (Ly::kTileBytes / 2), &tm_k, bx * 64, row, &full[s], pol);
+          tma_load_2d(st + Ly::kTileBytes + bx * (Ly::kTileBytes / 2), &tm_v, bx * 64, row, &full[s], pol);
         }
         ++issued;
       }
@@ -287,67 +318,53 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per tile: the scores S = K q (M = 64 keys, N = 8, K-major A and B), the
-    // gather G = K^T diag(e) (128 x 64, A = the K tile read as
-    // MN-major, B = diag(e)), the first moments sum e k += K^T [e 0..] and
-    // sum e v += V^T [e 0..] (128 x 16); once the compute warps have packed
-    // G into A = (e o K)^T: D_KK += A . K and D_KV += A . V (TS, K and V as
-    // MN-major B operands).
+    // Per tile: the scores S = K q (M = 64 keys, N = 8, K-major A and B); the
+    // gather G = K^T diag(e) (128 x 64, A = the K tile read as MN-major,
+    // B = diag(e)); once the compute warps have packed G into
+    // A = (e o K)^T: [D_KK | D_KV] += A . [K | V] (TS, 128 x 256, the stage's
+    // K and V tiles as one MN-major B operand).  Sixteen MMAs per tile (24
+    // below kLlaSplitLen keys), four under each elect.
     constexpr uint32_t kIdS = idesc_bf16_ab(kTile, 8, false, false);
     constexpr uint32_t kIdG = idesc_bf16_ab(128, kTile, true, false);
-    constexpr uint32_t kIdM = idesc_bf16_ab(128, 16, true, false);
-    constexpr uint32_t kId = idesc_bf16(128, kLlaD, true);
-    const uint64_t dkS = smem_desc_sw128(smem_u32(sm + Ly::kK), 16, 1024);                  // K, K-major A
-    const uint64_t dqS = smem_desc_sw128(smem_u32(sm + Ly::kQ), 16, 1024);                  // q, K-major B
-    const uint64_t dkA = smem_desc_sw128(smem_u32(sm + Ly::kK), Ly::kTileBytes / 2, 1024);   // K^T, MN-major A
-    const uint64_t dvA = smem_desc_sw128(smem_u32(sm + Ly::kV), Ly::kTileBytes / 2, 1024);   // V^T, MN-major A
-    const uint64_t dd = smem_desc_sw128(smem_u32(sm + Ly::kDiag), 16, 1024);                // diag(e), K-major B
-    const uint64_t de = smem_desc_sw128(smem_u32(sm + Ly::kEcol), 16, 1024);                // [e 0..], K-major B
+    constexpr uint32_t kIdD = idesc_bf16(128, 2 * kLlaD, true);
+    const uint64_t dkS = smem_desc_sw128(smem_u32(sm + Ly::kKV), 16, 1024);                  // K, K-major A
+    const uint64_t dqS = smem_desc_sw128(smem_u32(sm + Ly::kQ), 16, 1024);                   // q, K-major B
+    const uint64_t dkvM = smem_desc_sw128(smem_u32(sm + Ly::kKV), Ly::kTileBytes / 2, 1024);   // MN-major, 64-col atoms
+    const uint64_t dd = smem_desc_sw128(smem_u32(sm + Ly::kDiag), 16, 1024);                 // diag(e), K-major B
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
-    // main(j) = D_KK += A . K(j), D_KV += A . V(j); A holds tile j's packed
-    // gather.  Issue order S(0), S(1), then per tile j: G(j), main(j - 1),
-    // S(j + 2): the gather of the next tile runs while the compute warps
-    // pack this one, and the scores are two tiles ahead.
+    auto stage_off = [&](int j) { return (uint64_t)(((j % S) * Ly::kStageBytes) >> 4); };
+    // main(j) = [D_KK | D_KV] += A . [K(j) | V(j)]; A holds tile j's packed
+    // gather (16 keys = 8 A words and 16 B rows, 2048 bytes, per step).
+    // Issue order S(0), S(1), then per tile j: G(j), main(j - 1), S(j + 2):
+    // the gather of the next tile runs while the compute warps pack this
+    // one, and the scores are two tiles ahead.
     auto issue_main = [&](int jm) {
-      const int sm_ = jm % S;
-      const uint64_t kb = dkA + (uint64_t)((sm_ * Ly::kTileBytes) >> 4);   // the tiles as MN-major B
-      const uint64_t vb = dvA + (uint64_t)((sm_ * Ly::kTileBytes) >> 4);
+      const uint64_t kv = dkvM + stage_off(jm);
       const uint32_t ahi = tmem + kLlaColA;
-#pragma unroll
-      for (int kk = 0; kk < 4; kk += 2) {   // 16 keys per step: 8 A words, 16 B rows (2048 bytes)
-        const uint64_t o0 = (uint64_t)(kk * 128), o1 = o0 + 128;
-        tc_mma_ts4(tmem + kLlaColKK, ahi + 8u * kk, kb + o0, tmem + kLlaColKV, ahi + 8u * kk, vb + o0,
-                   tmem + kLlaColKK, ahi + 8u * (kk + 1), kb + o1, tmem + kLlaColKV, ahi + 8u * (kk + 1), vb + o1,
-                   kId, (jm > 0 || kk > 0) ? 1u : 0u, 1u);
-      }
+      lla_mma4_ts(tmem + kLlaColKK, ahi, kv, ahi + 8u, kv + 128, ahi + 16u, kv + 256, ahi + 24u, kv + 384, kIdD,
+                  jm > 0 ? 1u : 0u);
       if (split_lo) {
-#pragma unroll
-        for (int kk = 0; kk < 4; kk += 2) {
-          const uint64_t o0 = (uint64_t)(kk * 128), o1 = o0 + 128;
-          const uint32_t alo = ahi + 32u;
-          tc_mma_ts4(tmem + kLlaColKK, alo + 8u * kk, kb + o0, tmem + kLlaColKV, alo + 8u * kk, vb + o0,
-                     tmem + kLlaColKK, alo + 8u * (kk + 1), kb + o1, tmem + kLlaColKV, alo + 8u * (kk + 1),
-                     vb + o1, kId, 1u, 1u);
-        }
+        const uint32_t alo = ahi + 32u;
+        lla_mma4_ts(tmem + kLlaColKK, alo, kv, alo + 8u, kv + 128, alo + 16u, kv + 256, alo + 24u, kv + 384, kIdD,
+                    1u);
       }
       tc_commit(a_free);
-      tc_commit(&empty[sm_]);
+      tc_commit(&empty[jm % S]);
     };
     // S(js) once tile js has landed (buffer js % 2: the scores of tile js - 2
     // have been read, which e_ready(js - 2) reported before G(js - 2)).
+    // 16 components per step: box kk / 4, 32 bytes into the 128-byte row.
     auto issue_s = [&](int js) -> bool {
-      const int s = js % S;
-      if (!wait_warp(&full[s], (js / S) & 1)) return false;
+      if (!wait_warp(&full[js % S], (js / S) & 1)) return false;
       tc_fence_after();
-      const uint64_t ka = dkS + (uint64_t)((s * Ly::kTileBytes) >> 4);
-#pragma unroll
-      for (int kk = 0; kk < kLlaD / 16; ++kk) {   // 16 components per step: box kk / 4, 32 bytes into the row
-        const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTileBytes / 2 / 16) + (kk & 3) * 2);
-        const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kQBytes / 2 / 16) + (kk & 3) * 2);
-        tc_mma_ss(tmem + lla_col_s(js & 1), ka + oa, dqS + ob, kIdS, kk > 0 ? 1u : 0u);
-      }
+      const uint64_t ka = dkS + stage_off(js);
+      constexpr uint64_t kBoxA = Ly::kTileBytes / 2 / 16, kBoxB = Ly::kQBytes / 2 / 16;
+      const uint32_t d = tmem + lla_col_s(js & 1);
+      lla_mma4_ss(d, ka, dqS, ka + 2, dqS + 2, ka + 4, dqS + 4, ka + 6, dqS + 6, kIdS, 0u);
+      lla_mma4_ss(d, ka + kBoxA, dqS + kBoxB, ka + kBoxA + 2, dqS + kBoxB + 2, ka + kBoxA + 4, dqS + kBoxB + 4,
+                  ka + kBoxA + 6, dqS + kBoxB + 6, kIdS, 1u);
       tc_commit(&s_full[js & 1]);
       return true;
     };
@@ -357,23 +374,15 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         ok = false;
         break;
       }
-      if (j < n) {   // G(j) and the first moments of tile j (tile j has landed: S(j) waited for it)
-        const int s = j % S, gb = j & 1;
+      if (j < n) {   // G(j) (tile j has landed: S(j) waited for it)
+        const int gb = j & 1;
         if (!(ok = wait_warp(&e_ready[gb], (j >> 1) & 1))) break;
         if (j >= 2 && !(ok = wait_warp(&da_free[gb], ((j >> 1) - 1) & 1))) break;   // G buffer gb was read
         tc_fence_after();
-        const uint64_t ks = dkA + (uint64_t)((s * Ly::kTileBytes) >> 4);
-        const uint64_t vs = dvA + (uint64_t)((s * Ly::kTileBytes) >> 4);
+        // 16 keys per step: 16 rows (2048 bytes) of the K tile, 32 bytes of diag(e)
+        const uint64_t ks = dkvM + stage_off(j);
         const uint64_t ddb = dd + (uint64_t)((gb * Ly::kDiagBytes) >> 4);
-        const uint64_t deb = de + (uint64_t)((gb * Ly::kEcolBytes) >> 4);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {   // 16 keys per step: 16 rows (2048 bytes) of K, V; 32 bytes of diag, e
-          const uint64_t o0 = (uint64_t)(kk * 128), b0 = (uint64_t)(kk * 2);
-          const uint32_t acc = (j > 0 || kk > 0) ? 1u : 0u;   // the first moments accumulate over tiles
-          tc_mma_ss(tmem + lla_col_g(gb), ks + o0, ddb + b0, kIdG, kk > 0 ? 1u : 0u);
-          tc_mma_ss(tmem + kLlaColKs, ks + o0, deb + b0, kIdM, acc);
-          tc_mma_ss(tmem + kLlaColVs, vs + o0, deb + b0, kIdM, acc);
-        }
+        lla_mma4_ss(tmem + lla_col_g(gb), ks, ddb, ks + 128, ddb + 2, ks + 256, ddb + 4, ks + 384, ddb + 6, kIdG, 0u);
         tc_commit(&da_full[gb]);
       }
       if (j >= 1) {   // main(j - 1), once the compute warps have packed tile j - 1
@@ -404,18 +413,21 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     // (TMEM lanes 32 wq .. 32 wq + 15 of the M = 64 product), one per lane.
     const bool skey = cw < 4 && lane < 16;
     const int key = 16 * wq + lane;
+    // sum e v: thread c takes components 2 (c % 64), + 1 and keys 16 (c / 64) ..
+    // of each tile (a warp reads whole 128-byte rows of one V box).
+    const int vcp = c & 63, vkq = c >> 6, vchunk = (vcp & 31) >> 2;
+    const int voff = Ly::kTileBytes + (vcp >> 5) * (Ly::kTileBytes / 2) + (vcp & 3) * 4;   // + row, swizzled chunk
     float m_ref = -INFINITY, l_acc = 0.f;
-    // Tile t's scores, weights, diag(e) and [e 0 ..] (buffers t % 2), then
-    // e_ready.  The running max moves only when a score passes it by
-    // kLlaRescaleLog2 (one barrier reduction per tile decides; the first
-    // tile always takes its max).  A new running max rescales sum e k,
-    // sum e v (after G(t - 1), before G(t)) at once, and returns the factor
-    // that D_KK, D_KV take after main(t - 1) and before main(t).
+    float ks_acc = 0.f;                        // sum e k_row over this thread's key half
+    float vs0 = 0.f, vs1 = 0.f;                // sum e v over this thread's key quarter
+    // Tile t's scores, weights, diag(e) and e (buffers t % 2), then e_ready.
+    // The running max moves only when a score passes it by kLlaRescaleLog2
+    // (one barrier reduction per tile decides; the first tile always takes
+    // its max).  A new running max returns the factor that everything
+    // accumulated over tiles < t takes before tile t is added.
     auto scores_phase = [&](int t, float& alpha_d) -> bool {
-      const int s = t % S, gb = t & 1;
+      const int gb = t & 1;
       const bool w = __all_sync(0xffffffffu, !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[gb], (t >> 1) & 1));
-      uint8_t* kt = sm + Ly::kK + s * Ly::kTileBytes;
-      uint8_t* vt = sm + Ly::kV + s * Ly::kTileBytes;
       const int nvalid = min(kTile, len - (t0 + t) * kTile);
       float sc = -INFINITY;
       if (w && cw < 4) {   // warp-uniform
@@ -435,22 +447,9 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         if (t == 0) {
           m_ref = tmax;   // the piece's first tile holds a key: tmax is finite
         } else if (tmax > m_ref + kLlaRescaleLog2) {   // uniform: every compute thread saw the same maxima
-          const float alpha = ex2(m_ref - tmax);
+          alpha_d = ex2(m_ref - tmax);
           m_ref = tmax;
-          alpha_d = alpha;
-          // sum e k, sum e v hold tiles < t once G(t - 1) is done
-          const bool wd = mbar_wait_bounded(a.wait_ns, &da_full[(t - 1) & 1], ((t - 1) >> 1) & 1);
-          if (!bar_and(2, kLlaCompute, wd)) return false;
-          tc_fence_after();
-          uint32_t r[16];   // column 0 of sum e k (kh 0) or sum e v (kh 1); the other 15 are zero
-          const uint32_t addr = tmem + lane_off + (kh ? kLlaColVs : kLlaColKs);
-          tmem_ld16(addr, r);
-          tmem_wait_ld();
-          r[0] = __float_as_uint(__uint_as_float(r[0]) * alpha);
-          tmem_st16(addr, r);
-          tmem_wait_st();
-          tc_fence_before();
-          l_acc *= alpha;
+          l_acc *= alpha_d;
         }
       }
       // ---- the weights, rounded to bf16: every product below uses these values
@@ -458,29 +457,57 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         const float e = key < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f;
         l_acc += e;
         __nv_bfloat16* diag_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kDiag + gb * Ly::kDiagBytes);
-        __nv_bfloat16* ecol_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kEcol + gb * Ly::kEcolBytes);
         diag_s[sw128_off(key, key) >> 1] = __float2bfloat16_rn(e);
-        ecol_s[key] = __float2bfloat16_rn(e);   // row 0 of [e 0..]: unswizzled
+        reinterpret_cast<float*>(sm + Ly::kE)[gb * kTile + key] = e;
       }
       if (nvalid < kTile) {
         // Rows past the end are operands of the gather and the products
         // (their weights are 0, but 0 * NaN is not): zero them in K and V.
         // S(t), the only earlier reader of the tile, is done (s_full).
+        uint8_t* st = sm + Ly::kKV + (t % S) * Ly::kStageBytes;
         for (int i = c; i < (kTile - nvalid) * 16; i += kLlaCompute) {
           const int r = nvalid + (i >> 4), cc = i & 15;   // cc: box (cc >> 3), chunk (cc & 7)
           const int off = (cc >> 3) * (Ly::kTileBytes / 2) + r * 128 + (cc & 7) * 16;
-          *reinterpret_cast<uint4*>(kt + off) = make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(vt + off) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(st + off) = make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(st + Ly::kTileBytes + off) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
       fence_proxy_async_smem();
       mbar_arrive(&e_ready[gb]);
       return true;
     };
-    // Tile t's gather into A = (e o K)^T (after main(t - 1) has read A), and
-    // the deferred rescale of D_KK, D_KV.
+    // Tile t: sum e v over this thread's keys (while G(t) and main(t - 1) run;
+    // V(t) stays resident until main(t), after a_full(t), is done), then the
+    // gather into A = (e o K)^T (after main(t - 1) has read A), the deferred
+    // rescale of D, and sum e k from the gather's rows.
     auto pack_phase = [&](int t, float alpha_d) -> bool {
-      const bool wg = mbar_wait_bounded(a.wait_ns, &da_full[t & 1], (t >> 1) & 1);
+      const int gb = t & 1;
+      {
+        const float* et = reinterpret_cast<const float*>(sm + Ly::kE) + gb * kTile + 16 * vkq;
+        const uint8_t* vt = sm + Ly::kKV + (t % S) * Ly::kStageBytes + voff;
+        // Rows past the end hold zeros (scores(t) cleared them; a barrier
+        // since orders that before these reads) and weight 0.
+        uint32_t w2[16];
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj)   // row 16 vkq + jj, whose swizzle is jj % 8
+          w2[jj] = *reinterpret_cast<const uint32_t*>(vt + (16 * vkq + jj) * 128 + ((vchunk ^ (jj & 7)) << 4));
+        float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const float4 e4 = lds_f4(smem_u32(et + 4 * q4));
+          const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
+#pragma unroll
+          for (int u = 0; u < 4; u += 2) {
+            a0 = fmaf(ev[u], bf16_lo_f(w2[4 * q4 + u]), a0);
+            a1 = fmaf(ev[u], bf16_hi_f(w2[4 * q4 + u]), a1);
+            b0 = fmaf(ev[u + 1], bf16_lo_f(w2[4 * q4 + u + 1]), b0);
+            b1 = fmaf(ev[u + 1], bf16_hi_f(w2[4 * q4 + u + 1]), b1);
+          }
+        }
+        vs0 = fmaf(vs0, alpha_d, a0 + b0);
+        vs1 = fmaf(vs1, alpha_d, a1 + b1);
+      }
+      const bool wg = mbar_wait_bounded(a.wait_ns, &da_full[gb], (t >> 1) & 1);
       const bool wa = t == 0 || mbar_wait_bounded(a.wait_ns, a_free, (t - 1) & 1);
       if (!bar_and(2, kLlaCompute, wg && wa)) return false;
       tc_fence_after();
@@ -497,10 +524,10 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         }
       }
       uint32_t g[32];
-      tmem_ld32(tmem + lane_off + lla_col_g(t & 1) + 32u * kh, g);
+      tmem_ld32(tmem + lane_off + lla_col_g(gb) + 32u * kh, g);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&da_free[t & 1]);
+      mbar_arrive(&da_free[gb]);
       auto pack = [&](auto split_tag) {
         constexpr bool kSplit = decltype(split_tag)::value;
         uint32_t hi[16], lo[16];
@@ -520,16 +547,25 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(a_full);
+      // G holds e_i k_ia exactly (one nonzero product per entry)
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < 32; ++i) s4[i & 3] += __uint_as_float(g[i]);
+      ks_acc = fmaf(ks_acc, alpha_d, (s4[0] + s4[1]) + (s4[2] + s4[3]));
       return true;
     };
     // scores(t + 1) runs before pack(t), so the gather of tile t + 1 overlaps
     // the packing of tile t and main(t).
-    float alpha_pack = 1.f;   // D's rescale before main(t), decided by scores(t)
+    float alpha_pack = 1.f;   // the rescale before tile t is added, decided by scores(t)
     bool fine = scores_phase(0, alpha_pack);
     int j = 0;
     for (; fine && j < n; ++j) {
       float alpha_next = 1.f;
-      if (j + 1 < n && !(fine = scores_phase(j + 1, alpha_next))) break;
+      if (j + 1 < n) {
+        if (!(fine = scores_phase(j + 1, alpha_next))) break;
+      } else {
+        bar_and(1, kLlaCompute, true);   // the last tile's weights, visible to every compute thread
+      }
       if (!(fine = pack_phase(j, alpha_pack))) break;
       alpha_pack = alpha_next;
     }
@@ -538,6 +574,15 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     wl = bar_and(3, kLlaCompute, wl);
     const float lw = warp_sum(l_acc);
     if (lane == 0) red_s[8 + cw] = lw;
+    // the first moments' partial sums meet in the diag buffers, idle once
+    // the last products are done: [2][128] halves of sum e k, [4][128]
+    // quarters of sum e v
+    float* scr = reinterpret_cast<float*>(sm + Ly::kDiag);
+    if (wl) {
+      scr[kh * kLlaD + row] = ks_acc;
+      scr[2 * kLlaD + vkq * kLlaD + 2 * vcp] = vs0;
+      scr[2 * kLlaD + vkq * kLlaD + 2 * vcp + 1] = vs1;
+    }
     bar_and(2, kLlaCompute, true);
     if (wl) {
       tc_fence_after();
@@ -552,12 +597,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) dst[i * kLlaD] = __uint_as_float(r[i]);
       }
-      {
-        uint32_t r[16];
-        tmem_ld16(tmem + lane_off + (kh ? kLlaColVs : kLlaColKs), r);
-        tmem_wait_ld();
-        rec[(kh ? kLlaRecVs : kLlaRecKs) + row] = __uint_as_float(r[0]);
-      }
+      if (kh == 0)
+        rec[kLlaRecKs + row] = scr[row] + scr[kLlaD + row];
+      else
+        rec[kLlaRecVs + row] = (scr[2 * kLlaD + row] + scr[3 * kLlaD + row]) +
+                               (scr[4 * kLlaD + row] + scr[5 * kLlaD + row]);
       if (c == 0) {
         float lt = 0.f;
         for (int w = 0; w < 8; ++w) lt += red_s[8 + w];
