@@ -20,22 +20,20 @@
 //     a running max m (2^(s - m) weights, rescaled lazily as in the prefill),
 //         l = sum e,  ks = sum e k,  vs = sum e v,
 //         D_KK = sum e k k^T,  D_KV = sum e k v^T          (128 x 128 each)
-//     The products over keys run on the tensor cores: per 64-key tile the
-//     scores S = K q (M = 64 keys, N = 8: q is row 0 of an 8-row operand),
-//     read back by four warps, 16 keys each; the weights e (rounded to bf16
-//     once, so that every sum uses the same values) go into diag(e) in
-//     shared memory; the MMA G = K^T diag(e) (the K tile read as an MN-major
-//     A operand) puts e_i k_ia, exact in fp32, in row a of G; the compute
-//     warps pack G into A = (e o K)^T in tensor memory (bf16 pairs) and sum
-//     its rows into ks; then [D_KK | D_KV] += A . [K | V] (N = 256: a
-//     stage's K and V tiles are one MN-major B operand).  The issuing warp
-//     spends ~40 cycles per MMA, so the count matters more than the size:
-//     sixteen per tile.  vs is summed on the CUDA cores from the V tile
-//     while the compute warps wait for the gather.  For sequences shorter
-//     than kLlaSplitLen the bf16 rounding of e o K is not averaged away (the
-//     solve amplifies it along directions the few keys do not span), so a
-//     second product adds its lo part (x = hi + lo).  The piece's record
-//     goes to the workspace.
+//     Per 64-key tile: the scores S = K q on the tensor cores (M = 64 keys,
+//     N = 8: q is row 0 of an 8-row operand), read back by four warps, 16
+//     keys each; the weights e, rounded to bf16 once so that every sum uses
+//     the same values; then the compute warps scale the K tile's rows by e
+//     into A = (e o K)^T in shared memory (as an MN-major operand A has the
+//     K tile's own layout, so this is a row scaling, not a transpose) and
+//     sum ks and vs from the same rows on the CUDA cores; and the tensor
+//     cores add [D_KK | D_KV] += A . [K | V] (N = 256: a stage's K and V
+//     tiles are one MN-major B operand).  The issuing warp spends tens of
+//     cycles per MMA, so the count matters as much as the size: twelve per
+//     tile.  For sequences shorter than kLlaSplitLen the bf16 rounding of
+//     e o K is not averaged away (the solve amplifies it along directions
+//     the few keys do not span), so a second product adds its lo part
+//     (x = hi + lo).  The piece's record goes to the workspace.
 //
 //   lla_solve_kernel  one CTA per (sequence, query head): merges the pieces
 //     like online softmax (weights 2^(m_j - M)), forms S_KK + ridge I and
@@ -89,29 +87,27 @@ struct LlaLayout {
   // [K lo | K hi | V lo | V hi] are one MN-major operand of 256 columns.
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kKV = 0;
-  static constexpr int kDiagBytes = kTile * kTile * 2;        // bf16 [64][64]: diag(e), 128-byte swizzle
-  static constexpr int kDiag = kKV + kLlaStages * kStageBytes;   // two buffers (tile parity)
+  // A = (e o K)^T as an MN-major operand: the K tile's layout with row i
+  // scaled by e_i (bf16 hi, and lo = x - hi below kLlaSplitLen keys); two
+  // buffers each (tile parity)
+  static constexpr int kA = kKV + kLlaStages * kStageBytes;
+  static constexpr int kALo = kA + 2 * kTileBytes;
   static constexpr int kQBytes = 8 * kLlaD * 2;               // bf16 [8][128]: row 0 = q, rows 1.. zero
-  static constexpr int kQ = kDiag + 2 * kDiagBytes;           // K-major B operand, two 64-column atoms
+  static constexpr int kQ = kALo + 2 * kTileBytes;            // K-major B operand, two 64-column atoms
   static constexpr int kE = kQ + kQBytes;                     // float [2][64]: the tile's weights e
   static constexpr int kRed = kE + 2 * kTile * 4;             // float [8 warps][2]
   static constexpr int kBar = kRed + 64;
-  // full[S], empty[S], e_ready[2], da_full[2], da_free[2], a_full, a_free,
-  // drain, s_full[2] (the per-tile hand-offs that run a tile ahead alternate
-  // between two barriers by tile parity, so neither side can be two phases
-  // ahead)
-  static constexpr int kNumBars = 2 * kLlaStages + 11;
+  // full[S], empty[S], s_full[2], s_free[2], a_full[2], a_free[2], drain
+  // (the per-tile hand-offs alternate between two barriers by tile parity)
+  static constexpr int kNumBars = 2 * kLlaStages + 9;
   static constexpr int kMisc = kBar + kNumBars * 8;           // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
 
-// TMEM columns: D = [D_KK | D_KV] in [0, 256); A: hi words at 256, lo words
-// at 288 (keys 2c, 2c+1 in word c); the gather G = K^T diag(e) of tile j at
-// 320 + 64 (j % 2); the scores of tile j at 480 + 8 (j % 2) (M = 64: key r
-// in lane (r % 16) + 32 (r / 16), column 0).
-constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128, kLlaColA = 256;
-__device__ __forceinline__ uint32_t lla_col_g(int buf) { return 320u + 64u * buf; }
-__device__ __forceinline__ uint32_t lla_col_s(int buf) { return 480u + 8u * buf; }
+// TMEM columns: D = [D_KK | D_KV] in [0, 256); the scores of tile j at
+// 256 + 8 (j % 2) (M = 64: key r in lane (r % 16) + 32 (r / 16), column 0).
+constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128;
+__device__ __forceinline__ uint32_t lla_col_s(int buf) { return 256u + 8u * buf; }
 
 // Four MMAs into one accumulator under one elect.sync (four k-steps): the
 // first takes the accumulate flag acc0, the others accumulate.
@@ -126,20 +122,6 @@ __device__ __forceinline__ void lla_mma4_ss(uint32_t d, uint64_t a0, uint64_t b0
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %9, p1;\n\t"
       "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %9, p1;\n\t}" ::"r"(d),
       "l"(a0), "l"(b0), "l"(a1), "l"(b1), "l"(a2), "l"(b2), "l"(a3), "l"(b3), "r"(idesc), "r"(acc0)
-      : "memory");
-}
-
-__device__ __forceinline__ void lla_mma4_ts(uint32_t d, uint32_t a0, uint64_t b0, uint32_t a1, uint64_t b1,
-                                            uint32_t a2, uint64_t b2, uint32_t a3, uint64_t b3, uint32_t idesc,
-                                            uint32_t acc0) {
-  asm volatile(
-      "{\n\t.reg .pred p0, p1, e;\n\tsetp.ne.b32 p0, %10, 0;\n\tsetp.eq.b32 p1, %10, %10;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %9, p0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %4, %9, p1;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %9, p1;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %9, p1;\n\t}" ::"r"(d),
-      "r"(a0), "l"(b0), "r"(a1), "l"(b1), "r"(a2), "l"(b2), "r"(a3), "l"(b3), "r"(idesc), "r"(acc0)
       : "memory");
 }
 
@@ -178,11 +160,6 @@ __device__ __forceinline__ int lla_seq_len(const LlaArgs& a, int b) {
   return n;
 }
 
-// Byte offset of element (row, col) of a [rows][64] bf16 tile with the
-// 128-byte swizzle (16-byte chunks XORed with the row within each 8 rows).
-__device__ __forceinline__ int sw128_off(int row, int col) {
-  return row * 128 + ((((col >> 3) ^ (row & 7)) << 4)) + (col & 7) * 2;
-}
 
 // Instruction descriptor of kind::f16 with both operands' majorness given
 // (bf16 A and B, fp32 accumulator, shape M x N).
@@ -200,13 +177,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
   uint64_t* empty = full + S;
-  uint64_t* e_ready = empty + S;
-  uint64_t* da_full = e_ready + 2;
-  uint64_t* da_free = da_full + 2;
-  uint64_t* a_full = da_free + 2;
-  uint64_t* a_free = a_full + 1;
-  uint64_t* drain = a_free + 1;
-  uint64_t* s_full = drain + 1;
+  uint64_t* s_full = empty + S;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* a_full = s_free + 2;
+  uint64_t* a_free = a_full + 2;
+  uint64_t* drain = a_free + 2;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + Ly::kMisc + 4);
   float* red_s = reinterpret_cast<float*>(sm + Ly::kRed);
@@ -251,13 +226,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&e_ready[i], kLlaCompute);
-      mbar_init(&da_full[i], 1);
-      mbar_init(&da_free[i], kLlaCompute);
       mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], kLlaCompute);
+      mbar_init(&a_full[i], kLlaCompute);
+      mbar_init(&a_free[i], 1);
     }
-    mbar_init(a_full, kLlaCompute);
-    mbar_init(a_free, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -272,9 +245,6 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       v[e] = ((i >> 3) & 7) == 0 ? a.q[(size_t)bh * kLlaD + (i >> 6) * 64 + (i & 7) * 8 + e] : __float2bfloat16_rn(0.f);
     *reinterpret_cast<uint4*>(sm + Ly::kQ + i * 16) = *reinterpret_cast<const uint4*>(v);
   }
-  // diag(e) starts as zeros; only its diagonal changes per tile
-  for (int i = threadIdx.x; i < 2 * Ly::kDiagBytes / 16; i += kLlaThreads)
-    reinterpret_cast<uint4*>(sm + Ly::kDiag)[i] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_base_s, 512);
@@ -318,47 +288,39 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per tile: the scores S = K q (M = 64 keys, N = 8, K-major A and B); the
-    // gather G = K^T diag(e) (128 x 64, A = the K tile read as MN-major,
-    // B = diag(e)); once the compute warps have packed G into
-    // A = (e o K)^T: [D_KK | D_KV] += A . [K | V] (TS, 128 x 256, the stage's
-    // K and V tiles as one MN-major B operand).  Sixteen MMAs per tile (24
-    // below kLlaSplitLen keys), four under each elect.
+    // Per tile: the scores S = K q (M = 64 keys, N = 8, K-major A and B) and,
+    // once the compute warps have written A = (e o K)^T, the products
+    // [D_KK | D_KV] += A . [K | V] (SS, 128 x 256, A and the stage's K and V
+    // tiles as MN-major operands).  Twelve MMAs per tile (sixteen below
+    // kLlaSplitLen keys), four under each elect.
     constexpr uint32_t kIdS = idesc_bf16_ab(kTile, 8, false, false);
-    constexpr uint32_t kIdG = idesc_bf16_ab(128, kTile, true, false);
-    constexpr uint32_t kIdD = idesc_bf16(128, 2 * kLlaD, true);
+    constexpr uint32_t kIdD = idesc_bf16_ab(128, 2 * kLlaD, true, true);
     const uint64_t dkS = smem_desc_sw128(smem_u32(sm + Ly::kKV), 16, 1024);                  // K, K-major A
     const uint64_t dqS = smem_desc_sw128(smem_u32(sm + Ly::kQ), 16, 1024);                   // q, K-major B
     const uint64_t dkvM = smem_desc_sw128(smem_u32(sm + Ly::kKV), Ly::kTileBytes / 2, 1024);   // MN-major, 64-col atoms
-    const uint64_t dd = smem_desc_sw128(smem_u32(sm + Ly::kDiag), 16, 1024);                 // diag(e), K-major B
+    const uint64_t daM = smem_desc_sw128(smem_u32(sm + Ly::kA), Ly::kTileBytes / 2, 1024);
+    const uint64_t dlM = smem_desc_sw128(smem_u32(sm + Ly::kALo), Ly::kTileBytes / 2, 1024);
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
     auto stage_off = [&](int j) { return (uint64_t)(((j % S) * Ly::kStageBytes) >> 4); };
-    // main(j) = [D_KK | D_KV] += A . [K(j) | V(j)]; A holds tile j's packed
-    // gather (16 keys = 8 A words and 16 B rows, 2048 bytes, per step).
-    // Issue order S(0), S(1), then per tile j: G(j), main(j - 1), S(j + 2):
-    // the gather of the next tile runs while the compute warps pack this
-    // one, and the scores are two tiles ahead.
+    // main(j): 16 keys per step, 16 rows (2048 bytes) of A and of [K | V].
     auto issue_main = [&](int jm) {
       const uint64_t kv = dkvM + stage_off(jm);
-      const uint32_t ahi = tmem + kLlaColA;
-      lla_mma4_ts(tmem + kLlaColKK, ahi, kv, ahi + 8u, kv + 128, ahi + 16u, kv + 256, ahi + 24u, kv + 384, kIdD,
+      const uint64_t ab = (uint64_t)(((jm & 1) * Ly::kTileBytes) >> 4);
+      const uint64_t ah = daM + ab;
+      lla_mma4_ss(tmem + kLlaColKK, ah, kv, ah + 128, kv + 128, ah + 256, kv + 256, ah + 384, kv + 384, kIdD,
                   jm > 0 ? 1u : 0u);
       if (split_lo) {
-        const uint32_t alo = ahi + 32u;
-        lla_mma4_ts(tmem + kLlaColKK, alo, kv, alo + 8u, kv + 128, alo + 16u, kv + 256, alo + 24u, kv + 384, kIdD,
-                    1u);
+        const uint64_t al = dlM + ab;
+        lla_mma4_ss(tmem + kLlaColKK, al, kv, al + 128, kv + 128, al + 256, kv + 256, al + 384, kv + 384, kIdD, 1u);
       }
-      tc_commit(a_free);
+      tc_commit(&a_free[jm & 1]);
       tc_commit(&empty[jm % S]);
     };
-    // S(js) once tile js has landed (buffer js % 2: the scores of tile js - 2
-    // have been read, which e_ready(js - 2) reported before G(js - 2)).
-    // 16 components per step: box kk / 4, 32 bytes into the 128-byte row.
-    auto issue_s = [&](int js) -> bool {
-      if (!wait_warp(&full[js % S], (js / S) & 1)) return false;
-      tc_fence_after();
+    // S(js) once tile js has landed; 16 components per step: box kk / 4, 32
+    // bytes into the 128-byte row.
+    auto issue_s = [&](int js) {
       const uint64_t ka = dkS + stage_off(js);
       constexpr uint64_t kBoxA = Ly::kTileBytes / 2 / 16, kBoxB = Ly::kQBytes / 2 / 16;
       const uint32_t d = tmem + lla_col_s(js & 1);
@@ -366,31 +328,31 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       lla_mma4_ss(d, ka + kBoxA, dqS + kBoxB, ka + kBoxA + 2, dqS + kBoxB + 2, ka + kBoxA + 4, dqS + kBoxB + 4,
                   ka + kBoxA + 6, dqS + kBoxB + 6, kIdS, 1u);
       tc_commit(&s_full[js & 1]);
-      return true;
     };
-    bool ok = issue_s(0) && (n < 2 || issue_s(1));
-    for (int j = 0; ok && j <= n; ++j) {
+    // Issue order S(0), S(1), then per tile j: S(j + 2) (once the scores of
+    // tile j, in the same TMEM buffer, have been read), main(j).  The scores
+    // run two tiles ahead of the products, so the compute warps find them
+    // done.
+    bool ok = true;
+    for (int js = 0; ok && js < 2 && js < n; ++js) {
+      if (!(ok = wait_warp(&full[js % S], (js / S) & 1))) break;
+      tc_fence_after();
+      issue_s(js);
+    }
+    for (int j = 0; ok && j < n; ++j) {
       if (__any_sync(0xffffffffu, *abort_flag != 0)) {
         ok = false;
         break;
       }
-      if (j < n) {   // G(j) (tile j has landed: S(j) waited for it)
-        const int gb = j & 1;
-        if (!(ok = wait_warp(&e_ready[gb], (j >> 1) & 1))) break;
-        if (j >= 2 && !(ok = wait_warp(&da_free[gb], ((j >> 1) - 1) & 1))) break;   // G buffer gb was read
+      if (j + 2 < n) {
+        if (!(ok = wait_warp(&s_free[j & 1], (j >> 1) & 1))) break;
+        if (!(ok = wait_warp(&full[(j + 2) % S], ((j + 2) / S) & 1))) break;
         tc_fence_after();
-        // 16 keys per step: 16 rows (2048 bytes) of the K tile, 32 bytes of diag(e)
-        const uint64_t ks = dkvM + stage_off(j);
-        const uint64_t ddb = dd + (uint64_t)((gb * Ly::kDiagBytes) >> 4);
-        lla_mma4_ss(tmem + lla_col_g(gb), ks, ddb, ks + 128, ddb + 2, ks + 256, ddb + 4, ks + 384, ddb + 6, kIdG, 0u);
-        tc_commit(&da_full[gb]);
+        issue_s(j + 2);
       }
-      if (j >= 1) {   // main(j - 1), once the compute warps have packed tile j - 1
-        if (!(ok = wait_warp(a_full, (j - 1) & 1))) break;
-        tc_fence_after();
-        issue_main(j - 1);
-      }
-      if (j + 2 < n && !(ok = issue_s(j + 2))) break;
+      if (!(ok = wait_warp(&a_full[j & 1], (j >> 1) & 1))) break;
+      tc_fence_after();
+      issue_main(j);
     }
     if (!ok && lane == 0) *abort_flag = 1;
     // Every issued MMA must complete before tensor memory is released.
@@ -400,12 +362,9 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ compute
-    // Two warps per TMEM lane quarter: warp cw (0..7) takes rows 32 (warp % 4)
-    // .. of the accumulators and the keys 32 kh .. 32 kh + 31 of each tile's
-    // gather (kh = cw / 4).
     const int c = threadIdx.x - 64;            // 0..255
     const int cw = warp - 2;                   // compute warp 0..7
-    const int kh = cw >> 2;                    // key half of the gather this thread packs
+    const int kh = cw >> 2;                    // D half this warp rescales and writes (D_KK, D_KV)
     const int wq = warp & 3;                   // TMEM lane quarter of this warp
     const int row = wq * 32 + lane;            // TMEM lane = component a of k
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
@@ -413,19 +372,22 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     // (TMEM lanes 32 wq .. 32 wq + 15 of the M = 64 product), one per lane.
     const bool skey = cw < 4 && lane < 16;
     const int key = 16 * wq + lane;
-    // sum e v: thread c takes components 2 (c % 64), + 1 and keys 16 (c / 64) ..
-    // of each tile (a warp reads whole 128-byte rows of one V box).
-    const int vcp = c & 63, vkq = c >> 6, vchunk = (vcp & 31) >> 2;
-    const int voff = Ly::kTileBytes + (vcp >> 5) * (Ly::kTileBytes / 2) + (vcp & 3) * 4;   // + row, swizzled chunk
+    // Scale phase: thread c takes the 16-byte chunk cc = c % 16 of rows
+    // kg + 16 m (kg = c / 16, m = 0..3) of the K and V tiles: components
+    // 64 (cc / 8) + 8 (cc % 8) .. + 7.  A warp covers two whole rows.
+    const int cc = c & 15, kg = c >> 4;
+    const int coff = (cc >> 3) * (Ly::kTileBytes / 2);   // + row * 128 + swizzled chunk
     float m_ref = -INFINITY, l_acc = 0.f;
-    float ks_acc = 0.f;                        // sum e k_row over this thread's key half
-    float vs0 = 0.f, vs1 = 0.f;                // sum e v over this thread's key quarter
-    // Tile t's scores, weights, diag(e) and e (buffers t % 2), then e_ready.
-    // The running max moves only when a score passes it by kLlaRescaleLog2
-    // (one barrier reduction per tile decides; the first tile always takes
-    // its max).  A new running max returns the factor that everything
+    float ks[8], vs[8];                        // sum e k, sum e v over this thread's rows, its 8 components
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ks[i] = vs[i] = 0.f;
+    // Tile t's scores and weights e (buffer t % 2); wv carries the waits of
+    // the scale phase that follows (false: one of them ran out).  The
+    // running max moves only when a score passes it by kLlaRescaleLog2 (one
+    // barrier reduction per tile decides; the first tile always takes its
+    // max).  A new running max returns the factor that everything
     // accumulated over tiles < t takes before tile t is added.
-    auto scores_phase = [&](int t, float& alpha_d) -> bool {
+    auto scores_phase = [&](int t, float& alpha_d, bool wv) -> bool {
       const int gb = t & 1;
       const bool w = __all_sync(0xffffffffu, !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[gb], (t >> 1) & 1));
       const int nvalid = min(kTile, len - (t0 + t) * kTile);
@@ -436,9 +398,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         tmem_wait_ld();
         if (skey && key < nvalid) sc = __uint_as_float(r) * a.scale_log2;
       }
+      tc_fence_before();
+      mbar_arrive(&s_free[gb]);   // S(t + 2) may overwrite the buffer
       alpha_d = 1.f;
-      if (bar_or(1, kLlaCompute, t == 0 || !w || sc > m_ref + kLlaRescaleLog2)) {   // uniform
-        if (!bar_and(2, kLlaCompute, w)) return false;
+      if (bar_or(1, kLlaCompute, t == 0 || !w || !wv || sc > m_ref + kLlaRescaleLog2)) {   // uniform
+        if (!bar_and(2, kLlaCompute, w && wv)) return false;
         const float wmax = warp_max(sc);
         if (lane == 0) red_s[cw] = wmax;
         bar_and(3, kLlaCompute, true);
@@ -452,66 +416,35 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
           l_acc *= alpha_d;
         }
       }
-      // ---- the weights, rounded to bf16: every product below uses these values
+      // ---- the weights, rounded to bf16: every sum and product uses these values
       if (skey) {   // every key of the tile, its weight 0 past the end
         const float e = key < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f;
         l_acc += e;
-        __nv_bfloat16* diag_s = reinterpret_cast<__nv_bfloat16*>(sm + Ly::kDiag + gb * Ly::kDiagBytes);
-        diag_s[sw128_off(key, key) >> 1] = __float2bfloat16_rn(e);
         reinterpret_cast<float*>(sm + Ly::kE)[gb * kTile + key] = e;
       }
       if (nvalid < kTile) {
-        // Rows past the end are operands of the gather and the products
-        // (their weights are 0, but 0 * NaN is not): zero them in K and V.
-        // S(t), the only earlier reader of the tile, is done (s_full).
+        // Rows past the end are operands of the products (their weights are
+        // 0, but 0 * NaN is not): zero them in K and V.  S(t), the only
+        // earlier reader of the tile, is done (s_full).
         uint8_t* st = sm + Ly::kKV + (t % S) * Ly::kStageBytes;
         for (int i = c; i < (kTile - nvalid) * 16; i += kLlaCompute) {
-          const int r = nvalid + (i >> 4), cc = i & 15;   // cc: box (cc >> 3), chunk (cc & 7)
-          const int off = (cc >> 3) * (Ly::kTileBytes / 2) + r * 128 + (cc & 7) * 16;
+          const int r = nvalid + (i >> 4), ci = i & 15;   // ci: box (ci >> 3), chunk (ci & 7)
+          const int off = (ci >> 3) * (Ly::kTileBytes / 2) + r * 128 + (ci & 7) * 16;
           *reinterpret_cast<uint4*>(st + off) = make_uint4(0u, 0u, 0u, 0u);
           *reinterpret_cast<uint4*>(st + Ly::kTileBytes + off) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      fence_proxy_async_smem();
-      mbar_arrive(&e_ready[gb]);
       return true;
     };
-    // Tile t: sum e v over this thread's keys (while G(t) and main(t - 1) run;
-    // V(t) stays resident until main(t), after a_full(t), is done), then the
-    // gather into A = (e o K)^T (after main(t - 1) has read A), the deferred
-    // rescale of D, and sum e k from the gather's rows.
-    auto pack_phase = [&](int t, float alpha_d) -> bool {
+    // Tile t: the deferred rescale of D (a new running max; main(t - 1) is
+    // done), then A = (e o K)^T into A buffer t % 2 (main(t - 2) has read
+    // it) with sum e k and sum e v from the same rows; a_full.  The waits
+    // come before the barrier of scores(t + 1), so that one barrier per tile
+    // serves both phases.
+    auto scale_phase = [&](int t, float alpha_d) {
       const int gb = t & 1;
-      {
-        const float* et = reinterpret_cast<const float*>(sm + Ly::kE) + gb * kTile + 16 * vkq;
-        const uint8_t* vt = sm + Ly::kKV + (t % S) * Ly::kStageBytes + voff;
-        // Rows past the end hold zeros (scores(t) cleared them; a barrier
-        // since orders that before these reads) and weight 0.
-        uint32_t w2[16];
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj)   // row 16 vkq + jj, whose swizzle is jj % 8
-          w2[jj] = *reinterpret_cast<const uint32_t*>(vt + (16 * vkq + jj) * 128 + ((vchunk ^ (jj & 7)) << 4));
-        float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const float4 e4 = lds_f4(smem_u32(et + 4 * q4));
-          const float ev[4] = {e4.x, e4.y, e4.z, e4.w};
-#pragma unroll
-          for (int u = 0; u < 4; u += 2) {
-            a0 = fmaf(ev[u], bf16_lo_f(w2[4 * q4 + u]), a0);
-            a1 = fmaf(ev[u], bf16_hi_f(w2[4 * q4 + u]), a1);
-            b0 = fmaf(ev[u + 1], bf16_lo_f(w2[4 * q4 + u + 1]), b0);
-            b1 = fmaf(ev[u + 1], bf16_hi_f(w2[4 * q4 + u + 1]), b1);
-          }
-        }
-        vs0 = fmaf(vs0, alpha_d, a0 + b0);
-        vs1 = fmaf(vs1, alpha_d, a1 + b1);
-      }
-      const bool wg = mbar_wait_bounded(a.wait_ns, &da_full[gb], (t >> 1) & 1);
-      const bool wa = t == 0 || mbar_wait_bounded(a.wait_ns, a_free, (t - 1) & 1);
-      if (!bar_and(2, kLlaCompute, wg && wa)) return false;
       tc_fence_after();
-      if (alpha_d != 1.f) {   // uniform; main(t - 1) is done
+      if (alpha_d != 1.f) {   // uniform
 #pragma unroll 1
         for (int part = 4 * kh; part < 4 * kh + 4; ++part) {   // D_KK (kh 0) or D_KV (kh 1), 32 columns at a time
           uint32_t r[32];
@@ -522,66 +455,84 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
           for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha_d);
           tmem_st32(addr, r);
         }
-      }
-      uint32_t g[32];
-      tmem_ld32(tmem + lane_off + lla_col_g(gb) + 32u * kh, g);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&da_free[gb]);
-      auto pack = [&](auto split_tag) {
-        constexpr bool kSplit = decltype(split_tag)::value;
-        uint32_t hi[16], lo[16];
+        tmem_wait_st();
 #pragma unroll
-        for (int p = 0; p < 16; ++p) {
-          const float p0 = __uint_as_float(g[2 * p]), p1 = __uint_as_float(g[2 * p + 1]);
-          hi[p] = pack_bf16(p0, p1);
-          if constexpr (kSplit) lo[p] = pack_bf16(p0 - bf16_lo_f(hi[p]), p1 - bf16_hi_f(hi[p]));
+        for (int i = 0; i < 8; ++i) {
+          ks[i] *= alpha_d;
+          vs[i] *= alpha_d;
         }
-        tmem_st16(tmem + lane_off + kLlaColA + 16u * kh, hi);
-        if constexpr (kSplit) tmem_st16(tmem + lane_off + kLlaColA + 32u + 16u * kh, lo);
-      };
-      if (split_lo)
-        pack(std::true_type{});
-      else
-        pack(std::false_type{});
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(a_full);
-      // G holds e_i k_ia exactly (one nonzero product per entry)
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      }
+      const float* et = reinterpret_cast<const float*>(sm + Ly::kE) + gb * kTile;
+      const uint8_t* st = sm + Ly::kKV + (t % S) * Ly::kStageBytes;
+      uint8_t* ah = sm + Ly::kA + gb * Ly::kTileBytes;
+      uint8_t* al = sm + Ly::kALo + gb * Ly::kTileBytes;
+      // row kg + 16 m has swizzle kg % 8
+      const int roff = coff + (((cc & 7) ^ (kg & 7)) << 4) + kg * 128;
+      uint4 kw[4], vw[4];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) s4[i & 3] += __uint_as_float(g[i]);
-      ks_acc = fmaf(ks_acc, alpha_d, (s4[0] + s4[1]) + (s4[2] + s4[3]));
-      return true;
+      for (int m = 0; m < 4; ++m) {
+        kw[m] = *reinterpret_cast<const uint4*>(st + roff + m * 2048);
+        vw[m] = *reinterpret_cast<const uint4*>(st + Ly::kTileBytes + roff + m * 2048);
+      }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float e = et[kg + 16 * m];
+        const uint32_t kx[4] = {kw[m].x, kw[m].y, kw[m].z, kw[m].w};
+        const uint32_t vx[4] = {vw[m].x, vw[m].y, vw[m].z, vw[m].w};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          // e k is exact in fp32 (a product of two bf16 values)
+          const float p0 = e * bf16_lo_f(kx[p]), p1 = e * bf16_hi_f(kx[p]);
+          ks[2 * p] += p0;
+          ks[2 * p + 1] += p1;
+          vs[2 * p] = fmaf(e, bf16_lo_f(vx[p]), vs[2 * p]);
+          vs[2 * p + 1] = fmaf(e, bf16_hi_f(vx[p]), vs[2 * p + 1]);
+          hi[p] = pack_bf16(p0, p1);
+          lo[p] = pack_bf16(p0 - bf16_lo_f(hi[p]), p1 - bf16_hi_f(hi[p]));
+        }
+        *reinterpret_cast<uint4*>(ah + roff + m * 2048) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        if (split_lo) *reinterpret_cast<uint4*>(al + roff + m * 2048) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&a_full[gb]);
     };
-    // scores(t + 1) runs before pack(t), so the gather of tile t + 1 overlaps
-    // the packing of tile t and main(t).
+    // scores(t + 1) runs before scale(t): the scores are ready, and the
+    // weights of tile t are visible to every compute thread after the
+    // barrier of scores(t + 1).
     float alpha_pack = 1.f;   // the rescale before tile t is added, decided by scores(t)
-    bool fine = scores_phase(0, alpha_pack);
+    bool fine = scores_phase(0, alpha_pack, true);
     int j = 0;
     for (; fine && j < n; ++j) {
+      bool wv = j < 2 || mbar_wait_bounded(a.wait_ns, &a_free[j & 1], ((j >> 1) - 1) & 1);
+      if (alpha_pack != 1.f)   // uniform; j >= 1
+        wv = wv && mbar_wait_bounded(a.wait_ns, &a_free[(j - 1) & 1], ((j - 1) >> 1) & 1);
       float alpha_next = 1.f;
       if (j + 1 < n) {
-        if (!(fine = scores_phase(j + 1, alpha_next))) break;
-      } else {
-        bar_and(1, kLlaCompute, true);   // the last tile's weights, visible to every compute thread
+        if (!(fine = scores_phase(j + 1, alpha_next, wv))) break;
+      } else if (!(fine = bar_and(1, kLlaCompute, wv))) {
+        break;
       }
-      if (!(fine = pack_phase(j, alpha_pack))) break;
+      scale_phase(j, alpha_pack);
       alpha_pack = alpha_next;
     }
     // ---- the piece's record: wait for the last products, then write
-    bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, a_free, (n - 1) & 1);
+    bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, &a_free[(n - 1) & 1], ((n - 1) >> 1) & 1);
     wl = bar_and(3, kLlaCompute, wl);
     const float lw = warp_sum(l_acc);
     if (lane == 0) red_s[8 + cw] = lw;
-    // the first moments' partial sums meet in the diag buffers, idle once
-    // the last products are done: [2][128] halves of sum e k, [4][128]
-    // quarters of sum e v
-    float* scr = reinterpret_cast<float*>(sm + Ly::kDiag);
+    // the first moments' partial sums meet in the A buffers, idle once the
+    // last products are done: [16 row groups][128] of sum e k, then of sum e v
+    float* scr = reinterpret_cast<float*>(sm + Ly::kA);
     if (wl) {
-      scr[kh * kLlaD + row] = ks_acc;
-      scr[2 * kLlaD + vkq * kLlaD + 2 * vcp] = vs0;
-      scr[2 * kLlaD + vkq * kLlaD + 2 * vcp + 1] = vs1;
+      const int d0 = 64 * (cc >> 3) + 8 * (cc & 7);
+      float4* pk = reinterpret_cast<float4*>(scr + kg * kLlaD + d0);
+      float4* pv = reinterpret_cast<float4*>(scr + 16 * kLlaD + kg * kLlaD + d0);
+      pk[0] = make_float4(ks[0], ks[1], ks[2], ks[3]);
+      pk[1] = make_float4(ks[4], ks[5], ks[6], ks[7]);
+      pv[0] = make_float4(vs[0], vs[1], vs[2], vs[3]);
+      pv[1] = make_float4(vs[4], vs[5], vs[6], vs[7]);
     }
     bar_and(2, kLlaCompute, true);
     if (wl) {
@@ -597,11 +548,14 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) dst[i * kLlaD] = __uint_as_float(r[i]);
       }
-      if (kh == 0)
-        rec[kLlaRecKs + row] = scr[row] + scr[kLlaD + row];
-      else
-        rec[kLlaRecVs + row] = (scr[2 * kLlaD + row] + scr[3 * kLlaD + row]) +
-                               (scr[4 * kLlaD + row] + scr[5 * kLlaD + row]);
+      {
+        const int comp = c & (kLlaD - 1);
+        const float* src = scr + (c >= kLlaD ? 16 * kLlaD : 0) + comp;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int g = 0; g < 16; ++g) s4[g & 3] += src[g * kLlaD];
+        rec[(c >= kLlaD ? kLlaRecVs : kLlaRecKs) + comp] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      }
       if (c == 0) {
         float lt = 0.f;
         for (int w = 0; w < 8; ++w) lt += red_s[8 + w];
