@@ -51,7 +51,7 @@
 namespace plx {
 
 constexpr int kLlaD = 128;
-constexpr int kLlaStages = 4;            // K and V ring depth (tiles)
+constexpr int kLlaStages = 5;            // K and V ring depth (tiles)
 constexpr int kLlaThreads = 320;         // TMA producer warp, MMA warp, eight compute warps
 constexpr int kLlaCompute = 256;
 constexpr int kLlaSplitLen = 1024;       // shorter sequences add the lo part of e o K
@@ -88,12 +88,11 @@ struct LlaLayout {
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kKV = 0;
   // A = (e o K)^T as an MN-major operand: the K tile's layout with row i
-  // scaled by e_i (bf16 hi, and lo = x - hi below kLlaSplitLen keys); two
-  // buffers each (tile parity)
+  // scaled by e_i, in bf16.  Two buffers: hi of tile t in buffer t % 2; below
+  // kLlaSplitLen keys hi in buffer 0 and lo = x - hi in buffer 1.
   static constexpr int kA = kKV + kLlaStages * kStageBytes;
-  static constexpr int kALo = kA + 2 * kTileBytes;
   static constexpr int kQBytes = 8 * kLlaD * 2;               // bf16 [8][128]: row 0 = q, rows 1.. zero
-  static constexpr int kQ = kALo + 2 * kTileBytes;            // K-major B operand, two 64-column atoms
+  static constexpr int kQ = kA + 2 * kTileBytes;              // K-major B operand, two 64-column atoms
   static constexpr int kE = kQ + kQBytes;                     // float [2][64]: the tile's weights e
   static constexpr int kRed = kE + 2 * kTile * 4;             // float [8 warps][2]
   static constexpr int kBar = kRed + 64;
@@ -299,7 +298,6 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     const uint64_t dqS = smem_desc_sw128(smem_u32(sm + Ly::kQ), 16, 1024);                   // q, K-major B
     const uint64_t dkvM = smem_desc_sw128(smem_u32(sm + Ly::kKV), Ly::kTileBytes / 2, 1024);   // MN-major, 64-col atoms
     const uint64_t daM = smem_desc_sw128(smem_u32(sm + Ly::kA), Ly::kTileBytes / 2, 1024);
-    const uint64_t dlM = smem_desc_sw128(smem_u32(sm + Ly::kALo), Ly::kTileBytes / 2, 1024);
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
@@ -307,12 +305,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     // main(j): 16 keys per step, 16 rows (2048 bytes) of A and of [K | V].
     auto issue_main = [&](int jm) {
       const uint64_t kv = dkvM + stage_off(jm);
-      const uint64_t ab = (uint64_t)(((jm & 1) * Ly::kTileBytes) >> 4);
-      const uint64_t ah = daM + ab;
+      const uint64_t ah = daM + (split_lo ? 0 : (uint64_t)(((jm & 1) * Ly::kTileBytes) >> 4));
       lla_mma4_ss(tmem + kLlaColKK, ah, kv, ah + 128, kv + 128, ah + 256, kv + 256, ah + 384, kv + 384, kIdD,
                   jm > 0 ? 1u : 0u);
       if (split_lo) {
-        const uint64_t al = dlM + ab;
+        const uint64_t al = daM + (uint64_t)(Ly::kTileBytes >> 4);
         lla_mma4_ss(tmem + kLlaColKK, al, kv, al + 128, kv + 128, al + 256, kv + 256, al + 384, kv + 384, kIdD, 1u);
       }
       tc_commit(&a_free[jm & 1]);
@@ -381,12 +378,15 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     float ks[8], vs[8];                        // sum e k, sum e v over this thread's rows, its 8 components
 #pragma unroll
     for (int i = 0; i < 8; ++i) ks[i] = vs[i] = 0.f;
-    // Tile t's scores and weights e (buffer t % 2); wv carries the waits of
-    // the scale phase that follows (false: one of them ran out).  The
-    // running max moves only when a score passes it by kLlaRescaleLog2 (one
-    // barrier reduction per tile decides; the first tile always takes its
-    // max).  A new running max returns the factor that everything
-    // accumulated over tiles < t takes before tile t is added.
+    // Tile t's scores and weights e (buffer t % 2).  The weights are taken
+    // against the running max before the tile's one barrier, which both
+    // publishes them and decides (a reduction) whether the running max
+    // moves: only when a score passes it by kLlaRescaleLog2, or on the first
+    // tile.  On that rare path the max is reduced, the weights are taken
+    // again, and alpha_d returns the factor that everything accumulated over
+    // tiles < t takes before tile t is added; D's rescale needs main(t - 1)
+    // done, so that path waits for it.  wv carries the wait for the A
+    // buffer of the scale phase that follows (false: it ran out).
     auto scores_phase = [&](int t, float& alpha_d, bool wv) -> bool {
       const int gb = t & 1;
       const bool w = __all_sync(0xffffffffu, !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[gb], (t >> 1) & 1));
@@ -400,27 +400,13 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&s_free[gb]);   // S(t + 2) may overwrite the buffer
-      alpha_d = 1.f;
-      if (bar_or(1, kLlaCompute, t == 0 || !w || !wv || sc > m_ref + kLlaRescaleLog2)) {   // uniform
-        if (!bar_and(2, kLlaCompute, w && wv)) return false;
-        const float wmax = warp_max(sc);
-        if (lane == 0) red_s[cw] = wmax;
-        bar_and(3, kLlaCompute, true);
-        const float tmax = fmaxf(fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3])),
-                                 fmaxf(fmaxf(red_s[4], red_s[5]), fmaxf(red_s[6], red_s[7])));
-        if (t == 0) {
-          m_ref = tmax;   // the piece's first tile holds a key: tmax is finite
-        } else if (tmax > m_ref + kLlaRescaleLog2) {   // uniform: every compute thread saw the same maxima
-          alpha_d = ex2(m_ref - tmax);
-          m_ref = tmax;
-          l_acc *= alpha_d;
-        }
-      }
-      // ---- the weights, rounded to bf16: every sum and product uses these values
+      float* e_s = reinterpret_cast<float*>(sm + Ly::kE) + gb * kTile;
+      // the weights, rounded to bf16: every sum and product uses these values
+      auto weight = [&]() { return key < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f; };
+      float e = 0.f;
       if (skey) {   // every key of the tile, its weight 0 past the end
-        const float e = key < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f;
-        l_acc += e;
-        reinterpret_cast<float*>(sm + Ly::kE)[gb * kTile + key] = e;
+        e = weight();
+        e_s[key] = e;
       }
       if (nvalid < kTile) {
         // Rows past the end are operands of the products (their weights are
@@ -434,17 +420,40 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
           *reinterpret_cast<uint4*>(st + Ly::kTileBytes + off) = make_uint4(0u, 0u, 0u, 0u);
         }
       }
+      alpha_d = 1.f;
+      if (bar_or(1, kLlaCompute, t == 0 || !w || !wv || sc > m_ref + kLlaRescaleLog2)) {   // uniform
+        if (!bar_and(2, kLlaCompute, w && wv)) return false;
+        const float wmax = warp_max(sc);
+        if (lane == 0) red_s[cw] = wmax;
+        bar_and(3, kLlaCompute, true);
+        const float tmax = fmaxf(fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3])),
+                                 fmaxf(fmaxf(red_s[4], red_s[5]), fmaxf(red_s[6], red_s[7])));
+        bool wd = true;
+        if (t == 0) {
+          m_ref = tmax;   // the piece's first tile holds a key: tmax is finite
+        } else if (tmax > m_ref + kLlaRescaleLog2) {   // uniform: every compute thread saw the same maxima
+          alpha_d = ex2(m_ref - tmax);
+          m_ref = tmax;
+          l_acc *= alpha_d;
+          wd = mbar_wait_bounded(a.wait_ns, &a_free[(t - 1) & 1], ((t - 1) >> 1) & 1);   // main(t - 1) done
+        }
+        if (skey) {
+          e = weight();
+          e_s[key] = e;
+        }
+        if (!bar_and(2, kLlaCompute, wd)) return false;   // the new weights, visible to every compute thread
+      }
+      l_acc += e;
       return true;
     };
-    // Tile t: the deferred rescale of D (a new running max; main(t - 1) is
-    // done), then A = (e o K)^T into A buffer t % 2 (main(t - 2) has read
-    // it) with sum e k and sum e v from the same rows; a_full.  The waits
-    // come before the barrier of scores(t + 1), so that one barrier per tile
-    // serves both phases.
-    auto scale_phase = [&](int t, float alpha_d) {
+    // Tile t right after its scores: the deferred rescale of D, then
+    // A = (e o K)^T into its A buffer with sum e k and sum e v from the same
+    // rows; a_full.
+    auto scale_phase = [&](int t, float alpha_d, auto split_tag) {
+      constexpr bool kSplit = decltype(split_tag)::value;
       const int gb = t & 1;
       tc_fence_after();
-      if (alpha_d != 1.f) {   // uniform
+      if (alpha_d != 1.f) {   // uniform; main(t - 1) is done
 #pragma unroll 1
         for (int part = 4 * kh; part < 4 * kh + 4; ++part) {   // D_KK (kh 0) or D_KV (kh 1), 32 columns at a time
           uint32_t r[32];
@@ -464,8 +473,8 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       }
       const float* et = reinterpret_cast<const float*>(sm + Ly::kE) + gb * kTile;
       const uint8_t* st = sm + Ly::kKV + (t % S) * Ly::kStageBytes;
-      uint8_t* ah = sm + Ly::kA + gb * Ly::kTileBytes;
-      uint8_t* al = sm + Ly::kALo + gb * Ly::kTileBytes;
+      uint8_t* ah = sm + Ly::kA + (kSplit ? 0 : gb * Ly::kTileBytes);
+      uint8_t* al = sm + Ly::kA + Ly::kTileBytes;
       // row kg + 16 m has swizzle kg % 8
       const int roff = coff + (((cc & 7) ^ (kg & 7)) << 4) + kg * 128;
       uint4 kw[4], vw[4];
@@ -489,33 +498,28 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
           vs[2 * p] = fmaf(e, bf16_lo_f(vx[p]), vs[2 * p]);
           vs[2 * p + 1] = fmaf(e, bf16_hi_f(vx[p]), vs[2 * p + 1]);
           hi[p] = pack_bf16(p0, p1);
-          lo[p] = pack_bf16(p0 - bf16_lo_f(hi[p]), p1 - bf16_hi_f(hi[p]));
+          if constexpr (kSplit) lo[p] = pack_bf16(p0 - bf16_lo_f(hi[p]), p1 - bf16_hi_f(hi[p]));
         }
         *reinterpret_cast<uint4*>(ah + roff + m * 2048) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        if (split_lo) *reinterpret_cast<uint4*>(al + roff + m * 2048) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        if constexpr (kSplit) *reinterpret_cast<uint4*>(al + roff + m * 2048) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&a_full[gb]);
     };
-    // scores(t + 1) runs before scale(t): the scores are ready, and the
-    // weights of tile t are visible to every compute thread after the
-    // barrier of scores(t + 1).
-    float alpha_pack = 1.f;   // the rescale before tile t is added, decided by scores(t)
-    bool fine = scores_phase(0, alpha_pack, true);
+    // Before scores(t): the A buffers that scale(t) writes are free once
+    // main(t - 2) is done (main(t - 1) when lo takes the second buffer).
+    float alpha = 1.f;
+    bool fine = true;
     int j = 0;
     for (; fine && j < n; ++j) {
-      bool wv = j < 2 || mbar_wait_bounded(a.wait_ns, &a_free[j & 1], ((j >> 1) - 1) & 1);
-      if (alpha_pack != 1.f)   // uniform; j >= 1
-        wv = wv && mbar_wait_bounded(a.wait_ns, &a_free[(j - 1) & 1], ((j - 1) >> 1) & 1);
-      float alpha_next = 1.f;
-      if (j + 1 < n) {
-        if (!(fine = scores_phase(j + 1, alpha_next, wv))) break;
-      } else if (!(fine = bar_and(1, kLlaCompute, wv))) {
-        break;
-      }
-      scale_phase(j, alpha_pack);
-      alpha_pack = alpha_next;
+      const int jb = j - (split_lo ? 1 : 2);
+      const bool wv = jb < 0 || mbar_wait_bounded(a.wait_ns, &a_free[jb & 1], (jb >> 1) & 1);
+      if (!(fine = scores_phase(j, alpha, wv))) break;
+      if (split_lo)
+        scale_phase(j, alpha, std::true_type{});
+      else
+        scale_phase(j, alpha, std::false_type{});
     }
     // ---- the piece's record: wait for the last products, then write
     bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, &a_free[(n - 1) & 1], ((n - 1) >> 1) & 1);
