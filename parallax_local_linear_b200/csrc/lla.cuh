@@ -22,11 +22,12 @@
 //         D_KK = sum e k k^T,  D_KV = sum e k v^T          (128 x 128 each)
 //     Per 64-key tile: the scores S = K q on the tensor cores (M = 64 keys,
 //     N = 8: q is row 0 of an 8-row operand), read back by four warps, 16
-//     keys each; the weights e, rounded to bf16 once so that every sum uses
-//     the same values; then the compute warps scale the K tile's rows by e
-//     into A = (e o K)^T in shared memory (as an MN-major operand A has the
-//     K tile's own layout, so this is a row scaling, not a transpose) and
-//     sum ks and vs from the same rows on the CUDA cores; and the tensor
+//     keys each (the score warps), with the weights e, rounded to bf16 once
+//     so that every sum uses the same values; then eight scale warps scale
+//     the K tile's rows by e into A = (e o K)^T in shared memory (as an
+//     MN-major operand A has the K tile's own layout, so this is a row
+//     scaling, not a transpose) and sum ks and vs from the same rows on the
+//     CUDA cores, while the score warps take the next tile; and the tensor
 //     cores add [D_KK | D_KV] += A . [K | V] (N = 256: a stage's K and V
 //     tiles are one MN-major B operand).  The issuing warp spends tens of
 //     cycles per MMA, so the count matters as much as the size: twelve per
@@ -52,8 +53,9 @@ namespace plx {
 
 constexpr int kLlaD = 128;
 constexpr int kLlaStages = 5;            // K and V ring depth (tiles)
-constexpr int kLlaThreads = 320;         // TMA producer warp, MMA warp, eight compute warps
-constexpr int kLlaCompute = 256;
+constexpr int kLlaThreads = 448;         // TMA producer warp, MMA warp, four score warps, eight scale warps
+constexpr int kLlaScore = 128;           // score warps 2..5 (one per TMEM lane quarter)
+constexpr int kLlaScale = 256;           // scale warps 6..13 (two per TMEM lane quarter)
 constexpr int kLlaSplitLen = 1024;       // shorter sequences add the lo part of e o K
 constexpr float kLlaRescaleLog2 = 8.f;   // lazy rescale threshold (factor 256)
 constexpr int kLlaMaxPieces = 16;
@@ -94,11 +96,14 @@ struct LlaLayout {
   static constexpr int kQBytes = 8 * kLlaD * 2;               // bf16 [8][128]: row 0 = q, rows 1.. zero
   static constexpr int kQ = kA + 2 * kTileBytes;              // K-major B operand, two 64-column atoms
   static constexpr int kE = kQ + kQBytes;                     // float [2][64]: the tile's weights e
-  static constexpr int kRed = kE + 2 * kTile * 4;             // float [8 warps][2]
-  static constexpr int kBar = kRed + 64;
-  // full[S], empty[S], s_full[2], s_free[2], a_full[2], a_free[2], drain
-  // (the per-tile hand-offs alternate between two barriers by tile parity)
-  static constexpr int kNumBars = 2 * kLlaStages + 9;
+  // float [32]: [0, 4) the score warps' maxima, [4, 8) their sums of e,
+  // [8, 10) the rescale factor of the tile in e buffer 0 / 1
+  static constexpr int kRed = kE + 2 * kTile * 4;
+  static constexpr int kBar = kRed + 128;
+  // full[S], empty[S], s_full[2], s_free[2], e_full[2], e_free[2], a_full[2],
+  // a_free[2], drain (the per-tile hand-offs alternate between two barriers
+  // by tile parity)
+  static constexpr int kNumBars = 2 * kLlaStages + 13;
   static constexpr int kMisc = kBar + kNumBars * 8;           // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
@@ -178,7 +183,9 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   uint64_t* empty = full + S;
   uint64_t* s_full = empty + S;
   uint64_t* s_free = s_full + 2;
-  uint64_t* a_full = s_free + 2;
+  uint64_t* e_full = s_free + 2;
+  uint64_t* e_free = e_full + 2;
+  uint64_t* a_full = e_free + 2;
   uint64_t* a_free = a_full + 2;
   uint64_t* drain = a_free + 2;
   uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kMisc);
@@ -226,8 +233,10 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kLlaCompute);
-      mbar_init(&a_full[i], kLlaCompute);
+      mbar_init(&s_free[i], kLlaScore);
+      mbar_init(&e_full[i], kLlaScore);
+      mbar_init(&e_free[i], kLlaScale);
+      mbar_init(&a_full[i], kLlaScale);
       mbar_init(&a_free[i], 1);
     }
     mbar_init(drain, 1);
@@ -357,42 +366,32 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     __syncwarp();
     mbar_wait_drain(drain, 0);
     __syncwarp();
-  } else {
-    // ------------------------------------------------------------ compute
-    const int c = threadIdx.x - 64;            // 0..255
-    const int cw = warp - 2;                   // compute warp 0..7
-    const int kh = cw >> 2;                    // D half this warp rescales and writes (D_KK, D_KV)
-    const int wq = warp & 3;                   // TMEM lane quarter of this warp
-    const int row = wq * 32 + lane;            // TMEM lane = component a of k
-    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
-    // Score phase: warps with cw < 4 read the scores of keys 16 wq .. 16 wq + 15
-    // (TMEM lanes 32 wq .. 32 wq + 15 of the M = 64 product), one per lane.
-    const bool skey = cw < 4 && lane < 16;
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ score warps
+    // Warp 2 + i reads TMEM lane quarter wq = warp % 4: the scores of keys
+    // 16 wq .. 16 wq + 15 (lanes 32 wq .. 32 wq + 15 of the M = 64 product),
+    // one per lane.  Per tile t (buffers t % 2): the weights e, taken against
+    // the running max before the warps' one barrier, which also decides (a
+    // reduction) whether the running max moves: only when a score passes it
+    // by kLlaRescaleLog2, or on the first tile.  On that rare path the max
+    // is reduced and the weights are taken again.  The weights and the
+    // tile's rescale factor go to the scale warps (e_full).
+    const int c = threadIdx.x - 64;            // 0..127
+    const int wq = warp & 3;
+    const bool skey = lane < 16;
     const int key = 16 * wq + lane;
-    // Scale phase: thread c takes the 16-byte chunk cc = c % 16 of rows
-    // kg + 16 m (kg = c / 16, m = 0..3) of the K and V tiles: components
-    // 64 (cc / 8) + 8 (cc % 8) .. + 7.  A warp covers two whole rows.
-    const int cc = c & 15, kg = c >> 4;
-    const int coff = (cc >> 3) * (Ly::kTileBytes / 2);   // + row * 128 + swizzled chunk
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     float m_ref = -INFINITY, l_acc = 0.f;
-    float ks[8], vs[8];                        // sum e k, sum e v over this thread's rows, its 8 components
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ks[i] = vs[i] = 0.f;
-    // Tile t's scores and weights e (buffer t % 2).  The weights are taken
-    // against the running max before the tile's one barrier, which both
-    // publishes them and decides (a reduction) whether the running max
-    // moves: only when a score passes it by kLlaRescaleLog2, or on the first
-    // tile.  On that rare path the max is reduced, the weights are taken
-    // again, and alpha_d returns the factor that everything accumulated over
-    // tiles < t takes before tile t is added; D's rescale needs main(t - 1)
-    // done, so that path waits for it.  wv carries the wait for the A
-    // buffer of the scale phase that follows (false: it ran out).
-    auto scores_phase = [&](int t, float& alpha_d, bool wv) -> bool {
+    bool fine = true;
+    int t = 0;
+    for (; fine && t < n; ++t) {
       const int gb = t & 1;
-      const bool w = __all_sync(0xffffffffu, !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[gb], (t >> 1) & 1));
+      // the e buffer was read by the scale warps (tile t - 2)
+      const bool wf = t < 2 || mbar_wait_bounded(a.wait_ns, &e_free[gb], ((t >> 1) - 1) & 1);
+      const bool w = __all_sync(0xffffffffu, wf && !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[gb], (t >> 1) & 1));
       const int nvalid = min(kTile, len - (t0 + t) * kTile);
       float sc = -INFINITY;
-      if (w && cw < 4) {   // warp-uniform
+      if (w) {   // warp-uniform
         tc_fence_after();
         const uint32_t r = tmem_ld1(tmem + lane_off + lla_col_s(gb));
         tmem_wait_ld();
@@ -400,60 +399,94 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&s_free[gb]);   // S(t + 2) may overwrite the buffer
-      float* e_s = reinterpret_cast<float*>(sm + Ly::kE) + gb * kTile;
       // the weights, rounded to bf16: every sum and product uses these values
       auto weight = [&]() { return key < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f; };
-      float e = 0.f;
-      if (skey) {   // every key of the tile, its weight 0 past the end
-        e = weight();
-        e_s[key] = e;
-      }
+      float e = skey ? weight() : 0.f;
       if (nvalid < kTile) {
         // Rows past the end are operands of the products (their weights are
         // 0, but 0 * NaN is not): zero them in K and V.  S(t), the only
         // earlier reader of the tile, is done (s_full).
         uint8_t* st = sm + Ly::kKV + (t % S) * Ly::kStageBytes;
-        for (int i = c; i < (kTile - nvalid) * 16; i += kLlaCompute) {
+        for (int i = c; i < (kTile - nvalid) * 16; i += kLlaScore) {
           const int r = nvalid + (i >> 4), ci = i & 15;   // ci: box (ci >> 3), chunk (ci & 7)
           const int off = (ci >> 3) * (Ly::kTileBytes / 2) + r * 128 + (ci & 7) * 16;
           *reinterpret_cast<uint4*>(st + off) = make_uint4(0u, 0u, 0u, 0u);
           *reinterpret_cast<uint4*>(st + Ly::kTileBytes + off) = make_uint4(0u, 0u, 0u, 0u);
         }
+        fence_proxy_async_smem();   // the products read these rows
       }
-      alpha_d = 1.f;
-      if (bar_or(1, kLlaCompute, t == 0 || !w || !wv || sc > m_ref + kLlaRescaleLog2)) {   // uniform
-        if (!bar_and(2, kLlaCompute, w && wv)) return false;
+      float alpha = 1.f;
+      if (bar_or(1, kLlaScore, t == 0 || !w || sc > m_ref + kLlaRescaleLog2)) {   // uniform
+        if (!(fine = bar_and(2, kLlaScore, w))) break;
         const float wmax = warp_max(sc);
-        if (lane == 0) red_s[cw] = wmax;
-        bar_and(3, kLlaCompute, true);
-        const float tmax = fmaxf(fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3])),
-                                 fmaxf(fmaxf(red_s[4], red_s[5]), fmaxf(red_s[6], red_s[7])));
-        bool wd = true;
+        if (lane == 0) red_s[wq] = wmax;
+        bar_and(3, kLlaScore, true);
+        // (the next write of red_s[0..3] comes after the next tile's barrier)
+        const float tmax = fmaxf(fmaxf(red_s[0], red_s[1]), fmaxf(red_s[2], red_s[3]));
         if (t == 0) {
           m_ref = tmax;   // the piece's first tile holds a key: tmax is finite
-        } else if (tmax > m_ref + kLlaRescaleLog2) {   // uniform: every compute thread saw the same maxima
-          alpha_d = ex2(m_ref - tmax);
+        } else if (tmax > m_ref + kLlaRescaleLog2) {   // uniform: every score thread saw the same maxima
+          alpha = ex2(m_ref - tmax);
           m_ref = tmax;
-          l_acc *= alpha_d;
-          wd = mbar_wait_bounded(a.wait_ns, &a_free[(t - 1) & 1], ((t - 1) >> 1) & 1);   // main(t - 1) done
+          l_acc *= alpha;
         }
-        if (skey) {
-          e = weight();
-          e_s[key] = e;
-        }
-        if (!bar_and(2, kLlaCompute, wd)) return false;   // the new weights, visible to every compute thread
+        if (skey) e = weight();
       }
       l_acc += e;
-      return true;
-    };
-    // Tile t right after its scores: the deferred rescale of D, then
-    // A = (e o K)^T into its A buffer with sum e k and sum e v from the same
-    // rows; a_full.
-    auto scale_phase = [&](int t, float alpha_d, auto split_tag) {
+      if (skey) reinterpret_cast<float*>(sm + Ly::kE)[gb * kTile + key] = e;
+      if (c == 0) red_s[8 + gb] = alpha;
+      mbar_arrive(&e_full[gb]);
+    }
+    // the piece's l and m (combined with the scale warps' outcome below)
+    const float lw = warp_sum(l_acc);
+    if (lane == 0) red_s[4 + wq] = lw;
+    const bool ok = fine && t == n;
+    // ---- the piece's record (score side): wait for the scale warps' outcome
+    const bool rec_ok = bar_and(4, kLlaScore + kLlaScale, ok);
+    bar_and(5, kLlaScore + kLlaScale, true);   // the scale warps' partial sums are in place
+    if (c == 0) {
+      if (rec_ok) {
+        rec[kLlaRecM] = m_ref;
+        rec[kLlaRecM + 1] = (red_s[4] + red_s[5]) + (red_s[6] + red_s[7]);
+      } else {   // abandoned after a wait ran out (already reported): an empty record
+        rec[kLlaRecM] = -INFINITY;
+        rec[kLlaRecM + 1] = 0.f;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ scale warps
+    // Per tile t, once its weights are in (e_full): the deferred rescale of D
+    // (a new running max; main(t - 1) done), then A = (e o K)^T into its A
+    // buffer (main(t - 2) done; main(t - 1) when lo takes the second
+    // buffer), sum e k and sum e v from the same rows; a_full, e_free.
+    // Thread c takes the 16-byte chunk cc = c % 16 of rows kg + 16 m
+    // (kg = c / 16, m = 0..3) of the K and V tiles: components
+    // 64 (cc / 8) + 8 (cc % 8) .. + 7; a warp covers two whole rows.  For D,
+    // warp 6 + i takes TMEM lane quarter warp % 4 and half i / 4 (D_KK,
+    // D_KV).
+    const int c = threadIdx.x - 192;           // 0..255
+    const int kh = (warp - 6) >> 2;
+    const int wq = warp & 3;
+    const int row = wq * 32 + lane;            // TMEM lane = component a of k
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const int cc = c & 15, kg = c >> 4;
+    // row kg + 16 m has swizzle kg % 8
+    const int roff = (cc >> 3) * (Ly::kTileBytes / 2) + (((cc & 7) ^ (kg & 7)) << 4) + kg * 128;
+    float ks[8], vs[8];                        // sum e k, sum e v over this thread's rows, its 8 components
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ks[i] = vs[i] = 0.f;
+    auto scale = [&](int t, auto split_tag) -> bool {
       constexpr bool kSplit = decltype(split_tag)::value;
       const int gb = t & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, &e_full[gb], (t >> 1) & 1))) return false;
+      const float alpha = red_s[8 + gb];
+      const int jb = t - (kSplit ? 1 : 2);   // the products that last read the A buffers
+      bool wv = jb < 0 || mbar_wait_bounded(a.wait_ns, &a_free[jb & 1], (jb >> 1) & 1);
+      if (alpha != 1.f && !kSplit)   // uniform; D needs main(t - 1) done
+        wv = wv && mbar_wait_bounded(a.wait_ns, &a_free[(t - 1) & 1], ((t - 1) >> 1) & 1);
+      if (!__all_sync(0xffffffffu, wv)) return false;
       tc_fence_after();
-      if (alpha_d != 1.f) {   // uniform; main(t - 1) is done
+      if (alpha != 1.f) {
 #pragma unroll 1
         for (int part = 4 * kh; part < 4 * kh + 4; ++part) {   // D_KK (kh 0) or D_KV (kh 1), 32 columns at a time
           uint32_t r[32];
@@ -461,31 +494,34 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
           tmem_ld32(addr, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha_d);
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
           tmem_st32(addr, r);
         }
         tmem_wait_st();
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          ks[i] *= alpha_d;
-          vs[i] *= alpha_d;
+          ks[i] *= alpha;
+          vs[i] *= alpha;
         }
       }
       const float* et = reinterpret_cast<const float*>(sm + Ly::kE) + gb * kTile;
       const uint8_t* st = sm + Ly::kKV + (t % S) * Ly::kStageBytes;
       uint8_t* ah = sm + Ly::kA + (kSplit ? 0 : gb * Ly::kTileBytes);
       uint8_t* al = sm + Ly::kA + Ly::kTileBytes;
-      // row kg + 16 m has swizzle kg % 8
-      const int roff = coff + (((cc & 7) ^ (kg & 7)) << 4) + kg * 128;
       uint4 kw[4], vw[4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         kw[m] = *reinterpret_cast<const uint4*>(st + roff + m * 2048);
         vw[m] = *reinterpret_cast<const uint4*>(st + Ly::kTileBytes + roff + m * 2048);
       }
+      float ev[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) ev[m] = et[kg + 16 * m];
+      tc_fence_before();
+      mbar_arrive(&e_free[gb]);   // e and alpha of this tile are read
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        const float e = et[kg + 16 * m];
+        const float e = ev[m];
         const uint32_t kx[4] = {kw[m].x, kw[m].y, kw[m].z, kw[m].w};
         const uint32_t vx[4] = {vw[m].x, vw[m].y, vw[m].z, vw[m].w};
         uint32_t hi[4], lo[4];
@@ -506,26 +542,14 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(&a_full[gb]);
+      return true;
     };
-    // Before scores(t): the A buffers that scale(t) writes are free once
-    // main(t - 2) is done (main(t - 1) when lo takes the second buffer).
-    float alpha = 1.f;
     bool fine = true;
-    int j = 0;
-    for (; fine && j < n; ++j) {
-      const int jb = j - (split_lo ? 1 : 2);
-      const bool wv = jb < 0 || mbar_wait_bounded(a.wait_ns, &a_free[jb & 1], (jb >> 1) & 1);
-      if (!(fine = scores_phase(j, alpha, wv))) break;
-      if (split_lo)
-        scale_phase(j, alpha, std::true_type{});
-      else
-        scale_phase(j, alpha, std::false_type{});
-    }
-    // ---- the piece's record: wait for the last products, then write
-    bool wl = fine && j == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, &a_free[(n - 1) & 1], ((n - 1) >> 1) & 1);
-    wl = bar_and(3, kLlaCompute, wl);
-    const float lw = warp_sum(l_acc);
-    if (lane == 0) red_s[8 + cw] = lw;
+    int t = 0;
+    for (; fine && t < n; ++t) fine = split_lo ? scale(t, std::true_type{}) : scale(t, std::false_type{});
+    // ---- the piece's record (scale side): wait for the last products, then write
+    bool wl = fine && t == n && !*abort_flag && mbar_wait_bounded(a.wait_ns, &a_free[(n - 1) & 1], ((n - 1) >> 1) & 1);
+    wl = bar_and(4, kLlaScore + kLlaScale, wl);
     // the first moments' partial sums meet in the A buffers, idle once the
     // last products are done: [16 row groups][128] of sum e k, then of sum e v
     float* scr = reinterpret_cast<float*>(sm + Ly::kA);
@@ -538,7 +562,7 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       pv[0] = make_float4(vs[0], vs[1], vs[2], vs[3]);
       pv[1] = make_float4(vs[4], vs[5], vs[6], vs[7]);
     }
-    bar_and(2, kLlaCompute, true);
+    bar_and(5, kLlaScore + kLlaScale, true);
     if (wl) {
       tc_fence_after();
 #pragma unroll 1
@@ -552,23 +576,12 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
 #pragma unroll
         for (int i = 0; i < 32; ++i) dst[i * kLlaD] = __uint_as_float(r[i]);
       }
-      {
-        const int comp = c & (kLlaD - 1);
-        const float* src = scr + (c >= kLlaD ? 16 * kLlaD : 0) + comp;
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      const int comp = c & (kLlaD - 1);
+      const float* src = scr + (c >= kLlaD ? 16 * kLlaD : 0) + comp;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int g = 0; g < 16; ++g) s4[g & 3] += src[g * kLlaD];
-        rec[(c >= kLlaD ? kLlaRecVs : kLlaRecKs) + comp] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-      }
-      if (c == 0) {
-        float lt = 0.f;
-        for (int w = 0; w < 8; ++w) lt += red_s[8 + w];
-        rec[kLlaRecM] = m_ref;
-        rec[kLlaRecM + 1] = lt;
-      }
-    } else if (c == 0) {   // abandoned after a wait ran out (already reported): an empty record
-      rec[kLlaRecM] = -INFINITY;
-      rec[kLlaRecM + 1] = 0.f;
+      for (int g = 0; g < 16; ++g) s4[g & 3] += src[g * kLlaD];
+      rec[(c >= kLlaD ? kLlaRecVs : kLlaRecKs) + comp] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
     }
   }
   tc_fence_before();
