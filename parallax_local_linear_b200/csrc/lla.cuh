@@ -100,10 +100,10 @@ struct LlaLayout {
   // [8, 10) the rescale factor of the tile in e buffer 0 / 1
   static constexpr int kRed = kE + 2 * kTile * 4;
   static constexpr int kBar = kRed + 128;
-  // full[S], empty[S], s_full[2], s_free[2], e_full[2], e_free[2], a_full[2],
-  // a_free[2], drain (the per-tile hand-offs alternate between two barriers
-  // by tile parity)
-  static constexpr int kNumBars = 2 * kLlaStages + 13;
+  // full[S], empty[S], s_full[2], e_full[2], e_free[2], a_full[2], a_free[2],
+  // drain (the per-tile hand-offs alternate between two barriers by tile
+  // parity)
+  static constexpr int kNumBars = 2 * kLlaStages + 11;
   static constexpr int kMisc = kBar + kNumBars * 8;           // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
@@ -182,8 +182,7 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
   uint64_t* empty = full + S;
   uint64_t* s_full = empty + S;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* e_full = s_free + 2;
+  uint64_t* e_full = s_full + 2;
   uint64_t* e_free = e_full + 2;
   uint64_t* a_full = e_free + 2;
   uint64_t* a_free = a_full + 2;
@@ -233,7 +232,6 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], kLlaScore);
       mbar_init(&e_full[i], kLlaScore);
       mbar_init(&e_free[i], kLlaScale);
       mbar_init(&a_full[i], kLlaScale);
@@ -310,10 +308,12 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     auto wait_warp = [&](uint64_t* bar, uint32_t parity) {
       return __all_sync(0xffffffffu, mbar_wait_bounded(a.wait_ns, bar, parity));
     };
-    auto stage_off = [&](int j) { return (uint64_t)(((j % S) * Ly::kStageBytes) >> 4); };
+    constexpr uint64_t kStageU = Ly::kStageBytes >> 4, kRingU = S * kStageU;   // descriptor units (16 bytes)
+    uint64_t so_s = 0, so_m = 0;   // descriptor offsets of the stages of the next S and the next main
+    int st_s = 0, ph_s = 0, st_m = 0;
     // main(j): 16 keys per step, 16 rows (2048 bytes) of A and of [K | V].
     auto issue_main = [&](int jm) {
-      const uint64_t kv = dkvM + stage_off(jm);
+      const uint64_t kv = dkvM + so_m;
       const uint64_t ah = daM + (split_lo ? 0 : (uint64_t)(((jm & 1) * Ly::kTileBytes) >> 4));
       lla_mma4_ss(tmem + kLlaColKK, ah, kv, ah + 128, kv + 128, ah + 256, kv + 256, ah + 384, kv + 384, kIdD,
                   jm > 0 ? 1u : 0u);
@@ -322,41 +322,44 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         lla_mma4_ss(tmem + kLlaColKK, al, kv, al + 128, kv + 128, al + 256, kv + 256, al + 384, kv + 384, kIdD, 1u);
       }
       tc_commit(&a_free[jm & 1]);
-      tc_commit(&empty[jm % S]);
+      tc_commit(&empty[st_m]);
+      so_m = so_m + kStageU == kRingU ? 0 : so_m + kStageU;
+      if (++st_m == S) st_m = 0;
     };
     // S(js) once tile js has landed; 16 components per step: box kk / 4, 32
     // bytes into the 128-byte row.
     auto issue_s = [&](int js) {
-      const uint64_t ka = dkS + stage_off(js);
+      const uint64_t ka = dkS + so_s;
       constexpr uint64_t kBoxA = Ly::kTileBytes / 2 / 16, kBoxB = Ly::kQBytes / 2 / 16;
       const uint32_t d = tmem + lla_col_s(js & 1);
       lla_mma4_ss(d, ka, dqS, ka + 2, dqS + 2, ka + 4, dqS + 4, ka + 6, dqS + 6, kIdS, 0u);
       lla_mma4_ss(d, ka + kBoxA, dqS + kBoxB, ka + kBoxA + 2, dqS + kBoxB + 2, ka + kBoxA + 4, dqS + kBoxB + 4,
                   ka + kBoxA + 6, dqS + kBoxB + 6, kIdS, 1u);
       tc_commit(&s_full[js & 1]);
+      so_s = so_s + kStageU == kRingU ? 0 : so_s + kStageU;
+      if (++st_s == S) {
+        st_s = 0;
+        ph_s ^= 1;
+      }
     };
-    // Issue order S(0), S(1), then per tile j: S(j + 2) (once the scores of
-    // tile j, in the same TMEM buffer, have been read), main(j).  The scores
-    // run two tiles ahead of the products, so the compute warps find them
-    // done.
+    // Issue order S(0), S(1), then per tile j, once A(j) is written: S(j + 2)
+    // (the scores of tile j, in the same TMEM buffer, have been read), main(j).
+    // The scores run two tiles ahead of the products.
     bool ok = true;
     for (int js = 0; ok && js < 2 && js < n; ++js) {
-      if (!(ok = wait_warp(&full[js % S], (js / S) & 1))) break;
+      if (!(ok = wait_warp(&full[st_s], ph_s))) break;
       tc_fence_after();
       issue_s(js);
     }
-    for (int j = 0; ok && j < n; ++j) {
-      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
-        ok = false;
-        break;
-      }
+    for (int j = 0; ok && j < n; ++j) {   // a role that gave up leaves a wait here to run out
+      // a_full(j) also means the scores of tile j were read (the score
+      // warps handed tile j's weights to the scale warps after reading them)
+      if (!(ok = wait_warp(&a_full[j & 1], (j >> 1) & 1))) break;
       if (j + 2 < n) {
-        if (!(ok = wait_warp(&s_free[j & 1], (j >> 1) & 1))) break;
-        if (!(ok = wait_warp(&full[(j + 2) % S], ((j + 2) / S) & 1))) break;
+        if (!(ok = wait_warp(&full[st_s], ph_s))) break;
         tc_fence_after();
         issue_s(j + 2);
       }
-      if (!(ok = wait_warp(&a_full[j & 1], (j >> 1) & 1))) break;
       tc_fence_after();
       issue_main(j);
     }
@@ -397,8 +400,7 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         tmem_wait_ld();
         if (skey && key < nvalid) sc = __uint_as_float(r) * a.scale_log2;
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[gb]);   // S(t + 2) may overwrite the buffer
+      tc_fence_before();   // S(t + 2) overwrites the buffer after a_full(t)
       // the weights, rounded to bf16: every sum and product uses these values
       auto weight = [&]() { return key < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f; };
       float e = skey ? weight() : 0.f;
