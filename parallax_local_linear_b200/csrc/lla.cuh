@@ -593,26 +593,40 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
 }
 
 // ---------------------------------------------------------------- solve
-// One CTA (256 threads) per (sequence, query head).  Thread (bi, bj) of a
-// 16 x 16 grid holds the 8 x 8 block of S_KK + ridge I at rows 8 bi..,
-// columns 8 bj.. in registers (blocks on or below the diagonal; the others
-// idle in the factorisation).  Blocked right-looking Cholesky, 8 columns per
-// step: 16 steps of two barriers each.  The factor goes to shared memory for
-// the two triangular solves, which one warp runs with the vector in
-// registers.
-constexpr int kLlaSolveThreads = 256;
-constexpr int kLlaLd = kLlaD + 1;   // padded row stride of the factor in shared memory
+// One CTA per (sequence, query head).  Thread (bi, bj) of a 16 x 16 grid
+// holds the 8 x 8 block of S_KK + ridge I at rows 8 bi.., columns 8 bj.. in
+// registers (blocks on or below the diagonal; the others idle in the
+// factorisation); a 17th block row (threads 256..271) holds b = kbar - q as
+// its first row, so that the factorisation of [S; b^T] leaves z = L^-1 b in
+// it (the forward substitution rides along).  Blocked right-looking
+// Cholesky, 8 columns per step: 16 steps of two barriers each; the factor
+// goes to shared memory transposed (row k of L^T contiguous), so that the
+// rank-8 updates read it as float4.  The back substitution L^T rho = z is
+// blocked too: 16 steps, each a diagonal 8 x 8 solve and the blocks of one
+// row of L updating the rest of the vector, with every block still in its
+// thread's registers.  D_KV comes into shared memory by cp.async while the
+// factorisation runs.
+constexpr int kLlaSolveThreads = 288;            // 256 matrix blocks, 16 for the b row, 16 spare
+constexpr int kLlaLt = kLlaD + 8 + 4;            // row stride of L^T: 136 entries (b row included) + 4 of padding
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaArgs a) {
   extern __shared__ float smf[];
-  float* Lm = smf;                         // [128][129]: column k of the factor, rows >= k
-  float* kb = Lm + kLlaD * kLlaLd;         // kbar
+  float* Dkv = smf;                        // [128 columns][128]: D_KV of piece 0, column-major as recorded
+  float* Lt = Dkv + kLlaD * kLlaD;         // [128][kLlaLt]: Lt[k * kLlaLt + i] = L[i][k], i = 128: z
+  float* kb = Lt + kLlaD * kLlaLt;         // kbar
   float* vb = kb + kLlaD;                  // vbar
   float* rho_s = vb + kLlaD;               // rho*
-  float* invp = rho_s + kLlaD;             // 1 / L[k][k]
-  float* part = invp + kLlaD;              // [8][128] partial matrix-vector products
-  float* wts = part + 8 * kLlaD;           // [kLlaMaxPieces] piece weights 2^(m_j - M)
-  float* misc = wts + kLlaMaxPieces;       // [0] l, [1] kbar . rho*
+  float* r_s = rho_s + kLlaD;              // the back substitution's right-hand side (z, updated)
+  float* inv_s = r_s + kLlaD;              // 1 / L[k][k]
+  float* part = inv_s + kLlaD;             // [128] D_KV^T rho*
+  float* wts = part + kLlaD;               // [kLlaMaxPieces] piece weights 2^(m_j - M)
+  float* misc = wts + kLlaMaxPieces;       // [0] l, [1] kbar . rho*, [2] non-positive pivot flag
 
   const int tid = threadIdx.x;
   const int bh = blockIdx.x, b = bh / a.Hq;
@@ -632,6 +646,11 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     return;
   }
   const float* rec0 = a.rec + (size_t)bh * a.pieces * kLlaRecFloats;
+  {   // D_KV of piece 0 into shared memory, in the background
+    const float* src = rec0 + kLlaRecKV;
+    for (int i = tid; i < kLlaD * kLlaD / 4; i += kLlaSolveThreads) cp_async16(Dkv + 4 * i, src + 4 * i);
+    cp_async_commit();
+  }
   if (tid == 0) {
     float M = -INFINITY;
     for (int p = 0; p < a.pieces; ++p) {
@@ -646,6 +665,7 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
       L += w * r[kLlaRecM + 1];
     }
     misc[0] = L;
+    misc[2] = 0.f;
   }
   __syncthreads();
   const float invL = 1.f / misc[0];
@@ -663,14 +683,15 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
   __syncthreads();
 
   // ---- this thread's block of S_KK + ridge I = D_KK / l - kbar kbar^T + ridge I
+  // (block row 16: row 0 of the block is b = kbar - q, the rest zero)
   const int bi = tid >> 4, bj = tid & 15, r0 = 8 * bi, c0 = 8 * bj;
-  const bool active = bi >= bj;
+  const bool active = bi < 16 ? bi >= bj : bi == 16;
   float blk[8][8];
 #pragma unroll
   for (int r = 0; r < 8; ++r)
 #pragma unroll
     for (int c = 0; c < 8; ++c) blk[r][c] = 0.f;
-  if (active) {
+  if (bi < 16 && active) {
     for (int p = 0; p < a.pieces; ++p) {
       if (wts[p] == 0.f) continue;
       // column c0 + c of the block: rows r0 .. r0 + 7 are contiguous
@@ -699,14 +720,15 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
 #pragma unroll
       for (int c = 0; c < 8; ++c)
         blk[r][c] = fmaf(blk[r][c], invL, -kb[r0 + r] * kb[c0 + c]) + (r0 + r == c0 + c ? a.ridge : 0.f);
+  } else if (active) {   // the b row
+#pragma unroll
+    for (int c = 0; c < 8; ++c) blk[0][c] = kb[c0 + c] - __bfloat162float(a.q[orow + c0 + c]);
   }
 
   // ---- blocked Cholesky, one panel of 8 columns per step P: the diagonal
-  // block's owner factors it in registers; the blocks below it solve
-  // against that factor (X L_PP^T = A); the blocks right of the panel and
-  // on or below the diagonal take the rank-8 update.  Lm ends up holding L.
-  int* flag_s = reinterpret_cast<int*>(misc + 2);
-  if (tid == 0) *flag_s = 0;
+  // block's owner factors it in registers; the blocks below it (the b row
+  // included) solve against that factor (X L_PP^T = A); the blocks right of
+  // the panel and on or below the diagonal take the rank-8 update.
   bool bad = false;
 #pragma unroll 1
   for (int P = 0; P < 16; ++P) {
@@ -718,7 +740,7 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
         ok = ok && akk > 0.f && isfinite(akk);
         const float invd = rsqrtf(akk);
         blk[k][k] = akk * invd;
-        invp[8 * P + k] = invd;
+        inv_s[8 * P + k] = invd;
 #pragma unroll
         for (int i = k + 1; i < 8; ++i) blk[i][k] *= invd;
 #pragma unroll
@@ -726,44 +748,46 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
 #pragma unroll
           for (int jj = k + 1; jj <= i; ++jj) blk[i][jj] = fmaf(-blk[i][k], blk[jj][k], blk[i][jj]);
       }
-      if (!ok) *flag_s = 1;
+      if (!ok) misc[2] = 1.f;
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
+      for (int c = 0; c < 8; ++c)
 #pragma unroll
-        for (int c = 0; c <= r; ++c) Lm[(r0 + r) * kLlaLd + c0 + c] = blk[r][c];
+        for (int r = c; r < 8; ++r) Lt[(c0 + c) * kLlaLt + r0 + r] = blk[r][c];
     }
     __syncthreads();
-    if (*flag_s != 0) {   // not numerically positive definite (uniform)
+    if (misc[2] != 0.f) {   // not numerically positive definite (uniform)
       bad = true;
       break;
     }
-    if (bj == P && bi > P) {   // the panel: X L_PP^T = A, column by column
-      const float* lpp = Lm + (8 * P) * kLlaLd + 8 * P;
+    if (active && bj == P && bi > P) {   // the panel: X L_PP^T = A, column by column
+      const float* lpp = Lt + (8 * P) * kLlaLt + 8 * P;   // lpp[m * kLlaLt + c] = L_PP[c][m]
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float invd = invp[8 * P + c];
+        const float invd = inv_s[8 * P + c];
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
           float x = blk[r][c];
 #pragma unroll
-          for (int m = 0; m < c; ++m) x = fmaf(-blk[r][m], lpp[c * kLlaLd + m], x);
+          for (int m = 0; m < c; ++m) x = fmaf(-blk[r][m], lpp[m * kLlaLt + c], x);
           blk[r][c] = x * invd;
         }
       }
 #pragma unroll
-      for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) Lm[(r0 + r) * kLlaLd + c0 + c] = blk[r][c];
+      for (int c = 0; c < 8; ++c) {
+        float4* dst = reinterpret_cast<float4*>(Lt + (c0 + c) * kLlaLt + r0);
+        dst[0] = make_float4(blk[0][c], blk[1][c], blk[2][c], blk[3][c]);
+        dst[1] = make_float4(blk[4][c], blk[5][c], blk[6][c], blk[7][c]);
+      }
     }
     __syncthreads();
     if (active && bj > P) {   // rank-8 update of the trailing blocks
 #pragma unroll
       for (int m = 0; m < 8; ++m) {
-        float li[8], lj[8];
-#pragma unroll
-        for (int r = 0; r < 8; ++r) li[r] = Lm[(r0 + r) * kLlaLd + 8 * P + m];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) lj[c] = Lm[(c0 + c) * kLlaLd + 8 * P + m];
+        const float* lk = Lt + (8 * P + m) * kLlaLt;   // column 8 P + m of L
+        const float4 i0 = *reinterpret_cast<const float4*>(lk + r0), i1 = *reinterpret_cast<const float4*>(lk + r0 + 4);
+        const float4 j0 = *reinterpret_cast<const float4*>(lk + c0), j1 = *reinterpret_cast<const float4*>(lk + c0 + 4);
+        const float li[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+        const float lj[8] = {j0.x, j0.y, j0.z, j0.w, j1.x, j1.y, j1.z, j1.w};
 #pragma unroll
         for (int r = 0; r < 8; ++r)
 #pragma unroll
@@ -771,8 +795,8 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
       }
     }
   }
-  __syncthreads();
   if (bad) {
+    cp_async_wait_all();
     if (tid == 0) report_error(PLX_DEVERR_SINGULAR_BIT);
     if (tid < kLlaD) {   // rho* = 0: the output falls back to vbar
       store_out(tid, vb[tid]);
@@ -780,57 +804,55 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     }
     return;
   }
-  // ---- L z = kbar - q, then L^T rho = z: one warp, rows lane + 32u in registers
-  if (tid < 32) {
-    const int lane = tid;
-    float yv[4];
+  // ---- L^T rho = z, blockwise from the last block: the diagonal block's
+  // owner solves L_II^T rho_I = r_I; the owners of row I of L then take
+  // L_IJ^T rho_I off r_J (J < I).
+  if (bi == 16 && bj < 16) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) yv[u] = kb[lane + 32 * u] - __bfloat162float(a.q[orow + lane + 32 * u]);
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-#pragma unroll 1
-      for (int kk = 0; kk < 32; ++kk) {
-        const int k = 32 * u + kk;
-        const float zk = __shfl_sync(0xffffffffu, yv[u], kk) * invp[k];
-        if (lane == kk) yv[u] = zk;
-#pragma unroll
-        for (int v = u; v < 4; ++v) {
-          const int i = lane + 32 * v;
-          if (i > k) yv[v] = fmaf(-Lm[i * kLlaLd + k], zk, yv[v]);
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 3; u >= 0; --u) {
-#pragma unroll 1
-      for (int kk = 31; kk >= 0; --kk) {
-        const int k = 32 * u + kk;
-        const float xk = __shfl_sync(0xffffffffu, yv[u], kk) * invp[k];
-        if (lane == kk) yv[u] = xk;
-#pragma unroll
-        for (int v = 0; v <= u; ++v) {
-          const int jj = lane + 32 * v;
-          if (jj < k) yv[v] = fmaf(-Lm[k * kLlaLd + jj], xk, yv[v]);
-        }
-      }
-    }
-    float kr = 0.f;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      rho_s[lane + 32 * u] = yv[u];
-      kr = fmaf(kb[lane + 32 * u], yv[u], kr);
-    }
-    kr = warp_sum(kr);
-    if (lane == 0) misc[1] = kr;
+    for (int c = 0; c < 8; ++c) r_s[c0 + c] = blk[0][c];   // z
   }
   __syncthreads();
+#pragma unroll 1
+  for (int I = 15; I >= 0; --I) {
+    if (bi == I && bj == I) {
+      float x[8];
+#pragma unroll
+      for (int c = 7; c >= 0; --c) {
+        float v = r_s[8 * I + c];
+#pragma unroll
+        for (int rr = c + 1; rr < 8; ++rr) v = fmaf(-blk[rr][c], x[rr], v);
+        x[c] = v * inv_s[8 * I + c];
+        rho_s[8 * I + c] = x[c];
+      }
+    }
+    __syncthreads();
+    if (bi == I && bj < I) {
+      float x[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) x[r] = rho_s[8 * I + r];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float t = 0.f;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) t = fmaf(blk[r][c], x[r], t);
+        r_s[c0 + c] -= t;
+      }
+    }
+    __syncthreads();
+  }
+  if (tid < 32) {
+    float kr = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) kr = fmaf(kb[tid + 32 * u], rho_s[tid + 32 * u], kr);
+    kr = warp_sum(kr);
+    if (tid == 0) misc[1] = kr;
+  }
+  cp_async_wait_all();
+  __syncthreads();
   // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a
-  {
+  if (tid < 2 * kLlaD) {
     const int col = tid >> 1, half = tid & 1;   // rows a = 64 half .. 64 half + 63 of column col
-    float acc = 0.f;
-    for (int p = 0; p < a.pieces; ++p) {
-      if (wts[p] == 0.f) continue;
-      const float* dkv = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + col * kLlaD + 64 * half;
+    auto column_dot = [&](const float* dkv) {
       float4 v[16];
 #pragma unroll
       for (int u = 0; u < 16; ++u) v[u] = *reinterpret_cast<const float4*>(dkv + 4 * u);
@@ -840,7 +862,12 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
         const float* rr = rho_s + 64 * half + 4 * u;
         sp = fmaf(v[u].x, rr[0], fmaf(v[u].y, rr[1], fmaf(v[u].z, rr[2], fmaf(v[u].w, rr[3], sp))));
       }
-      acc = fmaf(wts[p], sp, acc);
+      return sp;
+    };
+    float acc = wts[0] == 0.f ? 0.f : wts[0] * column_dot(Dkv + col * kLlaD + 64 * half);
+    for (int p = 1; p < a.pieces; ++p) {
+      if (wts[p] == 0.f) continue;
+      acc = fmaf(wts[p], column_dot(rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + col * kLlaD + 64 * half), acc);
     }
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     if (half == 0) part[col] = acc;
@@ -854,7 +881,7 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
 }
 
 constexpr int lla_solve_smem_bytes() {
-  return (kLlaD * kLlaLd + 4 * kLlaD + 8 * kLlaD + kLlaMaxPieces + 4) * 4;
+  return (kLlaD * kLlaD + kLlaD * kLlaLt + 6 * kLlaD + kLlaMaxPieces + 4) * 4;
 }
 
 }  // namespace plx
