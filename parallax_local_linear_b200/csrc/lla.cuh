@@ -761,15 +761,21 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     }
     if (active && bj == P && bi > P) {   // the panel: X L_PP^T = A, column by column
       const float* lpp = Lt + (8 * P) * kLlaLt + 8 * P;   // lpp[m * kLlaLt + c] = L_PP[c][m]
+      float lp[8][8], invd[8];   // L_PP below the diagonal and 1 / L_PP[c][c], loaded before the chain
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        const float invd = inv_s[8 * P + c];
+        invd[c] = inv_s[8 * P + c];
+#pragma unroll
+        for (int m = 0; m < c; ++m) lp[c][m] = lpp[m * kLlaLt + c];
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
           float x = blk[r][c];
 #pragma unroll
-          for (int m = 0; m < c; ++m) x = fmaf(-blk[r][m], lpp[m * kLlaLt + c], x);
-          blk[r][c] = x * invd;
+          for (int m = 0; m < c; ++m) x = fmaf(-blk[r][m], lp[c][m], x);
+          blk[r][c] = x * invd[c];
         }
       }
 #pragma unroll
@@ -787,11 +793,16 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
         const float4 i0 = *reinterpret_cast<const float4*>(lk + r0), i1 = *reinterpret_cast<const float4*>(lk + r0 + 4);
         const float4 j0 = *reinterpret_cast<const float4*>(lk + c0), j1 = *reinterpret_cast<const float4*>(lk + c0 + 4);
         const float li[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-        const float lj[8] = {j0.x, j0.y, j0.z, j0.w, j1.x, j1.y, j1.z, j1.w};
+        const float2 lj[4] = {make_float2(j0.x, j0.y), make_float2(j0.z, j0.w), make_float2(j1.x, j1.y),
+                              make_float2(j1.z, j1.w)};
 #pragma unroll
         for (int r = 0; r < 8; ++r)
 #pragma unroll
-          for (int c = 0; c < 8; ++c) blk[r][c] = fmaf(-li[r], lj[c], blk[r][c]);
+          for (int h = 0; h < 4; ++h) {   // packed pairs of columns
+            const float2 t = fma2(make_float2(-li[r], -li[r]), lj[h], make_float2(blk[r][2 * h], blk[r][2 * h + 1]));
+            blk[r][2 * h] = t.x;
+            blk[r][2 * h + 1] = t.y;
+          }
       }
     }
   }
@@ -849,28 +860,26 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
   }
   cp_async_wait_all();
   __syncthreads();
-  // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a
-  if (tid < 2 * kLlaD) {
-    const int col = tid >> 1, half = tid & 1;   // rows a = 64 half .. 64 half + 63 of column col
-    auto column_dot = [&](const float* dkv) {
-      float4 v[16];
-#pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = *reinterpret_cast<const float4*>(dkv + 4 * u);
-      float sp = 0.f;
-#pragma unroll
-      for (int u = 0; u < 16; ++u) {
-        const float* rr = rho_s + 64 * half + 4 * u;
-        sp = fmaf(v[u].x, rr[0], fmaf(v[u].y, rr[1], fmaf(v[u].z, rr[2], fmaf(v[u].w, rr[3], sp))));
-      }
-      return sp;
+  // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a: warp w
+  // takes columns 16 w .. 16 w + 15, lane l rows 4 l .. 4 l + 3 of each (a
+  // column of D_KV is 512 contiguous bytes)
+  if (tid < 8 * 32) {
+    const int wid = tid >> 5, lane = tid & 31;
+    const float4 rr = *reinterpret_cast<const float4*>(rho_s + 4 * lane);
+    auto dot4 = [&](const float* p4) {
+      const float4 v = *reinterpret_cast<const float4*>(p4);
+      return fmaf(v.x, rr.x, fmaf(v.y, rr.y, fmaf(v.z, rr.z, v.w * rr.w)));
     };
-    float acc = wts[0] == 0.f ? 0.f : wts[0] * column_dot(Dkv + col * kLlaD + 64 * half);
-    for (int p = 1; p < a.pieces; ++p) {
-      if (wts[p] == 0.f) continue;
-      acc = fmaf(wts[p], column_dot(rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + col * kLlaD + 64 * half), acc);
+#pragma unroll 4
+    for (int k = 0; k < 16; ++k) {
+      const int col = 16 * wid + k;
+      float acc = wts[0] == 0.f ? 0.f : wts[0] * dot4(Dkv + col * kLlaD + 4 * lane);
+      for (int p = 1; p < a.pieces; ++p)
+        if (wts[p] != 0.f)
+          acc = fmaf(wts[p], dot4(rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + col * kLlaD + 4 * lane), acc);
+      acc = warp_sum(acc);
+      if (lane == 0) part[col] = acc;
     }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    if (half == 0) part[col] = acc;
   }
   __syncthreads();
   if (tid < kLlaD) {
