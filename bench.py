@@ -365,10 +365,11 @@ def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
     """End to end through the public API: each step copies the step's q and
     rho from pinned host memory, runs the decode and reads the output back.
     The headline figure is one call per step of a prepared decode
-    (DecodePlan.run_io: both copies in, the launch and the copy out, queued
-    by the library; the plan is made once per buffer set, as a serving loop
-    with fixed buffers would); the one-shot decode() call with torch copies
-    around it is timed the same way beside it."""
+    (DecodePlan.run_io: one launch that reads q and rho from pinned host
+    memory and writes the output there; the plan is made once per buffer
+    set, as a serving loop with fixed buffers would);
+    the one-shot decode() call with torch copies around it is timed the same
+    way beside it."""
     copies = len(insts)
     host = []
     for x in insts:
@@ -421,8 +422,8 @@ def e2e_decode(px, insts, outs, args, w, dev, bytes_per_step, world):
             "host_wall_ms_per_step": round(wall, 6), "api": "DecodePlan.run_io (parallax_decode_plan_run_io)",
             "one_shot_call": {"value": round(gbs_call, 2), "ms_per_step": round(ms_call, 6),
                               "host_wall_ms_per_step": round(wall_call, 6), "api": "decode (parallax_decode)"},
-            "note": "query and probe copied from pinned host memory and output read back every step; "
-                    "the KV cache stays resident on the device"}
+            "note": "every step the kernel reads the query and probe from pinned host memory and writes "
+                    "the output into pinned host memory, across PCIe; the KV cache stays resident on the device"}
 
 
 def bench_decode_projected(args, w, rank, world, dev, peaks, peaks_kind):

@@ -158,13 +158,18 @@ plx_status parallax_decode_plan_create(const void* q, const void* rho,
                                       const plx_decode_params* p, plx_decode_plan** plan);
 plx_status parallax_decode_plan_run(const plx_decode_plan* plan, cudaStream_t stream);
 
-/* One serving step from host memory: on `stream`, copies host_q and
- * host_rho ([B, Hq, d] of in_dtype) into the plan's q and rho buffers, runs
- * the decode, and copies the plan's out buffer into host_out ([B, Hq, d] of
- * out_dtype); three copies and one launch, all asynchronous (the host
- * buffers must be page-locked for the copies to overlap other work, and
- * must stay valid until the stream reaches them).  Errors as
- * parallax_decode_plan_run; PLX_ERR_INVALID_ARG for a null host pointer. */
+/* One serving step from host memory: host_q and host_rho ([B, Hq, d] of
+ * in_dtype) in, host_out ([B, Hq, d] of out_dtype) out, on `stream`,
+ * asynchronous; the host buffers must stay valid (and host_out unread)
+ * until the stream reaches the step.  When all three are page-locked and
+ * mapped into the device's address space (cudaHostAlloc / pinned memory
+ * under unified addressing, 16-byte aligned), the one launch reads q and rho
+ * and writes the output across PCIe directly, and the plan's own q, rho and
+ * out buffers are not touched.  Otherwise it copies host_q and host_rho into
+ * the plan's q and rho, runs the decode and copies the plan's out into
+ * host_out: three copies and one launch (page-locked buffers let the copies
+ * overlap other work).  Errors as parallax_decode_plan_run;
+ * PLX_ERR_INVALID_ARG for a null host pointer. */
 plx_status parallax_decode_plan_run_io(const plx_decode_plan* plan, const void* host_q, const void* host_rho,
                                       void* host_out, cudaStream_t stream);
 void parallax_decode_plan_destroy(plx_decode_plan* plan);

@@ -355,10 +355,12 @@ class DecodePlan:
         return self.out
 
     def run_io(self, host_q, host_rho, host_out):
-        """One step from host memory: copies ``host_q`` and ``host_rho`` in,
-        runs the decode and copies the output into ``host_out``, all queued
-        on the current stream (host tensors: contiguous, pinned, shaped and
-        typed like q / out)."""
+        """One step from host memory on the current stream: ``host_q`` and
+        ``host_rho`` in, the decode, the output into ``host_out`` (host
+        tensors: contiguous, shaped and typed like q / out).  When all three
+        are pinned the kernel reads and writes them across PCIe itself;
+        otherwise they go through copies into and out of the plan's
+        buffers."""
         q, rho = self._keep[0], self._keep[1]
         for name, t, like in (("host_q", host_q, q), ("host_rho", host_rho, rho), ("host_out", host_out, self.out)):
             if t.is_cuda or not t.is_contiguous() or t.dtype != like.dtype or tuple(t.shape) != tuple(like.shape):

@@ -465,20 +465,24 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
           qa[kk][3] = live ? __ldg(rrow + c1) : 0u;
         }
       }
-      float aref = 0.f;
+      // a_ref of head hr from the rho pairs this thread already holds (the
+      // quad of lanes 4 hr .. 4 hr + 3 covers all D columns) and k_0
+      float aref;
       {
-        const __nv_bfloat16* k0 = reinterpret_cast<const __nv_bfloat16*>(a.k) + cache_row(a, b, kvh, 0) * D;
-        float kv[D / 32];
+        const uint32_t* k0 =
+            reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(a.k) + cache_row(a, b, kvh, 0) * D);
+        float part = 0.f;
 #pragma unroll
-        for (int j = 0; j < D / 32; ++j) kv[j] = __bfloat162float(k0[lane + 32 * j]);
-        for (int h = 0; h < g; ++h) {
-          const __nv_bfloat16* rh = reinterpret_cast<const __nv_bfloat16*>(a.rho) + ((size_t)b * a.Hq + hq0 + h) * D;
-          float acc = 0.f;
-#pragma unroll
-          for (int j = 0; j < D / 32; ++j) acc += __bfloat162float(rh[lane + 32 * j]) * kv[j];
-          acc = warp_sum(acc);
-          if (hr == h) aref = acc;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t k_lo = __ldg(k0 + (16 * kk + qc) / 2), k_hi = __ldg(k0 + (16 * kk + 8 + qc) / 2);
+          part = fmaf(bf16_lo_f(qa[kk][1]), bf16_lo_f(k_lo), part);
+          part = fmaf(bf16_hi_f(qa[kk][1]), bf16_hi_f(k_lo), part);
+          part = fmaf(bf16_lo_f(qa[kk][3]), bf16_lo_f(k_hi), part);
+          part = fmaf(bf16_hi_f(qa[kk][3]), bf16_hi_f(k_hi), part);
         }
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        aref = part;   // 0 for rows past the group (their fragments are zero)
       }
 
       float o[D / 8][4];

@@ -711,6 +711,26 @@ plx_status parallax_decode_plan_run_io(const plx_decode_plan* plan, const void* 
   const size_t heads = (size_t)p.batch * p.num_q_heads * p.head_dim;
   const size_t in_bytes = heads * (p.in_dtype == PLX_BF16 ? 2 : 4);
   const size_t out_bytes = heads * (p.out_dtype == PLX_BF16 ? 2 : 4);
+  // Page-locked host buffers mapped into the device's address space (pinned
+  // memory under unified addressing): the kernel reads q, rho and writes the
+  // output across PCIe itself, with no copy operations around it.
+  auto mapped = [](const void* h, void** dptr) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, h) != cudaSuccess) {
+      cudaGetLastError();   // an unregistered pointer is an answer here, not an error
+      return false;
+    }
+    *dptr = at.devicePointer;
+    return at.type == cudaMemoryTypeHost && *dptr != nullptr && aligned(*dptr, 16);
+  };
+  void *dq = nullptr, *dr = nullptr, *dout = nullptr;
+  if (mapped(host_q, &dq) && mapped(host_rho, &dr) && mapped(host_out, &dout)) {
+    DecodeLaunch L = plan->L;
+    L.a.q = dq;
+    L.a.rho = dr;
+    L.a.out = dout;
+    return launch_decode(L, &plan->p, stream, false, false);
+  }
   const DecodeArgs& a = plan->L.a;
   if (note(cudaMemcpyAsync(const_cast<void*>(a.q), host_q, in_bytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
       note(cudaMemcpyAsync(const_cast<void*>(a.rho), host_rho, in_bytes, cudaMemcpyHostToDevice, stream)) !=

@@ -78,8 +78,9 @@ def test_plan_in_a_cuda_graph(px):
 
 
 def test_plan_step_from_host_memory(px):
-    # run_io: q and rho copied in from pinned host memory, the decode, the
-    # output copied back, on one stream: the result equals the device-side run.
+    # run_io: q and rho read by the kernel from pinned host memory, the
+    # decode, the output written straight into pinned host memory: the result
+    # equals the device-side run.
     inp = _cuda(W.small_decode_inputs(8, 16, 8, 128, 1024, seed=64))
     dq, dr = torch.empty_like(inp["q"]), torch.empty_like(inp["rho"])
     out = torch.empty_like(inp["q"])
@@ -90,5 +91,11 @@ def test_plan_step_from_host_memory(px):
     torch.cuda.synchronize()
     ref = px.decode(inp["q"], inp["rho"], inp["k_cache"], inp["v_cache"], inp["scale"])
     assert torch.equal(hout, ref.cpu())
+    # a pageable buffer takes the copy path through the plan's buffers
+    hout2 = torch.zeros(out.shape, dtype=out.dtype)
+    plan.run_io(inp["q"].cpu(), inp["rho"].cpu(), hout2)
+    torch.cuda.synchronize()
+    assert torch.equal(hout2, ref.cpu())
+    assert torch.equal(out.cpu(), ref.cpu())
     with pytest.raises(ValueError):
         plan.run_io(inp["q"], hr, hout)   # a device tensor where a host one belongs
