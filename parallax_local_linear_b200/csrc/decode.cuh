@@ -53,6 +53,9 @@ struct DecodeArgs {
   float scale_log2;                // scale * log2(e)
   int out_bf16;
   int cluster;                     // > 1: each unit is one cluster of this many CTAs (bf16 path)
+  int pdl_all;                     // 1: launched with a programmatic dependency on the previous
+                                   // kernel, which any input may come from: every thread waits for it
+                                   // before touching global memory (bf16 path)
   unsigned long long wait_ns;      // limit of one pipeline wait (0: give up unless complete)
 };
 
@@ -358,7 +361,30 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = a.group;
-  build_tile_space(a, pre, lens, scan);
+  // The next kernel in the stream may start once every CTA of this grid has
+  // got here; a decode launched after this one with a programmatic
+  // dependency then has its launch and set-up done by the time this grid
+  // ends, and waits below for this grid's results.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // Set-up that reads no global memory runs before the wait: the tile space
+  // when every sequence has kv_len tokens, the ring's barriers, the tensor
+  // maps' prefetch.
+  if (a.seq_lens == nullptr) build_tile_space(a, pre, lens, scan);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    s_flag[0] = 0;
+    s_flag[1] = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == NC && lane == 0) {
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_v);
+  }
+  if (a.pdl_all) asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (a.seq_lens != nullptr) build_tile_space(a, pre, lens, scan);
 
   // Sequences of length zero have no tiles: CTA b % gridDim.x writes their zeros.
   for (int b = blockIdx.x; b < a.B; b += gridDim.x)
@@ -371,16 +397,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
   TileSpace ts{pre, lens, a.B, a.units_per_seq, T, G};
   const long long x0 = ts.start(blockIdx.x), x1 = ts.start(blockIdx.x + 1);
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    s_flag[0] = 0;
-    s_flag[1] = 0;
-    fence_mbarrier_init();
-  }
-  __syncthreads();
+  __syncthreads();   // the barriers' initialisation is visible
   if (a.cluster > 1) cluster_arrive_relaxed();
   volatile int* abort_flag = s_flag + 1;
   const int nchunk = (int)(x1 - x0);
@@ -388,8 +405,6 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
   if (warp == NC) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tmap(&tmap_k);
-      prefetch_tmap(&tmap_v);
       const uint64_t pol = l2_policy_evict_first();
       UnitCursor cur;
       cur.seek(ts, x0);

@@ -196,17 +196,27 @@ size_t decode_smem_bytes(const plx_decode_params* p) {
          table;
 }
 
-// `pdl`: launch with a programmatic dependency on the previous kernel in the
-// stream, which may then still be running when this grid starts (the
-// consumers wait for it before reading q and rho).
+// How a decode grid depends on the kernel before it in the stream:
+//   kPdlNone      plain stream order;
+//   kPdlQR        programmatic: the previous kernel produces q and rho only
+//                 (the projection), so the producer streams K and V at once
+//                 and the consumers wait before reading q and rho;
+//   kPdlAll       programmatic: any input may come from the previous kernel,
+//                 so every thread waits before touching global memory; only
+//                 the launch and the CTAs' start overlap the previous grid's
+//                 tail.
+enum PdlMode { kPdlNone = 0, kPdlQR = 1, kPdlAll = 2 };
+
 template <int D, int STAGES, bool kLoInPad>
-plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CUtensorMap& tv, int ctas,
-                            size_t smem, cudaStream_t stream, bool pdl, bool set_attr) {
+plx_status launch_decode_tc(const DecodeArgs& args, const CUtensorMap& tk, const CUtensorMap& tv, int ctas,
+                            size_t smem, cudaStream_t stream, PdlMode pdl, bool set_attr) {
   auto kern = decode_tc_kernel<D, STAGES, kDecodeNC, kLoInPad>;
   if (set_attr &&
       set_smem(kern, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
-  if (a.cluster <= 1 && !pdl) {
+  DecodeArgs a = args;
+  a.pdl_all = pdl == kPdlAll ? 1 : 0;
+  if (a.cluster <= 1 && pdl == kPdlNone) {
     kern<<<ctas, (kDecodeNC + 1) * 32, smem, stream>>>(tk, tv, a);
     return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
   }
@@ -217,7 +227,7 @@ plx_status launch_decode_tc(const DecodeArgs& a, const CUtensorMap& tk, const CU
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
   int n = 0;
-  if (pdl) {
+  if (pdl != kPdlNone) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
@@ -334,7 +344,7 @@ plx_status prepare_decode(const void* q, const void* rho, const void* k_cache, c
 
 // `set_attr`: set the kernel's dynamic shared-memory limit first (a prepared
 // plan did that once when it was made).
-plx_status launch_decode(const DecodeLaunch& L, const plx_decode_params* p, cudaStream_t stream, bool pdl,
+plx_status launch_decode(const DecodeLaunch& L, const plx_decode_params* p, cudaStream_t stream, PdlMode pdl,
                          bool set_attr = true) {
   const DecodeArgs& a = L.a;
   const int D = p->head_dim;
@@ -669,7 +679,7 @@ plx_status parallax_decode(const void* q, const void* rho, const void* k_cache, 
   const plx_status st =
       prepare_decode(q, rho, k_cache, v_cache, page_table, seq_lens, out, workspace, workspace_bytes, p, &L);
   if (st != PLX_OK) return st;
-  return launch_decode(L, p, stream, false);
+  return launch_decode(L, p, stream, kPdlAll);
 }
 
 plx_status parallax_decode_plan_create(const void* q, const void* rho, const void* k_cache, const void* v_cache,
@@ -698,7 +708,7 @@ plx_status parallax_decode_plan_run(const plx_decode_plan* plan, cudaStream_t st
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return PLX_ERR_CUDA;
   if (dev != plan->device) return PLX_ERR_INVALID_ARG;
-  return launch_decode(plan->L, &plan->p, stream, false, false);
+  return launch_decode(plan->L, &plan->p, stream, kPdlAll, false);
 }
 
 plx_status parallax_decode_plan_run_io(const plx_decode_plan* plan, const void* host_q, const void* host_rho,
@@ -729,14 +739,14 @@ plx_status parallax_decode_plan_run_io(const plx_decode_plan* plan, const void* 
     L.a.q = dq;
     L.a.rho = dr;
     L.a.out = dout;
-    return launch_decode(L, &plan->p, stream, false, false);
+    return launch_decode(L, &plan->p, stream, kPdlAll, false);
   }
   const DecodeArgs& a = plan->L.a;
   if (note(cudaMemcpyAsync(const_cast<void*>(a.q), host_q, in_bytes, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
       note(cudaMemcpyAsync(const_cast<void*>(a.rho), host_rho, in_bytes, cudaMemcpyHostToDevice, stream)) !=
           cudaSuccess)
     return PLX_ERR_CUDA;
-  const plx_status st = launch_decode(plan->L, &plan->p, stream, false, false);
+  const plx_status st = launch_decode(plan->L, &plan->p, stream, kPdlAll, false);
   if (st != PLX_OK) return st;
   return note(cudaMemcpyAsync(host_out, a.out, out_bytes, cudaMemcpyDeviceToHost, stream)) == cudaSuccess
              ? PLX_OK
@@ -781,7 +791,7 @@ plx_status parallax_decode_projected(const void* x, const void* w_q, const void*
   pa.n1 = (int)n1;
   pa.hidden = hidden;
   if ((st = launch_project(pa, stream)) != PLX_OK) return st;
-  return launch_decode(L, p, stream, true);
+  return launch_decode(L, p, stream, kPdlQR);
 }
 
 plx_status parallax_prefill(const void* q, const void* rho, const void* k, const void* v, void* out,
@@ -883,7 +893,7 @@ plx_status parallax_decode_noalloc(const void* q, const void* rho, const void* k
     return st;
   // The counters must start at zero; the array keeps whatever the last call left.
   if (cudaMemsetAsync(scratch, 0, L.pl.counter_bytes, stream) != cudaSuccess) return PLX_ERR_CUDA;
-  return launch_decode(L, p, stream, false);
+  return launch_decode(L, p, stream, kPdlAll);
 }
 
 plx_status parallax_set_wait_limit_ns(uint64_t limit_ns, uint64_t* previous) {
