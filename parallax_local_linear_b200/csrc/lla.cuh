@@ -93,13 +93,16 @@ struct LlaLayout {
   // scaled by e_i, in bf16.  Two buffers: hi of tile t in buffer t % 2; below
   // kLlaSplitLen keys hi in buffer 0 and lo = x - hi in buffer 1.
   static constexpr int kA = kKV + kLlaStages * kStageBytes;
-  static constexpr int kQBytes = 8 * kLlaD * 2;               // bf16 [8][128]: row 0 = q, rows 1.. zero
+  // The score product's B operand, bf16 [16][64], K-major, 128-byte swizzle:
+  // row 0 = q[0:64], row 8 = q[64:128], the rest zero.
+  static constexpr int kQBytes = 16 * 64 * 2;
   static constexpr int kQ = kA + 2 * kTileBytes;              // K-major B operand, two 64-column atoms
   static constexpr int kE = kQ + kQBytes;                     // float [2][64]: the tile's weights e
   // float [32]: [0, 4) the score warps' maxima, [4, 8) their sums of e,
   // [8, 10) the rescale factor of the tile in e buffer 0 / 1
   static constexpr int kRed = kE + 2 * kTile * 4;
-  static constexpr int kBar = kRed + 128;
+  static constexpr int kPart = kRed + 128;                    // float [64]: the second half of each score
+  static constexpr int kBar = kPart + 256;
   // full[S], empty[S], s_full[2], e_full[2], e_free[2], a_full[2], a_free[2],
   // drain (the per-tile hand-offs alternate between two barriers by tile
   // parity)
@@ -108,10 +111,11 @@ struct LlaLayout {
   static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
 
-// TMEM columns: D = [D_KK | D_KV] in [0, 256); the scores of tile j at
-// 256 + 8 (j % 2) (M = 64: key r in lane (r % 16) + 32 (r / 16), column 0).
+// TMEM columns: D = [D_KK | D_KV] in [0, 256); the score product of tile j
+// at 256 + 16 (j % 2): key r's score is lane r, column 0 (components 0..63)
+// plus lane 64 + r, column 8 (components 64..127).
 constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128;
-__device__ __forceinline__ uint32_t lla_col_s(int buf) { return 256u + 8u * buf; }
+__device__ __forceinline__ uint32_t lla_col_s(int buf) { return 256u + 16u * buf; }
 
 // Four MMAs into one accumulator under one elect.sync (four k-steps): the
 // first takes the accumulate flag acc0, the others accumulate.
@@ -196,6 +200,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   const int bh = blockIdx.x / a.pieces;
   const int b = bh / a.Hq, h = bh % a.Hq, kvh = h / a.group;
   float* rec = a.rec + (size_t)blockIdx.x * kLlaRecFloats;
+  // Launched with a programmatic dependency on the kernel before it, which
+  // any input may come from: wait for it before touching global memory; let
+  // the next kernel (the solve) launch as soon as every CTA is here.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int len = lla_seq_len(a, b);
   const int tiles = (len + kTile - 1) / kTile;
   const int t0 = (int)((long long)piece * tiles / a.pieces);
@@ -242,8 +251,8 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     fence_mbarrier_init();
   }
   if (threadIdx.x < Ly::kQBytes / 16) {
-    // 16-byte chunk i of the q operand: atom i / 64 (components 64 (i / 64) ..),
-    // row (i / 8) % 8, chunk i % 8; row 0 is not swizzled and holds q
+    // 16-byte chunk i of the q operand: rows 8 (i / 64) + (i / 8) % 8, chunk
+    // i % 8; rows 0 and 8 (unswizzled) hold components 64 (i / 64) + 8 (i % 8) ..
     const int i = threadIdx.x;
     alignas(16) __nv_bfloat16 v[8];
 #pragma unroll
@@ -294,12 +303,14 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per tile: the scores S = K q (M = 64 keys, N = 8, K-major A and B) and,
+    // Per tile: the scores S = K q (M = 128: the K tile's two 64-column boxes
+    // stacked, so rows r and 64 + r hold key r's two halves; N = 16: q's
+    // halves in B rows 0 and 8; K-major A and B) and,
     // once the compute warps have written A = (e o K)^T, the products
     // [D_KK | D_KV] += A . [K | V] (SS, 128 x 256, A and the stage's K and V
     // tiles as MN-major operands).  Twelve MMAs per tile (sixteen below
     // kLlaSplitLen keys), four under each elect.
-    constexpr uint32_t kIdS = idesc_bf16_ab(kTile, 8, false, false);
+    constexpr uint32_t kIdS = idesc_bf16_ab(128, 16, false, false);
     constexpr uint32_t kIdD = idesc_bf16_ab(128, 2 * kLlaD, true, true);
     const uint64_t dkS = smem_desc_sw128(smem_u32(sm + Ly::kKV), 16, 1024);                  // K, K-major A
     const uint64_t dqS = smem_desc_sw128(smem_u32(sm + Ly::kQ), 16, 1024);                   // q, K-major B
@@ -326,15 +337,12 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       so_m = so_m + kStageU == kRingU ? 0 : so_m + kStageU;
       if (++st_m == S) st_m = 0;
     };
-    // S(js) once tile js has landed; 16 components per step: box kk / 4, 32
-    // bytes into the 128-byte row.
+    // S(js) once tile js has landed: 16 components of each half per step,
+    // 32 bytes into the 128-byte rows.
     auto issue_s = [&](int js) {
       const uint64_t ka = dkS + so_s;
-      constexpr uint64_t kBoxA = Ly::kTileBytes / 2 / 16, kBoxB = Ly::kQBytes / 2 / 16;
       const uint32_t d = tmem + lla_col_s(js & 1);
       lla_mma4_ss(d, ka, dqS, ka + 2, dqS + 2, ka + 4, dqS + 4, ka + 6, dqS + 6, kIdS, 0u);
-      lla_mma4_ss(d, ka + kBoxA, dqS + kBoxB, ka + kBoxA + 2, dqS + kBoxB + 2, ka + kBoxA + 4, dqS + kBoxB + 4,
-                  ka + kBoxA + 6, dqS + kBoxB + 6, kIdS, 1u);
       tc_commit(&s_full[js & 1]);
       so_s = so_s + kStageU == kRingU ? 0 : so_s + kStageU;
       if (++st_s == S) {
@@ -342,9 +350,10 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
         ph_s ^= 1;
       }
     };
-    // Issue order S(0), S(1), then per tile j, once A(j) is written: S(j + 2)
-    // (the scores of tile j, in the same TMEM buffer, have been read), main(j).
-    // The scores run two tiles ahead of the products.
+    // Issue order S(0), S(1), then per tile j, once A(j) is written: main(j),
+    // then S(j + 2) once its tile has landed (the scores of tile j, in the
+    // same TMEM buffer, have been read by then).  The scores run two tiles
+    // ahead of the products.
     bool ok = true;
     for (int js = 0; ok && js < 2 && js < n; ++js) {
       if (!(ok = wait_warp(&full[st_s], ph_s))) break;
@@ -355,13 +364,13 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       // a_full(j) also means the scores of tile j were read (the score
       // warps handed tile j's weights to the scale warps after reading them)
       if (!(ok = wait_warp(&a_full[j & 1], (j >> 1) & 1))) break;
+      tc_fence_after();
+      issue_main(j);   // first: tile j + 2 may not have landed yet
       if (j + 2 < n) {
         if (!(ok = wait_warp(&full[st_s], ph_s))) break;
         tc_fence_after();
         issue_s(j + 2);
       }
-      tc_fence_after();
-      issue_main(j);
     }
     if (!ok && lane == 0) *abort_flag = 1;
     // Every issued MMA must complete before tensor memory is released.
@@ -371,9 +380,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     __syncwarp();
   } else if (warp < 6) {
     // ------------------------------------------------------------ score warps
-    // Warp 2 + i reads TMEM lane quarter wq = warp % 4: the scores of keys
-    // 16 wq .. 16 wq + 15 (lanes 32 wq .. 32 wq + 15 of the M = 64 product),
-    // one per lane.  Per tile t (buffers t % 2): the weights e, taken against
+    // Warp 2 + i reads TMEM lane quarter wq = warp % 4: quarters 0 and 1 hold
+    // the first halves of the scores of keys 0..63 (column 0), quarters 2 and
+    // 3 the second halves (column 8), which they pass on through shared
+    // memory; the warps of quarters 0 and 1 then own one key per lane.  Per
+    // tile t (buffers t % 2): the weights e, taken against
     // the running max before the warps' one barrier, which also decides (a
     // reduction) whether the running max moves: only when a score passes it
     // by kLlaRescaleLog2, or on the first tile.  On that rare path the max
@@ -381,8 +392,9 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     // tile's rescale factor go to the scale warps (e_full).
     const int c = threadIdx.x - 64;            // 0..127
     const int wq = warp & 3;
-    const bool skey = lane < 16;
-    const int key = 16 * wq + lane;
+    const bool skey = wq < 2;
+    const int key = 32 * (wq & 1) + lane;
+    float* part_s = reinterpret_cast<float*>(sm + Ly::kPart);
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     float m_ref = -INFINITY, l_acc = 0.f;
     bool fine = true;
@@ -394,13 +406,16 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       const bool w = __all_sync(0xffffffffu, wf && !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[gb], (t >> 1) & 1));
       const int nvalid = min(kTile, len - (t0 + t) * kTile);
       float sc = -INFINITY;
+      float half = 0.f;
       if (w) {   // warp-uniform
         tc_fence_after();
-        const uint32_t r = tmem_ld1(tmem + lane_off + lla_col_s(gb));
+        half = __uint_as_float(tmem_ld1(tmem + lane_off + lla_col_s(gb) + (skey ? 0u : 8u)));
         tmem_wait_ld();
-        if (skey && key < nvalid) sc = __uint_as_float(r) * a.scale_log2;
       }
       tc_fence_before();   // S(t + 2) overwrites the buffer after a_full(t)
+      if (!skey) part_s[key] = half;
+      asm volatile("bar.sync 6, %0;" ::"n"(kLlaScore) : "memory");
+      if (w && skey && key < nvalid) sc = (half + part_s[key]) * a.scale_log2;
       // the weights, rounded to bf16: every sum and product uses these values
       auto weight = [&]() { return key < nvalid ? __bfloat162float(__float2bfloat16_rn(ex2(sc - m_ref))) : 0.f; };
       float e = skey ? weight() : 0.f;
@@ -631,6 +646,10 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
   const int tid = threadIdx.x;
   const int bh = blockIdx.x, b = bh / a.Hq;
   const size_t orow = (size_t)bh * kLlaD;
+  // Launched with a programmatic dependency on the moments grid: the records
+  // are read only after it has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int len = lla_seq_len(a, b);
   auto store_out = [&](int i, float v) {
     if (a.out_bf16)

@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <new>
+#include <utility>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -194,6 +195,25 @@ size_t decode_smem_bytes(const plx_decode_params* p) {
   return (p->head_dim == 64 ? tc_smem_fixed_bytes<64, kDecodeStages64, kDecodeNC>()
                             : tc_smem_fixed_bytes<128, kDecodeStages128, kDecodeNC>()) +
          table;
+}
+
+// Launch with a programmatic dependency on the previous kernel in the stream
+// (the kernel waits for it with griddepcontrol.wait before reading its
+// inputs; its launch and its CTAs' start overlap the previous grid's tail).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return note(cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...));
 }
 
 // How a decode grid depends on the kernel before it in the stream:
@@ -969,14 +989,16 @@ plx_status parallax_lla_decode(const void* q, const void* k_cache, const void* v
     constexpr int smem = LlaLayout::kBytes;
     if (set_smem(lla_moments_kernel, smem) != cudaSuccess)
       return PLX_ERR_CUDA;
-    lla_moments_kernel<<<(unsigned)(heads * pieces), kLlaThreads, smem, stream>>>(tk, tv, a);
-    if (note(cudaGetLastError()) != cudaSuccess) return PLX_ERR_CUDA;
+    if (launch_pdl(lla_moments_kernel, dim3((unsigned)(heads * pieces)), dim3(kLlaThreads), smem, stream, tk, tv, a) !=
+        cudaSuccess)
+      return PLX_ERR_CUDA;
   }
   constexpr int ssmem = lla_solve_smem_bytes();
   if (set_smem(lla_solve_kernel, ssmem) != cudaSuccess)
     return PLX_ERR_CUDA;
-  lla_solve_kernel<<<(unsigned)heads, kLlaSolveThreads, ssmem, stream>>>(a);
-  return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return launch_pdl(lla_solve_kernel, dim3((unsigned)heads), dim3(kLlaSolveThreads), ssmem, stream, a) == cudaSuccess
+             ? PLX_OK
+             : PLX_ERR_CUDA;
 }
 
 int32_t parallax_last_cuda_error(void) {
