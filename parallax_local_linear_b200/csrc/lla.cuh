@@ -103,16 +103,16 @@ struct LlaLayout {
   static constexpr int kRed = kE + 2 * kTile * 4;
   static constexpr int kPart = kRed + 128;                    // float [64]: the second half of each score
   static constexpr int kBar = kPart + 256;
-  // full[S], empty[S], s_full[2], e_full[2], e_free[2], a_full[2], a_free[2],
-  // drain (the per-tile hand-offs alternate between two barriers by tile
-  // parity)
-  static constexpr int kNumBars = 2 * kLlaStages + 11;
+  // full[S], empty[S], s_full[3], e_full[2], e_free[2], a_full[2], a_free[2],
+  // drain (the per-tile hand-offs rotate through two or three barriers by
+  // tile index)
+  static constexpr int kNumBars = 2 * kLlaStages + 12;
   static constexpr int kMisc = kBar + kNumBars * 8;           // tmem base, abort flag
   static constexpr int kBytes = kMisc + 16 + 1024;            // + alignment slack
 };
 
 // TMEM columns: D = [D_KK | D_KV] in [0, 256); the score product of tile j
-// at 256 + 16 (j % 2): key r's score is lane r, column 0 (components 0..63)
+// at 256 + 16 (j % 3): key r's score is lane r, column 0 (components 0..63)
 // plus lane 64 + r, column 8 (components 64..127).
 constexpr uint32_t kLlaColKK = 0, kLlaColKV = 128;
 __device__ __forceinline__ uint32_t lla_col_s(int buf) { return 256u + 16u * buf; }
@@ -186,7 +186,7 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(sm + Ly::kBar);
   uint64_t* empty = full + S;
   uint64_t* s_full = empty + S;
-  uint64_t* e_full = s_full + 2;
+  uint64_t* e_full = s_full + 3;
   uint64_t* e_free = e_full + 2;
   uint64_t* a_full = e_free + 2;
   uint64_t* a_free = a_full + 2;
@@ -240,12 +240,12 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       mbar_init(&empty[s], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
       mbar_init(&e_full[i], kLlaScore);
       mbar_init(&e_free[i], kLlaScale);
       mbar_init(&a_full[i], kLlaScale);
       mbar_init(&a_free[i], 1);
     }
+    for (int i = 0; i < 3; ++i) mbar_init(&s_full[i], 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -341,21 +341,21 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     // 32 bytes into the 128-byte rows.
     auto issue_s = [&](int js) {
       const uint64_t ka = dkS + so_s;
-      const uint32_t d = tmem + lla_col_s(js & 1);
+      const uint32_t d = tmem + lla_col_s(js % 3);
       lla_mma4_ss(d, ka, dqS, ka + 2, dqS + 2, ka + 4, dqS + 4, ka + 6, dqS + 6, kIdS, 0u);
-      tc_commit(&s_full[js & 1]);
+      tc_commit(&s_full[js % 3]);
       so_s = so_s + kStageU == kRingU ? 0 : so_s + kStageU;
       if (++st_s == S) {
         st_s = 0;
         ph_s ^= 1;
       }
     };
-    // Issue order S(0), S(1), then per tile j, once A(j) is written: main(j),
-    // then S(j + 2) once its tile has landed (the scores of tile j, in the
-    // same TMEM buffer, have been read by then).  The scores run two tiles
-    // ahead of the products.
+    // Issue order S(0), S(1), S(2), then per tile j, once A(j) is written:
+    // main(j), then S(j + 3) once its tile has landed (the scores of tile j,
+    // in the same TMEM buffer, have been read by then).  The scores run three
+    // tiles ahead of the products.
     bool ok = true;
-    for (int js = 0; ok && js < 2 && js < n; ++js) {
+    for (int js = 0; ok && js < 3 && js < n; ++js) {
       if (!(ok = wait_warp(&full[st_s], ph_s))) break;
       tc_fence_after();
       issue_s(js);
@@ -365,11 +365,11 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       // warps handed tile j's weights to the scale warps after reading them)
       if (!(ok = wait_warp(&a_full[j & 1], (j >> 1) & 1))) break;
       tc_fence_after();
-      issue_main(j);   // first: tile j + 2 may not have landed yet
-      if (j + 2 < n) {
+      issue_main(j);   // first: tile j + 3 may not have landed yet
+      if (j + 3 < n) {
         if (!(ok = wait_warp(&full[st_s], ph_s))) break;
         tc_fence_after();
-        issue_s(j + 2);
+        issue_s(j + 3);
       }
     }
     if (!ok && lane == 0) *abort_flag = 1;
@@ -403,16 +403,17 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       const int gb = t & 1;
       // the e buffer was read by the scale warps (tile t - 2)
       const bool wf = t < 2 || mbar_wait_bounded(a.wait_ns, &e_free[gb], ((t >> 1) - 1) & 1);
-      const bool w = __all_sync(0xffffffffu, wf && !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[gb], (t >> 1) & 1));
+      const int sb = t % 3;   // score buffer
+      const bool w = __all_sync(0xffffffffu, wf && !*abort_flag && mbar_wait_bounded(a.wait_ns, &s_full[sb], (t / 3) & 1));
       const int nvalid = min(kTile, len - (t0 + t) * kTile);
       float sc = -INFINITY;
       float half = 0.f;
       if (w) {   // warp-uniform
         tc_fence_after();
-        half = __uint_as_float(tmem_ld1(tmem + lane_off + lla_col_s(gb) + (skey ? 0u : 8u)));
+        half = __uint_as_float(tmem_ld1(tmem + lane_off + lla_col_s(sb) + (skey ? 0u : 8u)));
         tmem_wait_ld();
       }
-      tc_fence_before();   // S(t + 2) overwrites the buffer after a_full(t)
+      tc_fence_before();   // S(t + 3) overwrites the buffer after a_full(t)
       if (!skey) part_s[key] = half;
       asm volatile("bar.sync 6, %0;" ::"n"(kLlaScore) : "memory");
       if (w && skey && key < nvalid) sc = (half + part_s[key]) * a.scale_log2;
