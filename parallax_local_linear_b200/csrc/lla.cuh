@@ -96,7 +96,7 @@ struct LlaLayout {
   // The score product's B operand, bf16 [16][64], K-major, 128-byte swizzle:
   // row 0 = q[0:64], row 8 = q[64:128], the rest zero.
   static constexpr int kQBytes = 16 * 64 * 2;
-  static constexpr int kQ = kA + 2 * kTileBytes;              // K-major B operand, two 64-column atoms
+  static constexpr int kQ = kA + 2 * kTileBytes;
   static constexpr int kE = kQ + kQBytes;                     // float [2][64]: the tile's weights e
   // float [32]: [0, 4) the score warps' maxima, [4, 8) their sums of e,
   // [8, 10) the rescale factor of the tile in e buffer 0 / 1
