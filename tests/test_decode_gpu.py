@@ -273,3 +273,34 @@ def test_unit_aligned_grid_and_cluster_merge(px, B, Hq, Hkv, L):
     again = _run(px, inp, out_dtype=torch.float32)
     assert torch.equal(out, again)
     assert px.last_device_error() == 0
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_chained_calls_read_the_previous_output(px, paged):
+    # Consecutive decodes on one stream are launched with a programmatic
+    # dependency: the second may start before the first ends, and must wait
+    # for it before reading its inputs.  Here the second call's q and rho are
+    # the first call's output, written by the kernel just before; the chain
+    # runs with no host synchronisation in between and must equal the same
+    # two calls separated by a device synchronisation.
+    inp = _to(W.small_decode_inputs(8, 16, 8, 128, 2048, dtype="bf16", paged=paged, seed=81))
+    inp2 = _to(W.small_decode_inputs(8, 16, 8, 128, 2048, dtype="bf16", paged=paged, seed=82))
+    kw = dict(seq_lens=inp2.get("seq_lens"), page_table=inp2.get("page_table"))
+    out1 = _run(px, inp)
+    out2 = px.decode(out1, out1, inp2["k_cache"], inp2["v_cache"], inp2["scale"], **kw)
+    out3 = torch.empty_like(out2)
+    for _ in range(3):   # a few more links, still without synchronising
+        px.decode(out2, out1, inp2["k_cache"], inp2["v_cache"], inp2["scale"], out=out3, **kw)
+        px.decode(out3, out1, inp2["k_cache"], inp2["v_cache"], inp2["scale"], out=out2, **kw)
+    torch.cuda.synchronize()
+    ref1 = _run(px, inp)
+    torch.cuda.synchronize()
+    ref2 = px.decode(ref1, ref1, inp2["k_cache"], inp2["v_cache"], inp2["scale"], **kw)
+    torch.cuda.synchronize()
+    for _ in range(3):
+        ref3 = px.decode(ref2, ref1, inp2["k_cache"], inp2["v_cache"], inp2["scale"], **kw)
+        torch.cuda.synchronize()
+        ref2 = px.decode(ref3, ref1, inp2["k_cache"], inp2["v_cache"], inp2["scale"], **kw)
+        torch.cuda.synchronize()
+    assert torch.equal(out1, ref1)
+    assert torch.equal(out2, ref2)

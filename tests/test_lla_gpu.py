@@ -145,3 +145,22 @@ def test_decode_after_lla_is_unaffected(px):
     out = px.decode(inp["q"], inp["q"], inp["k_cache"], inp["v_cache"], inp["scale"], out_dtype=torch.float32)
     ref = oracle_heads(dict(inp, rho=inp["q"]), [(0, 0), (0, 1)])
     assert_parity(out.cpu().numpy(), ref, TOL_BF16, "decode after LLA")
+
+
+def test_chained_calls_read_the_previous_output(px):
+    # The moments and solve grids, and consecutive calls, are chained by a
+    # programmatic dependency: a call whose q is the previous call's output
+    # (written by its solve just before) must see that output.
+    inp = _cuda(W.small_decode_inputs(4, 8, 4, 128, 2048, seed=91))
+    out1, _ = px.lla_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["scale"], 0.05)
+    out2, rho2 = px.lla_decode(out1, inp["k_cache"], inp["v_cache"], inp["scale"], 0.05)
+    out3, _ = px.lla_decode(out2, inp["k_cache"], inp["v_cache"], inp["scale"], 0.05)
+    torch.cuda.synchronize()
+    ref1, _ = px.lla_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["scale"], 0.05)
+    torch.cuda.synchronize()
+    ref2, rref2 = px.lla_decode(ref1, inp["k_cache"], inp["v_cache"], inp["scale"], 0.05)
+    torch.cuda.synchronize()
+    ref3, _ = px.lla_decode(ref2, inp["k_cache"], inp["v_cache"], inp["scale"], 0.05)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, ref1) and torch.equal(out2, ref2) and torch.equal(out3, ref3)
+    assert torch.equal(rho2, rref2)
