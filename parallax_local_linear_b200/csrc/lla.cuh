@@ -609,21 +609,37 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
 }
 
 // ---------------------------------------------------------------- solve
-// One CTA per (sequence, query head).  Thread (bi, bj) of a 16 x 16 grid
-// holds the 8 x 8 block of S_KK + ridge I at rows 8 bi.., columns 8 bj.. in
-// registers (blocks on or below the diagonal; the others idle in the
-// factorisation); a 17th block row (threads 256..271) holds b = kbar - q as
-// its first row, so that the factorisation of [S; b^T] leaves z = L^-1 b in
-// it (the forward substitution rides along).  Blocked right-looking
-// Cholesky, 8 columns per step: 16 steps of two barriers each; the factor
-// goes to shared memory transposed (row k of L^T contiguous), so that the
-// rank-8 updates read it as float4.  The back substitution L^T rho = z is
-// blocked too: 16 steps, each a diagonal 8 x 8 solve and the blocks of one
-// row of L updating the rest of the vector, with every block still in its
-// thread's registers.  D_KV comes into shared memory by cp.async while the
-// factorisation runs.
-constexpr int kLlaSolveThreads = 288;            // 256 matrix blocks, 16 for the b row, 16 spare
-constexpr int kLlaLt = kLlaD + 8 + 4;            // row stride of L^T: 136 entries (b row included) + 4 of padding
+// One CTA per (sequence, query head): four row warps, row a in TMEM lane a.
+// S = S_KK + ridge I (fp32) lives in tensor memory, row a in lane a.  Blocked
+// right-looking Cholesky, 8 columns per panel: every row thread reads its 8
+// panel entries; the diagonal block goes through shared memory and each
+// thread factors it redundantly (no further synchronisation), solves its own
+// row against it and carries the forward substitution z = L^-1 (kbar - q)
+// along; the trailing update S -= L_P L_P^T runs on the tensor cores, with
+// each panel value split into three bf16 parts (hi + mid + lo carries the
+// fp32 value) and six products (hi hi, hi mid, mid hi, hi lo, lo hi, mid
+// mid) of a 128 x 128 x 16 MMA with A negated, issued by the first warp once
+// a named barrier says the panel is written.  The factor also goes to shared
+// memory, transposed, for the blocked back substitution L^T rho = z, whose
+// diagonal blocks are inverted all at once (one column per thread) first.
+// D_KV comes into shared memory by cp.async while the factorisation runs.
+constexpr int kLlaSolveThreads = 128;
+constexpr int kLlaLt = kLlaD + 4;                // row stride of L^T (padding against bank conflicts)
+
+struct LlaSolveLayout {
+  static constexpr int kDkv = 0;                              // float [128][128]: D_KV of piece 0
+  static constexpr int kLt = kDkv + kLlaD * kLlaD * 4;        // float [128][kLlaLt]: L^T
+  static constexpr int kOpBytes = kLlaD * 128;                // bf16 [128][64], 128-byte swizzle (16 columns used)
+  static constexpr int kOp = (kLt + kLlaD * kLlaLt * 4 + 1023) & ~1023;   // three parts: hi, mid, lo
+  static constexpr int kD8 = kOp + 3 * kOpBytes;              // float [8][8] diagonal block + [8] its z rhs
+  static constexpr int kMinv = kD8 + 72 * 4;                  // float [16][8][8]: (L_II^T)^-1
+  static constexpr int kVec = kMinv + 16 * 64 * 4;            // float [7][128]: kbar, vbar, rho, r, z, part, 1/L_kk
+  static constexpr int kWts = kVec + 7 * kLlaD * 4;           // float [kLlaMaxPieces]
+  static constexpr int kMisc = kWts + kLlaMaxPieces * 4;      // float [8]: l, kbar.rho, bad, stop, ...
+  static constexpr int kBar = (kMisc + 32 + 7) & ~7;          // upd_done, drain
+  static constexpr int kTmem = kBar + 24;
+  static constexpr int kBytes = kTmem + 16 + 1024;
+};
 
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
@@ -631,20 +647,56 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaArgs a) {
-  extern __shared__ float smf[];
-  float* Dkv = smf;                        // [128 columns][128]: D_KV of piece 0, column-major as recorded
-  float* Lt = Dkv + kLlaD * kLlaD;         // [128][kLlaLt]: Lt[k * kLlaLt + i] = L[i][k], i = 128: z
-  float* kb = Lt + kLlaD * kLlaLt;         // kbar
-  float* vb = kb + kLlaD;                  // vbar
-  float* rho_s = vb + kLlaD;               // rho*
-  float* r_s = rho_s + kLlaD;              // the back substitution's right-hand side (z, updated)
-  float* inv_s = r_s + kLlaD;              // 1 / L[k][k]
-  float* part = inv_s + kLlaD;             // [128] D_KV^T rho*
-  float* wts = part + kLlaD;               // [kLlaMaxPieces] piece weights 2^(m_j - M)
-  float* misc = wts + kLlaMaxPieces;       // [0] l, [1] kbar . rho*, [2] non-positive pivot flag
+// 8 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
 
-  const int tid = threadIdx.x;
+// Cholesky of the 8 x 8 block d (lower triangle used) in place, with the
+// reciprocals of the diagonal; false if a pivot is not positive.
+__device__ __forceinline__ bool lla_chol8(float (&d)[8][8], float (&inv)[8]) {
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float akk = d[k][k];
+    ok = ok && akk > 0.f && isfinite(akk);
+    const float invd = rsqrtf(akk);
+    d[k][k] = akk * invd;
+    inv[k] = invd;
+#pragma unroll
+    for (int i = k + 1; i < 8; ++i) d[i][k] *= invd;
+#pragma unroll
+    for (int i = k + 1; i < 8; ++i)
+#pragma unroll
+      for (int jj = k + 1; jj <= i; ++jj) d[i][jj] = fmaf(-d[i][k], d[jj][k], d[i][jj]);
+  }
+  return ok;
+}
+
+__global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const LlaArgs a) {
+  using Ly = LlaSolveLayout;
+  extern __shared__ uint8_t smem_raw_s[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_s) + 1023) & ~uintptr_t(1023));
+  float* Dkv = reinterpret_cast<float*>(sm + Ly::kDkv);   // column-major as recorded
+  float* Lt = reinterpret_cast<float*>(sm + Ly::kLt);     // Lt[k * kLlaLt + i] = L[i][k]
+  float* d8 = reinterpret_cast<float*>(sm + Ly::kD8);     // [8][8] diagonal block, then [8] its rhs
+  float* kb = reinterpret_cast<float*>(sm + Ly::kVec);    // kbar
+  float* vb = kb + kLlaD;                                 // vbar
+  float* rho_s = vb + kLlaD;                              // rho*
+  float* rb = rho_s + kLlaD;                              // back substitution right-hand side
+  float* z_s = rb + kLlaD;                                // z = L^-1 (kbar - q)
+  float* part = z_s + kLlaD;                              // D_KV^T rho*
+  float* inv_s = part + kLlaD;                            // 1 / L[k][k]
+  float* minv = reinterpret_cast<float*>(sm + Ly::kMinv); // [I][c][r]: (L_II^T)^-1
+  float* wts = reinterpret_cast<float*>(sm + Ly::kWts);   // piece weights 2^(m_j - M)
+  float* misc = reinterpret_cast<float*>(sm + Ly::kMisc); // [0] l, [1] kbar . rho*, [2] bad pivot, [3] stop
+  uint64_t* upd_done = reinterpret_cast<uint64_t*>(sm + Ly::kBar);   // the panel's update is done
+  uint64_t* drain = upd_done + 1;                                    // every product has completed
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kTmem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.x, b = bh / a.Hq;
   const size_t orow = (size_t)bh * kLlaD;
   // Launched with a programmatic dependency on the moments grid: the records
@@ -686,8 +738,22 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     }
     misc[0] = L;
     misc[2] = 0.f;
+    misc[3] = 0.f;
+    mbar_init(upd_done, 1);
+    mbar_init(drain, 1);
+    fence_mbarrier_init();
   }
+  // the three operand parts start as zeros: each row's columns 8.. stay zero
+  for (int i = tid; i < 3 * Ly::kOpBytes / 16; i += kLlaSolveThreads)
+    reinterpret_cast<uint4*>(sm + Ly::kOp)[i] = make_uint4(0u, 0u, 0u, 0u);
+  if (warp == 0) {
+    tmem_alloc(tmem_base_s, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_s;
   const float invL = 1.f / misc[0];
   if (tid < kLlaD) {
     float ks = 0.f, vs = 0.f;
@@ -702,172 +768,202 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
   }
   __syncthreads();
 
-  // ---- this thread's block of S_KK + ridge I = D_KK / l - kbar kbar^T + ridge I
-  // (block row 16: row 0 of the block is b = kbar - q, the rest zero)
-  const int bi = tid >> 4, bj = tid & 15, r0 = 8 * bi, c0 = 8 * bj;
-  const bool active = bi < 16 ? bi >= bj : bi == 16;
-  float blk[8][8];
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  constexpr uint32_t kIdUpd = idesc_bf16(kLlaD, kLlaD, false) | (1u << 13);   // 128 x 128 x 16, A negated
+  const int r_ = tid;   // row a of S, TMEM lane a
+  // ---- row a of S_KK + ridge I = D_KK / l - kbar kbar^T + ridge I into tensor
+  // memory (D_KK is recorded column-major: entry [a][j] at j * 128 + a, so a
+  // warp's 32 rows read 128 contiguous bytes per column; 64 loads in flight)
+#pragma unroll 1
+  for (int c64 = 0; c64 < 2; ++c64) {
+    float sv[64];
 #pragma unroll
-  for (int r = 0; r < 8; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c) blk[r][c] = 0.f;
-  if (bi < 16 && active) {
+    for (int j = 0; j < 64; ++j) sv[j] = 0.f;
+#pragma unroll 1
     for (int p = 0; p < a.pieces; ++p) {
-      if (wts[p] == 0.f) continue;
-      // column c0 + c of the block: rows r0 .. r0 + 7 are contiguous
-      const float* d = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKK + c0 * kLlaD + r0;
-      float4 v[8][2];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {   // all 16 loads in flight before any use
-        v[c][0] = *reinterpret_cast<const float4*>(d + c * kLlaD);
-        v[c][1] = *reinterpret_cast<const float4*>(d + c * kLlaD + 4);
-      }
       const float w = wts[p];
+      if (w == 0.f) continue;
+      const float* col0 = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKK + (size_t)(64 * c64) * kLlaD + r_;
+      float v[64];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        blk[0][c] = fmaf(w, v[c][0].x, blk[0][c]);
-        blk[1][c] = fmaf(w, v[c][0].y, blk[1][c]);
-        blk[2][c] = fmaf(w, v[c][0].z, blk[2][c]);
-        blk[3][c] = fmaf(w, v[c][0].w, blk[3][c]);
-        blk[4][c] = fmaf(w, v[c][1].x, blk[4][c]);
-        blk[5][c] = fmaf(w, v[c][1].y, blk[5][c]);
-        blk[6][c] = fmaf(w, v[c][1].z, blk[6][c]);
-        blk[7][c] = fmaf(w, v[c][1].w, blk[7][c]);
-      }
+      for (int j = 0; j < 64; ++j) v[j] = __ldg(col0 + (size_t)j * kLlaD);
+#pragma unroll
+      for (int j = 0; j < 64; ++j) sv[j] = fmaf(w, v[j], sv[j]);
     }
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
+    for (int h = 0; h < 2; ++h) {
+      uint32_t v[32];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        blk[r][c] = fmaf(blk[r][c], invL, -kb[r0 + r] * kb[c0 + c]) + (r0 + r == c0 + c ? a.ridge : 0.f);
-  } else if (active) {   // the b row
-#pragma unroll
-    for (int c = 0; c < 8; ++c) blk[0][c] = kb[c0 + c] - __bfloat162float(a.q[orow + c0 + c]);
+      for (int j = 0; j < 32; ++j) {
+        const int col = 64 * c64 + 32 * h + j;
+        v[j] = __float_as_uint(fmaf(sv[32 * h + j], invL, -kb[r_] * kb[col]) + (col == r_ ? a.ridge : 0.f));
+      }
+      tmem_st32(tmem + lane_off + (uint32_t)(64 * c64 + 32 * h), v);
+    }
   }
-
-  // ---- blocked Cholesky, one panel of 8 columns per step P: the diagonal
-  // block's owner factors it in registers; the blocks below it (the b row
-  // included) solve against that factor (X L_PP^T = A); the blocks right of
-  // the panel and on or below the diagonal take the rank-8 update.
-  bool bad = false;
+  tmem_wait_st();
+  float rr_a = kb[r_] - __bfloat162float(a.q[orow + r_]);   // forward right-hand side of row a
+  bool fine = true;
 #pragma unroll 1
   for (int P = 0; P < 16; ++P) {
-    if (bi == P && bj == P) {   // the diagonal block: L_PP L_PP^T = A_PP
-      bool ok = true;
+    const int c0 = 8 * P;
+    bool w = true;
+    if (P > 0) w = mbar_wait_bounded(a.wait_ns, upd_done, (P - 1) & 1);   // S holds panel P - 1's update
+    tc_fence_after();
+    uint32_t xr[8];
+    tmem_ld8(tmem + lane_off + (uint32_t)c0, xr);
+    tmem_wait_ld();
+    float x[8];
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float akk = blk[k][k];
-        ok = ok && akk > 0.f && isfinite(akk);
-        const float invd = rsqrtf(akk);
-        blk[k][k] = akk * invd;
-        inv_s[8 * P + k] = invd;
+    for (int c = 0; c < 8; ++c) x[c] = __uint_as_float(xr[c]);
+    if (r_ >= c0 && r_ < c0 + 8) {
 #pragma unroll
-        for (int i = k + 1; i < 8; ++i) blk[i][k] *= invd;
-#pragma unroll
-        for (int i = k + 1; i < 8; ++i)
-#pragma unroll
-          for (int jj = k + 1; jj <= i; ++jj) blk[i][jj] = fmaf(-blk[i][k], blk[jj][k], blk[i][jj]);
-      }
-      if (!ok) misc[2] = 1.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c)
-#pragma unroll
-        for (int r = c; r < 8; ++r) Lt[(c0 + c) * kLlaLt + r0 + r] = blk[r][c];
+      for (int c = 0; c < 8; ++c) d8[(r_ - c0) * 8 + c] = x[c];
+      d8[64 + (r_ - c0)] = rr_a;
     }
-    __syncthreads();
-    if (misc[2] != 0.f) {   // not numerically positive definite (uniform)
-      bad = true;
+    if (!bar_and(1, kLlaSolveThreads, w)) {   // a wait ran out (reported)
+      fine = false;
+      if (r_ == 0) misc[3] = 1.f;
       break;
     }
-    if (active && bj == P && bi > P) {   // the panel: X L_PP^T = A, column by column
-      const float* lpp = Lt + (8 * P) * kLlaLt + 8 * P;   // lpp[m * kLlaLt + c] = L_PP[c][m]
-      float lp[8][8], invd[8];   // L_PP below the diagonal and 1 / L_PP[c][c], loaded before the chain
+    // every row thread factors the diagonal block and solves L_PP z_P = r_P
+    float dd[8][8], inv[8], zz[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) dd[i][c] = d8[i * 8 + c];
+    const bool ok = lla_chol8(dd, inv);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float v = d8[64 + c];
+#pragma unroll
+      for (int m = 0; m < c; ++m) v = fmaf(-dd[c][m], zz[m], v);
+      zz[c] = v * inv[c];
+    }
+    if (!ok) {   // not numerically positive definite (every row thread sees it)
+      fine = false;
+      if (r_ == 0) {
+        misc[2] = 1.f;
+        misc[3] = 1.f;
+      }
+      break;
+    }
+    // this row's entries of L in the panel
+    float l[8];
+    if (r_ >= c0 + 8) {   // below the panel's diagonal block: l L_PP^T = x
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        invd[c] = inv_s[8 * P + c];
+        float v = x[c];
 #pragma unroll
-        for (int m = 0; m < c; ++m) lp[c][m] = lpp[m * kLlaLt + c];
+        for (int m = 0; m < c; ++m) v = fmaf(-l[m], dd[c][m], v);
+        l[c] = v * inv[c];
       }
 #pragma unroll
+      for (int c = 0; c < 8; ++c) rr_a = fmaf(-l[c], zz[c], rr_a);
+    } else if (r_ >= c0) {   // a row of the diagonal block: that row of L_PP
+      const int ri = r_ - c0;
+#pragma unroll
       for (int c = 0; c < 8; ++c) {
+        float v = 0.f;
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-          float x = blk[r][c];
-#pragma unroll
-          for (int m = 0; m < c; ++m) x = fmaf(-blk[r][m], lp[c][m], x);
-          blk[r][c] = x * invd[c];
-        }
+        for (int i = c; i < 8; ++i) v = i == ri ? dd[i][c] : v;
+        l[c] = v;
       }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) l[c] = 0.f;
+    }
+    if (r_ >= c0) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) Lt[(c0 + c) * kLlaLt + r_] = l[c];
+    }
+    if (r_ == c0) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
-        float4* dst = reinterpret_cast<float4*>(Lt + (c0 + c) * kLlaLt + r0);
-        dst[0] = make_float4(blk[0][c], blk[1][c], blk[2][c], blk[3][c]);
-        dst[1] = make_float4(blk[4][c], blk[5][c], blk[6][c], blk[7][c]);
+        z_s[c0 + c] = zz[c];
+        inv_s[c0 + c] = inv[c];
       }
     }
-    __syncthreads();
-    if (active && bj > P) {   // rank-8 update of the trailing blocks
+    if (P < 15) {
+      // the update's operand: rows below the panel's diagonal block, split
+      // into bf16 hi + mid + lo (16-byte chunk 0 of the row; the rest is zero)
+      uint32_t ph[4], pm[4], pl[4];
 #pragma unroll
-      for (int m = 0; m < 8; ++m) {
-        const float* lk = Lt + (8 * P + m) * kLlaLt;   // column 8 P + m of L
-        const float4 i0 = *reinterpret_cast<const float4*>(lk + r0), i1 = *reinterpret_cast<const float4*>(lk + r0 + 4);
-        const float4 j0 = *reinterpret_cast<const float4*>(lk + c0), j1 = *reinterpret_cast<const float4*>(lk + c0 + 4);
-        const float li[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-        const float2 lj[4] = {make_float2(j0.x, j0.y), make_float2(j0.z, j0.w), make_float2(j1.x, j1.y),
-                              make_float2(j1.z, j1.w)};
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {   // packed pairs of columns
-            const float2 t = fma2(make_float2(-li[r], -li[r]), lj[h], make_float2(blk[r][2 * h], blk[r][2 * h + 1]));
-            blk[r][2 * h] = t.x;
-            blk[r][2 * h + 1] = t.y;
-          }
+      for (int c = 0; c < 4; ++c) {
+        const float v0 = r_ >= c0 + 8 ? l[2 * c] : 0.f, v1 = r_ >= c0 + 8 ? l[2 * c + 1] : 0.f;
+        ph[c] = pack_bf16(v0, v1);
+        const float m0 = v0 - bf16_lo_f(ph[c]), m1 = v1 - bf16_hi_f(ph[c]);
+        pm[c] = pack_bf16(m0, m1);
+        pl[c] = pack_bf16(m0 - bf16_lo_f(pm[c]), m1 - bf16_hi_f(pm[c]));
+      }
+      const int off = r_ * 128 + ((r_ & 7) << 4);   // chunk 0 of row a, swizzled
+      *reinterpret_cast<uint4*>(sm + Ly::kOp + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+      *reinterpret_cast<uint4*>(sm + Ly::kOp + Ly::kOpBytes + off) = make_uint4(pm[0], pm[1], pm[2], pm[3]);
+      *reinterpret_cast<uint4*>(sm + Ly::kOp + 2 * Ly::kOpBytes + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      bar_and(1, kLlaSolveThreads, true);   // every row of the operand is written
+      if (warp == 0) {
+        // S -= L L^T over six products of the parts (hi hi, hi mid, mid hi, hi lo, lo hi, mid mid)
+        tc_fence_after();
+        const uint64_t dh = smem_desc_sw128(smem_u32(sm + Ly::kOp), 16, 1024);
+        const uint64_t dm = dh + (uint64_t)(Ly::kOpBytes >> 4), dl = dh + (uint64_t)((2 * Ly::kOpBytes) >> 4);
+        lla_mma4_ss(tmem, dh, dh, dh, dm, dm, dh, dh, dl, kIdUpd, 1u);
+        tc_mma_ss(tmem, dl, dh, kIdUpd, 1u);
+        tc_mma_ss(tmem, dm, dm, kIdUpd, 1u);
+        tc_commit(upd_done);
       }
     }
   }
-  if (bad) {
+  if (warp == 0) {   // every product issued completes before tensor memory is freed
+    tc_commit(drain);
+    __syncwarp();
+    mbar_wait_drain(drain, 0);
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 128);
+  if (!fine) {   // (a wait that ran out has reported itself)
     cp_async_wait_all();
-    if (tid == 0) report_error(PLX_DEVERR_SINGULAR_BIT);
-    if (tid < kLlaD) {   // rho* = 0: the output falls back to vbar
-      store_out(tid, vb[tid]);
-      if (a.rho) a.rho[orow + tid] = 0.f;
-    }
+    if (tid == 0 && misc[2] != 0.f) report_error(PLX_DEVERR_SINGULAR_BIT);
+    store_out(tid, vb[tid]);   // rho* = 0: the output falls back to vbar
+    if (a.rho) a.rho[orow + tid] = 0.f;
     return;
   }
-  // ---- L^T rho = z, blockwise from the last block: the diagonal block's
-  // owner solves L_II^T rho_I = r_I; the owners of row I of L then take
-  // L_IJ^T rho_I off r_J (J < I).
-  if (bi == 16 && bj < 16) {
+  // ---- L^T rho = z.  First the inverses of the transposed diagonal blocks,
+  // one column per thread: column j of (L_II^T)^-1 for I = tid / 8, j = tid % 8.
+  {
+    const int I = tid >> 3, j = tid & 7;
+    float xx[8];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) r_s[c0 + c] = blk[0][c];   // z
+    for (int c = 7; c >= 0; --c) {
+      float v = c == j ? 1.f : 0.f;
+#pragma unroll
+      for (int rr2 = c + 1; rr2 < 8; ++rr2) v = fmaf(-Lt[(8 * I + c) * kLlaLt + 8 * I + rr2], xx[rr2], v);
+      xx[c] = v * inv_s[8 * I + c];
+      minv[I * 64 + c * 8 + j] = xx[c];
+    }
+    rb[r_] = z_s[r_];
   }
   __syncthreads();
+  // Then blockwise from the last block: rho_I = (L_II^T)^-1 r_I (eight
+  // threads), and every row above takes L_IJ^T rho_I off its r_J.
 #pragma unroll 1
   for (int I = 15; I >= 0; --I) {
-    if (bi == I && bj == I) {
-      float x[8];
+    if (r_ < 8) {
+      float t = 0.f;
 #pragma unroll
-      for (int c = 7; c >= 0; --c) {
-        float v = r_s[8 * I + c];
-#pragma unroll
-        for (int rr = c + 1; rr < 8; ++rr) v = fmaf(-blk[rr][c], x[rr], v);
-        x[c] = v * inv_s[8 * I + c];
-        rho_s[8 * I + c] = x[c];
-      }
+      for (int rr2 = 0; rr2 < 8; ++rr2) t = fmaf(minv[I * 64 + r_ * 8 + rr2], rb[8 * I + rr2], t);
+      rho_s[8 * I + r_] = t;
     }
     __syncthreads();
-    if (bi == I && bj < I) {
-      float x[8];
+    if (r_ < 8 * I) {
+      float t = 0.f;
 #pragma unroll
-      for (int r = 0; r < 8; ++r) x[r] = rho_s[8 * I + r];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float t = 0.f;
-#pragma unroll
-        for (int r = 0; r < 8; ++r) t = fmaf(blk[r][c], x[r], t);
-        r_s[c0 + c] -= t;
-      }
+      for (int c = 0; c < 8; ++c) t = fmaf(Lt[r_ * kLlaLt + 8 * I + c], rho_s[8 * I + c], t);
+      rb[r_] -= t;
     }
     __syncthreads();
   }
@@ -881,18 +977,17 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
   cp_async_wait_all();
   __syncthreads();
   // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a: warp w
-  // takes columns 16 w .. 16 w + 15, lane l rows 4 l .. 4 l + 3 of each (a
+  // takes columns 32 w .. 32 w + 31, lane l rows 4 l .. 4 l + 3 of each (a
   // column of D_KV is 512 contiguous bytes)
-  if (tid < 8 * 32) {
-    const int wid = tid >> 5, lane = tid & 31;
+  {
     const float4 rr = *reinterpret_cast<const float4*>(rho_s + 4 * lane);
     auto dot4 = [&](const float* p4) {
       const float4 v = *reinterpret_cast<const float4*>(p4);
       return fmaf(v.x, rr.x, fmaf(v.y, rr.y, fmaf(v.z, rr.z, v.w * rr.w)));
     };
 #pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-      const int col = 16 * wid + k;
+    for (int k = 0; k < 32; ++k) {
+      const int col = 32 * warp + k;
       float acc = wts[0] == 0.f ? 0.f : wts[0] * dot4(Dkv + col * kLlaD + 4 * lane);
       for (int p = 1; p < a.pieces; ++p)
         if (wts[p] != 0.f)
@@ -902,15 +997,10 @@ __global__ void __launch_bounds__(kLlaSolveThreads) lla_solve_kernel(const LlaAr
     }
   }
   __syncthreads();
-  if (tid < kLlaD) {
-    const float corr = part[tid];
-    store_out(tid, fmaf(vb[tid], 1.f + misc[1], -corr * invL));
-    if (a.rho) a.rho[orow + tid] = rho_s[tid];
-  }
+  store_out(tid, fmaf(vb[tid], 1.f + misc[1], -part[tid] * invL));
+  if (a.rho) a.rho[orow + tid] = rho_s[tid];
 }
 
-constexpr int lla_solve_smem_bytes() {
-  return (kLlaD * kLlaD + kLlaD * kLlaLt + 6 * kLlaD + kLlaMaxPieces + 4) * 4;
-}
+constexpr int lla_solve_smem_bytes() { return LlaSolveLayout::kBytes; }
 
 }  // namespace plx
