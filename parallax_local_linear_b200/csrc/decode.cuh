@@ -464,20 +464,35 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
       const int hq0 = kvh * g;
 
       // [Q; R] A-operand fragments of this unit, and a_ref = rho_h . k_0.
+      // The group's q and rho rows come into shared memory first, one 16-byte
+      // load per 16 bytes (few, wide requests also when they sit in mapped
+      // host memory across PCIe); st is unused until this unit's end, and the
+      // bar() there orders its next writes after these reads.
       uint32_t qa[D / 16][4];
       {
+        constexpr int kQsStride = D / 2 + 4;   // words per row: rows land 4 banks apart
+        static_assert(16 * kQsStride <= 2 * kMaxGroup * D, "the staging rows fit in st.o1 and st.o2");
+        uint32_t* qs = reinterpret_cast<uint32_t*>(&st.o1[0][0]);   // rows 0..g-1 q, 8..8+g-1 rho
+#pragma unroll 1
+        for (int i = tid; i < 2 * g * (D / 8); i += NT) {
+          const int row = i / (D / 8), v = i % (D / 8);
+          const bool isr = row >= g;
+          const int h = isr ? row - g : row;
+          const uint4 val = __ldg(reinterpret_cast<const uint4*>(
+              reinterpret_cast<const __nv_bfloat16*>(isr ? a.rho : a.q) + ((size_t)b * a.Hq + hq0 + h) * D + 8 * v));
+          *reinterpret_cast<uint4*>(qs + (isr ? 8 + h : h) * kQsStride + 4 * v) = val;
+        }
+        bar();
         const bool live = hr < g;
-        const size_t qoff = ((size_t)b * a.Hq + hq0 + (live ? hr : 0)) * D;
-        const uint32_t* qrow = reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(a.q) + qoff);
-        const uint32_t* rrow =
-            reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(a.rho) + qoff);
+        const uint32_t* qrow = qs + hr * kQsStride;
+        const uint32_t* rrow = qs + (8 + hr) * kQsStride;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int c0 = (16 * kk + qc) / 2, c1 = (16 * kk + 8 + qc) / 2;
-          qa[kk][0] = live ? __ldg(qrow + c0) : 0u;
-          qa[kk][1] = live ? __ldg(rrow + c0) : 0u;
-          qa[kk][2] = live ? __ldg(qrow + c1) : 0u;
-          qa[kk][3] = live ? __ldg(rrow + c1) : 0u;
+          qa[kk][0] = live ? qrow[c0] : 0u;
+          qa[kk][1] = live ? rrow[c0] : 0u;
+          qa[kk][2] = live ? qrow[c1] : 0u;
+          qa[kk][3] = live ? rrow[c1] : 0u;
         }
       }
       // a_ref of head hr from the rho pairs this thread already holds (the
