@@ -726,20 +726,44 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     }
     cluster_sync();
     if (rank == 0) {
-      for (int i = threadIdx.x; i < g * D; i += blockDim.x) {
-        const int h = i / D, d = i % D;
+      // eight consecutive columns per thread, written as one 16-byte store
+      // (two for fp32): few, full-line writes, also into mapped host memory
+      for (int i = threadIdx.x; i < g * (D / 8); i += blockDim.x) {
+        const int h = i / (D / 8), d0 = 8 * (i % (D / 8));
         float M = st.m[h];
         for (int r = 0; r < k - 1; ++r) M = fmaxf(M, recv[r].m[h]);
         const float a0 = ex2(st.m[h] - M);
-        float L = a0 * st.l[h], C = a0 * st.c[h], O1 = a0 * st.o1[h][d], O2 = a0 * st.o2[h][d];
-        for (int r = 0; r < k - 1; ++r) {
-          const float al = ex2(recv[r].m[h] - M);
-          L += al * recv[r].l[h];
-          C += al * recv[r].c[h];
-          O1 += al * recv[r].o1[h][d];
-          O2 += al * recv[r].o2[h][d];
+        float al[kMaxClusterRecv];
+        float L = a0 * st.l[h], C = a0 * st.c[h];
+#pragma unroll
+        for (int r = 0; r < kMaxClusterRecv; ++r) {
+          al[r] = r < k - 1 ? ex2(recv[r].m[h] - M) : 0.f;
+          if (r < k - 1) {
+            L += al[r] * recv[r].l[h];
+            C += al[r] * recv[r].c[h];
+          }
         }
-        store_out(a, ((size_t)b * a.Hq + hq0 + h) * D + d, finalize(O1, O2, L, C));
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float O1 = a0 * st.o1[h][d0 + e], O2 = a0 * st.o2[h][d0 + e];
+#pragma unroll
+          for (int r = 0; r < kMaxClusterRecv; ++r)
+            if (r < k - 1) {
+              O1 += al[r] * recv[r].o1[h][d0 + e];
+              O2 += al[r] * recv[r].o2[h][d0 + e];
+            }
+          v[e] = finalize(O1, O2, L, C);
+        }
+        const size_t idx = ((size_t)b * a.Hq + hq0 + h) * D + d0;
+        if (a.out_bf16) {
+          *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.out) + idx) =
+              make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+        } else {
+          float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + idx);
+          o[0] = make_float4(v[0], v[1], v[2], v[3]);
+          o[1] = make_float4(v[4], v[5], v[6], v[7]);
+        }
       }
     }
   }
