@@ -341,12 +341,11 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
                      const DecodeArgs a) {
   using SM = TcSmem<D>;
-  // Consumer warp w takes tiles t = w (mod NC) and tile t sits in stage
-  // t % STAGES.  The parity wait on full[t % STAGES] is exact only if tile
-  // t - STAGES, the previous load into that stage, was consumed by the same
-  // warp, which holds exactly when NC divides STAGES: then each warp owns its
-  // stages and cannot run a whole ring ahead of a slower warp.
-  static_assert(STAGES % NC == 0, "each consumer warp must own whole stages");
+  // Tile t sits in stage t % STAGES and every consumer warp reads 16 of its
+  // 64 tokens; the stage is refilled once all NC warps have released it, so
+  // no warp can run a whole ring ahead of another and the parity wait on
+  // full[t % STAGES] is exact.
+  static_assert(kTile == 16 * NC, "each consumer warp takes 16 tokens of a tile");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* wstate = reinterpret_cast<float*>(ring + STAGES * SM::kStageBytes);
@@ -366,14 +365,19 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
   // dependency then has its launch and set-up done by the time this grid
   // ends, and waits below for this grid's results.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // Set-up that reads no global memory runs before the wait: the tile space
-  // when every sequence has kv_len tokens, the ring's barriers, the tensor
-  // maps' prefetch.
-  if (a.seq_lens == nullptr) build_tile_space(a, pre, lens, scan);
+  // Set-up that reads no global memory runs before the wait.  When every
+  // sequence has kv_len tokens (no seq_lens) the tile space is closed-form
+  // and nothing up to the first K/V load touches global memory: the
+  // producer then waits for the previous grid just before that load, the
+  // consumers before reading q and rho, and the chunk bounds, the cursor and
+  // the first stage's expected bytes are ready by then.  (kv_len is at least
+  // 1 here, so there are no empty sequences to write.)
+  const bool closed = a.seq_lens == nullptr;
+  if (closed) build_tile_space(a, pre, lens, scan);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+      mbar_init(&empty[s], NC);
     }
     s_flag[0] = 0;
     s_flag[1] = 0;
@@ -383,8 +387,8 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     prefetch_tmap(&tmap_k);
     prefetch_tmap(&tmap_v);
   }
-  if (a.pdl_all) asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (a.seq_lens != nullptr) build_tile_space(a, pre, lens, scan);
+  if (a.pdl_all && !closed) asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (!closed) build_tile_space(a, pre, lens, scan);
 
   // Sequences of length zero have no tiles: CTA b % gridDim.x writes their zeros.
   for (int b = blockIdx.x; b < a.B; b += gridDim.x)
@@ -422,6 +426,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         uint8_t* kdst = ring + s * SM::kStageBytes;
         uint8_t* vdst = kdst + SM::kTileBytes;
         mbar_arrive_expect_tx(&full[s], SM::kStageBytes);
+        if (t == 0 && a.pdl_all) asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
         for (int bx = 0; bx < SM::kBoxes; ++bx) {
           tma_load_2d(kdst + bx * SM::kBoxBytes, &tmap_k, bx * 64, row, &full[s], pol);
@@ -521,9 +526,11 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
       float m_run = -INFINITY, l_part = 0.f, c_part = 0.f;
 
       const int i_begin = (int)(x - x0), i_end = (int)(seg_end - x0);
-      // first chunk-local tile index >= i_begin that this warp owns (t % NC == warp)
-      int t = i_begin + ((warp - i_begin % NC) + NC) % NC;
-      for (; t < i_end; t += NC) {
+      // Every consumer warp takes its own 16 tokens (rows 16 w .. 16 w + 15)
+      // of every tile: a tile is consumed, and its stage freed, in about a
+      // quarter of the time one warp would take for all 64 tokens, and the
+      // last tile of a chunk does not leave three warps idle.
+      for (int t = i_begin; t < i_end; ++t) {
         const int s = t % STAGES;
         if (*abort_flag) break;
         if (!mbar_wait_bounded(a.wait_ns, &full[s], (t / STAGES) & 1)) {
@@ -534,9 +541,16 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         uint8_t* vt = kt + SM::kTileBytes;
         const int tok0 = (local0 + (t - i_begin)) * kTile;
         const int nvalid = min(kTile, len - tok0);
-        if (nvalid < kTile) {
-          // Zero V rows past the sequence end: their weight is 0, but 0 * NaN is not.
-          for (int i = lane; i < (kTile - nvalid) * SM::kBoxes * 8; i += 32) {
+        const int row0 = 16 * warp;   // this warp's first token row in the tile
+        if (nvalid <= row0) {         // all of this warp's tokens lie past the end
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[s]);
+          continue;
+        }
+        if (nvalid < row0 + 16) {
+          // Zero this warp's V rows past the sequence end: their weight is 0,
+          // but 0 * NaN is not.
+          for (int i = lane; i < (row0 + 16 - nvalid) * SM::kBoxes * 8; i += 32) {
             const int row = nvalid + i / (SM::kBoxes * 8);
             const int rest = i % (SM::kBoxes * 8);
             *reinterpret_cast<uint4*>(vt + (rest / 8) * SM::kBoxBytes + row * 128 + (rest % 8) * 16) =
@@ -545,16 +559,16 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
           fence_proxy_async_smem();
           __syncwarp();
         }
-        // ---- [S; A] = [Q; R] K^T
-        float sc[8][4];
+        // ---- [S; A] = [Q; R] K^T over this warp's two 8-token blocks
+        float sc[2][4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
-        const uint32_t kb = smem_u32(kt);
+        for (int j = 0; j < 2; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+        const uint32_t kb = smem_u32(kt) + (uint32_t)row0 * 128u;
 #pragma unroll
         for (int k2 = 0; k2 < D / 32; ++k2) {
           const uint32_t off = (k2 >> 1) * SM::kBoxBytes + rr * 128 + ((((k2 & 1) * 4 + mi) ^ rr) << 4);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int j = 0; j < 2; ++j) {
             uint32_t b0, b1, b2, b3;
             ldsm_x4(kb + off + j * 1024, b0, b1, b2, b3);
             mma_bf16_16816(sc[j], qa[2 * k2], b0, b1);
@@ -564,10 +578,10 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         // ---- online softmax on this thread's row; mask tokens past the end
         float mloc = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 2; ++j) {
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const bool ok = 8 * j + qc + e < nvalid;
+            const bool ok = row0 + 8 * j + qc + e < nvalid;
             sc[j][e] = ok ? sc[j][e] * a.scale_log2 : -INFINITY;
             sc[j][2 + e] = ok ? sc[j][2 + e] - aref : 0.f;
             mloc = fmaxf(mloc, sc[j][e]);
@@ -575,7 +589,7 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         }
         mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 1));
         mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, 2));
-        const float m_new = fmaxf(m_run, mloc);
+        const float m_new = fmaxf(m_run, mloc);   // finite: the warp has a valid token here
         const float alpha = ex2(m_run - m_new);
         m_run = m_new;
         l_part *= alpha;
@@ -587,29 +601,27 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
         // sequences.  With g <= 4 the lo pairs ride in the zero-padding rows
         // 4..7 / 12..15 (handed over from lane - 16), so they cost no extra
         // MMA; otherwise a second MMA consumes them.
-        uint32_t pf[4][4], pl[4][4];
+        uint32_t pf[4], pl[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 2; ++j) {
           const float p0 = ex2(sc[j][0] - m_new), p1 = ex2(sc[j][1] - m_new);
           const float pa0 = p0 * sc[j][2], pa1 = p1 * sc[j][3];
           l_part += p0 + p1;
           c_part += pa0 + pa1;
           const uint32_t hp = pack_bf16(p0, p1), ha = pack_bf16(pa0, pa1);
-          pf[j >> 1][(j & 1) * 2 + 0] = hp;
-          pf[j >> 1][(j & 1) * 2 + 1] = ha;
-          pl[j >> 1][(j & 1) * 2 + 0] = pack_bf16(p0 - bf16_lo_f(hp), p1 - bf16_hi_f(hp));
-          pl[j >> 1][(j & 1) * 2 + 1] = pack_bf16(pa0 - bf16_lo_f(ha), pa1 - bf16_hi_f(ha));
+          pf[2 * j + 0] = hp;
+          pf[2 * j + 1] = ha;
+          pl[2 * j + 0] = pack_bf16(p0 - bf16_lo_f(hp), p1 - bf16_hi_f(hp));
+          pl[2 * j + 1] = pack_bf16(pa0 - bf16_lo_f(ha), pa1 - bf16_hi_f(ha));
         }
         float alpha_o = alpha;
         if (kLoInPad) {
           const float a_from = __shfl_xor_sync(0xffffffffu, alpha, 16);
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj)
-#pragma unroll
-            for (int xx = 0; xx < 4; ++xx) {
-              const uint32_t from = __shfl_xor_sync(0xffffffffu, pl[jj][xx], 16);
-              if (lane & 16) pf[jj][xx] = from;
-            }
+          for (int xx = 0; xx < 4; ++xx) {
+            const uint32_t from = __shfl_xor_sync(0xffffffffu, pl[xx], 16);
+            if (lane & 16) pf[xx] = from;
+          }
           if (lane & 16) alpha_o = a_from;
         }
         if (alpha_o != 1.f) {
@@ -621,23 +633,20 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
             o[i][3] *= alpha_o;
           }
         }
-        // ---- [O1; O2] += [P; P*A] V
-        const uint32_t vb = smem_u32(vt);
+        // ---- [O1; O2] += [P; P*A] V over this warp's 16 token rows
+        const uint32_t vb = smem_u32(vt) + (uint32_t)row0 * 128u;
 #pragma unroll
         for (int n2 = 0; n2 < D / 16; ++n2) {
           const int dcol = 16 * n2 + 8 * (mi >> 1);
           const uint32_t off = (dcol >> 6) * SM::kBoxBytes + (rr + 8 * (mi & 1)) * 128 +
                                ((((dcol & 63) >> 3) ^ rr) << 4);
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(vb + off + jj * 2048, b0, b1, b2, b3);
-            mma_bf16_16816(o[2 * n2], pf[jj], b0, b1);
-            mma_bf16_16816(o[2 * n2 + 1], pf[jj], b2, b3);
-            if (!kLoInPad) {
-              mma_bf16_16816(o[2 * n2], pl[jj], b0, b1);
-              mma_bf16_16816(o[2 * n2 + 1], pl[jj], b2, b3);
-            }
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_trans(vb + off, b0, b1, b2, b3);
+          mma_bf16_16816(o[2 * n2], pf, b0, b1);
+          mma_bf16_16816(o[2 * n2 + 1], pf, b2, b3);
+          if (!kLoInPad) {
+            mma_bf16_16816(o[2 * n2], pl, b0, b1);
+            mma_bf16_16816(o[2 * n2 + 1], pl, b2, b3);
           }
         }
         __syncwarp();
