@@ -165,7 +165,11 @@ plx_status parallax_decode_plan_run(const plx_decode_plan* plan, cudaStream_t st
  * mapped into the device's address space (cudaHostAlloc / pinned memory
  * under unified addressing, 16-byte aligned), the one launch reads q and rho
  * and writes the output across PCIe directly, and the plan's own q, rho and
- * out buffers are not touched.  Otherwise it copies host_q and host_rho into
+ * out buffers are not touched.  In that case q and rho are read as the
+ * launch starts, which may be before the kernel queued just ahead of it on
+ * the stream has finished (programmatic dependent launch; the KV cache and
+ * the output wait for it): host_q and host_rho must be written by the host
+ * before the call, not by device work queued on the stream.  Otherwise it copies host_q and host_rho into
  * the plan's q and rho, runs the decode and copies the plan's out into
  * host_out: three copies and one launch (page-locked buffers let the copies
  * overlap other work).  Errors as parallax_decode_plan_run;

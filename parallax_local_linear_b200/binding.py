@@ -358,9 +358,11 @@ class DecodePlan:
         """One step from host memory on the current stream: ``host_q`` and
         ``host_rho`` in, the decode, the output into ``host_out`` (host
         tensors: contiguous, shaped and typed like q / out).  When all three
-        are pinned the kernel reads and writes them across PCIe itself;
-        otherwise they go through copies into and out of the plan's
-        buffers."""
+        are pinned the kernel reads and writes them across PCIe itself, and
+        reads q and rho as it starts, possibly before the kernel queued
+        ahead of it has finished: the host must have written them before
+        the call.  Otherwise they go through copies into and out of the
+        plan's buffers."""
         q, rho = self._keep[0], self._keep[1]
         for name, t, like in (("host_q", host_q, q), ("host_rho", host_rho, rho), ("host_out", host_out, self.out)):
             if t.is_cuda or not t.is_contiguous() or t.dtype != like.dtype or tuple(t.shape) != tuple(like.shape):

@@ -56,6 +56,8 @@ struct DecodeArgs {
   int pdl_all;                     // 1: launched with a programmatic dependency on the previous
                                    // kernel, which any input may come from: every thread waits for it
                                    // before touching global memory (bf16 path)
+  int qr_early;                    // 1: q and rho are supplied by the host, not by earlier work in
+                                   // the stream, and are read before that wait (bf16 path)
   unsigned long long wait_ns;      // limit of one pipeline wait (0: give up unless complete)
 };
 
@@ -445,22 +447,44 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
     }
   } else {
     // ------------------------------------------------------------ consumers
-    // q and rho may come from the grid launched just before this one (the
-    // projection of a projected decode, with a programmatic dependency): wait
-    // for it to complete before reading them.  Without such a dependency the
-    // wait returns at once.  The producer warp streams K and V meanwhile.
-    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int tid = threadIdx.x;
     constexpr int NT = NC * 32;
     auto bar = [] { asm volatile("bar.sync 1, %0;" ::"n"(NT) : "memory"); };
+    // The group's q and rho rows of a unit into shared memory, one 16-byte
+    // load per 16 bytes (few, wide requests also when they sit in mapped
+    // host memory across PCIe); st is unused until the unit's end, and the
+    // bar() there orders its next writes after the reads of these rows.
+    constexpr int kQsStride = D / 2 + 4;   // words per row: rows land 4 banks apart
+    static_assert(16 * kQsStride <= 2 * kMaxGroup * D, "the staging rows fit in st.o1 and st.o2");
+    uint32_t* qs = reinterpret_cast<uint32_t*>(&st.o1[0][0]);   // rows 0..g-1 q, 8..8+g-1 rho
+    auto stage_qr = [&](int b, int hq0) {
+#pragma unroll 1
+      for (int i = tid; i < 2 * g * (D / 8); i += NT) {
+        const int row = i / (D / 8), v = i % (D / 8);
+        const bool isr = row >= g;
+        const int h = isr ? row - g : row;
+        const uint4 val = __ldg(reinterpret_cast<const uint4*>(
+            reinterpret_cast<const __nv_bfloat16*>(isr ? a.rho : a.q) + ((size_t)b * a.Hq + hq0 + h) * D + 8 * v));
+        *reinterpret_cast<uint4*>(qs + (isr ? 8 + h : h) * kQsStride + 4 * v) = val;
+      }
+    };
+    UnitCursor cur;
+    cur.seek(ts, x0);
+    // q and rho supplied by the host are read at once, while the previous
+    // grid may still run; otherwise they may come from the grid launched just
+    // before this one (the projection of a projected decode, or an earlier
+    // call), so the consumers wait for it first.  The producer warp streams
+    // K and V meanwhile.
+    const bool early = a.qr_early != 0;
+    if (early) stage_qr(cur.b, cur.hu * g);
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int hr = lane >> 2;          // accumulator row (head) of this thread
     const int qc = (lane & 3) * 2;     // column pair within an 8-wide chunk
     const int rr = lane & 7, mi = lane >> 3;
     float* ws = wstate + warp * SM::kWarpStateFloats;
 
-    UnitCursor cur;
-    cur.seek(ts, x0);
     long long x = x0;
+    bool staged = early;   // the first unit's rows are in qs already
     while (x < x1) {
       const int b = cur.b, kvh = cur.hu, local0 = cur.local;
       const long long ua = cur.unit_begin(ts), ub = ua + cur.tiles;
@@ -469,24 +493,10 @@ __global__ void __launch_bounds__((NC + 1) * 32, 1)
       const int hq0 = kvh * g;
 
       // [Q; R] A-operand fragments of this unit, and a_ref = rho_h . k_0.
-      // The group's q and rho rows come into shared memory first, one 16-byte
-      // load per 16 bytes (few, wide requests also when they sit in mapped
-      // host memory across PCIe); st is unused until this unit's end, and the
-      // bar() there orders its next writes after these reads.
       uint32_t qa[D / 16][4];
       {
-        constexpr int kQsStride = D / 2 + 4;   // words per row: rows land 4 banks apart
-        static_assert(16 * kQsStride <= 2 * kMaxGroup * D, "the staging rows fit in st.o1 and st.o2");
-        uint32_t* qs = reinterpret_cast<uint32_t*>(&st.o1[0][0]);   // rows 0..g-1 q, 8..8+g-1 rho
-#pragma unroll 1
-        for (int i = tid; i < 2 * g * (D / 8); i += NT) {
-          const int row = i / (D / 8), v = i % (D / 8);
-          const bool isr = row >= g;
-          const int h = isr ? row - g : row;
-          const uint4 val = __ldg(reinterpret_cast<const uint4*>(
-              reinterpret_cast<const __nv_bfloat16*>(isr ? a.rho : a.q) + ((size_t)b * a.Hq + hq0 + h) * D + 8 * v));
-          *reinterpret_cast<uint4*>(qs + (isr ? 8 + h : h) * kQsStride + 4 * v) = val;
-        }
+        if (!staged) stage_qr(b, hq0);
+        staged = false;
         bar();
         const bool live = hr < g;
         const uint32_t* qrow = qs + hr * kQsStride;

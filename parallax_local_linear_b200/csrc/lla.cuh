@@ -58,7 +58,7 @@ constexpr int kLlaScore = 128;           // score warps 2..5 (one per TMEM lane 
 constexpr int kLlaScale = 256;           // scale warps 6..13 (two per TMEM lane quarter)
 constexpr int kLlaSplitLen = 1024;       // shorter sequences add the lo part of e o K
 constexpr float kLlaRescaleLog2 = 8.f;   // lazy rescale threshold (factor 256)
-constexpr int kLlaMaxPieces = 16;
+constexpr int kLlaMaxPieces = 16;      // at most 32: the solve merges one piece per lane
 // Record of one piece: D_KK, D_KV (column-major: [a][b] at b * 128 + a), ks,
 // vs, then m, l.
 constexpr int kLlaRecKK = 0;
@@ -646,6 +646,7 @@ __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src)
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // 8 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
@@ -718,34 +719,43 @@ __global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const Ll
     return;
   }
   const float* rec0 = a.rec + (size_t)bh * a.pieces * kLlaRecFloats;
-  {   // D_KV of piece 0 into shared memory, in the background
-    const float* src = rec0 + kLlaRecKV;
+  float* Dkk_s = Lt;   // D_KK of piece 0, [128][128] column-major as recorded, until the panels write L^T
+  {   // D_KK, then D_KV, of piece 0 into shared memory, in the background
+    const float* src = rec0 + kLlaRecKK;
+    for (int i = tid; i < kLlaD * kLlaD / 4; i += kLlaSolveThreads) cp_async16(Dkk_s + 4 * i, src + 4 * i);
+    cp_async_commit();
+    src = rec0 + kLlaRecKV;
     for (int i = tid; i < kLlaD * kLlaD / 4; i += kLlaSolveThreads) cp_async16(Dkv + 4 * i, src + 4 * i);
     cp_async_commit();
   }
-  if (tid == 0) {
-    float M = -INFINITY;
-    for (int p = 0; p < a.pieces; ++p) {
-      const float* r = rec0 + (size_t)p * kLlaRecFloats;
-      if (r[kLlaRecM + 1] > 0.f) M = fmaxf(M, r[kLlaRecM]);
+  const float ks0 = rec0[kLlaRecKs + tid], vs0 = rec0[kLlaRecVs + tid];   // piece 0's sums, loaded early
+  if (warp == 0) {   // lane p merges piece p (at most 32 pieces)
+    const bool has = lane < a.pieces;
+    const float* r = rec0 + (size_t)lane * kLlaRecFloats;
+    const float lp = has ? r[kLlaRecM + 1] : 0.f;
+    const float mp = lp > 0.f ? r[kLlaRecM] : -INFINITY;
+    float M = mp;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = lp > 0.f ? ex2(mp - M) : 0.f;
+    if (has) wts[lane] = w;
+    const float L = warp_sum(w * lp);
+    if (lane == 0) {
+      misc[0] = L;
+      misc[2] = 0.f;
+      misc[3] = 0.f;
+      mbar_init(upd_done, 1);
+      mbar_init(drain, 1);
+      fence_mbarrier_init();
     }
-    float L = 0.f;
-    for (int p = 0; p < a.pieces; ++p) {
-      const float* r = rec0 + (size_t)p * kLlaRecFloats;
-      const float w = r[kLlaRecM + 1] > 0.f ? ex2(r[kLlaRecM] - M) : 0.f;
-      wts[p] = w;
-      L += w * r[kLlaRecM + 1];
-    }
-    misc[0] = L;
-    misc[2] = 0.f;
-    misc[3] = 0.f;
-    mbar_init(upd_done, 1);
-    mbar_init(drain, 1);
-    fence_mbarrier_init();
   }
-  // the three operand parts start as zeros: each row's columns 8.. stay zero
-  for (int i = tid; i < 3 * Ly::kOpBytes / 16; i += kLlaSolveThreads)
-    reinterpret_cast<uint4*>(sm + Ly::kOp)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // The products read columns 0..15 of each operand row (its 16-byte chunks
+  // 0 and 1, at swizzled places): chunk 0 is written every panel, chunk 1
+  // (columns 8..15) stays zero.  Thread a clears chunk 1 of row a in each part.
+#pragma unroll
+  for (int part_i = 0; part_i < 3; ++part_i)
+    *reinterpret_cast<uint4*>(sm + Ly::kOp + part_i * Ly::kOpBytes + tid * 128 + ((1 ^ (tid & 7)) << 4)) =
+        make_uint4(0u, 0u, 0u, 0u);
   if (warp == 0) {
     tmem_alloc(tmem_base_s, 128);
     tmem_relinquish();
@@ -755,9 +765,10 @@ __global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const Ll
   tc_fence_after();
   const uint32_t tmem = *tmem_base_s;
   const float invL = 1.f / misc[0];
-  if (tid < kLlaD) {
-    float ks = 0.f, vs = 0.f;
-    for (int p = 0; p < a.pieces; ++p) {
+  {
+    // (an empty piece has weight 0 and is skipped, whatever its record holds)
+    float ks = wts[0] == 0.f ? 0.f : wts[0] * ks0, vs = wts[0] == 0.f ? 0.f : wts[0] * vs0;
+    for (int p = 1; p < a.pieces; ++p) {
       if (wts[p] == 0.f) continue;
       const float* r = rec0 + (size_t)p * kLlaRecFloats;
       ks = fmaf(wts[p], r[kLlaRecKs + tid], ks);
@@ -766,21 +777,24 @@ __global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const Ll
     kb[tid] = ks * invL;
     vb[tid] = vs * invL;
   }
-  __syncthreads();
+  cp_async_wait_group1();   // this thread's part of D_KK has landed (D_KV may still be on its way)
+  __syncthreads();          // and everyone's
 
   const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
   constexpr uint32_t kIdUpd = idesc_bf16(kLlaD, kLlaD, false) | (1u << 13);   // 128 x 128 x 16, A negated
   const int r_ = tid;   // row a of S, TMEM lane a
   // ---- row a of S_KK + ridge I = D_KK / l - kbar kbar^T + ridge I into tensor
   // memory (D_KK is recorded column-major: entry [a][j] at j * 128 + a, so a
-  // warp's 32 rows read 128 contiguous bytes per column; 64 loads in flight)
+  // warp's 32 rows read 128 contiguous bytes per column): piece 0 from
+  // shared memory, any other piece from global memory, 64 loads in flight
 #pragma unroll 1
   for (int c64 = 0; c64 < 2; ++c64) {
     float sv[64];
+    const float w0 = wts[0];
 #pragma unroll
-    for (int j = 0; j < 64; ++j) sv[j] = 0.f;
+    for (int j = 0; j < 64; ++j) sv[j] = w0 == 0.f ? 0.f : w0 * Dkk_s[(64 * c64 + j) * kLlaD + r_];
 #pragma unroll 1
-    for (int p = 0; p < a.pieces; ++p) {
+    for (int p = 1; p < a.pieces; ++p) {
       const float w = wts[p];
       if (w == 0.f) continue;
       const float* col0 = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKK + (size_t)(64 * c64) * kLlaD + r_;
@@ -804,28 +818,28 @@ __global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const Ll
   tmem_wait_st();
   float rr_a = kb[r_] - __bfloat162float(a.q[orow + r_]);   // forward right-hand side of row a
   bool fine = true;
+  // x holds this row's entries in panel P's columns, fully updated.  The
+  // tensor-core update of panel P leaves out panel P + 1's columns (their
+  // rows are zero in its operand): those the row threads update themselves
+  // in fp32 right after issuing it (look-ahead), so panel P + 1 can be
+  // factored while the tensor cores update the rest.
+  float x[8];
+  {
+    uint32_t xr[8];
+    tmem_ld8(tmem + lane_off, xr);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[c] = __uint_as_float(xr[c]);
+  }
 #pragma unroll 1
   for (int P = 0; P < 16; ++P) {
     const int c0 = 8 * P;
-    bool w = true;
-    if (P > 0) w = mbar_wait_bounded(a.wait_ns, upd_done, (P - 1) & 1);   // S holds panel P - 1's update
-    tc_fence_after();
-    uint32_t xr[8];
-    tmem_ld8(tmem + lane_off + (uint32_t)c0, xr);
-    tmem_wait_ld();
-    float x[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) x[c] = __uint_as_float(xr[c]);
     if (r_ >= c0 && r_ < c0 + 8) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) d8[(r_ - c0) * 8 + c] = x[c];
       d8[64 + (r_ - c0)] = rr_a;
     }
-    if (!bar_and(1, kLlaSolveThreads, w)) {   // a wait ran out (reported)
-      fine = false;
-      if (r_ == 0) misc[3] = 1.f;
-      break;
-    }
+    bar_and(1, kLlaSolveThreads, true);
     // every row thread factors the diagonal block and solves L_PP z_P = r_P
     float dd[8][8], inv[8], zz[8];
 #pragma unroll
@@ -884,13 +898,19 @@ __global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const Ll
         inv_s[c0 + c] = inv[c];
       }
     }
-    if (P < 15) {
-      // the update's operand: rows below the panel's diagonal block, split
-      // into bf16 hi + mid + lo (16-byte chunk 0 of the row; the rest is zero)
+    const bool mma = P < 14;   // columns past panel P + 1 remain
+    // The previous panel's products are done: their operand may be
+    // rewritten, and panel P + 1's columns in tensor memory are current.
+    bool w = true;
+    if (P >= 1 && P <= 14) w = mbar_wait_bounded(a.wait_ns, upd_done, (P - 1) & 1);
+    if (mma && w) {
+      // the update's operand: rows below panel P + 1, split into bf16 hi +
+      // mid + lo (16-byte chunk 0 of the row; the rest is zero)
+      const bool live = r_ >= c0 + 16;
       uint32_t ph[4], pm[4], pl[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        const float v0 = r_ >= c0 + 8 ? l[2 * c] : 0.f, v1 = r_ >= c0 + 8 ? l[2 * c + 1] : 0.f;
+        const float v0 = live ? l[2 * c] : 0.f, v1 = live ? l[2 * c + 1] : 0.f;
         ph[c] = pack_bf16(v0, v1);
         const float m0 = v0 - bf16_lo_f(ph[c]), m1 = v1 - bf16_hi_f(ph[c]);
         pm[c] = pack_bf16(m0, m1);
@@ -901,17 +921,41 @@ __global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const Ll
       *reinterpret_cast<uint4*>(sm + Ly::kOp + Ly::kOpBytes + off) = make_uint4(pm[0], pm[1], pm[2], pm[3]);
       *reinterpret_cast<uint4*>(sm + Ly::kOp + 2 * Ly::kOpBytes + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
       fence_proxy_async_smem();
-      tc_fence_before();
-      bar_and(1, kLlaSolveThreads, true);   // every row of the operand is written
-      if (warp == 0) {
-        // S -= L L^T over six products of the parts (hi hi, hi mid, mid hi, hi lo, lo hi, mid mid)
-        tc_fence_after();
-        const uint64_t dh = smem_desc_sw128(smem_u32(sm + Ly::kOp), 16, 1024);
-        const uint64_t dm = dh + (uint64_t)(Ly::kOpBytes >> 4), dl = dh + (uint64_t)((2 * Ly::kOpBytes) >> 4);
-        lla_mma4_ss(tmem, dh, dh, dh, dm, dm, dh, dh, dl, kIdUpd, 1u);
-        tc_mma_ss(tmem, dl, dh, kIdUpd, 1u);
-        tc_mma_ss(tmem, dm, dm, kIdUpd, 1u);
-        tc_commit(upd_done);
+    }
+    tc_fence_before();
+    if (!bar_and(1, kLlaSolveThreads, w)) {   // the operand and this panel's L^T are written, or a wait ran out (reported)
+      fine = false;
+      if (r_ == 0) misc[3] = 1.f;
+      break;
+    }
+    if (mma && warp == 0) {
+      // S -= L L^T over six products of the parts (hi hi, hi mid, mid hi, hi lo, lo hi, mid mid)
+      tc_fence_after();
+      const uint64_t dh = smem_desc_sw128(smem_u32(sm + Ly::kOp), 16, 1024);
+      const uint64_t dm = dh + (uint64_t)(Ly::kOpBytes >> 4), dl = dh + (uint64_t)((2 * Ly::kOpBytes) >> 4);
+      lla_mma4_ss(tmem, dh, dh, dh, dm, dm, dh, dh, dl, kIdUpd, 1u);
+      tc_mma_ss(tmem, dl, dh, kIdUpd, 1u);
+      tc_mma_ss(tmem, dm, dm, kIdUpd, 1u);
+      tc_commit(upd_done);
+    }
+    if (P == 15) break;
+    // panel P + 1's columns, then this panel's part of their update
+    tc_fence_after();
+    {
+      uint32_t xr[8];
+      tmem_ld8(tmem + lane_off + (uint32_t)(c0 + 8), xr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 8; ++c) x[c] = __uint_as_float(xr[c]);
+    }
+    if (r_ >= c0 + 8) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float* lrow = Lt + c0 * kLlaLt + c0 + 8 + c;   // L[c0 + 8 + c][c0 + k] at k * kLlaLt
+        float v = x[c];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v = fmaf(-l[k], lrow[k * kLlaLt], v);
+        x[c] = v;
       }
     }
   }
@@ -978,23 +1022,39 @@ __global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const Ll
   __syncthreads();
   // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a: warp w
   // takes columns 32 w .. 32 w + 31, lane l rows 4 l .. 4 l + 3 of each (a
-  // column of D_KV is 512 contiguous bytes)
+  // column of D_KV is 512 contiguous bytes).  Every lane forms its 32
+  // partial dot products; a halving exchange across the lanes (16 + 8 + 4 +
+  // 2 + 1 shuffles) then leaves lane j with the sum of column 32 w + j.
   {
     const float4 rr = *reinterpret_cast<const float4*>(rho_s + 4 * lane);
-    auto dot4 = [&](const float* p4) {
-      const float4 v = *reinterpret_cast<const float4*>(p4);
-      return fmaf(v.x, rr.x, fmaf(v.y, rr.y, fmaf(v.z, rr.z, v.w * rr.w)));
-    };
-#pragma unroll 4
-    for (int k = 0; k < 32; ++k) {
-      const int col = 32 * warp + k;
-      float acc = wts[0] == 0.f ? 0.f : wts[0] * dot4(Dkv + col * kLlaD + 4 * lane);
-      for (int p = 1; p < a.pieces; ++p)
-        if (wts[p] != 0.f)
-          acc = fmaf(wts[p], dot4(rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + col * kLlaD + 4 * lane), acc);
-      acc = warp_sum(acc);
-      if (lane == 0) part[col] = acc;
+    auto dot4 = [&](const float4 v) { return fmaf(v.x, rr.x, fmaf(v.y, rr.y, fmaf(v.z, rr.z, v.w * rr.w))); };
+    float acc[32];
+    const float w0 = wts[0];
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      acc[k] = w0 == 0.f ? 0.f : w0 * dot4(*reinterpret_cast<const float4*>(Dkv + (32 * warp + k) * kLlaD + 4 * lane));
+#pragma unroll 1
+    for (int p = 1; p < a.pieces; ++p) {
+      const float wp = wts[p];
+      if (wp == 0.f) continue;
+      const float* src = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + 4 * lane;
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        acc[k] = fmaf(wp, dot4(__ldg(reinterpret_cast<const float4*>(src + (32 * warp + k) * kLlaD))), acc[k]);
     }
+    // step o: the lanes with bit o set keep the upper half of their columns
+    // and send the lower half to lane ^ o, the others the reverse
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < o; ++i) {
+        const float send = up ? acc[i] : acc[i + o];
+        const float keep = up ? acc[i + o] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    part[32 * warp + lane] = acc[0];
   }
   __syncthreads();
   store_out(tid, fmaf(vb[tid], 1.f + misc[1], -part[tid] * invL));

@@ -759,6 +759,7 @@ plx_status parallax_decode_plan_run_io(const plx_decode_plan* plan, const void* 
     L.a.q = dq;
     L.a.rho = dr;
     L.a.out = dout;
+    L.a.qr_early = 1;   // the host supplies q and rho: they are read before the previous grid ends
     return launch_decode(L, &plan->p, stream, kPdlAll, false);
   }
   const DecodeArgs& a = plan->L.a;
