@@ -54,6 +54,57 @@ struct BwdArgs {
   unsigned long long wait_ns;     // limit of one pipeline wait (0: give up unless complete)
 };
 
+// ------------------------------------------------------------- MMA issue
+// Several MMAs under one elect.sync, issued in argument order, each with its
+// own accumulate flag: the issuing warp pays tens of cycles per elect.sync
+// block, so the backward's many small products go out four at a time.
+__device__ __forceinline__ void bwd_mma_ss4(uint32_t d0, uint64_t a0, uint64_t b0, uint32_t c0, uint32_t d1,
+                                            uint64_t a1, uint64_t b1, uint32_t c1, uint32_t d2, uint64_t a2,
+                                            uint64_t b2, uint32_t c2, uint32_t d3, uint64_t a3, uint64_t b3,
+                                            uint32_t c3, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1, p2, p3, e;\n\t"
+      "setp.ne.b32 p0, %12, 0;\n\tsetp.ne.b32 p1, %13, 0;\n\tsetp.ne.b32 p2, %14, 0;\n\tsetp.ne.b32 p3, %15, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %16, p0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], %4, %5, %16, p1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%6], %7, %8, %16, p2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%9], %10, %11, %16, p3;\n\t}" ::"r"(d0),
+      "l"(a0), "l"(b0), "r"(d1), "l"(a1), "l"(b1), "r"(d2), "l"(a2), "l"(b2), "r"(d3), "l"(a3), "l"(b3), "r"(c0),
+      "r"(c1), "r"(c2), "r"(c3), "r"(idesc)
+      : "memory");
+}
+
+// The same with A in tensor memory.
+__device__ __forceinline__ void bwd_mma_ts4(uint32_t d0, uint32_t a0, uint64_t b0, uint32_t c0, uint32_t d1,
+                                            uint32_t a1, uint64_t b1, uint32_t c1, uint32_t d2, uint32_t a2,
+                                            uint64_t b2, uint32_t c2, uint32_t d3, uint32_t a3, uint64_t b3,
+                                            uint32_t c3, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1, p2, p3, e;\n\t"
+      "setp.ne.b32 p0, %12, 0;\n\tsetp.ne.b32 p1, %13, 0;\n\tsetp.ne.b32 p2, %14, 0;\n\tsetp.ne.b32 p3, %15, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %16, p0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], [%4], %5, %16, p1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%6], [%7], %8, %16, p2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%9], [%10], %11, %16, p3;\n\t}" ::"r"(d0),
+      "r"(a0), "l"(b0), "r"(d1), "r"(a1), "l"(b1), "r"(d2), "r"(a2), "l"(b2), "r"(d3), "r"(a3), "l"(b3), "r"(c0),
+      "r"(c1), "r"(c2), "r"(c3), "r"(idesc)
+      : "memory");
+}
+
+__device__ __forceinline__ void bwd_mma_ts2(uint32_t d0, uint32_t a0, uint64_t b0, uint32_t c0, uint32_t d1,
+                                            uint32_t a1, uint64_t b1, uint32_t c1, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p0, p1, e;\n\t"
+      "setp.ne.b32 p0, %6, 0;\n\tsetp.ne.b32 p1, %7, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %8, p0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%3], [%4], %5, %8, p1;\n\t}" ::"r"(d0),
+      "r"(a0), "l"(b0), "r"(d1), "r"(a1), "l"(b1), "r"(c0), "r"(c1), "r"(idesc)
+      : "memory");
+}
+
 // ---------------------------------------------------------------- per row
 // One warp per row: Gbar = g.vbar, Delta = g.out.  out is the forward output
 // in its own dtype (the loss saw those values).  The record holds the
@@ -302,20 +353,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     auto value_products = [&](int jp) {
       const int sp = jp % S;
       const uint64_t kts = dkt + (uint64_t)((sp * Ly::kTile64) >> 4);
+      // 16 keys per step: 8 TMEM columns of packed bf16 pairs, 16 rows of K;
+      // two steps per issue block
 #pragma unroll
-      for (int kk = 0; kk < kPfBN / 16; ++kk) {
-        // 16 keys per step: 8 TMEM columns of packed bf16 pairs, 16 rows of K
-        const uint64_t kd = kts + (uint64_t)(kk * 16 * 128 / 16);
-        tc_mma_ts(tmem + kBwAcc0, tmem + kBwDS + kk * 8, kd, kIdT, (jp > 0 || kk > 0) ? 1u : 0u);
-        tc_mma_ts(tmem + kBwAcc1, tmem + kBwDA + kk * 8, kd, kIdT, (jp > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < kPfBN / 16; kk += 2) {
+        const uint64_t kd0 = kts + (uint64_t)(kk * 16 * 128 / 16), kd1 = kd0 + (uint64_t)(16 * 128 / 16);
+        const uint32_t c0 = (jp > 0 || kk > 0) ? 1u : 0u;
+        bwd_mma_ts4(tmem + kBwAcc0, tmem + kBwDS + kk * 8, kd0, c0, tmem + kBwAcc1, tmem + kBwDA + kk * 8, kd0, c0,
+                    tmem + kBwAcc0, tmem + kBwDS + kk * 8 + 8, kd1, 1u, tmem + kBwAcc1, tmem + kBwDA + kk * 8 + 8, kd1,
+                    1u, kIdT);
       }
       if (jp < split_tiles) {   // lo parts: keys 32h.. of dS at D + 32h, of dA at D + 32h + 16
 #pragma unroll
-        for (int kk = 0; kk < kPfBN / 16; ++kk) {
-          const uint64_t kd = kts + (uint64_t)(kk * 16 * 128 / 16);
-          const uint32_t pc = kBwD + 32u * (kk >> 1) + 8u * (kk & 1);
-          tc_mma_ts(tmem + kBwAcc0, tmem + pc, kd, kIdT, 1u);
-          tc_mma_ts(tmem + kBwAcc1, tmem + pc + 16, kd, kIdT, 1u);
+        for (int kk = 0; kk < kPfBN / 16; kk += 2) {
+          const uint64_t kd0 = kts + (uint64_t)(kk * 16 * 128 / 16), kd1 = kd0 + (uint64_t)(16 * 128 / 16);
+          const uint32_t pc = kBwD + 32u * (kk >> 1);   // kk even: 8 (kk & 1) = 0, then + 8 for kk + 1
+          bwd_mma_ts4(tmem + kBwAcc0, tmem + pc, kd0, 1u, tmem + kBwAcc1, tmem + pc + 16, kd0, 1u, tmem + kBwAcc0,
+                      tmem + pc + 8, kd1, 1u, tmem + kBwAcc1, tmem + pc + 24, kd1, 1u, kIdT);
         }
       }
       tc_commit(dd_free);
@@ -338,13 +392,23 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
         const uint64_t dks = dk + (uint64_t)((s * Ly::kTile64) >> 4);
         const uint64_t dvs = dv + (uint64_t)((s * Ly::kTile64) >> 4);
+        // S, A, D for k-steps kk = 0..7 in that order, four products per issue block
 #pragma unroll
-        for (int kk = 0; kk < kPfD / 16; ++kk) {
-          const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTile128 / 2 / 16) + (kk & 3) * 2);
-          const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2);
-          tc_mma_ss(tmem + kBwS, dq + oa, dks + ob, kIdS, kk > 0);
-          tc_mma_ss(tmem + kBwA, dr + oa, dks + ob, kIdS, kk > 0);
-          tc_mma_ss(tmem + kBwD, dg + oa, dvs + ob, kIdS, kk > 0);
+        for (int g4 = 0; g4 < 3 * (kPfD / 16) / 4; ++g4) {
+          uint32_t d[4], c[4];
+          uint64_t aa[4], bb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = 4 * g4 + u, kk = i / 3, which = i % 3;
+            const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTile128 / 2 / 16) + (kk & 3) * 2);
+            const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2);
+            d[u] = tmem + (which == 0 ? kBwS : which == 1 ? kBwA : kBwD);
+            aa[u] = (which == 0 ? dq : which == 1 ? dr : dg) + oa;
+            bb[u] = (which == 2 ? dvs : dks) + ob;
+            c[u] = kk > 0 ? 1u : 0u;
+          }
+          bwd_mma_ss4(d[0], aa[0], bb[0], c[0], d[1], aa[1], bb[1], c[1], d[2], aa[2], bb[2], c[2], d[3], aa[3], bb[3],
+                      c[3], kIdS);
         }
         tc_commit(sad_full);
         tc_commit(&v_empty[s]);   // V(j) only enters D
@@ -630,22 +694,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       const uint64_t tq = smem_desc_sw128(stp + Ly::kStQ, Ly::kTile64 / 2, 1024);
       const uint64_t tr = smem_desc_sw128(stp + Ly::kStR, Ly::kTile64 / 2, 1024);
       const uint64_t tg = smem_desc_sw128(stp + Ly::kStG, Ly::kTile64 / 2, 1024);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        // 16 queries per step.  U of queries 16kk.. sits in columns 16kk..16kk+7
-        // of the S^T block (its lo parts in 16kk+8..), dS / dA in 8kk..8kk+7 of
-        // their own blocks (lo parts: 16kk.. and 16kk+8.. of the A^T block).
-        const int kk = q + 2 * h;
-        const uint64_t ko = (uint64_t)(kk * 16 * 128 / 16);
-        const uint32_t acc = (ip > 0 || kk > 0) ? 1u : 0u;
-        tc_mma_ts(tmem + kBwAcc1, tmem + kBwS + 16 * kk, tg + ko, kIdT, acc);
-        tc_mma_ts(tmem + kBwAcc0, tmem + kBwDS + kk * 8, tq + ko, kIdT, acc);
-        tc_mma_ts(tmem + kBwAcc0, tmem + kBwDA + kk * 8, tr + ko, kIdT, 1u);
-        if (split_of(ip)) {
-          tc_mma_ts(tmem + kBwAcc1, tmem + kBwS + 16 * kk + 8, tg + ko, kIdT, 1u);
-          tc_mma_ts(tmem + kBwAcc0, tmem + kBwA + 16 * kk, tq + ko, kIdT, 1u);
-          tc_mma_ts(tmem + kBwAcc0, tmem + kBwA + 16 * kk + 8, tr + ko, kIdT, 1u);
-        }
+      // 16 queries per step.  U of queries 16kk.. sits in columns 16kk..16kk+7
+      // of the S^T block (its lo parts in 16kk+8..), dS / dA in 8kk..8kk+7 of
+      // their own blocks (lo parts: 16kk.. and 16kk+8.. of the A^T block).
+      // Steps kk = q and q + 2; the products go out four (or two) per issue
+      // block in the order: hi parts of kk = q, then of q + 2, then the lo parts.
+      const int k0 = q, k1 = q + 2;
+      const uint64_t ko0 = (uint64_t)(k0 * 16 * 128 / 16), ko1 = (uint64_t)(k1 * 16 * 128 / 16);
+      const uint32_t acc0 = (ip > 0 || k0 > 0) ? 1u : 0u;   // k1 > 0: always accumulates
+      bwd_mma_ts4(tmem + kBwAcc1, tmem + kBwS + 16 * k0, tg + ko0, acc0, tmem + kBwAcc0, tmem + kBwDS + k0 * 8,
+                  tq + ko0, acc0, tmem + kBwAcc0, tmem + kBwDA + k0 * 8, tr + ko0, 1u, tmem + kBwAcc1,
+                  tmem + kBwS + 16 * k1, tg + ko1, 1u, kIdT);
+      bwd_mma_ts2(tmem + kBwAcc0, tmem + kBwDS + k1 * 8, tq + ko1, 1u, tmem + kBwAcc0, tmem + kBwDA + k1 * 8,
+                  tr + ko1, 1u, kIdT);
+      if (split_of(ip)) {
+        bwd_mma_ts4(tmem + kBwAcc1, tmem + kBwS + 16 * k0 + 8, tg + ko0, 1u, tmem + kBwAcc0, tmem + kBwA + 16 * k0,
+                    tq + ko0, 1u, tmem + kBwAcc0, tmem + kBwA + 16 * k0 + 8, tr + ko0, 1u, tmem + kBwAcc1,
+                    tmem + kBwS + 16 * k1 + 8, tg + ko1, 1u, kIdT);
+        bwd_mma_ts2(tmem + kBwAcc0, tmem + kBwA + 16 * k1, tq + ko1, 1u, tmem + kBwAcc0, tmem + kBwA + 16 * k1 + 8,
+                    tr + ko1, 1u, kIdT);
       }
       if (q == 1) {
         tc_commit(dd_free);
@@ -674,11 +741,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint64_t br = smem_desc_sw128(st + Ly::kStR, 16, 1024);
         const uint64_t bg = smem_desc_sw128(st + Ly::kStG, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kPfD / 16; ++kk) {
-          const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTile128 / 2 / 16) + (kk & 3) * 2);
-          const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2);
-          tc_mma_ss(tmem + kBwA, dk + oa, br + ob, kIdS, kk > 0);
-          tc_mma_ss(tmem + kBwD, dvv + oa, bg + ob, kIdS, kk > 0);
+        for (int kk = 0; kk < kPfD / 16; kk += 2) {   // A^T, D^T of steps kk and kk + 1 per issue block
+          const uint64_t oa0 = (uint64_t)((kk >> 2) * (Ly::kTile128 / 2 / 16) + (kk & 3) * 2), oa1 = oa0 + 2;
+          const uint64_t ob0 = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2), ob1 = ob0 + 2;
+          const uint32_t c0 = kk > 0 ? 1u : 0u;
+          bwd_mma_ss4(tmem + kBwA, dk + oa0, br + ob0, c0, tmem + kBwD, dvv + oa0, bg + ob0, c0, tmem + kBwA,
+                      dk + oa1, br + ob1, 1u, tmem + kBwD, dvv + oa1, bg + ob1, 1u, kIdS);
         }
         // offsets: A^T -= 1 + abar (slab columns 16..31), D^T -= Gbar (32..47)
         const uint64_t bsl = smem_desc_sw128(st + Ly::kStSlab, 16, 1024);
@@ -691,10 +759,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (it < N) {
         const uint64_t bq = smem_desc_sw128(st + Ly::kStQ, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < kPfD / 16; ++kk) {
-          const uint64_t oa = (uint64_t)((kk >> 2) * (Ly::kTile128 / 2 / 16) + (kk & 3) * 2);
-          const uint64_t ob = (uint64_t)((kk >> 2) * (Ly::kTile64 / 2 / 16) + (kk & 3) * 2);
-          tc_mma_ss(tmem + kBwS, dk + oa, bq + ob, kIdS, kk > 0);
+        for (int kk = 0; kk < kPfD / 16; kk += 4) {   // four k-steps per issue block
+          uint64_t aa[4], bb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            aa[u] = dk + (uint64_t)(((kk + u) >> 2) * (Ly::kTile128 / 2 / 16) + ((kk + u) & 3) * 2);
+            bb[u] = bq + (uint64_t)(((kk + u) >> 2) * (Ly::kTile64 / 2 / 16) + ((kk + u) & 3) * 2);
+          }
+          bwd_mma_ss4(tmem + kBwS, aa[0], bb[0], kk > 0 ? 1u : 0u, tmem + kBwS, aa[1], bb[1], 1u, tmem + kBwS, aa[2],
+                      bb[2], 1u, tmem + kBwS, aa[3], bb[3], 1u, kIdS);
         }
         tc_mma_ss(tmem + kBwS, dones, smem_desc_sw128(st + Ly::kStSlab, 16, 1024), kIdS, 1u);   // S^T -= lse2 / c
         tc_commit(sad_full);
