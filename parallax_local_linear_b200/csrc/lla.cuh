@@ -80,6 +80,7 @@ struct LlaArgs {
   int B, Hq, Hkv, group, kv_len, paged, num_pages, max_pages, pieces;
   float scale_log2, ridge;
   int out_bf16;
+  int fused;                       // 1 (one piece per head): the moments kernel solves in place
   unsigned long long wait_ns;      // limit of one pipeline wait
 };
 
@@ -176,6 +177,555 @@ __host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, bool a_mn_maj
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
+// ---------------------------------------------------------------- solve
+// One CTA per (sequence, query head): four row warps, row a in TMEM lane a.
+// S = S_KK + ridge I (fp32) lives in tensor memory, row a in lane a.  Blocked
+// right-looking Cholesky, 8 columns per panel: every row thread reads its 8
+// panel entries; the diagonal block goes through shared memory and each
+// thread factors it redundantly (no further synchronisation), solves its own
+// row against it and carries the forward substitution z = L^-1 (kbar - q)
+// along; the trailing update S -= L_P L_P^T runs on the tensor cores, with
+// each panel value split into three bf16 parts (hi + mid + lo carries the
+// fp32 value) and six products (hi hi, hi mid, mid hi, hi lo, lo hi, mid
+// mid) of a 128 x 128 x 16 MMA with A negated, issued by the first warp once
+// a named barrier says the panel is written.  The factor also goes to shared
+// memory, transposed, for the blocked back substitution L^T rho = z, whose
+// diagonal blocks are inverted all at once (one column per thread) first.
+// D_KV comes into shared memory by cp.async while the factorisation runs.
+constexpr int kLlaSolveThreads = 128;
+constexpr int kLlaLt = kLlaD + 4;                // row stride of L^T (padding against bank conflicts)
+
+struct LlaSolveLayout {
+  static constexpr int kDkv = 0;                              // float [128][128]: D_KV of piece 0
+  static constexpr int kLt = kDkv + kLlaD * kLlaD * 4;        // float [128][kLlaLt]: L^T
+  static constexpr int kOpBytes = kLlaD * 128;                // bf16 [128][64], 128-byte swizzle (16 columns used)
+  static constexpr int kOp = (kLt + kLlaD * kLlaLt * 4 + 1023) & ~1023;   // three parts: hi, mid, lo
+  static constexpr int kD8 = kOp + 3 * kOpBytes;              // float [8][8] diagonal block + [8] its z rhs
+  static constexpr int kMinv = kD8 + 72 * 4;                  // float [16][8][8]: (L_II^T)^-1
+  static constexpr int kVec = kMinv + 16 * 64 * 4;            // float [7][128]: kbar, vbar, rho, r, z, part, 1/L_kk
+  static constexpr int kWts = kVec + 7 * kLlaD * 4;           // float [kLlaMaxPieces]
+  static constexpr int kMisc = kWts + kLlaMaxPieces * 4;      // float [8]: l, kbar.rho, bad, stop, ...
+  static constexpr int kBar = (kMisc + 32 + 7) & ~7;          // upd_done, drain
+  static constexpr int kTmem = kBar + 24;
+  static constexpr int kBytes = kTmem + 16 + 1024;
+};
+
+// The solve inside the moments kernel (one piece per head) uses the K/V
+// ring once its last products are done: no D_KV copy (it stays in tensor
+// memory) and no tensor-memory allocation of its own.
+struct LlaFusedSolveLayout {
+  static constexpr int kLt = 0;
+  static constexpr int kOpBytes = LlaSolveLayout::kOpBytes;
+  static constexpr int kOp = (kLt + kLlaD * kLlaLt * 4 + 1023) & ~1023;
+  static constexpr int kD8 = kOp + 3 * kOpBytes;
+  static constexpr int kMinv = kD8 + 72 * 4;
+  static constexpr int kVec = kMinv + 16 * 64 * 4;
+  static constexpr int kWts = kVec + 7 * kLlaD * 4;
+  static constexpr int kMisc = kWts + kLlaMaxPieces * 4;
+  static constexpr int kBar = (kMisc + 32 + 7) & ~7;
+  static constexpr int kBytes = kBar + 16;
+};
+static_assert(LlaFusedSolveLayout::kBytes <= kLlaStages * LlaLayout::kStageBytes, "the fused solve fits in the ring");
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// 8 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+
+// Cholesky of the 8 x 8 block d (lower triangle used) in place, with the
+// reciprocals of the diagonal; false if a pivot is not positive.
+__device__ __forceinline__ bool lla_chol8(float (&d)[8][8], float (&inv)[8]) {
+  bool ok = true;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float akk = d[k][k];
+    ok = ok && akk > 0.f && isfinite(akk);
+    const float invd = rsqrtf(akk);
+    d[k][k] = akk * invd;
+    inv[k] = invd;
+#pragma unroll
+    for (int i = k + 1; i < 8; ++i) d[i][k] *= invd;
+#pragma unroll
+    for (int i = k + 1; i < 8; ++i)
+#pragma unroll
+      for (int jj = k + 1; jj <= i; ++jj) d[i][jj] = fmaf(-d[i][k], d[jj][k], d[i][jj]);
+  }
+  return ok;
+}
+
+// The factorisation, the two triangular solves and the output of one
+// (sequence, query head), by 128 threads in four warps: thread tid owns row
+// tid of the system, in tensor memory lane tid (warp w of the four must be
+// a warp whose id is w mod 4), columns 0..127 of `tmem` holding
+// S_KK + ridge I on entry; kbar, vbar and l are in place.  kFused: the
+// threads are four warps of the moments kernel, D_KV is in tensor memory
+// columns 128..255 (row a in lane a) and the tensor memory is freed by that
+// kernel; otherwise D_KV of piece 0 is in shared memory (Dkv, column-major)
+// and the other pieces' in their records.  bar_row and bar_all are the
+// named barriers of the 128 threads (bar_all 0 when they are the whole CTA).
+template <bool kFused, class Ly>
+__device__ __forceinline__ void lla_solve_body(const LlaArgs& a, uint8_t* sm, const uint32_t tmem, const int tid,
+                                               const int warp, const int lane, const uint32_t bar_row,
+                                               const uint32_t bar_all, const float* Dkv, const float* rec0,
+                                               const float invL, const size_t orow) {
+  float* Lt = reinterpret_cast<float*>(sm + Ly::kLt);     // Lt[k * kLlaLt + i] = L[i][k]
+  float* d8 = reinterpret_cast<float*>(sm + Ly::kD8);     // [8][8] diagonal block, then [8] its rhs
+  float* kb = reinterpret_cast<float*>(sm + Ly::kVec);    // kbar
+  float* vb = kb + kLlaD;                                 // vbar
+  float* rho_s = vb + kLlaD;                              // rho*
+  float* rb = rho_s + kLlaD;                              // back substitution right-hand side
+  float* z_s = rb + kLlaD;                                // z = L^-1 (kbar - q)
+  float* part = z_s + kLlaD;                              // D_KV^T rho*
+  float* inv_s = part + kLlaD;                            // 1 / L[k][k]
+  float* minv = reinterpret_cast<float*>(sm + Ly::kMinv); // [I][c][r]: (L_II^T)^-1
+  const float* wts = reinterpret_cast<const float*>(sm + Ly::kWts);   // piece weights 2^(m_j - M)
+  float* misc = reinterpret_cast<float*>(sm + Ly::kMisc); // [0] l, [1] kbar . rho*, [2] bad pivot, [3] stop
+  uint64_t* upd_done = reinterpret_cast<uint64_t*>(sm + Ly::kBar);   // the panel's update is done
+  uint64_t* drain = upd_done + 1;                                    // every product has completed
+  auto store_out = [&](int i, float v) {
+    if (a.out_bf16)
+      reinterpret_cast<__nv_bfloat16*>(a.out)[orow + i] = __float2bfloat16_rn(v);
+    else
+      reinterpret_cast<float*>(a.out)[orow + i] = v;
+  };
+  auto sync_all = [&] { asm volatile("bar.sync %0, %1;" ::"r"(bar_all), "n"(kLlaSolveThreads) : "memory"); };
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  constexpr uint32_t kIdUpd = idesc_bf16(kLlaD, kLlaD, false) | (1u << 13);   // 128 x 128 x 16, A negated
+  const int r_ = tid;   // row a of S, TMEM lane a
+  float rr_a = kb[r_] - __bfloat162float(a.q[orow + r_]);   // forward right-hand side of row a
+  bool fine = true;
+  // x holds this row's entries in panel P's columns, fully updated.  The
+  // tensor-core update of panel P leaves out panel P + 1's columns (their
+  // rows are zero in its operand): those the row threads update themselves
+  // in fp32 right after issuing it (look-ahead), so panel P + 1 can be
+  // factored while the tensor cores update the rest.
+  float x[8];
+  {
+    uint32_t xr[8];
+    tmem_ld8(tmem + lane_off, xr);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) x[c] = __uint_as_float(xr[c]);
+  }
+#pragma unroll 1
+  for (int P = 0; P < 16; ++P) {
+    const int c0 = 8 * P;
+    if (r_ >= c0 && r_ < c0 + 8) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) d8[(r_ - c0) * 8 + c] = x[c];
+      d8[64 + (r_ - c0)] = rr_a;
+    }
+    bar_and(bar_row, kLlaSolveThreads, true);
+    // every row thread factors the diagonal block and solves L_PP z_P = r_P
+    float dd[8][8], inv[8], zz[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) dd[i][c] = d8[i * 8 + c];
+    const bool ok = lla_chol8(dd, inv);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      float v = d8[64 + c];
+#pragma unroll
+      for (int m = 0; m < c; ++m) v = fmaf(-dd[c][m], zz[m], v);
+      zz[c] = v * inv[c];
+    }
+    if (!ok) {   // not numerically positive definite (every row thread sees it)
+      fine = false;
+      if (r_ == 0) {
+        misc[2] = 1.f;
+        misc[3] = 1.f;
+      }
+      break;
+    }
+    // this row's entries of L in the panel
+    float l[8];
+    if (r_ >= c0 + 8) {   // below the panel's diagonal block: l L_PP^T = x
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float v = x[c];
+#pragma unroll
+        for (int m = 0; m < c; ++m) v = fmaf(-l[m], dd[c][m], v);
+        l[c] = v * inv[c];
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) rr_a = fmaf(-l[c], zz[c], rr_a);
+    } else if (r_ >= c0) {   // a row of the diagonal block: that row of L_PP
+      const int ri = r_ - c0;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        float v = 0.f;
+#pragma unroll
+        for (int i = c; i < 8; ++i) v = i == ri ? dd[i][c] : v;
+        l[c] = v;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) l[c] = 0.f;
+    }
+    if (r_ >= c0) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) Lt[(c0 + c) * kLlaLt + r_] = l[c];
+    }
+    if (r_ == c0) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        z_s[c0 + c] = zz[c];
+        inv_s[c0 + c] = inv[c];
+      }
+    }
+    const bool mma = P < 14;   // columns past panel P + 1 remain
+    // The previous panel's products are done: their operand may be
+    // rewritten, and panel P + 1's columns in tensor memory are current.
+    bool w = true;
+    if (P >= 1 && P <= 14) w = mbar_wait_bounded(a.wait_ns, upd_done, (P - 1) & 1);
+    if (mma && w) {
+      // the update's operand: rows below panel P + 1, split into bf16 hi +
+      // mid + lo (16-byte chunk 0 of the row; the rest is zero)
+      const bool live = r_ >= c0 + 16;
+      uint32_t ph[4], pm[4], pl[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const float v0 = live ? l[2 * c] : 0.f, v1 = live ? l[2 * c + 1] : 0.f;
+        ph[c] = pack_bf16(v0, v1);
+        const float m0 = v0 - bf16_lo_f(ph[c]), m1 = v1 - bf16_hi_f(ph[c]);
+        pm[c] = pack_bf16(m0, m1);
+        pl[c] = pack_bf16(m0 - bf16_lo_f(pm[c]), m1 - bf16_hi_f(pm[c]));
+      }
+      const int off = r_ * 128 + ((r_ & 7) << 4);   // chunk 0 of row a, swizzled
+      *reinterpret_cast<uint4*>(sm + Ly::kOp + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
+      *reinterpret_cast<uint4*>(sm + Ly::kOp + Ly::kOpBytes + off) = make_uint4(pm[0], pm[1], pm[2], pm[3]);
+      *reinterpret_cast<uint4*>(sm + Ly::kOp + 2 * Ly::kOpBytes + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    if (!bar_and(bar_row, kLlaSolveThreads, w)) {   // the operand and this panel's L^T are written, or a wait ran out (reported)
+      fine = false;
+      if (r_ == 0) misc[3] = 1.f;
+      break;
+    }
+    if (mma && warp == 0) {
+      // S -= L L^T over six products of the parts (hi hi, hi mid, mid hi, hi lo, lo hi, mid mid)
+      tc_fence_after();
+      const uint64_t dh = smem_desc_sw128(smem_u32(sm + Ly::kOp), 16, 1024);
+      const uint64_t dm = dh + (uint64_t)(Ly::kOpBytes >> 4), dl = dh + (uint64_t)((2 * Ly::kOpBytes) >> 4);
+      lla_mma4_ss(tmem, dh, dh, dh, dm, dm, dh, dh, dl, kIdUpd, 1u);
+      tc_mma_ss(tmem, dl, dh, kIdUpd, 1u);
+      tc_mma_ss(tmem, dm, dm, kIdUpd, 1u);
+      tc_commit(upd_done);
+    }
+    if (P == 15) break;
+    // panel P + 1's columns, then this panel's part of their update
+    tc_fence_after();
+    {
+      uint32_t xr[8];
+      tmem_ld8(tmem + lane_off + (uint32_t)(c0 + 8), xr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 8; ++c) x[c] = __uint_as_float(xr[c]);
+    }
+    if (r_ >= c0 + 8) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const float* lrow = Lt + c0 * kLlaLt + c0 + 8 + c;   // L[c0 + 8 + c][c0 + k] at k * kLlaLt
+        float v = x[c];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v = fmaf(-l[k], lrow[k * kLlaLt], v);
+        x[c] = v;
+      }
+    }
+  }
+  if (warp == 0) {   // every product issued completes before tensor memory is freed
+    tc_commit(drain);
+    __syncwarp();
+    mbar_wait_drain(drain, 0);
+    __syncwarp();
+  }
+  tc_fence_before();
+  sync_all();
+  tc_fence_after();
+  if constexpr (!kFused) {
+    if (warp == 0) tmem_dealloc(tmem, 128);
+  }
+  if (!fine) {   // (a wait that ran out has reported itself)
+    if constexpr (!kFused) cp_async_wait_all();
+    if (tid == 0 && misc[2] != 0.f) report_error(PLX_DEVERR_SINGULAR_BIT);
+    store_out(tid, vb[tid]);   // rho* = 0: the output falls back to vbar
+    if (a.rho) a.rho[orow + tid] = 0.f;
+    return;
+  }
+  // ---- L^T rho = z.  First the inverses of the transposed diagonal blocks,
+  // one column per thread: column j of (L_II^T)^-1 for I = tid / 8, j = tid % 8.
+  {
+    const int I = tid >> 3, j = tid & 7;
+    float xx[8];
+#pragma unroll
+    for (int c = 7; c >= 0; --c) {
+      float v = c == j ? 1.f : 0.f;
+#pragma unroll
+      for (int rr2 = c + 1; rr2 < 8; ++rr2) v = fmaf(-Lt[(8 * I + c) * kLlaLt + 8 * I + rr2], xx[rr2], v);
+      xx[c] = v * inv_s[8 * I + c];
+      minv[I * 64 + c * 8 + j] = xx[c];
+    }
+    rb[r_] = z_s[r_];
+  }
+  sync_all();
+  // Then blockwise from the last block: rho_I = (L_II^T)^-1 r_I (eight
+  // threads), and every row above takes L_IJ^T rho_I off its r_J.
+#pragma unroll 1
+  for (int I = 15; I >= 0; --I) {
+    if (r_ < 8) {
+      float t = 0.f;
+#pragma unroll
+      for (int rr2 = 0; rr2 < 8; ++rr2) t = fmaf(minv[I * 64 + r_ * 8 + rr2], rb[8 * I + rr2], t);
+      rho_s[8 * I + r_] = t;
+    }
+    sync_all();
+    if (r_ < 8 * I) {
+      float t = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) t = fmaf(Lt[r_ * kLlaLt + 8 * I + c], rho_s[8 * I + c], t);
+      rb[r_] -= t;
+    }
+    sync_all();
+  }
+  if (tid < 32) {
+    float kr = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) kr = fmaf(kb[tid + 32 * u], rho_s[tid + 32 * u], kr);
+    kr = warp_sum(kr);
+    if (tid == 0) misc[1] = kr;
+  }
+  if constexpr (!kFused) cp_async_wait_all();
+  sync_all();
+  if constexpr (kFused) {
+  // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a with
+  // D_KV in tensor memory (columns 128..255, row a in lane a): thread a
+  // scales its row by rho*_a; per 32-column chunk the halving exchange
+  // leaves lane j with the warp's sum of column j, and the four warps'
+  // sums meet in shared memory (the inverse blocks' place, free by now).
+  {
+    const float ra = rho_s[tid];
+    float* wsum = minv;   // [4][128]
+    tc_fence_after();
+#pragma unroll 1
+    for (int c32 = 0; c32 < 4; ++c32) {
+      uint32_t rv[32];
+      tmem_ld32(tmem + lane_off + (uint32_t)(kLlaD + 32 * c32), rv);
+      tmem_wait_ld();
+      float acc[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) acc[k] = __uint_as_float(rv[k]) * ra;
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) {
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < o; ++i) {
+          const float send = up ? acc[i] : acc[i + o];
+          const float keep = up ? acc[i + o] : acc[i];
+          acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      wsum[warp * kLlaD + 32 * c32 + lane] = acc[0];
+    }
+    sync_all();
+    part[tid] = (wsum[tid] + wsum[kLlaD + tid]) + (wsum[2 * kLlaD + tid] + wsum[3 * kLlaD + tid]);
+  }
+  } else {
+  // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a: warp w
+  // takes columns 32 w .. 32 w + 31, lane l rows 4 l .. 4 l + 3 of each (a
+  // column of D_KV is 512 contiguous bytes).  Every lane forms its 32
+  // partial dot products; a halving exchange across the lanes (16 + 8 + 4 +
+  // 2 + 1 shuffles) then leaves lane j with the sum of column 32 w + j.
+  {
+    const float4 rr = *reinterpret_cast<const float4*>(rho_s + 4 * lane);
+    auto dot4 = [&](const float4 v) { return fmaf(v.x, rr.x, fmaf(v.y, rr.y, fmaf(v.z, rr.z, v.w * rr.w))); };
+    float acc[32];
+    const float w0 = wts[0];
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      acc[k] = w0 == 0.f ? 0.f : w0 * dot4(*reinterpret_cast<const float4*>(Dkv + (32 * warp + k) * kLlaD + 4 * lane));
+#pragma unroll 1
+    for (int p = 1; p < a.pieces; ++p) {
+      const float wp = wts[p];
+      if (wp == 0.f) continue;
+      const float* src = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + 4 * lane;
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        acc[k] = fmaf(wp, dot4(__ldg(reinterpret_cast<const float4*>(src + (32 * warp + k) * kLlaD))), acc[k]);
+    }
+    // step o: the lanes with bit o set keep the upper half of their columns
+    // and send the lower half to lane ^ o, the others the reverse
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < o; ++i) {
+        const float send = up ? acc[i] : acc[i + o];
+        const float keep = up ? acc[i + o] : acc[i];
+        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    part[32 * warp + lane] = acc[0];
+  }
+  }
+  sync_all();
+  store_out(tid, fmaf(vb[tid], 1.f + misc[1], -part[tid] * invL));
+  if (a.rho) a.rho[orow + tid] = rho_s[tid];
+}
+
+// The in-place solve of the moments kernel, kept out of line so that the
+// moments loop keeps its own register allocation.
+__device__ __noinline__ void lla_fused_solve(const LlaArgs& a, uint8_t* sm, const uint32_t tmem, const int tid,
+                                             const int warp, const int lane, const float invL, const size_t orow) {
+  lla_solve_body<true, LlaFusedSolveLayout>(a, sm, tmem, tid, warp, lane, 7, 8, nullptr, nullptr, invL, orow);
+}
+
+__global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const LlaArgs a) {
+  using Ly = LlaSolveLayout;
+  extern __shared__ uint8_t smem_raw_s[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_s) + 1023) & ~uintptr_t(1023));
+  float* Dkv = reinterpret_cast<float*>(sm + Ly::kDkv);   // column-major as recorded
+  float* Lt = reinterpret_cast<float*>(sm + Ly::kLt);     // D_KK is staged where L^T goes later
+  float* kb = reinterpret_cast<float*>(sm + Ly::kVec);    // kbar
+  float* vb = kb + kLlaD;                                 // vbar
+  float* wts = reinterpret_cast<float*>(sm + Ly::kWts);   // piece weights 2^(m_j - M)
+  float* misc = reinterpret_cast<float*>(sm + Ly::kMisc); // [0] l, [1] kbar . rho*, [2] bad pivot, [3] stop
+  uint64_t* upd_done = reinterpret_cast<uint64_t*>(sm + Ly::kBar);   // the panel's update is done
+  uint64_t* drain = upd_done + 1;                                    // every product has completed
+  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kTmem);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x, b = bh / a.Hq;
+  const size_t orow = (size_t)bh * kLlaD;
+  // Launched with a programmatic dependency on the moments grid: the records
+  // are read only after it has completed.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int len = lla_seq_len(a, b);
+  auto store_out = [&](int i, float v) {
+    if (a.out_bf16)
+      reinterpret_cast<__nv_bfloat16*>(a.out)[orow + i] = __float2bfloat16_rn(v);
+    else
+      reinterpret_cast<float*>(a.out)[orow + i] = v;
+  };
+  if (len == 0) {   // no keys: out = 0, rho* = 0
+    if (tid < kLlaD) {
+      store_out(tid, 0.f);
+      if (a.rho) a.rho[orow + tid] = 0.f;
+    }
+    return;
+  }
+  const float* rec0 = a.rec + (size_t)bh * a.pieces * kLlaRecFloats;
+  float* Dkk_s = Lt;   // D_KK of piece 0, [128][128] column-major as recorded, until the panels write L^T
+  {   // D_KK, then D_KV, of piece 0 into shared memory, in the background
+    const float* src = rec0 + kLlaRecKK;
+    for (int i = tid; i < kLlaD * kLlaD / 4; i += kLlaSolveThreads) cp_async16(Dkk_s + 4 * i, src + 4 * i);
+    cp_async_commit();
+    src = rec0 + kLlaRecKV;
+    for (int i = tid; i < kLlaD * kLlaD / 4; i += kLlaSolveThreads) cp_async16(Dkv + 4 * i, src + 4 * i);
+    cp_async_commit();
+  }
+  const float ks0 = rec0[kLlaRecKs + tid], vs0 = rec0[kLlaRecVs + tid];   // piece 0's sums, loaded early
+  if (warp == 0) {   // lane p merges piece p (at most 32 pieces)
+    const bool has = lane < a.pieces;
+    const float* r = rec0 + (size_t)lane * kLlaRecFloats;
+    const float lp = has ? r[kLlaRecM + 1] : 0.f;
+    const float mp = lp > 0.f ? r[kLlaRecM] : -INFINITY;
+    float M = mp;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = lp > 0.f ? ex2(mp - M) : 0.f;
+    if (has) wts[lane] = w;
+    const float L = warp_sum(w * lp);
+    if (lane == 0) {
+      misc[0] = L;
+      misc[2] = 0.f;
+      misc[3] = 0.f;
+      mbar_init(upd_done, 1);
+      mbar_init(drain, 1);
+      fence_mbarrier_init();
+    }
+  }
+  // The products read columns 0..15 of each operand row (its 16-byte chunks
+  // 0 and 1, at swizzled places): chunk 0 is written every panel, chunk 1
+  // (columns 8..15) stays zero.  Thread a clears chunk 1 of row a in each part.
+#pragma unroll
+  for (int part_i = 0; part_i < 3; ++part_i)
+    *reinterpret_cast<uint4*>(sm + Ly::kOp + part_i * Ly::kOpBytes + tid * 128 + ((1 ^ (tid & 7)) << 4)) =
+        make_uint4(0u, 0u, 0u, 0u);
+  if (warp == 0) {
+    tmem_alloc(tmem_base_s, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_s;
+  const float invL = 1.f / misc[0];
+  {
+    // (an empty piece has weight 0 and is skipped, whatever its record holds)
+    float ks = wts[0] == 0.f ? 0.f : wts[0] * ks0, vs = wts[0] == 0.f ? 0.f : wts[0] * vs0;
+    for (int p = 1; p < a.pieces; ++p) {
+      if (wts[p] == 0.f) continue;
+      const float* r = rec0 + (size_t)p * kLlaRecFloats;
+      ks = fmaf(wts[p], r[kLlaRecKs + tid], ks);
+      vs = fmaf(wts[p], r[kLlaRecVs + tid], vs);
+    }
+    kb[tid] = ks * invL;
+    vb[tid] = vs * invL;
+  }
+  cp_async_wait_group1();   // this thread's part of D_KK has landed (D_KV may still be on its way)
+  __syncthreads();          // and everyone's
+
+  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+  const int r_ = tid;   // row a of S, TMEM lane a
+  // ---- row a of S_KK + ridge I = D_KK / l - kbar kbar^T + ridge I into tensor
+  // memory (D_KK is recorded column-major: entry [a][j] at j * 128 + a, so a
+  // warp's 32 rows read 128 contiguous bytes per column): piece 0 from
+  // shared memory, any other piece from global memory, 64 loads in flight
+#pragma unroll 1
+  for (int c64 = 0; c64 < 2; ++c64) {
+    float sv[64];
+    const float w0 = wts[0];
+#pragma unroll
+    for (int j = 0; j < 64; ++j) sv[j] = w0 == 0.f ? 0.f : w0 * Dkk_s[(64 * c64 + j) * kLlaD + r_];
+#pragma unroll 1
+    for (int p = 1; p < a.pieces; ++p) {
+      const float w = wts[p];
+      if (w == 0.f) continue;
+      const float* col0 = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKK + (size_t)(64 * c64) * kLlaD + r_;
+      float v[64];
+#pragma unroll
+      for (int j = 0; j < 64; ++j) v[j] = __ldg(col0 + (size_t)j * kLlaD);
+#pragma unroll
+      for (int j = 0; j < 64; ++j) sv[j] = fmaf(w, v[j], sv[j]);
+    }
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t v[32];
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int col = 64 * c64 + 32 * h + j;
+        v[j] = __float_as_uint(fmaf(sv[32 * h + j], invL, -kb[r_] * kb[col]) + (col == r_ ? a.ridge : 0.f));
+      }
+      tmem_st32(tmem + lane_off + (uint32_t)(64 * c64 + 32 * h), v);
+    }
+  }
+  tmem_wait_st();
+  lla_solve_body<false, LlaSolveLayout>(a, sm, tmem, tid, warp, lane, 1, 0, Dkv, rec0, invL, orow);
+}
+
+// ---------------------------------------------------------------- moments
 __global__ void __launch_bounds__(kLlaThreads, 1)
     lla_moments_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                        const LlaArgs a) {
@@ -209,8 +759,19 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   const int tiles = (len + kTile - 1) / kTile;
   const int t0 = (int)((long long)piece * tiles / a.pieces);
   const int n = (int)((long long)(piece + 1) * tiles / a.pieces) - t0;
-  if (n == 0) {   // no keys in this piece: an empty record
-    if (threadIdx.x == 0) {
+  auto zero_out = [&] {   // the head's output and rho* when it has no usable keys
+    for (int i = threadIdx.x; i < kLlaD; i += kLlaThreads) {
+      if (a.out_bf16)
+        reinterpret_cast<__nv_bfloat16*>(a.out)[(size_t)bh * kLlaD + i] = __float2bfloat16_rn(0.f);
+      else
+        reinterpret_cast<float*>(a.out)[(size_t)bh * kLlaD + i] = 0.f;
+      if (a.rho) a.rho[(size_t)bh * kLlaD + i] = 0.f;
+    }
+  };
+  if (n == 0) {   // no keys in this piece: an empty record (no keys at all: zeros)
+    if (a.fused) {
+      zero_out();
+    } else if (threadIdx.x == 0) {
       rec[kLlaRecM] = -INFINITY;
       rec[kLlaRecM + 1] = 0.f;
     }
@@ -224,8 +785,10 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       bad |= pg < 0 || pg >= a.num_pages;
     }
     if (__syncthreads_or(bad)) {
-      if (threadIdx.x == 0) {
-        report_error(1 /* PLX_DEVERR_BAD_PAGE */);
+      if (threadIdx.x == 0) report_error(1 /* PLX_DEVERR_BAD_PAGE */);
+      if (a.fused) {
+        zero_out();
+      } else if (threadIdx.x == 0) {
         rec[kLlaRecM] = -INFINITY;
         rec[kLlaRecM + 1] = 0.f;
       }
@@ -462,7 +1025,7 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
     // ---- the piece's record (score side): wait for the scale warps' outcome
     const bool rec_ok = bar_and(4, kLlaScore + kLlaScale, ok);
     bar_and(5, kLlaScore + kLlaScale, true);   // the scale warps' partial sums are in place
-    if (c == 0) {
+    if (c == 0 && !a.fused) {
       if (rec_ok) {
         rec[kLlaRecM] = m_ref;
         rec[kLlaRecM + 1] = (red_s[4] + red_s[5]) + (red_s[6] + red_s[7]);
@@ -581,7 +1144,74 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
       pv[1] = make_float4(vs[4], vs[5], vs[6], vs[7]);
     }
     bar_and(5, kLlaScore + kLlaScale, true);
-    if (wl) {
+    if (a.fused) {
+      // ---- the solve in place, by the scale warps 8..11 (TMEM lane
+      // quarters 0..3 in order): S_KK + ridge I from D_KK in tensor memory,
+      // kbar and vbar from the partial sums, then the common solve body
+      if (warp >= 8 && warp < 12) {
+        using FL = LlaFusedSolveLayout;
+        const int sw = warp - 8, stid = sw * 32 + lane;
+        uint8_t* ss = sm + Ly::kKV;   // the ring, idle once the last products are done
+        float* kbf = reinterpret_cast<float*>(ss + FL::kVec);
+        float* vbf = kbf + kLlaD;
+        float* miscf = reinterpret_cast<float*>(ss + FL::kMisc);
+        float* wtsf = reinterpret_cast<float*>(ss + FL::kWts);
+        uint64_t* updf = reinterpret_cast<uint64_t*>(ss + FL::kBar);
+        const size_t orow = (size_t)bh * kLlaD;
+        const float lsum = (red_s[4] + red_s[5]) + (red_s[6] + red_s[7]);
+        const float invL = 1.f / lsum;
+        if (wl) {
+          float s4k[4] = {0.f, 0.f, 0.f, 0.f}, s4v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int g = 0; g < 16; ++g) {
+            s4k[g & 3] += scr[g * kLlaD + stid];
+            s4v[g & 3] += scr[16 * kLlaD + g * kLlaD + stid];
+          }
+          kbf[stid] = ((s4k[0] + s4k[1]) + (s4k[2] + s4k[3])) * invL;
+          vbf[stid] = ((s4v[0] + s4v[1]) + (s4v[2] + s4v[3])) * invL;
+#pragma unroll
+          for (int part_i = 0; part_i < 3; ++part_i)   // chunk 1 of each operand row stays zero
+            *reinterpret_cast<uint4*>(ss + FL::kOp + part_i * FL::kOpBytes + stid * 128 + ((1 ^ (stid & 7)) << 4)) =
+                make_uint4(0u, 0u, 0u, 0u);
+          if (stid == 0) {
+            miscf[0] = lsum;
+            miscf[2] = 0.f;
+            miscf[3] = 0.f;
+            wtsf[0] = 1.f;
+            mbar_init(updf, 1);
+            mbar_init(updf + 1, 1);
+            fence_mbarrier_init();
+          }
+        }
+        asm volatile("bar.sync 8, %0;" ::"n"(kLlaSolveThreads) : "memory");
+        if (wl) {
+          // S = D_KK / l - kbar kbar^T + ridge I over D_KK, row a in lane a
+          tc_fence_after();
+          const uint32_t loff = (uint32_t)(sw * 32) << 16;
+#pragma unroll 1
+          for (int c32 = 0; c32 < 4; ++c32) {
+            uint32_t r[32];
+            tmem_ld32(tmem + loff + (uint32_t)(32 * c32), r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int col = 32 * c32 + j;
+              r[j] = __float_as_uint(fmaf(__uint_as_float(r[j]), invL, -kbf[stid] * kbf[col]) +
+                                     (col == stid ? a.ridge : 0.f));
+            }
+            tmem_st32(tmem + loff + (uint32_t)(32 * c32), r);
+          }
+          tmem_wait_st();
+          lla_fused_solve(a, ss, tmem, stid, sw, lane, invL, orow);
+        } else {   // abandoned after a wait ran out (already reported)
+          if (a.out_bf16)
+            reinterpret_cast<__nv_bfloat16*>(a.out)[orow + stid] = __float2bfloat16_rn(0.f);
+          else
+            reinterpret_cast<float*>(a.out)[orow + stid] = 0.f;
+          if (a.rho) a.rho[orow + stid] = 0.f;
+        }
+      }
+    } else if (wl) {
       tc_fence_after();
 #pragma unroll 1
       for (int part = 4 * kh; part < 4 * kh + 4; ++part) {
@@ -606,459 +1236,6 @@ __global__ void __launch_bounds__(kLlaThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == 1) tmem_dealloc(tmem, 512);
-}
-
-// ---------------------------------------------------------------- solve
-// One CTA per (sequence, query head): four row warps, row a in TMEM lane a.
-// S = S_KK + ridge I (fp32) lives in tensor memory, row a in lane a.  Blocked
-// right-looking Cholesky, 8 columns per panel: every row thread reads its 8
-// panel entries; the diagonal block goes through shared memory and each
-// thread factors it redundantly (no further synchronisation), solves its own
-// row against it and carries the forward substitution z = L^-1 (kbar - q)
-// along; the trailing update S -= L_P L_P^T runs on the tensor cores, with
-// each panel value split into three bf16 parts (hi + mid + lo carries the
-// fp32 value) and six products (hi hi, hi mid, mid hi, hi lo, lo hi, mid
-// mid) of a 128 x 128 x 16 MMA with A negated, issued by the first warp once
-// a named barrier says the panel is written.  The factor also goes to shared
-// memory, transposed, for the blocked back substitution L^T rho = z, whose
-// diagonal blocks are inverted all at once (one column per thread) first.
-// D_KV comes into shared memory by cp.async while the factorisation runs.
-constexpr int kLlaSolveThreads = 128;
-constexpr int kLlaLt = kLlaD + 4;                // row stride of L^T (padding against bank conflicts)
-
-struct LlaSolveLayout {
-  static constexpr int kDkv = 0;                              // float [128][128]: D_KV of piece 0
-  static constexpr int kLt = kDkv + kLlaD * kLlaD * 4;        // float [128][kLlaLt]: L^T
-  static constexpr int kOpBytes = kLlaD * 128;                // bf16 [128][64], 128-byte swizzle (16 columns used)
-  static constexpr int kOp = (kLt + kLlaD * kLlaLt * 4 + 1023) & ~1023;   // three parts: hi, mid, lo
-  static constexpr int kD8 = kOp + 3 * kOpBytes;              // float [8][8] diagonal block + [8] its z rhs
-  static constexpr int kMinv = kD8 + 72 * 4;                  // float [16][8][8]: (L_II^T)^-1
-  static constexpr int kVec = kMinv + 16 * 64 * 4;            // float [7][128]: kbar, vbar, rho, r, z, part, 1/L_kk
-  static constexpr int kWts = kVec + 7 * kLlaD * 4;           // float [kLlaMaxPieces]
-  static constexpr int kMisc = kWts + kLlaMaxPieces * 4;      // float [8]: l, kbar.rho, bad, stop, ...
-  static constexpr int kBar = (kMisc + 32 + 7) & ~7;          // upd_done, drain
-  static constexpr int kTmem = kBar + 24;
-  static constexpr int kBytes = kTmem + 16 + 1024;
-};
-
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gmem_src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_group1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-
-// 8 consecutive 32-bit columns of this thread's TMEM lane.
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t* r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-}
-
-// Cholesky of the 8 x 8 block d (lower triangle used) in place, with the
-// reciprocals of the diagonal; false if a pivot is not positive.
-__device__ __forceinline__ bool lla_chol8(float (&d)[8][8], float (&inv)[8]) {
-  bool ok = true;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float akk = d[k][k];
-    ok = ok && akk > 0.f && isfinite(akk);
-    const float invd = rsqrtf(akk);
-    d[k][k] = akk * invd;
-    inv[k] = invd;
-#pragma unroll
-    for (int i = k + 1; i < 8; ++i) d[i][k] *= invd;
-#pragma unroll
-    for (int i = k + 1; i < 8; ++i)
-#pragma unroll
-      for (int jj = k + 1; jj <= i; ++jj) d[i][jj] = fmaf(-d[i][k], d[jj][k], d[i][jj]);
-  }
-  return ok;
-}
-
-__global__ void __launch_bounds__(kLlaSolveThreads, 1) lla_solve_kernel(const LlaArgs a) {
-  using Ly = LlaSolveLayout;
-  extern __shared__ uint8_t smem_raw_s[];
-  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_s) + 1023) & ~uintptr_t(1023));
-  float* Dkv = reinterpret_cast<float*>(sm + Ly::kDkv);   // column-major as recorded
-  float* Lt = reinterpret_cast<float*>(sm + Ly::kLt);     // Lt[k * kLlaLt + i] = L[i][k]
-  float* d8 = reinterpret_cast<float*>(sm + Ly::kD8);     // [8][8] diagonal block, then [8] its rhs
-  float* kb = reinterpret_cast<float*>(sm + Ly::kVec);    // kbar
-  float* vb = kb + kLlaD;                                 // vbar
-  float* rho_s = vb + kLlaD;                              // rho*
-  float* rb = rho_s + kLlaD;                              // back substitution right-hand side
-  float* z_s = rb + kLlaD;                                // z = L^-1 (kbar - q)
-  float* part = z_s + kLlaD;                              // D_KV^T rho*
-  float* inv_s = part + kLlaD;                            // 1 / L[k][k]
-  float* minv = reinterpret_cast<float*>(sm + Ly::kMinv); // [I][c][r]: (L_II^T)^-1
-  float* wts = reinterpret_cast<float*>(sm + Ly::kWts);   // piece weights 2^(m_j - M)
-  float* misc = reinterpret_cast<float*>(sm + Ly::kMisc); // [0] l, [1] kbar . rho*, [2] bad pivot, [3] stop
-  uint64_t* upd_done = reinterpret_cast<uint64_t*>(sm + Ly::kBar);   // the panel's update is done
-  uint64_t* drain = upd_done + 1;                                    // every product has completed
-  uint32_t* tmem_base_s = reinterpret_cast<uint32_t*>(sm + Ly::kTmem);
-
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x, b = bh / a.Hq;
-  const size_t orow = (size_t)bh * kLlaD;
-  // Launched with a programmatic dependency on the moments grid: the records
-  // are read only after it has completed.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int len = lla_seq_len(a, b);
-  auto store_out = [&](int i, float v) {
-    if (a.out_bf16)
-      reinterpret_cast<__nv_bfloat16*>(a.out)[orow + i] = __float2bfloat16_rn(v);
-    else
-      reinterpret_cast<float*>(a.out)[orow + i] = v;
-  };
-  if (len == 0) {   // no keys: out = 0, rho* = 0
-    if (tid < kLlaD) {
-      store_out(tid, 0.f);
-      if (a.rho) a.rho[orow + tid] = 0.f;
-    }
-    return;
-  }
-  const float* rec0 = a.rec + (size_t)bh * a.pieces * kLlaRecFloats;
-  float* Dkk_s = Lt;   // D_KK of piece 0, [128][128] column-major as recorded, until the panels write L^T
-  {   // D_KK, then D_KV, of piece 0 into shared memory, in the background
-    const float* src = rec0 + kLlaRecKK;
-    for (int i = tid; i < kLlaD * kLlaD / 4; i += kLlaSolveThreads) cp_async16(Dkk_s + 4 * i, src + 4 * i);
-    cp_async_commit();
-    src = rec0 + kLlaRecKV;
-    for (int i = tid; i < kLlaD * kLlaD / 4; i += kLlaSolveThreads) cp_async16(Dkv + 4 * i, src + 4 * i);
-    cp_async_commit();
-  }
-  const float ks0 = rec0[kLlaRecKs + tid], vs0 = rec0[kLlaRecVs + tid];   // piece 0's sums, loaded early
-  if (warp == 0) {   // lane p merges piece p (at most 32 pieces)
-    const bool has = lane < a.pieces;
-    const float* r = rec0 + (size_t)lane * kLlaRecFloats;
-    const float lp = has ? r[kLlaRecM + 1] : 0.f;
-    const float mp = lp > 0.f ? r[kLlaRecM] : -INFINITY;
-    float M = mp;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float w = lp > 0.f ? ex2(mp - M) : 0.f;
-    if (has) wts[lane] = w;
-    const float L = warp_sum(w * lp);
-    if (lane == 0) {
-      misc[0] = L;
-      misc[2] = 0.f;
-      misc[3] = 0.f;
-      mbar_init(upd_done, 1);
-      mbar_init(drain, 1);
-      fence_mbarrier_init();
-    }
-  }
-  // The products read columns 0..15 of each operand row (its 16-byte chunks
-  // 0 and 1, at swizzled places): chunk 0 is written every panel, chunk 1
-  // (columns 8..15) stays zero.  Thread a clears chunk 1 of row a in each part.
-#pragma unroll
-  for (int part_i = 0; part_i < 3; ++part_i)
-    *reinterpret_cast<uint4*>(sm + Ly::kOp + part_i * Ly::kOpBytes + tid * 128 + ((1 ^ (tid & 7)) << 4)) =
-        make_uint4(0u, 0u, 0u, 0u);
-  if (warp == 0) {
-    tmem_alloc(tmem_base_s, 128);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_base_s;
-  const float invL = 1.f / misc[0];
-  {
-    // (an empty piece has weight 0 and is skipped, whatever its record holds)
-    float ks = wts[0] == 0.f ? 0.f : wts[0] * ks0, vs = wts[0] == 0.f ? 0.f : wts[0] * vs0;
-    for (int p = 1; p < a.pieces; ++p) {
-      if (wts[p] == 0.f) continue;
-      const float* r = rec0 + (size_t)p * kLlaRecFloats;
-      ks = fmaf(wts[p], r[kLlaRecKs + tid], ks);
-      vs = fmaf(wts[p], r[kLlaRecVs + tid], vs);
-    }
-    kb[tid] = ks * invL;
-    vb[tid] = vs * invL;
-  }
-  cp_async_wait_group1();   // this thread's part of D_KK has landed (D_KV may still be on its way)
-  __syncthreads();          // and everyone's
-
-  const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-  constexpr uint32_t kIdUpd = idesc_bf16(kLlaD, kLlaD, false) | (1u << 13);   // 128 x 128 x 16, A negated
-  const int r_ = tid;   // row a of S, TMEM lane a
-  // ---- row a of S_KK + ridge I = D_KK / l - kbar kbar^T + ridge I into tensor
-  // memory (D_KK is recorded column-major: entry [a][j] at j * 128 + a, so a
-  // warp's 32 rows read 128 contiguous bytes per column): piece 0 from
-  // shared memory, any other piece from global memory, 64 loads in flight
-#pragma unroll 1
-  for (int c64 = 0; c64 < 2; ++c64) {
-    float sv[64];
-    const float w0 = wts[0];
-#pragma unroll
-    for (int j = 0; j < 64; ++j) sv[j] = w0 == 0.f ? 0.f : w0 * Dkk_s[(64 * c64 + j) * kLlaD + r_];
-#pragma unroll 1
-    for (int p = 1; p < a.pieces; ++p) {
-      const float w = wts[p];
-      if (w == 0.f) continue;
-      const float* col0 = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKK + (size_t)(64 * c64) * kLlaD + r_;
-      float v[64];
-#pragma unroll
-      for (int j = 0; j < 64; ++j) v[j] = __ldg(col0 + (size_t)j * kLlaD);
-#pragma unroll
-      for (int j = 0; j < 64; ++j) sv[j] = fmaf(w, v[j], sv[j]);
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t v[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int col = 64 * c64 + 32 * h + j;
-        v[j] = __float_as_uint(fmaf(sv[32 * h + j], invL, -kb[r_] * kb[col]) + (col == r_ ? a.ridge : 0.f));
-      }
-      tmem_st32(tmem + lane_off + (uint32_t)(64 * c64 + 32 * h), v);
-    }
-  }
-  tmem_wait_st();
-  float rr_a = kb[r_] - __bfloat162float(a.q[orow + r_]);   // forward right-hand side of row a
-  bool fine = true;
-  // x holds this row's entries in panel P's columns, fully updated.  The
-  // tensor-core update of panel P leaves out panel P + 1's columns (their
-  // rows are zero in its operand): those the row threads update themselves
-  // in fp32 right after issuing it (look-ahead), so panel P + 1 can be
-  // factored while the tensor cores update the rest.
-  float x[8];
-  {
-    uint32_t xr[8];
-    tmem_ld8(tmem + lane_off, xr);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c = 0; c < 8; ++c) x[c] = __uint_as_float(xr[c]);
-  }
-#pragma unroll 1
-  for (int P = 0; P < 16; ++P) {
-    const int c0 = 8 * P;
-    if (r_ >= c0 && r_ < c0 + 8) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) d8[(r_ - c0) * 8 + c] = x[c];
-      d8[64 + (r_ - c0)] = rr_a;
-    }
-    bar_and(1, kLlaSolveThreads, true);
-    // every row thread factors the diagonal block and solves L_PP z_P = r_P
-    float dd[8][8], inv[8], zz[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) dd[i][c] = d8[i * 8 + c];
-    const bool ok = lla_chol8(dd, inv);
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float v = d8[64 + c];
-#pragma unroll
-      for (int m = 0; m < c; ++m) v = fmaf(-dd[c][m], zz[m], v);
-      zz[c] = v * inv[c];
-    }
-    if (!ok) {   // not numerically positive definite (every row thread sees it)
-      fine = false;
-      if (r_ == 0) {
-        misc[2] = 1.f;
-        misc[3] = 1.f;
-      }
-      break;
-    }
-    // this row's entries of L in the panel
-    float l[8];
-    if (r_ >= c0 + 8) {   // below the panel's diagonal block: l L_PP^T = x
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float v = x[c];
-#pragma unroll
-        for (int m = 0; m < c; ++m) v = fmaf(-l[m], dd[c][m], v);
-        l[c] = v * inv[c];
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) rr_a = fmaf(-l[c], zz[c], rr_a);
-    } else if (r_ >= c0) {   // a row of the diagonal block: that row of L_PP
-      const int ri = r_ - c0;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        float v = 0.f;
-#pragma unroll
-        for (int i = c; i < 8; ++i) v = i == ri ? dd[i][c] : v;
-        l[c] = v;
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) l[c] = 0.f;
-    }
-    if (r_ >= c0) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) Lt[(c0 + c) * kLlaLt + r_] = l[c];
-    }
-    if (r_ == c0) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        z_s[c0 + c] = zz[c];
-        inv_s[c0 + c] = inv[c];
-      }
-    }
-    const bool mma = P < 14;   // columns past panel P + 1 remain
-    // The previous panel's products are done: their operand may be
-    // rewritten, and panel P + 1's columns in tensor memory are current.
-    bool w = true;
-    if (P >= 1 && P <= 14) w = mbar_wait_bounded(a.wait_ns, upd_done, (P - 1) & 1);
-    if (mma && w) {
-      // the update's operand: rows below panel P + 1, split into bf16 hi +
-      // mid + lo (16-byte chunk 0 of the row; the rest is zero)
-      const bool live = r_ >= c0 + 16;
-      uint32_t ph[4], pm[4], pl[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const float v0 = live ? l[2 * c] : 0.f, v1 = live ? l[2 * c + 1] : 0.f;
-        ph[c] = pack_bf16(v0, v1);
-        const float m0 = v0 - bf16_lo_f(ph[c]), m1 = v1 - bf16_hi_f(ph[c]);
-        pm[c] = pack_bf16(m0, m1);
-        pl[c] = pack_bf16(m0 - bf16_lo_f(pm[c]), m1 - bf16_hi_f(pm[c]));
-      }
-      const int off = r_ * 128 + ((r_ & 7) << 4);   // chunk 0 of row a, swizzled
-      *reinterpret_cast<uint4*>(sm + Ly::kOp + off) = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-      *reinterpret_cast<uint4*>(sm + Ly::kOp + Ly::kOpBytes + off) = make_uint4(pm[0], pm[1], pm[2], pm[3]);
-      *reinterpret_cast<uint4*>(sm + Ly::kOp + 2 * Ly::kOpBytes + off) = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-      fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    if (!bar_and(1, kLlaSolveThreads, w)) {   // the operand and this panel's L^T are written, or a wait ran out (reported)
-      fine = false;
-      if (r_ == 0) misc[3] = 1.f;
-      break;
-    }
-    if (mma && warp == 0) {
-      // S -= L L^T over six products of the parts (hi hi, hi mid, mid hi, hi lo, lo hi, mid mid)
-      tc_fence_after();
-      const uint64_t dh = smem_desc_sw128(smem_u32(sm + Ly::kOp), 16, 1024);
-      const uint64_t dm = dh + (uint64_t)(Ly::kOpBytes >> 4), dl = dh + (uint64_t)((2 * Ly::kOpBytes) >> 4);
-      lla_mma4_ss(tmem, dh, dh, dh, dm, dm, dh, dh, dl, kIdUpd, 1u);
-      tc_mma_ss(tmem, dl, dh, kIdUpd, 1u);
-      tc_mma_ss(tmem, dm, dm, kIdUpd, 1u);
-      tc_commit(upd_done);
-    }
-    if (P == 15) break;
-    // panel P + 1's columns, then this panel's part of their update
-    tc_fence_after();
-    {
-      uint32_t xr[8];
-      tmem_ld8(tmem + lane_off + (uint32_t)(c0 + 8), xr);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 8; ++c) x[c] = __uint_as_float(xr[c]);
-    }
-    if (r_ >= c0 + 8) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const float* lrow = Lt + c0 * kLlaLt + c0 + 8 + c;   // L[c0 + 8 + c][c0 + k] at k * kLlaLt
-        float v = x[c];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) v = fmaf(-l[k], lrow[k * kLlaLt], v);
-        x[c] = v;
-      }
-    }
-  }
-  if (warp == 0) {   // every product issued completes before tensor memory is freed
-    tc_commit(drain);
-    __syncwarp();
-    mbar_wait_drain(drain, 0);
-    __syncwarp();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, 128);
-  if (!fine) {   // (a wait that ran out has reported itself)
-    cp_async_wait_all();
-    if (tid == 0 && misc[2] != 0.f) report_error(PLX_DEVERR_SINGULAR_BIT);
-    store_out(tid, vb[tid]);   // rho* = 0: the output falls back to vbar
-    if (a.rho) a.rho[orow + tid] = 0.f;
-    return;
-  }
-  // ---- L^T rho = z.  First the inverses of the transposed diagonal blocks,
-  // one column per thread: column j of (L_II^T)^-1 for I = tid / 8, j = tid % 8.
-  {
-    const int I = tid >> 3, j = tid & 7;
-    float xx[8];
-#pragma unroll
-    for (int c = 7; c >= 0; --c) {
-      float v = c == j ? 1.f : 0.f;
-#pragma unroll
-      for (int rr2 = c + 1; rr2 < 8; ++rr2) v = fmaf(-Lt[(8 * I + c) * kLlaLt + 8 * I + rr2], xx[rr2], v);
-      xx[c] = v * inv_s[8 * I + c];
-      minv[I * 64 + c * 8 + j] = xx[c];
-    }
-    rb[r_] = z_s[r_];
-  }
-  __syncthreads();
-  // Then blockwise from the last block: rho_I = (L_II^T)^-1 r_I (eight
-  // threads), and every row above takes L_IJ^T rho_I off its r_J.
-#pragma unroll 1
-  for (int I = 15; I >= 0; --I) {
-    if (r_ < 8) {
-      float t = 0.f;
-#pragma unroll
-      for (int rr2 = 0; rr2 < 8; ++rr2) t = fmaf(minv[I * 64 + r_ * 8 + rr2], rb[8 * I + rr2], t);
-      rho_s[8 * I + r_] = t;
-    }
-    __syncthreads();
-    if (r_ < 8 * I) {
-      float t = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) t = fmaf(Lt[r_ * kLlaLt + 8 * I + c], rho_s[8 * I + c], t);
-      rb[r_] -= t;
-    }
-    __syncthreads();
-  }
-  if (tid < 32) {
-    float kr = 0.f;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) kr = fmaf(kb[tid + 32 * u], rho_s[tid + 32 * u], kr);
-    kr = warp_sum(kr);
-    if (tid == 0) misc[1] = kr;
-  }
-  cp_async_wait_all();
-  __syncthreads();
-  // ---- out = vbar (1 + kbar . rho*) - (1 / l) sum_a D_KV[a, :] rho*_a: warp w
-  // takes columns 32 w .. 32 w + 31, lane l rows 4 l .. 4 l + 3 of each (a
-  // column of D_KV is 512 contiguous bytes).  Every lane forms its 32
-  // partial dot products; a halving exchange across the lanes (16 + 8 + 4 +
-  // 2 + 1 shuffles) then leaves lane j with the sum of column 32 w + j.
-  {
-    const float4 rr = *reinterpret_cast<const float4*>(rho_s + 4 * lane);
-    auto dot4 = [&](const float4 v) { return fmaf(v.x, rr.x, fmaf(v.y, rr.y, fmaf(v.z, rr.z, v.w * rr.w))); };
-    float acc[32];
-    const float w0 = wts[0];
-#pragma unroll
-    for (int k = 0; k < 32; ++k)
-      acc[k] = w0 == 0.f ? 0.f : w0 * dot4(*reinterpret_cast<const float4*>(Dkv + (32 * warp + k) * kLlaD + 4 * lane));
-#pragma unroll 1
-    for (int p = 1; p < a.pieces; ++p) {
-      const float wp = wts[p];
-      if (wp == 0.f) continue;
-      const float* src = rec0 + (size_t)p * kLlaRecFloats + kLlaRecKV + 4 * lane;
-#pragma unroll
-      for (int k = 0; k < 32; ++k)
-        acc[k] = fmaf(wp, dot4(__ldg(reinterpret_cast<const float4*>(src + (32 * warp + k) * kLlaD))), acc[k]);
-    }
-    // step o: the lanes with bit o set keep the upper half of their columns
-    // and send the lower half to lane ^ o, the others the reverse
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const bool up = (lane & o) != 0;
-#pragma unroll
-      for (int i = 0; i < o; ++i) {
-        const float send = up ? acc[i] : acc[i + o];
-        const float keep = up ? acc[i + o] : acc[i];
-        acc[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-    }
-    part[32 * warp + lane] = acc[0];
-  }
-  __syncthreads();
-  store_out(tid, fmaf(vb[tid], 1.f + misc[1], -part[tid] * invL));
-  if (a.rho) a.rho[orow + tid] = rho_s[tid];
 }
 
 constexpr int lla_solve_smem_bytes() { return LlaSolveLayout::kBytes; }

@@ -981,6 +981,9 @@ plx_status parallax_lla_decode(const void* q, const void* k_cache, const void* v
   a.ridge = ridge;
   a.out_bf16 = p->out_dtype == PLX_BF16 ? 1 : 0;
   a.wait_ns = current_wait_ns();
+  // One piece per head: the moments kernel solves in place (its D_KK and
+  // D_KV never leave tensor memory) and no solve grid is launched.
+  a.fused = pieces == 1 && p->kv_len > 0 ? 1 : 0;
   if (p->kv_len > 0) {   // kv_len 0: every sequence is empty and the solve writes zeros
     const uint64_t rows = paged ? (uint64_t)p->num_pages * p->num_kv_heads * kTile
                                 : (uint64_t)p->batch * p->num_kv_heads * p->kv_len;
@@ -994,6 +997,7 @@ plx_status parallax_lla_decode(const void* q, const void* k_cache, const void* v
         cudaSuccess)
       return PLX_ERR_CUDA;
   }
+  if (a.fused) return PLX_OK;
   constexpr int ssmem = lla_solve_smem_bytes();
   if (set_smem(lla_solve_kernel, ssmem) != cudaSuccess)
     return PLX_ERR_CUDA;

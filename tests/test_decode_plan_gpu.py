@@ -99,3 +99,32 @@ def test_plan_step_from_host_memory(px):
     assert torch.equal(out.cpu(), ref.cpu())
     with pytest.raises(ValueError):
         plan.run_io(inp["q"], hr, hout)   # a device tensor where a host one belongs
+
+
+def test_host_steps_chained_without_synchronisation(px):
+    # Zero-copy run_io steps back to back on one stream: each launch reads its
+    # q and rho from pinned host memory as it starts (possibly while the
+    # previous step still runs), and its K and V only after the previous
+    # kernel has finished.  Between two steps the cache is rescaled by a
+    # device op on the same stream: the second step must see the new cache.
+    inp = _cuda(W.small_decode_inputs(8, 16, 8, 128, 2048, seed=65))
+    out = torch.empty_like(inp["q"])
+    plan = px.DecodePlan(torch.empty_like(inp["q"]), torch.empty_like(inp["rho"]), inp["k_cache"], inp["v_cache"],
+                         inp["scale"], out=out)
+    gen = torch.Generator().manual_seed(7)
+    steps = []
+    for i in range(4):
+        hq = (torch.randn(inp["q"].shape, generator=gen)).to(inp["q"].dtype).pin_memory()
+        hr = (0.1 * torch.randn(inp["rho"].shape, generator=gen)).to(inp["rho"].dtype).pin_memory()
+        hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        steps.append((hq, hr, hout))
+    v0 = inp["v_cache"].clone()
+    for i, (hq, hr, hout) in enumerate(steps):
+        plan.run_io(hq, hr, hout)
+        if i == 1:
+            inp["v_cache"].mul_(2.0)   # exact in bf16: the later steps' outputs double
+    torch.cuda.synchronize()
+    for i, (hq, hr, hout) in enumerate(steps):
+        v = inp["v_cache"] if i >= 2 else v0
+        ref = px.decode(hq.cuda(), hr.cuda(), inp["k_cache"], v, inp["scale"])
+        assert torch.equal(hout, ref.cpu()), f"step {i}"

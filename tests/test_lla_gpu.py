@@ -79,14 +79,17 @@ def test_short_sequences_with_ridge(px, L):
     _check(px, inp, 0.1, f"short L={L}")
 
 
-def test_ragged_paged_and_empty(px):
+@pytest.mark.parametrize("num_ctas", [0, 32])
+def test_ragged_paged_and_empty(px, num_ctas):
+    # num_ctas 0: several pieces per head, merged by the solve grid; 32 (one
+    # CTA per head): one piece, solved in place by the moments kernel.
     lens = [3000, 1200, 65, 0]
     inp = _cuda(W.small_decode_inputs(4, 8, 2, 128, 3072, seq_lens=lens, paged=True, seed=41))
-    out, rho = _check(px, inp, 0.1, "paged ragged")
+    out, rho = _check(px, inp, 0.1, f"paged ragged, num_ctas={num_ctas}", num_ctas=num_ctas)
     assert not out[3].any() and not rho[3].any()   # an empty sequence: out = 0, rho* = 0
     contig = {k: inp[k] for k in ("q", "scale", "seq_lens")}
     contig.update(k_cache=inp["k_contig"], v_cache=inp["v_contig"])
-    out_c, rho_c = _run(px, contig, 0.1, out_dtype=torch.float32)
+    out_c, rho_c = _run(px, contig, 0.1, out_dtype=torch.float32, num_ctas=num_ctas)
     assert torch.equal(out, out_c) and torch.equal(rho, rho_c)   # same keys, same pieces: same bits
 
 
