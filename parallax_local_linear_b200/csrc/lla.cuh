@@ -13,7 +13,7 @@
 // `ridge` penalises the slope (the pages name no regularisation; 0 is plain
 // LLA).
 //
-// Two kernels per call:
+// One or two kernels per call:
 //
 //   lla_moments_kernel  one CTA per (sequence, query head, piece of its keys):
 //     a single pass over the piece's K and V tiles accumulates, relative to
@@ -34,7 +34,9 @@
 //     tile.  For sequences shorter than kLlaSplitLen the bf16 rounding of
 //     e o K is not averaged away (the solve amplifies it along directions
 //     the few keys do not span), so a second product adds its lo part
-//     (x = hi + lo).  The piece's record goes to the workspace.
+//     (x = hi + lo).  The piece's record goes to the workspace; with one
+//     piece per head the kernel instead solves in place (below), D_KK and
+//     D_KV never leaving tensor memory, and the second kernel is not run.
 //
 //   lla_solve_kernel  one CTA per (sequence, query head): merges the pieces
 //     like online softmax (weights 2^(m_j - M)), forms S_KK + ridge I and
