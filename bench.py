@@ -629,7 +629,8 @@ def bench_lla(args, w, rank, world, dev, peaks, peaks_kind):
                     "frac": round(hbm_frac, 4), "peak_source": f"{peaks_kind} hbm_gbs",
                     "algorithmic_bytes_per_launch": kv}
     roofline.update(traffic_fields("lla", w.name))
-    roofline["kernel"] = "lla_moments_kernel + lla_solve_kernel (one call)"
+    roofline["kernel"] = ("lla_moments_kernel with the solve in place (one piece per head: one launch per call); "
+                          "lla_moments_kernel + lla_solve_kernel when heads are cut into pieces")
     roofline["other_bound"] = ({"unit": "GB/s", "achieved": round(kv / step_s / 1e9, 1), "frac": round(hbm_frac, 4)}
                                if roofline["bound"] == "tensor" else
                                {"unit": "TFLOP/s", "achieved": round(tflops, 1), "frac": round(tc_frac, 4)})
