@@ -180,8 +180,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, bool a_mn_maj
 }
 
 // ---------------------------------------------------------------- solve
-// One CTA per (sequence, query head): four row warps, row a in TMEM lane a.
-// S = S_KK + ridge I (fp32) lives in tensor memory, row a in lane a.  Blocked
+// Per (sequence, query head), four row warps, row a of the system in TMEM
+// lane a: S = S_KK + ridge I (fp32) lives in tensor memory.  Blocked
 // right-looking Cholesky, 8 columns per panel: every row thread reads its 8
 // panel entries; the diagonal block goes through shared memory and each
 // thread factors it redundantly (no further synchronisation), solves its own
@@ -190,10 +190,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16_ab(int M, int N, bool a_mn_maj
 // each panel value split into three bf16 parts (hi + mid + lo carries the
 // fp32 value) and six products (hi hi, hi mid, mid hi, hi lo, lo hi, mid
 // mid) of a 128 x 128 x 16 MMA with A negated, issued by the first warp once
-// a named barrier says the panel is written.  The factor also goes to shared
-// memory, transposed, for the blocked back substitution L^T rho = z, whose
-// diagonal blocks are inverted all at once (one column per thread) first.
-// D_KV comes into shared memory by cp.async while the factorisation runs.
+// a named barrier says the panel is written; the next panel's columns are
+// updated by the row threads themselves (look-ahead).  The factor also goes
+// to shared memory, transposed, for the blocked back substitution
+// L^T rho = z, whose diagonal blocks are inverted all at once (one column
+// per thread) first.  The body runs in lla_solve_kernel (one CTA per head,
+// for heads cut into pieces: the records are merged and D_KV comes into
+// shared memory by cp.async while the factorisation runs) or in place in
+// lla_moments_kernel (one piece per head: D_KK and D_KV are already in its
+// tensor memory).
 constexpr int kLlaSolveThreads = 128;
 constexpr int kLlaLt = kLlaD + 4;                // row stride of L^T (padding against bank conflicts)
 
