@@ -117,12 +117,16 @@ def test_wait_limit_setter_round_trips(px):
         px.set_wait_limit_ns(prev)
 
 
-def test_lla_wait_timeout_then_recovery(px):
+@pytest.mark.parametrize("num_ctas", [0, 8])
+def test_lla_wait_timeout_then_recovery(px, num_ctas):
+    # num_ctas 0: heads cut into pieces, a moments grid and a solve grid; 8
+    # (one CTA per head): one grid, the solve in place in the moments kernel.
     inp = W.small_decode_inputs(2, 4, 2, 128, 4096, seed=55)
     inp = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
 
     def run():
-        return px.lla_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["scale"], 0.01, out_dtype=torch.float32)
+        return px.lla_decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["scale"], 0.01, out_dtype=torch.float32,
+                             num_ctas=num_ctas)
 
     code = _timed_out(px, run)
     assert code & px.DEVERR_TIMEOUT, f"error word {code}"
