@@ -1094,6 +1094,25 @@ def cpu_baseline_prefill_train(w, inp, budget_s):
             "seconds": round(secs, 2)}
 
 
+def workload_shape(w, args):
+    """The keys of this arm's `config` that name the workload itself (shapes,
+    dtypes, lengths), without the ones about how the GPU arm launches and
+    times it (grid size, L2 note, graph replay)."""
+    if w.name in ("prefill", "prefill_train"):
+        return {"workload": w.name, "batch": w.batch, "num_heads": w.num_heads, "seq_len": w.seq_len,
+                "head_dim": w.head_dim, "causal": w.causal, "rho_scale": w.rho_scale}
+    if w.name == "prefill_paged":
+        return {"workload": w.name, "batch": w.batch, "num_heads": w.num_heads, "num_kv_heads": w.num_kv_heads,
+                "head_dim": w.head_dim, "causal": w.causal, "page_size": W.PAGE_SIZE, "rho_scale": w.rho_scale}
+    cfg = decode_config(w, args, None)
+    cfg.pop("num_ctas", None)
+    if w.hidden:
+        cfg["hidden"] = w.hidden
+    if w.name == "lla_decode":
+        cfg["ridge"] = 0.0
+    return cfg
+
+
 def reference_arm(args, w, rank, world):
     """The float64 oracle on the host cores, on this workload's metric.
 
@@ -1135,7 +1154,8 @@ def reference_arm(args, w, rank, world):
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs_all / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": w.name},
+            "data": "synthetic",
+            "config": dict(workload_shape(w, args), timing="host wall clock of the float64 oracle on a bounded sample"),
             "cpu_baseline": {"value": round(value, 6), "unit": unit, "kind": "oracle", "cores": blas_threads(),
                              "sample": "per step: " + desc},
             "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
