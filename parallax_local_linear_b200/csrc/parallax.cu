@@ -35,7 +35,7 @@ constexpr int kMaxDevices = 64;
 #define PLX_DECODE_STAGES 4
 #endif
 constexpr int kDecodeNC = 4;
-constexpr int kDecodeStages128 = PLX_DECODE_STAGES;   // a multiple of kDecodeNC
+constexpr int kDecodeStages128 = PLX_DECODE_STAGES;   // 5 fit in shared memory for up to ~1100 sequences: no faster
 constexpr int kDecodeStages64 = 8;
 constexpr int kDecodeF32Warps = 4;
 
