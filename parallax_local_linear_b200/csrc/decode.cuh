@@ -817,6 +817,11 @@ __global__ void __launch_bounds__(NW * 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
   constexpr int NT = NW * 32;
+  // Launched with a programmatic dependency on the previous kernel: the
+  // next grid may launch at once, and this one waits for the previous grid
+  // before it touches global memory.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   build_tile_space(a, pre, lens, scan);
   for (int b = blockIdx.x; b < a.B; b += gridDim.x)
     if (lens[b] == 0)
@@ -869,7 +874,7 @@ __global__ void __launch_bounds__(NW * 32)
       if (lane < nvalid) {
         const float4* kr = reinterpret_cast<const float4*>(kc + cache_row(a, b, kvh, tok) * D);
         float s = 0.f, pr = 0.f;
-#pragma unroll 8
+#pragma unroll 16
         for (int d4 = 0; d4 < D / 4; ++d4) {
           const float4 kv = kr[d4];
           s += s_qr[0][4 * d4] * kv.x + s_qr[0][4 * d4 + 1] * kv.y + s_qr[0][4 * d4 + 2] * kv.z +
@@ -892,15 +897,26 @@ __global__ void __launch_bounds__(NW * 32)
         o1[i] *= alpha;
         o2[i] *= alpha;
       }
-      for (int j = 0; j < nvalid; ++j) {
-        const float pj = __shfl_sync(0xffffffffu, p, j);
-        const float paj = __shfl_sync(0xffffffffu, pa, j);
-        const float* vr = vc + cache_row(a, b, kvh, c0 + j) * D;
+      // eight V rows' loads in flight at a time, then their products in
+      // token order (rows past nvalid are not read; their p is 0)
+      for (int j0 = 0; j0 < nvalid; j0 += 8) {
+        float vv[8][D / 32];
 #pragma unroll
-        for (int i = 0; i < D / 32; ++i) {
-          const float vv = vr[lane + 32 * i];
-          o1[i] += pj * vv;
-          o2[i] += paj * vv;
+        for (int u = 0; u < 8; ++u) {
+          const float* vr = vc + cache_row(a, b, kvh, c0 + min(j0 + u, nvalid - 1)) * D;
+#pragma unroll
+          for (int i = 0; i < D / 32; ++i) vv[u][i] = j0 + u < nvalid ? vr[lane + 32 * i] : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (j0 + u >= nvalid) break;   // uniform across the warp
+          const float pj = __shfl_sync(0xffffffffu, p, j0 + u);
+          const float paj = __shfl_sync(0xffffffffu, pa, j0 + u);
+#pragma unroll
+          for (int i = 0; i < D / 32; ++i) {
+            o1[i] += pj * vv[u][i];
+            o2[i] += paj * vv[u][i];
+          }
         }
       }
     }

@@ -281,8 +281,8 @@ plx_status launch_decode_f32(const DecodeArgs& a, int ctas, size_t smem, cudaStr
   if (set_attr &&
       set_smem(kern, (int)smem) != cudaSuccess)
     return PLX_ERR_CUDA;
-  kern<<<ctas, kDecodeF32Warps * 32, smem, stream>>>(a);
-  return note(cudaGetLastError()) == cudaSuccess ? PLX_OK : PLX_ERR_CUDA;
+  return note(launch_pdl(kern, dim3(ctas), dim3(kDecodeF32Warps * 32), smem, stream, a)) == cudaSuccess ? PLX_OK
+                                                                                                    : PLX_ERR_CUDA;
 }
 
 // A validated decode call: kernel arguments, plan and tensor maps.
