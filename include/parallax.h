@@ -258,9 +258,14 @@ plx_status parallax_decode_noalloc(const void* q, const void* rho,
  * The pages solve by conjugate gradients; here each query head's system is
  * formed in fp32 and solved exactly by a Cholesky factorisation.
  *
- * Two launches on `stream`: a single pass over each query head's K and V
- * that accumulates sum w k k^T and sum w k v^T on the tensor cores (with
- * the first moments), then one solve per query head that also writes out.
+ * On `stream`: a single pass over each query head's K and V that
+ * accumulates sum w k k^T and sum w k v^T on the tensor cores (with the
+ * first moments), and one solve per query head that also writes out.  When
+ * each query head's keys are one piece (as many heads as SMs or more, or
+ * num_ctas = the number of heads) that is one launch: the pass's kernel
+ * solves in place, its sums never leaving tensor memory, and the workspace
+ * is not touched.  Otherwise the pieces' sums go to the workspace and a
+ * second launch merges them and solves.
  *
  *   q            device bf16 [B, Hq, 128].
  *   k_cache,     device bf16, contiguous [B, Hkv, L, 128] or paged pools
