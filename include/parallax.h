@@ -261,8 +261,9 @@ plx_status parallax_decode_noalloc(const void* q, const void* rho,
  * On `stream`: a single pass over each query head's K and V that
  * accumulates sum w k k^T and sum w k v^T on the tensor cores (with the
  * first moments), and one solve per query head that also writes out.  When
- * each query head's keys are one piece (as many heads as SMs or more, or
- * num_ctas = the number of heads) that is one launch: the pass's kernel
+ * each query head's keys are one piece (num_ctas, or for 0 the SM count,
+ * below twice the number of (sequence, query head) pairs, or kv_len below
+ * 512) that is one launch: the pass's kernel
  * solves in place, its sums never leaving tensor memory, and the workspace
  * is not touched.  Otherwise the pieces' sums go to the workspace and a
  * second launch merges them and solves.
