@@ -294,19 +294,19 @@ __device__ void finish_unit(const DecodeArgs& a, const TileSpace& ts, const CtaS
 // Warp roles: NC consumer warps and one producer warp.  The producer's lane 0
 // streams the chunk's K and V tiles (64 tokens x D, bf16) into a STAGES-deep
 // ring with 2D TMA loads (128-byte swizzle, 64-column boxes), straight across
-// unit boundaries.  Consumer warp w takes the chunk's tiles w, w + NC, ...;
-// each warp keeps its own running state per unit, and at the end of a unit
-// the consumer warps merge their states and finish the unit while the
+// unit boundaries.  Consumer warp w takes tokens 16 w .. 16 w + 15 of every
+// tile; each warp keeps its own running state per unit, and at the end of a
+// unit the consumer warps merge their states and finish the unit while the
 // producer keeps loading.
 //
-// Per tile a consumer computes, on tensor cores,
-//     [S; A] (16 x 64) = [Q; R] (16 x D) . K^T (D x 64)
+// Per tile a consumer computes, on tensor cores, over its 16 tokens
+//     [S; A] (16 x 16) = [Q; R] (16 x D) . K^T (D x 16)
 // where rows 0..g-1 of the 16-row operand are the group's queries and rows
 // 8..8+g-1 their probes (other rows zero).  The m16n8 accumulator layout then
 // gives each thread the score s and the probe value a of the same head (rows
 // h and h + 8) for the same two tokens.  It forms e and e*a in registers and
 // packs them as the A operand [P; P*A] of the second product
-//     [O1; O2] (16 x D) += [P; P*A] (16 x 64) . V (64 x D)
+//     [O1; O2] (16 x D) += [P; P*A] (16 x 16) . V (16 x D)
 // so both accumulators come from one pass over each V tile.
 // =========================================================================
 template <int D>
