@@ -802,7 +802,7 @@ constexpr int f32_smem_fixed_bytes() {
 }
 
 template <int D, int NW>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, 2)
     decode_f32_kernel(const DecodeArgs a) {
   __shared__ CtaState<D> st;
   __shared__ float s_qr[2][D];
@@ -847,6 +847,46 @@ __global__ void __launch_bounds__(NW * 32)
 
     const float* qp = reinterpret_cast<const float*>(a.q) + ((size_t)b * a.Hq + hq) * D;
     const float* rp = reinterpret_cast<const float*>(a.rho) + ((size_t)b * a.Hq + hq) * D;
+    const int tok_begin = local0 * kTile;
+    const int tok_end = min((local0 + (int)(seg_end - x)) * kTile, len);
+
+    // Every global load of a 32-token sub-chunk goes out at once, before
+    // any of its arithmetic: the lane's K row (its token's score and probe
+    // value) and the warp's V rows (each lane's D/32 columns of every
+    // token).  The first sub-chunk's loads go out beside q, rho and the
+    // first key; each later one's as soon as the previous scores and
+    // products have freed the registers.
+    constexpr int VB = D == 64 ? 32 : 16;   // V rows per batch of loads
+    float4 kr4[D / 4];
+    float vv[VB][D / 32];
+    auto load_k = [&](int c0) {
+      const int nvalid = min(32, tok_end - c0);
+      if (lane < nvalid) {
+        const float4* kr = reinterpret_cast<const float4*>(kc + cache_row(a, b, kvh, c0 + lane) * D);
+#pragma unroll
+        for (int d4 = 0; d4 < D / 4; ++d4) kr4[d4] = kr[d4];
+      }
+    };
+    auto load_v = [&](int c0, int j0) {   // rows j0 .. j0 + VB - 1 (rows past the chunk read as 0)
+      const int nvalid = min(32, tok_end - c0);
+#pragma unroll
+      for (int u = 0; u < VB; ++u) {
+        const float* vr = vc + cache_row(a, b, kvh, c0 + min(j0 + u, nvalid - 1)) * D;
+#pragma unroll
+        for (int i = 0; i < D / 32; ++i) vv[u][i] = j0 + u < nvalid ? vr[lane + 32 * i] : 0.f;
+      }
+    };
+    const int c_first = tok_begin + warp * 32;
+    if (c_first < tok_end) {
+      load_k(c_first);
+      load_v(c_first, 0);
+    }
+    float k0v[D / 32];
+    {
+      const float* k0 = kc + cache_row(a, b, kvh, 0) * D;
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) k0v[i] = k0[lane + 32 * i];
+    }
     for (int d = tid; d < D; d += NT) {
       s_qr[0][d] = qp[d];
       s_qr[1][d] = rp[d];
@@ -854,9 +894,9 @@ __global__ void __launch_bounds__(NW * 32)
     __syncthreads();
     float aref;
     {
-      const float* k0 = kc + cache_row(a, b, kvh, 0) * D;
       float acc = 0.f;
-      for (int d = lane; d < D; d += 32) acc += s_qr[1][d] * k0[d];
+#pragma unroll
+      for (int i = 0; i < D / 32; ++i) acc += s_qr[1][lane + 32 * i] * k0v[i];
       aref = warp_sum(acc);
     }
 
@@ -865,18 +905,15 @@ __global__ void __launch_bounds__(NW * 32)
 #pragma unroll
     for (int i = 0; i < D / 32; ++i) o1[i] = o2[i] = 0.f;
 
-    const int tok_begin = local0 * kTile;
-    const int tok_end = min((local0 + (int)(seg_end - x)) * kTile, len);
-    for (int c0 = tok_begin + warp * 32; c0 < tok_end; c0 += NW * 32) {
-      const int tok = c0 + lane;
+    for (int c0 = c_first; c0 < tok_end; c0 += NW * 32) {
       const int nvalid = min(32, tok_end - c0);
+      const int c_next = c0 + NW * 32;
       float xs = -INFINITY, av = 0.f;
       if (lane < nvalid) {
-        const float4* kr = reinterpret_cast<const float4*>(kc + cache_row(a, b, kvh, tok) * D);
         float s = 0.f, pr = 0.f;
-#pragma unroll 16
+#pragma unroll
         for (int d4 = 0; d4 < D / 4; ++d4) {
-          const float4 kv = kr[d4];
+          const float4 kv = kr4[d4];
           s += s_qr[0][4 * d4] * kv.x + s_qr[0][4 * d4 + 1] * kv.y + s_qr[0][4 * d4 + 2] * kv.z +
                s_qr[0][4 * d4 + 3] * kv.w;
           pr += s_qr[1][4 * d4] * kv.x + s_qr[1][4 * d4 + 1] * kv.y + s_qr[1][4 * d4 + 2] * kv.z +
@@ -885,6 +922,7 @@ __global__ void __launch_bounds__(NW * 32)
         xs = s * a.scale_log2;
         av = pr - aref;
       }
+      if (c_next < tok_end) load_k(c_next);
       const float m_new = fmaxf(m_run, warp_max(xs));
       const float alpha = ex2(m_run - m_new);
       m_run = m_new;
@@ -897,18 +935,13 @@ __global__ void __launch_bounds__(NW * 32)
         o1[i] *= alpha;
         o2[i] *= alpha;
       }
-      // eight V rows' loads in flight at a time, then their products in
-      // token order (rows past nvalid are not read; their p is 0)
-      for (int j0 = 0; j0 < nvalid; j0 += 8) {
-        float vv[8][D / 32];
+      // the products in token order (rows past nvalid hold 0 and p is 0 there)
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float* vr = vc + cache_row(a, b, kvh, c0 + min(j0 + u, nvalid - 1)) * D;
+      for (int j0 = 0; j0 < 32; j0 += VB) {
+        if (j0 >= nvalid) break;   // uniform across the warp
+        if (j0 > 0) load_v(c0, j0);
 #pragma unroll
-          for (int i = 0; i < D / 32; ++i) vv[u][i] = j0 + u < nvalid ? vr[lane + 32 * i] : 0.f;
-        }
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < VB; ++u) {
           if (j0 + u >= nvalid) break;   // uniform across the warp
           const float pj = __shfl_sync(0xffffffffu, p, j0 + u);
           const float paj = __shfl_sync(0xffffffffu, pa, j0 + u);
@@ -919,6 +952,7 @@ __global__ void __launch_bounds__(NW * 32)
           }
         }
       }
+      if (c_next < tok_end) load_v(c_next, 0);
     }
     const float l_w = warp_sum(l_lane), c_w = warp_sum(c_lane);
     if (lane == 0) {

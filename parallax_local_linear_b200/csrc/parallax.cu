@@ -39,8 +39,9 @@ constexpr int kDecodeStages128 = PLX_DECODE_STAGES;   // 5 fit in shared memory 
 constexpr int kDecodeStages64 = 8;
 constexpr int kDecodeF32Warps = 4;
 
-// Persistent grid of the fp32 path, in CTAs per SM (its CTAs are small).
-constexpr int kF32CtasPerSm = 4;
+// Persistent grid of the fp32 path, in CTAs per SM: two fit (each warp holds
+// a 32-token sub-chunk's K and V rows in registers, up to 255 a thread).
+constexpr int kF32CtasPerSm = 2;
 
 std::mutex g_mu;
 int g_num_sms[kMaxDevices];
