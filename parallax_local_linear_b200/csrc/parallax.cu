@@ -181,7 +181,10 @@ DecodePlan plan_decode(const plx_decode_params* p, int num_sms) {
     const int64_t k = num_sms / units;
     if (4 * units * k >= 3 * (int64_t)num_sms) ctas = units * k;
   }
-  if (ctas > tiles) ctas = tiles;
+  // The fp32 kernel's warps take 32-token sub-chunks: by default a CTA gets at
+  // least one per warp (two tiles), so that no warp idles on a short stream.
+  const int64_t min_tiles = p->num_ctas == 0 && !bf16 ? kDecodeF32Warps * 32 / kTile : 1;
+  if (ctas > (tiles + min_tiles - 1) / min_tiles) ctas = (tiles + min_tiles - 1) / min_tiles;
   if (ctas < 1) ctas = 1;
   if (ctas > INT32_MAX / 4) ctas = INT32_MAX / 4;
   pl.ctas = (int)ctas;
