@@ -81,9 +81,9 @@ typedef struct plx_decode_params {
   int32_t in_dtype;           /* plx_dtype of q, rho and the caches            */
   int32_t out_dtype;          /* plx_dtype of out                              */
   float scale;                /* softmax scale on q.k (e.g. 1/sqrt(d))         */
-  int32_t num_ctas;           /* persistent CTAs; 0 = one per SM (bf16) or
-                                 two per SM (fp32; and at most one per two
-                                 64-token tiles); never more than the tiles */
+  int32_t num_ctas;           /* persistent CTAs; 0 = one per SM (bf16), or
+                                 one per SM and at most one per four 64-token
+                                 tiles (fp32); never more than the tiles    */
 } plx_decode_params;
 
 /* Work decomposition.  The 64-token KV tiles of every (sequence, KV head)

@@ -802,7 +802,7 @@ constexpr int f32_smem_fixed_bytes() {
 }
 
 template <int D, int NW>
-__global__ void __launch_bounds__(NW * 32, 2)
+__global__ void __launch_bounds__(NW * 32, NW >= 8 ? 1 : 2)
     decode_f32_kernel(const DecodeArgs a) {
   __shared__ CtaState<D> st;
   __shared__ float s_qr[2][D];

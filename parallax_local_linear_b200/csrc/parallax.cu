@@ -37,11 +37,12 @@ constexpr int kMaxDevices = 64;
 constexpr int kDecodeNC = 4;
 constexpr int kDecodeStages128 = PLX_DECODE_STAGES;   // 5 fit in shared memory for up to ~1100 sequences: no faster
 constexpr int kDecodeStages64 = 8;
-constexpr int kDecodeF32Warps = 4;
+constexpr int kDecodeF32Warps = 8;
 
-// Persistent grid of the fp32 path, in CTAs per SM: two fit (each warp holds
-// a 32-token sub-chunk's K and V rows in registers, up to 255 a thread).
-constexpr int kF32CtasPerSm = 2;
+// Persistent grid of the fp32 path, in CTAs per SM: one CTA of eight warps
+// (each warp holds a 32-token sub-chunk's K and V rows in registers, up to
+// 255 a thread).
+constexpr int kF32CtasPerSm = 1;
 
 std::mutex g_mu;
 int g_num_sms[kMaxDevices];
@@ -182,7 +183,7 @@ DecodePlan plan_decode(const plx_decode_params* p, int num_sms) {
     if (4 * units * k >= 3 * (int64_t)num_sms) ctas = units * k;
   }
   // The fp32 kernel's warps take 32-token sub-chunks: by default a CTA gets at
-  // least one per warp (two tiles), so that no warp idles on a short stream.
+  // least one per warp (four tiles), so that no warp idles on a short stream.
   const int64_t min_tiles = p->num_ctas == 0 && !bf16 ? kDecodeF32Warps * 32 / kTile : 1;
   if (ctas > (tiles + min_tiles - 1) / min_tiles) ctas = (tiles + min_tiles - 1) / min_tiles;
   if (ctas < 1) ctas = 1;

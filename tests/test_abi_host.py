@@ -186,16 +186,16 @@ def test_paged_prefill_pointer_checks_and_empty_calls(binding):
         assert binding.lib.parallax_prefill_paged(*nul, ctypes.byref(pe), None) == 0
 
 
-def _expected_plan(B, units, heads_per_unit, L, d=128, num_sms=148, forced=0, per_sm=1, paged=False):
+def _expected_plan(B, units, heads_per_unit, L, d=128, num_sms=148, forced=0, f32=False, paged=False):
     tiles = B * units * (-(-L // 64))
-    ctas = forced if forced else num_sms * per_sm
+    ctas = forced if forced else num_sms
     n_units = B * units
-    if not forced and per_sm == 1 and not paged and n_units <= num_sms:
+    if not forced and not f32 and not paged and n_units <= num_sms:
         k = num_sms // n_units
         if 4 * n_units * k >= 3 * num_sms:
             ctas = n_units * k
-    # by default an fp32 CTA (four warps of 32 tokens) takes at least two 64-token tiles
-    per_cta = 2 if (not forced and per_sm != 1) else 1
+    # by default an fp32 CTA (eight warps of 32 tokens) takes at least four 64-token tiles
+    per_cta = 4 if (not forced and f32) else 1
     ctas = max(1, min(ctas, -(-tiles // per_cta)))
     counters = -(-(B * units * 4) // 256) * 256
     return ctas, counters + 2 * ctas * heads_per_unit * (2 * d + 4) * 4
@@ -209,8 +209,8 @@ def test_work_plan_and_workspace_size(binding, B, Hq, Hkv, L, forced, dtype):
     p = _params(binding, batch=B, num_q_heads=Hq, num_kv_heads=Hkv, kv_len=L, num_ctas=forced, in_dtype=dtype,
                 out_dtype=dtype)
     ctas = binding.lib.parallax_decode_num_ctas(ctypes.byref(p), 148)
-    units, hpu, per_sm = (Hkv, Hq // Hkv, 1) if dtype == 1 else (Hq, 1, 2)
-    exp_ctas, exp_ws = _expected_plan(B, units, hpu, L, forced=forced, per_sm=per_sm)
+    units, hpu = (Hkv, Hq // Hkv) if dtype == 1 else (Hq, 1)
+    exp_ctas, exp_ws = _expected_plan(B, units, hpu, L, forced=forced, f32=dtype == 0)
     assert ctas == exp_ctas
     assert binding.lib.parallax_decode_workspace_size(ctypes.byref(p), 148) == exp_ws
 
